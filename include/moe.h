@@ -1,0 +1,221 @@
+/*
+ * moe.h -- C ABI of a single-GPU Mixture-of-Experts layer forward for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (jsqmd.com, "第11章 MoE模型推理", 11.1.1 "稀疏激活原理"):
+ *
+ *     y = sum_{i in TopK} g_i(x) * E_i(x)
+ *
+ * runs as five steps, each exposed as its own call and chained by
+ * moe_layer_forward:
+ *   moe_route        router logits, scoring, top-k selection, gate weights
+ *   moe_permute      expert histogram, prefix scan, stable row permutation
+ *                    and gather of token rows into expert-contiguous rows
+ *   moe_grouped_ffn  every expert's FFN over its rows as one grouped GEMM
+ *   moe_combine      gate-weighted sum back into token order
+ *
+ * Conventions for every call:
+ *  - Tensor pointers are DEVICE pointers, row-major, owned by the caller.
+ *    The library never allocates device or host memory and never
+ *    synchronises, except moe_get_status.  Work is enqueued on `stream`
+ *    (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ *  - Weight stacks are stored "out x in" (K-major), one slab per expert:
+ *    w_router [E][d]; w1, w_gate, w_up [E+ns][h][d]; w2, w_down [E+ns][d][h],
+ *    where ns = num_shared (0 or 1) and the shared expert is slab E.
+ *  - Argument errors return before anything is enqueued.  Problems that only
+ *    the data reveals (non-finite logits, expert ids out of range, a bounded
+ *    device wait that gave up) set bits in the status block inside the
+ *    workspace and never trap; read them with moe_get_status.
+ *  - ws / ws_bytes: caller-allocated device scratch of at least
+ *    moe_workspace_size() bytes, 256-byte aligned.  Its first 256 bytes hold
+ *    the status block; moe_workspace_init zeroes it.  Calls that share one
+ *    workspace must be ordered on one stream.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null pointer, bad size or inconsistent desc */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid but not implemented combination */
+  MOE_ERR_WORKSPACE = 3,    /* ws NULL, misaligned or smaller than needed */
+  MOE_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
+  MOE_ERR_DEVICE_STATUS = 5 /* moe_get_status found error bits set */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_E4M3 = 2 } moe_dtype;
+typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score;
+typedef enum { MOE_ACT_GELU = 0, MOE_ACT_SWIGLU = 1 } moe_act;
+
+/* status block bits (moe_get_status flags) */
+#define MOE_STATUS_NONFINITE_LOGIT 0x1u /* a router logit was NaN or +-inf */
+#define MOE_STATUS_BAD_EXPERT_ID 0x2u   /* moe_permute saw an id outside [0,E) */
+#define MOE_STATUS_TIMEOUT 0x4u         /* a bounded device wait gave up */
+#define MOE_STATUS_BAD_GROUP 0x8u       /* a group table entry out of range */
+
+/* counters (moe_get_status counters[], MOE_NUM_COUNTERS entries) */
+#define MOE_CNT_NONFINITE 0   /* tokens with a non-finite logit */
+#define MOE_CNT_BAD_ID 1      /* slots with an out-of-range expert id */
+#define MOE_CNT_TIMEOUT 2     /* CTAs that gave up a wait */
+#define MOE_CNT_OVERFLOW_ROWS 3 /* rows routed to the overflow region */
+#define MOE_NUM_COUNTERS 8
+
+/*
+ * Layer shape and options.
+ *   num_tokens S, d_model d, num_experts E (routed), top_k K, d_ff h.
+ *   score_fn: MOE_SCORE_SOFTMAX -- selection key = logit (+ sel_bias);
+ *               gates = softmax over the K selected logits (renormalize=1,
+ *               the TopK(-inf)-then-Softmax form of 11.1.1) or the full
+ *               softmax probability (renormalize=0);
+ *             MOE_SCORE_SIGMOID -- s = sigmoid(logit), key = s + sel_bias
+ *               (ybb.press "MoE 推理工程深层实战" 2.3, aux-loss-free bias,
+ *               used for selection only); gates = s_k / sum_j s_j
+ *               (renormalize=1) or s_k.
+ *   num_groups, topk_groups: group-limited selection (2.3 of the same page:
+ *     group score = sum of the group's keys, keep the topk_groups best
+ *     groups, select the K experts inside them).  1,1 = no group limit.
+ *     E/num_groups must be a power of two.
+ *   num_shared: 0, or 1 always-on shared expert with gate 1 (slab E).
+ *   activation: MOE_ACT_GELU  E(x) = GeLU_erf(x W1 + b1) W2 + b2 (11.1.2);
+ *               MOE_ACT_SWIGLU E(x) = (SiLU(x Wg) * (x Wu)) Wd.
+ *   act_dtype: dtype of x, w_router, y and the intermediates (F32 or BF16).
+ *   weight_dtype: dtype of the expert weights (F32, BF16 or E4M3; E4M3
+ *     needs the per-output-channel scales s_gate, s_up, s_down).
+ *   capacity: 0 = unbounded; C > 0 = at most C rows per expert in the
+ *     primary block, the rest in an overflow region processed in a second
+ *     pass (ybb.press 2.2, overflow buffering).  No token is dropped.
+ * Supported: (F32 act, F32 weights, GELU) with E <= 32 on the SIMT path;
+ * (BF16 act, BF16 or E4M3 weights, SWIGLU or GELU) on the tensor-core path.
+ * E <= 256, K <= min(E, 16), d and h multiples of 8.
+ */
+typedef struct {
+  int32_t num_tokens;
+  int32_t d_model;
+  int32_t num_experts;
+  int32_t top_k;
+  int32_t d_ff;
+  int32_t score_fn;
+  int32_t renormalize;
+  int32_t num_groups;
+  int32_t topk_groups;
+  int32_t num_shared;
+  int32_t activation;
+  int32_t act_dtype;
+  int32_t weight_dtype;
+  int32_t capacity;
+} moe_desc;
+
+/* Weights, all DEVICE pointers (see layouts above).  Unused ones may be
+ * NULL: router_bias (added to the logits, so it also moves the gates),
+ * sel_bias (added to the selection keys only), b1/b2 (GELU only),
+ * s_gate/s_up/s_down (E4M3 only, fp32 [E+ns][h], [E+ns][h], [E+ns][d]). */
+typedef struct {
+  const void *w_router;
+  const float *router_bias;
+  const float *sel_bias;
+  const void *w1;
+  const float *b1;
+  const void *w2;
+  const float *b2;
+  const void *w_gate;
+  const void *w_up;
+  const void *w_down;
+  const float *s_gate;
+  const float *s_up;
+  const float *s_down;
+} moe_weights;
+
+/* Number of rows of the routed row space: S*K, or E*C + S*K with capacity
+ * (primary block of E*C rows, then the overflow region).  The shared expert,
+ * when present, adds S rows after them in the hidden and expert-output
+ * buffers.  Host only. */
+int64_t moe_routed_rows(const moe_desc *desc);
+
+/* Workspace bytes needed by moe_layer_forward for this desc (the standalone
+ * calls need no more).  Host only, no CUDA call. */
+moe_status moe_workspace_size(const moe_desc *desc, size_t *bytes);
+
+/* Zero the status block at the start of `ws` (stream-ordered). */
+moe_status moe_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Router logits + scoring + top-k (11.1.1; ybb.press 2.3; plumephp.com
+ * "MoE 混合专家推理", routing worked example).
+ *   x [S][d] act_dtype; logits_in: optional fp32 [S][E] logits used instead
+ *   of computing x W_r^T (router_bias is still added to them); x may then be
+ *   NULL.  Outputs topk_idx int32 [S][K] (descending key, ties to the lower
+ *   expert index; a non-finite key ranks lowest), topk_w fp32 [S][K].
+ */
+moe_status moe_route(const moe_desc *desc, const moe_weights *w, const void *x, const float *logits_in,
+                     int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Histogram, prefix scan and stable permutation (11.2.1 "数据重排").
+ *   topk_idx int32 [S][K] -> counts int32 [E];
+ *   offsets int32 [E+1] (exclusive prefix of counts), with capacity
+ *     [2(E+1)]: the first E+1 as before, then the exclusive prefix of the
+ *     overflow counts max(counts - C, 0);
+ *   row_of_slot int32 [S*K]: row of slot t*K+k; rows of one expert follow
+ *     slot order (stable); with capacity rows are e*C+r for r < C and
+ *     E*C + ovf_offset[e] + (r-C) otherwise;
+ *   token_of_row int32 [R] (R = moe_routed_rows), -1 for unused rows;
+ *   x_perm [R][d] act_dtype: x_perm[row_of_slot[t*K+k]] = x[t] (rows with
+ *     token_of_row = -1 are left untouched).  x and x_perm may be NULL to
+ *     compute only the maps.
+ */
+moe_status moe_permute(const moe_desc *desc, const void *x, const int32_t *topk_idx, int32_t *counts,
+                       int32_t *offsets, int32_t *row_of_slot, int32_t *token_of_row, void *x_perm, void *ws,
+                       size_t ws_bytes, void *stream);
+
+/*
+ * Grouped expert FFN (11.1.2: the S*K expert forwards grouped by expert).
+ *   x_perm [R][d] rows grouped as offsets describes (layout of moe_permute);
+ *   x [S][d]: A operand of the shared expert (NULL when num_shared = 0);
+ *   y_perm [R + ns*S][d] act_dtype: row r = E_{expert(r)}(x_perm[r]); rows
+ *     R .. R+S-1 hold the shared expert's output for token 0 .. S-1.
+ *   The hidden activations live in the workspace.  Rows outside any group
+ *   (unused capacity rows) are not written.
+ */
+moe_status moe_grouped_ffn(const moe_desc *desc, const moe_weights *w, const void *x_perm,
+                           const int32_t *offsets, const void *x, void *y_perm, void *ws, size_t ws_bytes,
+                           void *stream);
+
+/*
+ * Gate-weighted combine back into token order (11.3.1 step 6; plumephp.com
+ * worked example "结果按得分加权求和").
+ *   y[t] = sum_{k=0..K-1} topk_w[t][k] * y_perm[row_of_slot[t*K+k]]
+ *          (+ y_perm[R + t] when num_shared = 1), fp32 sums in k order.
+ *   y [S][d] act_dtype.
+ */
+moe_status moe_combine(const moe_desc *desc, const void *y_perm, const int32_t *row_of_slot,
+                       const float *topk_w, void *y, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * The whole layer: route -> permute -> grouped FFN -> combine, enqueued
+ * without any host synchronisation.  y [S][d] act_dtype.  topk_idx, topk_w
+ * and counts are optional outputs (NULL = keep them in the workspace).
+ */
+moe_status moe_layer_forward(const moe_desc *desc, const moe_weights *w, const void *x, void *y,
+                             int32_t *topk_idx, float *topk_w, int32_t *counts, void *ws, size_t ws_bytes,
+                             void *stream);
+
+/* Synchronise `stream`, copy the status block to the host.  flags: OR of
+ * MOE_STATUS_* bits; counters: MOE_NUM_COUNTERS int32 (may be NULL).
+ * Returns MOE_ERR_DEVICE_STATUS when any error bit is set. */
+moe_status moe_get_status(const void *ws, void *stream, uint32_t *flags, int32_t *counters);
+
+/* Static description of a status code. */
+const char *moe_strerror(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,399 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+None of these tests restates the oracle's own formulas: each compares it with
+a printed worked example, a brute-force enumeration, a closed form, a special
+case that reduces to a textbook routine, or an invariant stated on the pages.
+"""
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------------------
+# worked example (plumephp.com, routing worked example block)
+# ----------------------------------------------------------------------------
+
+
+def _worked_example():
+    with open(os.path.join(GOLDEN, "worked_example.json")) as f:
+        return json.load(f)
+
+
+def test_worked_example_top2_and_gates():
+    ex = _worked_example()
+    p = np.array(ex["probabilities"])
+    # any logits whose softmax is p: log p (softmax is shift invariant)
+    logits = np.log(p).astype(np.float32)[None, :]
+    idx, w = O.select_experts(logits, 2, renormalize=True)
+    assert idx[0].tolist() == ex["expected_top2"]
+    np.testing.assert_allclose(w[0], ex["expected_gates_normalised"], rtol=1e-6)
+    idx, w = O.select_experts(logits, 2, renormalize=False)
+    assert idx[0].tolist() == ex["expected_top2"]
+    np.testing.assert_allclose(w[0], ex["expected_gates_unnormalised"], rtol=1e-6)
+
+
+def test_worked_example_output_is_weighted_sum():
+    """Output = 0.55*e0(x) + 0.30*e3(x) (unnormalised) with experts whose
+    outputs are known in closed form: expert e maps x to (e + 1) * x."""
+    ex = _worked_example()
+    logits = np.log(np.array(ex["probabilities"])).astype(np.float32)[None, :]
+    x = np.array([[1.0, -2.0, 0.5]])
+    expert = lambda e, rows: (e + 1.0) * rows
+    for renorm, gates in ((False, ex["expected_gates_unnormalised"]), (True, ex["expected_gates_normalised"])):
+        idx, w = O.select_experts(logits, 2, renormalize=renorm)
+        y = O.moe_layer(x, idx, w, expert, 8)
+        expect = gates[0] * 1.0 * x + gates[1] * 4.0 * x  # e0 -> 1x, e3 -> 4x
+        np.testing.assert_allclose(y, expect, rtol=1e-6)
+
+
+# ----------------------------------------------------------------------------
+# top-k selection against brute force
+# ----------------------------------------------------------------------------
+
+
+def _brute_topk(keys_row, k, cand=None):
+    """Plain repeated selection: scan for the best remaining key (strict '>'
+    keeps the lower index on ties; NaN counts as -inf)."""
+    n = len(keys_row)
+    kv = [(-math.inf if math.isnan(float(v)) else float(v)) for v in keys_row]
+    taken = [False] * n
+    out = []
+    for _ in range(k):
+        best = -1
+        for j in range(n):
+            if taken[j] or (cand is not None and not cand[j]):
+                continue
+            if best < 0 or kv[j] > kv[best]:
+                best = j
+        taken[best] = True
+        out.append(best)
+    return out
+
+
+@pytest.mark.parametrize("E,K", [(8, 2), (64, 8), (256, 8), (5, 5), (32, 1)])
+def test_softmax_topk_matches_brute_force_with_ties(E, K):
+    rng = np.random.default_rng(E * 100 + K)
+    # small integer logits force many ties
+    logits = rng.integers(-3, 4, size=(40, E)).astype(np.float32)
+    logits[0, :] = 1.0  # all tied
+    logits[1, 0] = np.nan
+    logits[2, :] = -np.inf
+    idx, w = O.select_experts(logits, K)
+    for t in range(logits.shape[0]):
+        assert idx[t].tolist() == _brute_topk(logits[t], K), t
+    assert np.all(np.isfinite(w[3:]))
+    np.testing.assert_allclose(w[3:].sum(axis=1), 1.0, rtol=1e-12)
+
+
+def test_softmax_gates_textbook():
+    """Unnormalised gates equal the textbook softmax probability of each
+    chosen expert; normalised gates equal the softmax of the chosen logits."""
+    rng = np.random.default_rng(1)
+    l = rng.normal(size=(20, 8)).astype(np.float32)
+    idx, w = O.select_experts(l, 2, renormalize=False)
+    p = torch.softmax(torch.tensor(l, dtype=torch.float64), dim=1).numpy()
+    np.testing.assert_allclose(w, np.take_along_axis(p, idx, 1), rtol=1e-12)
+    idx2, w2 = O.select_experts(l, 2, renormalize=True)
+    assert (idx2 == idx).all()
+    sel = torch.tensor(np.take_along_axis(l, idx, 1), dtype=torch.float64)
+    np.testing.assert_allclose(w2, torch.softmax(sel, dim=1).numpy(), rtol=1e-12)
+    # TopK(-inf) then softmax over all E (chapter 11, 11.1.1 as written)
+    masked = np.full_like(l, -np.inf, dtype=np.float64)
+    np.put_along_axis(masked, idx, np.take_along_axis(l, idx, 1).astype(np.float64), 1)
+    pm = torch.softmax(torch.tensor(masked), dim=1).numpy()
+    np.testing.assert_allclose(w2, np.take_along_axis(pm, idx, 1), rtol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# group-limited sigmoid selection against brute-force enumeration
+# ----------------------------------------------------------------------------
+
+
+def test_grouped_selection_brute_force_dyadic():
+    """Keys on a coarse dyadic grid make every float32 sum exact, so the group
+    scores can be summed in any order.  The chosen groups must be the pair of
+    groups with the largest total among all C(8,2)=28 pairs (lexicographically
+    first on ties), and the top-8 the best keys inside them."""
+    rng = np.random.default_rng(7)
+    E, G, TG, K = 256, 8, 2, 8
+    gs = E // G
+    n_tok = 60
+    # sigmoid keys: choose the selection bias so that s + b lands on a grid
+    logits = rng.normal(size=(n_tok, E)).astype(np.float32)
+    s = O.sigmoid_f32(logits)
+    target = (rng.integers(0, 16, size=(n_tok, E)) / 16.0).astype(np.float32)
+    for t in range(n_tok):
+        # per-token bias is not allowed (bias is per expert), so check each
+        # token with its own bias vector
+        bias = (target[t] - s[t]).astype(np.float32)
+        keys = np.add(s[t], bias, dtype=np.float32)
+        idx, w = O.select_experts(logits[t:t + 1], K, score_fn="sigmoid", sel_bias=bias, num_groups=G,
+                                  topk_groups=TG)
+        gsum = [float(np.sum(keys[g * gs:(g + 1) * gs].astype(np.float64))) for g in range(G)]
+        best_pair = max(itertools.combinations(range(G), TG), key=lambda pr: (sum(gsum[g] for g in pr),
+                                                                              [-g for g in pr]))
+        cand = np.zeros(E, dtype=bool)
+        for g in best_pair:
+            cand[g * gs:(g + 1) * gs] = True
+        assert idx[0].tolist() == _brute_topk(keys, K, cand), t
+        assert all(cand[i] for i in idx[0])  # chosen experts lie inside chosen groups
+        # gates: unbiased sigmoid scores, normalised
+        sk = s[t][idx[0]].astype(np.float64)
+        np.testing.assert_allclose(w[0], sk / sk.sum(), rtol=1e-12)
+
+
+def test_group_sum_order_is_halving_tree():
+    """The float32 group score adds members (j, j+16), then (j, j+8), ...: for
+    values where order matters, compare with the hand-written tree of 4."""
+    v = np.array([1.0, 1e-8, -1.0, 1e-8], dtype=np.float32)
+    # halving: (1 + -1) , (1e-8 + 1e-8) -> 0 + 2e-8
+    assert O.group_sum_f32(v) == np.float32(np.float32(1e-8) + np.float32(1e-8))
+    # a left-to-right sum would give ((1 + 1e-8) - 1) + 1e-8 = 1e-8 in float32
+    assert O.group_sum_f32(v) != np.float32(1e-8)
+
+
+# ----------------------------------------------------------------------------
+# float32 sigmoid / exponential against the mathematics
+# ----------------------------------------------------------------------------
+
+
+def test_exp_f32_within_two_ulp_of_math_exp():
+    z = np.concatenate([np.linspace(-30, 88, 400001), np.array([0.0, 1.0, -1.0, 0.5])]).astype(np.float32)
+    e = O.exp_f32(z).astype(np.float64)
+    ref = np.array([math.exp(float(v)) for v in z[::37]])
+    ulp = np.spacing(ref.astype(np.float32)).astype(np.float64)
+    assert np.max(np.abs(e[::37] - ref) / ulp) <= 2.0
+    assert O.exp_f32(np.float32(0.0)) == 1.0
+
+
+def test_sigmoid_f32_special_values():
+    assert O.sigmoid_f32(np.float32(0.0)) == np.float32(0.5)
+    big = O.sigmoid_f32(np.array([100.0, -100.0, np.inf, -np.inf], dtype=np.float32))
+    assert big.tolist() == [1.0, 0.0, 1.0, 0.0]
+    x = np.linspace(-20, 20, 10001).astype(np.float32)
+    s = O.sigmoid_f32(x).astype(np.float64)
+    ref = 1.0 / (1.0 + np.exp(-x.astype(np.float64)))
+    assert np.max(np.abs(s - ref) / np.maximum(ref, 1e-30)) < 4e-7
+    assert np.all(np.diff(s) >= 0)  # monotone
+
+
+# ----------------------------------------------------------------------------
+# histogram, scan, permutation: invariants from the pages
+# ----------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("capacity", [0, 3, 1])
+def test_permutation_invariants(capacity):
+    rng = np.random.default_rng(3)
+    S, E, K = 50, 8, 3
+    logits = rng.normal(size=(S, E)).astype(np.float32)
+    logits[:, 2] += 2.0  # a hot expert
+    idx, _ = O.select_experts(logits, K)
+    P = O.expert_permutation(idx, E, capacity)
+    # every token goes to K experts (chapter 11, 11.1.2): counts sum to S*K
+    assert P["counts"].sum() == S * K
+    assert P["counts"].tolist() == [int((idx == e).sum()) for e in range(E)]
+    off = P["offsets"]
+    assert off[0] == 0 and off[-1] == S * K and np.all(np.diff(off) >= 0)
+    ros, tor = P["row_of_slot"], P["token_of_row"]
+    # bijection between slots and used rows; no token dropped (ybb.press 2.2)
+    assert len(set(ros.tolist())) == S * K
+    assert np.all(ros >= 0) and np.all(ros < P["num_rows"])
+    for slot in range(S * K):
+        assert tor[ros[slot]] == slot // K
+    assert (tor >= 0).sum() == S * K
+    # stable: within each expert, rows follow slot order
+    flat = idx.reshape(-1)
+    for e in range(E):
+        rows = ros[flat == e]
+        assert np.all(np.diff(rows) > 0)
+    if capacity:
+        C = capacity
+        assert np.all(P["prim_counts"] <= C)
+        assert (P["prim_counts"] + P["ovf_counts"] == P["counts"]).all()
+        for e in range(E):
+            rows = ros[flat == e]
+            prim = rows[rows < E * C]
+            assert np.all((prim >= e * C) & (prim < (e + 1) * C))
+    else:
+        for e in range(E):
+            rows = ros[flat == e]
+            assert np.all((rows >= off[e]) & (rows < off[e + 1]))
+
+
+def test_load_stats_uniform_and_skewed():
+    st = O.load_stats(np.array([4, 4, 4, 4]), 2, 8)
+    assert st["max_over_mean"] == 1.0 and st["std"] == 0.0
+    st = O.load_stats(np.array([13, 1, 1, 1]), 2, 8)  # max/mean = 13/4
+    assert st["max_over_mean"] == pytest.approx(3.25)
+
+
+# ----------------------------------------------------------------------------
+# experts: closed forms and special cases
+# ----------------------------------------------------------------------------
+
+
+def test_gelu_erf_textbook_values():
+    # GeLU(z) = z * Phi(z); Phi(1) = 0.8413447460685429 (normal table)
+    g = O.gelu_erf(np.array([0.0, 1.0, -1.0, 8.0, -8.0]))
+    np.testing.assert_allclose(g[:3], [0.0, 0.8413447460685429, -1 + 0.8413447460685429], rtol=1e-15, atol=1e-16)
+    assert g[3] == pytest.approx(8.0) and abs(g[4]) < 1e-12
+
+
+def test_silu_values():
+    s = O.silu(np.array([0.0, 1.0, -1.0]))
+    np.testing.assert_allclose(s, [0.0, 1 / (1 + math.exp(-1)), -1 / (1 + math.exp(1))], rtol=1e-15)
+
+
+def test_expert_gelu_one_hot_weights():
+    """W1 = identity-like, b1 = 0, W2 = identity, b2 = c: output is
+    GeLU(x) + c elementwise."""
+    d = 4
+    x = np.array([[0.5, -1.0, 2.0, 0.0]])
+    w1 = np.eye(d)
+    w2 = np.eye(d)
+    c = np.array([0.1, 0.2, 0.3, 0.4])
+    y = O.expert_gelu(x, w1, np.zeros(d), w2, c)
+    np.testing.assert_allclose(y, O.gelu_erf(x) + c, rtol=1e-15)
+    # W1 stored out x in: a permutation matrix routes input j to hidden p(j)
+    perm = np.eye(d)[[2, 0, 3, 1]]
+    y2 = O.expert_gelu(x, perm, np.zeros(d), np.eye(d), np.zeros(d))
+    np.testing.assert_allclose(y2[0], O.gelu_erf(x[0][[2, 0, 3, 1]]), rtol=1e-15)
+
+
+def test_expert_swiglu_closed_form():
+    """h=1: Wg row a, Wu row b, Wd column c -> y = silu(x.a) * (x.b) * c."""
+    x = np.array([[1.0, 2.0], [-1.0, 0.5]])
+    a, b, c = np.array([[0.5, -0.25]]), np.array([[1.0, 1.0]]), np.array([[2.0], [-3.0]])
+    y = O.expert_swiglu(x, a, b, c)
+    for t in range(2):
+        za, zb = float(x[t] @ a[0]), float(x[t] @ b[0])
+        hval = za / (1 + math.exp(-za)) * zb
+        np.testing.assert_allclose(y[t], [2.0 * hval, -3.0 * hval], rtol=1e-14)
+    # per-channel scales multiply the weight rows
+    y2 = O.expert_swiglu(x, a, b, c, s_gate=np.array([2.0]), s_up=np.array([0.5]), s_down=np.array([1.0, 1.0]))
+    y3 = O.expert_swiglu(x, 2 * a, 0.5 * b, c)
+    np.testing.assert_allclose(y2, y3, rtol=1e-14)
+
+
+def _rand_gelu_experts(rng, E, d, h):
+    w1 = rng.normal(size=(E, h, d)) / math.sqrt(d)
+    b1 = rng.normal(size=(E, h)) * 0.1
+    w2 = rng.normal(size=(E, d, h)) / math.sqrt(h)
+    b2 = rng.normal(size=(E, d)) * 0.1
+    return (lambda e, rows: O.expert_gelu(rows, w1[e], b1[e], w2[e], b2[e])), (w1, b1, w2, b2)
+
+
+def test_sparse_layer_equals_dense_then_mask():
+    rng = np.random.default_rng(11)
+    S, d, E, K, h = 30, 16, 8, 2, 24
+    fn, _ = _rand_gelu_experts(rng, E, d, h)
+    x = rng.normal(size=(S, d))
+    l = rng.normal(size=(S, E)).astype(np.float32)
+    idx, w = O.select_experts(l, K)
+    np.testing.assert_allclose(O.moe_layer(x, idx, w, fn, E), O.moe_layer_dense(x, idx, w, fn, E),
+                               rtol=1e-12, atol=1e-13)
+    # and through the permute/combine route with a shared expert
+    P = O.expert_permutation(idx, E)
+    y_rows = np.zeros((P["num_rows"], d))
+    for e in range(E):
+        rows = np.arange(P["offsets"][e], P["offsets"][e + 1])
+        if len(rows):
+            y_rows[rows] = fn(e, x[P["token_of_row"][rows]])
+    shared = fn(0, x)
+    np.testing.assert_allclose(O.combine(y_rows, P["row_of_slot"], w, shared),
+                               O.moe_layer(x, idx, w, fn, E, shared_fn=lambda z: fn(0, z)), rtol=1e-12,
+                               atol=1e-13)
+
+
+def test_single_expert_is_dense_ffn():
+    """E = 1, K = 1: the layer is the plain FFN of that expert (gate 1)."""
+    rng = np.random.default_rng(2)
+    fn, (w1, b1, w2, b2) = _rand_gelu_experts(rng, 1, 8, 12)
+    x = rng.normal(size=(5, 8))
+    idx, w = O.select_experts(rng.normal(size=(5, 1)).astype(np.float32), 1)
+    assert (idx == 0).all() and np.all(w == 1.0)
+    hid = x @ w1[0].T + b1[0]
+    hid = 0.5 * hid * (1 + np.vectorize(math.erf)(hid / math.sqrt(2)))
+    np.testing.assert_allclose(O.moe_layer(x, idx, w, fn, 1), hid @ w2[0].T + b2[0], rtol=1e-12)
+
+
+def test_k_equals_e_is_soft_routing():
+    """K = E with renormalised softmax gates is soft routing with tau = 1
+    (chapter 11, 11.3.3)."""
+    rng = np.random.default_rng(4)
+    S, d, E = 12, 8, 6
+    fn, _ = _rand_gelu_experts(rng, E, d, 10)
+    x = rng.normal(size=(S, d))
+    l = rng.normal(size=(S, E)).astype(np.float32)
+    idx, w = O.select_experts(l, E)
+    np.testing.assert_allclose(O.moe_layer(x, idx, w, fn, E), O.soft_routing(x, l, fn, E, 1.0), rtol=1e-12)
+
+
+def test_capacity_does_not_change_the_layer():
+    rng = np.random.default_rng(5)
+    S, d, E, K = 40, 8, 4, 2
+    fn, _ = _rand_gelu_experts(rng, E, d, 8)
+    x = rng.normal(size=(S, d))
+    l = rng.normal(size=(S, E)).astype(np.float32)
+    l[:, 1] += 3.0
+    idx, w = O.select_experts(l, K)
+    outs = []
+    for cap in (0, 5, 17):
+        P = O.expert_permutation(idx, E, cap)
+        y_rows = np.zeros((P["num_rows"], d))
+        tor = P["token_of_row"]
+        flat = idx.reshape(-1)
+        for slot in range(S * K):
+            y_rows[P["row_of_slot"][slot]] = fn(flat[slot], x[slot // K:slot // K + 1])[0]
+        assert (tor >= 0).sum() == S * K
+        outs.append(O.combine(y_rows, P["row_of_slot"], w))
+    np.testing.assert_allclose(outs[0], outs[1], rtol=1e-13)
+    np.testing.assert_allclose(outs[0], outs[2], rtol=1e-13)
+
+
+# ----------------------------------------------------------------------------
+# number formats against torch's converters (library routines)
+# ----------------------------------------------------------------------------
+
+
+def test_e4m3_decode_all_codes():
+    codes = np.arange(256, dtype=np.uint8)
+    mine = O.e4m3_bits_to_f64(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    both_nan = np.isnan(mine) & np.isnan(ref)
+    assert np.all(both_nan | (mine == ref))
+    assert mine[0x7E] == 448.0 and mine[0x38] == 1.0 and mine[0xB8] == -1.0 and mine[0x01] == 2.0 ** -9
+
+
+def test_bf16_round_trip_matches_torch():
+    rng = np.random.default_rng(9)
+    v = (rng.normal(size=4000) * np.exp(rng.normal(size=4000) * 5)).astype(np.float32)
+    v[:4] = [0.0, -0.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8]  # exact ties
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert (O.f64_to_bf16_bits(v.astype(np.float64)) == ref).all()
+    assert (O.f64_to_bf16_bits_fast(v.astype(np.float64)) == ref).all()
+    back = O.bf16_bits_to_f64(ref)
+    np.testing.assert_array_equal(back, torch.from_numpy(ref.view(np.int16)).view(torch.bfloat16).double().numpy())
+
+
+def test_router_logits_definition():
+    rng = np.random.default_rng(6)
+    x = rng.normal(size=(3, 5)).astype(np.float32)
+    w = rng.normal(size=(4, 5)).astype(np.float32)
+    b = np.array([0.5, 0.0, -0.5, 1.0], dtype=np.float32)
+    l = O.router_logits(x, w, b)
+    for t in range(3):
+        for e in range(4):
+            exact = math.fsum(float(x[t, k]) * float(w[e, k]) for k in range(5)) + float(b[e])
+            assert abs(float(l[t, e]) - exact) <= np.spacing(np.float32(abs(exact)))
