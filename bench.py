@@ -1,0 +1,413 @@
+"""Benchmark of the MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: the Mixtral-shaped prefill layer (S=4096 tokens, d=4096, E=8
+experts, top-2 softmax renormalised, SwiGLU experts h=14336, bf16 weights
+and activations, fp32 accumulation), synthetic seeded inputs resident in
+HBM.  A step is one layer forward (route -> permute -> grouped FFN ->
+combine) through the library's C ABI.  Expert weights (2.8 GB) exceed the
+126 MB L2, so no flush is needed between steps.
+
+Multi-GPU (torchrun): every rank runs an independent replica on its own S
+tokens (the layer has no exchange step on one node's data-parallel path);
+timing is the max over ranks, value = all ranks' tokens / that time.
+
+Also reported: per-stage times, the grouped-FFN roofline fraction against the
+measured bf16 tensor peak, the end-to-end number with host buffers (pinned
+host -> device copy of x, layer, device -> host copy of y inside the timed
+region), the decode sweep S in {1, 8, 32, 128} against the HBM roofline, and
+the CPU oracle timed on a bounded sample (rank 0 only).
+
+--impl reference times the CPU oracle as it stands (the only reference this
+layer has) on a bounded token sample per step and prints the same line with
+"impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from mixture_experts_layer_bias_b200 import ops  # noqa: E402
+from mixture_experts_layer_bias_b200 import synthetic as syn  # noqa: E402
+
+METRIC = "MoE-layer tokens/s (prefill & decode); % of TC peak or HBM roofline"
+WORKLOAD = "mixtral_prefill"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["source"] = "fallback"
+    return d
+
+
+def workload_desc(cfg):
+    return (f"{cfg.name}: S={cfg.S} d={cfg.d} E={cfg.E} K={cfg.K} h={cfg.h} "
+            f"{'SwiGLU' if cfg.activation == syn.SWIGLU else 'GeLU'} "
+            f"{'bf16' if cfg.act_dtype == syn.BF16 else 'fp32'} act, "
+            f"{ {0: 'fp32', 1: 'bf16', 2: 'e4m3'}[cfg.weight_dtype]} weights")
+
+
+def kernels_per_step(cfg):
+    """Launches of this library's kernels in one layer forward."""
+    n = 1 if (cfg.E <= 32) else 2          # route (fused) or logits + top-k
+    n += 3                                 # count, scan, scatter+gather
+    n += 1 + 2                             # group table, up and down GEMM
+    if cfg.weight_dtype == syn.E4M3:
+        n += 3                             # E4M3 -> bf16 decode of the three stacks
+    if cfg.capacity:
+        n += 2                             # overflow pass
+    n += 1                                 # combine
+    return n
+
+
+def expert_flops(cfg, rows):
+    per_row = (6 if cfg.activation == syn.SWIGLU else 4) * cfg.d * cfg.h
+    return rows * per_row
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            gid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={gid}", "--query-gpu=" + ",".join(self.FIELDS),
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def make_layer_inputs(cfg, device):
+    inp = syn.make_inputs(cfg, device, seed=0)
+    return inp
+
+
+def time_stages(cfg, inp, desc, ws, bufs, steps, warmup):
+    """Run `warmup` + `steps` layer forwards as the four stage calls, with
+    CUDA events between them on the launching stream.  Returns per-step ms
+    and per-stage mean ms."""
+    st = torch.cuda.current_stream()
+    w = ops.make_weights(inp)
+    x = inp["x"]
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(st)
+        ops.moe_route(desc, w, x, None, bufs["idx"], bufs["gw"], ws)
+        if ev is not None:
+            ev[1].record(st)
+        ops.moe_permute(desc, x, bufs["idx"], bufs["counts"], bufs["offsets"], bufs["ros"], bufs["tor"],
+                        bufs["xp"], ws)
+        if ev is not None:
+            ev[2].record(st)
+        ops.moe_grouped_ffn(desc, w, bufs["xp"], bufs["offsets"], x, bufs["yp"], ws)
+        if ev is not None:
+            ev[3].record(st)
+        ops.moe_combine(desc, bufs["yp"], bufs["ros"], bufs["gw"], bufs["y"], ws)
+        if ev is not None:
+            ev[4].record(st)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    return step, evs
+
+
+def alloc_bufs(cfg, desc, S, device):
+    R = ops.moe_routed_rows(desc)
+    Rt = R + cfg.num_shared * S
+    adt = torch.bfloat16 if cfg.act_dtype == syn.BF16 else torch.float32
+    return dict(idx=torch.empty((S, cfg.K), dtype=torch.int32, device=device),
+                gw=torch.empty((S, cfg.K), dtype=torch.float32, device=device),
+                counts=torch.empty((cfg.E,), dtype=torch.int32, device=device),
+                offsets=torch.empty((2 * (cfg.E + 1),), dtype=torch.int32, device=device),
+                ros=torch.empty((S * cfg.K,), dtype=torch.int32, device=device),
+                tor=torch.empty((max(R, 1),), dtype=torch.int32, device=device),
+                xp=torch.empty((max(R, 1), cfg.d), dtype=adt, device=device),
+                yp=torch.empty((max(Rt, 1), cfg.d), dtype=adt, device=device),
+                y=torch.empty((S, cfg.d), dtype=adt, device=device))
+
+
+def decode_sweep(base_inp, device, peaks, reps=20):
+    """Decode-regime calls S in {1, 8, 32, 128} on the prefill weights with
+    the decode router offsets, captured in a CUDA graph; reports us per call,
+    tokens/s and the HBM fraction of the expert weights touched."""
+    out = {}
+    dcfg0 = syn.CONFIGS["mixtral_decode"]
+    for S in syn.DECODE_SIZES:
+        cfg = syn.scaled(dcfg0, S=S)
+        dinp = syn.make_inputs(cfg, device, seed=0, x_only=True)
+        inp = dict(base_inp)
+        inp["x"] = dinp["x"]
+        inp["router_bias"] = syn.router_offsets(cfg, seed=0).to(device)
+        desc = ops.make_desc(**syn.desc_dict(cfg, S))
+        ws = torch.empty(ops.moe_workspace_size(desc), dtype=torch.uint8, device=device)
+        ops.moe_workspace_init(ws)
+        w = ops.make_weights(inp)
+        y = torch.empty((S, cfg.d), dtype=torch.bfloat16, device=device)
+        counts = torch.empty((cfg.E,), dtype=torch.int32, device=device)
+        s = torch.cuda.Stream()
+        with torch.cuda.stream(s):
+            for _ in range(3):
+                ops.moe_layer_forward(desc, w, inp["x"], y, None, None, counts, ws, s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            ops.moe_layer_forward(desc, w, inp["x"], y, None, None, counts, ws, s)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / reps
+        touched = int((counts > 0).sum().item())
+        wbytes = touched * 3 * cfg.d * cfg.h * 2
+        gbs = wbytes / (us * 1e-6) / 1e9
+        out[str(S)] = {"us_per_call": round(us, 2), "tokens_per_s": round(S / (us * 1e-6), 1),
+                       "experts_touched": touched, "weight_bytes": wbytes, "hbm_gbs": round(gbs, 1),
+                       "hbm_frac": round(gbs / peaks["hbm_gbs"], 3)}
+        del g
+    return out
+
+
+def cpu_baseline(cfg, inp, n_tokens=32):
+    """The CPU oracle as it stands on a fixed sample of tokens."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from parity import oracle_layer
+
+    toks = np.arange(n_tokens)
+    t0 = time.perf_counter()
+    oracle_layer(inp, cfg, toks)
+    dt = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return {"value": round(n_tokens / dt, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n_tokens} tokens of {cfg.name} (routing + their experts' SwiGLU FFN in float64), "
+                      f"{dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    cfg = syn.CONFIGS[WORKLOAD]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_layer_inputs(cfg, dev)
+    n_tok = 8
+    import numpy as np
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from threadpoolctl import threadpool_info
+
+    from parity import oracle_layer
+
+    for i in range(args.warmup):
+        oracle_layer(inp, cfg, np.arange(i * n_tok, (i + 1) * n_tok))
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle_layer(inp, cfg, np.arange(i * n_tok, (i + 1) * n_tok) % cfg.S)
+    dt = time.perf_counter() - t0
+    value = n_tok * args.steps / dt
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": workload_desc(cfg), "global_batch": cfg.S,
+                                            "seq_len": cfg.S, "parallelism": "none (CPU oracle)"},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{n_tok} tokens per step of {cfg.name}"},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = world > 1
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if dist:
+        import datetime
+
+        import torch.distributed as td
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    peaks = load_peaks()
+    cfg = syn.CONFIGS[WORKLOAD]
+    S = cfg.S
+    inp = make_layer_inputs(cfg, device)
+    desc = ops.make_desc(**syn.desc_dict(cfg, S))
+    ws = torch.empty(ops.moe_workspace_size(desc), dtype=torch.uint8, device=device)
+    ops.moe_workspace_init(ws)
+    bufs = alloc_bufs(cfg, desc, S, device)
+    step, evs = time_stages(cfg, inp, desc, ws, bufs, args.steps, args.warmup)
+
+    clocks = ClockSampler(local)
+    if dist:
+        td.barrier()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(args.steps):
+        step(evs[i])
+    stop.record()
+    torch.cuda.synchronize()
+    if dist:
+        td.barrier()
+    clk = clocks.stop()
+    total_ms = start.elapsed_time(stop)
+    if dist:
+        t = torch.tensor([total_ms], device=device)
+        td.all_reduce(t, op=td.ReduceOp.MAX)
+        total_ms = float(t.item())
+    stage_names = ("route", "permute", "grouped_ffn", "combine")
+    stages = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
+              for j, n in enumerate(stage_names)}
+    ms_per_step = total_ms / args.steps
+    value = world * S * args.steps / (total_ms * 1e-3)
+
+    code, flags, counters = ops.moe_get_status(ws)
+    if flags:
+        raise RuntimeError(f"device status flags {flags} {counters}")
+
+    # roofline of the dominant stage: the grouped expert FFN (both GEMMs)
+    rows = S * cfg.K + cfg.num_shared * S
+    flops = expert_flops(cfg, rows)
+    ffn_ms = stages["grouped_ffn"]
+    achieved = flops / (ffn_ms * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": None,
+                "kernel": "grouped expert FFN (up SwiGLU + down GEMMs, tcgen05)",
+                "peak_source": f"{peaks['source']} bf16 burst"}
+
+    # end to end through the public call with host buffers
+    x_host = inp["x"].cpu().pin_memory()
+    y_host = torch.empty((S, cfg.d), dtype=x_host.dtype).pin_memory()
+    x_dev = torch.empty_like(inp["x"])
+    layer_w = ops.make_weights(inp)
+    e2e_ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        ops.moe_layer_forward(desc, layer_w, x_dev, bufs["y"], None, None, None, ws)
+        y_host.copy_(bufs["y"], non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        td.barrier()
+    e2e_ev[0].record()
+    for _ in range(args.steps):
+        e2e_step()
+    e2e_ev[1].record()
+    torch.cuda.synchronize()
+    e2e_ms = e2e_ev[0].elapsed_time(e2e_ev[1])
+    if dist:
+        t = torch.tensor([e2e_ms], device=device)
+        td.all_reduce(t, op=td.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": round(world * S * args.steps / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+           "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+           "d2h_bytes_per_step": y_host.numel() * y_host.element_size()}
+
+    dec = None
+    if not args.no_decode:
+        dec = decode_sweep(inp, device, peaks)
+    if dist:
+        td.barrier()
+        td.destroy_process_group()
+    if rank != 0:
+        return
+    cpu = None
+    if not args.no_cpu and world == 1:
+        cpu = cpu_baseline(cfg, inp)
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": workload_desc(cfg), "global_batch": world * S, "seq_len": S,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "no flush: 2.8 GB of expert weights per step exceed the 126 MB L2"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": kernels_per_step(cfg) * args.steps, "clocks": clk,
+            "stages_ms": {k: round(v, 4) for k, v in stages.items()}, "decode_sweep": dec,
+            "counters": counters}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

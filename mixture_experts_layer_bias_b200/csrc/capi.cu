@@ -1,0 +1,439 @@
+// C ABI of the MoE layer forward: argument checks, workspace layout and the
+// launch sequence (declarations and contracts in include/moe.h).
+//
+// The layer follows jsqmd.com "第11章 MoE模型推理" 11.1.1-11.1.2 and 11.2.1:
+// route (router + TopK), regroup the S*K token slots by expert, run each
+// expert's FFN over its rows as one grouped GEMM, restore token order with
+// the gate-weighted sum.  Nothing here allocates or synchronises (except
+// moe_get_status); every launch goes to the caller's stream.
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
+
+struct Layout {
+  size_t status, logits, chunk_hist, groups1, groups2, counts, offsets, topk_idx, topk_w, row_of_slot, token_of_row,
+      x_perm, hidden, y_perm, wdeq, total;
+};
+
+int64_t routed_rows(const moe_desc& d) {
+  const int64_t sk = static_cast<int64_t>(d.num_tokens) * d.top_k;
+  return d.capacity > 0 ? static_cast<int64_t>(d.num_experts) * d.capacity + sk : sk;
+}
+
+size_t act_bytes(const moe_desc& d) { return d.act_dtype == MOE_F32 ? 4 : 2; }
+
+Layout make_layout(const moe_desc& d) {
+  Layout L;
+  const int64_t S = d.num_tokens, E = d.num_experts, K = d.top_k, h = d.d_ff, dm = d.d_model;
+  const int64_t R = routed_rows(d);
+  const int64_t Rt = R + static_cast<int64_t>(d.num_shared) * S;
+  const int64_t nch = permute_num_chunks(static_cast<int>(S), static_cast<int>(K));
+  const size_t ab = act_bytes(d);
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes);
+    return at;
+  };
+  L.status = take(kAlign);
+  L.logits = take(E > 32 ? static_cast<size_t>(S * E) * 4 : 0);
+  L.chunk_hist = take(static_cast<size_t>(nch * E) * 4);
+  L.groups1 = take(static_cast<size_t>(E + 1) * sizeof(GroupEntry));
+  L.groups2 = take(static_cast<size_t>(E) * sizeof(GroupEntry));
+  L.counts = take(static_cast<size_t>(E) * 4);
+  L.offsets = take(static_cast<size_t>(2 * (E + 1)) * 4);
+  L.topk_idx = take(static_cast<size_t>(S * K) * 4);
+  L.topk_w = take(static_cast<size_t>(S * K) * 4);
+  L.row_of_slot = take(static_cast<size_t>(S * K) * 4);
+  L.token_of_row = take(static_cast<size_t>(R) * 4);
+  L.x_perm = take(static_cast<size_t>(R * dm) * ab);
+  L.hidden = take(static_cast<size_t>(Rt * h) * ab);
+  L.y_perm = take(static_cast<size_t>(Rt * dm) * ab);
+  L.wdeq = take(d.weight_dtype == MOE_E4M3 ? static_cast<size_t>((E + d.num_shared) * 3 * h * dm) * 2 : 0);
+  L.total = o;
+  return L;
+}
+
+bool is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+moe_status validate(const moe_desc* d) {
+  if (d == nullptr) return MOE_ERR_INVALID_ARG;
+  if (d->num_tokens < 0 || d->d_model <= 0 || d->d_model % 8 != 0 || d->d_ff <= 0 || d->d_ff % 8 != 0)
+    return MOE_ERR_INVALID_ARG;
+  if (d->num_experts < 1 || d->num_experts > 256) return MOE_ERR_INVALID_ARG;
+  if (d->top_k < 1 || d->top_k > d->num_experts || d->top_k > 32) return MOE_ERR_INVALID_ARG;
+  if (d->score_fn != MOE_SCORE_SOFTMAX && d->score_fn != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (d->renormalize != 0 && d->renormalize != 1) return MOE_ERR_INVALID_ARG;
+  if (d->num_groups < 1 || d->num_experts % d->num_groups != 0) return MOE_ERR_INVALID_ARG;
+  if (d->topk_groups < 1 || d->topk_groups > d->num_groups) return MOE_ERR_INVALID_ARG;
+  const int gs = d->num_experts / d->num_groups;
+  if (d->num_groups > 1 && !is_pow2(gs)) return MOE_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(d->topk_groups) * gs < d->top_k) return MOE_ERR_INVALID_ARG;
+  if (d->num_shared != 0 && d->num_shared != 1) return MOE_ERR_INVALID_ARG;
+  if (d->activation != MOE_ACT_GELU && d->activation != MOE_ACT_SWIGLU) return MOE_ERR_INVALID_ARG;
+  if (d->act_dtype != MOE_F32 && d->act_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (d->weight_dtype != MOE_F32 && d->weight_dtype != MOE_BF16 && d->weight_dtype != MOE_E4M3)
+    return MOE_ERR_INVALID_ARG;
+  if (d->capacity < 0) return MOE_ERR_INVALID_ARG;
+  // row indices are int32 on the device
+  const int64_t rows = routed_rows(*d) + static_cast<int64_t>(d->num_shared) * d->num_tokens;
+  if (rows > (int64_t(1) << 31) - 1) return MOE_ERR_INVALID_ARG;
+  // implemented combinations
+  if (d->act_dtype == MOE_F32) {
+    if (d->weight_dtype != MOE_F32 || d->activation != MOE_ACT_GELU) return MOE_ERR_UNSUPPORTED;
+  } else {
+    if (d->weight_dtype == MOE_F32) return MOE_ERR_UNSUPPORTED;
+    if (d->weight_dtype == MOE_E4M3 && d->activation != MOE_ACT_SWIGLU) return MOE_ERR_UNSUPPORTED;
+  }
+  return MOE_OK;
+}
+
+moe_status check_ws(const moe_desc& d, const void* ws, size_t ws_bytes) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < make_layout(d).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// SM count of the current device, queried once per device ordinal.
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 64 && cache[dev] > 0) return cache[dev];
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  if (dev < 64) cache[dev] = n;
+  return n;
+}
+
+moe_status route_impl(const moe_desc& d, const moe_weights* w, const void* x, const float* logits_in,
+                      int32_t* topk_idx, float* topk_w, void* ws, cudaStream_t st) {
+  const Layout L = make_layout(d);
+  RouteArgs a{};
+  a.S = d.num_tokens;
+  a.d = d.d_model;
+  a.E = d.num_experts;
+  a.K = d.top_k;
+  a.score_fn = d.score_fn;
+  a.renormalize = d.renormalize;
+  a.num_groups = d.num_groups;
+  a.topk_groups = d.topk_groups;
+  a.act_dtype = d.act_dtype;
+  a.x = x;
+  a.w_router = w != nullptr ? w->w_router : nullptr;
+  a.logits = logits_in;
+  a.logits_scratch = at<float>(ws, L.logits);
+  a.router_bias = w != nullptr ? w->router_bias : nullptr;
+  a.sel_bias = w != nullptr ? w->sel_bias : nullptr;
+  a.topk_idx = topk_idx;
+  a.topk_w = topk_w;
+  a.status = at<StatusBlock>(ws, L.status);
+  return cuda_status(launch_route(a, st));
+}
+
+moe_status permute_impl(const moe_desc& d, const void* x, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                        int32_t* row_of_slot, int32_t* token_of_row, void* x_perm, void* ws, cudaStream_t st) {
+  const Layout L = make_layout(d);
+  PermuteArgs a{};
+  a.S = d.num_tokens;
+  a.d = d.d_model;
+  a.E = d.num_experts;
+  a.K = d.top_k;
+  a.capacity = d.capacity;
+  a.act_dtype = d.act_dtype;
+  a.topk_idx = topk_idx;
+  a.chunk_hist = at<int32_t>(ws, L.chunk_hist);
+  a.counts = counts;
+  a.offsets = offsets;
+  a.row_of_slot = row_of_slot;
+  a.token_of_row = token_of_row;
+  a.x = x;
+  a.x_perm = x_perm;
+  a.num_rows = routed_rows(d);
+  a.status = at<StatusBlock>(ws, L.status);
+  return cuda_status(launch_permute(a, st));
+}
+
+moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm, const int32_t* offsets, const void* x,
+                    void* y_perm, void* ws, cudaStream_t st) {
+  const Layout L = make_layout(d);
+  const int S = d.num_tokens, E = d.num_experts, h = d.d_ff, dm = d.d_model;
+  if (S == 0) return MOE_OK;
+  const int64_t R = routed_rows(d);
+  const int64_t Rt = R + static_cast<int64_t>(d.num_shared) * S;
+  StatusBlock* status = at<StatusBlock>(ws, L.status);
+  GroupEntry* g1 = at<GroupEntry>(ws, L.groups1);
+  GroupEntry* g2 = at<GroupEntry>(ws, L.groups2);
+  cudaError_t err = launch_build_groups(S, E, d.top_k, d.capacity, d.num_shared, offsets, g1, g2, status, st);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  const int slabs = E + d.num_shared;
+  void* hidden = at<void>(ws, L.hidden);
+
+  GemmArgs up{};
+  up.groups = g1;
+  up.num_groups = E + d.num_shared;
+  up.shared_slab = d.num_shared ? E : -1;
+  up.a_rows_from_out = 0;
+  up.a = x_perm;
+  up.a_rows = R;
+  up.a_shared = d.num_shared ? x : nullptr;
+  up.a_shared_rows = d.num_shared ? S : 0;
+  up.n_per_slab = h;
+  up.b_rows = static_cast<int64_t>(slabs) * h;
+  up.N = h;
+  up.K = dm;
+  up.out = hidden;
+  up.out_rows = Rt;
+  up.out_f32 = d.act_dtype == MOE_F32;
+  up.max_total_rows = static_cast<int64_t>(S) * d.top_k + static_cast<int64_t>(d.num_shared) * S;
+  up.max_group_rows = S;
+  up.status = status;
+
+  GemmArgs down = up;
+  down.a_rows_from_out = 1;
+  down.shared_slab = -1;
+  down.a = hidden;
+  down.a_rows = Rt;
+  down.a_shared = nullptr;
+  down.a_shared_rows = 0;
+  down.n_per_slab = dm;
+  down.b_rows = static_cast<int64_t>(slabs) * dm;
+  down.N = dm;
+  down.K = h;
+  down.out = y_perm;
+
+  if (d.act_dtype == MOE_F32) {
+    up.epilogue = EPI_GELU_BIAS;
+    up.b0 = w.w1;
+    up.bias = w.b1;
+    down.epilogue = EPI_BIAS;
+    down.b0 = w.w2;
+    down.bias = w.b2;
+  } else {
+    const void *wg = w.w_gate, *wu = w.w_up, *wd = w.w_down, *w1 = w.w1, *w2 = w.w2;
+    if (d.weight_dtype == MOE_E4M3) {
+      // exact E4M3 -> bf16 decode of this call's weights; the per-channel
+      // scales are applied to the fp32 accumulators in the epilogues
+      const int64_t n_up = static_cast<int64_t>(slabs) * h * dm;
+      char* base = at<char>(ws, L.wdeq);
+      void* dg = base;
+      void* du = base + n_up * 2;
+      void* dd = base + 2 * n_up * 2;
+      if ((err = launch_dequant_e4m3(static_cast<const uint8_t*>(wg), dg, n_up, st)) != cudaSuccess ||
+          (err = launch_dequant_e4m3(static_cast<const uint8_t*>(wu), du, n_up, st)) != cudaSuccess ||
+          (err = launch_dequant_e4m3(static_cast<const uint8_t*>(wd), dd, n_up, st)) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      wg = dg;
+      wu = du;
+      wd = dd;
+      up.scale0 = w.s_gate;
+      up.scale1 = w.s_up;
+      down.scale0 = w.s_down;
+    }
+    if (d.activation == MOE_ACT_SWIGLU) {
+      up.epilogue = EPI_SWIGLU;
+      up.b0 = wg;
+      up.b1 = wu;
+      down.epilogue = EPI_NONE;
+      down.b0 = wd;
+    } else {
+      up.epilogue = EPI_GELU_BIAS;
+      up.b0 = w1;
+      up.bias = w.b1;
+      down.epilogue = EPI_BIAS;
+      down.b0 = w2;
+      down.bias = w.b2;
+    }
+  }
+  const int sms = num_sms();
+  auto run = [&](const GemmArgs& g) {
+    return d.act_dtype == MOE_F32 ? launch_grouped_gemm_f32(g, st) : launch_grouped_gemm_tc(g, sms, st);
+  };
+  if ((err = run(up)) != cudaSuccess || (err = run(down)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (d.capacity > 0) {
+    // second pass: the overflow rows, grouped by expert the same way
+    GemmArgs up2 = up, down2 = down;
+    up2.groups = down2.groups = g2;
+    up2.num_groups = down2.num_groups = E;
+    up2.shared_slab = -1;
+    up2.a_shared = nullptr;
+    up2.a_shared_rows = 0;
+    up2.max_total_rows = down2.max_total_rows = static_cast<int64_t>(S) * d.top_k;
+    if ((err = run(up2)) != cudaSuccess || (err = run(down2)) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+moe_status combine_impl(const moe_desc& d, const void* y_perm, const int32_t* row_of_slot, const float* topk_w,
+                        void* y, cudaStream_t st) {
+  CombineArgs a{};
+  a.S = d.num_tokens;
+  a.d = d.d_model;
+  a.K = d.top_k;
+  a.act_dtype = d.act_dtype;
+  a.y_perm = y_perm;
+  a.row_of_slot = row_of_slot;
+  a.topk_w = topk_w;
+  a.shared_row0 = d.num_shared ? routed_rows(d) : -1;
+  a.y = y;
+  return cuda_status(launch_combine(a, st));
+}
+
+bool weights_ok(const moe_desc& d, const moe_weights* w) {
+  if (w == nullptr) return false;
+  if (d.act_dtype == MOE_F32 || d.activation == MOE_ACT_GELU) {
+    if (!w->w1 || !w->w2 || !w->b1 || !w->b2) return false;
+  } else {
+    if (!w->w_gate || !w->w_up || !w->w_down) return false;
+    if (d.weight_dtype == MOE_E4M3 && (!w->s_gate || !w->s_up || !w->s_down)) return false;
+  }
+  const void* ps[] = {w->w1, w->w2, w->w_gate, w->w_up, w->w_down};
+  for (const void* p : ps)
+    if (p && !aligned16(p)) return false;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t moe_routed_rows(const moe_desc* desc) {
+  if (validate(desc) != MOE_OK) return -1;
+  return routed_rows(*desc);
+}
+
+moe_status moe_workspace_size(const moe_desc* desc, size_t* bytes) {
+  moe_status s = validate(desc);
+  if (s != MOE_OK) return s;
+  if (bytes == nullptr) return MOE_ERR_INVALID_ARG;
+  *bytes = make_layout(*desc).total;
+  return MOE_OK;
+}
+
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (ws == nullptr || ws_bytes < kAlign || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0)
+    return MOE_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(ws, 0, kAlign, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_route(const moe_desc* desc, const moe_weights* w, const void* x, const float* logits_in,
+                     int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+  moe_status s = validate(desc);
+  if (s != MOE_OK) return s;
+  if ((s = check_ws(*desc, ws, ws_bytes)) != MOE_OK) return s;
+  if (desc->num_tokens == 0) return MOE_OK;
+  if (topk_idx == nullptr || topk_w == nullptr) return MOE_ERR_INVALID_ARG;
+  if (logits_in == nullptr) {
+    if (x == nullptr || w == nullptr || w->w_router == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w->w_router)) return MOE_ERR_INVALID_ARG;
+  }
+  return route_impl(*desc, w, x, logits_in, topk_idx, topk_w, ws, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_permute(const moe_desc* desc, const void* x, const int32_t* topk_idx, int32_t* counts,
+                       int32_t* offsets, int32_t* row_of_slot, int32_t* token_of_row, void* x_perm, void* ws,
+                       size_t ws_bytes, void* stream) {
+  moe_status s = validate(desc);
+  if (s != MOE_OK) return s;
+  if ((s = check_ws(*desc, ws, ws_bytes)) != MOE_OK) return s;
+  if (counts == nullptr || offsets == nullptr || row_of_slot == nullptr || token_of_row == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (desc->num_tokens > 0 && topk_idx == nullptr) return MOE_ERR_INVALID_ARG;
+  if ((x == nullptr) != (x_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (x && (!aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+  return permute_impl(*desc, x, topk_idx, counts, offsets, row_of_slot, token_of_row, x_perm, ws,
+                      static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_grouped_ffn(const moe_desc* desc, const moe_weights* w, const void* x_perm, const int32_t* offsets,
+                           const void* x, void* y_perm, void* ws, size_t ws_bytes, void* stream) {
+  moe_status s = validate(desc);
+  if (s != MOE_OK) return s;
+  if ((s = check_ws(*desc, ws, ws_bytes)) != MOE_OK) return s;
+  if (desc->num_tokens == 0) return MOE_OK;
+  if (!weights_ok(*desc, w) || x_perm == nullptr || offsets == nullptr || y_perm == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (desc->num_shared && x == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_perm) || !aligned16(y_perm) || (x && !aligned16(x))) return MOE_ERR_INVALID_ARG;
+  return ffn_impl(*desc, *w, x_perm, offsets, x, y_perm, ws, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_combine(const moe_desc* desc, const void* y_perm, const int32_t* row_of_slot, const float* topk_w,
+                       void* y, void* ws, size_t ws_bytes, void* stream) {
+  moe_status s = validate(desc);
+  if (s != MOE_OK) return s;
+  if ((s = check_ws(*desc, ws, ws_bytes)) != MOE_OK) return s;
+  if (desc->num_tokens == 0) return MOE_OK;
+  if (y_perm == nullptr || row_of_slot == nullptr || topk_w == nullptr || y == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_perm) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  return combine_impl(*desc, y_perm, row_of_slot, topk_w, y, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_layer_forward(const moe_desc* desc, const moe_weights* w, const void* x, void* y, int32_t* topk_idx,
+                             float* topk_w, int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  moe_status s = validate(desc);
+  if (s != MOE_OK) return s;
+  if ((s = check_ws(*desc, ws, ws_bytes)) != MOE_OK) return s;
+  const moe_desc& d = *desc;
+  if (d.num_tokens == 0) return MOE_OK;
+  if (x == nullptr || y == nullptr || !aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  if (!weights_ok(d, w) || w->w_router == nullptr || !aligned16(w->w_router)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Layout L = make_layout(d);
+  int32_t* idx = topk_idx ? topk_idx : at<int32_t>(ws, L.topk_idx);
+  float* gates = topk_w ? topk_w : at<float>(ws, L.topk_w);
+  int32_t* cnt = counts ? counts : at<int32_t>(ws, L.counts);
+  int32_t* offs = at<int32_t>(ws, L.offsets);
+  int32_t* ros = at<int32_t>(ws, L.row_of_slot);
+  int32_t* tor = at<int32_t>(ws, L.token_of_row);
+  void* x_perm = at<void>(ws, L.x_perm);
+  void* y_perm = at<void>(ws, L.y_perm);
+  if ((s = route_impl(d, w, x, nullptr, idx, gates, ws, st)) != MOE_OK) return s;
+  if ((s = permute_impl(d, x, idx, cnt, offs, ros, tor, x_perm, ws, st)) != MOE_OK) return s;
+  if ((s = ffn_impl(d, *w, x_perm, offs, x, y_perm, ws, st)) != MOE_OK) return s;
+  return combine_impl(d, y_perm, ros, gates, y, st);
+}
+
+moe_status moe_get_status(const void* ws, void* stream, uint32_t* flags, int32_t* counters) {
+  if (ws == nullptr) return MOE_ERR_WORKSPACE;
+  StatusBlock host;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpy(&host, ws, sizeof(host), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (flags) *flags = host.flags;
+  if (counters) memcpy(counters, host.counters, sizeof(host.counters));
+  const uint32_t errors = MOE_STATUS_NONFINITE_LOGIT | MOE_STATUS_BAD_EXPERT_ID | MOE_STATUS_TIMEOUT |
+                          MOE_STATUS_BAD_GROUP;
+  return (host.flags & errors) ? MOE_ERR_DEVICE_STATUS : MOE_OK;
+}
+
+const char* moe_strerror(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported combination";
+    case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_STATUS: return "device reported a data error (see moe_get_status)";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,112 @@
+// Gate-weighted combine back into token order, and the FP8 weight decode.
+//
+// jsqmd.com "第11章 MoE模型推理" 11.3.1 step 6 (weighted sum of the K expert
+// outputs by the top-k probabilities) and 11.2.1 (outputs restored to the
+// original token order); plumephp.com "MoE 混合专家推理", worked example:
+// output = 0.55 * e0(x) + 0.30 * e3(x), normalised.
+//
+// One warp per token; lanes stride over 16-byte vectors of the d_model row;
+// fp32 sums in k order, then the shared expert's row (gate 1), one rounding
+// to the output type at the end.
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kCombWarps = 8;
+
+template <typename T>
+__global__ void __launch_bounds__(kCombWarps * 32)
+    combine_kernel(int S, int d, int K, const T* __restrict__ y_perm, const int32_t* __restrict__ row_of_slot,
+                   const float* __restrict__ topk_w, int64_t shared_row0, T* __restrict__ y) {
+  const int t = blockIdx.x * kCombWarps + (threadIdx.x >> 5);
+  if (t >= S) return;
+  const int lane = lane_id();
+  constexpr int V = Vec16<T>::N;
+  const int nvec = d / V;
+  // row indices and gates of this token, one per lane (K <= 32)
+  int my_row = -1;
+  float my_g = 0.0f;
+  if (lane < K) {
+    my_row = __ldg(row_of_slot + static_cast<int64_t>(t) * K + lane);
+    my_g = __ldg(topk_w + static_cast<int64_t>(t) * K + lane);
+  }
+  for (int v = lane; v < nvec; v += 32) {
+    float acc[V];
+#pragma unroll
+    for (int j = 0; j < V; ++j) acc[j] = 0.0f;
+    for (int k = 0; k < K; ++k) {
+      const int row = __shfl_sync(0xFFFFFFFFu, my_row, k);
+      const float g = __shfl_sync(0xFFFFFFFFu, my_g, k);
+      if (row < 0) continue;
+      float f[V];
+      unpack16<T>(ldg16(y_perm + static_cast<int64_t>(row) * d + v * V), f);
+#pragma unroll
+      for (int j = 0; j < V; ++j) acc[j] = fmaf(g, f[j], acc[j]);
+    }
+    if (shared_row0 >= 0) {
+      float f[V];
+      unpack16<T>(ldg16(y_perm + (shared_row0 + t) * d + v * V), f);
+#pragma unroll
+      for (int j = 0; j < V; ++j) acc[j] += f[j];
+    }
+    stg16(y + static_cast<int64_t>(t) * d + v * V, pack16<T>(acc));
+  }
+}
+
+// 16 E4M3 codes -> 16 bf16 values (every E4M3 value is exact in f16 and in
+// bf16, so both conversions are exact).
+__global__ void dequant_e4m3_kernel(const uint4* __restrict__ q, uint4* __restrict__ out, int64_t n16) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n16;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 v = __ldg(q + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>((w[j] >> (16 * h)) & 0xFFFFu);
+        const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+        const __half2 hv = *reinterpret_cast<const __half2*>(&hr);
+        const float2 f = __half22float2(hv);
+        o[2 * j + h] = pack_bf16x2(f.x, f.y);
+      }
+    }
+    out[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+    out[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream) {
+  if (a.S == 0) return cudaSuccess;
+  const int blocks = (a.S + kCombWarps - 1) / kCombWarps;
+  if (a.act_dtype == MOE_BF16)
+    combine_kernel<__nv_bfloat16><<<blocks, kCombWarps * 32, 0, stream>>>(
+        a.S, a.d, a.K, static_cast<const __nv_bfloat16*>(a.y_perm), a.row_of_slot, a.topk_w, a.shared_row0,
+        static_cast<__nv_bfloat16*>(a.y));
+  else
+    combine_kernel<float><<<blocks, kCombWarps * 32, 0, stream>>>(a.S, a.d, a.K, static_cast<const float*>(a.y_perm),
+                                                                   a.row_of_slot, a.topk_w, a.shared_row0,
+                                                                   static_cast<float*>(a.y));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequant_e4m3(const uint8_t* q, void* out_bf16, int64_t n, cudaStream_t stream) {
+  const int64_t n16 = n / 16;
+  if (n16 == 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t want = (n16 + threads - 1) / threads;
+  const int blocks = static_cast<int>(want < 148 * 16 ? want : 148 * 16);
+  dequant_e4m3_kernel<<<blocks, threads, 0, stream>>>(reinterpret_cast<const uint4*>(q),
+                                                      reinterpret_cast<uint4*>(out_bf16), n16);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

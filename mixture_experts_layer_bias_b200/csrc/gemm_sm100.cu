@@ -1,0 +1,454 @@
+// Grouped expert GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// jsqmd.com "第11章 MoE模型推理" 11.1.2: the B*L*K expert forwards of a layer
+// are grouped by expert and run together; plumephp.com "MoE 混合专家推理",
+// activation-memory block ("sequence expert"): feed all of an expert's tokens
+// to it as one large GEMM.  Here every expert group is a slice of rows of one
+// A buffer, and one persistent launch runs all groups:
+//
+//   out[out_row0 + r, n] = epi( sum_k A[a_row0 + r, k] * W[expert][n, k] )
+//
+// Up projection, SwiGLU: W = [W_gate rows n0..n0+127 ; W_up rows n0..n0+127]
+// forms one 256-row B tile, so one M=128 x N=256 MMA produces the gate and the
+// up accumulators side by side in TMEM and the epilogue writes
+// silu(gate) * up (x per-channel scales for FP8 weights) as bf16.
+// Down projection: 256 output columns per tile, optional bias / scale.
+//
+// Structure (one CTA per SM, 192 threads):
+//   warp 0      TMA producer: A tile 128x64 and B tile 256x64 (bf16, 128-byte
+//               swizzle) per stage into a 4-stage shared-memory ring;
+//   warp 1      allocates 512 TMEM columns; one lane issues tcgen05.mma
+//               (kind::f16, fp32 accumulate) and tcgen05.commit;
+//   warps 2-5   epilogue: tcgen05.ld of their 32-lane quarter, activation,
+//               predicated 16-byte stores of the group's valid rows only.
+// Two 256-column accumulators let the epilogue of tile i overlap the MMAs of
+// tile i+1.  The tile list (group, n-block, m-block; m fastest, so the CTAs
+// in flight share weight tiles through L2) is derived on the device from the
+// group table: no host synchronisation on routing results.
+//
+// Every mbarrier wait is bounded in time; a CTA that gives up raises a flag
+// in shared memory and the status block, waits for its own copies and MMAs
+// in flight, frees its TMEM and exits.  No load uses cluster multicast.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;  // 64 bf16 = 128 bytes = one swizzle row
+constexpr int STAGES = 4;
+constexpr int A_TILE = BM * BK * 2;           // 16 KB
+constexpr int B_HALF = 128 * BK * 2;          // 16 KB
+constexpr int STAGE_BYTES = A_TILE + 2 * B_HALF;  // 48 KB
+constexpr int ACC_COLS = 256;
+constexpr int TMEM_COLS = 512;
+constexpr int kThreads = 192;
+constexpr int kMaxGroups = 264;
+constexpr uint32_t kIdesc = idesc_bf16_f32(128, 256);
+
+struct TcParams {
+  const GroupEntry* groups;
+  int num_groups;
+  int shared_slab;
+  int a_rows_from_out;
+  int num_slabs;
+  int n_per_slab;
+  int N, K;
+  int bn_out;   // output columns per tile (128 SwiGLU, 256 otherwise)
+  int n_tiles;  // ceil(N / bn_out)
+  int64_t out_rows;
+  const float* bias;
+  const float* scale0;
+  const float* scale1;
+  void* out;
+  int out_f32;
+  StatusBlock* status;
+};
+
+struct SmemCtl {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int tile_start[kMaxGroups + 1];
+};
+
+constexpr size_t kSmemBytes = STAGES * STAGE_BYTES + sizeof(SmemCtl) + 1024;
+
+__device__ __forceinline__ bool wait_timed(uint64_t* bar, uint32_t parity) {
+  int never = 0;
+  return mbar_wait(bar, parity, &never);
+}
+
+struct TileInfo {
+  GroupEntry grp;
+  int m_idx, n_idx;
+};
+
+__device__ __forceinline__ TileInfo decode_tile(const SmemCtl& s, const TcParams& p, int tt) {
+  int lo = 0, hi = p.num_groups;  // find g: tile_start[g] <= tt < tile_start[g+1]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (s.tile_start[mid] <= tt)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  TileInfo ti;
+  ti.grp = p.groups[lo];
+  const int mt = (ti.grp.rows + BM - 1) / BM;
+  const int local = tt - s.tile_start[lo];
+  ti.n_idx = local / mt;
+  ti.m_idx = local - ti.n_idx * mt;
+  return ti;
+}
+
+__device__ __forceinline__ bool group_ok(const GroupEntry& g, const TcParams& p) {
+  return g.rows > 0 && g.expert >= 0 && g.expert < p.num_slabs && g.out_row0 >= 0 &&
+         static_cast<int64_t>(g.out_row0) + g.rows <= p.out_rows && g.a_row0 >= 0;
+}
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_store(const TcParams& p, const TileInfo& ti, uint32_t tbase, int row,
+                                               bool valid) {
+  const int N = p.N;
+  const int64_t orow = static_cast<int64_t>(ti.grp.out_row0) + row;
+  const int64_t sbase = static_cast<int64_t>(ti.grp.expert) * N;
+  constexpr int kChunks = (EPI == EPI_SWIGLU) ? 4 : 8;
+  for (int c = 0; c < kChunks; ++c) {
+    const int n = ti.n_idx * p.bn_out + c * 32;
+    uint32_t r0[32];
+    float v[32];
+    if (EPI == EPI_SWIGLU) {
+      uint32_t r1[32];
+      tmem_ld_32x32b_x32(tbase + c * 32, r0);
+      tmem_ld_32x32b_x32(tbase + 128 + c * 32, r1);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float g = __uint_as_float(r0[j]);
+        float u = __uint_as_float(r1[j]);
+        if (p.scale0 != nullptr && n + j < N) {
+          g *= __ldg(p.scale0 + sbase + n + j);
+          u *= __ldg(p.scale1 + sbase + n + j);
+        }
+        v[j] = g / (1.0f + __expf(-g)) * u;
+      }
+    } else {
+      tmem_ld_32x32b_x32(tbase + c * 32, r0);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float z = __uint_as_float(r0[j]);
+        if (n + j < N) {
+          if (p.scale0 != nullptr) z *= __ldg(p.scale0 + sbase + n + j);
+          if (EPI == EPI_GELU_BIAS || EPI == EPI_BIAS) z += __ldg(p.bias + sbase + n + j);
+        }
+        if (EPI == EPI_GELU_BIAS) z = 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
+        v[j] = z;
+      }
+    }
+    if (!valid) continue;
+    if (p.out_f32) {
+      float* o = static_cast<float*>(p.out) + orow * N + n;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (n + 4 * j + 4 <= N) stg16(o + 4 * j, pack16<float>(v + 4 * j));
+    } else {
+      __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + orow * N + n;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (n + 8 * j + 8 <= N) stg16(o + 8 * j, pack16<__nv_bfloat16>(v + 8 * j));
+    }
+  }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
+                           const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+                           TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  SmemCtl& s = *reinterpret_cast<SmemCtl*>(ring + STAGES * STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = lane_id();
+
+  // per-group tile counts -> exclusive prefix (warp 0)
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < p.num_groups; base += 32) {
+      const int g = base + lane;
+      int tiles = 0;
+      if (g < p.num_groups) {
+        const GroupEntry ge = p.groups[g];
+        if (group_ok(ge, p))
+          tiles = ((ge.rows + BM - 1) / BM) * p.n_tiles;
+        else if (ge.rows != 0)
+          report(p.status, MOE_STATUS_BAD_GROUP, -1);
+      }
+      int incl = tiles;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      if (g < p.num_groups) s.tile_start[g] = carry + incl - tiles;
+      carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+    if (lane == 0) s.tile_start[p.num_groups] = carry;
+  } else if (warp == 1) {
+    if (lane == 0) {
+      for (int i = 0; i < STAGES; ++i) {
+        mbar_init(&s.full[i], 1);
+        mbar_init(&s.empty[i], 1);
+      }
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&s.tfull[i], 1);
+        mbar_init(&s.tempty[i], 128);
+      }
+      mbar_init(&s.drain, 1);
+      s.abort = 0;
+      fence_mbar_init();
+    }
+    __syncwarp();
+    tmem_alloc(&s.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  } else if (warp == 2 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmA2);
+    tma_prefetch_desc(&tmB0);
+    tma_prefetch_desc(&tmB1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const int total = s.tile_start[p.num_groups];
+  const uint32_t tmem = s.tmem_base;
+  const int nk = (p.K + BK - 1) / BK;
+  volatile int* abort_flag = &s.abort;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_phase = 0;
+      bool ok = true;
+      for (int tt = blockIdx.x; tt < total && ok; tt += gridDim.x) {
+        const TileInfo ti = decode_tile(s, p, tt);
+        const int a_row = (p.a_rows_from_out ? ti.grp.out_row0 : ti.grp.a_row0) + ti.m_idx * BM;
+        const CUtensorMap* mA = (ti.grp.expert == p.shared_slab) ? &tmA2 : &tmA;
+        const int b_row = ti.grp.expert * p.n_per_slab + ti.n_idx * p.bn_out;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&s.full[stage], STAGE_BYTES);
+          armed |= 1u << stage;
+          armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+          uint8_t* sa = ring + stage * STAGE_BYTES;
+          uint8_t* sb = sa + A_TILE;
+          tma_load_2d(sa, mA, kb * BK, a_row, &s.full[stage]);
+          if (EPI == EPI_SWIGLU) {
+            tma_load_2d(sb, &tmB0, kb * BK, b_row, &s.full[stage]);
+            tma_load_2d(sb + B_HALF, &tmB1, kb * BK, b_row, &s.full[stage]);
+          } else {
+            tma_load_2d(sb, &tmB0, kb * BK, b_row, &s.full[stage]);
+            tma_load_2d(sb + B_HALF, &tmB0, kb * BK, b_row + 128, &s.full[stage]);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        report(p.status, MOE_STATUS_TIMEOUT, MOE_CNT_TIMEOUT);
+        // let the copies already issued land before the CTA exits
+        for (int i = 0; i < STAGES; ++i)
+          if (armed & (1u << i)) wait_timed(&s.full[i], (armed_phase >> i) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int tt = blockIdx.x; tt < total && ok; tt += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + acc * ACC_COLS;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&s.full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(ring + stage * STAGE_BYTES);
+          const uint32_t b_base = a_base + A_TILE;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            tc_mma_f16(d_tmem, smem_desc_sw128(a_base + kk * 32), smem_desc_sw128(b_base + kk * 32), kIdesc,
+                       (kb | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit(&s.empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&s.tfull[acc]);
+      }
+      // every MMA this thread issued must finish before TMEM is released
+      tc_commit(&s.drain);
+      wait_timed(&s.drain, 0);
+      if (!ok) {
+        *abort_flag = 1;
+        report(p.status, MOE_STATUS_TIMEOUT, MOE_CNT_TIMEOUT);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int local = 0;
+    for (int tt = blockIdx.x; tt < total; tt += gridDim.x, ++local) {
+      const TileInfo ti = decode_tile(s, p, tt);
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!mbar_wait(&s.tfull[acc], acc_phase, abort_flag)) {
+        if (lane == 0) {
+          *abort_flag = 1;
+          report(p.status, MOE_STATUS_TIMEOUT, MOE_CNT_TIMEOUT);
+        }
+        break;
+      }
+      tc_fence_after();
+      const int row = ti.m_idx * BM + q * 32 + lane;
+      const bool valid = row < ti.grp.rows;
+      const uint32_t tbase = tmem + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16);
+      epilogue_store<EPI>(p, ti, tbase, row, valid);
+      tc_fence_before();
+      mbar_arrive(&s.tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D bf16 map over [rows][k] (row-major), box 64 (k) x 128 rows, 128B swizzle.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int k) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr || rows <= 0 || k <= 0) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || (static_cast<int64_t>(k) * 2) % 16 != 0) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(k) * 2};
+  cuuint32_t box[2] = {BK, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI>
+cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB0, const CUtensorMap& mB1,
+                       const TcParams& p, int grid, cudaStream_t stream) {
+  static uint64_t attr_set = 0;  // one bit per device ordinal
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64 || !(attr_set & (1ull << dev))) {
+    e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes));
+    if (e != cudaSuccess) return e;
+    if (dev < 64) attr_set |= 1ull << dev;
+  }
+  grouped_gemm_tc_kernel<EPI><<<grid, kThreads, kSmemBytes, stream>>>(mA, mA2, mB0, mB1, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t stream) {
+  if (a.num_groups <= 0 || a.num_groups > kMaxGroups) return cudaErrorInvalidValue;
+  TcParams p;
+  p.groups = a.groups;
+  p.num_groups = a.num_groups;
+  p.shared_slab = a.shared_slab;
+  p.a_rows_from_out = a.a_rows_from_out;
+  p.n_per_slab = a.n_per_slab;
+  p.num_slabs = static_cast<int>(a.b_rows / a.n_per_slab);
+  p.N = a.N;
+  p.K = a.K;
+  p.bn_out = a.epilogue == EPI_SWIGLU ? 128 : 256;
+  p.n_tiles = (a.N + p.bn_out - 1) / p.bn_out;
+  p.out_rows = a.out_rows;
+  p.bias = a.bias;
+  p.scale0 = a.scale0;
+  p.scale1 = a.scale1;
+  p.out = a.out;
+  p.out_f32 = a.out_f32;
+  p.status = a.status;
+  CUtensorMap mA, mA2, mB0, mB1;
+  if (!make_map(&mA, a.a, a.a_rows, a.K)) return cudaErrorInvalidValue;
+  if (a.a_shared != nullptr) {
+    if (!make_map(&mA2, a.a_shared, a.a_shared_rows, a.K)) return cudaErrorInvalidValue;
+  } else {
+    mA2 = mA;
+  }
+  if (!make_map(&mB0, a.b0, a.b_rows, a.K)) return cudaErrorInvalidValue;
+  if (a.epilogue == EPI_SWIGLU) {
+    if (!make_map(&mB1, a.b1, a.b_rows, a.K)) return cudaErrorInvalidValue;
+  } else {
+    mB1 = mB0;
+  }
+  // upper bound of the tile count: every group may add one partial m-block
+  const int64_t bound = (a.max_total_rows / BM + a.num_groups) * static_cast<int64_t>(p.n_tiles);
+  const int grid = static_cast<int>(bound < num_sms ? (bound > 0 ? bound : 1) : num_sms);
+  switch (a.epilogue) {
+    case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(mA, mA2, mB0, mB1, p, grid, stream);
+    case EPI_GELU_BIAS: return launch_epi<EPI_GELU_BIAS>(mA, mA2, mB0, mB1, p, grid, stream);
+    case EPI_BIAS: return launch_epi<EPI_BIAS>(mA, mA2, mB0, mB1, p, grid, stream);
+    case EPI_NONE: return launch_epi<EPI_NONE>(mA, mA2, mB0, mB1, p, grid, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace moe

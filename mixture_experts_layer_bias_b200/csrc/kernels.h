@@ -1,0 +1,107 @@
+// Host-side launchers of the MoE layer kernels (internal to the library).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+struct StatusBlock;
+
+// --- routing ---------------------------------------------------------------
+struct RouteArgs {
+  int S, d, E, K;
+  int score_fn, renormalize, num_groups, topk_groups;
+  int act_dtype;
+  const void* x;            // [S][d] (unused when logits given)
+  const void* w_router;     // [E][d]
+  const float* logits;      // [S][E] fp32 or nullptr (then computed)
+  float* logits_scratch;    // [S][E] fp32 scratch for E > 32
+  const float* router_bias; // [E] or nullptr
+  const float* sel_bias;    // [E] or nullptr
+  int32_t* topk_idx;        // [S][K]
+  float* topk_w;            // [S][K]
+  StatusBlock* status;
+};
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream);
+
+// --- grouping by expert -----------------------------------------------------
+struct PermuteArgs {
+  int S, d, E, K, capacity, act_dtype;
+  const int32_t* topk_idx;   // [S][K]
+  int32_t* chunk_hist;       // [num_chunks][E] scratch
+  int32_t* counts;           // [E]
+  int32_t* offsets;          // [E+1] (+ [E+1] overflow offsets with capacity)
+  int32_t* row_of_slot;      // [S*K]
+  int32_t* token_of_row;     // [R]
+  const void* x;             // [S][d] or nullptr
+  void* x_perm;              // [R][d] or nullptr
+  int64_t num_rows;          // R
+  StatusBlock* status;
+};
+int permute_num_chunks(int S, int K);
+int permute_tokens_per_chunk(int K);
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream);
+
+// Group table entry of the grouped GEMMs: rows [a_row0, a_row0 + rows) of the
+// A operand, written to rows [out_row0, out_row0 + rows) of the output, all
+// with the weights of slab `expert`.
+struct GroupEntry {
+  int32_t a_row0, out_row0, rows, expert;
+};
+
+// Build the pass tables from offsets: pass 1 = routed groups (primary block
+// with capacity) + the shared expert, pass 2 = overflow groups (capacity only).
+// g1 has E + ns entries, g2 has E entries.
+cudaError_t launch_build_groups(int S, int E, int K, int capacity, int num_shared, const int32_t* offsets,
+                                GroupEntry* g1, GroupEntry* g2, StatusBlock* status, cudaStream_t stream);
+
+// --- grouped expert GEMMs ----------------------------------------------------
+enum Epilogue { EPI_SWIGLU = 0, EPI_GELU_BIAS = 1, EPI_BIAS = 2, EPI_NONE = 3 };
+
+struct GemmArgs {
+  int epilogue;
+  const GroupEntry* groups;
+  int num_groups;
+  int shared_slab;          // slab index whose A rows come from a_shared, -1 = none
+  int a_rows_from_out;      // 1: A row = out_row0 + r (down projection), 0: a_row0 + r
+  const void* a;            // A operand [a_rows][K]
+  int64_t a_rows;
+  const void* a_shared;     // shared-expert A operand [a_shared_rows][K] (up projection)
+  int64_t a_shared_rows;
+  const void* b0;           // weights [slabs * n_per_slab][K] (gate for SwiGLU)
+  const void* b1;           // up weights (SwiGLU), else unused
+  int64_t b_rows;           // slabs * n_per_slab
+  int n_per_slab;           // N rows of one slab (h or d)
+  int N, K;                 // output columns, reduction length
+  const float* bias;        // [slabs][N] or nullptr
+  const float* scale0;      // per-output-channel scale [slabs][N] (gate / plain)
+  const float* scale1;      // per-output-channel scale [slabs][N] (up)
+  void* out;                // [out_rows][N]
+  int64_t out_rows;
+  int out_f32;              // 1: fp32 output, 0: bf16
+  int64_t max_total_rows;   // upper bound of the rows of all groups together
+  int64_t max_group_rows;   // upper bound of the rows of one group
+  StatusBlock* status;
+};
+cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t stream);
+cudaError_t launch_grouped_gemm_f32(const GemmArgs& a, cudaStream_t stream);
+
+// FP8-E4M3 weight slabs -> bf16 (exact)
+cudaError_t launch_dequant_e4m3(const uint8_t* q, void* out_bf16, int64_t n, cudaStream_t stream);
+
+// --- combine -----------------------------------------------------------------
+struct CombineArgs {
+  int S, d, K, act_dtype;
+  const void* y_perm;
+  const int32_t* row_of_slot;
+  const float* topk_w;
+  int64_t shared_row0;  // -1 = no shared expert
+  void* y;
+};
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,283 @@
+// Grouping by expert: histogram -> prefix scan -> stable permutation, and the
+// gather of token rows into expert-contiguous rows.
+//
+// jsqmd.com "第11章 MoE模型推理" 11.1.2 (the S*K expert forwards are grouped
+// and merged by expert) and 11.2.1 (regroup the sequence into one
+// sub-sequence per expert, restore the original order afterwards);
+// ybb.press "MoE 推理工程深层实战" 2.2 (rows above a capacity go to an overflow
+// buffer that is processed later; none is dropped).
+//
+// Three kernels, no atomics on row positions, so the permutation is
+// deterministic and stable (rows of an expert follow slot order t*K + k):
+//  1. count:   each CTA owns a chunk of whole tokens and writes its expert
+//              histogram (shared-memory atomics; counts are order-free);
+//  2. scan:    one CTA turns the chunk histograms into per-chunk bases
+//              (exclusive prefix over chunks) and the expert offsets
+//              (exclusive prefix over experts), plus the overflow split;
+//  3. scatter: each CTA ranks its slots inside the chunk (warp match/popc,
+//              then a prefix over warps), writes row_of_slot / token_of_row,
+//              and copies every token row once from HBM to its K rows with
+//              16-byte vectors.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kChunkSlots = 1024;  // slots per CTA (whole tokens)
+constexpr int kPermWarps = 8;
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+__global__ void __launch_bounds__(256)
+    count_kernel(int S, int E, int K, int tok_per_chunk, const int32_t* __restrict__ topk_idx,
+                 int32_t* __restrict__ chunk_hist, StatusBlock* status) {
+  extern __shared__ int32_t hist[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int64_t s0 = static_cast<int64_t>(blockIdx.x) * tok_per_chunk * K;
+  const int64_t s1 = min(static_cast<int64_t>(S) * K, s0 + static_cast<int64_t>(tok_per_chunk) * K);
+  int bad = 0;
+  for (int64_t s = s0 + threadIdx.x; s < s1; s += blockDim.x) {
+    const int e = topk_idx[s];
+    if (e >= 0 && e < E)
+      atomicAdd(&hist[e], 1);
+    else
+      ++bad;
+  }
+  if (bad) report(status, MOE_STATUS_BAD_EXPERT_ID, MOE_CNT_BAD_ID, bad);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_hist[static_cast<int64_t>(blockIdx.x) * E + e] = hist[e];
+}
+
+// Inclusive warp scan helper over one value per lane.
+__device__ __forceinline__ int warp_incl_scan(int v) {
+  const int lane = lane_id();
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(kFull, v, off);
+    if (lane >= off) v += o;
+  }
+  return v;
+}
+
+// Exclusive prefix of src[0..n) into dst[0..n], dst[n] = total, by warp 0.
+__device__ void warp0_exclusive_scan(const int32_t* src, int32_t* dst, int n) {
+  if (threadIdx.x >= 32) return;
+  const int lane = lane_id();
+  int carry = 0;
+  for (int base = 0; base < n; base += 32) {
+    const int i = base + lane;
+    const int v = i < n ? src[i] : 0;
+    const int incl = warp_incl_scan(v);
+    if (i < n) dst[i] = carry + incl - v;
+    carry += __shfl_sync(kFull, incl, 31);
+  }
+  if (lane == 0) dst[n] = carry;
+}
+
+// The chunk histograms of one expert are split into P = blockDim / E
+// contiguous segments, one thread each: segment sums, a prefix over the
+// segments, then a second pass writes the running (exclusive) chunk bases.
+__global__ void __launch_bounds__(1024)
+    scan_kernel(int E, int num_chunks, int capacity, int32_t* __restrict__ chunk_hist, int32_t* __restrict__ counts,
+                int32_t* __restrict__ offsets, StatusBlock* status) {
+  extern __shared__ int32_t sm[];
+  const int P = blockDim.x / E;        // >= 1 since E <= 256 < blockDim
+  int32_t* part = sm;                  // [P][E] segment sums
+  int32_t* cnt = sm + P * E;           // [E]
+  int32_t* ovf = cnt + E;              // [E]
+  int32_t* tmp = ovf + E;              // [E+1]
+  const int tid = threadIdx.x;
+  const int e = tid % E, pi = tid / E;
+  const bool active = pi < P;
+  const int seg = (num_chunks + P - 1) / P;
+  const int c0 = min(num_chunks, pi * seg), c1 = min(num_chunks, c0 + seg);
+  int local = 0;
+  if (active)
+    for (int c = c0; c < c1; ++c) local += chunk_hist[static_cast<int64_t>(c) * E + e];
+  if (active) part[pi * E + e] = local;
+  __syncthreads();
+  if (active) {
+    int run = 0;
+    for (int q = 0; q < pi; ++q) run += part[q * E + e];
+    for (int c = c0; c < c1; ++c) {
+      const int64_t i = static_cast<int64_t>(c) * E + e;
+      const int v = chunk_hist[i];
+      chunk_hist[i] = run;
+      run += v;
+    }
+    if (pi == P - 1) {
+      cnt[e] = run;
+      counts[e] = run;
+      ovf[e] = capacity > 0 ? max(run - capacity, 0) : 0;
+    }
+  }
+  __syncthreads();
+  warp0_exclusive_scan(cnt, tmp, E);
+  __syncthreads();
+  for (int i = tid; i <= E; i += blockDim.x) offsets[i] = tmp[i];
+  if (capacity > 0) {
+    __syncthreads();
+    warp0_exclusive_scan(ovf, tmp, E);
+    __syncthreads();
+    for (int i = tid; i <= E; i += blockDim.x) offsets[E + 1 + i] = tmp[i];
+    if (tid == 0 && tmp[E] > 0) report(status, 0u, MOE_CNT_OVERFLOW_ROWS, tmp[E]);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kPermWarps * 32)
+    scatter_kernel(int S, int d, int E, int K, int capacity, int tok_per_chunk, const int32_t* __restrict__ topk_idx,
+                   const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ offsets,
+                   int32_t* __restrict__ row_of_slot, int32_t* __restrict__ token_of_row, const T* __restrict__ x,
+                   T* __restrict__ x_perm) {
+  extern __shared__ int32_t sm[];
+  int32_t* whist = sm;                        // [kPermWarps][E] per-warp counts, then bases
+  int32_t* srow = sm + kPermWarps * E;        // [kChunkSlots] rows of the chunk's slots
+  const int warp = threadIdx.x >> 5, lane = lane_id();
+  const int t0 = blockIdx.x * tok_per_chunk;
+  const int t1 = min(S, t0 + tok_per_chunk);
+  const int64_t s0 = static_cast<int64_t>(t0) * K;
+  const int nslots = (t1 - t0) * K;
+  const int per_warp = (nslots + kPermWarps - 1) / kPermWarps;
+  const int w0 = warp * per_warp, w1 = min(nslots, w0 + per_warp);
+
+  for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) whist[i] = 0;
+  __syncthreads();
+  // pass 1: per-warp expert counts over the warp's contiguous slot range
+  for (int b = w0; b < w1; b += 32) {
+    const int s = b + lane;
+    const bool act = s < w1;
+    int e = act ? topk_idx[s0 + s] : -1;
+    if (e < 0 || e >= E) e = -1;
+    const unsigned peers = __match_any_sync(kFull, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) whist[warp * E + e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // bases: chunk base of the expert + counts of the warps before this one
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = chunk_base[static_cast<int64_t>(blockIdx.x) * E + e];
+    for (int w = 0; w < kPermWarps; ++w) {
+      const int c = whist[w * E + e];
+      whist[w * E + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  // pass 2: ranks -> rows
+  for (int b = w0; b < w1; b += 32) {
+    const int s = b + lane;
+    const bool act = s < w1;
+    int e = act ? topk_idx[s0 + s] : -1;
+    if (e < 0 || e >= E) e = -1;
+    const unsigned peers = __match_any_sync(kFull, e);
+    int row = -1;
+    if (e >= 0) {
+      const unsigned lt = (1u << lane) - 1u;
+      const int r = whist[warp * E + e] + __popc(peers & lt);
+      if (capacity <= 0)
+        row = offsets[e] + r;
+      else
+        row = r < capacity ? e * capacity + r : E * capacity + offsets[E + 1 + e] + (r - capacity);
+    }
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) whist[warp * E + e] += __popc(peers);
+    if (act) {
+      srow[s] = row;
+      row_of_slot[s0 + s] = row;
+      if (row >= 0) token_of_row[row] = static_cast<int32_t>((s0 + s) / K);
+    }
+    __syncwarp();
+  }
+  if (x == nullptr || x_perm == nullptr) return;
+  __syncthreads();
+  // copy: one warp per token, read the row once, write it to its K rows
+  constexpr int V = Vec16<T>::N;
+  const int nvec = d / V;
+  for (int t = t0 + warp; t < t1; t += kPermWarps) {
+    const T* src = x + static_cast<int64_t>(t) * d;
+    const int sl = (t - t0) * K;
+    for (int v = lane; v < nvec; v += 32) {
+      const uint4 val = ldg16(src + v * V);
+      for (int k = 0; k < K; ++k) {
+        const int row = srow[sl + k];
+        if (row >= 0) stg16(x_perm + static_cast<int64_t>(row) * d + v * V, val);
+      }
+    }
+  }
+}
+
+__global__ void build_groups_kernel(int S, int E, int K, int capacity, int num_shared,
+                                    const int32_t* __restrict__ offsets, GroupEntry* __restrict__ g1,
+                                    GroupEntry* __restrict__ g2) {
+  const int64_t R = capacity > 0 ? static_cast<int64_t>(E) * capacity + static_cast<int64_t>(S) * K
+                                 : static_cast<int64_t>(S) * K;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int cnt = offsets[e + 1] - offsets[e];
+    if (capacity <= 0) {
+      g1[e] = GroupEntry{offsets[e], offsets[e], cnt, e};
+    } else {
+      const int prim = min(cnt, capacity);
+      g1[e] = GroupEntry{e * capacity, e * capacity, prim, e};
+      const int orow = E * capacity + offsets[E + 1 + e];
+      g2[e] = GroupEntry{orow, orow, cnt - prim, e};
+    }
+  }
+  if (threadIdx.x == 0 && num_shared > 0) g1[E] = GroupEntry{0, static_cast<int32_t>(R), S, E};
+}
+
+}  // namespace
+
+int permute_tokens_per_chunk(int K) { return K >= kChunkSlots ? 1 : kChunkSlots / K; }
+
+int permute_num_chunks(int S, int K) {
+  const int tpc = permute_tokens_per_chunk(K);
+  return (S + tpc - 1) / tpc;
+}
+
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
+  if (a.S == 0) {
+    cudaError_t err = cudaMemsetAsync(a.counts, 0, sizeof(int32_t) * a.E, stream);
+    if (err == cudaSuccess)
+      err = cudaMemsetAsync(a.offsets, 0, sizeof(int32_t) * (a.E + 1) * (a.capacity > 0 ? 2 : 1), stream);
+    if (err == cudaSuccess && a.num_rows > 0)
+      err = cudaMemsetAsync(a.token_of_row, 0xFF, sizeof(int32_t) * a.num_rows, stream);
+    return err;
+  }
+  const int tpc = permute_tokens_per_chunk(a.K);
+  const int nch = permute_num_chunks(a.S, a.K);
+  cudaError_t err;
+  if (a.capacity > 0) {
+    // unused primary rows keep token -1
+    err = cudaMemsetAsync(a.token_of_row, 0xFF, sizeof(int32_t) * a.num_rows, stream);
+    if (err != cudaSuccess) return err;
+  }
+  count_kernel<<<nch, 256, sizeof(int32_t) * a.E, stream>>>(a.S, a.E, a.K, tpc, a.topk_idx, a.chunk_hist, a.status);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  const int scan_threads = 1024;
+  const size_t scan_smem = sizeof(int32_t) * ((scan_threads / a.E) * a.E + 3 * a.E + 1);
+  scan_kernel<<<1, scan_threads, scan_smem, stream>>>(a.E, nch, a.capacity, a.chunk_hist, a.counts,
+                                                                     a.offsets, a.status);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  const size_t smem = sizeof(int32_t) * (kPermWarps * a.E + kChunkSlots);
+  if (a.act_dtype == MOE_BF16)
+    scatter_kernel<__nv_bfloat16><<<nch, kPermWarps * 32, smem, stream>>>(
+        a.S, a.d, a.E, a.K, a.capacity, tpc, a.topk_idx, a.chunk_hist, a.offsets, a.row_of_slot, a.token_of_row,
+        static_cast<const __nv_bfloat16*>(a.x), static_cast<__nv_bfloat16*>(a.x_perm));
+  else
+    scatter_kernel<float><<<nch, kPermWarps * 32, smem, stream>>>(
+        a.S, a.d, a.E, a.K, a.capacity, tpc, a.topk_idx, a.chunk_hist, a.offsets, a.row_of_slot, a.token_of_row,
+        static_cast<const float*>(a.x), static_cast<float*>(a.x_perm));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_build_groups(int S, int E, int K, int capacity, int num_shared, const int32_t* offsets,
+                                GroupEntry* g1, GroupEntry* g2, StatusBlock* status, cudaStream_t stream) {
+  (void)status;
+  build_groups_kernel<<<1, 256, 0, stream>>>(S, E, K, capacity, num_shared, offsets, g1, g2);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

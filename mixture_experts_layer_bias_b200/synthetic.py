@@ -125,6 +125,17 @@ def quantize_e4m3_rows(w: torch.Tensor):
     return q.view(torch.uint8), s.to(torch.float32)
 
 
+def router_offsets(cfg: LayerConfig, seed: int = 0):
+    """Per-expert router logit offsets of the workload (CPU tensor), or None."""
+    cpu = torch.device("cpu")
+    rb = None
+    if cfg.router_offset_var > 0:
+        rb = _normal((cfg.E,), cfg.router_offset_var, _gen(cpu, seed, 3), cpu)
+    if cfg.skew_offset_scale > 0:
+        rb = _normal((cfg.E,), 1.0, _gen(cpu, seed, 4), cpu) * cfg.skew_offset_scale
+    return rb
+
+
 def make_inputs(cfg: LayerConfig, device="cpu", seed: int = 0, x_only: bool = False) -> dict:
     """Draw every input of one layer call.  Returns a dict of torch tensors on
     ``device``: x, w_router, router_bias, sel_bias and the expert stacks in the
@@ -138,11 +149,7 @@ def make_inputs(cfg: LayerConfig, device="cpu", seed: int = 0, x_only: bool = Fa
         return out
     cpu = torch.device("cpu")
     out["w_router"] = _normal((E, d), 1.0 / d, _gen(cpu, seed, 2), cpu, adt).to(dev)
-    rb = None
-    if cfg.router_offset_var > 0:
-        rb = _normal((E,), cfg.router_offset_var, _gen(cpu, seed, 3), cpu)
-    if cfg.skew_offset_scale > 0:
-        rb = _normal((E,), 1.0, _gen(cpu, seed, 4), cpu) * cfg.skew_offset_scale
+    rb = router_offsets(cfg, seed)
     out["router_bias"] = None if rb is None else rb.to(dev)
     out["sel_bias"] = None
     if cfg.sel_bias_var > 0:

@@ -1,0 +1,140 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry
+point the header declares, sizes workspaces, and rejects bad arguments before
+touching CUDA.  No GPU needed: none of these calls reaches a CUDA API."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mixture_experts_layer_bias_b200 import build as B
+from mixture_experts_layer_bias_b200 import ops
+from mixture_experts_layer_bias_b200 import synthetic as syn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_library():
+    B.build()
+    return ops.lib()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol():
+    names = header_functions()
+    assert len(names) >= 10
+    lib = ops.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(ops.EXPORTED)
+
+
+def test_strerror():
+    assert ops.strerror(0) == "ok"
+    for code in range(1, 6):
+        assert len(ops.strerror(code)) > 3
+    assert ops.strerror(99) == "unknown status"
+
+
+def _desc(name, **over):
+    return ops.make_desc(**dict(syn.desc_dict(syn.CONFIGS[name]), **over))
+
+
+@pytest.mark.parametrize("name", list(syn.CONFIGS))
+def test_workspace_size_and_rows(name):
+    cfg = syn.CONFIGS[name]
+    d = _desc(name)
+    R = ops.moe_routed_rows(d)
+    if cfg.capacity:
+        assert R == cfg.E * cfg.capacity + cfg.S * cfg.K
+    else:
+        assert R == cfg.S * cfg.K
+    n = ops.moe_workspace_size(d)
+    ab = 4 if cfg.act_dtype == 0 else 2
+    Rt = R + cfg.num_shared * cfg.S
+    # at least the permuted rows, hidden and expert outputs
+    assert n >= (R * cfg.d + Rt * cfg.h + Rt * cfg.d) * ab
+    assert n % 256 == 0
+
+
+def test_capacity_value_of_skew_workload():
+    cfg = syn.CONFIGS["fp8_skew_capacity"]
+    assert cfg.capacity == syn.capacity_for(cfg.S, cfg.K, cfg.E) == 2560
+
+
+BAD = [
+    dict(top_k=0), dict(top_k=9), dict(num_experts=0), dict(num_experts=300), dict(d_model=100),
+    dict(d_ff=0), dict(score_fn=5), dict(num_groups=3), dict(num_groups=2, topk_groups=3),
+    dict(num_groups=4, topk_groups=1, top_k=3), dict(num_shared=2), dict(capacity=-1), dict(num_tokens=-1),
+    dict(renormalize=2), dict(activation=7), dict(act_dtype=5),
+]
+
+
+@pytest.mark.parametrize("over", BAD)
+def test_invalid_desc_rejected(over):
+    d = _desc("mixtral_prefill", **over)
+    n = ctypes.c_size_t(0)
+    assert ops.lib().moe_workspace_size(ctypes.byref(d), ctypes.byref(n)) == ops.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("over", [dict(act_dtype=0), dict(weight_dtype=0),
+                                  dict(weight_dtype=2, activation=0)])
+def test_unsupported_combination(over):
+    d = _desc("mixtral_prefill", **over)
+    n = ctypes.c_size_t(0)
+    assert ops.lib().moe_workspace_size(ctypes.byref(d), ctypes.byref(n)) == ops.MOE_ERR_UNSUPPORTED
+
+
+def test_group_size_must_be_power_of_two():
+    d = _desc("dsv3_grouped", num_experts=96, num_groups=2)  # groups of 48
+    n = ctypes.c_size_t(0)
+    assert ops.lib().moe_workspace_size(ctypes.byref(d), ctypes.byref(n)) == ops.MOE_ERR_INVALID_ARG
+
+
+def test_calls_reject_missing_workspace_and_pointers():
+    L = ops.lib()
+    d = _desc("tiny_f32")
+    w = ops.MoeWeights()
+    p = ctypes.c_void_p(0x1000)
+    # no workspace
+    assert L.moe_route(ctypes.byref(d), ctypes.byref(w), p, None, p, p, None, 0, None) == ops.MOE_ERR_WORKSPACE
+    # workspace too small (pointer value only: nothing is dereferenced on the host)
+    ws = ctypes.c_void_p(0x100000)
+    assert L.moe_layer_forward(ctypes.byref(d), ctypes.byref(w), p, p, None, None, None, ws, 256,
+                               None) == ops.MOE_ERR_WORKSPACE
+    # misaligned workspace
+    n = ops.moe_workspace_size(d)
+    assert L.moe_combine(ctypes.byref(d), p, p, p, p, ctypes.c_void_p(0x100010), n, None) == ops.MOE_ERR_WORKSPACE
+    # missing outputs / weights
+    assert L.moe_route(ctypes.byref(d), ctypes.byref(w), p, None, None, p, ws, n, None) == ops.MOE_ERR_INVALID_ARG
+    assert L.moe_route(ctypes.byref(d), ctypes.byref(w), p, None, p, p, ws, n, None) == ops.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_forward(ctypes.byref(d), ctypes.byref(w), p, p, None, None, None, ws, n,
+                               None) == ops.MOE_ERR_INVALID_ARG
+    assert L.moe_permute(ctypes.byref(d), p, p, None, p, p, p, p, ws, n, None) == ops.MOE_ERR_INVALID_ARG
+    # x without x_perm
+    assert L.moe_permute(ctypes.byref(d), p, p, p, p, p, p, None, ws, n, None) == ops.MOE_ERR_INVALID_ARG
+    # misaligned activations
+    assert L.moe_combine(ctypes.byref(d), ctypes.c_void_p(0x1004), p, p, p, ws, n, None) == ops.MOE_ERR_INVALID_ARG
+    assert L.moe_get_status(None, None, None, None) == ops.MOE_ERR_WORKSPACE
+    assert L.moe_workspace_init(None, 0, None) == ops.MOE_ERR_WORKSPACE
+
+
+def test_empty_batch_is_a_no_op():
+    """S = 0 is valid: the calls return OK without launching anything."""
+    L = ops.lib()
+    d = _desc("tiny_f32", num_tokens=0)
+    n = ops.moe_workspace_size(d)
+    ws = ctypes.c_void_p(0x100000)
+    w = ops.MoeWeights()
+    p = ctypes.c_void_p(0x1000)
+    assert L.moe_route(ctypes.byref(d), ctypes.byref(w), None, None, p, p, ws, n, None) == ops.MOE_OK
+    assert L.moe_combine(ctypes.byref(d), p, p, p, p, ws, n, None) == ops.MOE_OK
+    assert L.moe_layer_forward(ctypes.byref(d), ctypes.byref(w), None, None, None, None, None, ws, n,
+                               None) == ops.MOE_OK
+    assert ops.moe_routed_rows(d) == 0
