@@ -35,19 +35,23 @@ __global__ void __launch_bounds__(kCombWarps * 32)
     my_row = __ldg(row_of_slot + static_cast<int64_t>(t) * K + lane);
     my_g = __ldg(topk_w + static_cast<int64_t>(t) * K + lane);
   }
-  for (int v = lane; v < nvec; v += 32) {
+  // warp-uniform loop: every lane takes part in the shuffles below
+  for (int base = 0; base < nvec; base += 32) {
+    const int v = base + lane;
+    const bool act = v < nvec;
     float acc[V];
 #pragma unroll
     for (int j = 0; j < V; ++j) acc[j] = 0.0f;
     for (int k = 0; k < K; ++k) {
       const int row = __shfl_sync(0xFFFFFFFFu, my_row, k);
       const float g = __shfl_sync(0xFFFFFFFFu, my_g, k);
-      if (row < 0) continue;
+      if (row < 0 || !act) continue;
       float f[V];
       unpack16<T>(ldg16(y_perm + static_cast<int64_t>(row) * d + v * V), f);
 #pragma unroll
       for (int j = 0; j < V; ++j) acc[j] = fmaf(g, f[j], acc[j]);
     }
+    if (!act) continue;
     if (shared_row0 >= 0) {
       float f[V];
       unpack16<T>(ldg16(y_perm + (shared_row0 + t) * d + v * V), f);
