@@ -175,6 +175,28 @@ moe_status moe_permute(const moe_desc *desc, const void *x, const int32_t *topk_
                        size_t ws_bytes, void *stream);
 
 /*
+ * moe_permute without a workspace, for callers that cannot allocate device
+ * memory: a runtime whose device-memory budget is fixed at start-up, code
+ * running inside an allocator or other callback where a nested
+ * cudaMalloc/cudaFree is not allowed, or a loop that must not risk the
+ * device-wide synchronisation cudaFree can cause.  The pages have no
+ * counterpart of this call; it exists for those callers only.
+ *   Same arguments, outputs and results as moe_permute, minus ws/ws_bytes.
+ *   The only scratch (per-chunk expert histograms) lives in a 256 KB device
+ *   array inside the library, held by every GPU that loads it until exit.
+ *   Sizes whose histograms exceed it -- more than 65536 (chunk, expert)
+ *   entries, i.e. ceil(S / floor(1024/K)) * E > 65536 -- return
+ *   MOE_ERR_WORKSPACE before anything is enqueued.  The first call on a device looks up the
+ *   array's device address (make it before any stream capture).  All calls
+ *   share the array: calls that overlap on the GPU race.  There is no status
+ *   block: an expert id outside [0, E) gets row -1 in row_of_slot.
+ *   Allocates nothing and calls no allocating routine.
+ */
+moe_status moe_permute_static(const moe_desc *desc, const void *x, const int32_t *topk_idx, int32_t *counts,
+                              int32_t *offsets, int32_t *row_of_slot, int32_t *token_of_row, void *x_perm,
+                              void *stream);
+
+/*
  * Grouped expert FFN (11.1.2: the S*K expert forwards grouped by expert).
  *   x_perm [R][d] rows grouped as offsets describes (layout of moe_permute);
  *   x [S][d]: A operand of the shared expert (NULL when num_shared = 0);

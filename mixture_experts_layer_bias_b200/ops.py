@@ -28,7 +28,8 @@ WEIGHT_FIELDS = ("w_router", "router_bias", "sel_bias", "w1", "b1", "w2", "b2", 
                  "s_gate", "s_up", "s_down")
 
 EXPORTED = ("moe_routed_rows", "moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute",
-            "moe_grouped_ffn", "moe_combine", "moe_layer_forward", "moe_get_status", "moe_strerror")
+            "moe_permute_static", "moe_grouped_ffn", "moe_combine", "moe_layer_forward", "moe_get_status",
+            "moe_strerror")
 
 
 class MoeDesc(ctypes.Structure):
@@ -61,6 +62,7 @@ def lib():
         "moe_workspace_init": (I, [P, SZ, P]),
         "moe_route": (I, [pd, pw, P, P, P, P, P, SZ, P]),
         "moe_permute": (I, [pd, P, P, P, P, P, P, P, P, SZ, P]),
+        "moe_permute_static": (I, [pd, P, P, P, P, P, P, P, P]),
         "moe_grouped_ffn": (I, [pd, pw, P, P, P, P, P, SZ, P]),
         "moe_combine": (I, [pd, P, P, P, P, P, SZ, P]),
         "moe_layer_forward": (I, [pd, pw, P, P, P, P, P, P, SZ, P]),
@@ -154,6 +156,14 @@ def moe_permute(desc, x, topk_idx, counts, offsets, row_of_slot, token_of_row, x
     _check(lib().moe_permute(ctypes.byref(desc), _ptr(x), _ptr(topk_idx), _ptr(counts), _ptr(offsets),
                              _ptr(row_of_slot), _ptr(token_of_row), _ptr(x_perm), p, n, _stream(stream)),
            "moe_permute")
+
+
+def moe_permute_static(desc, x, topk_idx, counts, offsets, row_of_slot, token_of_row, x_perm, stream=None):
+    """moe_permute without a workspace: its scratch is a fixed 256 KB device
+    array inside the library (for callers that cannot allocate)."""
+    _check(lib().moe_permute_static(ctypes.byref(desc), _ptr(x), _ptr(topk_idx), _ptr(counts), _ptr(offsets),
+                                    _ptr(row_of_slot), _ptr(token_of_row), _ptr(x_perm), _stream(stream)),
+           "moe_permute_static")
 
 
 def moe_grouped_ffn(desc, weights, x_perm, offsets, x, y_perm, ws, stream=None):
