@@ -68,7 +68,7 @@ def workload_desc(cfg):
 def kernels_per_step(cfg):
     """Launches of this library's kernels in one layer forward."""
     n = 1 if (cfg.E <= 32) else 2          # route (fused) or logits + top-k
-    n += 3                                 # count, scan, scatter+gather
+    n += 4                                 # count, scan, scatter, gather
     n += 1 + 2                             # group table, up and down GEMM
     if cfg.weight_dtype == syn.E4M3:
         n += 3                             # E4M3 -> bf16 decode of the three stacks

@@ -93,7 +93,7 @@ typedef enum { MOE_ACT_GELU = 0, MOE_ACT_SWIGLU = 1 } moe_act;
  *     pass (ybb.press 2.2, overflow buffering).  No token is dropped.
  * Supported: (F32 act, F32 weights, GELU) with E <= 32 on the SIMT path;
  * (BF16 act, BF16 or E4M3 weights, SWIGLU or GELU) on the tensor-core path.
- * E <= 256, K <= min(E, 16), d and h multiples of 8.
+ * E <= 256, K <= min(E, 32), d and h multiples of 8.
  */
 typedef struct {
   int32_t num_tokens;

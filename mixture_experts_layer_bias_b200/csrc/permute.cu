@@ -7,7 +7,7 @@
 // ybb.press "MoE 推理工程深层实战" 2.2 (rows above a capacity go to an overflow
 // buffer that is processed later; none is dropped).
 //
-// Three kernels, no atomics on row positions, so the permutation is
+// Four kernels, no atomics on row positions, so the permutation is
 // deterministic and stable (rows of an expert follow slot order t*K + k):
 //  1. count:   each CTA owns a chunk of whole tokens and writes its expert
 //              histogram (shared-memory atomics; counts are order-free);
@@ -15,9 +15,9 @@
 //              (exclusive prefix over chunks) and the expert offsets
 //              (exclusive prefix over experts), plus the overflow split;
 //  3. scatter: each CTA ranks its slots inside the chunk (warp match/popc,
-//              then a prefix over warps), writes row_of_slot / token_of_row,
-//              and copies every token row once from HBM to its K rows with
-//              16-byte vectors.
+//              then a prefix over warps) and writes row_of_slot / token_of_row;
+//  4. gather:  one warp per token copies its row once from HBM to its K rows
+//              with 16-byte vectors.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -126,15 +126,12 @@ __global__ void __launch_bounds__(1024)
   }
 }
 
-template <typename T>
 __global__ void __launch_bounds__(kPermWarps * 32)
     scatter_kernel(int S, int d, int E, int K, int capacity, int tok_per_chunk, const int32_t* __restrict__ topk_idx,
                    const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ offsets,
-                   int32_t* __restrict__ row_of_slot, int32_t* __restrict__ token_of_row, const T* __restrict__ x,
-                   T* __restrict__ x_perm) {
+                   int32_t* __restrict__ row_of_slot, int32_t* __restrict__ token_of_row) {
   extern __shared__ int32_t sm[];
   int32_t* whist = sm;                        // [kPermWarps][E] per-warp counts, then bases
-  int32_t* srow = sm + kPermWarps * E;        // [kChunkSlots] rows of the chunk's slots
   const int warp = threadIdx.x >> 5, lane = lane_id();
   const int t0 = blockIdx.x * tok_per_chunk;
   const int t1 = min(S, t0 + tok_per_chunk);
@@ -185,26 +182,35 @@ __global__ void __launch_bounds__(kPermWarps * 32)
     __syncwarp();
     if (e >= 0 && lane == __ffs(peers) - 1) whist[warp * E + e] += __popc(peers);
     if (act) {
-      srow[s] = row;
       row_of_slot[s0 + s] = row;
       if (row >= 0) token_of_row[row] = static_cast<int32_t>((s0 + s) / K);
     }
     __syncwarp();
   }
-  if (x == nullptr || x_perm == nullptr) return;
-  __syncthreads();
-  // copy: one warp per token, read the row once, write it to its K rows
+}
+
+// Row gather: one warp per token reads its row once (16-byte vectors) and
+// writes it to each of its K rows.  The grid grows with S, so the copy is
+// spread over every SM.
+template <typename T>
+__global__ void __launch_bounds__(kPermWarps * 32)
+    gather_rows_kernel(int S, int d, int K, const int32_t* __restrict__ row_of_slot, const T* __restrict__ x,
+                       T* __restrict__ x_perm) {
+  const int t = blockIdx.x * kPermWarps + (threadIdx.x >> 5);
+  if (t >= S) return;
+  const int lane = lane_id();
+  const int my_row = lane < K ? __ldg(row_of_slot + static_cast<int64_t>(t) * K + lane) : -1;
   constexpr int V = Vec16<T>::N;
   const int nvec = d / V;
-  for (int t = t0 + warp; t < t1; t += kPermWarps) {
-    const T* src = x + static_cast<int64_t>(t) * d;
-    const int sl = (t - t0) * K;
-    for (int v = lane; v < nvec; v += 32) {
-      const uint4 val = ldg16(src + v * V);
-      for (int k = 0; k < K; ++k) {
-        const int row = srow[sl + k];
-        if (row >= 0) stg16(x_perm + static_cast<int64_t>(row) * d + v * V, val);
-      }
+  const T* src = x + static_cast<int64_t>(t) * d;
+#pragma unroll 2
+  for (int base = 0; base < nvec; base += 32) {
+    const int v = base + lane;
+    const bool act = v < nvec;
+    const uint4 val = act ? ldg16(src + v * V) : make_uint4(0, 0, 0, 0);
+    for (int k = 0; k < K; ++k) {
+      const int row = __shfl_sync(kFull, my_row, k);
+      if (act && row >= 0) stg16(x_perm + static_cast<int64_t>(row) * d + v * V, val);
     }
   }
 }
@@ -261,15 +267,18 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
   scan_kernel<<<1, scan_threads, scan_smem, stream>>>(a.E, nch, a.capacity, a.chunk_hist, a.counts,
                                                                      a.offsets, a.status);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  const size_t smem = sizeof(int32_t) * (kPermWarps * a.E + kChunkSlots);
+  const size_t smem = sizeof(int32_t) * kPermWarps * a.E;
+  scatter_kernel<<<nch, kPermWarps * 32, smem, stream>>>(a.S, a.d, a.E, a.K, a.capacity, tpc, a.topk_idx,
+                                                          a.chunk_hist, a.offsets, a.row_of_slot, a.token_of_row);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  if (a.x == nullptr || a.x_perm == nullptr) return cudaSuccess;
+  const int gblocks = (a.S + kPermWarps - 1) / kPermWarps;
   if (a.act_dtype == MOE_BF16)
-    scatter_kernel<__nv_bfloat16><<<nch, kPermWarps * 32, smem, stream>>>(
-        a.S, a.d, a.E, a.K, a.capacity, tpc, a.topk_idx, a.chunk_hist, a.offsets, a.row_of_slot, a.token_of_row,
-        static_cast<const __nv_bfloat16*>(a.x), static_cast<__nv_bfloat16*>(a.x_perm));
+    gather_rows_kernel<__nv_bfloat16><<<gblocks, kPermWarps * 32, 0, stream>>>(
+        a.S, a.d, a.K, a.row_of_slot, static_cast<const __nv_bfloat16*>(a.x), static_cast<__nv_bfloat16*>(a.x_perm));
   else
-    scatter_kernel<float><<<nch, kPermWarps * 32, smem, stream>>>(
-        a.S, a.d, a.E, a.K, a.capacity, tpc, a.topk_idx, a.chunk_hist, a.offsets, a.row_of_slot, a.token_of_row,
-        static_cast<const float*>(a.x), static_cast<float*>(a.x_perm));
+    gather_rows_kernel<float><<<gblocks, kPermWarps * 32, 0, stream>>>(
+        a.S, a.d, a.K, a.row_of_slot, static_cast<const float*>(a.x), static_cast<float*>(a.x_perm));
   return cudaGetLastError();
 }
 
