@@ -21,8 +21,14 @@ size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 
 struct Layout {
   size_t status, logits, chunk_hist, groups1, groups2, counts, offsets, topk_idx, topk_w, row_of_slot, token_of_row,
-      x_perm, hidden, y_perm, wdeq, total;
+      x_perm, hidden, y_perm, wdeq, ksplit, partial, partial_bytes, total;
 };
+
+// Split-K of the tensor-core GEMMs is available to small row spaces (decode-
+// sized batches), where too few output tiles exist to occupy every SM.  The
+// partial sums take at most this much workspace.
+constexpr int64_t kSplitRowsMax = 4096;
+constexpr int64_t kPartialBudget = int64_t(256) << 20;
 
 int64_t routed_rows(const moe_desc& d) {
   const int64_t sk = static_cast<int64_t>(d.num_tokens) * d.top_k;
@@ -59,6 +65,16 @@ Layout make_layout(const moe_desc& d) {
   L.hidden = take(static_cast<size_t>(Rt * h) * ab);
   L.y_perm = take(static_cast<size_t>(Rt * dm) * ab);
   L.wdeq = take(d.weight_dtype == MOE_E4M3 ? static_cast<size_t>((E + d.num_shared) * 3 * h * dm) * 2 : 0);
+  L.ksplit = take(kAlign);
+  L.partial_bytes = 0;
+  if (d.act_dtype == MOE_BF16 && Rt > 0 && Rt <= kSplitRowsMax) {
+    const int64_t up_cols = d.activation == MOE_ACT_SWIGLU ? 2 * h : h;
+    const int64_t per_split = Rt * (up_cols > dm ? up_cols : dm) * 4;
+    int64_t bytes = 16 * per_split;
+    if (bytes > kPartialBudget) bytes = kPartialBudget;
+    if (bytes >= 2 * per_split) L.partial_bytes = static_cast<size_t>(bytes);
+  }
+  L.partial = take(L.partial_bytes);
   L.total = o;
   return L;
 }
@@ -205,6 +221,9 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
   up.max_total_rows = static_cast<int64_t>(S) * d.top_k + static_cast<int64_t>(d.num_shared) * S;
   up.max_group_rows = S;
   up.status = status;
+  up.partial = L.partial_bytes ? at<float>(ws, L.partial) : nullptr;
+  up.partial_bytes = static_cast<int64_t>(L.partial_bytes);
+  up.ksplit_out = at<int>(ws, L.ksplit);
 
   GemmArgs down = up;
   down.a_rows_from_out = 1;

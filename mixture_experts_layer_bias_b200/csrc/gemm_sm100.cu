@@ -66,6 +66,10 @@ struct TcParams {
   const float* scale1;
   void* out;
   int out_f32;
+  int max_ksplit;      // 1 = no split-K
+  float* partial;      // fp32 [max_ksplit][out_rows][pcols] (split-K partial sums)
+  int pcols;           // 2N (SwiGLU: gate then up) or N
+  int* ksplit_out;     // the split chosen on the device, read by the finalize kernel
   StatusBlock* status;
 };
 
@@ -77,6 +81,7 @@ struct SmemCtl {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  int ksplit;
   int tile_start[kMaxGroups + 1];
 };
 
@@ -108,6 +113,43 @@ __device__ __forceinline__ TileInfo decode_tile(const SmemCtl& s, const TcParams
   ti.n_idx = local / mt;
   ti.m_idx = local - ti.n_idx * mt;
   return ti;
+}
+
+// Split-K factor for `tiles` output tiles on `grid` persistent CTAs: the
+// smallest split whose work units fill the CTAs' waves clearly better
+// (>= 5 points of wave efficiency per step up), with >= 4 K-blocks per unit.
+__device__ __forceinline__ int choose_ksplit(int tiles, int grid, int nk, int kmax) {
+  if (tiles <= 0 || kmax <= 1) return 1;
+  auto eff = [&](int units) {
+    const int waves = (units + grid - 1) / grid;
+    return static_cast<float>(units) / static_cast<float>(waves * grid);
+  };
+  int best = 1;
+  float best_eff = eff(tiles);
+  for (int ks = 2; ks <= kmax; ++ks) {
+    if (nk / ks < 4) break;
+    const float e = eff(tiles * ks);
+    if (e > best_eff + 0.05f) {
+      best = ks;
+      best_eff = e;
+    }
+  }
+  return best;
+}
+
+struct UnitInfo {
+  TileInfo ti;
+  int split, kb0, kb1;
+};
+
+__device__ __forceinline__ UnitInfo decode_unit(const SmemCtl& s, const TcParams& p, int u, int ks, int nk) {
+  UnitInfo ui;
+  const int tt = u / ks;
+  ui.split = u - tt * ks;
+  ui.ti = decode_tile(s, p, tt);
+  ui.kb0 = static_cast<int>((static_cast<int64_t>(ui.split) * nk) / ks);
+  ui.kb1 = static_cast<int>((static_cast<int64_t>(ui.split + 1) * nk) / ks);
+  return ui;
 }
 
 __device__ __forceinline__ bool group_ok(const GroupEntry& g, const TcParams& p) {
@@ -166,6 +208,36 @@ __device__ __forceinline__ void epilogue_store(const TcParams& p, const TileInfo
 #pragma unroll
       for (int j = 0; j < 4; ++j)
         if (n + 8 * j + 8 <= N) stg16(o + 8 * j, pack16<__nv_bfloat16>(v + 8 * j));
+    }
+  }
+}
+
+// Split-K epilogue: raw fp32 accumulators of this unit's K range go to its
+// slice of the partial buffer (SwiGLU: gate columns at n, up columns at N+n).
+template <int EPI>
+__device__ __forceinline__ void epilogue_partial(const TcParams& p, const TileInfo& ti, uint32_t tbase, int row,
+                                                 bool valid, int split) {
+  const int N = p.N;
+  const int64_t orow = static_cast<int64_t>(ti.grp.out_row0) + row;
+  float* base = p.partial + (static_cast<int64_t>(split) * p.out_rows + orow) * p.pcols;
+  constexpr int kChunks = 8;  // 256 accumulator columns
+  for (int c = 0; c < kChunks; ++c) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(tbase + c * 32, r);
+    tmem_ld_wait();
+    if (!valid) continue;
+    int n, col;
+    if (EPI == EPI_SWIGLU) {
+      n = ti.n_idx * p.bn_out + (c & 3) * 32;
+      col = (c < 4 ? 0 : N) + n;
+    } else {
+      n = ti.n_idx * p.bn_out + c * 32;
+      col = n;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (n + 4 * j + 4 <= N)
+        stg16(base + col + 4 * j, make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]));
     }
   }
 }
@@ -230,9 +302,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
 
-  const int total = s.tile_start[p.num_groups];
   const uint32_t tmem = s.tmem_base;
   const int nk = (p.K + BK - 1) / BK;
+  const int tiles = s.tile_start[p.num_groups];
+  const int ks = choose_ksplit(tiles, gridDim.x, nk, p.max_ksplit);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && p.ksplit_out != nullptr) *p.ksplit_out = ks;
+  const int total = tiles * ks;  // work units
   volatile int* abort_flag = &s.abort;
 
   if (warp == 0) {
@@ -241,12 +316,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       uint32_t armed = 0, armed_phase = 0;
       bool ok = true;
-      for (int tt = blockIdx.x; tt < total && ok; tt += gridDim.x) {
-        const TileInfo ti = decode_tile(s, p, tt);
+      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+        const UnitInfo ui = decode_unit(s, p, u, ks, nk);
+        const TileInfo& ti = ui.ti;
         const int a_row = (p.a_rows_from_out ? ti.grp.out_row0 : ti.grp.a_row0) + ti.m_idx * BM;
         const CUtensorMap* mA = (ti.grp.expert == p.shared_slab) ? &tmA2 : &tmA;
         const int b_row = ti.grp.expert * p.n_per_slab + ti.n_idx * p.bn_out;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = ui.kb0; kb < ui.kb1; ++kb) {
           if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -284,7 +360,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
-      for (int tt = blockIdx.x; tt < total && ok; tt += gridDim.x, ++local) {
+      for (int u = blockIdx.x; u < total && ok; u += gridDim.x, ++local) {
+        const int split = u % ks;
+        const int kb0 = static_cast<int>((static_cast<int64_t>(split) * nk) / ks);
+        const int kb1 = static_cast<int>((static_cast<int64_t>(split + 1) * nk) / ks);
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
         if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag)) {
@@ -293,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem + acc * ACC_COLS;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&s.full[stage], phase, abort_flag)) {
             ok = false;
             break;
@@ -304,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             tc_mma_f16(d_tmem, smem_desc_sw128(a_base + kk * 32), smem_desc_sw128(b_base + kk * 32), kIdesc,
-                       (kb | kk) != 0 ? 1u : 0u);
+                       (kb > kb0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(&s.empty[stage]);
           if (++stage == STAGES) {
@@ -327,8 +406,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int local = 0;
-    for (int tt = blockIdx.x; tt < total; tt += gridDim.x, ++local) {
-      const TileInfo ti = decode_tile(s, p, tt);
+    for (int u = blockIdx.x; u < total; u += gridDim.x, ++local) {
+      const UnitInfo ui = decode_unit(s, p, u, ks, nk);
+      const TileInfo& ti = ui.ti;
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!mbar_wait(&s.tfull[acc], acc_phase, abort_flag)) {
@@ -342,7 +422,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = ti.m_idx * BM + q * 32 + lane;
       const bool valid = row < ti.grp.rows;
       const uint32_t tbase = tmem + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16);
-      epilogue_store<EPI>(p, ti, tbase, row, valid);
+      if (ks > 1)
+        epilogue_partial<EPI>(p, ti, tbase, row, valid, ui.split);
+      else
+        epilogue_store<EPI>(p, ti, tbase, row, valid);
       tc_fence_before();
       mbar_arrive(&s.tempty[acc]);
     }
@@ -353,6 +436,56 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// Split-K finalize: for every valid row of every group, sum the partial
+// slices in split order (deterministic), apply scales / bias / activation and
+// store the output row.  Exits at once when the GEMM ran without a split.
+template <int EPI>
+__global__ void __launch_bounds__(256) splitk_finalize_kernel(TcParams p) {
+  const int ks = *p.ksplit_out;
+  if (ks <= 1) return;
+  const GroupEntry grp = p.groups[blockIdx.z];
+  const int r = blockIdx.y;
+  if (r >= grp.rows || grp.expert < 0 || grp.expert >= p.num_slabs) return;
+  const int n = (blockIdx.x * 256 + threadIdx.x) * 4;
+  const int N = p.N;
+  if (n >= N) return;
+  const int64_t orow = static_cast<int64_t>(grp.out_row0) + r;
+  if (orow >= p.out_rows) return;
+  const int64_t sbase = static_cast<int64_t>(grp.expert) * N;
+  const int64_t slice = p.out_rows * static_cast<int64_t>(p.pcols);
+  float v[4] = {0.f, 0.f, 0.f, 0.f}, u[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < ks; ++s) {
+    const float* src = p.partial + s * slice + orow * p.pcols;
+    const float4 a = *reinterpret_cast<const float4*>(src + n);
+    v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+    if (EPI == EPI_SWIGLU) {
+      const float4 b = *reinterpret_cast<const float4*>(src + N + n);
+      u[0] += b.x; u[1] += b.y; u[2] += b.z; u[3] += b.w;
+    }
+  }
+  float o[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float g = v[j];
+    if (p.scale0 != nullptr) g *= p.scale0[sbase + n + j];
+    if (EPI == EPI_SWIGLU) {
+      float up = u[j];
+      if (p.scale1 != nullptr) up *= p.scale1[sbase + n + j];
+      o[j] = g / (1.0f + __expf(-g)) * up;
+    } else {
+      if (EPI == EPI_GELU_BIAS || EPI == EPI_BIAS) g += p.bias[sbase + n + j];
+      if (EPI == EPI_GELU_BIAS) g = 0.5f * g * (1.0f + erff(g * 0.70710678118654752f));
+      o[j] = g;
+    }
+  }
+  if (p.out_f32) {
+    *reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * N + n) = make_float4(o[0], o[1], o[2], o[3]);
+  } else {
+    uint2 packed = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + orow * N + n) = packed;
   }
 }
 
@@ -389,7 +522,7 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int k) {
 
 template <int EPI>
 cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB0, const CUtensorMap& mB1,
-                       const TcParams& p, int grid, cudaStream_t stream) {
+                       const TcParams& p, int grid, int64_t max_group_rows, cudaStream_t stream) {
   static uint64_t attr_set = 0;  // one bit per device ordinal
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -401,6 +534,10 @@ cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUte
     if (dev < 64) attr_set |= 1ull << dev;
   }
   grouped_gemm_tc_kernel<EPI><<<grid, kThreads, kSmemBytes, stream>>>(mA, mA2, mB0, mB1, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || p.max_ksplit <= 1) return e;
+  dim3 fgrid((p.N + 1023) / 1024, static_cast<unsigned>(max_group_rows), p.num_groups);
+  splitk_finalize_kernel<EPI><<<fgrid, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -426,6 +563,17 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t 
   p.out = a.out;
   p.out_f32 = a.out_f32;
   p.status = a.status;
+  p.pcols = a.epilogue == EPI_SWIGLU ? 2 * a.N : a.N;
+  p.partial = a.partial;
+  p.ksplit_out = a.ksplit_out;
+  p.max_ksplit = 1;
+  if (a.partial != nullptr && a.ksplit_out != nullptr && a.partial_bytes > 0) {
+    // as many K slices as the partial buffer holds for every output row
+    const int64_t per_split = a.out_rows * static_cast<int64_t>(p.pcols) * 4;
+    p.max_ksplit = static_cast<int>(per_split > 0 ? a.partial_bytes / per_split : 1);
+    if (p.max_ksplit > 16) p.max_ksplit = 16;
+    if (p.max_ksplit < 1) p.max_ksplit = 1;
+  }
   CUtensorMap mA, mA2, mB0, mB1;
   if (!make_map(&mA, a.a, a.a_rows, a.K)) return cudaErrorInvalidValue;
   if (a.a_shared != nullptr) {
@@ -443,10 +591,10 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t 
   const int64_t bound = (a.max_total_rows / BM + a.num_groups) * static_cast<int64_t>(p.n_tiles);
   const int grid = static_cast<int>(bound < num_sms ? (bound > 0 ? bound : 1) : num_sms);
   switch (a.epilogue) {
-    case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(mA, mA2, mB0, mB1, p, grid, stream);
-    case EPI_GELU_BIAS: return launch_epi<EPI_GELU_BIAS>(mA, mA2, mB0, mB1, p, grid, stream);
-    case EPI_BIAS: return launch_epi<EPI_BIAS>(mA, mA2, mB0, mB1, p, grid, stream);
-    case EPI_NONE: return launch_epi<EPI_NONE>(mA, mA2, mB0, mB1, p, grid, stream);
+    case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(mA, mA2, mB0, mB1, p, grid, a.max_group_rows, stream);
+    case EPI_GELU_BIAS: return launch_epi<EPI_GELU_BIAS>(mA, mA2, mB0, mB1, p, grid, a.max_group_rows, stream);
+    case EPI_BIAS: return launch_epi<EPI_BIAS>(mA, mA2, mB0, mB1, p, grid, a.max_group_rows, stream);
+    case EPI_NONE: return launch_epi<EPI_NONE>(mA, mA2, mB0, mB1, p, grid, a.max_group_rows, stream);
     default: return cudaErrorInvalidValue;
   }
 }

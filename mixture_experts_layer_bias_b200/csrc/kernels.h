@@ -85,6 +85,9 @@ struct GemmArgs {
   int out_f32;              // 1: fp32 output, 0: bf16
   int64_t max_total_rows;   // upper bound of the rows of all groups together
   int64_t max_group_rows;   // upper bound of the rows of one group
+  float* partial;           // split-K partial sums (nullptr = no split-K)
+  int64_t partial_bytes;    // size of `partial`
+  int* ksplit_out;          // device int: the split the GEMM chose
   StatusBlock* status;
 };
 cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t stream);

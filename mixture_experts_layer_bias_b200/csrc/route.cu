@@ -283,6 +283,51 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
   select_topk<1>(l, p, t);
 }
 
+// Small batches (decode): one CTA per token, its 8 warps split d so the
+// token's dot products are not serialised on one warp.  Per-warp partial sums
+// are added in warp order (deterministic), then warp 0 selects.
+template <typename T, int EMAX>
+__global__ void __launch_bounds__(kRouteWarps * 32)
+    route_token_cta_kernel(int d, const T* __restrict__ x, const T* __restrict__ w_router,
+                           const float* __restrict__ router_bias, SelectParams p) {
+  __shared__ float part[kRouteWarps][EMAX];
+  const int t = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = lane_id();
+  constexpr int V = Vec16<T>::N;
+  const int nvec = d / V;
+  float acc[EMAX];
+#pragma unroll
+  for (int e = 0; e < EMAX; ++e) acc[e] = 0.0f;
+  const T* xr = x + static_cast<int64_t>(t) * d;
+  for (int v = threadIdx.x; v < nvec; v += kRouteWarps * 32) {
+    float xf[V];
+    unpack16<T>(ldg16(xr + v * V), xf);
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) {
+      if (e < p.E) {
+        float wf[V];
+        unpack16<T>(ldg16(w_router + static_cast<int64_t>(e) * d + v * V), wf);
+#pragma unroll
+        for (int j = 0; j < V; ++j) acc[e] = fmaf(xf[j], wf[j], acc[e]);
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < EMAX; ++e) {
+    const float s = warp_sum(acc[e]);
+    if (lane == 0) part[warp][e] = s;
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  float l[1] = {0.0f};
+  if (lane < p.E && lane < EMAX) {
+    float s = 0.0f;
+    for (int w = 0; w < kRouteWarps; ++w) s += part[w][lane];
+    l[0] = router_bias != nullptr ? __fadd_rn(s, __ldg(router_bias + lane)) : s;
+  }
+  select_topk<1>(l, p, t);
+}
+
 // Logits given in memory (caller-supplied, or computed by the logits kernel).
 template <int NI>
 __global__ void __launch_bounds__(kRouteWarps * 32)
@@ -363,23 +408,30 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
   const int blocks = (a.S + kRouteWarps - 1) / kRouteWarps;
   const float* logits = a.logits;
   if (logits == nullptr && a.E <= 32) {
+    // decode-sized batches: a CTA per token; otherwise a warp per token
+    const bool per_cta = a.S <= 512;
+    const int g = per_cta ? a.S : blocks;
+#define MOE_ROUTE_LAUNCH(T, EM)                                                                                \
+  do {                                                                                                         \
+    if (per_cta)                                                                                               \
+      route_token_cta_kernel<T, EM><<<g, kRouteWarps * 32, 0, stream>>>(                                       \
+          a.d, static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);              \
+    else                                                                                                       \
+      route_fused_kernel<T, EM><<<g, kRouteWarps * 32, 0, stream>>>(                                           \
+          a.S, a.d, static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);         \
+  } while (0)
     if (a.act_dtype == MOE_BF16) {
       if (a.E <= 8)
-        route_fused_kernel<__nv_bfloat16, 8><<<blocks, kRouteWarps * 32, 0, stream>>>(
-            a.S, a.d, static_cast<const __nv_bfloat16*>(a.x), static_cast<const __nv_bfloat16*>(a.w_router),
-            a.router_bias, sp);
+        MOE_ROUTE_LAUNCH(__nv_bfloat16, 8);
       else
-        route_fused_kernel<__nv_bfloat16, 32><<<blocks, kRouteWarps * 32, 0, stream>>>(
-            a.S, a.d, static_cast<const __nv_bfloat16*>(a.x), static_cast<const __nv_bfloat16*>(a.w_router),
-            a.router_bias, sp);
+        MOE_ROUTE_LAUNCH(__nv_bfloat16, 32);
     } else {
       if (a.E <= 8)
-        route_fused_kernel<float, 8><<<blocks, kRouteWarps * 32, 0, stream>>>(
-            a.S, a.d, static_cast<const float*>(a.x), static_cast<const float*>(a.w_router), a.router_bias, sp);
+        MOE_ROUTE_LAUNCH(float, 8);
       else
-        route_fused_kernel<float, 32><<<blocks, kRouteWarps * 32, 0, stream>>>(
-            a.S, a.d, static_cast<const float*>(a.x), static_cast<const float*>(a.w_router), a.router_bias, sp);
+        MOE_ROUTE_LAUNCH(float, 32);
     }
+#undef MOE_ROUTE_LAUNCH
     return cudaGetLastError();
   }
   if (logits == nullptr) {

@@ -314,6 +314,20 @@ def test_grouped_ffn_fp8_weights(S, d, h, E, K):
     assert rel_l2(got, ref) <= FP8_REL_L2
 
 
+@pytest.mark.parametrize("S,d,h,E,K,extra", [
+    (2, 2048, 1024, 8, 2, {}),                                   # few tiles, long K: split-K on both GEMMs
+    (3, 1024, 2048, 8, 2, {"activation": syn.GELU}),              # GeLU + bias applied after the split sum
+    (4, 2048, 1408, 8, 2, {"weight_dtype": syn.E4M3}),            # FP8 scales applied after the split sum
+    (5, 1024, 512, 16, 4, {"num_shared": 1}),                     # shared expert group in the split GEMMs
+    (128, 4096, 1024, 8, 2, {}),                                  # decode-sized batch, full model width
+])
+def test_grouped_ffn_split_k(S, d, h, E, K, extra):
+    cfg = syn.LayerConfig("t", S=S, d=d, E=E, K=K, h=h, router_offset_var=0.5, **extra)
+    got, ref = _ffn_case(cfg)
+    lim = FP8_REL_L2 if cfg.weight_dtype == syn.E4M3 else BF16_REL_L2
+    assert rel_l2(got, ref) <= lim
+
+
 def test_grouped_ffn_bf16_gelu_bias():
     cfg = syn.LayerConfig("t", S=150, d=256, E=8, K=2, h=256, activation=syn.GELU)
     got, ref = _ffn_case(cfg)
