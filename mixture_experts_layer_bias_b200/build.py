@@ -44,8 +44,8 @@ def headers():
     return hs
 
 
-def _compile(src: str, force: bool, extra) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+def _compile(src: str, force: bool, extra, build_dir: str = BUILD) -> str:
+    obj = os.path.join(build_dir, os.path.basename(src) + ".o")
     newest_dep = max(os.path.getmtime(p) for p in [src] + headers())
     if not force and os.path.exists(obj) and os.path.getmtime(obj) >= newest_dep:
         return obj
@@ -56,19 +56,21 @@ def _compile(src: str, force: bool, extra) -> str:
     return obj
 
 
-def build(force: bool = False, jobs: int = 8, extra=()) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, jobs: int = 8, extra=(), out: str = LIB, build_dir: str = BUILD) -> str:
+    """Compile every source (extra nvcc flags, e.g. -D tuning macros, go to
+    all of them) into build_dir and link `out`."""
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sources()
     with cf.ThreadPoolExecutor(max_workers=jobs) as ex:
-        objs = list(ex.map(lambda s: _compile(s, force, extra), srcs))
-    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
-        tmp = LIB + ".tmp"
+        objs = list(ex.map(lambda s: _compile(s, force, extra, build_dir), srcs))
+    if force or not os.path.exists(out) or os.path.getmtime(out) < max(os.path.getmtime(o) for o in objs):
+        tmp = out + ".tmp"
         cmd = [nvcc()] + ARCH + ["-shared", "-o", tmp] + objs
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, out)
+    return out
 
 
 def main(argv=None):
@@ -76,9 +78,14 @@ def main(argv=None):
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-j", type=int, default=8)
     ap.add_argument("--ptxas-verbose", action="store_true")
+    ap.add_argument("-D", dest="defines", action="append", default=[], help="extra -D macro for every source")
+    ap.add_argument("--out", default=LIB, help="library path (variants go elsewhere)")
+    ap.add_argument("--build-dir", default=BUILD)
     a = ap.parse_args(argv)
     extra = ["-Xptxas", "-v"] if a.ptxas_verbose else []
-    print(build(force=a.force or a.ptxas_verbose, jobs=a.j, extra=extra))
+    extra += ["-D" + d for d in a.defines]
+    print(build(force=a.force or a.ptxas_verbose or bool(a.defines), jobs=a.j, extra=extra, out=a.out,
+                build_dir=a.build_dir))
 
 
 if __name__ == "__main__":

@@ -161,6 +161,7 @@ moe_status route_impl(const moe_desc& d, const moe_weights* w, const void* x, co
   a.topk_idx = topk_idx;
   a.topk_w = topk_w;
   a.status = at<StatusBlock>(ws, L.status);
+  a.num_sms = num_sms();
   return cuda_status(launch_route(a, st));
 }
 

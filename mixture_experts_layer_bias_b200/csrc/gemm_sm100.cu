@@ -51,7 +51,8 @@ constexpr int kMaxGroups = 264;
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, 256);
 
 struct TcParams {
-  const GroupEntry* groups;
+  const GroupEntry* groups;  // nullptr: one group of `single_rows` rows, slab 0
+  int single_rows;
   int num_groups;
   int shared_slab;
   int a_rows_from_out;
@@ -92,6 +93,11 @@ __device__ __forceinline__ bool wait_timed(uint64_t* bar, uint32_t parity) {
   return mbar_wait(bar, parity, &never);
 }
 
+__device__ __forceinline__ GroupEntry group_at(const TcParams& p, int g) {
+  if (p.groups == nullptr) return GroupEntry{0, 0, p.single_rows, 0};
+  return p.groups[g];
+}
+
 struct TileInfo {
   GroupEntry grp;
   int m_idx, n_idx;
@@ -107,7 +113,7 @@ __device__ __forceinline__ TileInfo decode_tile(const SmemCtl& s, const TcParams
       hi = mid;
   }
   TileInfo ti;
-  ti.grp = p.groups[lo];
+  ti.grp = group_at(p, lo);
   const int mt = (ti.grp.rows + BM - 1) / BM;
   const int local = tt - s.tile_start[lo];
   ti.n_idx = local / mt;
@@ -259,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int g = base + lane;
       int tiles = 0;
       if (g < p.num_groups) {
-        const GroupEntry ge = p.groups[g];
+        const GroupEntry ge = group_at(p, g);
         if (group_ok(ge, p))
           tiles = ((ge.rows + BM - 1) / BM) * p.n_tiles;
         else if (ge.rows != 0)
@@ -446,7 +452,7 @@ template <int EPI>
 __global__ void __launch_bounds__(256) splitk_finalize_kernel(TcParams p) {
   const int ks = *p.ksplit_out;
   if (ks <= 1) return;
-  const GroupEntry grp = p.groups[blockIdx.z];
+  const GroupEntry grp = group_at(p, blockIdx.z);
   const int r = blockIdx.y;
   if (r >= grp.rows || grp.expert < 0 || grp.expert >= p.num_slabs) return;
   const int n = (blockIdx.x * 256 + threadIdx.x) * 4;
@@ -545,8 +551,10 @@ cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUte
 
 cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t stream) {
   if (a.num_groups <= 0 || a.num_groups > kMaxGroups) return cudaErrorInvalidValue;
+  if (a.groups == nullptr && (a.num_groups != 1 || a.max_total_rows > INT32_MAX)) return cudaErrorInvalidValue;
   TcParams p;
   p.groups = a.groups;
+  p.single_rows = a.groups == nullptr ? static_cast<int>(a.max_total_rows) : 0;
   p.num_groups = a.num_groups;
   p.shared_slab = a.shared_slab;
   p.a_rows_from_out = a.a_rows_from_out;

@@ -25,6 +25,7 @@ struct RouteArgs {
   int32_t* topk_idx;        // [S][K]
   float* topk_w;            // [S][K]
   StatusBlock* status;
+  int num_sms;
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream);
 
@@ -64,7 +65,7 @@ enum Epilogue { EPI_SWIGLU = 0, EPI_GELU_BIAS = 1, EPI_BIAS = 2, EPI_NONE = 3 };
 
 struct GemmArgs {
   int epilogue;
-  const GroupEntry* groups;
+  const GroupEntry* groups;  // nullptr: a single group of max_total_rows rows (slab 0, rows from 0)
   int num_groups;
   int shared_slab;          // slab index whose A rows come from a_shared, -1 = none
   int a_rows_from_out;      // 1: A row = out_row0 + r (down projection), 0: a_row0 + r

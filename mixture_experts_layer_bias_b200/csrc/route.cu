@@ -435,16 +435,40 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
     return cudaGetLastError();
   }
   if (logits == nullptr) {
-    dim3 grid((a.S + 31) / 32, (a.E + 63) / 64);
-    if (a.act_dtype == MOE_BF16)
-      logits_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(a.S, a.d, a.E,
-                                                              static_cast<const __nv_bfloat16*>(a.x),
-                                                              static_cast<const __nv_bfloat16*>(a.w_router),
-                                                              a.logits_scratch);
-    else
-      logits_kernel<float><<<grid, 256, 0, stream>>>(a.S, a.d, a.E, static_cast<const float*>(a.x),
-                                                      static_cast<const float*>(a.w_router), a.logits_scratch);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err;
+    if (a.act_dtype == MOE_BF16 && a.d % 8 == 0) {
+      // l = x W_r^T as one dense GEMM on the tensor cores (fp32 accumulate
+      // and output); the selection then reads the logits back
+      GemmArgs g{};
+      g.epilogue = EPI_NONE;
+      g.groups = nullptr;
+      g.num_groups = 1;
+      g.shared_slab = -1;
+      g.a = a.x;
+      g.a_rows = a.S;
+      g.b0 = a.w_router;
+      g.b_rows = a.E;
+      g.n_per_slab = a.E;
+      g.N = a.E;
+      g.K = a.d;
+      g.out = a.logits_scratch;
+      g.out_rows = a.S;
+      g.out_f32 = 1;
+      g.max_total_rows = a.S;
+      g.max_group_rows = a.S;
+      g.status = a.status;
+      err = launch_grouped_gemm_tc(g, a.num_sms, stream);
+    } else {
+      dim3 grid((a.S + 31) / 32, (a.E + 63) / 64);
+      if (a.act_dtype == MOE_BF16)
+        logits_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(a.S, a.d, a.E, static_cast<const __nv_bfloat16*>(a.x),
+                                                                static_cast<const __nv_bfloat16*>(a.w_router),
+                                                                a.logits_scratch);
+      else
+        logits_kernel<float><<<grid, 256, 0, stream>>>(a.S, a.d, a.E, static_cast<const float*>(a.x),
+                                                        static_cast<const float*>(a.w_router), a.logits_scratch);
+      err = cudaGetLastError();
+    }
     if (err != cudaSuccess) return err;
     logits = a.logits_scratch;
   }

@@ -14,7 +14,10 @@ from typing import Optional
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
+# MOE_B200_LIB may point at another build of the same library (e.g. a variant
+# compiled with different tuning macros).
+_LIB_PATH = os.environ.get("MOE_B200_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                                                           "libmoe_b200.so")
 _lib = None
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE_STATUS = range(6)
