@@ -31,12 +31,16 @@
 // in flight, frees its TMEM and exits.  No load uses cluster multicast.
 #include <math.h>
 
-#include "common.cuh"
-#include "kernels.h"
+#include <stdlib.h>
+#include <string.h>
+
+#include "gemm_common.cuh"
 
 namespace moe {
 
 namespace {
+
+using namespace gemm;
 
 constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = 128 bytes = one swizzle row
@@ -47,32 +51,7 @@ constexpr int STAGE_BYTES = A_TILE + 2 * B_HALF;  // 48 KB
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
 constexpr int kThreads = 192;
-constexpr int kMaxGroups = 264;
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, 256);
-
-struct TcParams {
-  const GroupEntry* groups;  // nullptr: one group of `single_rows` rows, slab 0
-  int single_rows;
-  int num_groups;
-  int shared_slab;
-  int a_rows_from_out;
-  int num_slabs;
-  int n_per_slab;
-  int N, K;
-  int bn_out;   // output columns per tile (128 SwiGLU, 256 otherwise)
-  int n_tiles;  // ceil(N / bn_out)
-  int64_t out_rows;
-  const float* bias;
-  const float* scale0;
-  const float* scale1;
-  void* out;
-  int out_f32;
-  int max_ksplit;      // 1 = no split-K
-  float* partial;      // fp32 [max_ksplit][out_rows][pcols] (split-K partial sums)
-  int pcols;           // 2N (SwiGLU: gate then up) or N
-  int* ksplit_out;     // the split chosen on the device, read by the finalize kernel
-  StatusBlock* status;
-};
 
 struct SmemCtl {
   uint64_t full[STAGES];
@@ -91,11 +70,6 @@ constexpr size_t kSmemBytes = STAGES * STAGE_BYTES + sizeof(SmemCtl) + 1024;
 __device__ __forceinline__ bool wait_timed(uint64_t* bar, uint32_t parity) {
   int never = 0;
   return mbar_wait(bar, parity, &never);
-}
-
-__device__ __forceinline__ GroupEntry group_at(const TcParams& p, int g) {
-  if (p.groups == nullptr) return GroupEntry{0, 0, p.single_rows, 0};
-  return p.groups[g];
 }
 
 struct TileInfo {
@@ -121,28 +95,6 @@ __device__ __forceinline__ TileInfo decode_tile(const SmemCtl& s, const TcParams
   return ti;
 }
 
-// Split-K factor for `tiles` output tiles on `grid` persistent CTAs: the
-// smallest split whose work units fill the CTAs' waves clearly better
-// (>= 5 points of wave efficiency per step up), with >= 4 K-blocks per unit.
-__device__ __forceinline__ int choose_ksplit(int tiles, int grid, int nk, int kmax) {
-  if (tiles <= 0 || kmax <= 1) return 1;
-  auto eff = [&](int units) {
-    const int waves = (units + grid - 1) / grid;
-    return static_cast<float>(units) / static_cast<float>(waves * grid);
-  };
-  int best = 1;
-  float best_eff = eff(tiles);
-  for (int ks = 2; ks <= kmax; ++ks) {
-    if (nk / ks < 4) break;
-    const float e = eff(tiles * ks);
-    if (e > best_eff + 0.05f) {
-      best = ks;
-      best_eff = e;
-    }
-  }
-  return best;
-}
-
 struct UnitInfo {
   TileInfo ti;
   int split, kb0, kb1;
@@ -156,11 +108,6 @@ __device__ __forceinline__ UnitInfo decode_unit(const SmemCtl& s, const TcParams
   ui.kb0 = static_cast<int>((static_cast<int64_t>(ui.split) * nk) / ks);
   ui.kb1 = static_cast<int>((static_cast<int64_t>(ui.split + 1) * nk) / ks);
   return ui;
-}
-
-__device__ __forceinline__ bool group_ok(const GroupEntry& g, const TcParams& p) {
-  return g.rows > 0 && g.expert >= 0 && g.expert < p.num_slabs && g.out_row0 >= 0 &&
-         static_cast<int64_t>(g.out_row0) + g.rows <= p.out_rows && g.a_row0 >= 0;
 }
 
 template <int EPI>
@@ -445,87 +392,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Split-K finalize: for every valid row of every group, sum the partial
-// slices in split order (deterministic), apply scales / bias / activation and
-// store the output row.  Exits at once when the GEMM ran without a split.
-template <int EPI>
-__global__ void __launch_bounds__(256) splitk_finalize_kernel(TcParams p) {
-  const int ks = *p.ksplit_out;
-  if (ks <= 1) return;
-  const GroupEntry grp = group_at(p, blockIdx.z);
-  const int r = blockIdx.y;
-  if (r >= grp.rows || grp.expert < 0 || grp.expert >= p.num_slabs) return;
-  const int n = (blockIdx.x * 256 + threadIdx.x) * 4;
-  const int N = p.N;
-  if (n >= N) return;
-  const int64_t orow = static_cast<int64_t>(grp.out_row0) + r;
-  if (orow >= p.out_rows) return;
-  const int64_t sbase = static_cast<int64_t>(grp.expert) * N;
-  const int64_t slice = p.out_rows * static_cast<int64_t>(p.pcols);
-  float v[4] = {0.f, 0.f, 0.f, 0.f}, u[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int s = 0; s < ks; ++s) {
-    const float* src = p.partial + s * slice + orow * p.pcols;
-    const float4 a = *reinterpret_cast<const float4*>(src + n);
-    v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
-    if (EPI == EPI_SWIGLU) {
-      const float4 b = *reinterpret_cast<const float4*>(src + N + n);
-      u[0] += b.x; u[1] += b.y; u[2] += b.z; u[3] += b.w;
-    }
-  }
-  float o[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    float g = v[j];
-    if (p.scale0 != nullptr) g *= p.scale0[sbase + n + j];
-    if (EPI == EPI_SWIGLU) {
-      float up = u[j];
-      if (p.scale1 != nullptr) up *= p.scale1[sbase + n + j];
-      o[j] = g / (1.0f + __expf(-g)) * up;
-    } else {
-      if (EPI == EPI_GELU_BIAS || EPI == EPI_BIAS) g += p.bias[sbase + n + j];
-      if (EPI == EPI_GELU_BIAS) g = 0.5f * g * (1.0f + erff(g * 0.70710678118654752f));
-      o[j] = g;
-    }
-  }
-  if (p.out_f32) {
-    *reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * N + n) = make_float4(o[0], o[1], o[2], o[3]);
-  } else {
-    uint2 packed = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
-    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + orow * N + n) = packed;
-  }
-}
-
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
-// 2-D bf16 map over [rows][k] (row-major), box 64 (k) x 128 rows, 128B swizzle.
-bool make_map(CUtensorMap* m, const void* base, int64_t rows, int k) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (enc == nullptr || rows <= 0 || k <= 0) return false;
-  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || (static_cast<int64_t>(k) * 2) % 16 != 0) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(k) * 2};
-  cuuint32_t box[2] = {BK, 128};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int EPI>
 cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB0, const CUtensorMap& mB1,
                        const TcParams& p, int grid, int64_t max_group_rows, cudaStream_t stream) {
@@ -548,6 +414,16 @@ cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUte
 }
 
 }  // namespace
+
+// Kernel choice: the CTA-pair kernel unless MOE_B200_GEMM=single (read once).
+static bool use_pair_kernel() {
+  static int choice = -1;
+  if (choice < 0) {
+    const char* v = getenv("MOE_B200_GEMM");
+    choice = (v != nullptr && strcmp(v, "single") == 0) ? 0 : 1;
+  }
+  return choice == 1;
+}
 
 cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t stream) {
   if (a.num_groups <= 0 || a.num_groups > kMaxGroups) return cudaErrorInvalidValue;
@@ -582,6 +458,7 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t 
     if (p.max_ksplit > 16) p.max_ksplit = 16;
     if (p.max_ksplit < 1) p.max_ksplit = 1;
   }
+  if (use_pair_kernel()) return launch_grouped_gemm_pair(a, p, num_sms, stream);
   CUtensorMap mA, mA2, mB0, mB1;
   if (!make_map(&mA, a.a, a.a_rows, a.K)) return cudaErrorInvalidValue;
   if (a.a_shared != nullptr) {

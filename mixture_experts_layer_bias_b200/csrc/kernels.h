@@ -92,6 +92,10 @@ struct GemmArgs {
   StatusBlock* status;
 };
 cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t stream);
+namespace gemm {
+struct TcParams;
+}
+cudaError_t launch_grouped_gemm_pair(const GemmArgs& a, const gemm::TcParams& p, int num_sms, cudaStream_t stream);
 cudaError_t launch_grouped_gemm_f32(const GemmArgs& a, cudaStream_t stream);
 
 // FP8-E4M3 weight slabs -> bf16 (exact)
