@@ -97,16 +97,18 @@ __device__ __forceinline__ bool wait_timed_pair(uint64_t* bar, uint32_t parity) 
   return mbar_wait(bar, parity, &never);
 }
 
-// Epilogue of one 32-token chunk: v[j] is the accumulator of this thread's
-// TMEM lane (weight row) for token tb*256 + chunk*32 + j.
+constexpr int P_CHUNK = 16;  // tokens per epilogue chunk (one 32x32b.x16 TMEM load)
+
+// Epilogue of one 16-token chunk: r[j] is the accumulator of this thread's
+// TMEM lane (weight row) for token tb*256 + chunk*16 + j.
 template <int EPI>
 __device__ __forceinline__ void pair_store_chunk(const TcParams& p, const PairUnit& pu, uint32_t rank, int q, int lane,
-                                                 int chunk, const uint32_t (&r)[32], int ks) {
+                                                 int chunk, const uint32_t (&r)[P_CHUNK], int ks) {
   const int N = p.N;
-  const int t0 = pu.tb * P_TOK + chunk * 32;  // first token of the chunk inside the group
+  const int t0 = pu.tb * P_TOK + chunk * P_CHUNK;  // first token of the chunk inside the group
   const int64_t row0 = static_cast<int64_t>(pu.grp.out_row0) + t0;
   const int64_t sbase = static_cast<int64_t>(pu.grp.expert) * N;
-  const int tlim = min(32, pu.grp.rows - t0);  // valid tokens in this chunk
+  const int tlim = min(P_CHUNK, pu.grp.rows - t0);  // valid tokens in this chunk
   if (EPI == EPI_SWIGLU) {
     const int blk = q * 2 + (lane >> 4);  // 16-row block of this CTA's weight rows
     const bool is_up = blk & 1;
@@ -116,7 +118,7 @@ __device__ __forceinline__ void pair_store_chunk(const TcParams& p, const PairUn
       if (!fvalid) return;
       float* base = p.partial + (static_cast<int64_t>(pu.split) * p.out_rows + row0) * p.pcols + (is_up ? N : 0) + f;
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
+      for (int j = 0; j < P_CHUNK; ++j)
         if (j < tlim) base[static_cast<int64_t>(j) * p.pcols] = __uint_as_float(r[j]);
       return;
     }
@@ -127,7 +129,7 @@ __device__ __forceinline__ void pair_store_chunk(const TcParams& p, const PairUn
     }
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row0 * N + f;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
+    for (int j = 0; j < P_CHUNK; ++j) {
       const float mine = __uint_as_float(r[j]);
       const float up = __shfl_xor_sync(0xFFFFFFFFu, mine, 16);
       if (!is_up && fvalid && j < tlim) {
@@ -141,14 +143,14 @@ __device__ __forceinline__ void pair_store_chunk(const TcParams& p, const PairUn
     if (ks > 1) {
       float* base = p.partial + (static_cast<int64_t>(pu.split) * p.out_rows + row0) * p.pcols + f;
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
+      for (int j = 0; j < P_CHUNK; ++j)
         if (j < tlim) base[static_cast<int64_t>(j) * p.pcols] = __uint_as_float(r[j]);
       return;
     }
     const float sc = p.scale0 != nullptr ? __ldg(p.scale0 + sbase + f) : 1.0f;
     const float bi = (EPI == EPI_GELU_BIAS || EPI == EPI_BIAS) ? __ldg(p.bias + sbase + f) : 0.0f;
-#pragma unroll 8
-    for (int j = 0; j < 32; ++j) {
+#pragma unroll
+    for (int j = 0; j < P_CHUNK; ++j) {
       if (j >= tlim) break;
       float z = __uint_as_float(r[j]) * sc + bi;
       if (EPI == EPI_GELU_BIAS) z = 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
@@ -355,10 +357,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
       }
       tc_fence_after();
       const uint32_t tbase = tmem + acc * P_ACC_COLS + (static_cast<uint32_t>(q * 32) << 16);
-      const int nchunks = (pu.nt + 31) / 32;
+      const int nchunks = (pu.nt + P_CHUNK - 1) / P_CHUNK;
       for (int c = 0; c < nchunks; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tbase + c * 32, r);
+        uint32_t r[P_CHUNK];
+        tmem_ld_32x32b_x16(tbase + c * P_CHUNK, r);
         tmem_ld_wait();
         pair_store_chunk<EPI>(p, pu, rank, q, lane, c, r, ks);
       }
