@@ -415,12 +415,12 @@ cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUte
 
 }  // namespace
 
-// Kernel choice: the CTA-pair kernel unless MOE_B200_GEMM=single (read once).
+// Kernel choice: the one-CTA kernel unless MOE_B200_GEMM=pair (read once).
 static bool use_pair_kernel() {
   static int choice = -1;
   if (choice < 0) {
     const char* v = getenv("MOE_B200_GEMM");
-    choice = (v != nullptr && strcmp(v, "single") == 0) ? 0 : 1;
+    choice = (v != nullptr && strcmp(v, "pair") == 0) ? 1 : 0;
   }
   return choice == 1;
 }
