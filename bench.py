@@ -354,8 +354,10 @@ def main():
     ffn_ms = stages["grouped_ffn"]
     achieved = flops / (ffn_ms * 1e-3) / 1e12
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": None,
+                "frac": round(achieved / peak, 4), "frac_of_sustained_peak": round(achieved / sustained, 4),
+                "traffic": None,
                 "kernel": "grouped expert FFN (up SwiGLU + down GEMMs, tcgen05)",
                 "peak_source": f"{peaks['source']} bf16 burst"}
 
