@@ -78,6 +78,21 @@ def kernels_per_step(cfg):
     return n
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The largest `value` over all ranks (identity outside a process group)."""
+    import torch.distributed as td
+    if not (td.is_available() and td.is_initialized()) or td.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    td.all_reduce(t, op=td.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, max_ms: float, world: int) -> float:
+    """Units all ranks processed per second, timed by the slowest rank."""
+    return world * units_per_rank / (max_ms * 1e-3)
+
+
 def expert_flops(cfg, rows):
     per_row = (6 if cfg.activation == syn.SWIGLU else 4) * cfg.d * cfg.h
     return rows * per_row
@@ -333,16 +348,12 @@ def main():
     if dist:
         td.barrier()
     clk = clocks.stop()
-    total_ms = start.elapsed_time(stop)
-    if dist:
-        t = torch.tensor([total_ms], device=device)
-        td.all_reduce(t, op=td.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(start.elapsed_time(stop), device)
     stage_names = ("route", "permute", "grouped_ffn", "combine")
     stages = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
               for j, n in enumerate(stage_names)}
     ms_per_step = total_ms / args.steps
-    value = world * S * args.steps / (total_ms * 1e-3)
+    value = whole_job_rate(S * args.steps, total_ms, world)
 
     code, flags, counters = ops.moe_get_status(ws)
     if flags:
@@ -383,12 +394,8 @@ def main():
         e2e_step()
     e2e_ev[1].record()
     torch.cuda.synchronize()
-    e2e_ms = e2e_ev[0].elapsed_time(e2e_ev[1])
-    if dist:
-        t = torch.tensor([e2e_ms], device=device)
-        td.all_reduce(t, op=td.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": round(world * S * args.steps / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+    e2e_ms = max_over_ranks(e2e_ev[0].elapsed_time(e2e_ev[1]), device)
+    e2e = {"value": round(whole_job_rate(S * args.steps, e2e_ms, world), 1), "unit": "tokens/s",
            "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
            "d2h_bytes_per_step": y_host.numel() * y_host.element_size()}
 

@@ -166,7 +166,8 @@ moe_status route_impl(const moe_desc& d, const moe_weights* w, const void* x, co
 }
 
 moe_status permute_impl(const moe_desc& d, const void* x, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
-                        int32_t* row_of_slot, int32_t* token_of_row, void* x_perm, void* ws, cudaStream_t st) {
+                        int32_t* row_of_slot, int32_t* token_of_row, void* x_perm, void* ws, cudaStream_t st,
+                        bool write_groups = false) {
   const Layout L = make_layout(d);
   PermuteArgs a{};
   a.S = d.num_tokens;
@@ -185,11 +186,16 @@ moe_status permute_impl(const moe_desc& d, const void* x, const int32_t* topk_id
   a.x_perm = x_perm;
   a.num_rows = routed_rows(d);
   a.status = at<StatusBlock>(ws, L.status);
+  if (write_groups) {
+    a.g1 = at<GroupEntry>(ws, L.groups1);
+    a.g2 = at<GroupEntry>(ws, L.groups2);
+    a.num_shared = d.num_shared;
+  }
   return cuda_status(launch_permute(a, st));
 }
 
 moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm, const int32_t* offsets, const void* x,
-                    void* y_perm, void* ws, cudaStream_t st) {
+                    void* y_perm, void* ws, cudaStream_t st, bool groups_ready = false) {
   const Layout L = make_layout(d);
   const int S = d.num_tokens, E = d.num_experts, h = d.d_ff, dm = d.d_model;
   if (S == 0) return MOE_OK;
@@ -198,8 +204,11 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
   StatusBlock* status = at<StatusBlock>(ws, L.status);
   GroupEntry* g1 = at<GroupEntry>(ws, L.groups1);
   GroupEntry* g2 = at<GroupEntry>(ws, L.groups2);
-  cudaError_t err = launch_build_groups(S, E, d.top_k, d.capacity, d.num_shared, offsets, g1, g2, status, st);
-  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  cudaError_t err = cudaSuccess;
+  if (!groups_ready) {
+    err = launch_build_groups(S, E, d.top_k, d.capacity, d.num_shared, offsets, g1, g2, status, st);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+  }
   const int slabs = E + d.num_shared;
   void* hidden = at<void>(ws, L.hidden);
 
@@ -426,8 +435,9 @@ moe_status moe_layer_forward(const moe_desc* desc, const moe_weights* w, const v
   void* x_perm = at<void>(ws, L.x_perm);
   void* y_perm = at<void>(ws, L.y_perm);
   if ((s = route_impl(d, w, x, nullptr, idx, gates, ws, st)) != MOE_OK) return s;
-  if ((s = permute_impl(d, x, idx, cnt, offs, ros, tor, x_perm, ws, st)) != MOE_OK) return s;
-  if ((s = ffn_impl(d, *w, x_perm, offs, x, y_perm, ws, st)) != MOE_OK) return s;
+  // the permutation also writes the GEMM group tables, so the FFN skips that launch
+  if ((s = permute_impl(d, x, idx, cnt, offs, ros, tor, x_perm, ws, st, true)) != MOE_OK) return s;
+  if ((s = ffn_impl(d, *w, x_perm, offs, x, y_perm, ws, st, true)) != MOE_OK) return s;
   return combine_impl(d, y_perm, ros, gates, y, st);
 }
 

@@ -5,9 +5,9 @@
 // original token order); plumephp.com "MoE 混合专家推理", worked example:
 // output = 0.55 * e0(x) + 0.30 * e3(x), normalised.
 //
-// One warp per token; lanes stride over 16-byte vectors of the d_model row;
-// fp32 sums in k order, then the shared expert's row (gate 1), one rounding
-// to the output type at the end.
+// One warp per token (one CTA per token for S <= 256); lanes stride over
+// 16-byte vectors of the d_model row; fp32 sums in k order, then the shared
+// expert's row (gate 1), one rounding to the output type at the end.
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -62,6 +62,42 @@ __global__ void __launch_bounds__(kCombWarps * 32)
   }
 }
 
+// Small batches: one CTA per token, its threads split the row.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    combine_cta_kernel(int d, int K, const T* __restrict__ y_perm, const int32_t* __restrict__ row_of_slot,
+                       const float* __restrict__ topk_w, int64_t shared_row0, T* __restrict__ y) {
+  __shared__ int32_t rows[32];
+  __shared__ float gates[32];
+  const int t = blockIdx.x;
+  if (threadIdx.x < K) {
+    rows[threadIdx.x] = row_of_slot[static_cast<int64_t>(t) * K + threadIdx.x];
+    gates[threadIdx.x] = topk_w[static_cast<int64_t>(t) * K + threadIdx.x];
+  }
+  __syncthreads();
+  constexpr int V = Vec16<T>::N;
+  const int nvec = d / V;
+  for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+    float acc[V];
+#pragma unroll
+    for (int j = 0; j < V; ++j) acc[j] = 0.0f;
+    for (int k = 0; k < K; ++k) {
+      if (rows[k] < 0) continue;
+      float f[V];
+      unpack16<T>(ldg16(y_perm + static_cast<int64_t>(rows[k]) * d + v * V), f);
+#pragma unroll
+      for (int j = 0; j < V; ++j) acc[j] = fmaf(gates[k], f[j], acc[j]);
+    }
+    if (shared_row0 >= 0) {
+      float f[V];
+      unpack16<T>(ldg16(y_perm + (shared_row0 + t) * d + v * V), f);
+#pragma unroll
+      for (int j = 0; j < V; ++j) acc[j] += f[j];
+    }
+    stg16(y + static_cast<int64_t>(t) * d + v * V, pack16<T>(acc));
+  }
+}
+
 // 16 E4M3 codes -> 16 bf16 values (every E4M3 value is exact in f16 and in
 // bf16, so both conversions are exact).
 __global__ void dequant_e4m3_kernel(const uint4* __restrict__ q, uint4* __restrict__ out, int64_t n16) {
@@ -90,6 +126,16 @@ __global__ void dequant_e4m3_kernel(const uint4* __restrict__ q, uint4* __restri
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream) {
   if (a.S == 0) return cudaSuccess;
+  if (a.S <= 256) {
+    if (a.act_dtype == MOE_BF16)
+      combine_cta_kernel<__nv_bfloat16><<<a.S, 256, 0, stream>>>(a.d, a.K, static_cast<const __nv_bfloat16*>(a.y_perm),
+                                                                 a.row_of_slot, a.topk_w, a.shared_row0,
+                                                                 static_cast<__nv_bfloat16*>(a.y));
+    else
+      combine_cta_kernel<float><<<a.S, 256, 0, stream>>>(a.d, a.K, static_cast<const float*>(a.y_perm), a.row_of_slot,
+                                                         a.topk_w, a.shared_row0, static_cast<float*>(a.y));
+    return cudaGetLastError();
+  }
   const int blocks = (a.S + kCombWarps - 1) / kCombWarps;
   if (a.act_dtype == MOE_BF16)
     combine_kernel<__nv_bfloat16><<<blocks, kCombWarps * 32, 0, stream>>>(

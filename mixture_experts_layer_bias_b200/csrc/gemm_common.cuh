@@ -34,6 +34,7 @@ struct TcParams {
   float* partial;      // fp32 [max_ksplit][out_rows][pcols] (split-K partial sums)
   int pcols;           // 2N (SwiGLU: gate then up) or N
   int* ksplit_out;     // the split chosen on the device, read by the finalize kernel
+  int test_stall;      // test hook: the producer delivers nothing (the bounded waits must give up)
   StatusBlock* status;
 };
 

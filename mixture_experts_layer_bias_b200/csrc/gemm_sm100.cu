@@ -269,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       uint32_t armed = 0, armed_phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+      for (int u = blockIdx.x; u < total && ok && !p.test_stall; u += gridDim.x) {
         const UnitInfo ui = decode_unit(s, p, u, ks, nk);
         const TileInfo& ti = ui.ti;
         const int a_row = (p.a_rows_from_out ? ti.grp.out_row0 : ti.grp.a_row0) + ti.m_idx * BM;
@@ -415,6 +415,22 @@ cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUte
 
 }  // namespace
 
+// Test hook for the failure-detection tests: MOE_B200_TEST_STALL_GEMM=n makes
+// the next n one-CTA GEMM launches of this process run with a producer that
+// delivers nothing, so their bounded waits give up and report
+// MOE_STATUS_TIMEOUT.  Unset (the default) it costs nothing.
+static int take_test_stall() {
+  static int budget = -1;
+  if (budget < 0) {
+    const char* v = getenv("MOE_B200_TEST_STALL_GEMM");
+    budget = v != nullptr ? atoi(v) : 0;
+    if (budget < 0) budget = 0;
+  }
+  if (budget == 0) return 0;
+  --budget;
+  return 1;
+}
+
 // Kernel choice: the one-CTA kernel unless MOE_B200_GEMM=pair (read once).
 static bool use_pair_kernel() {
   static int choice = -1;
@@ -458,7 +474,9 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t 
     if (p.max_ksplit > 16) p.max_ksplit = 16;
     if (p.max_ksplit < 1) p.max_ksplit = 1;
   }
+  p.test_stall = 0;
   if (use_pair_kernel()) return launch_grouped_gemm_pair(a, p, num_sms, stream);
+  p.test_stall = take_test_stall();
   CUtensorMap mA, mA2, mB0, mB1;
   if (!make_map(&mA, a.a, a.a_rows, a.K)) return cudaErrorInvalidValue;
   if (a.a_shared != nullptr) {

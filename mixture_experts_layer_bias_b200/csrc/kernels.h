@@ -30,6 +30,13 @@ struct RouteArgs {
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream);
 
 // --- grouping by expert -----------------------------------------------------
+// Group table entry of the grouped GEMMs: rows [a_row0, a_row0 + rows) of the
+// A operand, written to rows [out_row0, out_row0 + rows) of the output, all
+// with the weights of slab `expert`.
+struct GroupEntry {
+  int32_t a_row0, out_row0, rows, expert;
+};
+
 struct PermuteArgs {
   int S, d, E, K, capacity, act_dtype;
   const int32_t* topk_idx;   // [S][K]
@@ -42,17 +49,14 @@ struct PermuteArgs {
   void* x_perm;              // [R][d] or nullptr
   int64_t num_rows;          // R
   StatusBlock* status;
+  // optional: also write the GEMM group tables (see GroupEntry)
+  GroupEntry* g1;
+  GroupEntry* g2;
+  int num_shared;
 };
 int permute_num_chunks(int S, int K);
 int permute_tokens_per_chunk(int K);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream);
-
-// Group table entry of the grouped GEMMs: rows [a_row0, a_row0 + rows) of the
-// A operand, written to rows [out_row0, out_row0 + rows) of the output, all
-// with the weights of slab `expert`.
-struct GroupEntry {
-  int32_t a_row0, out_row0, rows, expert;
-};
 
 // Build the pass tables from offsets: pass 1 = routed groups (primary block
 // with capacity) + the shared expert, pass 2 = overflow groups (capacity only).

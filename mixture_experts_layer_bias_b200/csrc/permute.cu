@@ -18,6 +18,8 @@
 //              then a prefix over warps) and writes row_of_slot / token_of_row;
 //  4. gather:  one warp per token copies its row once from HBM to its K rows
 //              with 16-byte vectors.
+// Small batches (S*K <= 4096 slots) run steps 1-3 and the group tables of the
+// GEMMs in one single-CTA kernel, and the gather with one CTA per token.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -215,9 +217,10 @@ __global__ void __launch_bounds__(kPermWarps * 32)
   }
 }
 
-__global__ void build_groups_kernel(int S, int E, int K, int capacity, int num_shared,
-                                    const int32_t* __restrict__ offsets, GroupEntry* __restrict__ g1,
-                                    GroupEntry* __restrict__ g2) {
+// Group tables of the grouped GEMMs from the offsets (pass 1: routed or
+// primary groups + shared expert; pass 2: overflow groups).
+__device__ __forceinline__ void write_groups(int S, int E, int K, int capacity, int num_shared,
+                                             const int32_t* offsets, GroupEntry* g1, GroupEntry* g2) {
   const int64_t R = capacity > 0 ? static_cast<int64_t>(E) * capacity + static_cast<int64_t>(S) * K
                                  : static_cast<int64_t>(S) * K;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -232,6 +235,123 @@ __global__ void build_groups_kernel(int S, int E, int K, int capacity, int num_s
     }
   }
   if (threadIdx.x == 0 && num_shared > 0) g1[E] = GroupEntry{0, static_cast<int32_t>(R), S, E};
+}
+
+constexpr int kSmallWarps = 32;
+constexpr int kSmallSlots = 4096;  // the fused single-CTA path handles S*K up to this
+
+// Small batches (decode): histogram, scans, stable ranks, row maps and the
+// group tables in one CTA -- the same counting sort as the chunked path with
+// the whole slot range as one chunk split over 32 warps.
+__global__ void __launch_bounds__(kSmallWarps * 32)
+    permute_small_kernel(int S, int E, int K, int capacity, int num_shared, const int32_t* __restrict__ topk_idx,
+                         int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                         int32_t* __restrict__ row_of_slot, int32_t* __restrict__ token_of_row, int64_t num_rows,
+                         GroupEntry* __restrict__ g1, GroupEntry* __restrict__ g2, StatusBlock* status) {
+  extern __shared__ int32_t sm[];
+  int32_t* whist = sm;                      // [32][E]
+  int32_t* cnt = sm + kSmallWarps * E;      // [E]
+  int32_t* ovf = cnt + E;                   // [E]
+  int32_t* tmp = ovf + E;                   // [E+1]
+  __shared__ int32_t offs_s[2 * 257];
+  const int warp = threadIdx.x >> 5, lane = lane_id();
+  const int nslots = S * K;
+  const int per_warp = (nslots + kSmallWarps - 1) / kSmallWarps;
+  const int w0 = warp * per_warp, w1 = min(nslots, w0 + per_warp);
+  for (int i = threadIdx.x; i < kSmallWarps * E; i += blockDim.x) whist[i] = 0;
+  if (capacity > 0)
+    for (int64_t r = threadIdx.x; r < num_rows; r += blockDim.x) token_of_row[r] = -1;
+  __syncthreads();
+  int bad = 0;
+  for (int b = w0; b < w1; b += 32) {
+    const int sl = b + lane;
+    const bool act = sl < w1;
+    int e = act ? topk_idx[sl] : -1;
+    if (act && (e < 0 || e >= E)) ++bad;
+    if (e < 0 || e >= E) e = -1;
+    const unsigned peers = __match_any_sync(kFull, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) whist[warp * E + e] += __popc(peers);
+    __syncwarp();
+  }
+  if (bad) report(status, MOE_STATUS_BAD_EXPERT_ID, MOE_CNT_BAD_ID, bad);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int w = 0; w < kSmallWarps; ++w) {
+      const int c = whist[w * E + e];
+      whist[w * E + e] = run;
+      run += c;
+    }
+    cnt[e] = run;
+    counts[e] = run;
+    ovf[e] = capacity > 0 ? max(run - capacity, 0) : 0;
+  }
+  __syncthreads();
+  warp0_exclusive_scan(cnt, tmp, E);
+  __syncthreads();
+  for (int i = threadIdx.x; i <= E; i += blockDim.x) {
+    offsets[i] = tmp[i];
+    offs_s[i] = tmp[i];
+  }
+  if (capacity > 0) {
+    __syncthreads();
+    warp0_exclusive_scan(ovf, tmp, E);
+    __syncthreads();
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) {
+      offsets[E + 1 + i] = tmp[i];
+      offs_s[E + 1 + i] = tmp[i];
+    }
+    if (threadIdx.x == 0 && tmp[E] > 0) report(status, 0u, MOE_CNT_OVERFLOW_ROWS, tmp[E]);
+  }
+  __syncthreads();
+  for (int b = w0; b < w1; b += 32) {
+    const int sl = b + lane;
+    const bool act = sl < w1;
+    int e = act ? topk_idx[sl] : -1;
+    if (e < 0 || e >= E) e = -1;
+    const unsigned peers = __match_any_sync(kFull, e);
+    int row = -1;
+    if (e >= 0) {
+      const int r = whist[warp * E + e] + __popc(peers & ((1u << lane) - 1u));
+      if (capacity <= 0)
+        row = offs_s[e] + r;
+      else
+        row = r < capacity ? e * capacity + r : E * capacity + offs_s[E + 1 + e] + (r - capacity);
+    }
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) whist[warp * E + e] += __popc(peers);
+    if (act) {
+      row_of_slot[sl] = row;
+      if (row >= 0) token_of_row[row] = sl / K;
+    }
+    __syncwarp();
+  }
+  if (g1 != nullptr) write_groups(S, E, K, capacity, num_shared, offs_s, g1, g2);
+}
+
+// Row gather for small batches: one CTA per token, its threads split the row.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    gather_rows_cta_kernel(int d, int K, const int32_t* __restrict__ row_of_slot, const T* __restrict__ x,
+                           T* __restrict__ x_perm) {
+  __shared__ int32_t rows[32];
+  const int t = blockIdx.x;
+  if (threadIdx.x < K) rows[threadIdx.x] = row_of_slot[static_cast<int64_t>(t) * K + threadIdx.x];
+  __syncthreads();
+  constexpr int V = Vec16<T>::N;
+  const int nvec = d / V;
+  const T* src = x + static_cast<int64_t>(t) * d;
+  for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+    const uint4 val = ldg16(src + v * V);
+    for (int k = 0; k < K; ++k)
+      if (rows[k] >= 0) stg16(x_perm + static_cast<int64_t>(rows[k]) * d + v * V, val);
+  }
+}
+
+__global__ void build_groups_kernel(int S, int E, int K, int capacity, int num_shared,
+                                    const int32_t* __restrict__ offsets, GroupEntry* __restrict__ g1,
+                                    GroupEntry* __restrict__ g2) {
+  write_groups(S, E, K, capacity, num_shared, offsets, g1, g2);
 }
 
 }  // namespace
@@ -252,26 +372,50 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
       err = cudaMemsetAsync(a.token_of_row, 0xFF, sizeof(int32_t) * a.num_rows, stream);
     return err;
   }
-  const int tpc = permute_tokens_per_chunk(a.K);
-  const int nch = permute_num_chunks(a.S, a.K);
   cudaError_t err;
-  if (a.capacity > 0) {
-    // unused primary rows keep token -1
-    err = cudaMemsetAsync(a.token_of_row, 0xFF, sizeof(int32_t) * a.num_rows, stream);
-    if (err != cudaSuccess) return err;
+  if (static_cast<int64_t>(a.S) * a.K <= kSmallSlots) {
+    const size_t smem = sizeof(int32_t) * (kSmallWarps * a.E + 3 * a.E + 1);
+    permute_small_kernel<<<1, kSmallWarps * 32, smem, stream>>>(a.S, a.E, a.K, a.capacity, a.num_shared, a.topk_idx,
+                                                                 a.counts, a.offsets, a.row_of_slot, a.token_of_row,
+                                                                 a.num_rows, a.g1, a.g2, a.status);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  } else {
+    const int tpc = permute_tokens_per_chunk(a.K);
+    const int nch = permute_num_chunks(a.S, a.K);
+    if (a.capacity > 0) {
+      // unused primary rows keep token -1
+      err = cudaMemsetAsync(a.token_of_row, 0xFF, sizeof(int32_t) * a.num_rows, stream);
+      if (err != cudaSuccess) return err;
+    }
+    count_kernel<<<nch, 256, sizeof(int32_t) * a.E, stream>>>(a.S, a.E, a.K, tpc, a.topk_idx, a.chunk_hist,
+                                                                a.status);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    const int scan_threads = 1024;
+    const size_t scan_smem = sizeof(int32_t) * ((scan_threads / a.E) * a.E + 3 * a.E + 1);
+    scan_kernel<<<1, scan_threads, scan_smem, stream>>>(a.E, nch, a.capacity, a.chunk_hist, a.counts, a.offsets,
+                                                         a.status);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    const size_t smem = sizeof(int32_t) * kPermWarps * a.E;
+    scatter_kernel<<<nch, kPermWarps * 32, smem, stream>>>(a.S, a.d, a.E, a.K, a.capacity, tpc, a.topk_idx,
+                                                            a.chunk_hist, a.offsets, a.row_of_slot, a.token_of_row);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (a.g1 != nullptr) {
+      build_groups_kernel<<<1, 256, 0, stream>>>(a.S, a.E, a.K, a.capacity, a.num_shared, a.offsets, a.g1, a.g2);
+      if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
   }
-  count_kernel<<<nch, 256, sizeof(int32_t) * a.E, stream>>>(a.S, a.E, a.K, tpc, a.topk_idx, a.chunk_hist, a.status);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  const int scan_threads = 1024;
-  const size_t scan_smem = sizeof(int32_t) * ((scan_threads / a.E) * a.E + 3 * a.E + 1);
-  scan_kernel<<<1, scan_threads, scan_smem, stream>>>(a.E, nch, a.capacity, a.chunk_hist, a.counts,
-                                                                     a.offsets, a.status);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  const size_t smem = sizeof(int32_t) * kPermWarps * a.E;
-  scatter_kernel<<<nch, kPermWarps * 32, smem, stream>>>(a.S, a.d, a.E, a.K, a.capacity, tpc, a.topk_idx,
-                                                          a.chunk_hist, a.offsets, a.row_of_slot, a.token_of_row);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
   if (a.x == nullptr || a.x_perm == nullptr) return cudaSuccess;
+  if (a.S <= 256) {
+#define MOE_GATHER_CTA(T)                                                                                    \
+  gather_rows_cta_kernel<T><<<a.S, 256, 0, stream>>>(a.d, a.K, a.row_of_slot, static_cast<const T*>(a.x),   \
+                                                      static_cast<T*>(a.x_perm))
+    if (a.act_dtype == MOE_BF16)
+      MOE_GATHER_CTA(__nv_bfloat16);
+    else
+      MOE_GATHER_CTA(float);
+#undef MOE_GATHER_CTA
+    return cudaGetLastError();
+  }
   const int gblocks = (a.S + kPermWarps - 1) / kPermWarps;
   if (a.act_dtype == MOE_BF16)
     gather_rows_kernel<__nv_bfloat16><<<gblocks, kPermWarps * 32, 0, stream>>>(

@@ -218,9 +218,10 @@ def test_permute_bad_ids_flagged():
 # ----------------------------------------------------------------------------
 
 
-@pytest.mark.parametrize("dt,shared,K", [(0, 0, 2), (1, 0, 2), (1, 1, 8), (0, 1, 3)])
-def test_combine(dt, shared, K):
-    S, E, d = 333, 16, 264
+@pytest.mark.parametrize("dt,shared,K,S", [(0, 0, 2, 333), (1, 0, 2, 333), (1, 1, 8, 333), (0, 1, 3, 333),
+                                           (1, 1, 8, 5), (0, 0, 2, 1), (1, 0, 2, 256)])
+def test_combine(dt, shared, K, S):
+    E, d = 16, 264
     rng = np.random.default_rng(K + dt)
     ridx, rw = O.select_experts(rng.normal(size=(S, E)).astype(np.float32), K)
     P = O.expert_permutation(ridx, E)
