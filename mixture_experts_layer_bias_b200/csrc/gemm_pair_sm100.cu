@@ -57,7 +57,11 @@ struct PairCtl {
   int tile_start[kMaxGroups + 1];
 };
 
-constexpr size_t kPairSmem = P_STAGES * P_STAGE + sizeof(PairCtl) + 1024;
+// per epilogue warp: one 16-token x 32-feature bf16 tile, transposed through
+// shared memory so that global stores are 16-byte pieces of output rows
+constexpr int P_TBUF = 16 * 32 * 2;
+constexpr size_t kPairCtlBytes = (sizeof(PairCtl) + 127) & ~size_t(127);  // keeps the buffers 128-byte aligned
+constexpr size_t kPairSmem = P_STAGES * P_STAGE + kPairCtlBytes + 4 * P_TBUF + 1024;
 
 template <int EPI>
 struct PairShape {
@@ -103,7 +107,8 @@ constexpr int P_CHUNK = 16;  // tokens per epilogue chunk (one 32x32b.x16 TMEM l
 // TMEM lane (weight row) for token tb*256 + chunk*16 + j.
 template <int EPI>
 __device__ __forceinline__ void pair_store_chunk(const TcParams& p, const PairUnit& pu, uint32_t rank, int q, int lane,
-                                                 int chunk, const uint32_t (&r)[P_CHUNK], int ks) {
+                                                 int chunk, const uint32_t (&r)[P_CHUNK], int ks,
+                                                 __nv_bfloat16* tbuf) {
   const int N = p.N;
   const int t0 = pu.tb * P_TOK + chunk * P_CHUNK;  // first token of the chunk inside the group
   const int64_t row0 = static_cast<int64_t>(pu.grp.out_row0) + t0;
@@ -112,7 +117,8 @@ __device__ __forceinline__ void pair_store_chunk(const TcParams& p, const PairUn
   if (EPI == EPI_SWIGLU) {
     const int blk = q * 2 + (lane >> 4);  // 16-row block of this CTA's weight rows
     const bool is_up = blk & 1;
-    const int f = pu.fb * PairShape<EPI>::FEAT + static_cast<int>(rank) * 64 + (blk >> 1) * 16 + (lane & 15);
+    const int fbase = pu.fb * PairShape<EPI>::FEAT + static_cast<int>(rank) * 64 + (blk >> 1) * 16;
+    const int f = fbase + (lane & 15);
     const bool fvalid = f < N;
     if (ks > 1) {
       if (!fvalid) return;
@@ -127,38 +133,64 @@ __device__ __forceinline__ void pair_store_chunk(const TcParams& p, const PairUn
       sg = __ldg(p.scale0 + sbase + f);
       su = __ldg(p.scale1 + sbase + f);
     }
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row0 * N + f;
+    // lanes 0-15: h for 16 features x 16 tokens -> tbuf[token][feature] (16 x 16 bf16)
 #pragma unroll
     for (int j = 0; j < P_CHUNK; ++j) {
       const float mine = __uint_as_float(r[j]);
       const float up = __shfl_xor_sync(0xFFFFFFFFu, mine, 16);
-      if (!is_up && fvalid && j < tlim) {
+      if (!is_up) {
         const float g = mine * sg;
-        out[static_cast<int64_t>(j) * N] = __float2bfloat16_rn(g / (1.0f + __expf(-g)) * (up * su));
+        tbuf[j * 16 + lane] = __float2bfloat16_rn(g / (1.0f + __expf(-g)) * (up * su));
       }
     }
+    __syncwarp();
+    // 16 tokens x 32 bytes = 32 pieces of 16 bytes, one per lane
+    const int tok = lane >> 1, sub = lane & 1;
+    const int fo = fbase + sub * 8;
+    if (tok < tlim && fo + 8 <= N)
+      stg16(static_cast<__nv_bfloat16*>(p.out) + (row0 + tok) * N + fo,
+            *reinterpret_cast<const uint4*>(tbuf + tok * 16 + sub * 8));
+    __syncwarp();
   } else {
-    const int f = pu.fb * PairShape<EPI>::FEAT + static_cast<int>(rank) * 128 + q * 32 + lane;
-    if (f >= N) return;
+    const int fbase = pu.fb * PairShape<EPI>::FEAT + static_cast<int>(rank) * 128 + q * 32;
+    const int f = fbase + lane;
     if (ks > 1) {
+      if (f >= N) return;
       float* base = p.partial + (static_cast<int64_t>(pu.split) * p.out_rows + row0) * p.pcols + f;
 #pragma unroll
       for (int j = 0; j < P_CHUNK; ++j)
         if (j < tlim) base[static_cast<int64_t>(j) * p.pcols] = __uint_as_float(r[j]);
       return;
     }
-    const float sc = p.scale0 != nullptr ? __ldg(p.scale0 + sbase + f) : 1.0f;
-    const float bi = (EPI == EPI_GELU_BIAS || EPI == EPI_BIAS) ? __ldg(p.bias + sbase + f) : 0.0f;
+    const bool fvalid = f < N;
+    const float sc = (p.scale0 != nullptr && fvalid) ? __ldg(p.scale0 + sbase + f) : 1.0f;
+    const float bi = ((EPI == EPI_GELU_BIAS || EPI == EPI_BIAS) && fvalid) ? __ldg(p.bias + sbase + f) : 0.0f;
+    if (p.out_f32) {
+      // fp32 output (router logits): 32 lanes write 128 contiguous bytes per token
+      if (!fvalid) return;
+#pragma unroll
+      for (int j = 0; j < P_CHUNK; ++j)
+        if (j < tlim) static_cast<float*>(p.out)[(row0 + j) * N + f] = __uint_as_float(r[j]) * sc + bi;
+      return;
+    }
 #pragma unroll
     for (int j = 0; j < P_CHUNK; ++j) {
-      if (j >= tlim) break;
       float z = __uint_as_float(r[j]) * sc + bi;
       if (EPI == EPI_GELU_BIAS) z = 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
-      if (p.out_f32)
-        static_cast<float*>(p.out)[(row0 + j) * N + f] = z;
-      else
-        static_cast<__nv_bfloat16*>(p.out)[(row0 + j) * N + f] = __float2bfloat16_rn(z);
+      tbuf[j * 32 + lane] = __float2bfloat16_rn(z);
     }
+    __syncwarp();
+    // 16 tokens x 64 bytes = 64 pieces of 16 bytes, two per lane
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int piece = lane + 32 * h;
+      const int tok = piece >> 2, sub = piece & 3;
+      const int fo = fbase + sub * 8;
+      if (tok < tlim && fo + 8 <= N)
+        stg16(static_cast<__nv_bfloat16*>(p.out) + (row0 + tok) * N + fo,
+              *reinterpret_cast<const uint4*>(tbuf + tok * 32 + sub * 8));
+    }
+    __syncwarp();
   }
 }
 
@@ -170,6 +202,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   PairCtl& s = *reinterpret_cast<PairCtl*>(ring + P_STAGES * P_STAGE);
+  __nv_bfloat16* tbufs = reinterpret_cast<__nv_bfloat16*>(ring + P_STAGES * P_STAGE + kPairCtlBytes);
   const int warp = threadIdx.x >> 5, lane = lane_id();
   const uint32_t rank = cluster_ctarank();
   const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
@@ -362,7 +395,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
         uint32_t r[P_CHUNK];
         tmem_ld_32x32b_x16(tbase + c * P_CHUNK, r);
         tmem_ld_wait();
-        pair_store_chunk<EPI>(p, pu, rank, q, lane, c, r, ks);
+        pair_store_chunk<EPI>(p, pu, rank, q, lane, c, r, ks, tbufs + (warp - 2) * (P_TBUF / 2));
       }
       tc_fence_before();
       __syncwarp();
