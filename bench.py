@@ -372,32 +372,61 @@ def main():
                 "kernel": "grouped expert FFN (up SwiGLU + down GEMMs, tcgen05)",
                 "peak_source": f"{peaks['source']} bf16 burst"}
 
-    # end to end through the public call with host buffers
-    x_host = inp["x"].cpu().pin_memory()
-    y_host = torch.empty((S, cfg.d), dtype=x_host.dtype).pin_memory()
-    x_dev = torch.empty_like(inp["x"])
+    # end to end through the public call with host buffers: every step copies its
+    # input from pinned host memory and its output back.  As in a serving loop,
+    # step i+1's upload and step i-1's download overlap step i's layer (two copy
+    # streams, double-buffered device buffers); the layer calls stay serialised
+    # on one stream because they share the workspace.
+    x_host = [inp["x"].cpu().pin_memory() for _ in range(2)]
+    y_host = [torch.empty((S, cfg.d), dtype=x_host[0].dtype).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(inp["x"]) for _ in range(2)]
+    y_dev = [torch.empty((S, cfg.d), dtype=inp["x"].dtype, device=device) for _ in range(2)]
     layer_w = ops.make_weights(inp)
-    e2e_ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    comp = torch.cuda.current_stream()
+    up_s, down_s = torch.cuda.Stream(), torch.cuda.Stream()
+    uploaded = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    downloaded = [torch.cuda.Event() for _ in range(2)]
+    for b in range(2):
+        computed[b].record(comp)
+        downloaded[b].record(comp)
 
-    def e2e_step():
-        x_dev.copy_(x_host, non_blocking=True)
-        ops.moe_layer_forward(desc, layer_w, x_dev, bufs["y"], None, None, None, ws)
-        y_host.copy_(bufs["y"], non_blocking=True)
+    def e2e_step(i):
+        b = i % 2
+        with torch.cuda.stream(up_s):
+            up_s.wait_event(computed[b])       # x_dev[b] no longer read by the layer two steps back
+            x_dev[b].copy_(x_host[b], non_blocking=True)
+            uploaded[b].record(up_s)
+        comp.wait_event(uploaded[b])
+        comp.wait_event(downloaded[b])          # y_dev[b] already copied out
+        ops.moe_layer_forward(desc, layer_w, x_dev[b], y_dev[b], None, None, None, ws, comp)
+        computed[b].record(comp)
+        with torch.cuda.stream(down_s):
+            down_s.wait_event(computed[b])
+            y_host[b].copy_(y_dev[b], non_blocking=True)
+            downloaded[b].record(down_s)
 
-    for _ in range(args.warmup):
-        e2e_step()
+    for i in range(args.warmup):
+        e2e_step(i)
     torch.cuda.synchronize()
     if dist:
         td.barrier()
-    e2e_ev[0].record()
-    for _ in range(args.steps):
-        e2e_step()
-    e2e_ev[1].record()
+    e2e_t0 = time.perf_counter()
+    e2e_start = torch.cuda.Event(enable_timing=True)
+    e2e_stop = torch.cuda.Event(enable_timing=True)
+    e2e_start.record(comp)
+    for i in range(args.steps):
+        e2e_step(i)
+    for b in range(2):
+        comp.wait_event(downloaded[b])
+    e2e_stop.record(comp)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e2e_ev[0].elapsed_time(e2e_ev[1]), device)
+    e2e_ms = max_over_ranks(e2e_start.elapsed_time(e2e_stop), device)
     e2e = {"value": round(whole_job_rate(S * args.steps, e2e_ms, world), 1), "unit": "tokens/s",
-           "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
-           "d2h_bytes_per_step": y_host.numel() * y_host.element_size()}
+           "h2d_bytes_per_step": x_host[0].numel() * x_host[0].element_size(),
+           "d2h_bytes_per_step": y_host[0].numel() * y_host[0].element_size(),
+           "copies": "overlapped with the neighbouring steps' layers (2 copy streams)",
+           "wall_ms": round((time.perf_counter() - e2e_t0) * 1e3, 3)}
 
     dec = None
     if not args.no_decode and args.workload == WORKLOAD:
