@@ -46,6 +46,29 @@ WORKLOAD = "mixtral_prefill"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM bytes of the grouped FFN stage (up + down GEMM launches) of one prefill
+# layer call, from the ncu capture summarised in profiles/dram_traffic_per_kernel.md.
+# Valid only for the GEMM sources it was taken on: `traffic` is reported as null
+# once their hash differs.
+FFN_TRAFFIC_CAPTURE = {
+    "workload": "mixtral_prefill",
+    "bytes": (1973.3 + 223.5 + 1430.2 + 60.4) * 1e6,
+    "sources": ("common.cuh", "gemm_common.cuh", "gemm_sm100.cu", "kernels.h"),
+    "sha1": "31014cc6ff2ab8842ea85babd0a06440b74e5ff3",
+}
+
+
+def ffn_traffic(workload: str):
+    import hashlib
+    if workload != FFN_TRAFFIC_CAPTURE["workload"] or os.environ.get("MOE_B200_GEMM") == "pair":
+        return None
+    h = hashlib.sha1()
+    for f in FFN_TRAFFIC_CAPTURE["sources"]:
+        with open(os.path.join(ROOT, "mixture_experts_layer_bias_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return FFN_TRAFFIC_CAPTURE["bytes"] if h.hexdigest() == FFN_TRAFFIC_CAPTURE["sha1"] else None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -362,13 +385,20 @@ def main():
     # roofline of the dominant stage: the grouped expert FFN (both GEMMs)
     rows = S * cfg.K + cfg.num_shared * S
     flops = expert_flops(cfg, rows)
+    wbytes = {syn.F32: 4, syn.BF16: 2, syn.E4M3: 1}[cfg.weight_dtype]
+    abytes = 4 if cfg.act_dtype == syn.F32 else 2
+    n_up = 2 if cfg.activation == syn.SWIGLU else 1
+    # weights of every expert + permuted rows in + hidden out/in + expert rows out
+    algo_bytes = ((cfg.E + cfg.num_shared) * (n_up + 1) * cfg.d * cfg.h * wbytes
+                  + rows * (cfg.d + 2 * cfg.h + cfg.d) * abytes)
     ffn_ms = stages["grouped_ffn"]
     achieved = flops / (ffn_ms * 1e-3) / 1e12
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "frac_of_sustained_peak": round(achieved / sustained, 4),
-                "traffic": None,
+                "traffic": ffn_traffic(args.workload),
+                "algorithmic_bytes": algo_bytes,
                 "kernel": "grouped expert FFN (up SwiGLU + down GEMMs, tcgen05)",
                 "peak_source": f"{peaks['source']} bf16 burst"}
 
