@@ -228,6 +228,30 @@ moe_status moe_layer_forward(const moe_desc *desc, const moe_weights *w, const v
                              int32_t *topk_idx, float *topk_w, int32_t *counts, void *ws, size_t ws_bytes,
                              void *stream);
 
+/*
+ * Sliding-window expert load and the aux-loss-free selection-bias update
+ * (ybb.press "MoE 推理工程深层实战" 2.3: the bias added to the selection keys
+ * is recomputed from a sliding-window token count, `TokenWindowCounter(
+ * window_size=1000)`, so routing is steered without gradients).  The page
+ * prints no update rule; this call applies, per expert, in float32,
+ *     sel_bias[e] += gamma * sign(mean - count_e),
+ * count_e = (token, k) slots routed to e among the last `window_tokens`
+ * tokens, mean = tokens_in_window * K / E.
+ *   state: caller-owned device memory of moe_bias_state_size() bytes, zeroed
+ *     by moe_bias_state_init before the first update (it holds the window's
+ *     expert ids and counts).  The window fills from empty; a batch of S
+ *     tokens replaces the S oldest ones (only its last window_tokens tokens
+ *     count when S >= window_tokens).  Ids outside [0, E) are not counted.
+ *   topk_idx int32 [S][K] (e.g. moe_route's output); sel_bias fp32 [E] is
+ *   updated in place; window_counts int32 [E] (optional) receives count_e.
+ *   One window per state; calls on one state must be stream-ordered.
+ */
+moe_status moe_bias_state_size(const moe_desc *desc, int32_t window_tokens, size_t *bytes);
+moe_status moe_bias_state_init(void *state, size_t state_bytes, void *stream);
+moe_status moe_update_sel_bias(const moe_desc *desc, const int32_t *topk_idx, int32_t window_tokens, float gamma,
+                               void *state, size_t state_bytes, float *sel_bias, int32_t *window_counts,
+                               void *stream);
+
 /* Synchronise `stream`, copy the status block to the host.  flags: OR of
  * MOE_STATUS_* bits; counters: MOE_NUM_COUNTERS int32 (may be NULL).
  * Returns MOE_ERR_DEVICE_STATUS when any error bit is set. */

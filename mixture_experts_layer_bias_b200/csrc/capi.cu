@@ -441,6 +441,36 @@ moe_status moe_layer_forward(const moe_desc* desc, const moe_weights* w, const v
   return combine_impl(d, y_perm, ros, gates, y, st);
 }
 
+moe_status moe_bias_state_size(const moe_desc* desc, int32_t window_tokens, size_t* bytes) {
+  const moe_status s = validate(desc);
+  if (s != MOE_OK) return s;
+  if (bytes == nullptr || window_tokens < 1) return MOE_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(window_tokens) * desc->top_k > (int64_t(1) << 31) - 1) return MOE_ERR_INVALID_ARG;
+  *bytes = bias_state_bytes(desc->num_experts, desc->top_k, window_tokens);
+  return MOE_OK;
+}
+
+moe_status moe_bias_state_init(void* state, size_t state_bytes, void* stream) {
+  if (state == nullptr || state_bytes < kAlign || (reinterpret_cast<uintptr_t>(state) & (kAlign - 1)) != 0)
+    return MOE_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(state, 0, state_bytes, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_update_sel_bias(const moe_desc* desc, const int32_t* topk_idx, int32_t window_tokens, float gamma,
+                               void* state, size_t state_bytes, float* sel_bias, int32_t* window_counts,
+                               void* stream) {
+  size_t need = 0;
+  moe_status s = moe_bias_state_size(desc, window_tokens, &need);
+  if (s != MOE_OK) return s;
+  if (state == nullptr || state_bytes < need || (reinterpret_cast<uintptr_t>(state) & (kAlign - 1)) != 0)
+    return MOE_ERR_WORKSPACE;
+  if (sel_bias == nullptr || (desc->num_tokens > 0 && topk_idx == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (!(gamma >= 0.0f) || gamma > 3.0e38f) return MOE_ERR_INVALID_ARG;  // also rejects NaN
+  if (desc->num_tokens == 0) return MOE_OK;
+  return cuda_status(launch_bias_update(desc->num_tokens, desc->num_experts, desc->top_k, window_tokens, topk_idx,
+                                        gamma, state, sel_bias, window_counts, static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_get_status(const void* ws, void* stream, uint32_t* flags, int32_t* counters) {
   if (ws == nullptr) return MOE_ERR_WORKSPACE;
   StatusBlock host;

@@ -105,6 +105,11 @@ cudaError_t launch_grouped_gemm_f32(const GemmArgs& a, cudaStream_t stream);
 // FP8-E4M3 weight slabs -> bf16 (exact)
 cudaError_t launch_dequant_e4m3(const uint8_t* q, void* out_bf16, int64_t n, cudaStream_t stream);
 
+// --- sliding-window load and selection-bias update ---------------------------
+size_t bias_state_bytes(int E, int K, int window);
+cudaError_t launch_bias_update(int S, int E, int K, int window, const int32_t* topk_idx, float gamma, void* state,
+                               float* sel_bias, int32_t* window_counts, cudaStream_t stream);
+
 // --- combine -----------------------------------------------------------------
 struct CombineArgs {
   int S, d, K, act_dtype;

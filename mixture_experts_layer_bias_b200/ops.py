@@ -31,8 +31,8 @@ WEIGHT_FIELDS = ("w_router", "router_bias", "sel_bias", "w1", "b1", "w2", "b2", 
                  "s_gate", "s_up", "s_down")
 
 EXPORTED = ("moe_routed_rows", "moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute",
-            "moe_permute_static", "moe_grouped_ffn", "moe_combine", "moe_layer_forward", "moe_get_status",
-            "moe_strerror")
+            "moe_permute_static", "moe_grouped_ffn", "moe_combine", "moe_layer_forward", "moe_bias_state_size",
+            "moe_bias_state_init", "moe_update_sel_bias", "moe_get_status", "moe_strerror")
 
 
 class MoeDesc(ctypes.Structure):
@@ -69,6 +69,9 @@ def lib():
         "moe_grouped_ffn": (I, [pd, pw, P, P, P, P, P, SZ, P]),
         "moe_combine": (I, [pd, P, P, P, P, P, SZ, P]),
         "moe_layer_forward": (I, [pd, pw, P, P, P, P, P, P, SZ, P]),
+        "moe_bias_state_size": (I, [pd, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]),
+        "moe_bias_state_init": (I, [P, SZ, P]),
+        "moe_update_sel_bias": (I, [pd, P, ctypes.c_int32, ctypes.c_float, P, SZ, P, P, P]),
         "moe_get_status": (I, [P, P, ctypes.POINTER(ctypes.c_uint32), ctypes.POINTER(ctypes.c_int32)]),
         "moe_strerror": (ctypes.c_char_p, [I]),
     }
@@ -185,6 +188,23 @@ def moe_layer_forward(desc, weights, x, y, topk_idx, topk_w, counts, ws, stream=
     p, n = _ws(ws)
     _check(lib().moe_layer_forward(ctypes.byref(desc), ctypes.byref(weights), _ptr(x), _ptr(y), _ptr(topk_idx),
                                    _ptr(topk_w), _ptr(counts), p, n, _stream(stream)), "moe_layer_forward")
+
+
+def moe_bias_state_size(desc, window_tokens: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().moe_bias_state_size(ctypes.byref(desc), int(window_tokens), ctypes.byref(n)), "moe_bias_state_size")
+    return int(n.value)
+
+
+def moe_bias_state_init(state, stream=None):
+    p, n = _ws(state)
+    _check(lib().moe_bias_state_init(p, n, _stream(stream)), "moe_bias_state_init")
+
+
+def moe_update_sel_bias(desc, topk_idx, window_tokens, gamma, state, sel_bias, window_counts=None, stream=None):
+    p, n = _ws(state)
+    _check(lib().moe_update_sel_bias(ctypes.byref(desc), _ptr(topk_idx), int(window_tokens), float(gamma), p, n,
+                                     _ptr(sel_bias), _ptr(window_counts), _stream(stream)), "moe_update_sel_bias")
 
 
 def moe_get_status(ws, stream=None):

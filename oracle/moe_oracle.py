@@ -564,3 +564,60 @@ def soft_routing(x, logits, expert_fn, num_experts, tau=1.0):
     for e in range(num_experts):
         y = y + p[:, e:e + 1] * expert_fn(e, np.asarray(x, np.float64))
     return y
+
+
+# ----------------------------------------------------------------------------
+# aux-loss-free bias update (NEXT row: the selection bias follows the load)
+# ----------------------------------------------------------------------------
+
+
+class WindowBias:
+    """Sliding-window expert counts and the selection-bias update of
+    ybb.press 2.3 (aux-loss-free routing: the bias added to the selection
+    keys is recomputed from a sliding window of recent tokens' expert
+    choices, `TokenWindowCounter(window_size=1000)`).
+
+    The page does not print the update rule.  Reading taken: after each
+    batch, b_e <- b_e + gamma * sign(mean - count_e) in float32, where count_e
+    is expert e's number of (token, k) slots among the last `window` tokens and
+    mean = tokens_in_window * K / E; under-loaded experts move up, over-loaded
+    ones down.
+
+    The window is a ring of `window` token positions filled from position 0;
+    a batch of S tokens occupies the next S positions (only its last `window`
+    tokens when S >= window).
+    """
+
+    def __init__(self, num_experts: int, top_k: int, window: int):
+        self.E, self.K, self.W = num_experts, top_k, window
+        self.ring = np.full((window, top_k), -1, dtype=np.int64)
+        self.filled = 0
+        self.head = 0
+
+    def counts(self) -> np.ndarray:
+        ids = self.ring[self.ring >= 0]
+        return np.bincount(ids, minlength=self.E).astype(np.int32)
+
+    def update(self, topk_idx: np.ndarray, sel_bias: np.ndarray, gamma: float):
+        idx = np.asarray(topk_idx, dtype=np.int64)
+        idx = np.where((idx >= 0) & (idx < self.E), idx, -1)  # ids outside [0, E) are not counted
+        S = idx.shape[0]
+        if S >= self.W:
+            self.ring[:] = idx[S - self.W:]
+            self.filled, self.head = self.W, 0
+        else:
+            for i in range(S):
+                self.ring[(self.head + i) % self.W] = idx[i]
+            self.filled = min(self.W, self.filled + S)
+            self.head = (self.head + S) % self.W
+        c = self.counts()
+        mean = np.float32(self.filled * self.K) / np.float32(self.E)
+        b = np.asarray(sel_bias, dtype=np.float32).copy()
+        g = np.float32(gamma)
+        for e in range(self.E):
+            diff = np.float32(mean - np.float32(c[e]))
+            if diff > 0:
+                b[e] = np.float32(b[e] + g)
+            elif diff < 0:
+                b[e] = np.float32(b[e] - g)
+        return b, c

@@ -138,3 +138,25 @@ def test_empty_batch_is_a_no_op():
     assert L.moe_layer_forward(ctypes.byref(d), ctypes.byref(w), None, None, None, None, None, ws, n,
                                None) == ops.MOE_OK
     assert ops.moe_routed_rows(d) == 0
+
+
+def test_bias_state_size_and_argument_errors():
+    L = ops.lib()
+    d = _desc("dsv3_grouped")
+    n = ops.moe_bias_state_size(d, 1000)
+    assert n >= 256 + 256 * 4 + 1000 * 8 * 4 and n % 256 == 0
+    size = ctypes.c_size_t(0)
+    assert L.moe_bias_state_size(ctypes.byref(d), 0, ctypes.byref(size)) == ops.MOE_ERR_INVALID_ARG
+    p = ctypes.c_void_p(0x1000)
+    st = ctypes.c_void_p(0x200000)
+    # state missing / too small / misaligned
+    assert L.moe_update_sel_bias(ctypes.byref(d), p, 1000, 0.1, None, n, p, None, None) == ops.MOE_ERR_WORKSPACE
+    assert L.moe_update_sel_bias(ctypes.byref(d), p, 1000, 0.1, st, n - 256, p, None, None) == ops.MOE_ERR_WORKSPACE
+    assert L.moe_update_sel_bias(ctypes.byref(d), p, 1000, 0.1, ctypes.c_void_p(0x200010), n, p, None,
+                                 None) == ops.MOE_ERR_WORKSPACE
+    # bias missing, negative or NaN step
+    assert L.moe_update_sel_bias(ctypes.byref(d), p, 1000, 0.1, st, n, None, None, None) == ops.MOE_ERR_INVALID_ARG
+    assert L.moe_update_sel_bias(ctypes.byref(d), p, 1000, -0.1, st, n, p, None, None) == ops.MOE_ERR_INVALID_ARG
+    assert L.moe_update_sel_bias(ctypes.byref(d), p, 1000, float("nan"), st, n, p, None,
+                                 None) == ops.MOE_ERR_INVALID_ARG
+    assert L.moe_bias_state_init(None, 0, None) == ops.MOE_ERR_WORKSPACE

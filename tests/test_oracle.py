@@ -397,3 +397,55 @@ def test_router_logits_definition():
         for e in range(4):
             exact = math.fsum(float(x[t, k]) * float(w[e, k]) for k in range(5)) + float(b[e])
             assert abs(float(l[t, e]) - exact) <= np.spacing(np.float32(abs(exact)))
+
+
+# ----------------------------------------------------------------------------
+# sliding-window bias update (aux-loss-free routing, ybb.press 2.3)
+# ----------------------------------------------------------------------------
+
+
+def test_window_bias_hand_computed():
+    """E=4, K=1, window 4, gamma 0.5: tokens [0,0,0,1] -> counts [3,1,0,0],
+    mean 1 -> bias [-0.5, 0, +0.5, +0.5]; then [2,2] replaces the two oldest
+    -> window [2,2,0,1], counts [1,1,2,0] -> bias [-0.5, 0, 0, 1.0]."""
+    wb = O.WindowBias(4, 1, 4)
+    b = np.zeros(4, np.float32)
+    b, c = wb.update(np.array([[0], [0], [0], [1]]), b, 0.5)
+    assert c.tolist() == [3, 1, 0, 0] and b.tolist() == [-0.5, 0.0, 0.5, 0.5]
+    b, c = wb.update(np.array([[2], [2]]), b, 0.5)
+    assert c.tolist() == [1, 1, 2, 0] and b.tolist() == [-0.5, 0.0, 0.0, 1.0]
+    # a batch longer than the window keeps only its last `window` tokens
+    b, c = wb.update(np.array([[3]] * 3 + [[1]] * 4), b, 0.5)
+    assert c.tolist() == [0, 4, 0, 0]
+
+
+def test_window_counts_sum_and_partial_fill():
+    wb = O.WindowBias(8, 2, 10)
+    rng = np.random.default_rng(0)
+    b = np.zeros(8, np.float32)
+    seen = []
+    for S in (3, 4, 5, 1, 12, 2):
+        ridx, _ = O.select_experts(rng.normal(size=(S, 8)).astype(np.float32), 2)
+        seen.extend(ridx.tolist())
+        b, c = wb.update(ridx, b, 0.01)
+        last = np.array(seen[-10:])
+        assert c.sum() == min(len(seen), 10) * 2
+        assert c.tolist() == np.bincount(last.reshape(-1), minlength=8).tolist()
+
+
+def test_bias_update_steers_load_toward_balance():
+    """The point of the bias (ybb.press 2.3: steer the routing distribution
+    without gradients): repeated routing + update under a skewed router must
+    lower the max/mean load.  With the sign flipped the skew would grow."""
+    rng = np.random.default_rng(1)
+    E, K, S = 16, 2, 512
+    offs = (rng.normal(size=E) * 1.5).astype(np.float32)
+    wb = O.WindowBias(E, K, 1000)
+    b = np.zeros(E, np.float32)
+    ratios = []
+    for it in range(60):
+        logits = (rng.normal(size=(S, E)).astype(np.float32) + offs).astype(np.float32)
+        idx, _ = O.select_experts(logits, K, "softmax", True, b)
+        ratios.append(O.load_stats(O.expert_counts(idx, E), K, S)["max_over_mean"])
+        b, _ = wb.update(idx, b, 0.05)
+    assert ratios[0] > 2.0 and np.mean(ratios[-10:]) < 0.6 * ratios[0]
