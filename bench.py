@@ -269,6 +269,24 @@ def decode_sweep(base_inp, device, peaks, reps=20):
     return out
 
 
+def time_bias_update(cfg, device, S, window=1000, reps=50):
+    """Mean time of one sliding-window selection-bias update (us)."""
+    desc = ops.make_desc(**syn.desc_dict(cfg, S))
+    state = torch.empty(ops.moe_bias_state_size(desc, window), dtype=torch.uint8, device=device)
+    ops.moe_bias_state_init(state)
+    bias = torch.zeros(cfg.E, dtype=torch.float32, device=device)
+    idx = torch.randint(0, cfg.E, (S, cfg.K), dtype=torch.int32, device=device)
+    for _ in range(3):
+        ops.moe_update_sel_bias(desc, idx, window, 0.001, state, bias)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        ops.moe_update_sel_bias(desc, idx, window, 0.001, state, bias)
+    e1.record()
+    torch.cuda.synchronize()
+    return round(e0.elapsed_time(e1) * 1e3 / reps, 2)
+
+
 def cpu_baseline(cfg, inp, n_tokens=32):
     """The CPU oracle as it stands on a fixed sample of tokens."""
     sys.path.insert(0, os.path.join(ROOT, "tests"))
@@ -458,6 +476,7 @@ def main():
            "copies": "overlapped with the neighbouring steps' layers (2 copy streams)",
            "wall_ms": round((time.perf_counter() - e2e_t0) * 1e3, 3)}
 
+    bias_us = time_bias_update(cfg, device, S)
     dec = None
     if not args.no_decode and args.workload == WORKLOAD:
         dec = decode_sweep(inp, device, peaks)
@@ -478,6 +497,7 @@ def main():
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": kernels_per_step(cfg) * args.steps, "clocks": clk,
             "stages_ms": {k: round(v, 4) for k, v in stages.items()}, "decode_sweep": dec,
+            "bias_update_us": bias_us,
             "counters": counters}
     print(json.dumps(line), flush=True)
 

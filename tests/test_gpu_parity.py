@@ -375,3 +375,21 @@ def test_layer_dense_cross_check_tiny():
     dense = O.moe_layer_dense(x, ridx, rw, fn, cfg.E)
     keep = margin >= 1e-4
     assert max_abs_rel(np64(gpu["y"])[keep], dense[keep]) <= F32_MAXABS_REL
+
+
+@pytest.mark.parametrize("tau", [1.0, 2.0, 0.5])
+def test_soft_routing_with_temperature(tau):
+    """Soft routing (jsqmd.com chapter 11, 11.3.3): y = sum_i softmax(s/tau)_i
+    E_i(x) over all experts.  The layer with K = E and renormalised gates
+    computes it when the router weights are scaled by 1/tau (a power of two
+    here, so the scaling is exact)."""
+    cfg = syn.scaled(syn.CONFIGS["tiny_f32"], K=8)
+    inp = syn.make_inputs(cfg, "cuda", seed=4)
+    inp_t = dict(inp)
+    inp_t["w_router"] = inp["w_router"] / tau
+    gpu = run_layer(inp_t, cfg)
+    x = np64(inp["x"])
+    logits = O.router_logits(x, np64(inp["w_router"]))
+    fn = OracleExperts(inp, cfg)
+    ref = O.soft_routing(x, logits, fn, cfg.E, tau)
+    assert max_abs_rel(np64(gpu["y"]), ref) <= F32_MAXABS_REL
