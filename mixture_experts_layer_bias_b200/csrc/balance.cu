@@ -16,8 +16,8 @@
 // The ring holds the expert ids of the last `window` tokens, filled from
 // position 0; a batch of S tokens takes the next S positions (only its last
 // `window` tokens when S >= window), decrementing the counts of the tokens it
-// replaces.  One CTA does the whole update: counts are integer atomics, so
-// the result does not depend on their order.
+// replaces.  One CTA does the whole update: the batch's count changes are
+// integer shared-memory atomics, so the result does not depend on their order.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -29,17 +29,18 @@ __global__ void __launch_bounds__(1024)
     bias_update_kernel(int S, int E, int K, int W, const int32_t* __restrict__ topk_idx, float gamma,
                        int32_t* __restrict__ hdr, int32_t* __restrict__ counts, int32_t* __restrict__ ring,
                        float* __restrict__ sel_bias, int32_t* __restrict__ out_counts) {
+  __shared__ int32_t delta[256];  // count changes of this batch (E <= 256), shared-memory atomics
   const int filled = hdr[0], head = hdr[1];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) delta[e] = 0;
+  __syncthreads();
   int new_filled, new_head;
   if (S >= W) {
-    for (int e = threadIdx.x; e < E; e += blockDim.x) counts[e] = 0;
-    __syncthreads();
     for (int64_t s = threadIdx.x; s < static_cast<int64_t>(W) * K; s += blockDim.x) {
       const int64_t src = static_cast<int64_t>(S - W) * K + s;  // the batch's last W tokens
       const int id = topk_idx[src];
       const bool ok = id >= 0 && id < E;
       ring[s] = ok ? id : -1;
-      if (ok) atomicAdd(&counts[id], 1);
+      if (ok) atomicAdd(&delta[id], 1);
     }
     new_filled = W;
     new_head = 0;
@@ -50,12 +51,12 @@ __global__ void __launch_bounds__(1024)
       const int64_t at = static_cast<int64_t>(pos) * K + k;
       if (filled == W || pos < filled) {
         const int old = ring[at];
-        if (old >= 0 && old < E) atomicSub(&counts[old], 1);
+        if (old >= 0 && old < E) atomicSub(&delta[old], 1);
       }
       const int id = topk_idx[s];
       const bool ok = id >= 0 && id < E;
       ring[at] = ok ? id : -1;
-      if (ok) atomicAdd(&counts[id], 1);
+      if (ok) atomicAdd(&delta[id], 1);
     }
     new_filled = min(W, filled + S);
     new_head = (head + S) % W;
@@ -63,7 +64,8 @@ __global__ void __launch_bounds__(1024)
   __syncthreads();
   const float mean = __fdiv_rn(static_cast<float>(new_filled * K), static_cast<float>(E));
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    const int c = counts[e];
+    const int c = (S >= W ? 0 : counts[e]) + delta[e];
+    counts[e] = c;
     const float diff = __fsub_rn(mean, static_cast<float>(c));
     float b = sel_bias[e];
     if (diff > 0.0f)
