@@ -27,7 +27,7 @@
 // or split-K partial sums).  Waits are bounded in time as in the one-CTA
 // kernel.  No load uses cluster multicast; only the MMA completion signal
 // (tcgen05.commit) reaches both CTAs.
-#include "gemm_common.cuh"
+#include "gemm_wt_epilogue.cuh"
 
 namespace moe {
 
@@ -99,99 +99,6 @@ __device__ __forceinline__ PairUnit pair_unit(const PairCtl& s, const TcParams& 
 __device__ __forceinline__ bool wait_timed_pair(uint64_t* bar, uint32_t parity) {
   int never = 0;
   return mbar_wait(bar, parity, &never);
-}
-
-constexpr int P_CHUNK = 16;  // tokens per epilogue chunk (one 32x32b.x16 TMEM load)
-
-// Epilogue of one 16-token chunk: r[j] is the accumulator of this thread's
-// TMEM lane (weight row) for token tb*256 + chunk*16 + j.
-template <int EPI>
-__device__ __forceinline__ void pair_store_chunk(const TcParams& p, const PairUnit& pu, uint32_t rank, int q, int lane,
-                                                 int chunk, const uint32_t (&r)[P_CHUNK], int ks,
-                                                 __nv_bfloat16* tbuf) {
-  const int N = p.N;
-  const int t0 = pu.tb * P_TOK + chunk * P_CHUNK;  // first token of the chunk inside the group
-  const int64_t row0 = static_cast<int64_t>(pu.grp.out_row0) + t0;
-  const int64_t sbase = static_cast<int64_t>(pu.grp.expert) * N;
-  const int tlim = min(P_CHUNK, pu.grp.rows - t0);  // valid tokens in this chunk
-  if (EPI == EPI_SWIGLU) {
-    const int blk = q * 2 + (lane >> 4);  // 16-row block of this CTA's weight rows
-    const bool is_up = blk & 1;
-    const int fbase = pu.fb * PairShape<EPI>::FEAT + static_cast<int>(rank) * 64 + (blk >> 1) * 16;
-    const int f = fbase + (lane & 15);
-    const bool fvalid = f < N;
-    if (ks > 1) {
-      if (!fvalid) return;
-      float* base = p.partial + (static_cast<int64_t>(pu.split) * p.out_rows + row0) * p.pcols + (is_up ? N : 0) + f;
-#pragma unroll
-      for (int j = 0; j < P_CHUNK; ++j)
-        if (j < tlim) base[static_cast<int64_t>(j) * p.pcols] = __uint_as_float(r[j]);
-      return;
-    }
-    float sg = 1.0f, su = 1.0f;
-    if (p.scale0 != nullptr && fvalid) {
-      sg = __ldg(p.scale0 + sbase + f);
-      su = __ldg(p.scale1 + sbase + f);
-    }
-    // lanes 0-15: h for 16 features x 16 tokens -> tbuf[token][feature] (16 x 16 bf16)
-#pragma unroll
-    for (int j = 0; j < P_CHUNK; ++j) {
-      const float mine = __uint_as_float(r[j]);
-      const float up = __shfl_xor_sync(0xFFFFFFFFu, mine, 16);
-      if (!is_up) {
-        const float g = mine * sg;
-        tbuf[j * 16 + lane] = __float2bfloat16_rn(g / (1.0f + __expf(-g)) * (up * su));
-      }
-    }
-    __syncwarp();
-    // 16 tokens x 32 bytes = 32 pieces of 16 bytes, one per lane
-    const int tok = lane >> 1, sub = lane & 1;
-    const int fo = fbase + sub * 8;
-    if (tok < tlim && fo + 8 <= N)
-      stg16(static_cast<__nv_bfloat16*>(p.out) + (row0 + tok) * N + fo,
-            *reinterpret_cast<const uint4*>(tbuf + tok * 16 + sub * 8));
-    __syncwarp();
-  } else {
-    const int fbase = pu.fb * PairShape<EPI>::FEAT + static_cast<int>(rank) * 128 + q * 32;
-    const int f = fbase + lane;
-    if (ks > 1) {
-      if (f >= N) return;
-      float* base = p.partial + (static_cast<int64_t>(pu.split) * p.out_rows + row0) * p.pcols + f;
-#pragma unroll
-      for (int j = 0; j < P_CHUNK; ++j)
-        if (j < tlim) base[static_cast<int64_t>(j) * p.pcols] = __uint_as_float(r[j]);
-      return;
-    }
-    const bool fvalid = f < N;
-    const float sc = (p.scale0 != nullptr && fvalid) ? __ldg(p.scale0 + sbase + f) : 1.0f;
-    const float bi = ((EPI == EPI_GELU_BIAS || EPI == EPI_BIAS) && fvalid) ? __ldg(p.bias + sbase + f) : 0.0f;
-    if (p.out_f32) {
-      // fp32 output (router logits): 32 lanes write 128 contiguous bytes per token
-      if (!fvalid) return;
-#pragma unroll
-      for (int j = 0; j < P_CHUNK; ++j)
-        if (j < tlim) static_cast<float*>(p.out)[(row0 + j) * N + f] = __uint_as_float(r[j]) * sc + bi;
-      return;
-    }
-#pragma unroll
-    for (int j = 0; j < P_CHUNK; ++j) {
-      float z = __uint_as_float(r[j]) * sc + bi;
-      if (EPI == EPI_GELU_BIAS) z = 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
-      tbuf[j * 32 + lane] = __float2bfloat16_rn(z);
-    }
-    __syncwarp();
-    // 16 tokens x 64 bytes = 64 pieces of 16 bytes, two per lane
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int piece = lane + 32 * h;
-      const int tok = piece >> 2, sub = piece & 3;
-      const int fo = fbase + sub * 8;
-      if (tok < tlim && fo + 8 <= N)
-        stg16(static_cast<__nv_bfloat16*>(p.out) + (row0 + tok) * N + fo,
-              *reinterpret_cast<const uint4*>(tbuf + tok * 32 + sub * 8));
-    }
-    __syncwarp();
-  }
 }
 
 template <int EPI>
@@ -390,12 +297,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
       }
       tc_fence_after();
       const uint32_t tbase = tmem + acc * P_ACC_COLS + (static_cast<uint32_t>(q * 32) << 16);
-      const int nchunks = (pu.nt + P_CHUNK - 1) / P_CHUNK;
+      const int nchunks = (pu.nt + WT_CHUNK - 1) / WT_CHUNK;
+      const int feat0 = pu.fb * FEAT + static_cast<int>(rank) * (FEAT / 2);
       for (int c = 0; c < nchunks; ++c) {
-        uint32_t r[P_CHUNK];
-        tmem_ld_32x32b_x16(tbase + c * P_CHUNK, r);
+        uint32_t r[WT_CHUNK];
+        tmem_ld_32x32b_x16(tbase + c * WT_CHUNK, r);
         tmem_ld_wait();
-        pair_store_chunk<EPI>(p, pu, rank, q, lane, c, r, ks, tbufs + (warp - 2) * (P_TBUF / 2));
+        wt_store_chunk<EPI>(p, pu.grp, pu.split, feat0, pu.tb * P_TOK, q, lane, c, r, ks,
+                            tbufs + (warp - 2) * (P_TBUF / 2));
       }
       tc_fence_before();
       __syncwarp();
