@@ -44,18 +44,23 @@ using namespace gemm;
 
 constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = 128 bytes = one swizzle row
-constexpr int STAGES = 4;
-constexpr int A_TILE = BM * BK * 2;           // 16 KB
+// Ring: one stage = A rows (bma x 64 bf16, bma <= 128) then B (256 x 64 bf16).
+// Prefill loads all 128 token rows of A (4 stages of 48 KB).  When every group
+// fits in bma < 128 rows (decode), only those rows are loaded and the shared
+// memory saved becomes extra stages, i.e. more weight bytes in flight; the
+// MMA still reads 128 A rows, the rows past bma being the start of the same
+// stage's B tile, and their accumulator rows are never stored.
+constexpr int MAX_STAGES = 8;
 constexpr int B_HALF = 128 * BK * 2;          // 16 KB
-constexpr int STAGE_BYTES = A_TILE + 2 * B_HALF;  // 48 KB
+constexpr int B_TILE = 2 * B_HALF;            // 32 KB
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
 constexpr int kThreads = 192;
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, 256);
 
 struct SmemCtl {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[MAX_STAGES];
+  uint64_t empty[MAX_STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -65,7 +70,8 @@ struct SmemCtl {
   int tile_start[kMaxGroups + 1];
 };
 
-constexpr size_t kSmemBytes = STAGES * STAGE_BYTES + sizeof(SmemCtl) + 1024;
+constexpr size_t kSmemLimitTc = 232448;  // 227 KB per CTA
+constexpr size_t kCtlBytes = sizeof(SmemCtl) + 1024;  // control block + alignment slack
 
 __device__ __forceinline__ bool wait_timed(uint64_t* bar, uint32_t parity) {
   int never = 0;
@@ -199,9 +205,11 @@ template <int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                            const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
-                           TcParams p) {
+                           TcParams p, int bma, int STAGES) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int A_TILE = bma * BK * 2;
+  const int STAGE_BYTES = A_TILE + B_TILE;
   SmemCtl& s = *reinterpret_cast<SmemCtl*>(ring + STAGES * STAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = lane_id();
 
@@ -394,18 +402,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int EPI>
 cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB0, const CUtensorMap& mB1,
-                       const TcParams& p, int grid, int64_t max_group_rows, cudaStream_t stream) {
+                       const TcParams& p, int grid, int bma, int stages, size_t smem, int64_t max_group_rows,
+                       cudaStream_t stream) {
   static uint64_t attr_set = 0;  // one bit per device ordinal
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64 || !(attr_set & (1ull << dev))) {
     e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes));
+                             static_cast<int>(kSmemLimitTc));
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set |= 1ull << dev;
   }
-  grouped_gemm_tc_kernel<EPI><<<grid, kThreads, kSmemBytes, stream>>>(mA, mA2, mB0, mB1, p);
+  grouped_gemm_tc_kernel<EPI><<<grid, kThreads, smem, stream>>>(mA, mA2, mB0, mB1, p, bma, stages);
   e = cudaGetLastError();
   if (e != cudaSuccess || p.max_ksplit <= 1) return e;
   dim3 fgrid((p.N + 1023) / 1024, static_cast<unsigned>(max_group_rows), p.num_groups);
@@ -417,10 +426,17 @@ cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUte
 
 // Token-rows kernel launch; `p` is filled by the dispatcher.
 cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& p, int num_sms, cudaStream_t stream) {
+  // A rows loaded per stage: all 128, or (every group fitting) the largest group rounded up to 16
+  int bma = BM;
+  if (a.max_group_rows > 0 && a.max_group_rows <= 64) bma = static_cast<int>((a.max_group_rows + 15) & ~int64_t(15));
+  const size_t stage_bytes = static_cast<size_t>(bma) * BK * 2 + B_TILE;
+  int stages = static_cast<int>((kSmemLimitTc - kCtlBytes) / stage_bytes);
+  if (stages > MAX_STAGES) stages = MAX_STAGES;
+  const size_t smem = stages * stage_bytes + kCtlBytes;
   CUtensorMap mA, mA2, mB0, mB1;
-  if (!make_map(&mA, a.a, a.a_rows, a.K)) return cudaErrorInvalidValue;
+  if (!make_map(&mA, a.a, a.a_rows, a.K, bma)) return cudaErrorInvalidValue;
   if (a.a_shared != nullptr) {
-    if (!make_map(&mA2, a.a_shared, a.a_shared_rows, a.K)) return cudaErrorInvalidValue;
+    if (!make_map(&mA2, a.a_shared, a.a_shared_rows, a.K, bma)) return cudaErrorInvalidValue;
   } else {
     mA2 = mA;
   }
@@ -434,10 +450,14 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
   const int64_t bound = (a.max_total_rows / BM + a.num_groups) * static_cast<int64_t>(p.n_tiles);
   const int grid = static_cast<int>(bound < num_sms ? (bound > 0 ? bound : 1) : num_sms);
   switch (a.epilogue) {
-    case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(mA, mA2, mB0, mB1, p, grid, a.max_group_rows, stream);
-    case EPI_GELU_BIAS: return launch_epi<EPI_GELU_BIAS>(mA, mA2, mB0, mB1, p, grid, a.max_group_rows, stream);
-    case EPI_BIAS: return launch_epi<EPI_BIAS>(mA, mA2, mB0, mB1, p, grid, a.max_group_rows, stream);
-    case EPI_NONE: return launch_epi<EPI_NONE>(mA, mA2, mB0, mB1, p, grid, a.max_group_rows, stream);
+    case EPI_SWIGLU:
+      return launch_epi<EPI_SWIGLU>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows, stream);
+    case EPI_GELU_BIAS:
+      return launch_epi<EPI_GELU_BIAS>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows, stream);
+    case EPI_BIAS:
+      return launch_epi<EPI_BIAS>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows, stream);
+    case EPI_NONE:
+      return launch_epi<EPI_NONE>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows, stream);
     default: return cudaErrorInvalidValue;
   }
 }
