@@ -621,3 +621,86 @@ class WindowBias:
             elif diff < 0:
                 b[e] = np.float32(b[e] - g)
         return b, c
+
+
+# ----------------------------------------------------------------------------
+# W8A8: E4M3 activations with per-row scales (NEXT row)
+# ----------------------------------------------------------------------------
+
+
+def f32_to_e4m3_bits(v: np.ndarray) -> np.ndarray:
+    """float32 values -> E4M3 bit patterns, round to nearest, ties to even,
+    saturating at +-448 (the largest finite E4M3 value); NaN -> 0x7F.
+
+    The E4M3 grid: exponent e in [-6, 8] with 3 mantissa bits (spacing
+    2**(e-3)); below 2**-6 the subnormal spacing is 2**-9.  Rounding is done
+    on the exact float64 value of the float32 input (no double rounding).
+    """
+    x = np.asarray(v, dtype=np.float32).astype(np.float64)
+    out = np.zeros(x.shape, dtype=np.uint8)
+    flat, o = x.reshape(-1), out.reshape(-1)
+    for i, val in enumerate(flat):
+        if math.isnan(val):
+            o[i] = 0x7F
+            continue
+        sign = 0x80 if math.copysign(1.0, val) < 0 else 0
+        a = abs(val)
+        if a >= 448.0:
+            o[i] = sign | 0x7E
+            continue
+        if a == 0.0:
+            o[i] = sign
+            continue
+        e = max(math.frexp(a)[1] - 1, -6)  # exponent of the grid containing a
+        q = math.ldexp(1.0, e - 3)         # spacing of that grid
+        n = a / q
+        r = math.floor(n)
+        frac = n - r
+        if frac > 0.5 or (frac == 0.5 and r % 2 == 1):
+            r += 1
+        val_r = r * q
+        if val_r > 448.0:
+            val_r = 448.0
+        # encode val_r exactly
+        if val_r < math.ldexp(1.0, -6):
+            o[i] = sign | int(round(val_r / math.ldexp(1.0, -9)))
+        else:
+            m, ee = math.frexp(val_r)  # val_r = m * 2**ee, m in [0.5, 1)
+            exp_field = ee - 1 + 7
+            mant = int(round((m * 2.0 - 1.0) * 8.0))
+            if mant == 8:  # rounding carried into the next binade
+                mant, exp_field = 0, exp_field + 1
+            o[i] = sign | (exp_field << 3) | mant
+    return out
+
+
+def quantize_rows_e4m3(rows: np.ndarray):
+    """Per-row E4M3 quantisation of float32 rows (the W8A8 activations):
+    amax = max_j |x_j|; scale s = amax / 448 as one float32 division (1 when
+    the row is all zero); codes q_j = E4M3(x_j / s), the quotient a float32
+    division, rounded to nearest even.  Returns (codes uint8 [n, d], s float32
+    [n]); the dequantised row is q * s."""
+    x = np.asarray(rows, dtype=np.float32)
+    amax = np.max(np.abs(x), axis=1).astype(np.float32)
+    s = np.where(amax > 0, np.divide(amax, np.float32(448.0), dtype=np.float32), np.float32(1.0)).astype(np.float32)
+    ratio = np.divide(x, s[:, None], dtype=np.float32)
+    return f32_to_e4m3_bits(ratio), s
+
+
+def expert_swiglu_w8a8(x, q_gate, q_up, q_down, s_gate, s_up, s_down, round_hidden_bf16=True):
+    """SwiGLU expert with E4M3 weights (per-output-channel scales) applied to
+    E4M3-quantised activations: x rows are quantised per row
+    (``quantize_rows_e4m3``), the hidden rows are rounded to bfloat16 and
+    quantised per row again before the down projection.  float64 sums."""
+    x = np.asarray(x, dtype=np.float64)
+    qx, sx = quantize_rows_e4m3(x.astype(np.float32))
+    xq = e4m3_bits_to_f64(qx) * sx[:, None].astype(np.float64)
+    wg = e4m3_bits_to_f64(q_gate) * np.asarray(s_gate, np.float64)[:, None]
+    wu = e4m3_bits_to_f64(q_up) * np.asarray(s_up, np.float64)[:, None]
+    wd = e4m3_bits_to_f64(q_down) * np.asarray(s_down, np.float64)[:, None]
+    hid = silu(xq @ wg.T) * (xq @ wu.T)
+    if round_hidden_bf16:
+        hid = bf16_bits_to_f64(f64_to_bf16_bits_fast(hid))
+    qh, sh = quantize_rows_e4m3(hid.astype(np.float32))
+    hq = e4m3_bits_to_f64(qh) * sh[:, None].astype(np.float64)
+    return hq @ wd.T

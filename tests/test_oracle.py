@@ -449,3 +449,60 @@ def test_bias_update_steers_load_toward_balance():
         ratios.append(O.load_stats(O.expert_counts(idx, E), K, S)["max_over_mean"])
         b, _ = wb.update(idx, b, 0.05)
     assert ratios[0] > 2.0 and np.mean(ratios[-10:]) < 0.6 * ratios[0]
+
+
+# ----------------------------------------------------------------------------
+# E4M3 encoder and per-row quantisation (W8A8)
+# ----------------------------------------------------------------------------
+
+
+def test_f32_to_e4m3_matches_torch_rne():
+    rng = np.random.default_rng(12)
+    v = np.concatenate([
+        (rng.normal(size=20000) * np.exp(rng.normal(size=20000) * 3)),
+        O.e4m3_bits_to_f64(np.arange(0, 0x7F, dtype=np.uint8)),          # every finite code exactly
+        (O.e4m3_bits_to_f64(np.arange(0, 0x7E, dtype=np.uint8)) +
+         O.e4m3_bits_to_f64(np.arange(1, 0x7F, dtype=np.uint8))) / 2,   # every tie
+    ]).astype(np.float32)
+    v = v[np.abs(v) < 464]  # torch's encoder is not saturating past the rounding edge
+    mine = O.f32_to_e4m3_bits(v)
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(mine, ref)
+    assert O.f32_to_e4m3_bits(np.array([1e6, -500.0], np.float32)).tolist() == [0x7E, 0xFE]  # saturates
+
+
+def test_quantize_rows_round_trip_error_bound():
+    """Dequantised rows are within half an E4M3 step of the input: relative
+    2**-4 for normal codes, absolute s * 2**-10 near zero; the row maximum maps
+    to 448 exactly."""
+    rng = np.random.default_rng(13)
+    x = (rng.normal(size=(50, 300)) * np.exp(rng.normal(size=(50, 1)))).astype(np.float32)
+    x[3] = 0.0
+    q, s = O.quantize_rows_e4m3(x)
+    back = O.e4m3_bits_to_f64(q) * s[:, None]
+    err = np.abs(back - x)
+    bound = np.maximum(np.abs(x) * 2.0 ** -4, s[:, None] * 2.0 ** -10) * 1.0000001
+    assert np.all(err <= bound)
+    assert s[3] == 1.0 and np.all(q[3] == 0)
+    top = np.argmax(np.abs(x), axis=1)
+    nz = np.arange(50) != 3
+    assert np.all(np.abs(O.e4m3_bits_to_f64(q[np.arange(50), top]))[nz] == 448.0)
+
+
+def test_w8a8_expert_close_to_exact_expert():
+    """With 8-bit activations the expert output stays within the quantisation
+    noise of the same expert on unquantised activations (relative L2 a few
+    percent), and equals it exactly when activations are E4M3-representable
+    multiples of their row scale."""
+    rng = np.random.default_rng(14)
+    d, h = 64, 96
+    wg, wu, wd = (rng.normal(size=(h, d)) / 8, rng.normal(size=(h, d)) / 8, rng.normal(size=(d, h)) / 10)
+    qg, sg = (lambda q: (q[0], q[1]))(O.quantize_rows_e4m3(wg.astype(np.float32)))
+    qu, su = O.quantize_rows_e4m3(wu.astype(np.float32))
+    qd, sd = O.quantize_rows_e4m3(wd.astype(np.float32))
+    x = rng.normal(size=(20, d))
+    y8 = O.expert_swiglu_w8a8(x, qg, qu, qd, sg, su, sd, round_hidden_bf16=False)
+    yref = O.expert_swiglu(x, O.e4m3_bits_to_f64(qg), O.e4m3_bits_to_f64(qu), O.e4m3_bits_to_f64(qd),
+                           s_gate=sg, s_up=su, s_down=sd)
+    rel = np.linalg.norm(y8 - yref) / np.linalg.norm(yref)
+    assert 1e-4 < rel < 5e-2
