@@ -85,7 +85,8 @@ def workload_desc(cfg):
     return (f"{cfg.name}: S={cfg.S} d={cfg.d} E={cfg.E} K={cfg.K} h={cfg.h} "
             f"{'SwiGLU' if cfg.activation == syn.SWIGLU else 'GeLU'} "
             f"{'bf16' if cfg.act_dtype == syn.BF16 else 'fp32'} act, "
-            f"{ {0: 'fp32', 1: 'bf16', 2: 'e4m3'}[cfg.weight_dtype]} weights")
+            f"{ {0: 'fp32', 1: 'bf16', 2: 'e4m3'}[cfg.weight_dtype]} weights"
+            f"{', W8A8 (e4m3 activation rows, per-row scales)' if cfg.act_quant else ''}")
 
 
 def kernels_per_step(cfg):
@@ -93,10 +94,12 @@ def kernels_per_step(cfg):
     n = 1 if (cfg.E <= 32) else 2          # route (fused) or logits + top-k
     n += 4                                 # count, scan, scatter, gather
     n += 1 + 2                             # group table, up and down GEMM
-    if cfg.weight_dtype == syn.E4M3:
+    if cfg.act_quant:
+        n += 2                             # per-row E4M3 quantisation of each GEMM's A rows
+    elif cfg.weight_dtype == syn.E4M3:
         n += 3                             # E4M3 -> bf16 decode of the three stacks
     if cfg.capacity:
-        n += 2                             # overflow pass
+        n += 4 if cfg.act_quant else 2     # overflow pass (with its two quantisations)
     n += 1                                 # combine
     return n
 
@@ -308,7 +311,8 @@ def cpu_baseline(cfg, inp, n_tokens=32):
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    cfg = syn.CONFIGS[WORKLOAD]
+    name = WORKLOAD if args.workload == "profile_small" else args.workload
+    cfg = syn.CONFIGS.get(name) or syn.VARIANTS[name]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = make_layer_inputs(cfg, dev)
     n_tok = 8
@@ -345,7 +349,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(syn.CONFIGS) + ["profile_small"],
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=sorted(syn.CONFIGS) + sorted(syn.VARIANTS) + ["profile_small"],
                     help="profile_small: S=2048, d=4096, h=4096 (same kernels, ~1 GB) for ncu captures")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -367,7 +372,7 @@ def main():
     if args.workload == "profile_small":
         cfg = syn.scaled(syn.CONFIGS[WORKLOAD], S=2048, h=4096)
     else:
-        cfg = syn.CONFIGS[args.workload]
+        cfg = syn.CONFIGS.get(args.workload) or syn.VARIANTS[args.workload]
     S = cfg.S
     inp = make_layer_inputs(cfg, device)
     desc = ops.make_desc(**syn.desc_dict(cfg, S))
@@ -405,6 +410,8 @@ def main():
     flops = expert_flops(cfg, rows)
     wbytes = {syn.F32: 4, syn.BF16: 2, syn.E4M3: 1}[cfg.weight_dtype]
     abytes = 4 if cfg.act_dtype == syn.F32 else 2
+    if cfg.act_quant:
+        abytes = 1  # the GEMMs read 8-bit rows (the quantisers' bf16 reads are not counted)
     n_up = 2 if cfg.activation == syn.SWIGLU else 1
     # weights of every expert + permuted rows in + hidden out/in + expert rows out
     algo_bytes = ((cfg.E + cfg.num_shared) * (n_up + 1) * cfg.d * cfg.h * wbytes
@@ -413,12 +420,17 @@ def main():
     achieved = flops / (ffn_ms * 1e-3) / 1e12
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    peak_kind = "bf16 burst"
+    if cfg.act_quant:
+        # E4M3 x E4M3: the measured bf16 peak times the nominal fp8 : bf16 ratio (4.5 : 2.25)
+        peak, sustained = 2 * peak, 2 * sustained
+        peak_kind = "bf16 burst x 2 (nominal e4m3 : bf16 ratio)"
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "frac_of_sustained_peak": round(achieved / sustained, 4),
                 "traffic": ffn_traffic(args.workload),
                 "algorithmic_bytes": algo_bytes,
                 "kernel": "grouped expert FFN (up SwiGLU + down GEMMs, tcgen05)",
-                "peak_source": f"{peaks['source']} bf16 burst"}
+                "peak_source": f"{peaks['source']} {peak_kind}"}
 
     # end to end through the public call with host buffers: every step copies its
     # input from pinned host memory and its output back.  As in a serving loop,
@@ -490,7 +502,8 @@ def main():
         cpu = cpu_baseline(cfg, inp)
     line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if cfg.act_quant else "bf16",
+            "data": "synthetic",
             "config": {"workload": workload_desc(cfg), "global_batch": world * S, "seq_len": S,
                        "parallelism": f"replicas x{world}",
                        "l2": "no flush: the expert weights read every step exceed the 126 MB L2"},

@@ -91,9 +91,18 @@ typedef enum { MOE_ACT_GELU = 0, MOE_ACT_SWIGLU = 1 } moe_act;
  *   capacity: 0 = unbounded; C > 0 = at most C rows per expert in the
  *     primary block, the rest in an overflow region processed in a second
  *     pass (ybb.press 2.2, overflow buffering).  No token is dropped.
+ *   act_quant: 0 = the expert GEMMs read bf16 activations (E4M3 weights are
+ *     decoded to bf16 first); 1 = W8A8: each A row of both expert GEMMs
+ *     (the permuted tokens, then the bf16 hidden rows) is quantised to E4M3
+ *     with one fp32 scale per row (moe_quantize_rows_e4m3) and the GEMMs run
+ *     on 8-bit operands, the epilogue applying row and channel scales.  The
+ *     pages list E4M3 only as a storage format (ybb.press 3.3); per-row
+ *     activation scaling is this library's reading.  Needs BF16 act, E4M3
+ *     weights, SWIGLU, d and h multiples of 16.
  * Supported: (F32 act, F32 weights, GELU) with E <= 32 on the SIMT path;
- * (BF16 act, BF16 or E4M3 weights, SWIGLU or GELU) on the tensor-core path.
- * E <= 256, K <= min(E, 32), d and h multiples of 8.
+ * (BF16 act, BF16 or E4M3 weights, SWIGLU or GELU; E4M3 with SWIGLU only)
+ * on the tensor-core path.  E <= 256, K <= min(E, 32), d and h multiples
+ * of 8.
  */
 typedef struct {
   int32_t num_tokens;
@@ -110,6 +119,7 @@ typedef struct {
   int32_t act_dtype;
   int32_t weight_dtype;
   int32_t capacity;
+  int32_t act_quant;
 } moe_desc;
 
 /* Weights, all DEVICE pointers (see layouts above).  Unused ones may be
@@ -208,6 +218,22 @@ moe_status moe_permute_static(const moe_desc *desc, const void *x, const int32_t
 moe_status moe_grouped_ffn(const moe_desc *desc, const moe_weights *w, const void *x_perm,
                            const int32_t *offsets, const void *x, void *y_perm, void *ws, size_t ws_bytes,
                            void *stream);
+
+/*
+ * Per-row E4M3 quantisation of bf16 rows, the activation step of the W8A8
+ * path (act_quant = 1), exposed on its own.  For each row i of x [rows][d]
+ * (bf16, row-major, DEVICE, 16-byte aligned, d a multiple of 16):
+ *   s[i]    = max_j |x[i][j]| / 448 as one fp32 division; 1 when the row is
+ *             all zero or holds a NaN;
+ *   q[i][j] = E4M3(x[i][j] / s[i]): fp32 division, round to nearest even,
+ *             saturating at +-448; NaN -> 0x7F.
+ * q [rows][d] uint8 and s [rows] fp32 are caller-owned DEVICE buffers (q
+ * 16-byte aligned).  Launches one kernel on `stream`, allocates nothing.
+ * rows = 0 is a no-op.  Errors: MOE_ERR_INVALID_ARG for a NULL or misaligned
+ * pointer, rows < 0 or d not a positive multiple of 16; MOE_ERR_CUDA when
+ * the launch fails.  There is no workspace or status block.
+ */
+moe_status moe_quantize_rows_e4m3(const void *x, int64_t rows, int32_t d, uint8_t *q, float *s, void *stream);
 
 /*
  * Gate-weighted combine back into token order (11.3.1 step 6; plumephp.com

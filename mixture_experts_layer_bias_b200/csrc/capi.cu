@@ -21,7 +21,7 @@ size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 
 struct Layout {
   size_t status, logits, chunk_hist, groups1, groups2, counts, offsets, topk_idx, topk_w, row_of_slot, token_of_row,
-      x_perm, hidden, y_perm, wdeq, ksplit, partial, partial_bytes, total;
+      x_perm, hidden, y_perm, wdeq, ksplit, partial, partial_bytes, qa, sa, qas, sas, qh, sh, total;
 };
 
 // Split-K of the tensor-core GEMMs is available to small row spaces (decode-
@@ -64,7 +64,16 @@ Layout make_layout(const moe_desc& d) {
   L.x_perm = take(static_cast<size_t>(R * dm) * ab);
   L.hidden = take(static_cast<size_t>(Rt * h) * ab);
   L.y_perm = take(static_cast<size_t>(Rt * dm) * ab);
-  L.wdeq = take(d.weight_dtype == MOE_E4M3 ? static_cast<size_t>((E + d.num_shared) * 3 * h * dm) * 2 : 0);
+  const bool w8a8 = d.act_quant == 1;
+  L.wdeq = take(d.weight_dtype == MOE_E4M3 && !w8a8 ? static_cast<size_t>((E + d.num_shared) * 3 * h * dm) * 2 : 0);
+  // W8A8: E4M3 codes and row scales of the up GEMM's A rows (permuted
+  // tokens; the shared expert's tokens) and of the down GEMM's (hidden rows)
+  L.qa = take(w8a8 ? static_cast<size_t>(R * dm) : 0);
+  L.sa = take(w8a8 ? static_cast<size_t>(R) * 4 : 0);
+  L.qas = take(w8a8 && d.num_shared ? static_cast<size_t>(S * dm) : 0);
+  L.sas = take(w8a8 && d.num_shared ? static_cast<size_t>(S) * 4 : 0);
+  L.qh = take(w8a8 ? static_cast<size_t>(Rt * h) : 0);
+  L.sh = take(w8a8 ? static_cast<size_t>(Rt) * 4 : 0);
   L.ksplit = take(kAlign);
   L.partial_bytes = 0;
   if (d.act_dtype == MOE_BF16 && Rt > 0 && Rt <= kSplitRowsMax) {
@@ -100,6 +109,7 @@ moe_status validate(const moe_desc* d) {
   if (d->weight_dtype != MOE_F32 && d->weight_dtype != MOE_BF16 && d->weight_dtype != MOE_E4M3)
     return MOE_ERR_INVALID_ARG;
   if (d->capacity < 0) return MOE_ERR_INVALID_ARG;
+  if (d->act_quant != 0 && d->act_quant != 1) return MOE_ERR_INVALID_ARG;
   // row indices are int32 on the device
   const int64_t rows = routed_rows(*d) + static_cast<int64_t>(d->num_shared) * d->num_tokens;
   if (rows > (int64_t(1) << 31) - 1) return MOE_ERR_INVALID_ARG;
@@ -110,6 +120,9 @@ moe_status validate(const moe_desc* d) {
     if (d->weight_dtype == MOE_F32) return MOE_ERR_UNSUPPORTED;
     if (d->weight_dtype == MOE_E4M3 && d->activation != MOE_ACT_SWIGLU) return MOE_ERR_UNSUPPORTED;
   }
+  if (d->act_quant == 1 && (d->act_dtype != MOE_BF16 || d->weight_dtype != MOE_E4M3 ||
+                            d->activation != MOE_ACT_SWIGLU || d->d_model % 16 != 0 || d->d_ff % 16 != 0))
+    return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 
@@ -257,7 +270,21 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
     down.bias = w.b2;
   } else {
     const void *wg = w.w_gate, *wu = w.w_up, *wd = w.w_down, *w1 = w.w1, *w2 = w.w2;
-    if (d.weight_dtype == MOE_E4M3) {
+    if (d.act_quant == 1) {
+      // W8A8: the GEMMs read the E4M3 weights as they are; A rows are
+      // quantised per row right before each GEMM (below)
+      up.fp8 = down.fp8 = 1;
+      up.scale0 = w.s_gate;
+      up.scale1 = w.s_up;
+      down.scale0 = w.s_down;
+      up.a = at<void>(ws, L.qa);
+      up.row_scale = at<float>(ws, L.sa);
+      up.a_shared = d.num_shared ? at<void>(ws, L.qas) : nullptr;
+      up.row_scale_shared = d.num_shared ? at<float>(ws, L.sas) : nullptr;
+      down.a = at<void>(ws, L.qh);
+      down.row_scale = at<float>(ws, L.sh);
+      down.row_scale_shared = nullptr;
+    } else if (d.weight_dtype == MOE_E4M3) {
       // exact E4M3 -> bf16 decode of this call's weights; the per-channel
       // scales are applied to the fp32 accumulators in the epilogues
       const int64_t n_up = static_cast<int64_t>(slabs) * h * dm;
@@ -295,7 +322,21 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
   auto run = [&](const GemmArgs& g) {
     return d.act_dtype == MOE_F32 ? launch_grouped_gemm_f32(g, st) : launch_grouped_gemm_tc(g, sms, st);
   };
-  if ((err = run(up)) != cudaSuccess || (err = run(down)) != cudaSuccess) return MOE_ERR_CUDA;
+  // W8A8: E4M3 codes + row scales of the A rows a GEMM over `g` reads
+  auto quant_up = [&](const GemmArgs& g) {
+    return launch_quantize_group_rows(g.groups, g.num_groups, 0, g.shared_slab, x_perm, at<uint8_t>(ws, L.qa),
+                                      at<float>(ws, L.sa), R, x, d.num_shared ? at<uint8_t>(ws, L.qas) : nullptr,
+                                      d.num_shared ? at<float>(ws, L.sas) : nullptr, S, dm, g.max_group_rows, st);
+  };
+  auto quant_down = [&](const GemmArgs& g) {
+    return launch_quantize_group_rows(g.groups, g.num_groups, 1, -1, hidden, at<uint8_t>(ws, L.qh),
+                                      at<float>(ws, L.sh), Rt, nullptr, nullptr, nullptr, 0, h, g.max_group_rows, st);
+  };
+  const bool w8a8 = d.act_quant == 1;
+  if (w8a8 && (err = quant_up(up)) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((err = run(up)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (w8a8 && (err = quant_down(down)) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((err = run(down)) != cudaSuccess) return MOE_ERR_CUDA;
   if (d.capacity > 0) {
     // second pass: the overflow rows, grouped by expert the same way
     GemmArgs up2 = up, down2 = down;
@@ -304,8 +345,12 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
     up2.shared_slab = -1;
     up2.a_shared = nullptr;
     up2.a_shared_rows = 0;
+    up2.row_scale_shared = nullptr;
     up2.max_total_rows = down2.max_total_rows = static_cast<int64_t>(S) * d.top_k;
-    if ((err = run(up2)) != cudaSuccess || (err = run(down2)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (w8a8 && (err = quant_up(up2)) != cudaSuccess) return MOE_ERR_CUDA;
+    if ((err = run(up2)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (w8a8 && (err = quant_down(down2)) != cudaSuccess) return MOE_ERR_CUDA;
+    if ((err = run(down2)) != cudaSuccess) return MOE_ERR_CUDA;
   }
   return MOE_OK;
 }
@@ -402,6 +447,14 @@ moe_status moe_grouped_ffn(const moe_desc* desc, const moe_weights* w, const voi
   if (desc->num_shared && x == nullptr) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x_perm) || !aligned16(y_perm) || (x && !aligned16(x))) return MOE_ERR_INVALID_ARG;
   return ffn_impl(*desc, *w, x_perm, offsets, x, y_perm, ws, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_quantize_rows_e4m3(const void* x, int64_t rows, int32_t d, uint8_t* q, float* s, void* stream) {
+  if (rows < 0 || d <= 0 || d % 16 != 0) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (x == nullptr || q == nullptr || s == nullptr || !aligned16(x) || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(s) & 3) != 0) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_quantize_rows(x, q, s, rows, d, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_combine(const moe_desc* desc, const void* y_perm, const int32_t* row_of_slot, const float* topk_w,

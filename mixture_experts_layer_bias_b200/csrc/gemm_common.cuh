@@ -35,8 +35,17 @@ struct TcParams {
   int pcols;           // 2N (SwiGLU: gate then up) or N
   int* ksplit_out;     // the split chosen on the device, read by the finalize kernel
   int test_stall;      // test hook: the producer delivers nothing (the bounded waits must give up)
+  const float* row_scale;         // E4M3 activations: per-row scale of the A operand rows (nullptr: none)
+  const float* row_scale_shared;  // ... of the shared expert's A rows (indexed by row within the group)
   StatusBlock* status;
 };
+
+// Scale of A row `r` (within group `g`) for 8-bit activations, 1 otherwise.
+__device__ __forceinline__ float a_row_scale(const TcParams& p, const GroupEntry& g, int r) {
+  if (p.row_scale == nullptr) return 1.0f;
+  if (g.expert == p.shared_slab && p.row_scale_shared != nullptr) return __ldg(p.row_scale_shared + r);
+  return __ldg(p.row_scale + (p.a_rows_from_out ? g.out_row0 : g.a_row0) + r);
+}
 
 __device__ __forceinline__ GroupEntry group_at(const TcParams& p, int g) {
   if (p.groups == nullptr) return GroupEntry{0, 0, p.single_rows, 0};
@@ -87,6 +96,7 @@ __global__ void __launch_bounds__(256) splitk_finalize_kernel(TcParams p) {
   if (orow >= p.out_rows) return;
   const int64_t sbase = static_cast<int64_t>(grp.expert) * N;
   const int64_t slice = p.out_rows * static_cast<int64_t>(p.pcols);
+  const float rs = a_row_scale(p, grp, r);
   float v[4] = {0.f, 0.f, 0.f, 0.f}, u[4] = {0.f, 0.f, 0.f, 0.f};
   for (int s = 0; s < ks; ++s) {
     const float* src = p.partial + s * slice + orow * p.pcols;
@@ -100,10 +110,10 @@ __global__ void __launch_bounds__(256) splitk_finalize_kernel(TcParams p) {
   float o[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    float g = v[j];
+    float g = v[j] * rs;
     if (p.scale0 != nullptr) g *= p.scale0[sbase + n + j];
     if (EPI == EPI_SWIGLU) {
-      float up = u[j];
+      float up = u[j] * rs;
       if (p.scale1 != nullptr) up *= p.scale1[sbase + n + j];
       o[j] = g / (1.0f + __expf(-g)) * up;
     } else {
@@ -137,16 +147,18 @@ inline EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// 2-D bf16 map over [rows][k] (row-major), box 64 (k) x box_rows, 128B swizzle.
-inline bool make_map(CUtensorMap* m, const void* base, int64_t rows, int k, int box_rows = 128) {
+// 2-D map over [rows][k] (row-major) of bf16 (elem_bytes 2) or 8-bit (1)
+// elements; box = one 128-byte swizzle row of k by box_rows rows.
+inline bool make_map(CUtensorMap* m, const void* base, int64_t rows, int k, int box_rows = 128, int elem_bytes = 2) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr || rows <= 0 || k <= 0) return false;
-  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || (static_cast<int64_t>(k) * 2) % 16 != 0) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || (static_cast<int64_t>(k) * elem_bytes) % 16 != 0) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(k) * 2};
-  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(k) * elem_bytes};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  return enc(m, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+             const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

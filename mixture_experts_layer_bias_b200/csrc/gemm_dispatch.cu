@@ -1,6 +1,7 @@
 // Grouped GEMM dispatch: fills the launch parameters shared by the tensor-core
 // kernels and picks one of them (token rows as M, the default; weights as M
-// on one CTA; weights as M on a CTA pair).
+// on one CTA; weights as M on a CTA pair).  E4M3 operands always take the
+// token-rows kernel.
 #include <stdlib.h>
 #include <string.h>
 
@@ -79,7 +80,10 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t 
     if (p.max_ksplit < 1) p.max_ksplit = 1;
   }
   p.test_stall = 0;
-  const int choice = gemm_kernel_choice();
+  p.row_scale = a.fp8 ? a.row_scale : nullptr;
+  p.row_scale_shared = a.fp8 ? a.row_scale_shared : nullptr;
+  if (a.fp8 && a.row_scale == nullptr) return cudaErrorInvalidValue;
+  const int choice = a.fp8 ? 0 : gemm_kernel_choice();  // 8-bit operands: token-rows kernel only
   if (choice == 1) return launch_grouped_gemm_pair(a, p, num_sms, stream);
   p.test_stall = take_test_stall();
   if (choice == 2 || (choice == 3 && a.epilogue != EPI_SWIGLU)) return launch_grouped_gemm_wt(a, p, num_sms, stream);

@@ -14,6 +14,12 @@
 // silu(gate) * up (x per-channel scales for FP8 weights) as bf16.
 // Down projection: 256 output columns per tile, optional bias / scale.
 //
+// With E4M3 activations and weights (W8A8) the same kernel runs on 8-bit
+// operands: a stage still holds 128-byte rows, now 128 K elements, and the
+// MMA kind is f8f6f4 (K = 32 per instruction); the epilogue multiplies each
+// accumulator row by its activation row scale and each column by the weight
+// channel scale.
+//
 // Structure (one CTA per SM, 192 threads):
 //   warp 0      TMA producer: A tile 128x64 and B tile 256x64 (bf16, 128-byte
 //               swizzle) per stage into a 4-stage shared-memory ring;
@@ -43,7 +49,7 @@ namespace {
 using namespace gemm;
 
 constexpr int BM = 128;
-constexpr int BK = 64;  // 64 bf16 = 128 bytes = one swizzle row
+constexpr int BK_BYTES = 128;  // one swizzle row: 64 bf16 or 128 E4M3 elements of K per stage
 // Ring: one stage = A rows (bma x 64 bf16, bma <= 128) then B (256 x 64 bf16).
 // Prefill loads all 128 token rows of A (4 stages of 48 KB).  When every group
 // fits in bma < 128 rows (decode), only those rows are loaded and the shared
@@ -51,12 +57,19 @@ constexpr int BK = 64;  // 64 bf16 = 128 bytes = one swizzle row
 // MMA still reads 128 A rows, the rows past bma being the start of the same
 // stage's B tile, and their accumulator rows are never stored.
 constexpr int MAX_STAGES = 8;
-constexpr int B_HALF = 128 * BK * 2;          // 16 KB
+constexpr int B_HALF = 128 * BK_BYTES;        // 16 KB
 constexpr int B_TILE = 2 * B_HALF;            // 32 KB
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
 constexpr int kThreads = 192;
-constexpr uint32_t kIdesc = idesc_bf16_f32(128, 256);
+constexpr uint32_t kIdescBf16 = idesc_bf16_f32(128, 256);
+constexpr uint32_t kIdescE4m3 = idesc_e4m3_f32(128, 256);
+
+// K elements per stage of the bf16 (F8 = false) and E4M3 (F8 = true) kernels
+template <bool F8>
+constexpr int bk_elems() {
+  return F8 ? BK_BYTES : BK_BYTES / 2;
+}
 
 struct SmemCtl {
   uint64_t full[MAX_STAGES];
@@ -122,6 +135,7 @@ __device__ __forceinline__ void epilogue_store(const TcParams& p, const TileInfo
   const int N = p.N;
   const int64_t orow = static_cast<int64_t>(ti.grp.out_row0) + row;
   const int64_t sbase = static_cast<int64_t>(ti.grp.expert) * N;
+  const float rs = valid ? a_row_scale(p, ti.grp, row) : 1.0f;
   constexpr int kChunks = (EPI == EPI_SWIGLU) ? 4 : 8;
   for (int c = 0; c < kChunks; ++c) {
     const int n = ti.n_idx * p.bn_out + c * 32;
@@ -134,8 +148,8 @@ __device__ __forceinline__ void epilogue_store(const TcParams& p, const TileInfo
       tmem_ld_wait();
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        float g = __uint_as_float(r0[j]);
-        float u = __uint_as_float(r1[j]);
+        float g = __uint_as_float(r0[j]) * rs;
+        float u = __uint_as_float(r1[j]) * rs;
         if (p.scale0 != nullptr && n + j < N) {
           g *= __ldg(p.scale0 + sbase + n + j);
           u *= __ldg(p.scale1 + sbase + n + j);
@@ -147,7 +161,7 @@ __device__ __forceinline__ void epilogue_store(const TcParams& p, const TileInfo
       tmem_ld_wait();
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        float z = __uint_as_float(r0[j]);
+        float z = __uint_as_float(r0[j]) * rs;
         if (n + j < N) {
           if (p.scale0 != nullptr) z *= __ldg(p.scale0 + sbase + n + j);
           if (EPI == EPI_GELU_BIAS || EPI == EPI_BIAS) z += __ldg(p.bias + sbase + n + j);
@@ -201,14 +215,15 @@ __device__ __forceinline__ void epilogue_partial(const TcParams& p, const TileIn
   }
 }
 
-template <int EPI>
+template <int EPI, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                            const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
                            TcParams p, int bma, int STAGES) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int A_TILE = bma * BK * 2;
+  constexpr int BK = bk_elems<F8>();
+  const int A_TILE = bma * BK_BYTES;
   const int STAGE_BYTES = A_TILE + B_TILE;
   SmemCtl& s = *reinterpret_cast<SmemCtl*>(ring + STAGES * STAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = lane_id();
@@ -342,9 +357,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a_base = smem_u32(ring + stage * STAGE_BYTES);
           const uint32_t b_base = a_base + A_TILE;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            tc_mma_f16(d_tmem, smem_desc_sw128(a_base + kk * 32), smem_desc_sw128(b_base + kk * 32), kIdesc,
-                       (kb > kb0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BK_BYTES / 32; ++kk) {  // 32 bytes of K per MMA (16 bf16 or 32 E4M3)
+            if (F8)
+              tc_mma_f8(d_tmem, smem_desc_sw128(a_base + kk * 32), smem_desc_sw128(b_base + kk * 32), kIdescE4m3,
+                        (kb > kb0 || kk > 0) ? 1u : 0u);
+            else
+              tc_mma_f16(d_tmem, smem_desc_sw128(a_base + kk * 32), smem_desc_sw128(b_base + kk * 32), kIdescBf16,
+                         (kb > kb0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(&s.empty[stage]);
           if (++stage == STAGES) {
@@ -400,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int EPI>
+template <int EPI, bool F8>
 cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB0, const CUtensorMap& mB1,
                        const TcParams& p, int grid, int bma, int stages, size_t smem, int64_t max_group_rows,
                        cudaStream_t stream) {
@@ -409,12 +428,12 @@ cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUte
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64 || !(attr_set & (1ull << dev))) {
-    e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<EPI, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemLimitTc));
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set |= 1ull << dev;
   }
-  grouped_gemm_tc_kernel<EPI><<<grid, kThreads, smem, stream>>>(mA, mA2, mB0, mB1, p, bma, stages);
+  grouped_gemm_tc_kernel<EPI, F8><<<grid, kThreads, smem, stream>>>(mA, mA2, mB0, mB1, p, bma, stages);
   e = cudaGetLastError();
   if (e != cudaSuccess || p.max_ksplit <= 1) return e;
   dim3 fgrid((p.N + 1023) / 1024, static_cast<unsigned>(max_group_rows), p.num_groups);
@@ -429,35 +448,46 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
   // A rows loaded per stage: all 128, or (every group fitting) the largest group rounded up to 16
   int bma = BM;
   if (a.max_group_rows > 0 && a.max_group_rows <= 64) bma = static_cast<int>((a.max_group_rows + 15) & ~int64_t(15));
-  const size_t stage_bytes = static_cast<size_t>(bma) * BK * 2 + B_TILE;
+  const size_t stage_bytes = static_cast<size_t>(bma) * BK_BYTES + B_TILE;
+  const int eb = a.fp8 ? 1 : 2;  // element bytes of A and B
   int stages = static_cast<int>((kSmemLimitTc - kCtlBytes) / stage_bytes);
   if (stages > MAX_STAGES) stages = MAX_STAGES;
   const size_t smem = stages * stage_bytes + kCtlBytes;
   CUtensorMap mA, mA2, mB0, mB1;
-  if (!make_map(&mA, a.a, a.a_rows, a.K, bma)) return cudaErrorInvalidValue;
+  if (!make_map(&mA, a.a, a.a_rows, a.K, bma, eb)) return cudaErrorInvalidValue;
   if (a.a_shared != nullptr) {
-    if (!make_map(&mA2, a.a_shared, a.a_shared_rows, a.K, bma)) return cudaErrorInvalidValue;
+    if (!make_map(&mA2, a.a_shared, a.a_shared_rows, a.K, bma, eb)) return cudaErrorInvalidValue;
   } else {
     mA2 = mA;
   }
-  if (!make_map(&mB0, a.b0, a.b_rows, a.K)) return cudaErrorInvalidValue;
+  if (!make_map(&mB0, a.b0, a.b_rows, a.K, 128, eb)) return cudaErrorInvalidValue;
   if (a.epilogue == EPI_SWIGLU) {
-    if (!make_map(&mB1, a.b1, a.b_rows, a.K)) return cudaErrorInvalidValue;
+    if (!make_map(&mB1, a.b1, a.b_rows, a.K, 128, eb)) return cudaErrorInvalidValue;
   } else {
     mB1 = mB0;
   }
   // upper bound of the tile count: every group may add one partial m-block
   const int64_t bound = (a.max_total_rows / BM + a.num_groups) * static_cast<int64_t>(p.n_tiles);
   const int grid = static_cast<int>(bound < num_sms ? (bound > 0 ? bound : 1) : num_sms);
+  if (a.fp8) {  // W8A8 runs SwiGLU experts only
+    switch (a.epilogue) {
+      case EPI_SWIGLU:
+        return launch_epi<EPI_SWIGLU, true>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows, stream);
+      case EPI_NONE:
+        return launch_epi<EPI_NONE, true>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (a.epilogue) {
     case EPI_SWIGLU:
-      return launch_epi<EPI_SWIGLU>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows, stream);
+      return launch_epi<EPI_SWIGLU, false>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows, stream);
     case EPI_GELU_BIAS:
-      return launch_epi<EPI_GELU_BIAS>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows, stream);
+      return launch_epi<EPI_GELU_BIAS, false>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows,
+                                              stream);
     case EPI_BIAS:
-      return launch_epi<EPI_BIAS>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows, stream);
+      return launch_epi<EPI_BIAS, false>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows, stream);
     case EPI_NONE:
-      return launch_epi<EPI_NONE>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows, stream);
+      return launch_epi<EPI_NONE, false>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -93,6 +93,9 @@ struct GemmArgs {
   float* partial;           // split-K partial sums (nullptr = no split-K)
   int64_t partial_bytes;    // size of `partial`
   int* ksplit_out;          // device int: the split the GEMM chose
+  int fp8;                  // 1: A and B are E4M3 (kind::f8f6f4); A rows scaled by row_scale
+  const float* row_scale;        // [a rows] per-row scale of A (fp8 only)
+  const float* row_scale_shared; // [S] per-row scale of the shared expert's A rows (fp8 only)
   StatusBlock* status;
 };
 cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t stream);
@@ -106,6 +109,20 @@ cudaError_t launch_grouped_gemm_f32(const GemmArgs& a, cudaStream_t stream);
 
 // FP8-E4M3 weight slabs -> bf16 (exact)
 cudaError_t launch_dequant_e4m3(const uint8_t* q, void* out_bf16, int64_t n, cudaStream_t stream);
+
+// --- E4M3 activations (W8A8) -------------------------------------------------
+// Per-row quantisation of bf16 rows: s = amax / 448 (1 for an all-zero row
+// or a row holding a NaN), q = RNE satfinite E4M3 (x / s), both float32
+// divisions.
+cudaError_t launch_quantize_rows(const void* src, uint8_t* dst, float* scale, int64_t rows, int d, cudaStream_t stream);
+// The same for the rows of a group table: rows a_row0 + r (or out_row0 + r
+// with use_out_rows) of src, at most dst_rows; the shared-expert group's
+// rows come from src_shared and go to dst_shared / scale_shared (index r,
+// at most shared_rows).
+cudaError_t launch_quantize_group_rows(const GroupEntry* groups, int num_groups, int use_out_rows, int shared_slab,
+                                       const void* src, uint8_t* dst, float* scale, int64_t dst_rows,
+                                       const void* src_shared, uint8_t* dst_shared, float* scale_shared,
+                                       int64_t shared_rows, int d, int64_t max_group_rows, cudaStream_t stream);
 
 // --- sliding-window load and selection-bias update ---------------------------
 size_t bias_state_bytes(int E, int K, int window);

@@ -72,6 +72,10 @@ class OracleExperts:
 
     def __call__(self, e, rows):
         cfg = self.cfg
+        if cfg.act_quant:
+            codes = [self.inp[n][e].cpu().numpy() for n in ("w_gate", "w_up", "w_down")]
+            return O.expert_swiglu_w8a8(rows, *codes, np64(self.inp["s_gate"][e]), np64(self.inp["s_up"][e]),
+                                        np64(self.inp["s_down"][e]), round_hidden_bf16=True)
         if cfg.activation == syn.GELU:
             return O.expert_gelu(rows, self._slab("w1", e), np64(self.inp["b1"][e]), self._slab("w2", e),
                                  np64(self.inp["b2"][e]))
@@ -147,3 +151,36 @@ def compare_layer(gpu: dict, inp: dict, cfg: syn.LayerConfig, tokens=None, tol=N
 def skewed_logits(rng, S, E, spread=1.5):
     """Random float32 logits with per-expert offsets (uneven loads)."""
     return (rng.normal(size=(S, E)) + spread * rng.normal(size=E)[None, :]).astype(np.float32)
+
+
+def ffn_case(cfg, seed=0):
+    """Route with the oracle, permute with the oracle, run moe_grouped_ffn and
+    compare every written row with the oracle expert on that row."""
+    inp = syn.make_inputs(cfg, "cuda", seed=seed)
+    x, ridx, rw, _ = oracle_routing(inp, cfg)
+    P = O.expert_permutation(ridx, cfg.E, cfg.capacity)
+    R = P["num_rows"]
+    desc = ops.make_desc(**syn.desc_dict(cfg))
+    ws = new_ws(desc)
+    tor = P["token_of_row"]
+    used = np.nonzero(tor >= 0)[0]
+    xp = torch.zeros((R, cfg.d), dtype=inp["x"].dtype, device="cuda")
+    xp[torch.tensor(used, device="cuda")] = inp["x"][torch.tensor(tor[used], device="cuda", dtype=torch.long)]
+    offs = P["offsets"] if not cfg.capacity else np.concatenate([P["offsets"], P["ovf_offsets"]])
+    Rt = R + cfg.num_shared * cfg.S
+    yp = torch.zeros((Rt, cfg.d), dtype=inp["x"].dtype, device="cuda")
+    ops.moe_grouped_ffn(desc, ops.make_weights(inp), xp, torch.tensor(offs, dtype=torch.int32, device="cuda"),
+                        inp["x"], yp, ws)
+    torch.cuda.synchronize()
+    assert_status_clean(ws)
+    fn = OracleExperts(inp, cfg)
+    ref = np.zeros((Rt, cfg.d))
+    flat = ridx.reshape(-1)
+    for e in range(cfg.E):
+        rows = P["row_of_slot"][flat == e]
+        if len(rows):
+            ref[rows] = fn(e, x[tor[rows]])
+    if cfg.num_shared:
+        ref[R:] = fn(cfg.E, x)
+    rows_all = np.concatenate([used, np.arange(R, Rt)])
+    return np64(yp)[rows_all], ref[rows_all]

@@ -23,7 +23,7 @@ def built_library():
 def header_functions():
     text = open(os.path.join(ROOT, "include", "moe.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_exports_every_declared_symbol():
@@ -43,7 +43,8 @@ def test_strerror():
 
 
 def _desc(name, **over):
-    return ops.make_desc(**dict(syn.desc_dict(syn.CONFIGS[name]), **over))
+    cfg = syn.CONFIGS[name] if name in syn.CONFIGS else syn.VARIANTS[name]
+    return ops.make_desc(**dict(syn.desc_dict(cfg), **over))
 
 
 @pytest.mark.parametrize("name", list(syn.CONFIGS))
@@ -72,7 +73,7 @@ BAD = [
     dict(top_k=0), dict(top_k=9), dict(num_experts=0), dict(num_experts=300), dict(d_model=100),
     dict(d_ff=0), dict(score_fn=5), dict(num_groups=3), dict(num_groups=2, topk_groups=3),
     dict(num_groups=4, topk_groups=1, top_k=3), dict(num_shared=2), dict(capacity=-1), dict(num_tokens=-1),
-    dict(renormalize=2), dict(activation=7), dict(act_dtype=5),
+    dict(renormalize=2), dict(activation=7), dict(act_dtype=5), dict(act_quant=2), dict(act_quant=-1),
 ]
 
 
@@ -84,7 +85,10 @@ def test_invalid_desc_rejected(over):
 
 
 @pytest.mark.parametrize("over", [dict(act_dtype=0), dict(weight_dtype=0),
-                                  dict(weight_dtype=2, activation=0)])
+                                  dict(weight_dtype=2, activation=0),
+                                  dict(act_quant=1),                                  # W8A8 needs E4M3 weights
+                                  dict(act_quant=1, weight_dtype=2, d_model=4104),    # d not a multiple of 16
+                                  dict(act_quant=1, weight_dtype=2, d_ff=14344)])     # h not a multiple of 16
 def test_unsupported_combination(over):
     d = _desc("mixtral_prefill", **over)
     n = ctypes.c_size_t(0)
@@ -160,3 +164,33 @@ def test_bias_state_size_and_argument_errors():
     assert L.moe_update_sel_bias(ctypes.byref(d), p, 1000, float("nan"), st, n, p, None,
                                  None) == ops.MOE_ERR_INVALID_ARG
     assert L.moe_bias_state_init(None, 0, None) == ops.MOE_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("name", list(syn.VARIANTS))
+def test_w8a8_workspace_holds_codes_and_scales(name):
+    """W8A8 replaces the bf16 weight copy with the 8-bit activation rows."""
+    cfg = syn.VARIANTS[name]
+    d8 = _desc(name)
+    d16 = ops.make_desc(**dict(syn.desc_dict(cfg), act_quant=0))
+    R = ops.moe_routed_rows(d8)
+    Rt = R + cfg.num_shared * cfg.S
+    n8, n16 = ops.moe_workspace_size(d8), ops.moe_workspace_size(d16)
+    wdeq = (cfg.E + cfg.num_shared) * 3 * cfg.h * cfg.d * 2
+    codes = R * cfg.d + Rt * cfg.h + (R + Rt) * 4
+    assert n8 >= codes
+    assert n8 - (n16 - wdeq) >= codes
+
+
+def test_quantize_rows_argument_errors():
+    L = ops.lib()
+    p = ctypes.c_void_p(0x1000)
+    assert L.moe_quantize_rows_e4m3(p, 0, 32, p, p, None) == ops.MOE_OK       # nothing to do
+    assert L.moe_quantize_rows_e4m3(p, -1, 32, p, p, None) == ops.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_rows_e4m3(p, 4, 24, p, p, None) == ops.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_rows_e4m3(p, 4, 0, p, p, None) == ops.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_rows_e4m3(None, 4, 32, p, p, None) == ops.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_rows_e4m3(p, 4, 32, None, p, None) == ops.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_rows_e4m3(p, 4, 32, p, None, None) == ops.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_rows_e4m3(ctypes.c_void_p(0x1008), 4, 32, p, p, None) == ops.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_rows_e4m3(p, 4, 32, ctypes.c_void_p(0x1004), p, None) == ops.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_rows_e4m3(p, 4, 32, p, ctypes.c_void_p(0x1002), None) == ops.MOE_ERR_INVALID_ARG

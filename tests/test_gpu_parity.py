@@ -17,7 +17,7 @@ from mixture_experts_layer_bias_b200 import synthetic as syn
 from oracle import moe_oracle as O
 
 from parity import (BF16_REL_L2, F32_MAXABS_REL, FP8_REL_L2, OracleExperts, assert_status_clean, compare_layer,
-                    max_abs_rel, new_ws, np64, rel_l2, run_layer, skewed_logits)
+                    ffn_case, max_abs_rel, new_ws, np64, rel_l2, run_layer, skewed_logits)
 
 pytestmark = pytest.mark.gpu
 
@@ -248,38 +248,7 @@ def test_combine(dt, shared, K, S):
 # ----------------------------------------------------------------------------
 
 
-def _ffn_case(cfg, seed=0):
-    """Route with the oracle, permute with the oracle, run moe_grouped_ffn and
-    compare every written row with the oracle expert on that row."""
-    inp = syn.make_inputs(cfg, "cuda", seed=seed)
-    from parity import oracle_routing
-    x, ridx, rw, _ = oracle_routing(inp, cfg)
-    P = O.expert_permutation(ridx, cfg.E, cfg.capacity)
-    R = P["num_rows"]
-    desc = ops.make_desc(**syn.desc_dict(cfg))
-    ws = new_ws(desc)
-    tor = P["token_of_row"]
-    used = np.nonzero(tor >= 0)[0]
-    xp = torch.zeros((R, cfg.d), dtype=inp["x"].dtype, device="cuda")
-    xp[torch.tensor(used, device="cuda")] = inp["x"][torch.tensor(tor[used], device="cuda", dtype=torch.long)]
-    offs = P["offsets"] if not cfg.capacity else np.concatenate([P["offsets"], P["ovf_offsets"]])
-    Rt = R + cfg.num_shared * cfg.S
-    yp = torch.zeros((Rt, cfg.d), dtype=inp["x"].dtype, device="cuda")
-    ops.moe_grouped_ffn(desc, ops.make_weights(inp), xp, torch.tensor(offs, dtype=torch.int32, device="cuda"),
-                        inp["x"], yp, ws)
-    torch.cuda.synchronize()
-    assert_status_clean(ws)
-    fn = OracleExperts(inp, cfg)
-    ref = np.zeros((Rt, cfg.d))
-    flat = ridx.reshape(-1)
-    for e in range(cfg.E):
-        rows = P["row_of_slot"][flat == e]
-        if len(rows):
-            ref[rows] = fn(e, x[tor[rows]])
-    if cfg.num_shared:
-        ref[R:] = fn(cfg.E, x)
-    rows_all = np.concatenate([used, np.arange(R, Rt)])
-    return np64(yp)[rows_all], ref[rows_all]
+_ffn_case = ffn_case
 
 
 def test_grouped_ffn_f32_tiny():
