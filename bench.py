@@ -311,7 +311,7 @@ def cpu_baseline(cfg, inp, n_tokens=32):
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    name = WORKLOAD if args.workload == "profile_small" else args.workload
+    name = WORKLOAD if args.workload.startswith("profile_small") else args.workload
     cfg = syn.CONFIGS.get(name) or syn.VARIANTS[name]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = make_layer_inputs(cfg, dev)
@@ -350,7 +350,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=sorted(syn.CONFIGS) + sorted(syn.VARIANTS) + ["profile_small"],
+                    choices=sorted(syn.CONFIGS) + sorted(syn.VARIANTS) + ["profile_small", "profile_small_w8a8"],
                     help="profile_small: S=2048, d=4096, h=4096 (same kernels, ~1 GB) for ncu captures")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -371,6 +371,8 @@ def main():
     peaks = load_peaks()
     if args.workload == "profile_small":
         cfg = syn.scaled(syn.CONFIGS[WORKLOAD], S=2048, h=4096)
+    elif args.workload == "profile_small_w8a8":
+        cfg = syn.scaled(syn.VARIANTS["mixtral_prefill_w8a8"], S=2048, h=4096)
     else:
         cfg = syn.CONFIGS.get(args.workload) or syn.VARIANTS[args.workload]
     S = cfg.S

@@ -506,3 +506,27 @@ def test_w8a8_expert_close_to_exact_expert():
                            s_gate=sg, s_up=su, s_down=sd)
     rel = np.linalg.norm(y8 - yref) / np.linalg.norm(yref)
     assert 1e-4 < rel < 5e-2
+
+
+def test_w8a8_expert_exact_on_representable_rows():
+    """With x rows that are E4M3 codes times a power of two (the row maximum
+    coding to 448) the activation quantisation is lossless, and with d_ff = 1
+    each hidden row has one element, which quantises to +-448 times |h|/448,
+    i.e. back to h up to one float32 rounding.  So the W8A8 expert must equal
+    the plain SwiGLU expert on the dequantised weights; a wrong activation or
+    hidden scale, or swapped weight scales, breaks the equality."""
+    rng = np.random.default_rng(15)
+    d, n = 32, 12
+    codes = rng.integers(0, 0x7F, size=(n, d)).astype(np.uint8) | (rng.integers(0, 2, size=(n, d)) << 7).astype(
+        np.uint8)
+    codes[:, 0] = 0x7E  # 448: the row maximum
+    x = O.e4m3_bits_to_f64(codes) * (2.0 ** rng.integers(-12, 4, size=(n, 1)))
+    wg, wu, wd = rng.normal(size=(1, d)) / 4, rng.normal(size=(1, d)) / 4, rng.normal(size=(d, 1))
+    qg, sg = O.quantize_rows_e4m3(wg.astype(np.float32))
+    qu, su = O.quantize_rows_e4m3(wu.astype(np.float32))
+    qd, sd = O.quantize_rows_e4m3(wd.astype(np.float32))
+    su = su * 3.0  # distinct gate and up scales, so that swapping them shows
+    y8 = O.expert_swiglu_w8a8(x, qg, qu, qd, sg, su, sd, round_hidden_bf16=False)
+    yref = O.expert_swiglu(x, O.e4m3_bits_to_f64(qg), O.e4m3_bits_to_f64(qu), O.e4m3_bits_to_f64(qd),
+                           s_gate=sg, s_up=su, s_down=sd)
+    np.testing.assert_allclose(y8, yref, rtol=1e-6, atol=1e-12 * np.abs(yref).max())
