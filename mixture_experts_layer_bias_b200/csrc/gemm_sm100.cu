@@ -129,16 +129,29 @@ __device__ __forceinline__ UnitInfo decode_unit(const SmemCtl& s, const TcParams
   return ui;
 }
 
+// Epilogue of one 32-row quarter of a tile: thread `lane` owns accumulator
+// row `row` (and its activation row scale rs).  The per-column operands
+// (weight-channel scales, biases) are loaded once per 32-column chunk, lane j
+// holding column n + j, and handed to every lane by shuffles; SiLU uses the
+// fast reciprocal-based division.
 template <int EPI>
 __device__ __forceinline__ void epilogue_store(const TcParams& p, const TileInfo& ti, uint32_t tbase, int row,
-                                               bool valid) {
+                                               bool valid, int lane) {
   const int N = p.N;
   const int64_t orow = static_cast<int64_t>(ti.grp.out_row0) + row;
   const int64_t sbase = static_cast<int64_t>(ti.grp.expert) * N;
   const float rs = valid ? a_row_scale(p, ti.grp, row) : 1.0f;
   constexpr int kChunks = (EPI == EPI_SWIGLU) ? 4 : 8;
+  constexpr bool kBias = EPI == EPI_GELU_BIAS || EPI == EPI_BIAS;
   for (int c = 0; c < kChunks; ++c) {
     const int n = ti.n_idx * p.bn_out + c * 32;
+    const bool col_ok = n + lane < N;
+    float cs0 = 1.0f, cs1 = 1.0f, cb = 0.0f;  // this lane's column: channel scales, bias
+    if (col_ok) {
+      if (p.scale0 != nullptr) cs0 = __ldg(p.scale0 + sbase + n + lane);
+      if (EPI == EPI_SWIGLU && p.scale1 != nullptr) cs1 = __ldg(p.scale1 + sbase + n + lane);
+      if (kBias) cb = __ldg(p.bias + sbase + n + lane);
+    }
     uint32_t r0[32];
     float v[32];
     if (EPI == EPI_SWIGLU) {
@@ -148,24 +161,17 @@ __device__ __forceinline__ void epilogue_store(const TcParams& p, const TileInfo
       tmem_ld_wait();
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        float g = __uint_as_float(r0[j]) * rs;
-        float u = __uint_as_float(r1[j]) * rs;
-        if (p.scale0 != nullptr && n + j < N) {
-          g *= __ldg(p.scale0 + sbase + n + j);
-          u *= __ldg(p.scale1 + sbase + n + j);
-        }
-        v[j] = g / (1.0f + __expf(-g)) * u;
+        const float g = __uint_as_float(r0[j]) * rs * __shfl_sync(0xFFFFFFFFu, cs0, j);
+        const float u = __uint_as_float(r1[j]) * rs * __shfl_sync(0xFFFFFFFFu, cs1, j);
+        v[j] = __fdividef(g, 1.0f + __expf(-g)) * u;
       }
     } else {
       tmem_ld_32x32b_x32(tbase + c * 32, r0);
       tmem_ld_wait();
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        float z = __uint_as_float(r0[j]) * rs;
-        if (n + j < N) {
-          if (p.scale0 != nullptr) z *= __ldg(p.scale0 + sbase + n + j);
-          if (EPI == EPI_GELU_BIAS || EPI == EPI_BIAS) z += __ldg(p.bias + sbase + n + j);
-        }
+        float z = __uint_as_float(r0[j]) * rs * __shfl_sync(0xFFFFFFFFu, cs0, j);
+        if (kBias) z += __shfl_sync(0xFFFFFFFFu, cb, j);
         if (EPI == EPI_GELU_BIAS) z = 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
         v[j] = z;
       }
@@ -405,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ks > 1)
         epilogue_partial<EPI>(p, ti, tbase, row, valid, ui.split);
       else
-        epilogue_store<EPI>(p, ti, tbase, row, valid);
+        epilogue_store<EPI>(p, ti, tbase, row, valid, lane);
       tc_fence_before();
       mbar_arrive(&s.tempty[acc]);
     }
