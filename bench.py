@@ -98,8 +98,6 @@ def kernels_per_step(cfg):
         n += 2                             # per-row E4M3 quantisation of each GEMM's A rows
     elif cfg.weight_dtype == syn.E4M3:
         n += 3                             # E4M3 -> bf16 decode of the three stacks
-    if cfg.capacity:
-        n += 4 if cfg.act_quant else 2     # overflow pass (with its two quantisations)
     n += 1                                 # combine
     return n
 

@@ -89,8 +89,9 @@ typedef enum { MOE_ACT_GELU = 0, MOE_ACT_SWIGLU = 1 } moe_act;
  *   weight_dtype: dtype of the expert weights (F32, BF16 or E4M3; E4M3
  *     needs the per-output-channel scales s_gate, s_up, s_down).
  *   capacity: 0 = unbounded; C > 0 = at most C rows per expert in the
- *     primary block, the rest in an overflow region processed in a second
- *     pass (ybb.press 2.2, overflow buffering).  No token is dropped.
+ *     primary block, the rest in an overflow region (ybb.press 2.2,
+ *     overflow buffering) whose rows the expert GEMMs process right after
+ *     that expert's primary rows.  No token is dropped.
  *   act_quant: 0 = the expert GEMMs read bf16 activations (E4M3 weights are
  *     decoded to bf16 first); 1 = W8A8: each A row of both expert GEMMs
  *     (the permuted tokens, then the bf16 hidden rows) is quantised to E4M3

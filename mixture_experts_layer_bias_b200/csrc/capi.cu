@@ -20,7 +20,7 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 
 struct Layout {
-  size_t status, logits, chunk_hist, groups1, groups2, counts, offsets, topk_idx, topk_w, row_of_slot, token_of_row,
+  size_t status, logits, chunk_hist, groups, counts, offsets, topk_idx, topk_w, row_of_slot, token_of_row,
       x_perm, hidden, y_perm, wdeq, ksplit, partial, partial_bytes, qa, sa, qas, sas, qh, sh, total;
 };
 
@@ -53,8 +53,7 @@ Layout make_layout(const moe_desc& d) {
   L.status = take(kAlign);
   L.logits = take(E > 32 ? static_cast<size_t>(S * E) * 4 : 0);
   L.chunk_hist = take(static_cast<size_t>(nch * E) * 4);
-  L.groups1 = take(static_cast<size_t>(E + 1) * sizeof(GroupEntry));
-  L.groups2 = take(static_cast<size_t>(E) * sizeof(GroupEntry));
+  L.groups = take(static_cast<size_t>(2 * E + 1) * sizeof(GroupEntry));
   L.counts = take(static_cast<size_t>(E) * 4);
   L.offsets = take(static_cast<size_t>(2 * (E + 1)) * 4);
   L.topk_idx = take(static_cast<size_t>(S * K) * 4);
@@ -200,8 +199,7 @@ moe_status permute_impl(const moe_desc& d, const void* x, const int32_t* topk_id
   a.num_rows = routed_rows(d);
   a.status = at<StatusBlock>(ws, L.status);
   if (write_groups) {
-    a.g1 = at<GroupEntry>(ws, L.groups1);
-    a.g2 = at<GroupEntry>(ws, L.groups2);
+    a.g1 = at<GroupEntry>(ws, L.groups);
     a.num_shared = d.num_shared;
   }
   return cuda_status(launch_permute(a, st));
@@ -215,11 +213,10 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
   const int64_t R = routed_rows(d);
   const int64_t Rt = R + static_cast<int64_t>(d.num_shared) * S;
   StatusBlock* status = at<StatusBlock>(ws, L.status);
-  GroupEntry* g1 = at<GroupEntry>(ws, L.groups1);
-  GroupEntry* g2 = at<GroupEntry>(ws, L.groups2);
+  GroupEntry* g1 = at<GroupEntry>(ws, L.groups);
   cudaError_t err = cudaSuccess;
   if (!groups_ready) {
-    err = launch_build_groups(S, E, d.top_k, d.capacity, d.num_shared, offsets, g1, g2, status, st);
+    err = launch_build_groups(S, E, d.top_k, d.capacity, d.num_shared, offsets, g1, status, st);
     if (err != cudaSuccess) return MOE_ERR_CUDA;
   }
   const int slabs = E + d.num_shared;
@@ -227,7 +224,8 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
 
   GemmArgs up{};
   up.groups = g1;
-  up.num_groups = E + d.num_shared;
+  // with a capacity the overflow groups sit right behind each expert's primary group
+  up.num_groups = (d.capacity > 0 ? 2 * E : E) + d.num_shared;
   up.shared_slab = d.num_shared ? E : -1;
   up.a_rows_from_out = 0;
   up.a = x_perm;
@@ -337,21 +335,6 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
   if ((err = run(up)) != cudaSuccess) return MOE_ERR_CUDA;
   if (w8a8 && (err = quant_down(down)) != cudaSuccess) return MOE_ERR_CUDA;
   if ((err = run(down)) != cudaSuccess) return MOE_ERR_CUDA;
-  if (d.capacity > 0) {
-    // second pass: the overflow rows, grouped by expert the same way
-    GemmArgs up2 = up, down2 = down;
-    up2.groups = down2.groups = g2;
-    up2.num_groups = down2.num_groups = E;
-    up2.shared_slab = -1;
-    up2.a_shared = nullptr;
-    up2.a_shared_rows = 0;
-    up2.row_scale_shared = nullptr;
-    up2.max_total_rows = down2.max_total_rows = static_cast<int64_t>(S) * d.top_k;
-    if (w8a8 && (err = quant_up(up2)) != cudaSuccess) return MOE_ERR_CUDA;
-    if ((err = run(up2)) != cudaSuccess) return MOE_ERR_CUDA;
-    if (w8a8 && (err = quant_down(down2)) != cudaSuccess) return MOE_ERR_CUDA;
-    if ((err = run(down2)) != cudaSuccess) return MOE_ERR_CUDA;
-  }
   return MOE_OK;
 }
 

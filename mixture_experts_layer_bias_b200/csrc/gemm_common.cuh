@@ -11,7 +11,7 @@
 namespace moe {
 namespace gemm {
 
-constexpr int kMaxGroups = 264;
+constexpr int kMaxGroups = 520;  // 2 x 256 experts (primary + overflow) + shared
 
 struct TcParams {
   const GroupEntry* groups;  // nullptr: one group of `single_rows` rows, slab 0

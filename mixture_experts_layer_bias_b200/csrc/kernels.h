@@ -49,20 +49,19 @@ struct PermuteArgs {
   void* x_perm;              // [R][d] or nullptr
   int64_t num_rows;          // R
   StatusBlock* status;
-  // optional: also write the GEMM group tables (see GroupEntry)
+  // optional: also write the GEMM group table (see GroupEntry)
   GroupEntry* g1;
-  GroupEntry* g2;
   int num_shared;
 };
 int permute_num_chunks(int S, int K);
 int permute_tokens_per_chunk(int K);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream);
 
-// Build the pass tables from offsets: pass 1 = routed groups (primary block
-// with capacity) + the shared expert, pass 2 = overflow groups (capacity only).
-// g1 has E + ns entries, g2 has E entries.
+// Build the group table from offsets: E routed groups, or with a capacity
+// 2E (expert e's primary group at 2e, its overflow group at 2e + 1), then
+// the shared expert; E + ns or 2E + ns entries.
 cudaError_t launch_build_groups(int S, int E, int K, int capacity, int num_shared, const int32_t* offsets,
-                                GroupEntry* g1, GroupEntry* g2, StatusBlock* status, cudaStream_t stream);
+                                GroupEntry* g1, StatusBlock* status, cudaStream_t stream);
 
 // --- grouped expert GEMMs ----------------------------------------------------
 enum Epilogue { EPI_SWIGLU = 0, EPI_GELU_BIAS = 1, EPI_BIAS = 2, EPI_NONE = 3 };

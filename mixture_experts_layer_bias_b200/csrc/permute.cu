@@ -217,10 +217,13 @@ __global__ void __launch_bounds__(kPermWarps * 32)
   }
 }
 
-// Group tables of the grouped GEMMs from the offsets (pass 1: routed or
-// primary groups + shared expert; pass 2: overflow groups).
+// Group table of the grouped GEMMs from the offsets: one group per expert
+// (rows offsets[e] ..), or with a capacity two per expert, its primary rows
+// (e*C ..) then its overflow rows (E*C + overflow offset ..), so that the
+// overflow pass runs in the same launches right behind the expert's primary
+// tiles while its weight tiles are still in L2; the shared expert last.
 __device__ __forceinline__ void write_groups(int S, int E, int K, int capacity, int num_shared,
-                                             const int32_t* offsets, GroupEntry* g1, GroupEntry* g2) {
+                                             const int32_t* offsets, GroupEntry* g1) {
   const int64_t R = capacity > 0 ? static_cast<int64_t>(E) * capacity + static_cast<int64_t>(S) * K
                                  : static_cast<int64_t>(S) * K;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -229,12 +232,13 @@ __device__ __forceinline__ void write_groups(int S, int E, int K, int capacity, 
       g1[e] = GroupEntry{offsets[e], offsets[e], cnt, e};
     } else {
       const int prim = min(cnt, capacity);
-      g1[e] = GroupEntry{e * capacity, e * capacity, prim, e};
+      g1[2 * e] = GroupEntry{e * capacity, e * capacity, prim, e};
       const int orow = E * capacity + offsets[E + 1 + e];
-      g2[e] = GroupEntry{orow, orow, cnt - prim, e};
+      g1[2 * e + 1] = GroupEntry{orow, orow, cnt - prim, e};
     }
   }
-  if (threadIdx.x == 0 && num_shared > 0) g1[E] = GroupEntry{0, static_cast<int32_t>(R), S, E};
+  const int gs = capacity > 0 ? 2 * E : E;
+  if (threadIdx.x == 0 && num_shared > 0) g1[gs] = GroupEntry{0, static_cast<int32_t>(R), S, E};
 }
 
 constexpr int kSmallWarps = 32;
@@ -247,7 +251,7 @@ __global__ void __launch_bounds__(kSmallWarps * 32)
     permute_small_kernel(int S, int E, int K, int capacity, int num_shared, const int32_t* __restrict__ topk_idx,
                          int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                          int32_t* __restrict__ row_of_slot, int32_t* __restrict__ token_of_row, int64_t num_rows,
-                         GroupEntry* __restrict__ g1, GroupEntry* __restrict__ g2, StatusBlock* status) {
+                         GroupEntry* __restrict__ g1, StatusBlock* status) {
   extern __shared__ int32_t sm[];
   int32_t* whist = sm;                      // [32][E]
   int32_t* cnt = sm + kSmallWarps * E;      // [E]
@@ -326,7 +330,7 @@ __global__ void __launch_bounds__(kSmallWarps * 32)
     }
     __syncwarp();
   }
-  if (g1 != nullptr) write_groups(S, E, K, capacity, num_shared, offs_s, g1, g2);
+  if (g1 != nullptr) write_groups(S, E, K, capacity, num_shared, offs_s, g1);
 }
 
 // Row gather for small batches: one CTA per token, its threads split the row.
@@ -349,9 +353,8 @@ __global__ void __launch_bounds__(256)
 }
 
 __global__ void build_groups_kernel(int S, int E, int K, int capacity, int num_shared,
-                                    const int32_t* __restrict__ offsets, GroupEntry* __restrict__ g1,
-                                    GroupEntry* __restrict__ g2) {
-  write_groups(S, E, K, capacity, num_shared, offsets, g1, g2);
+                                    const int32_t* __restrict__ offsets, GroupEntry* __restrict__ g1) {
+  write_groups(S, E, K, capacity, num_shared, offsets, g1);
 }
 
 }  // namespace
@@ -377,7 +380,7 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
     const size_t smem = sizeof(int32_t) * (kSmallWarps * a.E + 3 * a.E + 1);
     permute_small_kernel<<<1, kSmallWarps * 32, smem, stream>>>(a.S, a.E, a.K, a.capacity, a.num_shared, a.topk_idx,
                                                                  a.counts, a.offsets, a.row_of_slot, a.token_of_row,
-                                                                 a.num_rows, a.g1, a.g2, a.status);
+                                                                 a.num_rows, a.g1, a.status);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   } else {
     const int tpc = permute_tokens_per_chunk(a.K);
@@ -400,7 +403,7 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
                                                             a.chunk_hist, a.offsets, a.row_of_slot, a.token_of_row);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     if (a.g1 != nullptr) {
-      build_groups_kernel<<<1, 256, 0, stream>>>(a.S, a.E, a.K, a.capacity, a.num_shared, a.offsets, a.g1, a.g2);
+      build_groups_kernel<<<1, 256, 0, stream>>>(a.S, a.E, a.K, a.capacity, a.num_shared, a.offsets, a.g1);
       if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
   }
@@ -427,9 +430,9 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_build_groups(int S, int E, int K, int capacity, int num_shared, const int32_t* offsets,
-                                GroupEntry* g1, GroupEntry* g2, StatusBlock* status, cudaStream_t stream) {
+                                GroupEntry* g1, StatusBlock* status, cudaStream_t stream) {
   (void)status;
-  build_groups_kernel<<<1, 256, 0, stream>>>(S, E, K, capacity, num_shared, offsets, g1, g2);
+  build_groups_kernel<<<1, 256, 0, stream>>>(S, E, K, capacity, num_shared, offsets, g1);
   return cudaGetLastError();
 }
 

@@ -262,6 +262,7 @@ def test_grouped_ffn_f32_tiny():
     (1, 512, 256, 8, 2, {}),              # a single token
     (513, 384, 256, 16, 4, {"num_shared": 1}),
     (700, 256, 128, 64, 8, {"capacity": -1}),
+    (600, 256, 128, 256, 8, {"capacity": -1, "num_shared": 1}),  # 2 x 256 + 1 groups in one launch
 ])
 def test_grouped_ffn_bf16_swiglu(S, d, h, E, K, extra):
     extra = dict(extra)
