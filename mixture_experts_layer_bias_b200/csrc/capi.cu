@@ -205,8 +205,10 @@ moe_status permute_impl(const moe_desc& d, const void* x, const int32_t* topk_id
   return cuda_status(launch_permute(a, st));
 }
 
+// a_quantized (W8A8): the up projection's E4M3 rows and scales are already in
+// the workspace (written by the quantising gather), x_perm is not read.
 moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm, const int32_t* offsets, const void* x,
-                    void* y_perm, void* ws, cudaStream_t st, bool groups_ready = false) {
+                    void* y_perm, void* ws, cudaStream_t st, bool groups_ready = false, bool a_quantized = false) {
   const Layout L = make_layout(d);
   const int S = d.num_tokens, E = d.num_experts, h = d.d_ff, dm = d.d_model;
   if (S == 0) return MOE_OK;
@@ -331,7 +333,7 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
                                       at<float>(ws, L.sh), Rt, nullptr, nullptr, nullptr, 0, h, g.max_group_rows, st);
   };
   const bool w8a8 = d.act_quant == 1;
-  if (w8a8 && (err = quant_up(up)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (w8a8 && !a_quantized && (err = quant_up(up)) != cudaSuccess) return MOE_ERR_CUDA;
   if ((err = run(up)) != cudaSuccess) return MOE_ERR_CUDA;
   if (w8a8 && (err = quant_down(down)) != cudaSuccess) return MOE_ERR_CUDA;
   if ((err = run(down)) != cudaSuccess) return MOE_ERR_CUDA;
@@ -472,8 +474,20 @@ moe_status moe_layer_forward(const moe_desc* desc, const moe_weights* w, const v
   void* y_perm = at<void>(ws, L.y_perm);
   if ((s = route_impl(d, w, x, nullptr, idx, gates, ws, st)) != MOE_OK) return s;
   // the permutation also writes the GEMM group tables, so the FFN skips that launch
-  if ((s = permute_impl(d, x, idx, cnt, offs, ros, tor, x_perm, ws, st, true)) != MOE_OK) return s;
-  if ((s = ffn_impl(d, *w, x_perm, offs, x, y_perm, ws, st, true)) != MOE_OK) return s;
+  if (d.act_quant == 1) {
+    // W8A8: the row gather writes E4M3 codes and row scales straight away
+    // (no bf16 copy of the permuted rows)
+    if ((s = permute_impl(d, nullptr, idx, cnt, offs, ros, tor, nullptr, ws, st, true)) != MOE_OK) return s;
+    const bool sh = d.num_shared != 0;
+    if (launch_gather_quantize(d.num_tokens, d.d_model, d.top_k, ros, x, at<uint8_t>(ws, L.qa), at<float>(ws, L.sa),
+                               sh ? at<uint8_t>(ws, L.qas) : nullptr, sh ? at<float>(ws, L.sas) : nullptr,
+                               st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if ((s = ffn_impl(d, *w, x_perm, offs, x, y_perm, ws, st, true, true)) != MOE_OK) return s;
+  } else {
+    if ((s = permute_impl(d, x, idx, cnt, offs, ros, tor, x_perm, ws, st, true)) != MOE_OK) return s;
+    if ((s = ffn_impl(d, *w, x_perm, offs, x, y_perm, ws, st, true)) != MOE_OK) return s;
+  }
   return combine_impl(d, y_perm, ros, gates, y, st);
 }
 

@@ -114,6 +114,11 @@ cudaError_t launch_dequant_e4m3(const uint8_t* q, void* out_bf16, int64_t n, cud
 // or a row holding a NaN), q = RNE satfinite E4M3 (x / s), both float32
 // divisions.
 cudaError_t launch_quantize_rows(const void* src, uint8_t* dst, float* scale, int64_t rows, int d, cudaStream_t stream);
+// The row gather of the permutation fused with that quantisation: token t's
+// codes and scale go to rows row_of_slot[t*K + k] (>= 0) of q_perm / s_perm
+// and, when q_x is given, to row t of q_x / s_x.
+cudaError_t launch_gather_quantize(int S, int d, int K, const int32_t* row_of_slot, const void* x, uint8_t* q_perm,
+                                   float* s_perm, uint8_t* q_x, float* s_x, cudaStream_t stream);
 // The same for the rows of a group table: rows a_row0 + r (or out_row0 + r
 // with use_out_rows) of src, at most dst_rows; the shared-expert group's
 // rows come from src_shared and go to dst_shared / scale_shared (index r,

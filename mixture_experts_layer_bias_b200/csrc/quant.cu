@@ -40,9 +40,8 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& w, float* f) {
   }
 }
 
-// Quantise one row of d bf16 values (d % 8 == 0) with the calling warp.
-__device__ __forceinline__ void quantize_row(const __nv_bfloat16* __restrict__ src, uint8_t* __restrict__ dst,
-                                             float* __restrict__ scale, int d, int lane) {
+// Row scale of d bf16 values (d % 8 == 0), computed by the calling warp.
+__device__ __forceinline__ float row_scale_e4m3(const __nv_bfloat16* __restrict__ src, int d, int lane) {
   float amax = 0.0f;
   bool nan = false;
 #pragma unroll 4
@@ -58,20 +57,55 @@ __device__ __forceinline__ void quantize_row(const __nv_bfloat16* __restrict__ s
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
   nan = __any_sync(0xFFFFFFFFu, nan);
-  const float s = (!nan && amax > 0.0f) ? __fdiv_rn(amax, 448.0f) : 1.0f;
-#pragma unroll 4
-  for (int c = lane * 8; c < d; c += 256) {
-    float f[8];
-    bf16x8_to_f32(ldg16(src + c), f);
-    uint32_t lo = 0, hi = 0;
+  return (!nan && amax > 0.0f) ? __fdiv_rn(amax, 448.0f) : 1.0f;
+}
+
+// E4M3 codes of 8 bf16 values for the row scale s, packed in memory order.
+__device__ __forceinline__ uint2 encode8_e4m3(const uint4& w, float s) {
+  float f[8];
+  bf16x8_to_f32(w, f);
+  uint32_t lo = 0, hi = 0;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      lo |= static_cast<uint32_t>(e4m3_code(__fdiv_rn(f[j], s))) << (8 * j);
-      hi |= static_cast<uint32_t>(e4m3_code(__fdiv_rn(f[4 + j], s))) << (8 * j);
-    }
-    *reinterpret_cast<uint2*>(dst + c) = make_uint2(lo, hi);
+  for (int j = 0; j < 4; ++j) {
+    lo |= static_cast<uint32_t>(e4m3_code(__fdiv_rn(f[j], s))) << (8 * j);
+    hi |= static_cast<uint32_t>(e4m3_code(__fdiv_rn(f[4 + j], s))) << (8 * j);
   }
+  return make_uint2(lo, hi);
+}
+
+// Quantise one row of d bf16 values (d % 8 == 0) with the calling warp.
+__device__ __forceinline__ void quantize_row(const __nv_bfloat16* __restrict__ src, uint8_t* __restrict__ dst,
+                                             float* __restrict__ scale, int d, int lane) {
+  const float s = row_scale_e4m3(src, d, lane);
+#pragma unroll 4
+  for (int c = lane * 8; c < d; c += 256) *reinterpret_cast<uint2*>(dst + c) = encode8_e4m3(ldg16(src + c), s);
   if (lane == 0) *scale = s;
+}
+
+// The permutation's row gather fused with the quantisation: a warp per
+// token computes the token row's scale and codes once and writes them to the
+// token's K rows of the expert-sorted buffer (row_of_slot; -1 = none), and to
+// row t of q_x / s_x when given (the shared expert's operand).
+__global__ void __launch_bounds__(kWarps * 32)
+    gather_quantize_kernel(int S, int d, int K, const int32_t* __restrict__ row_of_slot,
+                           const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ q_perm,
+                           float* __restrict__ s_perm, uint8_t* __restrict__ q_x, float* __restrict__ s_x) {
+  const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (t >= S) return;
+  const int lane = lane_id();
+  const int my_row = lane < K ? __ldg(row_of_slot + static_cast<int64_t>(t) * K + lane) : -1;
+  const __nv_bfloat16* src = x + static_cast<int64_t>(t) * d;
+  const float s = row_scale_e4m3(src, d, lane);
+  for (int c = lane * 8; c < d; c += 256) {
+    const uint2 q = encode8_e4m3(ldg16(src + c), s);
+    for (int k = 0; k < K; ++k) {
+      const int row = __shfl_sync(0xFFFFFFFFu, my_row, k);
+      if (row >= 0) *reinterpret_cast<uint2*>(q_perm + static_cast<int64_t>(row) * d + c) = q;
+    }
+    if (q_x != nullptr) *reinterpret_cast<uint2*>(q_x + static_cast<int64_t>(t) * d + c) = q;
+  }
+  if (my_row >= 0) s_perm[my_row] = s;
+  if (lane == 0 && s_x != nullptr) s_x[t] = s;
 }
 
 // Rows of a group table (groups != nullptr) or `single_rows` contiguous rows.
@@ -111,6 +145,15 @@ cudaError_t launch_quantize_rows(const void* src, uint8_t* dst, float* scale, in
   quantize_rows_kernel<<<dim3(static_cast<unsigned>(blocks)), kWarps * 32, 0, stream>>>(
       nullptr, 0, -1, rows, static_cast<const __nv_bfloat16*>(src), dst, scale, rows, nullptr, nullptr, nullptr, 0,
       d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_quantize(int S, int d, int K, const int32_t* row_of_slot, const void* x, uint8_t* q_perm,
+                                   float* s_perm, uint8_t* q_x, float* s_x, cudaStream_t stream) {
+  if (S <= 0) return cudaSuccess;
+  if (d <= 0 || d % 8 != 0 || K < 1 || K > 32) return cudaErrorInvalidValue;
+  gather_quantize_kernel<<<(S + kWarps - 1) / kWarps, kWarps * 32, 0, stream>>>(
+      S, d, K, row_of_slot, static_cast<const __nv_bfloat16*>(x), q_perm, s_perm, q_x, s_x);
   return cudaGetLastError();
 }
 

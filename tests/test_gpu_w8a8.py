@@ -149,3 +149,38 @@ def test_layer_w8a8_full_size(name):
     del inp, gpu
     gc.collect()
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name,over", [
+    ("fp8_skew_capacity_w8a8", dict(S=1024, d=256, h=384)),
+    ("mixtral_prefill_w8a8", dict(S=300, d=512, h=256, num_shared=1)),
+])
+def test_fused_gather_quantisation_matches_stage_calls(name, over):
+    """moe_layer_forward quantises the token rows inside the row gather; the
+    four stage calls quantise the gathered bf16 rows in moe_grouped_ffn.  Both
+    encode the same rows the same way, so the outputs are bit-identical."""
+    cfg = syn.scaled(syn.VARIANTS[name], **over)
+    inp = syn.make_inputs(cfg, "cuda", seed=6)
+    fused = run_layer(inp, cfg)
+    desc = fused["desc"]
+    w = ops.make_weights(inp)
+    ws = torch.empty(ops.moe_workspace_size(desc), dtype=torch.uint8, device="cuda")
+    ops.moe_workspace_init(ws)
+    S, E, K = cfg.S, cfg.E, cfg.K
+    R = ops.moe_routed_rows(desc)
+    idx = torch.empty((S, K), dtype=torch.int32, device="cuda")
+    gw = torch.empty((S, K), dtype=torch.float32, device="cuda")
+    counts = torch.empty((E,), dtype=torch.int32, device="cuda")
+    offsets = torch.empty((2 * (E + 1),), dtype=torch.int32, device="cuda")
+    ros = torch.empty((S * K,), dtype=torch.int32, device="cuda")
+    tor = torch.empty((R,), dtype=torch.int32, device="cuda")
+    xp = torch.empty((R, cfg.d), dtype=torch.bfloat16, device="cuda")
+    yp = torch.empty((R + cfg.num_shared * S, cfg.d), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((S, cfg.d), dtype=torch.bfloat16, device="cuda")
+    ops.moe_route(desc, w, inp["x"], None, idx, gw, ws)
+    ops.moe_permute(desc, inp["x"], idx, counts, offsets, ros, tor, xp, ws)
+    ops.moe_grouped_ffn(desc, w, xp, offsets, inp["x"], yp, ws)
+    ops.moe_combine(desc, yp, ros, gw, y, ws)
+    torch.cuda.synchronize()
+    assert_status_clean(ws)
+    assert torch.equal(y.view(torch.int16), fused["y"].view(torch.int16))
