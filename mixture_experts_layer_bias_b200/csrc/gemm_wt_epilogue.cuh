@@ -51,7 +51,7 @@ __device__ __forceinline__ void wt_store_chunk(const TcParams& p, const GroupEnt
       const float up = __shfl_xor_sync(0xFFFFFFFFu, mine, 16);
       if (!is_up) {
         const float g = mine * sg;
-        tbuf[j * 16 + lane] = __float2bfloat16_rn(g / (1.0f + __expf(-g)) * (up * su));
+        tbuf[j * 16 + lane] = __float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * (up * su));
       }
     }
     __syncwarp();
