@@ -102,6 +102,8 @@ def kernels_per_step(cfg):
         n += 1                             # per-row E4M3 quantisation of the hidden rows
     elif cfg.weight_dtype == syn.E4M3:
         n += 3                             # E4M3 -> bf16 decode of the three stacks
+    if cfg.reroute:
+        n += 3 + 2                         # ranks (count, scan, scatter), re-route assignment and gates
     n += 1                                 # combine
     return n
 
@@ -196,6 +198,11 @@ def time_stages(cfg, inp, desc, ws, bufs, steps, warmup):
         ops.moe_route(desc, w, x, None, bufs["idx"], bufs["gw"], ws)
         if ev is not None:
             ev[1].record(st)
+        if cfg.reroute:
+            # capacity ranks of the first choices, then over-capacity re-routing
+            ops.moe_permute(desc, None, bufs["idx"], bufs["counts"], bufs["offsets"], bufs["ros"], bufs["tor"],
+                            None, ws)
+            ops.moe_reroute(desc, bufs["idx"], bufs["gw"], bufs["counts"], bufs["ros"], ws)
         ops.moe_permute(desc, x, bufs["idx"], bufs["counts"], bufs["offsets"], bufs["ros"], bufs["tor"],
                         bufs["xp"], ws)
         if ev is not None:

@@ -65,6 +65,7 @@ typedef enum { MOE_ACT_GELU = 0, MOE_ACT_SWIGLU = 1 } moe_act;
 #define MOE_CNT_BAD_ID 1      /* slots with an out-of-range expert id */
 #define MOE_CNT_TIMEOUT 2     /* CTAs that gave up a wait */
 #define MOE_CNT_OVERFLOW_ROWS 3 /* rows routed to the overflow region */
+#define MOE_CNT_REROUTED 4    /* slots moved by over-capacity re-routing */
 #define MOE_NUM_COUNTERS 8
 
 /*
@@ -100,6 +101,15 @@ typedef enum { MOE_ACT_GELU = 0, MOE_ACT_SWIGLU = 1 } moe_act;
  *     pages list E4M3 only as a storage format (ybb.press 3.3); per-row
  *     activation scaling is this library's reading.  Needs BF16 act, E4M3
  *     weights, SWIGLU, d and h multiples of 16.
+ *   reroute: 0 = none; 1 = over-capacity re-routing (needs capacity > 0;
+ *     jsqmd.com 11.3.3 "专家丢弃": an overloaded expert's excess tokens go
+ *     to their next-best expert).  Each expert keeps its first C slots in
+ *     (token, k) order; the excess slots, in (token, k) order, move to the
+ *     candidate expert (within the token's kept groups) with the highest
+ *     selection key that still has room and that the token does not hold
+ *     (ties to the lower index); a slot with no such expert keeps its expert
+ *     and its overflow row.  Gates are then recomputed over the final
+ *     experts.  See moe_reroute.
  * Supported: (F32 act, F32 weights, GELU) with E <= 32 on the SIMT path;
  * (BF16 act, BF16 or E4M3 weights, SWIGLU or GELU; E4M3 with SWIGLU only)
  * on the tensor-core path.  E <= 256, K <= min(E, 32), d and h multiples
@@ -121,6 +131,7 @@ typedef struct {
   int32_t weight_dtype;
   int32_t capacity;
   int32_t act_quant;
+  int32_t reroute;
 } moe_desc;
 
 /* Weights, all DEVICE pointers (see layouts above).  Unused ones may be
@@ -219,6 +230,27 @@ moe_status moe_permute_static(const moe_desc *desc, const void *x, const int32_t
 moe_status moe_grouped_ffn(const moe_desc *desc, const moe_weights *w, const void *x_perm,
                            const int32_t *offsets, const void *x, void *y_perm, void *ws, size_t ws_bytes,
                            void *stream);
+
+/*
+ * Over-capacity re-routing (desc->reroute = 1, capacity > 0), the step
+ * between a capacity-bounded moe_permute and a second moe_permute:
+ *   moe_route (writes the selection keys and gate sources of every expert
+ *   into ws) -> moe_permute (x may be NULL) -> moe_reroute -> moe_permute
+ *   -> moe_grouped_ffn -> moe_combine.
+ * moe_layer_forward runs this sequence by itself when desc->reroute = 1.
+ *   topk_idx [S][K] int32 (in/out): the slots listed as excess by
+ *     row_of_slot (rows >= E*C) are moved as described at moe_desc.reroute;
+ *   topk_w [S][K] fp32 (in/out): the gates of every token with a moved slot
+ *     are recomputed over its final experts;
+ *   counts [E], row_of_slot [S*K]: moe_permute's outputs for this topk_idx.
+ * ws must hold the keys written by the last moe_route on it with the same
+ * desc.  One CTA runs the assignment (its visit order is serial; it commits
+ * chunks of up to 1024 slots at a time).  Moved slots are counted in
+ * MOE_CNT_REROUTED.  Errors: MOE_ERR_INVALID_ARG when reroute != 1 or a
+ * pointer is NULL, workspace errors as elsewhere.
+ */
+moe_status moe_reroute(const moe_desc *desc, int32_t *topk_idx, float *topk_w, const int32_t *counts,
+                       const int32_t *row_of_slot, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * Per-row E4M3 quantisation of bf16 rows, the activation step of the W8A8

@@ -21,7 +21,8 @@ size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 
 struct Layout {
   size_t status, logits, chunk_hist, groups, counts, offsets, topk_idx, topk_w, row_of_slot, token_of_row,
-      x_perm, hidden, y_perm, wdeq, ksplit, partial, partial_bytes, qa, sa, qas, sas, qh, sh, total;
+      x_perm, hidden, y_perm, wdeq, ksplit, partial, partial_bytes, qa, sa, qas, sas, qh, sh, rr_key, rr_score,
+      rr_ex, rr_changed, total;
 };
 
 // Split-K of the tensor-core GEMMs is available to small row spaces (decode-
@@ -73,6 +74,12 @@ Layout make_layout(const moe_desc& d) {
   L.sas = take(w8a8 && d.num_shared ? static_cast<size_t>(S) * 4 : 0);
   L.qh = take(w8a8 ? static_cast<size_t>(Rt * h) : 0);
   L.sh = take(w8a8 ? static_cast<size_t>(Rt) * 4 : 0);
+  // re-routing: every expert's selection key and gate source, the excess-slot list, changed tokens
+  const bool rr = d.reroute == 1;
+  L.rr_key = take(rr ? static_cast<size_t>(S * E) * 4 : 0);
+  L.rr_score = take(rr ? static_cast<size_t>(S * E) * 4 : 0);
+  L.rr_ex = take(rr ? static_cast<size_t>(S * K) * 4 : 0);
+  L.rr_changed = take(rr ? static_cast<size_t>(S) * 4 : 0);
   L.ksplit = take(kAlign);
   L.partial_bytes = 0;
   if (d.act_dtype == MOE_BF16 && Rt > 0 && Rt <= kSplitRowsMax) {
@@ -109,6 +116,8 @@ moe_status validate(const moe_desc* d) {
     return MOE_ERR_INVALID_ARG;
   if (d->capacity < 0) return MOE_ERR_INVALID_ARG;
   if (d->act_quant != 0 && d->act_quant != 1) return MOE_ERR_INVALID_ARG;
+  if (d->reroute != 0 && d->reroute != 1) return MOE_ERR_INVALID_ARG;
+  if (d->reroute == 1 && d->capacity <= 0) return MOE_ERR_INVALID_ARG;
   // row indices are int32 on the device
   const int64_t rows = routed_rows(*d) + static_cast<int64_t>(d->num_shared) * d->num_tokens;
   if (rows > (int64_t(1) << 31) - 1) return MOE_ERR_INVALID_ARG;
@@ -174,6 +183,10 @@ moe_status route_impl(const moe_desc& d, const moe_weights* w, const void* x, co
   a.topk_w = topk_w;
   a.status = at<StatusBlock>(ws, L.status);
   a.num_sms = num_sms();
+  if (d.reroute == 1) {
+    a.cand_key_out = at<float>(ws, L.rr_key);
+    a.score_out = at<float>(ws, L.rr_score);
+  }
   return cuda_status(launch_route(a, st));
 }
 
@@ -340,6 +353,19 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
   return MOE_OK;
 }
 
+moe_status reroute_impl(const moe_desc& d, int32_t* topk_idx, float* topk_w, const int32_t* counts,
+                        const int32_t* row_of_slot, void* ws, cudaStream_t st) {
+  const Layout L = make_layout(d);
+  int32_t* changed = at<int32_t>(ws, L.rr_changed);
+  cudaError_t e = launch_reroute_assign(d.num_tokens, d.num_experts, d.top_k, d.capacity, topk_idx,
+                                        at<float>(ws, L.rr_key), counts, row_of_slot, at<int32_t>(ws, L.rr_ex),
+                                        changed, at<StatusBlock>(ws, L.status), st);
+  if (e == cudaSuccess)
+    e = launch_reroute_gates(d.num_tokens, d.num_experts, d.top_k, d.score_fn, d.renormalize,
+                             at<float>(ws, L.rr_score), changed, topk_idx, topk_w, st);
+  return cuda_status(e);
+}
+
 moe_status combine_impl(const moe_desc& d, const void* y_perm, const int32_t* row_of_slot, const float* topk_w,
                         void* y, cudaStream_t st) {
   CombineArgs a{};
@@ -434,6 +460,18 @@ moe_status moe_grouped_ffn(const moe_desc* desc, const moe_weights* w, const voi
   return ffn_impl(*desc, *w, x_perm, offsets, x, y_perm, ws, static_cast<cudaStream_t>(stream));
 }
 
+moe_status moe_reroute(const moe_desc* desc, int32_t* topk_idx, float* topk_w, const int32_t* counts,
+                       const int32_t* row_of_slot, void* ws, size_t ws_bytes, void* stream) {
+  moe_status s = validate(desc);
+  if (s != MOE_OK) return s;
+  if (desc->reroute != 1) return MOE_ERR_INVALID_ARG;
+  if ((s = check_ws(*desc, ws, ws_bytes)) != MOE_OK) return s;
+  if (desc->num_tokens == 0) return MOE_OK;
+  if (topk_idx == nullptr || topk_w == nullptr || counts == nullptr || row_of_slot == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  return reroute_impl(*desc, topk_idx, topk_w, counts, row_of_slot, ws, static_cast<cudaStream_t>(stream));
+}
+
 moe_status moe_quantize_rows_e4m3(const void* x, int64_t rows, int32_t d, uint8_t* q, float* s, void* stream) {
   if (rows < 0 || d <= 0 || d % 16 != 0) return MOE_ERR_INVALID_ARG;
   if (rows == 0) return MOE_OK;
@@ -473,6 +511,12 @@ moe_status moe_layer_forward(const moe_desc* desc, const moe_weights* w, const v
   void* x_perm = at<void>(ws, L.x_perm);
   void* y_perm = at<void>(ws, L.y_perm);
   if ((s = route_impl(d, w, x, nullptr, idx, gates, ws, st)) != MOE_OK) return s;
+  if (d.reroute == 1) {
+    // capacity ranks of the first choices, then the excess slots move; the
+    // permutation below is that of the final choices
+    if ((s = permute_impl(d, nullptr, idx, cnt, offs, ros, tor, nullptr, ws, st)) != MOE_OK) return s;
+    if ((s = reroute_impl(d, idx, gates, cnt, ros, ws, st)) != MOE_OK) return s;
+  }
   // the permutation also writes the GEMM group tables, so the FFN skips that launch
   if (d.act_quant == 1) {
     // W8A8: the row gather writes E4M3 codes and row scales straight away

@@ -26,8 +26,23 @@ struct RouteArgs {
   float* topk_w;            // [S][K]
   StatusBlock* status;
   int num_sms;
+  float* cand_key_out;      // optional [S][E]: candidate keys (-inf for non-candidates), for re-routing
+  float* score_out;         // optional [S][E]: gate sources (logits or sigmoid scores), with cand_key_out
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream);
+
+// --- over-capacity re-routing ------------------------------------------------
+// Excess slots (row_of_slot >= E*C after a capacity-bounded permutation) move,
+// in (token, k) order, to the best-keyed candidate expert with room that the
+// token does not hold; changed[t] marks tokens with a moved slot.  One CTA.
+// ex_scratch: int32 [S*K].  moved_count (optional): device int, += moved slots.
+cudaError_t launch_reroute_assign(int S, int E, int K, int capacity, int32_t* topk_idx, const float* cand_key,
+                                  const int32_t* counts, const int32_t* row_of_slot, int32_t* ex_scratch,
+                                  int32_t* changed, StatusBlock* status, cudaStream_t stream);
+// Gates of the tokens marked in changed[], recomputed over their final experts
+// from the gate sources (the same formulas as the routing kernels).
+cudaError_t launch_reroute_gates(int S, int E, int K, int score_fn, int renormalize, const float* score,
+                                 const int32_t* changed, const int32_t* topk_idx, float* topk_w, cudaStream_t stream);
 
 // --- grouping by expert -----------------------------------------------------
 // Group table entry of the grouped GEMMs: rows [a_row0, a_row0 + rows) of the

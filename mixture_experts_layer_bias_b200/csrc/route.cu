@@ -88,7 +88,40 @@ struct SelectParams {
   int32_t* topk_idx;
   float* topk_w;
   StatusBlock* status;
+  float* cand_key;   // optional [S][E]: selection key of each candidate expert, -inf for the others
+  float* score_out;  // optional [S][E]: the gate source (logit, or sigmoid score) of every expert
 };
+
+// Gate of this lane's selected expert (lanes < K hold one each, my_score its
+// score); score[]/valid[] are the token's scores of experts 32*i + lane.
+template <int NI>
+__device__ __forceinline__ float gate_of(const float (&score)[NI], const bool (&valid)[NI], float my_score,
+                                         bool mine, int score_fn, int renormalize) {
+  const float kNegInf = __int_as_float(0xff800000);
+  if (score_fn == MOE_SCORE_SOFTMAX) {
+    if (renormalize) {
+      const float m = warp_max(mine ? my_score : kNegInf);
+      const float ex = mine ? expf(my_score - m) : 0.0f;
+      return ex / warp_sum(ex);
+    }
+    float m = kNegInf;
+#pragma unroll
+    for (int i = 0; i < NI; ++i)
+      if (valid[i]) m = fmaxf(m, score[i]);
+    m = warp_max(m);
+    float s = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NI; ++i)
+      if (valid[i]) s += expf(score[i] - m);
+    s = warp_sum(s);
+    return expf(my_score - m) / s;
+  }
+  if (renormalize) {
+    const float s = warp_sum(mine ? my_score : 0.0f);
+    return my_score / s;
+  }
+  return my_score;
+}
 
 // Selection for one token held by the whole warp: l[i] is the logit (router
 // bias included) of expert 32*i + lane.  Writes K indices and gates.
@@ -178,6 +211,16 @@ __device__ void select_topk(const float (&l)[NI], const SelectParams& p, int t) 
 #pragma unroll
     for (int i = 0; i < NI; ++i) cand[i] = cand[i] && gchosen[i];
   }
+  if (p.cand_key != nullptr) {
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+      const int e = 32 * i + lane;
+      if (valid[i]) {
+        p.cand_key[static_cast<int64_t>(t) * E + e] = cand[i] ? key[i] : kNegInf;
+        p.score_out[static_cast<int64_t>(t) * E + e] = score[i];
+      }
+    }
+  }
 
   int my_e = 0;
   float my_score = 0.0f;
@@ -208,34 +251,8 @@ __device__ void select_topk(const float (&l)[NI], const SelectParams& p, int t) 
     }
   }
 
-  float g;
   const bool mine = lane < p.K;
-  if (p.score_fn == MOE_SCORE_SOFTMAX) {
-    if (p.renormalize) {
-      const float m = warp_max(mine ? my_score : kNegInf);
-      const float ex = mine ? expf(my_score - m) : 0.0f;
-      g = ex / warp_sum(ex);
-    } else {
-      float m = kNegInf;
-#pragma unroll
-      for (int i = 0; i < NI; ++i)
-        if (valid[i]) m = fmaxf(m, score[i]);
-      m = warp_max(m);
-      float s = 0.0f;
-#pragma unroll
-      for (int i = 0; i < NI; ++i)
-        if (valid[i]) s += expf(score[i] - m);
-      s = warp_sum(s);
-      g = expf(my_score - m) / s;
-    }
-  } else {
-    if (p.renormalize) {
-      const float s = warp_sum(mine ? my_score : 0.0f);
-      g = my_score / s;
-    } else {
-      g = my_score;
-    }
-  }
+  const float g = gate_of<NI>(score, valid, my_score, mine, p.score_fn, p.renormalize);
   if (mine) {
     p.topk_idx[static_cast<int64_t>(t) * p.K + lane] = my_e;
     p.topk_w[static_cast<int64_t>(t) * p.K + lane] = g;
@@ -392,6 +409,33 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// Gates of a token whose experts changed after selection (over-capacity
+// re-routing): a warp per token, lanes holding the gate sources of experts
+// 32*i + lane as in the selection, lanes < K one selected expert each.
+template <int NI>
+__global__ void __launch_bounds__(kRouteWarps * 32)
+    reroute_gates_kernel(int S, int E, int K, int score_fn, int renormalize, const float* __restrict__ score_in,
+                         const int32_t* __restrict__ changed, const int32_t* __restrict__ topk_idx,
+                         float* __restrict__ topk_w) {
+  const int t = blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
+  if (t >= S || changed[t] == 0) return;
+  const int lane = lane_id();
+  const float* row = score_in + static_cast<int64_t>(t) * E;
+  float score[NI];
+  bool valid[NI];
+#pragma unroll
+  for (int i = 0; i < NI; ++i) {
+    const int e = 32 * i + lane;
+    valid[i] = e < E;
+    score[i] = valid[i] ? row[e] : __int_as_float(0xff800000);
+  }
+  const bool mine = lane < K;
+  const int my_e = mine ? topk_idx[static_cast<int64_t>(t) * K + lane] : 0;
+  const float my_score = (mine && my_e >= 0 && my_e < E) ? row[my_e] : 0.0f;
+  const float g = gate_of<NI>(score, valid, my_score, mine, score_fn, renormalize);
+  if (mine) topk_w[static_cast<int64_t>(t) * K + lane] = g;
+}
+
 template <int NI>
 cudaError_t launch_topk_ni(const RouteArgs& a, const float* logits, const SelectParams& sp, cudaStream_t st) {
   const int blocks = (a.S + kRouteWarps - 1) / kRouteWarps;
@@ -403,8 +447,8 @@ cudaError_t launch_topk_ni(const RouteArgs& a, const float* logits, const Select
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
   if (a.S == 0) return cudaSuccess;
-  SelectParams sp{a.E, a.K, a.score_fn, a.renormalize, a.num_groups, a.topk_groups, a.sel_bias,
-                  a.topk_idx, a.topk_w, a.status};
+  SelectParams sp{a.E,       a.K,        a.score_fn, a.renormalize, a.num_groups,  a.topk_groups, a.sel_bias,
+                  a.topk_idx, a.topk_w, a.status,   a.cand_key_out, a.score_out};
   const int blocks = (a.S + kRouteWarps - 1) / kRouteWarps;
   const float* logits = a.logits;
   if (logits == nullptr && a.E <= 32) {
@@ -477,6 +521,26 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
   if (ni <= 2) return launch_topk_ni<2>(a, logits, sp, stream);
   if (ni <= 4) return launch_topk_ni<4>(a, logits, sp, stream);
   return launch_topk_ni<8>(a, logits, sp, stream);
+}
+
+cudaError_t launch_reroute_gates(int S, int E, int K, int score_fn, int renormalize, const float* score,
+                                 const int32_t* changed, const int32_t* topk_idx, float* topk_w, cudaStream_t stream) {
+  if (S <= 0) return cudaSuccess;
+  const int blocks = (S + kRouteWarps - 1) / kRouteWarps;
+  const int ni = (E + 31) / 32;
+#define MOE_RG(N) \
+  reroute_gates_kernel<N><<<blocks, kRouteWarps * 32, 0, stream>>>(S, E, K, score_fn, renormalize, score, changed, \
+                                                                   topk_idx, topk_w)
+  if (ni <= 1)
+    MOE_RG(1);
+  else if (ni <= 2)
+    MOE_RG(2);
+  else if (ni <= 4)
+    MOE_RG(4);
+  else
+    MOE_RG(8);
+#undef MOE_RG
+  return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -23,17 +23,18 @@ _lib = None
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE_STATUS = range(6)
 MOE_STATUS_NONFINITE_LOGIT, MOE_STATUS_BAD_EXPERT_ID, MOE_STATUS_TIMEOUT, MOE_STATUS_BAD_GROUP = 1, 2, 4, 8
 MOE_NUM_COUNTERS = 8
-COUNTER_NAMES = ("nonfinite", "bad_id", "timeout", "overflow_rows")
+COUNTER_NAMES = ("nonfinite", "bad_id", "timeout", "overflow_rows", "rerouted")
 
 DESC_FIELDS = ("num_tokens", "d_model", "num_experts", "top_k", "d_ff", "score_fn", "renormalize", "num_groups",
-               "topk_groups", "num_shared", "activation", "act_dtype", "weight_dtype", "capacity", "act_quant")
+               "topk_groups", "num_shared", "activation", "act_dtype", "weight_dtype", "capacity", "act_quant",
+               "reroute")
 WEIGHT_FIELDS = ("w_router", "router_bias", "sel_bias", "w1", "b1", "w2", "b2", "w_gate", "w_up", "w_down",
                  "s_gate", "s_up", "s_down")
 
 EXPORTED = ("moe_routed_rows", "moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute",
             "moe_permute_static", "moe_grouped_ffn", "moe_combine", "moe_layer_forward", "moe_bias_state_size",
-            "moe_bias_state_init", "moe_update_sel_bias", "moe_quantize_rows_e4m3", "moe_get_status",
-            "moe_strerror")
+            "moe_bias_state_init", "moe_update_sel_bias", "moe_quantize_rows_e4m3", "moe_reroute",
+            "moe_get_status", "moe_strerror")
 
 
 class MoeDesc(ctypes.Structure):
@@ -74,6 +75,7 @@ def lib():
         "moe_bias_state_init": (I, [P, SZ, P]),
         "moe_update_sel_bias": (I, [pd, P, ctypes.c_int32, ctypes.c_float, P, SZ, P, P, P]),
         "moe_quantize_rows_e4m3": (I, [P, ctypes.c_int64, ctypes.c_int32, P, P, P]),
+        "moe_reroute": (I, [pd, P, P, P, P, P, SZ, P]),
         "moe_get_status": (I, [P, P, ctypes.POINTER(ctypes.c_uint32), ctypes.POINTER(ctypes.c_int32)]),
         "moe_strerror": (ctypes.c_char_p, [I]),
     }
@@ -92,7 +94,7 @@ def strerror(code: int) -> str:
 def make_desc(**fields) -> MoeDesc:
     d = MoeDesc()
     defaults = dict(score_fn=0, renormalize=1, num_groups=1, topk_groups=1, num_shared=0, activation=1,
-                    act_dtype=1, weight_dtype=1, capacity=0, act_quant=0)
+                    act_dtype=1, weight_dtype=1, capacity=0, act_quant=0, reroute=0)
     defaults.update(fields)
     for f in DESC_FIELDS:
         setattr(d, f, int(defaults[f]))
@@ -207,6 +209,12 @@ def moe_update_sel_bias(desc, topk_idx, window_tokens, gamma, state, sel_bias, w
     p, n = _ws(state)
     _check(lib().moe_update_sel_bias(ctypes.byref(desc), _ptr(topk_idx), int(window_tokens), float(gamma), p, n,
                                      _ptr(sel_bias), _ptr(window_counts), _stream(stream)), "moe_update_sel_bias")
+
+
+def moe_reroute(desc, topk_idx, topk_w, counts, row_of_slot, ws, stream=None):
+    p, n = _ws(ws)
+    _check(lib().moe_reroute(ctypes.byref(desc), _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(row_of_slot), p, n,
+                             _stream(stream)), "moe_reroute")
 
 
 def moe_quantize_rows_e4m3(x, q, s, stream=None):

@@ -66,6 +66,7 @@ class LayerConfig:
     weight_dtype: int = BF16
     capacity: int = 0
     act_quant: int = 0               # 1: W8A8 (E4M3 activation rows with per-row scales)
+    reroute: int = 0                 # 1: over-capacity slots move to the next-best expert with room
     router_offset_var: float = 0.0   # variance of N(0, v) per-expert logit offsets
     skew_offset_scale: float = 0.0   # c of the c * z_e offsets
     sel_bias_var: float = 0.0        # variance of the selection bias
@@ -84,7 +85,7 @@ CONFIGS = {
                                      skew_offset_scale=SKEW_OFFSET_SCALE),
 }
 
-# W8A8 variants: the same inputs with the expert GEMMs run on E4M3
+# Variants of the workloads.  W8A8: the same inputs with the expert GEMMs run on E4M3
 # activations (per-row scales) against E4M3 weights.  The Mixtral-shaped one
 # stores its expert weights as E4M3 with per-output-channel scales.
 VARIANTS = {
@@ -92,6 +93,9 @@ VARIANTS = {
                                                   act_quant=1),
     "mixtral_prefill_w8a8": dataclasses.replace(CONFIGS["mixtral_prefill"], name="mixtral_prefill_w8a8",
                                                 weight_dtype=E4M3, act_quant=1),
+    # the skewed capacity-bounded layer with over-capacity re-routing instead of the overflow pass
+    "fp8_skew_capacity_reroute": dataclasses.replace(CONFIGS["fp8_skew_capacity"], name="fp8_skew_capacity_reroute",
+                                                     reroute=1),
 }
 
 DECODE_SIZES = (1, 8, 32, 128)
@@ -198,4 +202,4 @@ def desc_dict(cfg: LayerConfig, S: Optional[int] = None) -> dict:
                 d_ff=cfg.h, score_fn=cfg.score_fn, renormalize=cfg.renormalize, num_groups=cfg.num_groups,
                 topk_groups=cfg.topk_groups, num_shared=cfg.num_shared, activation=cfg.activation,
                 act_dtype=cfg.act_dtype, weight_dtype=cfg.weight_dtype, capacity=cfg.capacity,
-                act_quant=cfg.act_quant)
+                act_quant=cfg.act_quant, reroute=cfg.reroute)

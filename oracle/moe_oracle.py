@@ -273,6 +273,21 @@ def select_experts(
     """
     logits = np.asarray(logits, dtype=np.float32)
     S, E = logits.shape
+    scores, keys, cand = selection_keys(logits, score_fn, sel_bias, num_groups, topk_groups)
+    # candidates first, each part in descending key order, ties to lower index
+    neg = -keys.astype(np.float64)
+    order = np.lexsort((np.broadcast_to(np.arange(E), (S, E)), neg, ~cand), axis=-1)
+    idx = order[:, :top_k].astype(np.int32)
+    return idx, gate_weights(scores, idx, score_fn, renormalize)
+
+
+def selection_keys(logits, score_fn="softmax", sel_bias=None, num_groups=1, topk_groups=1):
+    """The quantities selection works on (see ``select_experts``): scores
+    (float32 logits, or their sigmoid), keys (scores + sel_bias in float32,
+    NaN -> -inf) and the candidate mask (experts of the token's kept
+    groups; all experts without groups)."""
+    logits = np.asarray(logits, dtype=np.float32)
+    S, E = logits.shape
     if score_fn == "softmax":
         scores = logits
     elif score_fn == "sigmoid":
@@ -293,25 +308,27 @@ def select_experts(
         cand = np.repeat(keep, gs, axis=1)
     else:
         cand = np.ones((S, E), dtype=bool)
-    # candidates first, each part in descending key order, ties to lower index
-    neg = -keys.astype(np.float64)
-    order = np.lexsort((np.broadcast_to(np.arange(E), (S, E)), neg, ~cand), axis=-1)
-    idx = order[:, :top_k].astype(np.int32)
+    return scores, keys, cand
+
+
+def gate_weights(scores, idx, score_fn="softmax", renormalize=True):
+    """Gates of the experts idx [S, K] from the float32 scores [S, E]
+    (``select_experts``): softmax over the K selected logits, or the full
+    softmax probability; sigmoid scores normalised over the K, or as they are.
+    float64."""
+    idx = np.asarray(idx)
     if score_fn == "softmax":
-        l = logits.astype(np.float64)
+        l = np.asarray(scores, np.float32).astype(np.float64)
         sel = np.take_along_axis(l, idx, axis=1)
         if renormalize:
             m = sel.max(axis=1, keepdims=True)
             ex = np.exp(sel - m)
-            w = ex / ex.sum(axis=1, keepdims=True)
-        else:
-            m = l.max(axis=1, keepdims=True)
-            ex = np.exp(l - m)
-            w = np.take_along_axis(ex, idx, axis=1) / ex.sum(axis=1, keepdims=True)
-    else:
-        s = np.take_along_axis(scores.astype(np.float64), idx, axis=1)
-        w = s / s.sum(axis=1, keepdims=True) if renormalize else s
-    return idx, w
+            return ex / ex.sum(axis=1, keepdims=True)
+        m = l.max(axis=1, keepdims=True)
+        ex = np.exp(l - m)
+        return np.take_along_axis(ex, idx, axis=1) / ex.sum(axis=1, keepdims=True)
+    s = np.take_along_axis(np.asarray(scores, np.float32).astype(np.float64), idx, axis=1)
+    return s / s.sum(axis=1, keepdims=True) if renormalize else s
 
 
 def selection_margin(logits, top_k, score_fn="softmax", sel_bias=None, num_groups=1, topk_groups=1):
@@ -403,6 +420,52 @@ def expert_permutation(topk_idx: np.ndarray, num_experts: int, capacity: int = 0
     token_of_row[row_of_slot] = np.arange(S * K) // K
     out.update(row_of_slot=row_of_slot.astype(np.int32), token_of_row=token_of_row.astype(np.int32), num_rows=R)
     return out
+
+
+def reroute_over_capacity(topk_idx, keys, cand, capacity: int):
+    """Over-capacity re-routing (jsqmd.com chapter 11, 11.3.3, "专家丢弃":
+    when an expert is overloaded, its excess tokens go to their next-best
+    expert).  The page gives the rule in one sentence; the reading taken:
+
+    1. every expert keeps the first ``capacity`` slots routed to it, slots in
+       (token, k) order;
+    2. the remaining (excess) slots are visited in (token, k) order; each
+       moves to the best expert by the token's selection key among the
+       token's candidates (its kept groups) that still has room and that the
+       token does not hold already (ties to the lower index), taking one unit
+       of that expert's room;
+    3. an excess slot with no such expert keeps its expert (it then goes to
+       the overflow region, as without re-routing).
+
+    Returns (new topk_idx int32 [S, K], moved bool [S, K]).  Gates are then
+    recomputed over the final experts (``gate_weights``)."""
+    idx = np.array(topk_idx, dtype=np.int32, copy=True)
+    S, K = idx.shape
+    E = keys.shape[1]
+    kept = np.zeros(E, dtype=np.int64)
+    excess = []
+    for t in range(S):
+        for k in range(K):
+            e = idx[t, k]
+            if kept[e] < capacity:
+                kept[e] += 1
+            else:
+                excess.append((t, k))
+    room = capacity - kept
+    moved = np.zeros((S, K), dtype=bool)
+    for t, k in excess:
+        best, best_key = -1, -np.inf
+        held = set(idx[t].tolist())
+        for e in range(E):
+            if room[e] <= 0 or e in held or not cand[t, e] or keys[t, e] == -np.inf:
+                continue
+            if best < 0 or keys[t, e] > best_key:
+                best, best_key = e, keys[t, e]
+        if best >= 0:
+            idx[t, k] = best
+            room[best] -= 1
+            moved[t, k] = True
+    return idx, moved
 
 
 def load_stats(counts: np.ndarray, top_k: int, num_tokens: int) -> dict:

@@ -89,7 +89,12 @@ class OracleExperts:
 
 def oracle_routing(inp: dict, cfg: syn.LayerConfig, tokens=None):
     """Oracle router logits, selection, gates and margins for the given
-    tokens (all by default)."""
+    tokens (all by default).  With re-routing the assignment depends on the
+    whole batch, so every token is routed and the given ones returned."""
+    if cfg.reroute and tokens is not None:
+        x, idx, w, margin = oracle_routing(inp, cfg)
+        tokens = np.asarray(tokens)
+        return x[tokens], idx[tokens], w[tokens], margin[tokens]
     x = np64(inp["x"]) if tokens is None else np64(inp["x"][tokens])
     rb = None if inp.get("router_bias") is None else np64(inp["router_bias"])
     logits = O.router_logits(x, np64(inp["w_router"]), rb)
@@ -97,7 +102,16 @@ def oracle_routing(inp: dict, cfg: syn.LayerConfig, tokens=None):
     idx, w = O.select_experts(logits, cfg.K, SCORE[cfg.score_fn], bool(cfg.renormalize), sb, cfg.num_groups,
                               cfg.topk_groups)
     margin = O.selection_margin(logits, cfg.K, SCORE[cfg.score_fn], sb, cfg.num_groups, cfg.topk_groups)
+    if cfg.reroute:
+        idx, w = oracle_reroute(logits, idx, cfg, sb)
     return x, idx, w, margin
+
+
+def oracle_reroute(logits, idx, cfg: syn.LayerConfig, sel_bias=None):
+    """Over-capacity re-routing of the oracle's selection, gates recomputed."""
+    scores, keys, cand = O.selection_keys(logits, SCORE[cfg.score_fn], sel_bias, cfg.num_groups, cfg.topk_groups)
+    new, _ = O.reroute_over_capacity(idx, keys, cand, cfg.capacity)
+    return new, O.gate_weights(scores, new, SCORE[cfg.score_fn], bool(cfg.renormalize))
 
 
 def oracle_layer(inp: dict, cfg: syn.LayerConfig, tokens=None):

@@ -74,6 +74,7 @@ BAD = [
     dict(d_ff=0), dict(score_fn=5), dict(num_groups=3), dict(num_groups=2, topk_groups=3),
     dict(num_groups=4, topk_groups=1, top_k=3), dict(num_shared=2), dict(capacity=-1), dict(num_tokens=-1),
     dict(renormalize=2), dict(activation=7), dict(act_dtype=5), dict(act_quant=2), dict(act_quant=-1),
+    dict(reroute=2), dict(reroute=1),  # re-routing needs a capacity (mixtral_prefill has none)
 ]
 
 
@@ -166,7 +167,7 @@ def test_bias_state_size_and_argument_errors():
     assert L.moe_bias_state_init(None, 0, None) == ops.MOE_ERR_WORKSPACE
 
 
-@pytest.mark.parametrize("name", list(syn.VARIANTS))
+@pytest.mark.parametrize("name", [n for n, c in syn.VARIANTS.items() if c.act_quant])
 def test_w8a8_workspace_holds_codes_and_scales(name):
     """W8A8 replaces the bf16 weight copy with the 8-bit activation rows."""
     cfg = syn.VARIANTS[name]
@@ -194,3 +195,20 @@ def test_quantize_rows_argument_errors():
     assert L.moe_quantize_rows_e4m3(ctypes.c_void_p(0x1008), 4, 32, p, p, None) == ops.MOE_ERR_INVALID_ARG
     assert L.moe_quantize_rows_e4m3(p, 4, 32, ctypes.c_void_p(0x1004), p, None) == ops.MOE_ERR_INVALID_ARG
     assert L.moe_quantize_rows_e4m3(p, 4, 32, p, ctypes.c_void_p(0x1002), None) == ops.MOE_ERR_INVALID_ARG
+
+
+def test_reroute_workspace_and_argument_errors():
+    L = ops.lib()
+    d = _desc("fp8_skew_capacity_reroute")
+    d0 = _desc("fp8_skew_capacity")
+    cfg = syn.VARIANTS["fp8_skew_capacity_reroute"]
+    # keys + gate sources of every expert, the excess list and the changed flags
+    assert ops.moe_workspace_size(d) - ops.moe_workspace_size(d0) >= cfg.S * cfg.E * 8 + cfg.S * cfg.K * 4
+    n = ops.moe_workspace_size(d)
+    p = ctypes.c_void_p(0x1000)
+    ws = ctypes.c_void_p(0x100000)
+    assert L.moe_reroute(ctypes.byref(d0), p, p, p, p, ws, n, None) == ops.MOE_ERR_INVALID_ARG  # reroute = 0
+    assert L.moe_reroute(ctypes.byref(d), None, p, p, p, ws, n, None) == ops.MOE_ERR_INVALID_ARG
+    assert L.moe_reroute(ctypes.byref(d), p, p, p, None, ws, n, None) == ops.MOE_ERR_INVALID_ARG
+    assert L.moe_reroute(ctypes.byref(d), p, p, p, p, ws, n - 256, None) == ops.MOE_ERR_WORKSPACE
+    assert L.moe_reroute(ctypes.byref(d), p, p, p, p, None, n, None) == ops.MOE_ERR_WORKSPACE

@@ -530,3 +530,92 @@ def test_w8a8_expert_exact_on_representable_rows():
     yref = O.expert_swiglu(x, O.e4m3_bits_to_f64(qg), O.e4m3_bits_to_f64(qu), O.e4m3_bits_to_f64(qd),
                            s_gate=sg, s_up=su, s_down=sd)
     np.testing.assert_allclose(y8, yref, rtol=1e-6, atol=1e-12 * np.abs(yref).max())
+
+
+# ----------------------------------------------------------------------------
+# over-capacity re-routing (jsqmd.com chapter 11, 11.3.3)
+# ----------------------------------------------------------------------------
+
+
+def _reroute(keys, K, C, cand=None):
+    keys = np.asarray(keys, np.float32)
+    if cand is None:
+        cand = np.ones(keys.shape, bool)
+    idx, _ = O.select_experts(keys, K)
+    return idx, O.reroute_over_capacity(idx, keys, cand, C)
+
+
+def test_reroute_hand_computed():
+    """E=4, K=1, C=1.  Three tokens all prefer e0: t0 keeps it; t1 (excess)
+    takes its best expert with room, e1; t2 then finds e1 full and takes e3
+    (key 2 beats e2's 1)."""
+    idx, (new, moved) = _reroute([[4, 3, 2, 1], [4, 3, 2, 1], [4, 3, 1, 2]], 1, 1)
+    assert idx[:, 0].tolist() == [0, 0, 0]
+    assert new[:, 0].tolist() == [0, 1, 3]
+    assert moved[:, 0].tolist() == [False, True, True]
+    # a slot that finds no room keeps its expert (and its overflow row)
+    idx, (new, moved) = _reroute([[2, 1], [2, 1], [2, 1]], 1, 1)
+    assert new[:, 0].tolist() == [0, 1, 0] and moved[:, 0].tolist() == [False, True, False]
+
+
+def test_reroute_skips_held_and_non_candidate_experts():
+    """E=4, K=2, C=2: t2's excess slot (e0) cannot take e2, which t2 already
+    holds, nor e1 (full), nor e3 outside its candidates; nothing is left, so
+    it stays.  With e3 a candidate it moves there."""
+    keys = [[4, 3, 2, 1], [4, 3, 1, 2], [4, 1, 3, 2]]
+    cand = np.ones((3, 4), bool)
+    cand[2, 3] = False
+    idx, (new, moved) = _reroute(keys, 2, 2, cand)
+    assert idx.tolist() == [[0, 1], [0, 1], [0, 2]]
+    assert new.tolist() == idx.tolist() and not moved.any()
+    idx, (new, moved) = _reroute(keys, 2, 2)
+    assert new.tolist() == [[0, 1], [0, 1], [3, 2]] and moved.tolist() == [[False] * 2, [False] * 2, [True, False]]
+
+
+def test_reroute_invariants_on_a_skewed_batch():
+    rng = np.random.default_rng(21)
+    S, E, K = 600, 16, 4
+    keys = (rng.normal(size=(S, E)) + 1.5 * rng.normal(size=E)[None, :]).astype(np.float32)
+    C = O_cap = int(np.ceil(1.1 * S * K / E))
+    idx, (new, moved) = _reroute(keys, K, C)
+    counts0 = O.expert_counts(idx, E)
+    assert counts0.max() > C                                     # the batch really overflows
+    # slots are moved only out of overloaded experts, never within a token twice
+    assert all(len(set(r.tolist())) == K for r in new)
+    P0 = O.expert_permutation(idx, E, C)
+    excess = (P0["row_of_slot"] >= E * C).reshape(S, K)
+    assert not (moved & ~excess).any()
+    assert (new[~moved] == idx[~moved]).all()
+    # every expert that received moved slots stays within its capacity
+    counts1 = O.expert_counts(new, E)
+    recv = np.bincount(new[moved], minlength=E)
+    assert (counts1[recv > 0] <= C).all()
+    # a moved slot's new expert ranks below all of the token's original K
+    t, k = np.nonzero(moved)
+    kth = np.sort(np.take_along_axis(keys, idx, 1), axis=1)[:, 0]
+    assert (keys[t, new[t, k]] <= kth[t]).all()
+    # the total room is large enough here, so every excess slot finds an expert
+    assert moved.sum() == excess.sum()
+    # unbounded capacity changes nothing
+    _, (same, none) = _reroute(keys, K, S)
+    assert (same == idx).all() and not none.any()
+    assert O_cap == C
+
+
+def test_reroute_visit_order_is_slot_order():
+    """Two excess slots compete for the last unit of room: the earlier slot
+    in (token, k) order wins, the later one takes the next best."""
+    keys = [[9, 1, 5, 4], [9, 2, 5, 4], [9, 3, 5, 4]]
+    idx, (new, moved) = _reroute(keys, 1, 1)
+    # t0 keeps e0; t1 -> e2 (5); t2 -> e2 full -> e3 (4)
+    assert new[:, 0].tolist() == [0, 2, 3]
+
+
+def test_gate_weights_match_selection():
+    rng = np.random.default_rng(22)
+    logits = rng.normal(size=(50, 12)).astype(np.float32)
+    for fn in ("softmax", "sigmoid"):
+        for renorm in (True, False):
+            idx, w = O.select_experts(logits, 3, fn, renorm)
+            scores, _, _ = O.selection_keys(logits, fn)
+            np.testing.assert_allclose(O.gate_weights(scores, idx, fn, renorm), w, rtol=0, atol=0)
