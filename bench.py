@@ -359,8 +359,11 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=sorted(syn.CONFIGS) + sorted(syn.VARIANTS) + ["profile_small", "profile_small_w8a8"],
-                    help="profile_small: S=2048, d=4096, h=4096 (same kernels, ~1 GB) for ncu captures")
+                    choices=sorted(syn.CONFIGS) + sorted(syn.VARIANTS)
+                    + ["profile_small", "profile_small_w8a8", "profile_small_dsv3"],
+                    help="profile_small*: smaller cases of the same kernels (0.4-1.5 GB of weights) for ncu "
+                         "captures: Mixtral-shaped S=2048, h=4096 (bf16 or W8A8); DeepSeek-shaped S=512 with "
+                         "16 routed experts (~256 rows each) + the shared one")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))
@@ -382,6 +385,8 @@ def main():
         cfg = syn.scaled(syn.CONFIGS[WORKLOAD], S=2048, h=4096)
     elif args.workload == "profile_small_w8a8":
         cfg = syn.scaled(syn.VARIANTS["mixtral_prefill_w8a8"], S=2048, h=4096)
+    elif args.workload == "profile_small_dsv3":
+        cfg = syn.scaled(syn.CONFIGS["dsv3_grouped"], S=512, E=16, num_groups=1, topk_groups=1)
     else:
         cfg = syn.CONFIGS.get(args.workload) or syn.VARIANTS[args.workload]
     S = cfg.S

@@ -35,6 +35,7 @@ struct TcParams {
   int pcols;           // 2N (SwiGLU: gate then up) or N
   int* ksplit_out;     // the split chosen on the device, read by the finalize kernel
   int test_stall;      // test hook: the producer delivers nothing (the bounded waits must give up)
+  int tma_out;         // 1: the output tensor map is valid (full 32-row quarters use bulk tensor stores)
   const float* row_scale;         // E4M3 activations: per-row scale of the A operand rows (nullptr: none)
   const float* row_scale_shared;  // ... of the shared expert's A rows (indexed by row within the group)
   StatusBlock* status;
@@ -149,6 +150,21 @@ inline EncodeTiledFn get_encode_fn() {
 
 // 2-D map over [rows][k] (row-major) of bf16 (elem_bytes 2) or 8-bit (1)
 // elements; box = one 128-byte swizzle row of k by box_rows rows.
+// 2-D map over an output [rows][cols] (row-major, bf16 or fp32) for bulk
+// tensor stores of 32 x 32 element boxes, no swizzle.
+inline bool make_store_map(CUtensorMap* m, void* base, int64_t rows, int cols, int elem_bytes) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr || rows <= 0 || cols <= 0) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || (static_cast<int64_t>(cols) * elem_bytes) % 16 != 0) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * elem_bytes};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, elem_bytes == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims,
+             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline bool make_map(CUtensorMap* m, const void* base, int64_t rows, int k, int box_rows = 128, int elem_bytes = 2) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr || rows <= 0 || k <= 0) return false;

@@ -80,6 +80,7 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t 
     if (p.max_ksplit < 1) p.max_ksplit = 1;
   }
   p.test_stall = 0;
+  p.tma_out = 0;  // set by the token-rows launcher when it can map the output
   p.row_scale = a.fp8 ? a.row_scale : nullptr;
   p.row_scale_shared = a.fp8 ? a.row_scale_shared : nullptr;
   if (a.fp8 && a.row_scale == nullptr) return cudaErrorInvalidValue;

@@ -20,13 +20,15 @@
 // accumulator row by its activation row scale and each column by the weight
 // channel scale.
 //
-// Structure (one CTA per SM, 192 threads):
+// Structure (one CTA per SM, 320 threads):
 //   warp 0      TMA producer: A tile 128x64 and B tile 256x64 (bf16, 128-byte
 //               swizzle) per stage into a 4-stage shared-memory ring;
 //   warp 1      allocates 512 TMEM columns; one lane issues tcgen05.mma
 //               (kind::f16, fp32 accumulate) and tcgen05.commit;
-//   warps 2-5   epilogue: tcgen05.ld of their 32-lane quarter, activation,
-//               predicated 16-byte stores of the group's valid rows only.
+//   warps 2-9   epilogue, two warps per 32-lane TMEM quarter, each draining
+//               half of the tile's columns: tcgen05.ld, activation, then a
+//               bulk tensor store per 32 x 32 box (or row stores for a group's
+//               last, partial quarter).
 // Two 256-column accumulators let the epilogue of tile i overlap the MMAs of
 // tile i+1.  The tile list (group, n-block, m-block; m fastest, so the CTAs
 // in flight share weight tiles through L2) is derived on the device from the
@@ -61,7 +63,8 @@ constexpr int B_HALF = 128 * BK_BYTES;        // 16 KB
 constexpr int B_TILE = 2 * B_HALF;            // 32 KB
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;  // two per TMEM lane quarter, each draining half of a tile's columns
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kIdescBf16 = idesc_bf16_f32(128, 256);
 constexpr uint32_t kIdescE4m3 = idesc_e4m3_f32(128, 256);
 
@@ -84,7 +87,9 @@ struct SmemCtl {
 };
 
 constexpr size_t kSmemLimitTc = 232448;  // 227 KB per CTA
-constexpr size_t kCtlBytes = sizeof(SmemCtl) + 1024;  // control block + alignment slack
+// epilogue staging: one 32 x 32 box (fp32 at most) per epilogue warp, 128-byte aligned
+constexpr int kEpiWarpBytes = 32 * 32 * 2;  // bf16 boxes (fp32 outputs store row by row)
+constexpr size_t kCtlBytes = sizeof(SmemCtl) + 1024 + 128 + kEpiWarps * kEpiWarpBytes;  // control, staging, slack
 
 __device__ __forceinline__ bool wait_timed(uint64_t* bar, uint32_t parity) {
   int never = 0;
@@ -134,16 +139,23 @@ __device__ __forceinline__ UnitInfo decode_unit(const SmemCtl& s, const TcParams
 // (weight-channel scales, biases) are loaded once per 32-column chunk, lane j
 // holding column n + j, and handed to every lane by shuffles; SiLU uses the
 // fast reciprocal-based division.
+//
+// A warp whose 32 rows all belong to the group (every quarter but a group's
+// last) writes each 32-column chunk into its shared-memory box and stores it
+// with one bulk tensor store (full 128-byte lines instead of 32 scattered
+// 16-byte pieces per store instruction); a partial quarter stores row by row.
 template <int EPI>
 __device__ __forceinline__ void epilogue_store(const TcParams& p, const TileInfo& ti, uint32_t tbase, int row,
-                                               bool valid, int lane) {
+                                               bool valid, int lane, int half, const CUtensorMap* tm_out,
+                                               uint8_t* ebuf) {
   const int N = p.N;
   const int64_t orow = static_cast<int64_t>(ti.grp.out_row0) + row;
+  const bool full = p.tma_out && (row - lane) + 32 <= ti.grp.rows;  // warp-uniform
   const int64_t sbase = static_cast<int64_t>(ti.grp.expert) * N;
   const float rs = valid ? a_row_scale(p, ti.grp, row) : 1.0f;
   constexpr int kChunks = (EPI == EPI_SWIGLU) ? 4 : 8;
   constexpr bool kBias = EPI == EPI_GELU_BIAS || EPI == EPI_BIAS;
-  for (int c = 0; c < kChunks; ++c) {
+  for (int c = half * (kChunks / 2); c < (half + 1) * (kChunks / 2); ++c) {
     const int n = ti.n_idx * p.bn_out + c * 32;
     const bool col_ok = n + lane < N;
     float cs0 = 1.0f, cs1 = 1.0f, cb = 0.0f;  // this lane's column: channel scales, bias
@@ -176,6 +188,19 @@ __device__ __forceinline__ void epilogue_store(const TcParams& p, const TileInfo
         v[j] = z;
       }
     }
+    if (full) {
+      if (lane == 0) bulk_wait_read_all();  // the previous box has been read out
+      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < 4; ++j) stg16(ebuf + lane * 64 + 16 * j, pack16<__nv_bfloat16>(v + 8 * j));
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && n < N) {
+        tma_store_2d(tm_out, ebuf, n, static_cast<int>(orow - lane));
+        bulk_commit();
+      }
+      continue;
+    }
     if (!valid) continue;
     if (p.out_f32) {
       float* o = static_cast<float*>(p.out) + orow * N + n;
@@ -195,12 +220,12 @@ __device__ __forceinline__ void epilogue_store(const TcParams& p, const TileInfo
 // slice of the partial buffer (SwiGLU: gate columns at n, up columns at N+n).
 template <int EPI>
 __device__ __forceinline__ void epilogue_partial(const TcParams& p, const TileInfo& ti, uint32_t tbase, int row,
-                                                 bool valid, int split) {
+                                                 bool valid, int split, int half) {
   const int N = p.N;
   const int64_t orow = static_cast<int64_t>(ti.grp.out_row0) + row;
   float* base = p.partial + (static_cast<int64_t>(split) * p.out_rows + orow) * p.pcols;
-  constexpr int kChunks = 8;  // 256 accumulator columns
-  for (int c = 0; c < kChunks; ++c) {
+  constexpr int kChunks = 8;  // 256 accumulator columns, half of them per warp
+  for (int c = half * 4; c < half * 4 + 4; ++c) {
     uint32_t r[32];
     tmem_ld_32x32b_x32(tbase + c * 32, r);
     tmem_ld_wait();
@@ -225,13 +250,15 @@ template <int EPI, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                            const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
-                           TcParams p, int bma, int STAGES) {
+                           const __grid_constant__ CUtensorMap tmOut, TcParams p, int bma, int STAGES) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int BK = bk_elems<F8>();
   const int A_TILE = bma * BK_BYTES;
   const int STAGE_BYTES = A_TILE + B_TILE;
   SmemCtl& s = *reinterpret_cast<SmemCtl*>(ring + STAGES * STAGE_BYTES);
+  uint8_t* epi_smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(ring + STAGES * STAGE_BYTES + sizeof(SmemCtl)) + 127) & ~uintptr_t(127));
   const int warp = threadIdx.x >> 5, lane = lane_id();
 
   // per-group tile counts -> exclusive prefix (warp 0)
@@ -265,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int i = 0; i < 2; ++i) {
         mbar_init(&s.tfull[i], 1);
-        mbar_init(&s.tempty[i], 128);
+        mbar_init(&s.tempty[i], 32 * kEpiWarps);
       }
       mbar_init(&s.drain, 1);
       s.abort = 0;
@@ -390,7 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;                // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;      // which half of the tile's columns it drains
     int local = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x, ++local) {
       const UnitInfo ui = decode_unit(s, p, u, ks, nk);
@@ -409,14 +437,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = row < ti.grp.rows;
       const uint32_t tbase = tmem + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16);
       if (ks > 1)
-        epilogue_partial<EPI>(p, ti, tbase, row, valid, ui.split);
+        epilogue_partial<EPI>(p, ti, tbase, row, valid, ui.split, half);
       else
-        epilogue_store<EPI>(p, ti, tbase, row, valid, lane);
+        epilogue_store<EPI>(p, ti, tbase, row, valid, lane, half, &tmOut, epi_smem + (warp - 2) * kEpiWarpBytes);
       tc_fence_before();
       mbar_arrive(&s.tempty[acc]);
     }
   }
 
+  if (warp >= 2 && lane == 0) bulk_wait_all();  // this warp's output boxes are written
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -427,8 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int EPI, bool F8>
 cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB0, const CUtensorMap& mB1,
-                       const TcParams& p, int grid, int bma, int stages, size_t smem, int64_t max_group_rows,
-                       cudaStream_t stream) {
+                       const CUtensorMap& mOut, const TcParams& p, int grid, int bma, int stages, size_t smem,
+                       int64_t max_group_rows, cudaStream_t stream) {
   static uint64_t attr_set = 0;  // one bit per device ordinal
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -439,7 +468,7 @@ cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUte
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set |= 1ull << dev;
   }
-  grouped_gemm_tc_kernel<EPI, F8><<<grid, kThreads, smem, stream>>>(mA, mA2, mB0, mB1, p, bma, stages);
+  grouped_gemm_tc_kernel<EPI, F8><<<grid, kThreads, smem, stream>>>(mA, mA2, mB0, mB1, mOut, p, bma, stages);
   e = cudaGetLastError();
   if (e != cudaSuccess || p.max_ksplit <= 1) return e;
   dim3 fgrid((p.N + 1023) / 1024, static_cast<unsigned>(max_group_rows), p.num_groups);
@@ -459,7 +488,11 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
   int stages = static_cast<int>((kSmemLimitTc - kCtlBytes) / stage_bytes);
   if (stages > MAX_STAGES) stages = MAX_STAGES;
   const size_t smem = stages * stage_bytes + kCtlBytes;
-  CUtensorMap mA, mA2, mB0, mB1;
+  CUtensorMap mA, mA2, mB0, mB1, mOut;
+  // bf16 outputs: full 32-row quarters go out as bulk tensor stores; fp32 outputs store row by row
+  TcParams pp = p;
+  pp.tma_out = !a.out_f32 && make_store_map(&mOut, a.out, a.out_rows, a.N, 2) ? 1 : 0;
+  if (!pp.tma_out) memset(&mOut, 0, sizeof(mOut));
   if (!make_map(&mA, a.a, a.a_rows, a.K, bma, eb)) return cudaErrorInvalidValue;
   if (a.a_shared != nullptr) {
     if (!make_map(&mA2, a.a_shared, a.a_shared_rows, a.K, bma, eb)) return cudaErrorInvalidValue;
@@ -478,22 +511,22 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
   if (a.fp8) {  // W8A8 runs SwiGLU experts only
     switch (a.epilogue) {
       case EPI_SWIGLU:
-        return launch_epi<EPI_SWIGLU, true>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows, stream);
+        return launch_epi<EPI_SWIGLU, true>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
       case EPI_NONE:
-        return launch_epi<EPI_NONE, true>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows, stream);
+        return launch_epi<EPI_NONE, true>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
       default: return cudaErrorInvalidValue;
     }
   }
   switch (a.epilogue) {
     case EPI_SWIGLU:
-      return launch_epi<EPI_SWIGLU, false>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows, stream);
+      return launch_epi<EPI_SWIGLU, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
     case EPI_GELU_BIAS:
-      return launch_epi<EPI_GELU_BIAS, false>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows,
-                                              stream);
+      return launch_epi<EPI_GELU_BIAS, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem,
+                                              a.max_group_rows, stream);
     case EPI_BIAS:
-      return launch_epi<EPI_BIAS, false>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows, stream);
+      return launch_epi<EPI_BIAS, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
     case EPI_NONE:
-      return launch_epi<EPI_NONE, false>(mA, mA2, mB0, mB1, p, grid, bma, stages, smem, a.max_group_rows, stream);
+      return launch_epi<EPI_NONE, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
     default: return cudaErrorInvalidValue;
   }
 }
