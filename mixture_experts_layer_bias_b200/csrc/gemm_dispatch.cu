@@ -31,7 +31,8 @@ int take_test_stall() {
 
 // Kernel choice (read once): MOE_B200_GEMM=pair or =wt selects the CTA-pair or
 // the one-CTA weights-as-M kernel, =hybrid the weights-as-M kernel for all but
-// the SwiGLU up projection; otherwise the token-rows kernel.
+// the SwiGLU up projection; otherwise the token-rows kernel, on CTA pairs for
+// large groups (=single forces one CTA, =pairtok forces pairs).
 int gemm_kernel_choice() {
   static int choice = -1;
   if (choice < 0) {
@@ -40,6 +41,8 @@ int gemm_kernel_choice() {
     if (v != nullptr && strcmp(v, "pair") == 0) choice = 1;
     if (v != nullptr && strcmp(v, "wt") == 0) choice = 2;
     if (v != nullptr && strcmp(v, "hybrid") == 0) choice = 3;
+    if (v != nullptr && strcmp(v, "single") == 0) choice = 4;
+    if (v != nullptr && strcmp(v, "pairtok") == 0) choice = 5;
   }
   return choice;
 }
@@ -88,7 +91,7 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t 
   if (choice == 1) return launch_grouped_gemm_pair(a, p, num_sms, stream);
   p.test_stall = take_test_stall();
   if (choice == 2 || (choice == 3 && a.epilogue != EPI_SWIGLU)) return launch_grouped_gemm_wt(a, p, num_sms, stream);
-  return launch_grouped_gemm_single(a, p, num_sms, stream);
+  return launch_grouped_gemm_single(a, p, num_sms, stream, choice == 4 ? 1 : (choice == 5 ? 2 : 0));
 }
 
 }  // namespace moe

@@ -118,7 +118,8 @@ struct TcParams;
 }
 cudaError_t launch_grouped_gemm_pair(const GemmArgs& a, const gemm::TcParams& p, int num_sms, cudaStream_t stream);
 cudaError_t launch_grouped_gemm_wt(const GemmArgs& a, const gemm::TcParams& p, int num_sms, cudaStream_t stream);
-cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& p, int num_sms, cudaStream_t stream);
+cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& p, int num_sms, cudaStream_t stream,
+                                       int pair_mode);
 cudaError_t launch_grouped_gemm_f32(const GemmArgs& a, cudaStream_t stream);
 
 // FP8-E4M3 weight slabs -> bf16 (exact)
