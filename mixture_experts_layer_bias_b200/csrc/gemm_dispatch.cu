@@ -31,8 +31,8 @@ int take_test_stall() {
 
 // Kernel choice (read once): MOE_B200_GEMM=pair or =wt selects the CTA-pair or
 // the one-CTA weights-as-M kernel, =hybrid the weights-as-M kernel for all but
-// the SwiGLU up projection; otherwise the token-rows kernel, on CTA pairs for
-// large groups (=single forces one CTA, =pairtok forces pairs).
+// the SwiGLU up projection, =pairtok the token-rows kernel on CTA pairs for
+// large groups; otherwise (or =single) the one-CTA token-rows kernel.
 int gemm_kernel_choice() {
   static int choice = -1;
   if (choice < 0) {

@@ -735,9 +735,11 @@ cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUte
 
 }  // namespace
 
-// Token-rows kernel launch; `p` is filled by the dispatcher.  pair_mode: 0 =
-// CTA pairs when the groups are large (at least 512 rows on average and some
-// group above 128), 1 = one-CTA kernel, 2 = CTA pairs.
+// Token-rows kernel launch; `p` is filled by the dispatcher.  pair_mode: 0 or
+// 1 = one-CTA kernel, 2 = CTA pairs when the groups are large (at least 512
+// rows on average and some group above 128).  In same-box A/B the pair
+// kernel was within a few percent of the one-CTA kernel and read 28% more
+// weight bytes from DRAM in the up projection, so it stays opt-in.
 cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& p, int num_sms, cudaStream_t stream,
                                        int pair_mode) {
   // A rows loaded per stage: all 128, or (every group fitting) the largest group rounded up to 16
@@ -766,7 +768,7 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
     mB1 = mB0;
   }
   const bool large = a.max_group_rows > 128 && a.max_total_rows >= int64_t(512) * a.num_groups;
-  if (bma == BM && num_sms >= 2 && (pair_mode == 2 || (pair_mode == 0 && large))) {
+  if (bma == BM && num_sms >= 2 && pair_mode == 2 && large) {
     const int64_t pbound = (a.max_total_rows / P2_BM + a.num_groups) * static_cast<int64_t>(p.n_tiles);
     const int64_t clusters = pbound < num_sms / 2 ? (pbound > 0 ? pbound : 1) : num_sms / 2;
     const int pgrid = static_cast<int>(2 * (clusters > 0 ? clusters : 1));
