@@ -12,6 +12,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "pdl.cuh"
 
 namespace moe {
 
@@ -69,6 +70,8 @@ __global__ void __launch_bounds__(256)
                        const float* __restrict__ topk_w, int64_t shared_row0, T* __restrict__ y) {
   __shared__ int32_t rows[32];
   __shared__ float gates[32];
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   if (threadIdx.x < K) {
     rows[threadIdx.x] = row_of_slot[static_cast<int64_t>(t) * K + threadIdx.x];
@@ -127,13 +130,16 @@ __global__ void dequant_e4m3_kernel(const uint4* __restrict__ q, uint4* __restri
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream) {
   if (a.S == 0) return cudaSuccess;
   if (a.S <= 256) {
+    cudaError_t err;
     if (a.act_dtype == MOE_BF16)
-      combine_cta_kernel<__nv_bfloat16><<<a.S, 256, 0, stream>>>(a.d, a.K, static_cast<const __nv_bfloat16*>(a.y_perm),
-                                                                 a.row_of_slot, a.topk_w, a.shared_row0,
-                                                                 static_cast<__nv_bfloat16*>(a.y));
+      err = launch_pdl(combine_cta_kernel<__nv_bfloat16>, dim3(a.S), dim3(256), 0, stream, a.d, a.K,
+                       static_cast<const __nv_bfloat16*>(a.y_perm), a.row_of_slot, a.topk_w, a.shared_row0,
+                       static_cast<__nv_bfloat16*>(a.y));
     else
-      combine_cta_kernel<float><<<a.S, 256, 0, stream>>>(a.d, a.K, static_cast<const float*>(a.y_perm), a.row_of_slot,
-                                                         a.topk_w, a.shared_row0, static_cast<float*>(a.y));
+      err = launch_pdl(combine_cta_kernel<float>, dim3(a.S), dim3(256), 0, stream, a.d, a.K,
+                       static_cast<const float*>(a.y_perm), a.row_of_slot, a.topk_w, a.shared_row0,
+                       static_cast<float*>(a.y));
+    if (err != cudaSuccess) return err;
     return cudaGetLastError();
   }
   const int blocks = (a.S + kCombWarps - 1) / kCombWarps;

@@ -22,6 +22,7 @@
 // GEMMs in one single-CTA kernel, and the gather with one CTA per token.
 #include "common.cuh"
 #include "kernels.h"
+#include "pdl.cuh"
 
 namespace moe {
 
@@ -253,6 +254,8 @@ __global__ void __launch_bounds__(kSmallWarps * 32)
                          int32_t* __restrict__ row_of_slot, int32_t* __restrict__ token_of_row, int64_t num_rows,
                          GroupEntry* __restrict__ g1, StatusBlock* status) {
   extern __shared__ int32_t sm[];
+  pdl_wait();
+  pdl_trigger();
   int32_t* whist = sm;                      // [32][E]
   int32_t* cnt = sm + kSmallWarps * E;      // [E]
   int32_t* ovf = cnt + E;                   // [E]
@@ -339,6 +342,8 @@ __global__ void __launch_bounds__(256)
     gather_rows_cta_kernel(int d, int K, const int32_t* __restrict__ row_of_slot, const T* __restrict__ x,
                            T* __restrict__ x_perm) {
   __shared__ int32_t rows[32];
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   if (threadIdx.x < K) rows[threadIdx.x] = row_of_slot[static_cast<int64_t>(t) * K + threadIdx.x];
   __syncthreads();
@@ -378,10 +383,10 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
   cudaError_t err;
   if (static_cast<int64_t>(a.S) * a.K <= kSmallSlots) {
     const size_t smem = sizeof(int32_t) * (kSmallWarps * a.E + 3 * a.E + 1);
-    permute_small_kernel<<<1, kSmallWarps * 32, smem, stream>>>(a.S, a.E, a.K, a.capacity, a.num_shared, a.topk_idx,
-                                                                 a.counts, a.offsets, a.row_of_slot, a.token_of_row,
-                                                                 a.num_rows, a.g1, a.status);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    err = launch_pdl(permute_small_kernel, dim3(1), dim3(kSmallWarps * 32), smem, stream, a.S, a.E, a.K, a.capacity,
+                     a.num_shared, a.topk_idx, a.counts, a.offsets, a.row_of_slot, a.token_of_row, a.num_rows, a.g1,
+                     a.status);
+    if (err != cudaSuccess || (err = cudaGetLastError()) != cudaSuccess) return err;
   } else {
     const int tpc = permute_tokens_per_chunk(a.K);
     const int nch = permute_num_chunks(a.S, a.K);
@@ -410,13 +415,14 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
   if (a.x == nullptr || a.x_perm == nullptr) return cudaSuccess;
   if (a.S <= 256) {
 #define MOE_GATHER_CTA(T)                                                                                    \
-  gather_rows_cta_kernel<T><<<a.S, 256, 0, stream>>>(a.d, a.K, a.row_of_slot, static_cast<const T*>(a.x),   \
-                                                      static_cast<T*>(a.x_perm))
+  err = launch_pdl(gather_rows_cta_kernel<T>, dim3(a.S), dim3(256), 0, stream, a.d, a.K,                       \
+                   static_cast<const int32_t*>(a.row_of_slot), static_cast<const T*>(a.x), static_cast<T*>(a.x_perm))
     if (a.act_dtype == MOE_BF16)
       MOE_GATHER_CTA(__nv_bfloat16);
     else
       MOE_GATHER_CTA(float);
 #undef MOE_GATHER_CTA
+    if (err != cudaSuccess) return err;
     return cudaGetLastError();
   }
   const int gblocks = (a.S + kPermWarps - 1) / kPermWarps;

@@ -18,6 +18,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "pdl.cuh"
 
 namespace moe {
 
@@ -308,6 +309,8 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
     route_token_cta_kernel(int d, const T* __restrict__ x, const T* __restrict__ w_router,
                            const float* __restrict__ router_bias, SelectParams p) {
   __shared__ float part[kRouteWarps][EMAX];
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = lane_id();
   constexpr int V = Vec16<T>::N;
@@ -455,11 +458,12 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
     // decode-sized batches: a CTA per token; otherwise a warp per token
     const bool per_cta = a.S <= 512;
     const int g = per_cta ? a.S : blocks;
+    cudaError_t err = cudaSuccess;
 #define MOE_ROUTE_LAUNCH(T, EM)                                                                                \
   do {                                                                                                         \
     if (per_cta)                                                                                               \
-      route_token_cta_kernel<T, EM><<<g, kRouteWarps * 32, 0, stream>>>(                                       \
-          a.d, static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);              \
+      err = launch_pdl(route_token_cta_kernel<T, EM>, dim3(g), dim3(kRouteWarps * 32), 0, stream, a.d,              \
+                       static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);      \
     else                                                                                                       \
       route_fused_kernel<T, EM><<<g, kRouteWarps * 32, 0, stream>>>(                                           \
           a.S, a.d, static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);         \
@@ -476,6 +480,7 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
         MOE_ROUTE_LAUNCH(float, 32);
     }
 #undef MOE_ROUTE_LAUNCH
+    if (err != cudaSuccess) return err;
     return cudaGetLastError();
   }
   if (logits == nullptr) {
