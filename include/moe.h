@@ -14,6 +14,12 @@
  *   moe_grouped_ffn  every expert's FFN over its rows as one grouped GEMM
  *   moe_combine      gate-weighted sum back into token order
  *
+ * Around them: moe_reroute (over-capacity re-routing between two
+ * permutations), moe_update_sel_bias (sliding-window selection-bias update),
+ * moe_quantize_rows_e4m3 (the W8A8 activation quantiser on its own),
+ * moe_permute_static (moe_permute without a workspace), and the workspace /
+ * status helpers.
+ *
  * Conventions for every call:
  *  - Tensor pointers are DEVICE pointers, row-major, owned by the caller.
  *    The library never allocates device or host memory and never
@@ -225,7 +231,13 @@ moe_status moe_permute_static(const moe_desc *desc, const void *x, const int32_t
  *   y_perm [R + ns*S][d] act_dtype: row r = E_{expert(r)}(x_perm[r]); rows
  *     R .. R+S-1 hold the shared expert's output for token 0 .. S-1.
  *   The hidden activations live in the workspace.  Rows outside any group
- *   (unused capacity rows) are not written.
+ *   (unused capacity rows) are not written.  With a capacity, each expert's
+ *   overflow rows are processed in the same GEMM launches, right after its
+ *   primary rows.  E4M3 weights with act_quant = 0 are decoded exactly to
+ *   bf16 into the workspace on every call (the channel scales multiply the
+ *   fp32 accumulators); with act_quant = 1 the A rows of both GEMMs (x_perm
+ *   rows and, for the shared expert, x rows; then the hidden rows) are
+ *   quantised per row into the workspace and the GEMMs read E4M3 codes.
  */
 moe_status moe_grouped_ffn(const moe_desc *desc, const moe_weights *w, const void *x_perm,
                            const int32_t *offsets, const void *x, void *y_perm, void *ws, size_t ws_bytes,
