@@ -34,6 +34,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -137,7 +138,9 @@ class ClockSampler:
 
     def __init__(self, device_index):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        # raw samples: MOE_B200_CLOCKS_DIR if set, else the system temp directory
+        out_dir = os.environ.get("MOE_B200_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"moe_b200_clocks_rank{device_index}.csv")
         try:
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
             gid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
