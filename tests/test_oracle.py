@@ -619,3 +619,30 @@ def test_gate_weights_match_selection():
             idx, w = O.select_experts(logits, 3, fn, renorm)
             scores, _, _ = O.selection_keys(logits, fn)
             np.testing.assert_allclose(O.gate_weights(scores, idx, fn, renorm), w, rtol=0, atol=0)
+
+
+def test_selection_margin_hand_computed_and_stability():
+    """The margin is the gap between the K-th and (K+1)-th candidate keys
+    (and between the last kept and first dropped group score with groups);
+    any perturbation of the keys smaller than half of it leaves the selection
+    unchanged, and one slightly larger can change it."""
+    l = np.array([[3.0, 1.0, 2.0, 0.5]], np.float32)
+    assert O.selection_margin(l, 1)[0] == 1.0              # 3 vs 2
+    assert O.selection_margin(l, 2)[0] == 1.0              # 2 vs 1
+    assert O.selection_margin(l, 3)[0] == 0.5              # 1 vs 0.5
+    # groups of 2: group sums (3+1, 2+0.5) = (4, 2.5): keep 1 group -> margin min(1.5, key gap inside)
+    assert O.selection_margin(l, 1, num_groups=2, topk_groups=1)[0] == 1.5
+    rng = np.random.default_rng(23)
+    logits = rng.normal(size=(400, 16)).astype(np.float32)
+    idx, _ = O.select_experts(logits, 4)
+    m = O.selection_margin(logits, 4)
+    noise = (rng.uniform(-1, 1, size=logits.shape) * (0.49 * m[:, None])).astype(np.float32)
+    idx2, _ = O.select_experts((logits.astype(np.float64) + noise).astype(np.float32), 4)
+    assert (np.sort(idx, 1) == np.sort(idx2, 1)).all()
+    # closing the gap of one token flips its K-th choice
+    t = int(np.argmin(m))
+    order = np.argsort(-logits[t])
+    bumped = logits.copy()
+    bumped[t, order[4]] += np.float32(m[t] * 1.01)
+    idx3, _ = O.select_experts(bumped, 4)
+    assert set(idx3[t].tolist()) != set(idx[t].tolist())
