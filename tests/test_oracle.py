@@ -646,3 +646,67 @@ def test_selection_margin_hand_computed_and_stability():
     bumped[t, order[4]] += np.float32(m[t] * 1.01)
     idx3, _ = O.select_experts(bumped, 4)
     assert set(idx3[t].tolist()) != set(idx[t].tolist())
+
+
+def _reroute_in_rounds(topk_idx, keys, cand, capacity, chunk):
+    """The round structure the GPU assignment uses, restated on the host: every
+    slot of a chunk picks against the room at the round's start (a token's
+    slots in order, each excluding the earlier picks), picks are ranked per
+    expert in slot order, and the longest prefix whose picks fit is
+    committed."""
+    idx = np.array(topk_idx, dtype=np.int32, copy=True)
+    S, K = idx.shape
+    E = keys.shape[1]
+    P = O.expert_permutation(idx, E, capacity)
+    ex = np.nonzero(P["row_of_slot"] >= E * capacity)[0]
+    room = capacity - np.minimum(O.expert_counts(idx, E), capacity)
+    base = 0
+    rounds = 0
+    while base < len(ex):
+        m = min(chunk, len(ex) - base)
+        picks, held_t, held = [], -1, None
+        for i in range(m):
+            t = ex[base + i] // K
+            if t != held_t:
+                held_t, held = t, set(idx[t].tolist())
+            ok = [e for e in range(E) if room[e] > 0 and e not in held and cand[t, e] and keys[t, e] > -np.inf]
+            b = max(ok, key=lambda e: (keys[t, e], -e)) if ok else -1
+            picks.append(b)
+            if b >= 0:
+                held.add(b)
+        seen = np.zeros(E, np.int64)
+        p = m
+        for i, b in enumerate(picks):
+            if b >= 0:
+                if seen[b] >= room[b]:
+                    p = i
+                    break
+                seen[b] += 1
+        assert p >= 1
+        for i in range(p):
+            if picks[i] >= 0:
+                s = ex[base + i]
+                idx[s // K, s % K] = picks[i]
+                room[picks[i]] -= 1
+        base += p
+        rounds += 1
+    return idx, rounds
+
+
+@pytest.mark.parametrize("chunk", [1, 4, 16, 1024])
+def test_reroute_rounds_equal_the_serial_assignment(chunk):
+    """The committed prefix of every round is the serial result: the round
+    structure reproduces reroute_over_capacity exactly, for any chunk size,
+    with at most ceil(excess / chunk) + E rounds."""
+    rng = np.random.default_rng(24 + chunk)
+    for trial in range(6):
+        S, E, K = int(rng.integers(50, 400)), int(rng.choice([8, 16, 32])), int(rng.integers(1, 5))
+        keys = (rng.normal(size=(S, E)) + 1.5 * rng.normal(size=E)[None, :]).astype(np.float32)
+        cand = rng.random((S, E)) > 0.1
+        idx, _ = O.select_experts(np.where(cand, keys, -np.inf).astype(np.float32), K)
+        C = max(1, int(np.ceil(rng.uniform(0.7, 1.3) * S * K / E)))
+        ref, _ = O.reroute_over_capacity(idx, keys, cand, C)
+        got, rounds = _reroute_in_rounds(idx, keys, cand, C, chunk)
+        np.testing.assert_array_equal(got, ref)
+        n_ex = int((O.expert_permutation(idx, E, C)["row_of_slot"] >= E * C).sum())
+        assert rounds <= -(-n_ex // chunk) + E + 1
