@@ -212,3 +212,21 @@ def test_reroute_workspace_and_argument_errors():
     assert L.moe_reroute(ctypes.byref(d), p, p, p, None, ws, n, None) == ops.MOE_ERR_INVALID_ARG
     assert L.moe_reroute(ctypes.byref(d), p, p, p, p, ws, n - 256, None) == ops.MOE_ERR_WORKSPACE
     assert L.moe_reroute(ctypes.byref(d), p, p, p, p, None, n, None) == ops.MOE_ERR_WORKSPACE
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/moe.h is a C header: a C99 translation unit that includes it and
+    takes the address of every entry point compiles without warnings."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    names = header_functions()
+    src = tmp_path / "use_header.c"
+    body = "\n".join(f"  p[{i}] = (fn)&{n};" for i, n in enumerate(names))
+    src.write_text('#include "moe.h"\ntypedef void (*fn)(void);\nvoid touch(fn *p) {\n' + body + '\n}\n')
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-c", str(src), "-I",
+                        os.path.join(ROOT, "include"), "-o", str(tmp_path / "use_header.o")],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
