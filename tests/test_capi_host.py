@@ -230,3 +230,17 @@ def test_header_is_plain_c(tmp_path):
                         os.path.join(ROOT, "include"), "-o", str(tmp_path / "use_header.o")],
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_binding_argument_counts_match_the_header():
+    """Every ctypes prototype in ops.py has as many arguments as the C
+    prototype in include/moe.h."""
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    protos = dict(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S))
+    L = ops.lib()
+    assert set(protos) == set(ops.EXPORTED)
+    for name, args in protos.items():
+        args = args.strip()
+        n = 0 if args in ("", "void") else args.count(",") + 1
+        assert len(getattr(L, name).argtypes) == n, name
