@@ -244,3 +244,19 @@ def test_binding_argument_counts_match_the_header():
         args = args.strip()
         n = 0 if args in ("", "void") else args.count(",") + 1
         assert len(getattr(L, name).argtypes) == n, name
+
+
+def _struct_fields(text, name):
+    bodies = dict((n, b) for b, n in re.findall(r"typedef struct \{([^{}]*)\}\s*(\w+)\s*;", text))
+    body = bodies[name]
+    return [m.group(1) for m in re.finditer(r"\**\s*([a-z_0-9]+)\s*;", body)]
+
+
+def test_struct_layouts_match_the_header():
+    """moe_desc and moe_weights as ctypes structures list the header's fields
+    in the header's order (int32 and pointer members only)."""
+    text = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "moe.h")).read(), flags=re.S)
+    assert _struct_fields(text, "moe_desc") == list(ops.DESC_FIELDS)
+    assert _struct_fields(text, "moe_weights") == list(ops.WEIGHT_FIELDS)
+    assert ctypes.sizeof(ops.MoeDesc) == 4 * len(ops.DESC_FIELDS)
+    assert ctypes.sizeof(ops.MoeWeights) == 8 * len(ops.WEIGHT_FIELDS)
