@@ -260,3 +260,27 @@ def test_struct_layouts_match_the_header():
     assert _struct_fields(text, "moe_weights") == list(ops.WEIGHT_FIELDS)
     assert ctypes.sizeof(ops.MoeDesc) == 4 * len(ops.DESC_FIELDS)
     assert ctypes.sizeof(ops.MoeWeights) == 8 * len(ops.WEIGHT_FIELDS)
+
+
+def test_product_path_never_touches_the_oracle():
+    """The library and its binding import, read and call nothing under
+    oracle/ (only tests, the smoke check and the benchmark's CPU legs may)."""
+    pkg = os.path.join(ROOT, "mixture_experts_layer_bias_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                where = os.path.join(dirpath, f)
+                assert "moe_oracle" not in text and "oracle/" not in text, where
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, flags=re.M), where
+
+
+def test_missing_library_fails_loudly():
+    """No CPU fallback: without the built library the first call raises."""
+    import subprocess
+    import sys
+    code = ("from mixture_experts_layer_bias_b200 import ops\n"
+            "try:\n    ops.lib()\nexcept RuntimeError as e:\n    print('raised', e)\n")
+    env = dict(os.environ, MOE_B200_LIB=os.path.join(ROOT, "no_such_library.so"))
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True, text=True)
+    assert "raised" in r.stdout, (r.stdout, r.stderr)
