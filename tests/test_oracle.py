@@ -710,3 +710,23 @@ def test_reroute_rounds_equal_the_serial_assignment(chunk):
         np.testing.assert_array_equal(got, ref)
         n_ex = int((O.expert_permutation(idx, E, C)["row_of_slot"] >= E * C).sum())
         assert rounds <= -(-n_ex // chunk) + E + 1
+
+
+def test_skew_recipe_gives_max_over_mean_near_four():
+    """The skewed FP8 workload's router offsets (scale SKEW_OFFSET_SCALE, the
+    value tests/golden/calibrate_skew.py finds) give a max/mean expert load of
+    about 4 under the oracle's routing of the full-size inputs, drawn on the
+    CPU (the top of the 3-5 range of jsqmd.com chapter 11, 11.2.3)."""
+    import torch
+    from mixture_experts_layer_bias_b200 import synthetic as syn
+    cfg = syn.CONFIGS["fp8_skew_capacity"]
+    x = syn.make_inputs(cfg, "cpu", seed=0, x_only=True)["x"].float().numpy()
+    cpu = torch.device("cpu")
+    w_r = syn._normal((cfg.E, cfg.d), 1.0 / cfg.d, syn._gen(cpu, 0, 2), cpu, torch.bfloat16).float().numpy()
+    rb = syn.router_offsets(cfg, 0).numpy().astype(np.float64)
+    logits = O.router_logits(x.astype(np.float64), w_r.astype(np.float64), rb)
+    idx, _ = O.select_experts(logits, cfg.K)
+    ratio = O.load_stats(O.expert_counts(idx, cfg.E), cfg.K, cfg.S)["max_over_mean"]
+    assert 3.8 <= ratio <= 4.2, ratio
+    # and the capacity of 1.25 S K / E really overflows on the hot experts
+    assert cfg.capacity == syn.capacity_for(cfg.S, cfg.K, cfg.E) and ratio * cfg.S * cfg.K / cfg.E > cfg.capacity
