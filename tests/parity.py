@@ -2,7 +2,6 @@
 oracle on the same seeded inputs, and compare."""
 from __future__ import annotations
 
-import math
 
 import numpy as np
 import torch

@@ -6,7 +6,6 @@ tolerances: fp32 max-abs <= 1e-4 * max|ref|, bf16 relative L2 <= 1e-2, FP8
 weights relative L2 <= 3e-2 against the oracle on the same decoded weights.
 Sizes span several tiles and ragged tails.
 """
-import math
 
 import numpy as np
 import pytest
