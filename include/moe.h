@@ -108,7 +108,7 @@ typedef enum { MOE_ACT_GELU = 0, MOE_ACT_SWIGLU = 1 } moe_act;
  *     activation scaling is this library's reading.  Needs BF16 act, E4M3
  *     weights, SWIGLU, d and h multiples of 16.
  *   reroute: 0 = none; 1 = over-capacity re-routing (needs capacity > 0;
- *     jsqmd.com 11.3.3 "专家丢弃": an overloaded expert's excess tokens go
+ *     jsqmd.com 11.3.3, expert-dropping paragraph: an overloaded expert's excess tokens go
  *     to their next-best expert).  Each expert keeps its first C slots in
  *     (token, k) order; the excess slots, in (token, k) order, move to the
  *     candidate expert (within the token's kept groups) with the highest
@@ -185,7 +185,7 @@ moe_status moe_route(const moe_desc *desc, const moe_weights *w, const void *x, 
                      int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes, void *stream);
 
 /*
- * Histogram, prefix scan and stable permutation (11.2.1 "数据重排").
+ * Histogram, prefix scan and stable permutation (11.2.1, data-regrouping paragraph).
  *   topk_idx int32 [S][K] -> counts int32 [E];
  *   offsets int32 [E+1] (exclusive prefix of counts), with capacity
  *     [2(E+1)]: the first E+1 as before, then the exclusive prefix of the
@@ -282,7 +282,7 @@ moe_status moe_quantize_rows_e4m3(const void *x, int64_t rows, int32_t d, uint8_
 
 /*
  * Gate-weighted combine back into token order (11.3.1 step 6; plumephp.com
- * worked example "结果按得分加权求和").
+ * "MoE 混合专家推理", worked-example block: the gate-weighted sum).
  *   y[t] = sum_{k=0..K-1} topk_w[t][k] * y_perm[row_of_slot[t*K+k]]
  *          (+ y_perm[R + t] when num_shared = 1), fp32 sums in k order.
  *   y [S][d] act_dtype.
@@ -302,8 +302,8 @@ moe_status moe_layer_forward(const moe_desc *desc, const moe_weights *w, const v
 /*
  * Sliding-window expert load and the aux-loss-free selection-bias update
  * (ybb.press "MoE 推理工程深层实战" 2.3: the bias added to the selection keys
- * is recomputed from a sliding-window token count, `TokenWindowCounter(
- * window_size=1000)`, so routing is steered without gradients).  The page
+ * is recomputed from a token counter over a sliding window of 1000 tokens,
+ * so routing is steered without gradients).  The page
  * prints no update rule; this call applies, per expert, in float32,
  *     sel_bias[e] += gamma * sign(mean - count_e),
  * count_e = (token, k) slots routed to e among the last `window_tokens`

@@ -2,7 +2,7 @@
 //
 // ybb.press "MoE 推理工程深层实战" 2.3: DeepSeek-V3-style routing adds a bias to
 // the selection keys and recomputes it from a sliding-window token count
-// (`TokenWindowCounter(window_size=1000)`), steering the routing distribution
+// over a window of 1000 tokens, steering the routing distribution
 // without gradients.  The page does not print the update rule; the one used
 // here moves each expert's bias against its deviation from the mean load:
 //

@@ -19,6 +19,8 @@
 // that overlap on the GPU (different streams, or different host threads
 // without ordering) race on the array.  Data problems are not reported
 // through a status block here: an out-of-range expert id gets row -1.
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -30,15 +32,21 @@ constexpr int kStaticHistEntries = 65536;  // 256 KB
 __device__ __align__(256) int32_t g_permute_hist[kStaticHistEntries];
 
 // Device address of g_permute_hist on the current device (looked up once per
-// device ordinal; returns nullptr if the lookup fails).
+// device ordinal; returns nullptr if the lookup fails).  Host threads may make
+// their first calls concurrently: each cache entry is an atomic pointer, and
+// a thread that finds it empty looks the address up itself (every thread gets
+// the same value for a device, so the relaxed store of either one is right).
 int32_t* static_hist_for_current_device() {
-  static int32_t* cache[64] = {};
+  static std::atomic<int32_t*> cache[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
-  if (dev < 64 && cache[dev] != nullptr) return cache[dev];
+  if (dev >= 0 && dev < 64) {
+    int32_t* known = cache[dev].load(std::memory_order_relaxed);
+    if (known != nullptr) return known;
+  }
   void* p = nullptr;
   if (cudaGetSymbolAddress(&p, g_permute_hist) != cudaSuccess || p == nullptr) return nullptr;
-  if (dev < 64) cache[dev] = static_cast<int32_t*>(p);
+  if (dev >= 0 && dev < 64) cache[dev].store(static_cast<int32_t*>(p), std::memory_order_relaxed);
   return static_cast<int32_t*>(p);
 }
 

@@ -1,6 +1,6 @@
 // Over-capacity re-routing of excess slots to the next-best expert.
 //
-// jsqmd.com "第11章 MoE模型推理" 11.3.3 ("专家丢弃"): when an expert is
+// jsqmd.com "第11章 MoE模型推理" 11.3.3 (expert-dropping paragraph): when an expert is
 // overloaded, the tokens above its share are routed again to their next-best
 // expert.  Reading taken (the page gives one sentence): every expert keeps its
 // first C slots in (token, k) order -- the primary rows of the capacity-bounded

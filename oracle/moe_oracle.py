@@ -19,14 +19,14 @@ extracted web pages about MoE inference:
   - 11.3.1, step 6 of the expert-parallel layer: weighted sum of the K
     expert outputs by their top-k probabilities.
 * ybb.press, "MoE 推理工程深层实战":
-  - 2.2 "Token Dropping + Overflow Buffering": tokens above a capacity go to an
-    overflow buffer and are processed later, none dropped;
+  - 2.2 (expert-parallel dispatch, capacity paragraph): tokens above a
+    capacity go to an overflow buffer and are processed later, none dropped;
   - 2.3 "DeepSeek-V3 的 256 专家路由机制": aux-loss-free bias that steers
     selection only, node(group)-limited routing: sum of biased scores per
     group, top-2 groups, top-8 experts inside them.
 * plumephp.com, "MoE 混合专家推理", routing worked example ("路由打分示意"):
   scores e0 .55, e3 .30, e5 .08, e7 .03 -> top-2 = {e0, e3}, output
-  .55*e0(x) + .30*e3(x), "normalised weighting".
+  .55*e0(x) + .30*e3(x), marked as a normalised weighting.
 
 Readings taken where the pages are silent or disagree (each is listed, with
 its reason, in the design notes):
@@ -219,8 +219,12 @@ def _order_desc(keys: np.ndarray) -> np.ndarray:
 
 
 def group_sums_f32(v: np.ndarray) -> np.ndarray:
-    """Group scores: float32 halving-tree sums along the last axis (see
-    ``group_sum_f32``), vectorised over the leading axes."""
+    """Group scores (ybb.press 2.3: a group's score is the sum of its
+    members' biased scores) as float32 sums along the last axis, vectorised
+    over the leading axes.  The order of the float32 additions is fixed: a
+    power-of-two number n of members is halved repeatedly, member j adding
+    member j + n/2 (for 32 members: strides 16, 8, 4, 2, 1), until one value
+    is left."""
     v = np.asarray(v, dtype=np.float32)
     n = v.shape[-1]
     assert n & (n - 1) == 0, "group size must be a power of two"
@@ -229,20 +233,6 @@ def group_sums_f32(v: np.ndarray) -> np.ndarray:
         v = np.add(v[..., :h], v[..., h:], dtype=np.float32)
         n = h
     return v[..., 0]
-
-
-def group_sum_f32(v: np.ndarray) -> np.float32:
-    """Sum of a power-of-two number of float32 values by repeated halving:
-    v <- v[:n/2] + v[n/2:] in float32 until one value is left.  This fixes the
-    order of the float32 additions of a group score."""
-    v = np.asarray(v, dtype=np.float32)
-    n = len(v)
-    assert n & (n - 1) == 0, "group size must be a power of two"
-    while n > 1:
-        h = n // 2
-        v = np.add(v[:h], v[h:], dtype=np.float32)
-        n = h
-    return np.float32(v[0])
 
 
 def select_experts(
@@ -423,7 +413,7 @@ def expert_permutation(topk_idx: np.ndarray, num_experts: int, capacity: int = 0
 
 
 def reroute_over_capacity(topk_idx, keys, cand, capacity: int):
-    """Over-capacity re-routing (jsqmd.com chapter 11, 11.3.3, "专家丢弃":
+    """Over-capacity re-routing (jsqmd.com chapter 11, 11.3.3, expert-dropping paragraph:
     when an expert is overloaded, its excess tokens go to their next-best
     expert).  The page gives the rule in one sentence; the reading taken:
 
@@ -638,7 +628,7 @@ class WindowBias:
     """Sliding-window expert counts and the selection-bias update of
     ybb.press 2.3 (aux-loss-free routing: the bias added to the selection
     keys is recomputed from a sliding window of recent tokens' expert
-    choices, `TokenWindowCounter(window_size=1000)`).
+    choices; the page's window holds 1000 tokens).
 
     The page does not print the update rule.  Reading taken: after each
     batch, b_e <- b_e + gamma * sign(mean - count_e) in float32, where count_e

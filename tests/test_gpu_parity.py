@@ -121,8 +121,9 @@ def test_route_worked_example():
                                     ("dsv3_grouped", 256)])
 def test_route_computed_logits_within_margin(name, S):
     """The router computes its own logits (fused kernel for E <= 32, logits
-    kernel otherwise); indices must agree with the oracle wherever the
-    selection margin is >= 1e-4 (excluded tokens are counted)."""
+    GEMM otherwise); indices must agree with the oracle wherever the
+    selection margin is >= 1e-4 (excluded tokens are counted), and the gates
+    within the fp32 tolerance."""
     cfg = syn.scaled(syn.CONFIGS[name], S=S)
     # routing only reads x and the router; small experts keep the draw cheap
     inp = syn.make_inputs(syn.scaled(cfg, h=8), "cuda", seed=1)
@@ -137,7 +138,8 @@ def test_route_computed_logits_within_margin(name, S):
     keep = margin >= 1e-4
     assert keep.sum() >= 0.9 * S
     np.testing.assert_array_equal(idx.cpu().numpy()[keep], ridx[keep])
-    assert max_abs_rel(gw.cpu().numpy()[keep], rw[keep]) <= 1e-3
+    # the gates are fp32 outputs: the fp32 contract, max-abs <= 1e-4 * max|ref|
+    assert max_abs_rel(gw.cpu().numpy()[keep], rw[keep]) <= F32_MAXABS_REL
     print(f"{name}: excluded {int((~keep).sum())} of {S} tokens (margin < 1e-4)")
 
 

@@ -152,14 +152,63 @@ def test_grouped_selection_brute_force_dyadic():
         np.testing.assert_allclose(w[0], sk / sk.sum(), rtol=1e-12)
 
 
-def test_group_sum_order_is_halving_tree():
-    """The float32 group score adds members (j, j+16), then (j, j+8), ...: for
-    values where order matters, compare with the hand-written tree of 4."""
-    v = np.array([1.0, 1e-8, -1.0, 1e-8], dtype=np.float32)
-    # halving: (1 + -1) , (1e-8 + 1e-8) -> 0 + 2e-8
-    assert O.group_sum_f32(v) == np.float32(np.float32(1e-8) + np.float32(1e-8))
-    # a left-to-right sum would give ((1 + 1e-8) - 1) + 1e-8 = 1e-8 in float32
-    assert O.group_sum_f32(v) != np.float32(1e-8)
+def _group_row_with_cancellation():
+    """32 float32 members: 2**25 at member 0, -2**25 at member 16, and
+    c = float32(0.7) (not dyadic) everywhere else."""
+    v = np.full(32, np.float32(0.7), dtype=np.float32)
+    v[0], v[16] = np.float32(2.0 ** 25), np.float32(-2.0 ** 25)
+    return v
+
+
+def test_group_sums_f32_is_the_halving_tree():
+    """The group score of the grouped selection adds member j + 16 to member
+    j, then j + 8, j + 4, j + 2, j + 1 (a fixed float32 order).  On the row
+    of ``_group_row_with_cancellation`` that order gives exactly 21, by hand:
+    with c = 11744051 * 2**-24 (float32(0.7)),
+      stride 16: 2**25 - 2**25 = 0 and fifteen sums 2c (exact);
+      stride 8:  0 + 2c = 2c and seven sums 4c (exact);
+      stride 4:  2c + 4c = 70464306 * 2**-24, rounded to the 2**-21 grid
+                 -> 70464304 * 2**-24; three sums 8c (exact);
+      stride 2:  70464304 + 93952408 = 164416712 (units of 2**-24), a tie on
+                 the 2**-20 grid -> even -> 164416704; one sum 16c;
+      stride 1:  164416704 + 187904816 = 352321520, a tie on the 2**-19 grid
+                 -> even -> 352321536 = 21 * 2**24, i.e. 21.0.
+    A left-to-right sum or adjacent pairing (j with j + 1) gives other
+    float32 values on the same row, so either slip fails here."""
+    v = _group_row_with_cancellation()
+    assert O.group_sums_f32(v) == np.float32(21.0)
+    # vectorised over leading axes: the same row in a [2, 3, 32] batch
+    batch = np.broadcast_to(v, (2, 3, 32)).copy()
+    batch[1, 2] = np.float32(0.5)  # 32 * 0.5 = 16 exactly in any order
+    got = O.group_sums_f32(batch)
+    assert got.shape == (2, 3)
+    assert got[1, 2] == np.float32(16.0)
+    assert np.all(np.delete(got.reshape(-1), 5) == np.float32(21.0))
+    # the row discriminates: the two other plausible orders differ from 21
+    ltr = np.float32(0.0)
+    for m in v:
+        ltr = np.float32(ltr + m)
+    adj = v.copy()
+    while len(adj) > 1:
+        adj = np.add(adj[0::2], adj[1::2], dtype=np.float32)
+    assert ltr != np.float32(21.0) and adj[0] != np.float32(21.0) and ltr != adj[0]
+
+
+def test_group_limited_selection_uses_the_halving_order():
+    """Two groups of 32 softmax keys, keep one group, top-1.  Group 0 holds
+    the cancellation row (halving sum 21, see above); group 1 holds 32 keys
+    0.609375 (exact dyadic sum 19.5 in any order).  The halving order keeps
+    group 0, whose best key (2**25, expert 0) wins; a left-to-right or
+    adjacent-pair group sum (both below 19.5 on this row) would keep group 1
+    and pick expert 32."""
+    keys = np.concatenate([_group_row_with_cancellation(), np.full(32, np.float32(0.609375))])[None, :]
+    idx, w = O.select_experts(keys, 1, num_groups=2, topk_groups=1)
+    assert idx.tolist() == [[0]]
+    np.testing.assert_allclose(w, [[1.0]])
+    # and when group 1's exact sum is above 21 (0.671875 * 32 = 21.5), group 1 wins
+    keys2 = np.concatenate([_group_row_with_cancellation(), np.full(32, np.float32(0.671875))])[None, :]
+    idx2, _ = O.select_experts(keys2, 1, num_groups=2, topk_groups=1)
+    assert idx2.tolist() == [[32]]
 
 
 # ----------------------------------------------------------------------------
@@ -229,6 +278,33 @@ def test_permutation_invariants(capacity):
         for e in range(E):
             rows = ros[flat == e]
             assert np.all((rows >= off[e]) & (rows < off[e + 1]))
+
+
+def test_overflow_region_is_expert_major():
+    """ybb.press 2.2 (overflow buffering), with the layout read as: the E*C
+    primary rows first, then the overflow rows expert by expert, each
+    expert's in slot order.  Hand-built case, E = 3, C = 1, K = 2:
+        token 0 -> (e0, e2), token 1 -> (e2, e0), token 2 -> (e1, e2)
+    slots 0..5 = e0, e2, e2, e0, e1, e2; counts (2, 1, 3).
+    Primary rows: e0 keeps slot 0 (row 0), e1 slot 4 (row 1), e2 slot 1
+    (row 2).  Overflow counts (1, 0, 2) -> overflow offsets (0, 1, 1, 3):
+    e0's excess slot 3 -> row 3 + 0 = 3; e2's excess slots 2, 5 -> rows
+    3 + 1 = 4 and 5.  A token-major overflow layout would put slot 2 at row 3
+    and slot 3 at row 4 instead."""
+    idx = np.array([[0, 2], [2, 0], [1, 2]], dtype=np.int32)
+    P = O.expert_permutation(idx, 3, capacity=1)
+    assert P["counts"].tolist() == [2, 1, 3]
+    assert P["prim_counts"].tolist() == [1, 1, 1]
+    assert P["ovf_counts"].tolist() == [1, 0, 2]
+    assert P["ovf_offsets"].tolist() == [0, 1, 1, 3]
+    assert P["num_rows"] == 3 * 1 + 3 * 2
+    assert P["row_of_slot"].tolist() == [0, 2, 4, 3, 1, 5]
+    assert P["token_of_row"].tolist() == [0, 2, 0, 1, 1, 2, -1, -1, -1]
+    # without capacity: plain stable grouping, offsets (0, 2, 3, 6)
+    Q = O.expert_permutation(idx, 3)
+    assert Q["offsets"].tolist() == [0, 2, 3, 6]
+    assert Q["row_of_slot"].tolist() == [0, 3, 4, 1, 2, 5]
+    assert Q["token_of_row"].tolist() == [0, 1, 2, 0, 1, 2]
 
 
 def test_load_stats_uniform_and_skewed():
