@@ -116,6 +116,14 @@ typedef enum { MOE_ACT_GELU = 0, MOE_ACT_SWIGLU = 1 } moe_act;
  *     (ties to the lower index); a slot with no such expert keeps its expert
  *     and its overflow row.  Gates are then recomputed over the final
  *     experts.  See moe_reroute.
+ *   temperature: softmax temperature tau of soft routing (jsqmd.com 11.3.3,
+ *     soft-routing equation y = sum_i softmax(s/tau)_i E_i(x)).  0 means
+ *     tau = 1.  With score_fn = MOE_SCORE_SOFTMAX every logit l (router bias
+ *     included) becomes z = l / tau, one float32 division; z is the gate
+ *     source and, plus sel_bias, the selection key.  A finite tau > 0;
+ *     tau != 1 with MOE_SCORE_SIGMOID is MOE_ERR_UNSUPPORTED (the page gives
+ *     the temperature for the softmax router only).  K = E, renormalize = 1
+ *     and tau give the page's soft routing.
  * Supported: (F32 act, F32 weights, GELU) with E <= 32 on the SIMT path;
  * (BF16 act, BF16 or E4M3 weights, SWIGLU or GELU; E4M3 with SWIGLU only)
  * on the tensor-core path.  E <= 256, K <= min(E, 32), d and h multiples
@@ -138,6 +146,7 @@ typedef struct {
   int32_t capacity;
   int32_t act_quant;
   int32_t reroute;
+  float temperature;
 } moe_desc;
 
 /* Weights, all DEVICE pointers (see layouts above).  Unused ones may be
@@ -300,6 +309,24 @@ moe_status moe_layer_forward(const moe_desc *desc, const moe_weights *w, const v
                              void *stream);
 
 /*
+ * moe_layer_forward that also records caller-created CUDA events on `stream`
+ * between its stages, so a caller can time each stage of the real layer call
+ * (the same launches as moe_layer_forward, plus the event records).
+ * events: MOE_NUM_STAGE_EVENTS cudaEvent_t handles passed as void*, each one
+ * NULL (skipped) or an event created on the current device:
+ *   [0] before routing             [1] after routing (and re-routing)
+ *   [2] after the permutation       [3] before the up-projection GEMM (after
+ *   any E4M3 weight decode or activation quantisation of the FFN)
+ *   [4] after the up-projection GEMM   [5] before the down-projection GEMM
+ *   [6] after the down-projection GEMM [7] after the combine.
+ * Errors as moe_layer_forward; MOE_ERR_CUDA when an event record fails.
+ */
+#define MOE_NUM_STAGE_EVENTS 8
+moe_status moe_layer_forward_timed(const moe_desc *desc, const moe_weights *w, const void *x, void *y,
+                                   int32_t *topk_idx, float *topk_w, int32_t *counts, void *ws, size_t ws_bytes,
+                                   void *stream, void *const *events);
+
+/*
  * Sliding-window expert load and the aux-loss-free selection-bias update
  * (ybb.press "MoE 推理工程深层实战" 2.3: the bias added to the selection keys
  * is recomputed from a token counter over a sliding window of 1000 tokens,
@@ -322,6 +349,39 @@ moe_status moe_bias_state_init(void *state, size_t state_bytes, void *stream);
 moe_status moe_update_sel_bias(const moe_desc *desc, const int32_t *topk_idx, int32_t window_tokens, float gamma,
                                void *state, size_t state_bytes, float *sel_bias, int32_t *window_counts,
                                void *stream);
+
+/*
+ * Load report of one routing, computed on the device from the per-expert
+ * counts (moe_permute's or moe_layer_forward's counts output).  It gathers
+ * what the pages ask to watch: the max/mean expert load (jsqmd.com 11.2.3,
+ * 1 when balanced, 3-5 in practice), the standard deviation of the expert
+ * loads and the token drop rate (ybb.press "MoE 推理工程深层实战" 1.2, table
+ * of inference metrics), the rows above the capacity (ybb.press 2.2) and the
+ * routing histogram itself (plumephp.com "MoE 混合专家推理", verification
+ * block).
+ *   counts int32 [E] DEVICE; stats double [MOE_NUM_LOAD_STATS] DEVICE,
+ *   caller-owned, written as
+ *     [MOE_LS_MAX_OVER_MEAN] max_e counts[e] / mean   (0 when S*K = 0)
+ *     [MOE_LS_STD]           sqrt(sum_e (counts[e] - mean)^2 / E)
+ *     [MOE_LS_MEAN]          mean = S*K / E
+ *     [MOE_LS_MAX]           max_e counts[e]
+ *     [MOE_LS_OVERFLOW_ROWS] sum_e max(counts[e] - capacity, 0) (0 without
+ *                            a capacity): rows in the overflow region
+ *     [MOE_LS_DROPPED]       S*K - sum_e counts[e]: slots that got no row.
+ *                            The layer drops no token, so this is 0 unless
+ *                            an expert id was outside [0, E).
+ * One kernel on `stream`; no workspace.  Errors: MOE_ERR_INVALID_ARG for an
+ * invalid desc or a NULL / misaligned pointer, MOE_ERR_CUDA for a failed
+ * launch.
+ */
+#define MOE_LS_MAX_OVER_MEAN 0
+#define MOE_LS_STD 1
+#define MOE_LS_MEAN 2
+#define MOE_LS_MAX 3
+#define MOE_LS_OVERFLOW_ROWS 4
+#define MOE_LS_DROPPED 5
+#define MOE_NUM_LOAD_STATS 6
+moe_status moe_load_stats(const moe_desc *desc, const int32_t *counts, double *stats, void *stream);
 
 /* Synchronise `stream`, copy the status block to the host.  flags: OR of
  * MOE_STATUS_* bits; counters: MOE_NUM_COUNTERS int32 (may be NULL).

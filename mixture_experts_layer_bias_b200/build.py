@@ -5,6 +5,11 @@
 Objects go to ``_build/`` at the repository root; the shared library lands
 next to this file so it ships with the package.  Only sources newer than their
 object are recompiled.
+
+A second library, libmoe_b200_testhooks.so, is linked from the same objects
+except the GEMM launch file, which is compiled with MOE_B200_TEST_HOOKS: it
+adds the failure-detection test hook (moe_test_stall_gemms) that the product
+library does not contain.  Only the failure-detection test loads it.
 """
 from __future__ import annotations
 
@@ -21,6 +26,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe_b200.so")
+TEST_HOOKS_LIB = os.path.join(PKG, "libmoe_b200_testhooks.so")
+TEST_HOOKS_SOURCE = "gemm_dispatch.cu"
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",
@@ -56,13 +63,7 @@ def _compile(src: str, force: bool, extra, build_dir: str = BUILD) -> str:
     return obj
 
 
-def build(force: bool = False, jobs: int = 8, extra=(), out: str = LIB, build_dir: str = BUILD) -> str:
-    """Compile every source (extra nvcc flags, e.g. -D tuning macros, go to
-    all of them) into build_dir and link `out`."""
-    os.makedirs(build_dir, exist_ok=True)
-    srcs = sources()
-    with cf.ThreadPoolExecutor(max_workers=jobs) as ex:
-        objs = list(ex.map(lambda s: _compile(s, force, extra, build_dir), srcs))
+def _link(objs, out: str, force: bool) -> str:
     if force or not os.path.exists(out) or os.path.getmtime(out) < max(os.path.getmtime(o) for o in objs):
         tmp = out + ".tmp"
         cmd = [nvcc()] + ARCH + ["-shared", "-o", tmp] + objs
@@ -70,6 +71,26 @@ def build(force: bool = False, jobs: int = 8, extra=(), out: str = LIB, build_di
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
         os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False, jobs: int = 8, extra=(), out: str = LIB, build_dir: str = BUILD,
+          test_hooks: bool = True) -> str:
+    """Compile every source (extra nvcc flags, e.g. -D tuning macros, go to
+    all of them) into build_dir and link `out`; with test_hooks also link the
+    test-hook library next to the product one."""
+    os.makedirs(build_dir, exist_ok=True)
+    srcs = sources()
+    with cf.ThreadPoolExecutor(max_workers=jobs) as ex:
+        objs = list(ex.map(lambda s: _compile(s, force, extra, build_dir), srcs))
+    _link(objs, out, force)
+    if test_hooks and out == LIB:
+        hook_dir = os.path.join(build_dir, "testhooks")
+        os.makedirs(hook_dir, exist_ok=True)
+        hook_src = os.path.join(CSRC, TEST_HOOKS_SOURCE)
+        hook_obj = _compile(hook_src, force, list(extra) + ["-DMOE_B200_TEST_HOOKS"], hook_dir)
+        objs_h = [hook_obj if os.path.basename(o) == TEST_HOOKS_SOURCE + ".o" else o for o in objs]
+        _link(objs_h, TEST_HOOKS_LIB, force)
     return out
 
 

@@ -118,6 +118,8 @@ moe_status validate(const moe_desc* d) {
   if (d->act_quant != 0 && d->act_quant != 1) return MOE_ERR_INVALID_ARG;
   if (d->reroute != 0 && d->reroute != 1) return MOE_ERR_INVALID_ARG;
   if (d->reroute == 1 && d->capacity <= 0) return MOE_ERR_INVALID_ARG;
+  // temperature: 0 (= 1) or a finite positive float (the comparison also rejects NaN)
+  if (!(d->temperature >= 0.0f) || d->temperature > 3.0e38f) return MOE_ERR_INVALID_ARG;
   // row indices are int32 on the device
   const int64_t rows = routed_rows(*d) + static_cast<int64_t>(d->num_shared) * d->num_tokens;
   if (rows > (int64_t(1) << 31) - 1) return MOE_ERR_INVALID_ARG;
@@ -128,6 +130,8 @@ moe_status validate(const moe_desc* d) {
     if (d->weight_dtype == MOE_F32) return MOE_ERR_UNSUPPORTED;
     if (d->weight_dtype == MOE_E4M3 && d->activation != MOE_ACT_SWIGLU) return MOE_ERR_UNSUPPORTED;
   }
+  if (d->score_fn == MOE_SCORE_SIGMOID && d->temperature != 0.0f && d->temperature != 1.0f)
+    return MOE_ERR_UNSUPPORTED;
   if (d->act_quant == 1 && (d->act_dtype != MOE_BF16 || d->weight_dtype != MOE_E4M3 ||
                             d->activation != MOE_ACT_SWIGLU || d->d_model % 16 != 0 || d->d_ff % 16 != 0))
     return MOE_ERR_UNSUPPORTED;
@@ -170,6 +174,7 @@ moe_status route_impl(const moe_desc& d, const moe_weights* w, const void* x, co
   a.K = d.top_k;
   a.score_fn = d.score_fn;
   a.renormalize = d.renormalize;
+  a.tau = d.temperature == 0.0f ? 1.0f : d.temperature;
   a.num_groups = d.num_groups;
   a.topk_groups = d.topk_groups;
   a.act_dtype = d.act_dtype;
@@ -220,8 +225,15 @@ moe_status permute_impl(const moe_desc& d, const void* x, const int32_t* topk_id
 
 // a_quantized (W8A8): the up projection's E4M3 rows and scales are already in
 // the workspace (written by the quantising gather), x_perm is not read.
+// Record stage event `i` of `events` (moe_layer_forward_timed), if given.
+bool record(void* const* events, int i, cudaStream_t st) {
+  if (events == nullptr || events[i] == nullptr) return true;
+  return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) == cudaSuccess;
+}
+
 moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm, const int32_t* offsets, const void* x,
-                    void* y_perm, void* ws, cudaStream_t st, bool groups_ready = false, bool a_quantized = false) {
+                    void* y_perm, void* ws, cudaStream_t st, bool groups_ready = false, bool a_quantized = false,
+                    void* const* events = nullptr) {
   const Layout L = make_layout(d);
   const int S = d.num_tokens, E = d.num_experts, h = d.d_ff, dm = d.d_model;
   if (S == 0) return MOE_OK;
@@ -347,9 +359,13 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
   };
   const bool w8a8 = d.act_quant == 1;
   if (w8a8 && !a_quantized && (err = quant_up(up)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (!record(events, 3, st)) return MOE_ERR_CUDA;
   if ((err = run(up)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (!record(events, 4, st)) return MOE_ERR_CUDA;
   if (w8a8 && (err = quant_down(down)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (!record(events, 5, st)) return MOE_ERR_CUDA;
   if ((err = run(down)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (!record(events, 6, st)) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 
@@ -393,6 +409,57 @@ bool weights_ok(const moe_desc& d, const moe_weights* w) {
   for (const void* p : ps)
     if (p && !aligned16(p)) return false;
   return true;
+}
+
+// The layer call (moe_layer_forward), recording the stage events of
+// moe_layer_forward_timed when `events` is given.
+moe_status layer_impl(const moe_desc* desc, const moe_weights* w, const void* x, void* y, int32_t* topk_idx,
+                      float* topk_w, int32_t* counts, void* ws, size_t ws_bytes, void* stream, void* const* events) {
+  moe_status s = validate(desc);
+  if (s != MOE_OK) return s;
+  if ((s = check_ws(*desc, ws, ws_bytes)) != MOE_OK) return s;
+  const moe_desc& d = *desc;
+  if (d.num_tokens == 0) return MOE_OK;
+  if (x == nullptr || y == nullptr || !aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  if (!weights_ok(d, w) || w->w_router == nullptr || !aligned16(w->w_router)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Layout L = make_layout(d);
+  int32_t* idx = topk_idx ? topk_idx : at<int32_t>(ws, L.topk_idx);
+  float* gates = topk_w ? topk_w : at<float>(ws, L.topk_w);
+  int32_t* cnt = counts ? counts : at<int32_t>(ws, L.counts);
+  int32_t* offs = at<int32_t>(ws, L.offsets);
+  int32_t* ros = at<int32_t>(ws, L.row_of_slot);
+  int32_t* tor = at<int32_t>(ws, L.token_of_row);
+  void* x_perm = at<void>(ws, L.x_perm);
+  void* y_perm = at<void>(ws, L.y_perm);
+  if (!record(events, 0, st)) return MOE_ERR_CUDA;
+  if ((s = route_impl(d, w, x, nullptr, idx, gates, ws, st)) != MOE_OK) return s;
+  if (d.reroute == 1) {
+    // capacity ranks of the first choices, then the excess slots move; the
+    // permutation below is that of the final choices
+    if ((s = permute_impl(d, nullptr, idx, cnt, offs, ros, tor, nullptr, ws, st)) != MOE_OK) return s;
+    if ((s = reroute_impl(d, idx, gates, cnt, ros, ws, st)) != MOE_OK) return s;
+  }
+  if (!record(events, 1, st)) return MOE_ERR_CUDA;
+  // the permutation also writes the GEMM group tables, so the FFN skips that launch
+  if (d.act_quant == 1) {
+    // W8A8: the row gather writes E4M3 codes and row scales straight away
+    // (no bf16 copy of the permuted rows)
+    if ((s = permute_impl(d, nullptr, idx, cnt, offs, ros, tor, nullptr, ws, st, true)) != MOE_OK) return s;
+    const bool sh = d.num_shared != 0;
+    if (launch_gather_quantize(d.num_tokens, d.d_model, d.top_k, ros, x, at<uint8_t>(ws, L.qa), at<float>(ws, L.sa),
+                               sh ? at<uint8_t>(ws, L.qas) : nullptr, sh ? at<float>(ws, L.sas) : nullptr,
+                               st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (!record(events, 2, st)) return MOE_ERR_CUDA;
+    if ((s = ffn_impl(d, *w, x_perm, offs, x, y_perm, ws, st, true, true, events)) != MOE_OK) return s;
+  } else {
+    if ((s = permute_impl(d, x, idx, cnt, offs, ros, tor, x_perm, ws, st, true)) != MOE_OK) return s;
+    if (!record(events, 2, st)) return MOE_ERR_CUDA;
+    if ((s = ffn_impl(d, *w, x_perm, offs, x, y_perm, ws, st, true, false, events)) != MOE_OK) return s;
+  }
+  if ((s = combine_impl(d, y_perm, ros, gates, y, st)) != MOE_OK) return s;
+  return record(events, 7, st) ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace
@@ -493,46 +560,24 @@ moe_status moe_combine(const moe_desc* desc, const void* y_perm, const int32_t* 
 
 moe_status moe_layer_forward(const moe_desc* desc, const moe_weights* w, const void* x, void* y, int32_t* topk_idx,
                              float* topk_w, int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
-  moe_status s = validate(desc);
+  return layer_impl(desc, w, x, y, topk_idx, topk_w, counts, ws, ws_bytes, stream, nullptr);
+}
+
+moe_status moe_layer_forward_timed(const moe_desc* desc, const moe_weights* w, const void* x, void* y,
+                                   int32_t* topk_idx, float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
+                                   void* stream, void* const* events) {
+  return layer_impl(desc, w, x, y, topk_idx, topk_w, counts, ws, ws_bytes, stream, events);
+}
+
+moe_status moe_load_stats(const moe_desc* desc, const int32_t* counts, double* stats, void* stream) {
+  const moe_status s = validate(desc);
   if (s != MOE_OK) return s;
-  if ((s = check_ws(*desc, ws, ws_bytes)) != MOE_OK) return s;
-  const moe_desc& d = *desc;
-  if (d.num_tokens == 0) return MOE_OK;
-  if (x == nullptr || y == nullptr || !aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
-  if (!weights_ok(d, w) || w->w_router == nullptr || !aligned16(w->w_router)) return MOE_ERR_INVALID_ARG;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const Layout L = make_layout(d);
-  int32_t* idx = topk_idx ? topk_idx : at<int32_t>(ws, L.topk_idx);
-  float* gates = topk_w ? topk_w : at<float>(ws, L.topk_w);
-  int32_t* cnt = counts ? counts : at<int32_t>(ws, L.counts);
-  int32_t* offs = at<int32_t>(ws, L.offsets);
-  int32_t* ros = at<int32_t>(ws, L.row_of_slot);
-  int32_t* tor = at<int32_t>(ws, L.token_of_row);
-  void* x_perm = at<void>(ws, L.x_perm);
-  void* y_perm = at<void>(ws, L.y_perm);
-  if ((s = route_impl(d, w, x, nullptr, idx, gates, ws, st)) != MOE_OK) return s;
-  if (d.reroute == 1) {
-    // capacity ranks of the first choices, then the excess slots move; the
-    // permutation below is that of the final choices
-    if ((s = permute_impl(d, nullptr, idx, cnt, offs, ros, tor, nullptr, ws, st)) != MOE_OK) return s;
-    if ((s = reroute_impl(d, idx, gates, cnt, ros, ws, st)) != MOE_OK) return s;
-  }
-  // the permutation also writes the GEMM group tables, so the FFN skips that launch
-  if (d.act_quant == 1) {
-    // W8A8: the row gather writes E4M3 codes and row scales straight away
-    // (no bf16 copy of the permuted rows)
-    if ((s = permute_impl(d, nullptr, idx, cnt, offs, ros, tor, nullptr, ws, st, true)) != MOE_OK) return s;
-    const bool sh = d.num_shared != 0;
-    if (launch_gather_quantize(d.num_tokens, d.d_model, d.top_k, ros, x, at<uint8_t>(ws, L.qa), at<float>(ws, L.sa),
-                               sh ? at<uint8_t>(ws, L.qas) : nullptr, sh ? at<float>(ws, L.sas) : nullptr,
-                               st) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    if ((s = ffn_impl(d, *w, x_perm, offs, x, y_perm, ws, st, true, true)) != MOE_OK) return s;
-  } else {
-    if ((s = permute_impl(d, x, idx, cnt, offs, ros, tor, x_perm, ws, st, true)) != MOE_OK) return s;
-    if ((s = ffn_impl(d, *w, x_perm, offs, x, y_perm, ws, st, true)) != MOE_OK) return s;
-  }
-  return combine_impl(d, y_perm, ros, gates, y, st);
+  if (counts == nullptr || stats == nullptr || (reinterpret_cast<uintptr_t>(counts) & 3) != 0 ||
+      (reinterpret_cast<uintptr_t>(stats) & 7) != 0)
+    return MOE_ERR_INVALID_ARG;
+  const int64_t slots = static_cast<int64_t>(desc->num_tokens) * desc->top_k;
+  return cuda_status(launch_load_stats(desc->num_experts, slots, desc->capacity, counts, stats,
+                                       static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_bias_state_size(const moe_desc* desc, int32_t window_tokens, size_t* bytes) {

@@ -1,7 +1,6 @@
-// Grouped GEMM dispatch: fills the launch parameters shared by the tensor-core
-// kernels and picks one of them (token rows as M, the default; weights as M
-// on one CTA; weights as M on a CTA pair).  E4M3 operands always take the
-// token-rows kernel.
+// Grouped GEMM launch parameters: fills the parameter block of the
+// tensor-core kernel from the launch arguments (split-K budget, epilogue
+// operands, output mode) and hands it to the token-rows kernel launcher.
 #include <stdlib.h>
 #include <string.h>
 
@@ -11,43 +10,21 @@ namespace moe {
 
 using namespace gemm;
 
+#ifdef MOE_B200_TEST_HOOKS
+// Failure-detection test hook, compiled only into the test build of the
+// library (libmoe_b200_testhooks.so): moe_test_stall_gemms(n) makes the next
+// n GEMM launches run with a producer that delivers nothing, so every bounded
+// wait of those launches gives up and reports MOE_STATUS_TIMEOUT.
 namespace {
-
-// Test hook for the failure-detection tests: MOE_B200_TEST_STALL_GEMM=n makes
-// the next n one-CTA GEMM launches of this process run with a producer that
-// delivers nothing, so their bounded waits give up and report
-// MOE_STATUS_TIMEOUT.  Unset (the default) it costs nothing.
+int g_stall_budget = 0;
 int take_test_stall() {
-  static int budget = -1;
-  if (budget < 0) {
-    const char* v = getenv("MOE_B200_TEST_STALL_GEMM");
-    budget = v != nullptr ? atoi(v) : 0;
-    if (budget < 0) budget = 0;
-  }
-  if (budget == 0) return 0;
-  --budget;
+  if (g_stall_budget <= 0) return 0;
+  --g_stall_budget;
   return 1;
 }
-
-// Kernel choice (read once): MOE_B200_GEMM=pair or =wt selects the CTA-pair or
-// the one-CTA weights-as-M kernel, =hybrid the weights-as-M kernel for all but
-// the SwiGLU up projection, =pairtok the token-rows kernel on CTA pairs for
-// large groups; otherwise (or =single) the one-CTA token-rows kernel.
-int gemm_kernel_choice() {
-  static int choice = -1;
-  if (choice < 0) {
-    const char* v = getenv("MOE_B200_GEMM");
-    choice = 0;
-    if (v != nullptr && strcmp(v, "pair") == 0) choice = 1;
-    if (v != nullptr && strcmp(v, "wt") == 0) choice = 2;
-    if (v != nullptr && strcmp(v, "hybrid") == 0) choice = 3;
-    if (v != nullptr && strcmp(v, "single") == 0) choice = 4;
-    if (v != nullptr && strcmp(v, "pairtok") == 0) choice = 5;
-  }
-  return choice;
-}
-
 }  // namespace
+extern "C" void moe_test_stall_gemms(int n) { g_stall_budget = n > 0 ? n : 0; }
+#endif
 
 cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t stream) {
   if (a.num_groups <= 0 || a.num_groups > kMaxGroups) return cudaErrorInvalidValue;
@@ -82,16 +59,16 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t 
     if (p.max_ksplit > 16) p.max_ksplit = 16;
     if (p.max_ksplit < 1) p.max_ksplit = 1;
   }
+#ifdef MOE_B200_TEST_HOOKS
+  p.test_stall = take_test_stall();
+#else
   p.test_stall = 0;
-  p.tma_out = 0;  // set by the token-rows launcher when it can map the output
+#endif
+  p.tma_out = 0;  // set by the launcher when it can map the output
   p.row_scale = a.fp8 ? a.row_scale : nullptr;
   p.row_scale_shared = a.fp8 ? a.row_scale_shared : nullptr;
   if (a.fp8 && a.row_scale == nullptr) return cudaErrorInvalidValue;
-  const int choice = a.fp8 ? 0 : gemm_kernel_choice();  // 8-bit operands: token-rows kernel only
-  if (choice == 1) return launch_grouped_gemm_pair(a, p, num_sms, stream);
-  p.test_stall = take_test_stall();
-  if (choice == 2 || (choice == 3 && a.epilogue != EPI_SWIGLU)) return launch_grouped_gemm_wt(a, p, num_sms, stream);
-  return launch_grouped_gemm_single(a, p, num_sms, stream, choice == 4 ? 1 : (choice == 5 ? 2 : 0));
+  return launch_grouped_gemm_single(a, p, num_sms, stream);
 }
 
 }  // namespace moe

@@ -455,262 +455,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// ---------------------------------------------------------------------------
-// CTA-pair variant (tcgen05 .cta_group::2) for large groups: a cluster of two
-// CTAs owns 256 token rows (128 in each CTA's shared memory and TMEM lanes) by
-// the same 256 accumulator columns; each CTA loads its own 128 token rows and
-// one half of the weight tile (SwiGLU: the gate rows in the even CTA, the up
-// rows in the odd one; otherwise weight rows 0-127 / 128-255), so a CTA moves
-// 32 KB per 128-byte K step instead of 48 KB and six stages fit.  One thread
-// of the even CTA issues the MMAs (M=256, N=256) for both; each CTA's
-// epilogue drains its own rows exactly as in the one-CTA kernel.  All loads
-// are plain (no cluster multicast); only the MMA completion signal
-// (tcgen05.commit) reaches both CTAs.
-constexpr int P2_STAGES = 6;
-constexpr int P2_BM = 256;  // token rows per pair tile
-constexpr int P2_STAGE = 128 * BK_BYTES + 128 * BK_BYTES;  // own A rows + half of B
-constexpr size_t kP2Smem = P2_STAGES * P2_STAGE + kCtlBytes;
-
-template <int EPI, bool F8>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    grouped_gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
-                                const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
-                                const __grid_constant__ CUtensorMap tmOut, TcParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  constexpr int BK = bk_elems<F8>();
-  constexpr int A_BYTES = 128 * BK_BYTES;
-  SmemCtl& s = *reinterpret_cast<SmemCtl*>(ring + P2_STAGES * P2_STAGE);
-  uint8_t* epi_smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(ring + P2_STAGES * P2_STAGE + sizeof(SmemCtl)) + 127) & ~uintptr_t(127));
-  const int warp = threadIdx.x >> 5, lane = lane_id();
-  const uint32_t rank = cluster_ctarank();
-  const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
-
-  if (warp == 0) {
-    int carry = 0;
-    for (int base = 0; base < p.num_groups; base += 32) {
-      const int g = base + lane;
-      int tiles = 0;
-      if (g < p.num_groups) {
-        const GroupEntry ge = group_at(p, g);
-        if (group_ok(ge, p))
-          tiles = ((ge.rows + P2_BM - 1) / P2_BM) * p.n_tiles;
-        else if (ge.rows != 0 && rank == 0)
-          report(p.status, MOE_STATUS_BAD_GROUP, -1);
-      }
-      int incl = tiles;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-        if (lane >= off) incl += o;
-      }
-      if (g < p.num_groups) s.tile_start[g] = carry + incl - tiles;
-      carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
-    }
-    if (lane == 0) s.tile_start[p.num_groups] = carry;
-  } else if (warp == 1) {
-    if (lane == 0) {
-      for (int i = 0; i < P2_STAGES; ++i) {
-        mbar_init(&s.full[i], 1);
-        mbar_init(&s.empty[i], 1);
-      }
-      for (int i = 0; i < 2; ++i) {
-        mbar_init(&s.tfull[i], 1);
-        mbar_init(&s.tempty[i], 2 * kEpiWarps);  // one lane of each epilogue warp of both CTAs
-      }
-      mbar_init(&s.drain, 1);
-      s.abort = 0;
-      fence_mbar_init();
-    }
-    __syncwarp();
-    tmem_alloc_pair(&s.tmem_base, TMEM_COLS);
-    tmem_relinquish_pair();
-  } else if (warp == 2 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmA2);
-    tma_prefetch_desc(&tmB0);
-    tma_prefetch_desc(&tmB1);
-  }
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync_all();  // both CTAs' barriers exist before any remote signal
-  tc_fence_after();
-
-  const uint32_t tmem = s.tmem_base;
-  const int nk = (p.K + BK - 1) / BK;
-  const int tiles = s.tile_start[p.num_groups];
-  const int ks = choose_ksplit(tiles, nclusters, nk, p.max_ksplit);
-  if (blockIdx.x == 0 && threadIdx.x == 0 && p.ksplit_out != nullptr) *p.ksplit_out = ks;
-  const int total = tiles * ks;
-  volatile int* abort_flag = &s.abort;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t armed = 0, armed_phase = 0;
-      bool ok = true;
-      for (int u = cluster; u < total && ok && !p.test_stall; u += nclusters) {
-        const UnitInfo ui = decode_unit(s, p, u, ks, nk, P2_BM);
-        const TileInfo& ti = ui.ti;
-        const int a_row = (p.a_rows_from_out ? ti.grp.out_row0 : ti.grp.a_row0) + ti.m_idx * P2_BM +
-                          static_cast<int>(rank) * 128;
-        const CUtensorMap* mA = (ti.grp.expert == p.shared_slab) ? &tmA2 : &tmA;
-        const int b_row0 = ti.grp.expert * p.n_per_slab + ti.n_idx * p.bn_out;
-        const CUtensorMap* mB = (EPI == EPI_SWIGLU && rank == 1) ? &tmB1 : &tmB0;
-        const int b_row = (EPI == EPI_SWIGLU) ? b_row0 : b_row0 + static_cast<int>(rank) * 128;
-        for (int kb = ui.kb0; kb < ui.kb1; ++kb) {
-          if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag)) {
-            ok = false;
-            break;
-          }
-          if (rank == 0) {
-            mbar_arrive_expect_tx(&s.full[stage], 2 * P2_STAGE);
-            armed |= 1u << stage;
-            armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
-          }
-          const uint32_t bar = mapa_shared(smem_u32(&s.full[stage]), 0);
-          uint8_t* sa = ring + stage * P2_STAGE;
-          tma_load_2d_pair(sa, mA, kb * BK, a_row, bar);
-          tma_load_2d_pair(sa + A_BYTES, mB, kb * BK, b_row, bar);
-          if (++stage == P2_STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      if (!ok) {
-        *abort_flag = 1;
-        report(p.status, MOE_STATUS_TIMEOUT, MOE_CNT_TIMEOUT);
-        if (rank == 0) {
-          for (int i = 0; i < P2_STAGES; ++i)
-            if (armed & (1u << i)) wait_timed(&s.full[i], (armed_phase >> i) & 1u);
-        } else {
-          // this CTA's copies count on the peer's barriers: give them time to land
-          const uint64_t t0 = globaltimer_ns();
-          while (globaltimer_ns() - t0 < 2000000ull) {
-          }
-        }
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
-      constexpr uint32_t kIdesc2 = F8 ? idesc_e4m3_f32(256, 256) : idesc_bf16_f32(256, 256);
-      int stage = 0;
-      uint32_t phase = 0;
-      int local = 0;
-      bool ok = true;
-      for (int u = cluster; u < total && ok; u += nclusters, ++local) {
-        const int split = u % ks;
-        const int kb0 = static_cast<int>((static_cast<int64_t>(split) * nk) / ks);
-        const int kb1 = static_cast<int>((static_cast<int64_t>(split + 1) * nk) / ks);
-        const int acc = local & 1;
-        const uint32_t acc_phase = (local >> 1) & 1;
-        if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + acc * ACC_COLS;
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&s.full[stage], phase, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_base = smem_u32(ring + stage * P2_STAGE);
-          const uint32_t b_base = a_base + A_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < BK_BYTES / 32; ++kk) {
-            if (F8)
-              tc_mma_f8_pair(d_tmem, smem_desc_sw128(a_base + kk * 32), smem_desc_sw128(b_base + kk * 32), kIdesc2,
-                             (kb > kb0 || kk > 0) ? 1u : 0u);
-            else
-              tc_mma_f16_pair(d_tmem, smem_desc_sw128(a_base + kk * 32), smem_desc_sw128(b_base + kk * 32), kIdesc2,
-                              (kb > kb0 || kk > 0) ? 1u : 0u);
-          }
-          tc_commit_pair_mask(&s.empty[stage], 0x3);
-          if (++stage == P2_STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if (!ok) break;
-        tc_commit_pair_mask(&s.tfull[acc], 0x3);
-      }
-      tc_commit_pair(&s.drain);
-      wait_timed(&s.drain, 0);
-      if (!ok) {
-        *abort_flag = 1;
-        report(p.status, MOE_STATUS_TIMEOUT, MOE_CNT_TIMEOUT);
-      }
-    }
-    __syncwarp();
-  } else {
-    const int q = warp & 3;            // TMEM lane quarter this warp may access
-    const int half = (warp - 2) >> 2;  // which half of the tile's columns it drains
-    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&s.tempty[0]), 0);
-    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&s.tempty[1]), 0);
-    int local = 0;
-    for (int u = cluster; u < total; u += nclusters, ++local) {
-      const UnitInfo ui = decode_unit(s, p, u, ks, nk, P2_BM);
-      const TileInfo& ti = ui.ti;
-      const int acc = local & 1;
-      const uint32_t acc_phase = (local >> 1) & 1;
-      if (!mbar_wait(&s.tfull[acc], acc_phase, abort_flag)) {
-        if (lane == 0) {
-          *abort_flag = 1;
-          report(p.status, MOE_STATUS_TIMEOUT, MOE_CNT_TIMEOUT);
-        }
-        break;
-      }
-      tc_fence_after();
-      const int row = ti.m_idx * P2_BM + static_cast<int>(rank) * 128 + q * 32 + lane;
-      const bool valid = row < ti.grp.rows;
-      const uint32_t tbase = tmem + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16);
-      if (ks > 1)
-        epilogue_partial<EPI>(p, ti, tbase, row, valid, ui.split, half);
-      else
-        epilogue_store<EPI>(p, ti, tbase, row, valid, lane, half, &tmOut, epi_smem + (warp - 2) * kEpiWarpBytes);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
-    }
-  }
-
-  if (warp >= 2 && lane == 0) bulk_wait_all();  // this warp's output boxes are written
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync_all();  // the even CTA's MMAs read this CTA's shared memory and TMEM until here
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc_pair(tmem, TMEM_COLS);
-  }
-}
-
-template <int EPI, bool F8>
-cudaError_t launch_pair_tok(const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB0,
-                            const CUtensorMap& mB1, const CUtensorMap& mOut, const TcParams& p, int grid,
-                            int64_t max_group_rows, cudaStream_t stream) {
-  static uint64_t attr_set = 0;  // one bit per device ordinal
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev >= 64 || !(attr_set & (1ull << dev))) {
-    e = cudaFuncSetAttribute(grouped_gemm_tc_pair_kernel<EPI, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kP2Smem));
-    if (e != cudaSuccess) return e;
-    if (dev < 64) attr_set |= 1ull << dev;
-  }
-  grouped_gemm_tc_pair_kernel<EPI, F8><<<grid, kThreads, kP2Smem, stream>>>(mA, mA2, mB0, mB1, mOut, p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess || p.max_ksplit <= 1) return e;
-  dim3 fgrid((p.N + 1023) / 1024, static_cast<unsigned>(max_group_rows), p.num_groups);
-  splitk_finalize_kernel<EPI><<<fgrid, 256, 0, stream>>>(p);
-  return cudaGetLastError();
-}
-
 template <int EPI, bool F8>
 cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB0, const CUtensorMap& mB1,
                        const CUtensorMap& mOut, const TcParams& p, int grid, int bma, int stages, size_t smem,
@@ -735,13 +479,8 @@ cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUte
 
 }  // namespace
 
-// Token-rows kernel launch; `p` is filled by the dispatcher.  pair_mode: 0 or
-// 1 = one-CTA kernel, 2 = CTA pairs when the groups are large (at least 512
-// rows on average and some group above 128).  In same-box A/B the pair
-// kernel was within a few percent of the one-CTA kernel and read 28% more
-// weight bytes from DRAM in the up projection, so it stays opt-in.
-cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& p, int num_sms, cudaStream_t stream,
-                                       int pair_mode) {
+// Token-rows kernel launch; `p` is filled by launch_grouped_gemm_tc.
+cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& p, int num_sms, cudaStream_t stream) {
   // A rows loaded per stage: all 128, or (every group fitting) the largest group rounded up to 16
   int bma = BM;
   if (a.max_group_rows > 0 && a.max_group_rows <= 64) bma = static_cast<int>((a.max_group_rows + 15) & ~int64_t(15));
@@ -766,32 +505,6 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
     if (!make_map(&mB1, a.b1, a.b_rows, a.K, 128, eb)) return cudaErrorInvalidValue;
   } else {
     mB1 = mB0;
-  }
-  const bool large = a.max_group_rows > 128 && a.max_total_rows >= int64_t(512) * a.num_groups;
-  if (bma == BM && num_sms >= 2 && pair_mode == 2 && large) {
-    const int64_t pbound = (a.max_total_rows / P2_BM + a.num_groups) * static_cast<int64_t>(p.n_tiles);
-    const int64_t clusters = pbound < num_sms / 2 ? (pbound > 0 ? pbound : 1) : num_sms / 2;
-    const int pgrid = static_cast<int>(2 * (clusters > 0 ? clusters : 1));
-    if (a.fp8) {
-      switch (a.epilogue) {
-        case EPI_SWIGLU:
-          return launch_pair_tok<EPI_SWIGLU, true>(mA, mA2, mB0, mB1, mOut, pp, pgrid, a.max_group_rows, stream);
-        case EPI_NONE:
-          return launch_pair_tok<EPI_NONE, true>(mA, mA2, mB0, mB1, mOut, pp, pgrid, a.max_group_rows, stream);
-        default: return cudaErrorInvalidValue;
-      }
-    }
-    switch (a.epilogue) {
-      case EPI_SWIGLU:
-        return launch_pair_tok<EPI_SWIGLU, false>(mA, mA2, mB0, mB1, mOut, pp, pgrid, a.max_group_rows, stream);
-      case EPI_GELU_BIAS:
-        return launch_pair_tok<EPI_GELU_BIAS, false>(mA, mA2, mB0, mB1, mOut, pp, pgrid, a.max_group_rows, stream);
-      case EPI_BIAS:
-        return launch_pair_tok<EPI_BIAS, false>(mA, mA2, mB0, mB1, mOut, pp, pgrid, a.max_group_rows, stream);
-      case EPI_NONE:
-        return launch_pair_tok<EPI_NONE, false>(mA, mA2, mB0, mB1, mOut, pp, pgrid, a.max_group_rows, stream);
-      default: return cudaErrorInvalidValue;
-    }
   }
   // upper bound of the tile count: every group may add one partial m-block
   const int64_t bound = (a.max_total_rows / BM + a.num_groups) * static_cast<int64_t>(p.n_tiles);

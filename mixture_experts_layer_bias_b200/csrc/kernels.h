@@ -15,6 +15,7 @@ struct StatusBlock;
 struct RouteArgs {
   int S, d, E, K;
   int score_fn, renormalize, num_groups, topk_groups;
+  float tau;                // softmax temperature: logits are divided by it (1 = none)
   int act_dtype;
   const void* x;            // [S][d] (unused when logits given)
   const void* w_router;     // [E][d]
@@ -116,10 +117,7 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t 
 namespace gemm {
 struct TcParams;
 }
-cudaError_t launch_grouped_gemm_pair(const GemmArgs& a, const gemm::TcParams& p, int num_sms, cudaStream_t stream);
-cudaError_t launch_grouped_gemm_wt(const GemmArgs& a, const gemm::TcParams& p, int num_sms, cudaStream_t stream);
-cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& p, int num_sms, cudaStream_t stream,
-                                       int pair_mode);
+cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& p, int num_sms, cudaStream_t stream);
 cudaError_t launch_grouped_gemm_f32(const GemmArgs& a, cudaStream_t stream);
 
 // FP8-E4M3 weight slabs -> bf16 (exact)
@@ -148,6 +146,11 @@ cudaError_t launch_quantize_group_rows(const GroupEntry* groups, int num_groups,
 size_t bias_state_bytes(int E, int K, int window);
 cudaError_t launch_bias_update(int S, int E, int K, int window, const int32_t* topk_idx, float gamma, void* state,
                                float* sel_bias, int32_t* window_counts, cudaStream_t stream);
+
+// --- load report -------------------------------------------------------------
+// MOE_NUM_LOAD_STATS doubles from counts[E] (one CTA; see moe_load_stats).
+cudaError_t launch_load_stats(int E, int64_t slots, int capacity, const int32_t* counts, double* out,
+                              cudaStream_t stream);
 
 // --- combine -----------------------------------------------------------------
 struct CombineArgs {

@@ -85,6 +85,7 @@ __device__ __forceinline__ float warp_max(float v) {
 
 struct SelectParams {
   int E, K, score_fn, renormalize, num_groups, topk_groups;
+  float tau;  // softmax temperature (1 = none): z = l / tau
   const float* sel_bias;
   int32_t* topk_idx;
   float* topk_w;
@@ -126,6 +127,8 @@ __device__ __forceinline__ float gate_of(const float (&score)[NI], const bool (&
 
 // Selection for one token held by the whole warp: l[i] is the logit (router
 // bias included) of expert 32*i + lane.  Writes K indices and gates.
+// Softmax scores are the logits divided by the temperature (jsqmd.com
+// 11.3.3, soft routing with softmax(s / tau)).
 template <int NI>
 __device__ void select_topk(const float (&l)[NI], const SelectParams& p, int t) {
   const int lane = lane_id();
@@ -140,7 +143,9 @@ __device__ void select_topk(const float (&l)[NI], const SelectParams& p, int t) 
     valid[i] = e < E;
     const float li = valid[i] ? l[i] : kNegInf;
     if (valid[i] && !isfinite(li)) nonfinite = true;
-    score[i] = (p.score_fn == MOE_SCORE_SIGMOID) ? sigmoid_sel_f32(li) : li;
+    // softmax: the tempered logit z = l / tau (one float32 division, exact for
+    // tau = 1) is both the gate source and the key; sigmoid: sigma(l)
+    score[i] = (p.score_fn == MOE_SCORE_SIGMOID) ? sigmoid_sel_f32(li) : __fdiv_rn(li, p.tau);
     float k = score[i];
     if (valid[i] && p.sel_bias != nullptr) k = __fadd_rn(k, __ldg(p.sel_bias + e));
     if (!valid[i] || isnan(k)) k = kNegInf;
@@ -450,8 +455,8 @@ cudaError_t launch_topk_ni(const RouteArgs& a, const float* logits, const Select
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
   if (a.S == 0) return cudaSuccess;
-  SelectParams sp{a.E,       a.K,        a.score_fn, a.renormalize, a.num_groups,  a.topk_groups, a.sel_bias,
-                  a.topk_idx, a.topk_w, a.status,   a.cand_key_out, a.score_out};
+  SelectParams sp{a.E,        a.K,      a.score_fn, a.renormalize, a.num_groups,   a.topk_groups, a.tau,
+                  a.sel_bias, a.topk_idx, a.topk_w, a.status,      a.cand_key_out, a.score_out};
   const int blocks = (a.S + kRouteWarps - 1) / kRouteWarps;
   const float* logits = a.logits;
   if (logits == nullptr && a.E <= 32) {

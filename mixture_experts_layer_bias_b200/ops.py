@@ -14,10 +14,7 @@ from typing import Optional
 
 import torch
 
-# MOE_B200_LIB may point at another build of the same library (e.g. a variant
-# compiled with different tuning macros).
-_LIB_PATH = os.environ.get("MOE_B200_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
-                                                           "libmoe_b200.so")
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
 _lib = None
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE_STATUS = range(6)
@@ -27,18 +24,23 @@ COUNTER_NAMES = ("nonfinite", "bad_id", "timeout", "overflow_rows", "rerouted")
 
 DESC_FIELDS = ("num_tokens", "d_model", "num_experts", "top_k", "d_ff", "score_fn", "renormalize", "num_groups",
                "topk_groups", "num_shared", "activation", "act_dtype", "weight_dtype", "capacity", "act_quant",
-               "reroute")
+               "reroute", "temperature")
+DESC_FLOAT_FIELDS = ("temperature",)
 WEIGHT_FIELDS = ("w_router", "router_bias", "sel_bias", "w1", "b1", "w2", "b2", "w_gate", "w_up", "w_down",
                  "s_gate", "s_up", "s_down")
 
 EXPORTED = ("moe_routed_rows", "moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute",
-            "moe_permute_static", "moe_grouped_ffn", "moe_combine", "moe_layer_forward", "moe_bias_state_size",
-            "moe_bias_state_init", "moe_update_sel_bias", "moe_quantize_rows_e4m3", "moe_reroute",
-            "moe_get_status", "moe_strerror")
+            "moe_permute_static", "moe_grouped_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_timed",
+            "moe_load_stats", "moe_bias_state_size", "moe_bias_state_init", "moe_update_sel_bias",
+            "moe_quantize_rows_e4m3", "moe_reroute", "moe_get_status", "moe_strerror")
+
+MOE_NUM_STAGE_EVENTS = 8
+MOE_NUM_LOAD_STATS = 6
+LOAD_STAT_NAMES = ("max_over_mean", "std", "mean", "max", "overflow_rows", "dropped")
 
 
 class MoeDesc(ctypes.Structure):
-    _fields_ = [(f, ctypes.c_int32) for f in DESC_FIELDS]
+    _fields_ = [(f, ctypes.c_float if f in DESC_FLOAT_FIELDS else ctypes.c_int32) for f in DESC_FIELDS]
 
 
 class MoeWeights(ctypes.Structure):
@@ -71,6 +73,8 @@ def lib():
         "moe_grouped_ffn": (I, [pd, pw, P, P, P, P, P, SZ, P]),
         "moe_combine": (I, [pd, P, P, P, P, P, SZ, P]),
         "moe_layer_forward": (I, [pd, pw, P, P, P, P, P, P, SZ, P]),
+        "moe_layer_forward_timed": (I, [pd, pw, P, P, P, P, P, P, SZ, P, ctypes.POINTER(ctypes.c_void_p)]),
+        "moe_load_stats": (I, [pd, P, P, P]),
         "moe_bias_state_size": (I, [pd, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]),
         "moe_bias_state_init": (I, [P, SZ, P]),
         "moe_update_sel_bias": (I, [pd, P, ctypes.c_int32, ctypes.c_float, P, SZ, P, P, P]),
@@ -94,10 +98,10 @@ def strerror(code: int) -> str:
 def make_desc(**fields) -> MoeDesc:
     d = MoeDesc()
     defaults = dict(score_fn=0, renormalize=1, num_groups=1, topk_groups=1, num_shared=0, activation=1,
-                    act_dtype=1, weight_dtype=1, capacity=0, act_quant=0, reroute=0)
+                    act_dtype=1, weight_dtype=1, capacity=0, act_quant=0, reroute=0, temperature=0.0)
     defaults.update(fields)
     for f in DESC_FIELDS:
-        setattr(d, f, int(defaults[f]))
+        setattr(d, f, float(defaults[f]) if f in DESC_FLOAT_FIELDS else int(defaults[f]))
     return d
 
 
@@ -192,6 +196,25 @@ def moe_layer_forward(desc, weights, x, y, topk_idx, topk_w, counts, ws, stream=
     p, n = _ws(ws)
     _check(lib().moe_layer_forward(ctypes.byref(desc), ctypes.byref(weights), _ptr(x), _ptr(y), _ptr(topk_idx),
                                    _ptr(topk_w), _ptr(counts), p, n, _stream(stream)), "moe_layer_forward")
+
+
+def moe_layer_forward_timed(desc, weights, x, y, topk_idx, topk_w, counts, ws, events, stream=None):
+    """moe_layer_forward recording the stage events: `events` is a list of
+    MOE_NUM_STAGE_EVENTS torch.cuda.Event (or None) already created on this
+    device (record each once, or query it, before the first call)."""
+    p, n = _ws(ws)
+    handles = (ctypes.c_void_p * MOE_NUM_STAGE_EVENTS)()
+    for i, ev in enumerate(events):
+        handles[i] = None if ev is None else ev.cuda_event
+    _check(lib().moe_layer_forward_timed(ctypes.byref(desc), ctypes.byref(weights), _ptr(x), _ptr(y), _ptr(topk_idx),
+                                         _ptr(topk_w), _ptr(counts), p, n, _stream(stream), handles),
+           "moe_layer_forward_timed")
+
+
+def moe_load_stats(desc, counts, stats, stream=None):
+    """Load report of the counts [E] into stats (float64 [6], device): see
+    LOAD_STAT_NAMES for the order."""
+    _check(lib().moe_load_stats(ctypes.byref(desc), _ptr(counts), _ptr(stats), _stream(stream)), "moe_load_stats")
 
 
 def moe_bias_state_size(desc, window_tokens: int) -> int:

@@ -67,6 +67,7 @@ class LayerConfig:
     capacity: int = 0
     act_quant: int = 0               # 1: W8A8 (E4M3 activation rows with per-row scales)
     reroute: int = 0                 # 1: over-capacity slots move to the next-best expert with room
+    temperature: float = 0.0         # softmax temperature of the router (0 = 1)
     router_offset_var: float = 0.0   # variance of N(0, v) per-expert logit offsets
     skew_offset_scale: float = 0.0   # c of the c * z_e offsets
     sel_bias_var: float = 0.0        # variance of the selection bias
@@ -202,4 +203,4 @@ def desc_dict(cfg: LayerConfig, S: Optional[int] = None) -> dict:
                 d_ff=cfg.h, score_fn=cfg.score_fn, renormalize=cfg.renormalize, num_groups=cfg.num_groups,
                 topk_groups=cfg.topk_groups, num_shared=cfg.num_shared, activation=cfg.activation,
                 act_dtype=cfg.act_dtype, weight_dtype=cfg.weight_dtype, capacity=cfg.capacity,
-                act_quant=cfg.act_quant, reroute=cfg.reroute)
+                act_quant=cfg.act_quant, reroute=cfg.reroute, temperature=cfg.temperature)

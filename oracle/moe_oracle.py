@@ -243,14 +243,17 @@ def select_experts(
     sel_bias=None,
     num_groups: int = 1,
     topk_groups: int = 1,
+    temperature: float = 1.0,
 ):
     """Top-K expert selection and gate weights for every token.
 
     logits: float32 [S, E] (router output, router bias already added).
-    score_fn 'softmax' (chapter 11, 11.1.1): key = logit (+ sel_bias); the
-        gate is exp(l_k - m) / sum_{j in TopK} exp(l_j - m) when renormalised
-        -- the softmax of the TopK(-inf) sparsified scores -- else the full
-        softmax probability of expert k.
+    score_fn 'softmax' (chapter 11, 11.1.1): the score is the tempered logit
+        z = l / temperature (chapter 11, 11.3.3, soft routing with
+        softmax(s / tau); one float32 division, z = l for temperature 1);
+        key = z (+ sel_bias); the gate is exp(z_k - m) / sum_{j in TopK}
+        exp(z_j - m) when renormalised -- the softmax of the TopK(-inf)
+        sparsified scores -- else the full softmax probability of expert k.
     score_fn 'sigmoid' (ybb.press 2.3, bias moved onto the sigmoid scores):
         s = sigmoid_f32(l), key = s + sel_bias in float32; the gate is
         s_k / sum_j s_j (renormalised) or s_k.
@@ -263,7 +266,7 @@ def select_experts(
     """
     logits = np.asarray(logits, dtype=np.float32)
     S, E = logits.shape
-    scores, keys, cand = selection_keys(logits, score_fn, sel_bias, num_groups, topk_groups)
+    scores, keys, cand = selection_keys(logits, score_fn, sel_bias, num_groups, topk_groups, temperature)
     # candidates first, each part in descending key order, ties to lower index
     neg = -keys.astype(np.float64)
     order = np.lexsort((np.broadcast_to(np.arange(E), (S, E)), neg, ~cand), axis=-1)
@@ -271,16 +274,17 @@ def select_experts(
     return idx, gate_weights(scores, idx, score_fn, renormalize)
 
 
-def selection_keys(logits, score_fn="softmax", sel_bias=None, num_groups=1, topk_groups=1):
+def selection_keys(logits, score_fn="softmax", sel_bias=None, num_groups=1, topk_groups=1, temperature=1.0):
     """The quantities selection works on (see ``select_experts``): scores
-    (float32 logits, or their sigmoid), keys (scores + sel_bias in float32,
-    NaN -> -inf) and the candidate mask (experts of the token's kept
-    groups; all experts without groups)."""
+    (float32 logits divided by the temperature, or their sigmoid), keys
+    (scores + sel_bias in float32, NaN -> -inf) and the candidate mask
+    (experts of the token's kept groups; all experts without groups)."""
     logits = np.asarray(logits, dtype=np.float32)
     S, E = logits.shape
     if score_fn == "softmax":
-        scores = logits
+        scores = np.divide(logits, np.float32(temperature), dtype=np.float32)
     elif score_fn == "sigmoid":
+        assert temperature == 1.0, "the temperature applies to the softmax router"
         scores = sigmoid_f32(logits)
     else:
         raise ValueError(score_fn)
@@ -321,14 +325,18 @@ def gate_weights(scores, idx, score_fn="softmax", renormalize=True):
     return s / s.sum(axis=1, keepdims=True) if renormalize else s
 
 
-def selection_margin(logits, top_k, score_fn="softmax", sel_bias=None, num_groups=1, topk_groups=1):
+def selection_margin(logits, top_k, score_fn="softmax", sel_bias=None, num_groups=1, topk_groups=1,
+                     temperature=1.0):
     """Per token, the smaller of (a) the gap between the K-th and (K+1)-th
     candidate key and (b) the gap between the last kept and the first dropped
     group score.  A path that computes its own logits in another summation
     order may legitimately route a token with a tiny margin differently."""
     logits = np.asarray(logits, dtype=np.float32)
     S, E = logits.shape
-    scores = logits if score_fn == "softmax" else sigmoid_f32(logits)
+    if score_fn == "softmax":
+        scores = np.divide(logits, np.float32(temperature), dtype=np.float32)
+    else:
+        scores = sigmoid_f32(logits)
     keys = scores if sel_bias is None else np.add(scores, np.asarray(sel_bias, np.float32)[None, :],
                                                   dtype=np.float32)
     keys = _nan_to_neginf(keys).astype(np.float64)
@@ -458,13 +466,26 @@ def reroute_over_capacity(topk_idx, keys, cand, capacity: int):
     return idx, moved
 
 
-def load_stats(counts: np.ndarray, top_k: int, num_tokens: int) -> dict:
-    """max/mean expert load (chapter 11, 11.2.3) and the standard deviation of
-    per-expert counts (ybb.press 1.2, 'Expert Load Balance')."""
+def load_stats(counts: np.ndarray, top_k: int, num_tokens: int, capacity: int = 0) -> dict:
+    """Load report of one routing, from the per-expert counts (plumephp.com
+    verification block: the routing histogram is the first thing to check):
+
+    * max_over_mean: max_e count_e / (S*K/E), the max/mean expert load of
+      chapter 11, 11.2.3 (1 when balanced, 3-5 in practice);
+    * std: population standard deviation of the counts (ybb.press 1.2,
+      expert load balance row of the table);
+    * overflow_rows: rows above the capacity, sum_e max(count_e - C, 0)
+      (ybb.press 2.2 overflow buffering; 0 without a capacity);
+    * dropped: (token, k) slots without an expert row, S*K - sum_e count_e
+      (ybb.press 1.2, token drop rate; the layer drops nothing, so 0 unless
+      an expert id was out of range);
+    * mean = S*K/E and max = max_e count_e."""
     c = np.asarray(counts, dtype=np.float64)
     mean = num_tokens * top_k / len(c)
+    over = float(np.maximum(c - capacity, 0).sum()) if capacity > 0 else 0.0
     return {"max_over_mean": float(c.max() / mean) if mean > 0 else 0.0,
-            "std": float(c.std()), "mean": mean}
+            "std": float(c.std()), "mean": mean, "max": float(c.max()), "overflow_rows": over,
+            "dropped": float(num_tokens * top_k - c.sum())}
 
 
 # ----------------------------------------------------------------------------

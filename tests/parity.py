@@ -98,9 +98,10 @@ def oracle_routing(inp: dict, cfg: syn.LayerConfig, tokens=None):
     rb = None if inp.get("router_bias") is None else np64(inp["router_bias"])
     logits = O.router_logits(x, np64(inp["w_router"]), rb)
     sb = None if inp.get("sel_bias") is None else inp["sel_bias"].cpu().numpy().astype(np.float32)
+    tau = cfg.temperature or 1.0
     idx, w = O.select_experts(logits, cfg.K, SCORE[cfg.score_fn], bool(cfg.renormalize), sb, cfg.num_groups,
-                              cfg.topk_groups)
-    margin = O.selection_margin(logits, cfg.K, SCORE[cfg.score_fn], sb, cfg.num_groups, cfg.topk_groups)
+                              cfg.topk_groups, tau)
+    margin = O.selection_margin(logits, cfg.K, SCORE[cfg.score_fn], sb, cfg.num_groups, cfg.topk_groups, tau)
     if cfg.reroute:
         idx, w = oracle_reroute(logits, idx, cfg, sb)
     return x, idx, w, margin
@@ -108,7 +109,8 @@ def oracle_routing(inp: dict, cfg: syn.LayerConfig, tokens=None):
 
 def oracle_reroute(logits, idx, cfg: syn.LayerConfig, sel_bias=None):
     """Over-capacity re-routing of the oracle's selection, gates recomputed."""
-    scores, keys, cand = O.selection_keys(logits, SCORE[cfg.score_fn], sel_bias, cfg.num_groups, cfg.topk_groups)
+    scores, keys, cand = O.selection_keys(logits, SCORE[cfg.score_fn], sel_bias, cfg.num_groups, cfg.topk_groups,
+                                          cfg.temperature or 1.0)
     new, _ = O.reroute_over_capacity(idx, keys, cand, cfg.capacity)
     return new, O.gate_weights(scores, new, SCORE[cfg.score_fn], bool(cfg.renormalize))
 

@@ -75,6 +75,7 @@ BAD = [
     dict(num_groups=4, topk_groups=1, top_k=3), dict(num_shared=2), dict(capacity=-1), dict(num_tokens=-1),
     dict(renormalize=2), dict(activation=7), dict(act_dtype=5), dict(act_quant=2), dict(act_quant=-1),
     dict(reroute=2), dict(reroute=1),  # re-routing needs a capacity (mixtral_prefill has none)
+    dict(temperature=-0.5), dict(temperature=float("nan")), dict(temperature=float("inf")),
 ]
 
 
@@ -89,11 +90,23 @@ def test_invalid_desc_rejected(over):
                                   dict(weight_dtype=2, activation=0),
                                   dict(act_quant=1),                                  # W8A8 needs E4M3 weights
                                   dict(act_quant=1, weight_dtype=2, d_model=4104),    # d not a multiple of 16
-                                  dict(act_quant=1, weight_dtype=2, d_ff=14344)])     # h not a multiple of 16
+                                  dict(act_quant=1, weight_dtype=2, d_ff=14344),      # h not a multiple of 16
+                                  dict(score_fn=1, temperature=0.5)])                 # temperature: softmax only
 def test_unsupported_combination(over):
     d = _desc("mixtral_prefill", **over)
     n = ctypes.c_size_t(0)
     assert ops.lib().moe_workspace_size(ctypes.byref(d), ctypes.byref(n)) == ops.MOE_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("tau", [0.0, 1.0, 0.5, 2.0, 0.7])
+def test_temperature_accepted(tau):
+    n = ctypes.c_size_t(0)
+    assert ops.lib().moe_workspace_size(ctypes.byref(_desc("mixtral_prefill", temperature=tau)),
+                                        ctypes.byref(n)) == ops.MOE_OK
+    # a sigmoid router takes only tau = 1 (or 0, its spelling)
+    if tau in (0.0, 1.0):
+        assert ops.lib().moe_workspace_size(ctypes.byref(_desc("dsv3_grouped", temperature=tau)),
+                                            ctypes.byref(n)) == ops.MOE_OK
 
 
 def test_group_size_must_be_power_of_two():
@@ -254,10 +267,15 @@ def _struct_fields(text, name):
 
 def test_struct_layouts_match_the_header():
     """moe_desc and moe_weights as ctypes structures list the header's fields
-    in the header's order (int32 and pointer members only)."""
+    in the header's order with the header's member types (int32 and float
+    members of the descriptor, pointers of the weights)."""
     text = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "moe.h")).read(), flags=re.S)
     assert _struct_fields(text, "moe_desc") == list(ops.DESC_FIELDS)
     assert _struct_fields(text, "moe_weights") == list(ops.WEIGHT_FIELDS)
+    body = dict((n, b) for b, n in re.findall(r"typedef struct \{([^{}]*)\}\s*(\w+)\s*;", text))["moe_desc"]
+    types = dict((m.group(2), m.group(1)) for m in re.finditer(r"(int32_t|float)\s+([a-z_0-9]+)\s*;", body))
+    for name, ctype in ops.MoeDesc._fields_:
+        assert types[name] == ("float" if ctype is ctypes.c_float else "int32_t"), name
     assert ctypes.sizeof(ops.MoeDesc) == 4 * len(ops.DESC_FIELDS)
     assert ctypes.sizeof(ops.MoeWeights) == 8 * len(ops.WEIGHT_FIELDS)
 
@@ -279,8 +297,9 @@ def test_missing_library_fails_loudly():
     """No CPU fallback: without the built library the first call raises."""
     import subprocess
     import sys
+    missing = os.path.join(ROOT, "no_such_library.so")
     code = ("from mixture_experts_layer_bias_b200 import ops\n"
+            f"ops._LIB_PATH = {missing!r}\n"
             "try:\n    ops.lib()\nexcept RuntimeError as e:\n    print('raised', e)\n")
-    env = dict(os.environ, MOE_B200_LIB=os.path.join(ROOT, "no_such_library.so"))
-    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True, text=True)
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True)
     assert "raised" in r.stdout, (r.stdout, r.stderr)

@@ -1,12 +1,12 @@
 """Failure detection on the GPU without a GPU fault.
 
-Every wait inside the tensor-core GEMM is bounded in time.  A test hook
-(MOE_B200_TEST_STALL_GEMM=1) makes the next GEMM launch run with a producer
-that never delivers a tile -- a flag nothing sets -- so the MMA warp's wait
-must give up, raise MOE_STATUS_TIMEOUT in the status block and let the kernel
+Every wait inside the tensor-core GEMM is bounded in time.  A test hook,
+present only in the test build of the library (libmoe_b200_testhooks.so,
+moe_test_stall_gemms(1)), makes the next GEMM launch run with a producer that
+never delivers a tile -- a flag nothing sets -- so the MMA warp's wait must
+give up, raise MOE_STATUS_TIMEOUT in the status block and let the kernel
 exit.  The host reads the status, and the same CUDA context must then run a
-correct layer.  The hook is read once per process, so the check runs in a
-child process of its own.
+correct layer.  The test build is loaded in a child process of its own.
 """
 import json
 import os
@@ -24,6 +24,9 @@ import json, sys
 sys.path.insert(0, {root!r}); sys.path.insert(0, {tests!r})
 import torch
 from mixture_experts_layer_bias_b200 import ops, synthetic as syn
+from mixture_experts_layer_bias_b200.build import TEST_HOOKS_LIB
+ops._LIB_PATH = TEST_HOOKS_LIB
+ops.lib().moe_test_stall_gemms(1)
 from parity import run_layer, compare_layer
 cfg = syn.scaled(syn.CONFIGS["mixtral_prefill"], S=64, d=256, h=256)
 inp = syn.make_inputs(cfg, "cuda", seed=0)
@@ -39,10 +42,8 @@ print("RESULT " + json.dumps(dict(code1=code1, flags1=flags1, timeouts=cnt1["tim
 
 
 def test_bounded_wait_gives_up_and_context_survives():
-    env = dict(os.environ, MOE_B200_TEST_STALL_GEMM="1")
-    env.pop("MOE_B200_GEMM", None)  # the hook lives in the one-CTA kernel
     code = CHILD.format(root=ROOT, tests=os.path.join(ROOT, "tests"))
-    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-3000:]
     line = [l for l in r.stdout.splitlines() if l.startswith("RESULT ")][-1]
     res = json.loads(line[len("RESULT "):])

@@ -93,9 +93,20 @@ def _check_layer(cfg, inp, n_random=48, extra=(), seed=0):
     _, ridx_full, _, _ = oracle_routing(inp, cfg)
     toks = _sample_tokens(ridx_full, cfg.E, n_random, np.random.default_rng(seed), extra)
     rep = compare_layer(gpu, inp, cfg, toks)
+    # the load report computed on the device from the layer's counts
     counts = gpu["counts"].cpu().numpy()
-    rep["max_over_mean"] = O.load_stats(counts, cfg.K, cfg.S)["max_over_mean"]
+    stats = torch.full((ops.MOE_NUM_LOAD_STATS,), -1.0, dtype=torch.float64, device="cuda")
+    ops.moe_load_stats(gpu["desc"], gpu["counts"], stats)
+    got = dict(zip(ops.LOAD_STAT_NAMES, stats.cpu().tolist()))
+    ref = O.load_stats(counts, cfg.K, cfg.S, cfg.capacity)
+    for k in ops.LOAD_STAT_NAMES:
+        assert got[k] == pytest.approx(ref[k], rel=1e-12, abs=1e-9), (k, got, ref)
+    assert got["dropped"] == 0.0
+    rep["max_over_mean"] = got["max_over_mean"]
+    rep["load_std"] = got["std"]
     rep["overflow_rows"] = counters["overflow_rows"]
+    if cfg.capacity and not cfg.reroute:
+        assert got["overflow_rows"] == counters["overflow_rows"]
     print(cfg.name, rep)
     assert rep["ok"], rep
     return gpu, rep

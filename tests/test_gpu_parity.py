@@ -7,6 +7,8 @@ weights relative L2 <= 3e-2 against the oracle on the same decoded weights.
 Sizes span several tiles and ragged tails.
 """
 
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -348,19 +350,34 @@ def test_layer_dense_cross_check_tiny():
     assert max_abs_rel(np64(gpu["y"])[keep], dense[keep]) <= F32_MAXABS_REL
 
 
-@pytest.mark.parametrize("tau", [1.0, 2.0, 0.5])
+@pytest.mark.parametrize("tau", [1.0, 2.0, 0.5, 0.7])
 def test_soft_routing_with_temperature(tau):
     """Soft routing (jsqmd.com chapter 11, 11.3.3): y = sum_i softmax(s/tau)_i
-    E_i(x) over all experts.  The layer with K = E and renormalised gates
-    computes it when the router weights are scaled by 1/tau (a power of two
-    here, so the scaling is exact)."""
-    cfg = syn.scaled(syn.CONFIGS["tiny_f32"], K=8)
+    E_i(x) over all experts.  The layer with K = E, renormalised gates and
+    desc.temperature = tau computes it from the unscaled router weights."""
+    cfg = dataclasses.replace(syn.scaled(syn.CONFIGS["tiny_f32"], K=8), temperature=tau)
     inp = syn.make_inputs(cfg, "cuda", seed=4)
-    inp_t = dict(inp)
-    inp_t["w_router"] = inp["w_router"] / tau
-    gpu = run_layer(inp_t, cfg)
+    gpu = run_layer(inp, cfg)
     x = np64(inp["x"])
     logits = O.router_logits(x, np64(inp["w_router"]))
     fn = OracleExperts(inp, cfg)
     ref = O.soft_routing(x, logits, fn, cfg.E, tau)
     assert max_abs_rel(np64(gpu["y"]), ref) <= F32_MAXABS_REL
+    # the gates: every expert's softmax(l / tau) probability in the slot order
+    p = torch.softmax(torch.tensor(logits, dtype=torch.float64) / tau, dim=1).numpy()
+    idx = gpu["idx"].cpu().numpy()
+    assert max_abs_rel(gpu["w"].cpu().numpy(), np.take_along_axis(p, idx, 1)) <= F32_MAXABS_REL
+
+
+@pytest.mark.parametrize("tau", [0.5, 0.7, 2.0])
+def test_route_temperature_bit_exact_on_oracle_logits(tau):
+    """Top-8 of 64 with a temperature on oracle logits: indices bit-exact
+    (keys l / tau in float32 on both sides), gates within the fp32 bar."""
+    rng = np.random.default_rng(int(tau * 10))
+    S, E, K = 2000, 64, 8
+    logits = skewed_logits(rng, S, E, spread=2.0)
+    idx, gw, flags, _ = _route_gpu(_fields(S, E, K, temperature=tau), logits)
+    ridx, rw = O.select_experts(logits, K, temperature=tau)
+    np.testing.assert_array_equal(idx, ridx)
+    assert max_abs_rel(gw, rw) <= F32_MAXABS_REL
+    assert flags == 0

@@ -310,8 +310,17 @@ def test_overflow_region_is_expert_major():
 def test_load_stats_uniform_and_skewed():
     st = O.load_stats(np.array([4, 4, 4, 4]), 2, 8)
     assert st["max_over_mean"] == 1.0 and st["std"] == 0.0
-    st = O.load_stats(np.array([13, 1, 1, 1]), 2, 8)  # max/mean = 13/4
+    assert st["overflow_rows"] == 0 and st["dropped"] == 0
+    # S*K = 16 slots over 4 experts: mean 4; deviations 9, -3, -3, -3 -> variance
+    # (81 + 27) / 4 = 27, std = 3 * sqrt(3); capacity 3 leaves 13 - 3 = 10 rows over
+    st = O.load_stats(np.array([13, 1, 1, 1]), 2, 8, capacity=3)
     assert st["max_over_mean"] == pytest.approx(3.25)
+    assert st["std"] == pytest.approx(3.0 * math.sqrt(3.0), rel=1e-15)
+    assert st["mean"] == 4.0 and st["max"] == 13.0
+    assert st["overflow_rows"] == 10.0 and st["dropped"] == 0.0
+    # one slot with an out-of-range id is counted nowhere: dropped = 1
+    st = O.load_stats(np.array([12, 1, 1, 1]), 2, 8)
+    assert st["dropped"] == 1.0 and st["overflow_rows"] == 0.0
 
 
 # ----------------------------------------------------------------------------
@@ -414,6 +423,41 @@ def test_k_equals_e_is_soft_routing():
     l = rng.normal(size=(S, E)).astype(np.float32)
     idx, w = O.select_experts(l, E)
     np.testing.assert_allclose(O.moe_layer(x, idx, w, fn, E), O.soft_routing(x, l, fn, E, 1.0), rtol=1e-12)
+
+
+@pytest.mark.parametrize("tau", [0.5, 2.0, 0.7, 3.0])
+def test_temperature_k_equals_e_is_soft_routing(tau):
+    """With a temperature, K = E renormalised selection is the soft routing
+    y = sum_i softmax(s / tau)_i E_i(x) of chapter 11, 11.3.3 (computed there
+    in float64; here the tempered logit is one float32 division, so the two
+    agree to float32 rounding)."""
+    rng = np.random.default_rng(40)
+    S, d, E = 12, 8, 6
+    fn, _ = _rand_gelu_experts(rng, E, d, 10)
+    x = rng.normal(size=(S, d))
+    l = (3.0 * rng.normal(size=(S, E))).astype(np.float32)
+    idx, w = O.select_experts(l, E, temperature=tau)
+    np.testing.assert_allclose(O.moe_layer(x, idx, w, fn, E), O.soft_routing(x, l, fn, E, tau), rtol=2e-6)
+    # the gates themselves: softmax of l / tau over all experts, in each token's slot order
+    p = torch.softmax(torch.tensor(l, dtype=torch.float64) / tau, dim=1).numpy()
+    np.testing.assert_allclose(w, np.take_along_axis(p, idx, 1), rtol=2e-6)
+
+
+def test_temperature_keeps_the_order_and_sharpens_or_flattens_the_gates():
+    """tau > 0 divides every key alike, so the selected experts are those of
+    tau = 1 (keys far apart here); tau < 1 moves the top gate up and tau > 1
+    moves it toward 1/K, the limits of a softmax temperature."""
+    rng = np.random.default_rng(41)
+    l = rng.normal(size=(50, 16)).astype(np.float32) * 4.0
+    idx1, w1 = O.select_experts(l, 4)
+    for tau in (0.25, 4.0):
+        idx, w = O.select_experts(l, 4, temperature=tau)
+        np.testing.assert_array_equal(idx, idx1)
+        if tau < 1:
+            assert np.all(w[:, 0] >= w1[:, 0])
+        else:
+            assert np.all(w[:, 0] <= w1[:, 0]) and np.all(w[:, 0] >= 0.25)
+    assert np.array_equal(O.select_experts(l, 4, temperature=1.0)[1], w1)
 
 
 def test_capacity_does_not_change_the_layer():
