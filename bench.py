@@ -123,13 +123,15 @@ def kernels_per_step(cfg, S=None):
     """Launches of this library's kernels in one moe_layer_forward call."""
     S = cfg.S if S is None else S
     small = S * cfg.K <= 4096               # one-CTA permutation for small batches
-    n = 1 if (cfg.E <= 32) else 2          # route (fused) or logits GEMM + top-k
-    n += 1 if small else 4                 # permutation (+ group table): one kernel, or count, scan, scatter, groups
-    n += 1                                 # row gather (quantising for W8A8)
-    n += 2                                 # up and down GEMM
-    rows = S * cfg.K + cfg.num_shared * S + (cfg.E * cfg.capacity if cfg.capacity else 0)
-    if cfg.act_dtype == syn.BF16 and rows <= 4096:
-        n += 2                             # split-K finalize of both GEMMs
+    if not cfg.reroute and 1 <= S <= 16 and cfg.E <= 32 and small:
+        n = 1                              # routing, permutation and row gather in one kernel
+        if cfg.act_quant:
+            n += 1                         # the quantising row gather
+    else:
+        n = 1 if (cfg.E <= 32) else 2      # route (fused) or logits GEMM + top-k
+        n += 1 if small else 4             # permutation (+ group table): one kernel, or count, scan, scatter, groups
+        n += 1                             # row gather (quantising for W8A8)
+    n += 2                                 # up and down GEMM (split-K partial sums reduced inside them)
     if cfg.act_quant:
         n += 1                             # per-row E4M3 quantisation of the hidden rows
     elif cfg.weight_dtype == syn.E4M3:
@@ -488,8 +490,8 @@ def cpu_baseline(cfg, inp, n_tokens, one_core_tokens):
 
 # sample sizes of the oracle baseline per workload: (layer tokens, 1-core layer tokens)
 CPU_SAMPLES = {"mixtral_prefill": (32, 8), "tiny_f32": (64, 64), "dsv3_grouped": (4, 1),
-               "fp8_skew_capacity": (32, 8), "mixtral_prefill_w8a8": (8, 2), "fp8_skew_capacity_w8a8": (16, 4),
-               "fp8_skew_capacity_reroute": (32, 8)}
+               "fp8_skew_capacity": (16, 4), "mixtral_prefill_w8a8": (2, 1), "fp8_skew_capacity_w8a8": (8, 2),
+               "fp8_skew_capacity_reroute": (16, 4), "mixtral_decode": (1, 1)}
 
 
 def run_reference(args, rank, world):

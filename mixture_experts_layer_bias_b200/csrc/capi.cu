@@ -20,10 +20,17 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 
 struct Layout {
-  size_t status, logits, chunk_hist, groups, counts, offsets, topk_idx, topk_w, row_of_slot, token_of_row,
-      x_perm, hidden, y_perm, wdeq, ksplit, partial, partial_bytes, qa, sa, qas, sas, qh, sh, rr_key, rr_score,
-      rr_ex, rr_changed, total;
+  size_t status, counters, logits, chunk_hist, groups, counts, offsets, topk_idx, topk_w, row_of_slot,
+      token_of_row, x_perm, hidden, y_perm, wdeq, partial, partial_bytes, qa, sa, qas, sas, qh, sh, rr_key,
+      rr_score, rr_ex, rr_changed, total;
 };
+
+// Split-K arrival counters of the grouped GEMMs: a fixed region right after
+// the status block, the same for every desc, so a workspace reused across
+// descs (e.g. decode batches of varying size) keeps them valid.  They are zero
+// after moe_workspace_init and every completed GEMM leaves them zero.
+constexpr size_t kCounterInts = 65536;
+constexpr size_t kCounterBytes = kCounterInts * 4;
 
 // Split-K of the tensor-core GEMMs is available to small row spaces (decode-
 // sized batches), where too few output tiles exist to occupy every SM.  The
@@ -52,6 +59,7 @@ Layout make_layout(const moe_desc& d) {
     return at;
   };
   L.status = take(kAlign);
+  L.counters = take(kCounterBytes);
   L.logits = take(E > 32 ? static_cast<size_t>(S * E) * 4 : 0);
   L.chunk_hist = take(static_cast<size_t>(nch * E) * 4);
   L.groups = take(static_cast<size_t>(2 * E + 1) * sizeof(GroupEntry));
@@ -80,7 +88,6 @@ Layout make_layout(const moe_desc& d) {
   L.rr_score = take(rr ? static_cast<size_t>(S * E) * 4 : 0);
   L.rr_ex = take(rr ? static_cast<size_t>(S * K) * 4 : 0);
   L.rr_changed = take(rr ? static_cast<size_t>(S) * 4 : 0);
-  L.ksplit = take(kAlign);
   L.partial_bytes = 0;
   if (d.act_dtype == MOE_BF16 && Rt > 0 && Rt <= kSplitRowsMax) {
     const int64_t up_cols = d.activation == MOE_ACT_SWIGLU ? 2 * h : h;
@@ -164,8 +171,8 @@ int num_sms() {
   return n;
 }
 
-moe_status route_impl(const moe_desc& d, const moe_weights* w, const void* x, const float* logits_in,
-                      int32_t* topk_idx, float* topk_w, void* ws, cudaStream_t st) {
+RouteArgs route_args(const moe_desc& d, const moe_weights* w, const void* x, const float* logits_in,
+                     int32_t* topk_idx, float* topk_w, void* ws) {
   const Layout L = make_layout(d);
   RouteArgs a{};
   a.S = d.num_tokens;
@@ -192,12 +199,16 @@ moe_status route_impl(const moe_desc& d, const moe_weights* w, const void* x, co
     a.cand_key_out = at<float>(ws, L.rr_key);
     a.score_out = at<float>(ws, L.rr_score);
   }
-  return cuda_status(launch_route(a, st));
+  return a;
 }
 
-moe_status permute_impl(const moe_desc& d, const void* x, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
-                        int32_t* row_of_slot, int32_t* token_of_row, void* x_perm, void* ws, cudaStream_t st,
-                        bool write_groups = false) {
+moe_status route_impl(const moe_desc& d, const moe_weights* w, const void* x, const float* logits_in,
+                      int32_t* topk_idx, float* topk_w, void* ws, cudaStream_t st) {
+  return cuda_status(launch_route(route_args(d, w, x, logits_in, topk_idx, topk_w, ws), st));
+}
+
+PermuteArgs permute_args(const moe_desc& d, const void* x, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                         int32_t* row_of_slot, int32_t* token_of_row, void* x_perm, void* ws, bool write_groups) {
   const Layout L = make_layout(d);
   PermuteArgs a{};
   a.S = d.num_tokens;
@@ -220,11 +231,16 @@ moe_status permute_impl(const moe_desc& d, const void* x, const int32_t* topk_id
     a.g1 = at<GroupEntry>(ws, L.groups);
     a.num_shared = d.num_shared;
   }
-  return cuda_status(launch_permute(a, st));
+  return a;
 }
 
-// a_quantized (W8A8): the up projection's E4M3 rows and scales are already in
-// the workspace (written by the quantising gather), x_perm is not read.
+moe_status permute_impl(const moe_desc& d, const void* x, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                        int32_t* row_of_slot, int32_t* token_of_row, void* x_perm, void* ws, cudaStream_t st,
+                        bool write_groups = false) {
+  return cuda_status(launch_permute(
+      permute_args(d, x, topk_idx, counts, offsets, row_of_slot, token_of_row, x_perm, ws, write_groups), st));
+}
+
 // Record stage event `i` of `events` (moe_layer_forward_timed), if given.
 bool record(void* const* events, int i, cudaStream_t st) {
   if (events == nullptr || events[i] == nullptr) return true;
@@ -271,7 +287,8 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
   up.status = status;
   up.partial = L.partial_bytes ? at<float>(ws, L.partial) : nullptr;
   up.partial_bytes = static_cast<int64_t>(L.partial_bytes);
-  up.ksplit_out = at<int>(ws, L.ksplit);
+  up.tile_count = at<int>(ws, L.counters);
+  up.tile_count_len = static_cast<int64_t>(kCounterInts);
 
   GemmArgs down = up;
   down.a_rows_from_out = 1;
@@ -433,6 +450,26 @@ moe_status layer_impl(const moe_desc* desc, const moe_weights* w, const void* x,
   void* x_perm = at<void>(ws, L.x_perm);
   void* y_perm = at<void>(ws, L.y_perm);
   if (!record(events, 0, st)) return MOE_ERR_CUDA;
+  const bool w8a8 = d.act_quant == 1;
+  if (d.reroute == 0 && route_permute_fusable(d.num_tokens, d.num_experts, d.top_k)) {
+    // tiny batch: routing, permutation (with the group tables) and the row
+    // gather in one kernel; W8A8 gathers E4M3 codes in its own kernel below
+    const RouteArgs ra = route_args(d, w, x, nullptr, idx, gates, ws);
+    const PermuteArgs pa = permute_args(d, x, idx, cnt, offs, ros, tor, w8a8 ? nullptr : x_perm, ws, true);
+    if (launch_route_permute_small(ra, pa, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (!record(events, 1, st)) return MOE_ERR_CUDA;
+    if (w8a8) {
+      const bool sh = d.num_shared != 0;
+      if (launch_gather_quantize(d.num_tokens, d.d_model, d.top_k, ros, x, at<uint8_t>(ws, L.qa),
+                                 at<float>(ws, L.sa), sh ? at<uint8_t>(ws, L.qas) : nullptr,
+                                 sh ? at<float>(ws, L.sas) : nullptr, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+    if (!record(events, 2, st)) return MOE_ERR_CUDA;
+    if ((s = ffn_impl(d, *w, x_perm, offs, x, y_perm, ws, st, true, w8a8, events)) != MOE_OK) return s;
+    if ((s = combine_impl(d, y_perm, ros, gates, y, st)) != MOE_OK) return s;
+    return record(events, 7, st) ? MOE_OK : MOE_ERR_CUDA;
+  }
   if ((s = route_impl(d, w, x, nullptr, idx, gates, ws, st)) != MOE_OK) return s;
   if (d.reroute == 1) {
     // capacity ranks of the first choices, then the excess slots move; the
@@ -442,7 +479,7 @@ moe_status layer_impl(const moe_desc* desc, const moe_weights* w, const void* x,
   }
   if (!record(events, 1, st)) return MOE_ERR_CUDA;
   // the permutation also writes the GEMM group tables, so the FFN skips that launch
-  if (d.act_quant == 1) {
+  if (w8a8) {
     // W8A8: the row gather writes E4M3 codes and row scales straight away
     // (no bf16 copy of the permuted rows)
     if ((s = permute_impl(d, nullptr, idx, cnt, offs, ros, tor, nullptr, ws, st, true)) != MOE_OK) return s;
@@ -482,7 +519,9 @@ moe_status moe_workspace_size(const moe_desc* desc, size_t* bytes) {
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   if (ws == nullptr || ws_bytes < kAlign || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0)
     return MOE_ERR_WORKSPACE;
-  return cuda_status(cudaMemsetAsync(ws, 0, kAlign, static_cast<cudaStream_t>(stream)));
+  // status block and the GEMMs' split-K arrival counters
+  const size_t n = ws_bytes < kAlign + kCounterBytes ? ws_bytes : kAlign + kCounterBytes;
+  return cuda_status(cudaMemsetAsync(ws, 0, n, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_route(const moe_desc* desc, const moe_weights* w, const void* x, const float* logits_in,

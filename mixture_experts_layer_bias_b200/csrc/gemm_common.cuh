@@ -1,6 +1,6 @@
-// Pieces shared by the tensor-core grouped GEMM kernels: launch parameters,
-// group lookup, the device-side split-K choice, the split-K finalize kernel
-// and tensor-map encoding.
+// Pieces shared by the tensor-core grouped GEMM kernel: launch parameters,
+// group lookup, the device-side split-K choice, the split-K reduction of the
+// last-arriving slice and tensor-map encoding.
 #pragma once
 
 #include <math.h>
@@ -33,7 +33,8 @@ struct TcParams {
   int max_ksplit;      // 1 = no split-K
   float* partial;      // fp32 [max_ksplit][out_rows][pcols] (split-K partial sums)
   int pcols;           // 2N (SwiGLU: gate then up) or N
-  int* ksplit_out;     // the split chosen on the device, read by the finalize kernel
+  int* tile_count;     // split-K arrival counters, kRegionsPerTile per tile, zero between launches
+  int max_tiles;       // tiles the counters cover (more tiles: no split-K)
   int test_stall;      // test hook: the producer delivers nothing (the bounded waits must give up)
   int tma_out;         // 1: the output tensor map is valid (full 32-row quarters use bulk tensor stores)
   const float* row_scale;         // E4M3 activations: per-row scale of the A operand rows (nullptr: none)
@@ -80,54 +81,90 @@ __device__ __forceinline__ bool group_ok(const GroupEntry& g, const TcParams& p)
          static_cast<int64_t>(g.out_row0) + g.rows <= p.out_rows && g.a_row0 >= 0;
 }
 
-// Split-K finalize: for every valid row of every group, sum the partial
-// slices in split order (deterministic), apply scales / bias / activation and
-// store the output row.  Exits at once when the GEMM ran without a split.
+// Split-K: every epilogue warp of a CTA owns one region of its tile (32 rows
+// of one TMEM lane quarter x half of the tile's columns) and, per split, writes
+// its raw fp32 accumulators there to the split's slice of the partial buffer.
+// One arrival counter per (tile, region) counts the slices written; the warp
+// whose slice completes the count sums the region's slices in split order
+// (deterministic whatever the arrival order), applies the epilogue and stores
+// the output rows, then resets the counter for the next launch.
+constexpr int kRegionsPerTile = 8;
+
+// The last arriver's reduction of region (q, half) of tile `ti`: rows
+// m_idx*128 + q*32 .. +31 of the group, lane j taking output columns
+// n0 + 2j, n0 + 2j + 1 (SwiGLU, 64 columns per half: gate at n, up at N + n
+// in the slices) or n0 + 4j .. n0 + 4j + 3 (128 columns per half).  Partial
+// sums are read at L2 (ld.global.cg): other CTAs wrote them in this launch.
 template <int EPI>
-__global__ void __launch_bounds__(256) splitk_finalize_kernel(TcParams p) {
-  const int ks = *p.ksplit_out;
-  if (ks <= 1) return;
-  const GroupEntry grp = group_at(p, blockIdx.z);
-  const int r = blockIdx.y;
-  if (r >= grp.rows || grp.expert < 0 || grp.expert >= p.num_slabs) return;
-  const int n = (blockIdx.x * 256 + threadIdx.x) * 4;
+__device__ __forceinline__ void splitk_reduce_region(const TcParams& p, const GroupEntry& grp, int m_row0, int n_tile,
+                                                     int ks, int half, int lane) {
   const int N = p.N;
-  if (n >= N) return;
-  const int64_t orow = static_cast<int64_t>(grp.out_row0) + r;
-  if (orow >= p.out_rows) return;
-  const int64_t sbase = static_cast<int64_t>(grp.expert) * N;
   const int64_t slice = p.out_rows * static_cast<int64_t>(p.pcols);
-  const float rs = a_row_scale(p, grp, r);
-  float v[4] = {0.f, 0.f, 0.f, 0.f}, u[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int s = 0; s < ks; ++s) {
-    const float* src = p.partial + s * slice + orow * p.pcols;
-    const float4 a = *reinterpret_cast<const float4*>(src + n);
-    v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
-    if (EPI == EPI_SWIGLU) {
-      const float4 b = *reinterpret_cast<const float4*>(src + N + n);
-      u[0] += b.x; u[1] += b.y; u[2] += b.z; u[3] += b.w;
+  const int64_t sbase = static_cast<int64_t>(grp.expert) * N;
+  const int r1 = min(m_row0 + 32, grp.rows);
+  if (EPI == EPI_SWIGLU) {
+    const int n = n_tile * p.bn_out + half * 64 + 2 * lane;
+    if (n >= N) return;  // N is a multiple of 8, so n + 1 < N as well
+    float c0[2] = {1.0f, 1.0f}, c1[2] = {1.0f, 1.0f};
+    if (p.scale0 != nullptr) { c0[0] = p.scale0[sbase + n]; c0[1] = p.scale0[sbase + n + 1]; }
+    if (p.scale1 != nullptr) { c1[0] = p.scale1[sbase + n]; c1[1] = p.scale1[sbase + n + 1]; }
+    for (int r = m_row0; r < r1; ++r) {
+      const int64_t orow = static_cast<int64_t>(grp.out_row0) + r;
+      const float rs = a_row_scale(p, grp, r);
+      float g[2] = {0.f, 0.f}, u[2] = {0.f, 0.f};
+      for (int s = 0; s < ks; ++s) {
+        const float* src = p.partial + s * slice + orow * p.pcols;
+        const float2 a = __ldcg(reinterpret_cast<const float2*>(src + n));
+        const float2 b = __ldcg(reinterpret_cast<const float2*>(src + N + n));
+        g[0] += a.x; g[1] += a.y; u[0] += b.x; u[1] += b.y;
+      }
+      float o[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float gv = g[j] * rs;
+        if (p.scale0 != nullptr) gv *= c0[j];
+        float uv = u[j] * rs;
+        if (p.scale1 != nullptr) uv *= c1[j];
+        o[j] = gv / (1.0f + __expf(-gv)) * uv;
+      }
+      if (p.out_f32)
+        *reinterpret_cast<float2*>(static_cast<float*>(p.out) + orow * N + n) = make_float2(o[0], o[1]);
+      else
+        *reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(p.out) + orow * N + n) = pack_bf16x2(o[0], o[1]);
     }
+    return;
   }
-  float o[4];
+  const int n = n_tile * p.bn_out + half * 128 + 4 * lane;
+  if (n >= N) return;  // n is a multiple of 4 and N of 8: n + 3 < N
+  float cs[4] = {1.f, 1.f, 1.f, 1.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    float g = v[j] * rs;
-    if (p.scale0 != nullptr) g *= p.scale0[sbase + n + j];
-    if (EPI == EPI_SWIGLU) {
-      float up = u[j] * rs;
-      if (p.scale1 != nullptr) up *= p.scale1[sbase + n + j];
-      o[j] = g / (1.0f + __expf(-g)) * up;
-    } else {
-      if (EPI == EPI_GELU_BIAS || EPI == EPI_BIAS) g += p.bias[sbase + n + j];
-      if (EPI == EPI_GELU_BIAS) g = 0.5f * g * (1.0f + erff(g * 0.70710678118654752f));
-      o[j] = g;
-    }
+    if (p.scale0 != nullptr) cs[j] = p.scale0[sbase + n + j];
+    if (EPI == EPI_GELU_BIAS || EPI == EPI_BIAS) cb[j] = p.bias[sbase + n + j];
   }
-  if (p.out_f32) {
-    *reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * N + n) = make_float4(o[0], o[1], o[2], o[3]);
-  } else {
-    uint2 packed = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
-    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + orow * N + n) = packed;
+  for (int r = m_row0; r < r1; ++r) {
+    const int64_t orow = static_cast<int64_t>(grp.out_row0) + r;
+    const float rs = a_row_scale(p, grp, r);
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < ks; ++s) {
+      const float4 a = __ldcg(reinterpret_cast<const float4*>(p.partial + s * slice + orow * p.pcols + n));
+      v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+    }
+    float o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float z = v[j] * rs;
+      if (p.scale0 != nullptr) z *= cs[j];
+      if (EPI == EPI_GELU_BIAS || EPI == EPI_BIAS) z += cb[j];
+      if (EPI == EPI_GELU_BIAS) z = 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
+      o[j] = z;
+    }
+    if (p.out_f32) {
+      *reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * N + n) = make_float4(o[0], o[1], o[2], o[3]);
+    } else {
+      const uint2 packed = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
+      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + orow * N + n) = packed;
+    }
   }
 }
 

@@ -50,9 +50,10 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t 
   p.status = a.status;
   p.pcols = a.epilogue == EPI_SWIGLU ? 2 * a.N : a.N;
   p.partial = a.partial;
-  p.ksplit_out = a.ksplit_out;
+  p.tile_count = a.tile_count;
+  p.max_tiles = static_cast<int>(a.tile_count_len / kRegionsPerTile);
   p.max_ksplit = 1;
-  if (a.partial != nullptr && a.ksplit_out != nullptr && a.partial_bytes > 0) {
+  if (a.partial != nullptr && a.tile_count != nullptr && a.partial_bytes > 0 && p.max_tiles > 0) {
     // as many K slices as the partial buffer holds for every output row
     const int64_t per_split = a.out_rows * static_cast<int64_t>(p.pcols) * 4;
     p.max_ksplit = static_cast<int>(per_split > 0 ? a.partial_bytes / per_split : 1);

@@ -43,6 +43,7 @@
 #include <string.h>
 
 #include "gemm_common.cuh"
+#include "pdl.cuh"
 
 namespace moe {
 
@@ -218,15 +219,20 @@ __device__ __forceinline__ void epilogue_store(const TcParams& p, const TileInfo
 }
 
 // Split-K epilogue: raw fp32 accumulators of this unit's K range go to its
-// slice of the partial buffer (SwiGLU: gate columns at n, up columns at N+n).
+// slice of the partial buffer, for the warp's region of the tile: rows of its
+// TMEM lane quarter, and half of the tile's columns -- SwiGLU: output columns
+// half*64 .. +63, i.e. gate chunks {2 half, 2 half + 1} and up chunks
+// {4 + 2 half, 5 + 2 half}, gate stored at column n and up at N + n; other
+// epilogues: columns half*128 .. +127.  A region is then complete in itself
+// (splitk_reduce_region).
 template <int EPI>
 __device__ __forceinline__ void epilogue_partial(const TcParams& p, const TileInfo& ti, uint32_t tbase, int row,
                                                  bool valid, int split, int half) {
   const int N = p.N;
   const int64_t orow = static_cast<int64_t>(ti.grp.out_row0) + row;
   float* base = p.partial + (static_cast<int64_t>(split) * p.out_rows + orow) * p.pcols;
-  constexpr int kChunks = 8;  // 256 accumulator columns, half of them per warp
-  for (int c = half * 4; c < half * 4 + 4; ++c) {
+  for (int i = 0; i < 4; ++i) {
+    const int c = (EPI == EPI_SWIGLU) ? ((i < 2 ? 0 : 4) + 2 * half + (i & 1)) : (half * 4 + i);
     uint32_t r[32];
     tmem_ld_32x32b_x32(tbase + c * 32, r);
     tmem_ld_wait();
@@ -262,6 +268,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(ring + STAGES * STAGE_BYTES + sizeof(SmemCtl)) + 127) & ~uintptr_t(127));
   const int warp = threadIdx.x >> 5, lane = lane_id();
 
+  // Prologue that needs nothing from earlier kernels (barriers, TMEM, tensor
+  // map prefetch) runs first; under programmatic dependent launch it overlaps
+  // the previous kernel, and the wait below is where this grid first needs
+  // that kernel's results (group table, A rows, partial buffer).
+  if (warp == 1) {
+    if (lane == 0) {
+      for (int i = 0; i < STAGES; ++i) {
+        mbar_init(&s.full[i], 1);
+        mbar_init(&s.empty[i], 1);
+      }
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&s.tfull[i], 1);
+        mbar_init(&s.tempty[i], 32 * kEpiWarps);
+      }
+      mbar_init(&s.drain, 1);
+      s.abort = 0;
+      fence_mbar_init();
+    }
+    __syncwarp();
+    tmem_alloc(&s.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  } else if (warp == 2 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmA2);
+    tma_prefetch_desc(&tmB0);
+    tma_prefetch_desc(&tmB1);
+  }
+  pdl_wait();
+  pdl_trigger();
   // per-group tile counts -> exclusive prefix (warp 0)
   if (warp == 0) {
     int carry = 0;
@@ -285,28 +320,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
     }
     if (lane == 0) s.tile_start[p.num_groups] = carry;
-  } else if (warp == 1) {
-    if (lane == 0) {
-      for (int i = 0; i < STAGES; ++i) {
-        mbar_init(&s.full[i], 1);
-        mbar_init(&s.empty[i], 1);
-      }
-      for (int i = 0; i < 2; ++i) {
-        mbar_init(&s.tfull[i], 1);
-        mbar_init(&s.tempty[i], 32 * kEpiWarps);
-      }
-      mbar_init(&s.drain, 1);
-      s.abort = 0;
-      fence_mbar_init();
-    }
-    __syncwarp();
-    tmem_alloc(&s.tmem_base, TMEM_COLS);
-    tmem_relinquish();
-  } else if (warp == 2 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmA2);
-    tma_prefetch_desc(&tmB0);
-    tma_prefetch_desc(&tmB1);
   }
   tc_fence_before();
   __syncthreads();
@@ -315,8 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s.tmem_base;
   const int nk = (p.K + BK - 1) / BK;
   const int tiles = s.tile_start[p.num_groups];
-  const int ks = choose_ksplit(tiles, gridDim.x, nk, p.max_ksplit);
-  if (blockIdx.x == 0 && threadIdx.x == 0 && p.ksplit_out != nullptr) *p.ksplit_out = ks;
+  // split-K only while every tile has its arrival counters
+  const int ks = tiles <= p.max_tiles ? choose_ksplit(tiles, gridDim.x, nk, p.max_ksplit) : 1;
   const int total = tiles * ks;  // work units
   volatile int* abort_flag = &s.abort;
 
@@ -443,6 +456,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         epilogue_store<EPI>(p, ti, tbase, row, valid, lane, half, &tmOut, epi_smem + (warp - 2) * kEpiWarpBytes);
       tc_fence_before();
       mbar_arrive(&s.tempty[acc]);
+      if (ks > 1) {
+        // publish this slice of the warp's region, count it; the warp that
+        // completes the count reduces the region's slices
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        int* counter = p.tile_count + static_cast<int64_t>(u / ks) * kRegionsPerTile + q * 2 + half;
+        if (lane == 0) {
+          last = atomicAdd(counter, 1) == ks - 1;
+          if (last) {
+            *counter = 0;  // ready for the next launch
+            __threadfence();
+          }
+        }
+        if (__shfl_sync(0xFFFFFFFFu, last, 0))
+          splitk_reduce_region<EPI>(p, ti.grp, ti.m_idx * BM + q * 32, ti.n_idx, ks, half, lane);
+      }
     }
   }
 
@@ -458,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int EPI, bool F8>
 cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB0, const CUtensorMap& mB1,
                        const CUtensorMap& mOut, const TcParams& p, int grid, int bma, int stages, size_t smem,
-                       int64_t max_group_rows, cudaStream_t stream) {
+                       cudaStream_t stream) {
   static uint64_t attr_set = 0;  // one bit per device ordinal
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -469,11 +499,10 @@ cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUte
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set |= 1ull << dev;
   }
-  grouped_gemm_tc_kernel<EPI, F8><<<grid, kThreads, smem, stream>>>(mA, mA2, mB0, mB1, mOut, p, bma, stages);
-  e = cudaGetLastError();
-  if (e != cudaSuccess || p.max_ksplit <= 1) return e;
-  dim3 fgrid((p.N + 1023) / 1024, static_cast<unsigned>(max_group_rows), p.num_groups);
-  splitk_finalize_kernel<EPI><<<fgrid, 256, 0, stream>>>(p);
+  // programmatic dependent launch: the prologue may overlap the previous kernel
+  e = launch_pdl(grouped_gemm_tc_kernel<EPI, F8>, dim3(grid), dim3(kThreads), smem, stream, mA, mA2, mB0, mB1, mOut,
+                 p, bma, stages);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -512,22 +541,21 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
   if (a.fp8) {  // W8A8 runs SwiGLU experts only
     switch (a.epilogue) {
       case EPI_SWIGLU:
-        return launch_epi<EPI_SWIGLU, true>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
+        return launch_epi<EPI_SWIGLU, true>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, stream);
       case EPI_NONE:
-        return launch_epi<EPI_NONE, true>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
+        return launch_epi<EPI_NONE, true>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, stream);
       default: return cudaErrorInvalidValue;
     }
   }
   switch (a.epilogue) {
     case EPI_SWIGLU:
-      return launch_epi<EPI_SWIGLU, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
+      return launch_epi<EPI_SWIGLU, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, stream);
     case EPI_GELU_BIAS:
-      return launch_epi<EPI_GELU_BIAS, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem,
-                                              a.max_group_rows, stream);
+      return launch_epi<EPI_GELU_BIAS, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, stream);
     case EPI_BIAS:
-      return launch_epi<EPI_BIAS, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
+      return launch_epi<EPI_BIAS, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, stream);
     case EPI_NONE:
-      return launch_epi<EPI_NONE, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
+      return launch_epi<EPI_NONE, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, stream);
     default: return cudaErrorInvalidValue;
   }
 }

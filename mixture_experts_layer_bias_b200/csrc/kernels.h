@@ -69,6 +69,11 @@ struct PermuteArgs {
   GroupEntry* g1;
   int num_shared;
 };
+// Tiny batches: routing (logits computed from x, E <= 32), the single-CTA
+// permutation with group tables, and the row gather (pa.x_perm, or none when
+// NULL) in one kernel.  route_permute_fusable says which batches qualify.
+bool route_permute_fusable(int S, int E, int K);
+cudaError_t launch_route_permute_small(const RouteArgs& ra, const PermuteArgs& pa, cudaStream_t stream);
 int permute_num_chunks(int S, int K);
 int permute_tokens_per_chunk(int K);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream);
@@ -107,7 +112,8 @@ struct GemmArgs {
   int64_t max_group_rows;   // upper bound of the rows of one group
   float* partial;           // split-K partial sums (nullptr = no split-K)
   int64_t partial_bytes;    // size of `partial`
-  int* ksplit_out;          // device int: the split the GEMM chose
+  int* tile_count;          // split-K arrival counters (zero between launches; nullptr = no split-K)
+  int64_t tile_count_len;   // number of counters
   int fp8;                  // 1: A and B are E4M3 (kind::f8f6f4); A rows scaled by row_scale
   const float* row_scale;        // [a rows] per-row scale of A (fp8 only)
   const float* row_scale_shared; // [S] per-row scale of the shared expert's A rows (fp8 only)

@@ -19,291 +19,81 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "pdl.cuh"
+#include "route_select.cuh"
 
 namespace moe {
 
 namespace {
 
-constexpr unsigned kFull = 0xFFFFFFFFu;
-
-// exp(z) in float32 by Cody-Waite range reduction and the degree-7 Taylor
-// polynomial, each step one IEEE float32 operation with round-to-nearest:
-//   n = rint(z * log2 e), r = (z - n * ln2_hi) - n * ln2_lo,
-//   p = 1 + r (1 + r (1/2! + r (1/3! + ... + r / 7!))), result = p * 2^n.
-// ln2_hi is ln 2 truncated to 16 significant bits (so n * ln2_hi is exact for
-// |n| < 256) and ln2_lo the float32 rounding of the remainder; the Taylor
-// coefficients are the float32 roundings of 1/j!.  z > 88 gives +inf and
-// z < -30 gives 0 (there 1 + exp(z) rounds to 1 anyway).
-__device__ __forceinline__ float exp_cw_f32(float z) {
-  if (z > 88.0f) return __int_as_float(0x7f800000);
-  if (z < -30.0f) return 0.0f;
-  const float kLog2e = __int_as_float(0x3fb8aa3b);   // 1/ln 2
-  const float kLn2Hi = __int_as_float(0x3f317200);   // 0.693145751953125
-  const float kLn2Lo = __int_as_float(0x35bfbe8e);   // ln 2 - kLn2Hi
-  const float n = rintf(__fmul_rn(z, kLog2e));
-  float r = __fsub_rn(z, __fmul_rn(n, kLn2Hi));
-  r = __fsub_rn(r, __fmul_rn(n, kLn2Lo));
-  float p = __int_as_float(0x39500d01);                  // 1/7!
-  p = __fadd_rn(__fmul_rn(p, r), __int_as_float(0x3ab60b61));  // 1/6!
-  p = __fadd_rn(__fmul_rn(p, r), __int_as_float(0x3c088889));  // 1/5!
-  p = __fadd_rn(__fmul_rn(p, r), __int_as_float(0x3d2aaaab));  // 1/4!
-  p = __fadd_rn(__fmul_rn(p, r), __int_as_float(0x3e2aaaab));  // 1/3!
-  p = __fadd_rn(__fmul_rn(p, r), 0.5f);                        // 1/2!
-  p = __fadd_rn(__fmul_rn(p, r), 1.0f);                        // 1/1!
-  p = __fadd_rn(__fmul_rn(p, r), 1.0f);                        // 1/0!
-  return ldexpf(p, static_cast<int>(n));
-}
-
-// sigma(l) = 1 / (1 + exp(-l)) with the exponential above.
-__device__ __forceinline__ float sigmoid_sel_f32(float l) {
-  return __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_cw_f32(-l)));
-}
-
-__device__ __forceinline__ void warp_argmax(float& v, int& idx) {
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) {
-    const float ov = __shfl_xor_sync(kFull, v, off);
-    const int oi = __shfl_xor_sync(kFull, idx, off);
-    if (ov > v || (ov == v && oi < idx)) {
-      v = ov;
-      idx = oi;
-    }
-  }
-}
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
-  return v;
-}
-
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, off));
-  return v;
-}
-
-struct SelectParams {
-  int E, K, score_fn, renormalize, num_groups, topk_groups;
-  float tau;  // softmax temperature (1 = none): z = l / tau
-  const float* sel_bias;
-  int32_t* topk_idx;
-  float* topk_w;
-  StatusBlock* status;
-  float* cand_key;   // optional [S][E]: selection key of each candidate expert, -inf for the others
-  float* score_out;  // optional [S][E]: the gate source (logit, or sigmoid score) of every expert
-};
-
-// Gate of this lane's selected expert (lanes < K hold one each, my_score its
-// score); score[]/valid[] are the token's scores of experts 32*i + lane.
-template <int NI>
-__device__ __forceinline__ float gate_of(const float (&score)[NI], const bool (&valid)[NI], float my_score,
-                                         bool mine, int score_fn, int renormalize) {
-  const float kNegInf = __int_as_float(0xff800000);
-  if (score_fn == MOE_SCORE_SOFTMAX) {
-    if (renormalize) {
-      const float m = warp_max(mine ? my_score : kNegInf);
-      const float ex = mine ? expf(my_score - m) : 0.0f;
-      return ex / warp_sum(ex);
-    }
-    float m = kNegInf;
-#pragma unroll
-    for (int i = 0; i < NI; ++i)
-      if (valid[i]) m = fmaxf(m, score[i]);
-    m = warp_max(m);
-    float s = 0.0f;
-#pragma unroll
-    for (int i = 0; i < NI; ++i)
-      if (valid[i]) s += expf(score[i] - m);
-    s = warp_sum(s);
-    return expf(my_score - m) / s;
-  }
-  if (renormalize) {
-    const float s = warp_sum(mine ? my_score : 0.0f);
-    return my_score / s;
-  }
-  return my_score;
-}
-
-// Selection for one token held by the whole warp: l[i] is the logit (router
-// bias included) of expert 32*i + lane.  Writes K indices and gates.
-// Softmax scores are the logits divided by the temperature (jsqmd.com
-// 11.3.3, soft routing with softmax(s / tau)).
-template <int NI>
-__device__ void select_topk(const float (&l)[NI], const SelectParams& p, int t) {
-  const int lane = lane_id();
-  const int E = p.E;
-  const float kNegInf = __int_as_float(0xff800000);
-  float score[NI], key[NI];
-  bool valid[NI], cand[NI], taken[NI];
-  bool nonfinite = false;
-#pragma unroll
-  for (int i = 0; i < NI; ++i) {
-    const int e = 32 * i + lane;
-    valid[i] = e < E;
-    const float li = valid[i] ? l[i] : kNegInf;
-    if (valid[i] && !isfinite(li)) nonfinite = true;
-    // softmax: the tempered logit z = l / tau (one float32 division, exact for
-    // tau = 1) is both the gate source and the key; sigmoid: sigma(l)
-    score[i] = (p.score_fn == MOE_SCORE_SIGMOID) ? sigmoid_sel_f32(li) : __fdiv_rn(li, p.tau);
-    float k = score[i];
-    if (valid[i] && p.sel_bias != nullptr) k = __fadd_rn(k, __ldg(p.sel_bias + e));
-    if (!valid[i] || isnan(k)) k = kNegInf;
-    key[i] = k;
-    cand[i] = valid[i];
-    taken[i] = false;
-  }
-  if (__any_sync(kFull, nonfinite) && lane == 0) report(p.status, MOE_STATUS_NONFINITE_LOGIT, MOE_CNT_NONFINITE);
-
-  if (p.num_groups > 1) {
-    const int gs = E / p.num_groups;  // power of two
-    float gsum[NI];
-    if (gs >= 32) {
-      // members of group g: registers g*r .. g*r + r - 1 in every lane.  The
-      // halving tree first adds register j to register j + r/2 (member m to
-      // m + gs/2), down to single registers, then goes across lanes.
-      const int r = gs >> 5;
-      float v[NI];
-#pragma unroll
-      for (int i = 0; i < NI; ++i) v[i] = key[i];
-#pragma unroll
-      for (int half = NI / 2; half >= 1; half >>= 1) {
-        if (half < r) {
-#pragma unroll
-          for (int i = 0; i < NI; ++i)
-            if (i + half < NI && (i % r) < half) v[i] = __fadd_rn(v[i], v[i + half]);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < NI; ++i) {
-        if (i % r == 0) {
-#pragma unroll
-          for (int off = 16; off >= 1; off >>= 1) v[i] = __fadd_rn(v[i], __shfl_xor_sync(kFull, v[i], off));
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < NI; ++i) gsum[i] = v[(i / r) * r];
-    } else {
-      // gs consecutive lanes form a group: butterfly inside the group
-#pragma unroll
-      for (int i = 0; i < NI; ++i) {
-        float v = key[i];
-        for (int off = gs >> 1; off >= 1; off >>= 1) v = __fadd_rn(v, __shfl_xor_sync(kFull, v, off));
-        gsum[i] = v;
-      }
-    }
-    bool gchosen[NI];
-#pragma unroll
-    for (int i = 0; i < NI; ++i) {
-      if (isnan(gsum[i])) gsum[i] = kNegInf;
-      gchosen[i] = false;
-    }
-    for (int rnd = 0; rnd < p.topk_groups; ++rnd) {
-      float bv = kNegInf;
-      int bg = 0x7fffffff;
-#pragma unroll
-      for (int i = 0; i < NI; ++i) {
-        const int gid = (32 * i + lane) / gs;
-        if (valid[i] && !gchosen[i] && (gsum[i] > bv || (gsum[i] == bv && gid < bg))) {
-          bv = gsum[i];
-          bg = gid;
-        }
-      }
-      warp_argmax(bv, bg);
-#pragma unroll
-      for (int i = 0; i < NI; ++i)
-        if ((32 * i + lane) / gs == bg) gchosen[i] = true;
-    }
-#pragma unroll
-    for (int i = 0; i < NI; ++i) cand[i] = cand[i] && gchosen[i];
-  }
-  if (p.cand_key != nullptr) {
-#pragma unroll
-    for (int i = 0; i < NI; ++i) {
-      const int e = 32 * i + lane;
-      if (valid[i]) {
-        p.cand_key[static_cast<int64_t>(t) * E + e] = cand[i] ? key[i] : kNegInf;
-        p.score_out[static_cast<int64_t>(t) * E + e] = score[i];
-      }
-    }
-  }
-
-  int my_e = 0;
-  float my_score = 0.0f;
-  for (int k = 0; k < p.K; ++k) {
-    float bv = kNegInf;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < NI; ++i) {
-      const int e = 32 * i + lane;
-      if (cand[i] && !taken[i] && (key[i] > bv || (key[i] == bv && e < be))) {
-        bv = key[i];
-        be = e;
-      }
-    }
-    warp_argmax(bv, be);
-    float sc = 0.0f;
-#pragma unroll
-    for (int i = 0; i < NI; ++i) {
-      if (32 * i + lane == be) {
-        taken[i] = true;
-        sc = score[i];
-      }
-    }
-    sc = __shfl_sync(kFull, sc, be & 31);
-    if (lane == k) {
-      my_e = be;
-      my_score = sc;
-    }
-  }
-
-  const bool mine = lane < p.K;
-  const float g = gate_of<NI>(score, valid, my_score, mine, p.score_fn, p.renormalize);
-  if (mine) {
-    p.topk_idx[static_cast<int64_t>(t) * p.K + lane] = my_e;
-    p.topk_w[static_cast<int64_t>(t) * p.K + lane] = g;
-  }
-}
+using namespace route_detail;
 
 constexpr int kRouteWarps = 8;
 
-// E <= EMAX <= 32: the warp computes the token's logits itself.  Lanes stride
-// over 16-byte vectors of x and W_r rows (fp32 partial sums), then a butterfly
-// reduction per expert.
+// E <= EMAX <= 32, large batches: each warp routes TPW = 32 / EMAX tokens at
+// once, so every router-weight vector it loads (through L1) serves TPW
+// tokens, and the token rows -- the only bytes that must come from HBM --
+// stream at full width (lanes stride over 16-byte vectors of the rows).  The
+// TPW x EMAX = 32 partial dot products per lane are summed over the warp by a
+// reduce-scatter butterfly (31 shuffles: at each step a lane keeps half of
+// its values and receives the partner's partial sums of that half), after
+// which lane i holds logit (token i / EMAX, expert i % EMAX); one shuffle per
+// token hands lane e its expert-e logit for the selection.
+constexpr int kRouteWarpsP = 4;
+
 template <typename T, int EMAX>
-__global__ void __launch_bounds__(kRouteWarps * 32)
+__global__ void __launch_bounds__(kRouteWarpsP * 32)
     route_fused_kernel(int S, int d, const T* __restrict__ x, const T* __restrict__ w_router,
                        const float* __restrict__ router_bias, SelectParams p) {
-  const int t = blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
-  if (t >= S) return;
+  constexpr int TPW = 32 / EMAX;
+  const int t0 = (blockIdx.x * kRouteWarpsP + (threadIdx.x >> 5)) * TPW;
+  if (t0 >= S) return;
   const int lane = lane_id();
   constexpr int V = Vec16<T>::N;
   const int nvec = d / V;
-  float acc[EMAX];
+  float acc[TPW * EMAX];
 #pragma unroll
-  for (int e = 0; e < EMAX; ++e) acc[e] = 0.0f;
-  const T* xr = x + static_cast<int64_t>(t) * d;
+  for (int i = 0; i < TPW * EMAX; ++i) acc[i] = 0.0f;
+  const T* xr[TPW];
+#pragma unroll
+  for (int tt = 0; tt < TPW; ++tt) xr[tt] = x + static_cast<int64_t>(min(t0 + tt, S - 1)) * d;
+#pragma unroll 2
   for (int v = lane; v < nvec; v += 32) {
-    float xf[V];
-    unpack16<T>(ldg16(xr + v * V), xf);
+    float xf[TPW][V];
+#pragma unroll
+    for (int tt = 0; tt < TPW; ++tt) unpack16<T>(ldg16(xr[tt] + v * V), xf[tt]);
 #pragma unroll
     for (int e = 0; e < EMAX; ++e) {
       if (e < p.E) {
         float wf[V];
         unpack16<T>(ldg16(w_router + static_cast<int64_t>(e) * d + v * V), wf);
 #pragma unroll
-        for (int j = 0; j < V; ++j) acc[e] = fmaf(xf[j], wf[j], acc[e]);
+        for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+          for (int j = 0; j < V; ++j) acc[tt * EMAX + e] = fmaf(xf[tt][j], wf[j], acc[tt * EMAX + e]);
       }
     }
   }
-  float l[1] = {0.0f};
+  // reduce-scatter over the warp: afterwards acc[0] of lane i is the sum of value i
 #pragma unroll
-  for (int e = 0; e < EMAX; ++e) {
-    const float s = warp_sum(acc[e]);
-    if (e == lane) l[0] = s;
+  for (int s = 16; s >= 1; s >>= 1) {
+    const bool upper = (lane & s) != 0;
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      const float send = upper ? acc[i] : acc[i + s];
+      const float keep = upper ? acc[i + s] : acc[i];
+      acc[i] = keep + __shfl_xor_sync(kFull, send, s);
+    }
   }
-  if (lane < p.E && router_bias != nullptr) l[0] = __fadd_rn(l[0], __ldg(router_bias + lane));
-  select_topk<1>(l, p, t);
+  const float mine = acc[0];
+  const float bias = (lane < p.E && router_bias != nullptr) ? __ldg(router_bias + lane) : 0.0f;
+#pragma unroll
+  for (int tt = 0; tt < TPW; ++tt) {
+    if (t0 + tt >= S) break;  // warp-uniform
+    float l[1];
+    l[0] = __shfl_sync(kFull, mine, tt * EMAX + (lane % EMAX));
+    if (lane < p.E && router_bias != nullptr) l[0] = __fadd_rn(l[0], bias);
+    select_topk<1>(l, p, t0 + tt);
+  }
 }
 
 // Small batches (decode): one CTA per token, its 8 warps split d so the
@@ -456,22 +246,23 @@ cudaError_t launch_topk_ni(const RouteArgs& a, const float* logits, const Select
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
   if (a.S == 0) return cudaSuccess;
   SelectParams sp{a.E,        a.K,      a.score_fn, a.renormalize, a.num_groups,   a.topk_groups, a.tau,
-                  a.sel_bias, a.topk_idx, a.topk_w, a.status,      a.cand_key_out, a.score_out};
+                  a.sel_bias, a.topk_idx, a.topk_w, a.status,      a.cand_key_out, a.score_out, nullptr};
   const int blocks = (a.S + kRouteWarps - 1) / kRouteWarps;
   const float* logits = a.logits;
   if (logits == nullptr && a.E <= 32) {
     // decode-sized batches: a CTA per token; otherwise a warp per token
     const bool per_cta = a.S <= 512;
-    const int g = per_cta ? a.S : blocks;
     cudaError_t err = cudaSuccess;
 #define MOE_ROUTE_LAUNCH(T, EM)                                                                                \
   do {                                                                                                         \
-    if (per_cta)                                                                                               \
-      err = launch_pdl(route_token_cta_kernel<T, EM>, dim3(g), dim3(kRouteWarps * 32), 0, stream, a.d,              \
+    if (per_cta) {                                                                                             \
+      err = launch_pdl(route_token_cta_kernel<T, EM>, dim3(a.S), dim3(kRouteWarps * 32), 0, stream, a.d,       \
                        static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);      \
-    else                                                                                                       \
-      route_fused_kernel<T, EM><<<g, kRouteWarps * 32, 0, stream>>>(                                           \
+    } else {                                                                                                   \
+      const int per_cta_tokens = kRouteWarpsP * (32 / EM);                                                     \
+      route_fused_kernel<T, EM><<<(a.S + per_cta_tokens - 1) / per_cta_tokens, kRouteWarpsP * 32, 0, stream>>>( \
           a.S, a.d, static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);         \
+    }                                                                                                          \
   } while (0)
     if (a.act_dtype == MOE_BF16) {
       if (a.E <= 8)
