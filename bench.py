@@ -131,7 +131,10 @@ def kernels_per_step(cfg, S=None):
         n = 1 if (cfg.E <= 32) else 2      # route (fused) or logits GEMM + top-k
         n += 1 if small else 4             # permutation (+ group table): one kernel, or count, scan, scatter, groups
         n += 1                             # row gather (quantising for W8A8)
-    n += 2                                 # up and down GEMM (split-K partial sums reduced inside them)
+    n += 2                                 # up and down GEMM
+    rows = S * cfg.K + cfg.num_shared * S + (cfg.E * cfg.capacity if cfg.capacity else 0)
+    if cfg.act_dtype == syn.BF16 and rows <= 4096 and S > 16:
+        n += 2                             # split-K finalize of both GEMMs (S <= 16 reduce inside the GEMMs)
     if cfg.act_quant:
         n += 1                             # per-row E4M3 quantisation of the hidden rows
     elif cfg.weight_dtype == syn.E4M3:

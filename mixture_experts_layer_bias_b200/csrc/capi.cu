@@ -6,6 +6,7 @@
 // expert's FFN over its rows as one grouped GEMM, restore token order with
 // the gate-weighted sum.  Nothing here allocates or synchronises (except
 // moe_get_status); every launch goes to the caller's stream.
+#include <nvtx3/nvToolsExt.h>
 #include <string.h>
 
 #include "common.cuh"
@@ -15,13 +16,23 @@ using namespace moe;
 
 namespace {
 
+// NVTX range around each entry point and each stage of the layer call (host
+// timeline; a profiler can filter the kernels launched inside a range).  The
+// calls cost a few nanoseconds when no tool is attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 
 struct Layout {
   size_t status, counters, logits, chunk_hist, groups, counts, offsets, topk_idx, topk_w, row_of_slot,
-      token_of_row, x_perm, hidden, y_perm, wdeq, partial, partial_bytes, qa, sa, qas, sas, qh, sh, rr_key,
+      token_of_row, x_perm, hidden, y_perm, wdeq, ksplit, partial, partial_bytes, qa, sa, qas, sas, qh, sh, rr_key,
       rr_score, rr_ex, rr_changed, total;
 };
 
@@ -88,6 +99,7 @@ Layout make_layout(const moe_desc& d) {
   L.rr_score = take(rr ? static_cast<size_t>(S * E) * 4 : 0);
   L.rr_ex = take(rr ? static_cast<size_t>(S * K) * 4 : 0);
   L.rr_changed = take(rr ? static_cast<size_t>(S) * 4 : 0);
+  L.ksplit = take(kAlign);
   L.partial_bytes = 0;
   if (d.act_dtype == MOE_BF16 && Rt > 0 && Rt <= kSplitRowsMax) {
     const int64_t up_cols = d.activation == MOE_ACT_SWIGLU ? 2 * h : h;
@@ -287,6 +299,7 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
   up.status = status;
   up.partial = L.partial_bytes ? at<float>(ws, L.partial) : nullptr;
   up.partial_bytes = static_cast<int64_t>(L.partial_bytes);
+  up.ksplit_out = at<int>(ws, L.ksplit);
   up.tile_count = at<int>(ws, L.counters);
   up.tile_count_len = static_cast<int64_t>(kCounterInts);
 
@@ -526,6 +539,7 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
 
 moe_status moe_route(const moe_desc* desc, const moe_weights* w, const void* x, const float* logits_in,
                      int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx("moe_route");
   moe_status s = validate(desc);
   if (s != MOE_OK) return s;
   if ((s = check_ws(*desc, ws, ws_bytes)) != MOE_OK) return s;
@@ -541,6 +555,7 @@ moe_status moe_route(const moe_desc* desc, const moe_weights* w, const void* x, 
 moe_status moe_permute(const moe_desc* desc, const void* x, const int32_t* topk_idx, int32_t* counts,
                        int32_t* offsets, int32_t* row_of_slot, int32_t* token_of_row, void* x_perm, void* ws,
                        size_t ws_bytes, void* stream) {
+  NvtxRange nvtx("moe_permute");
   moe_status s = validate(desc);
   if (s != MOE_OK) return s;
   if ((s = check_ws(*desc, ws, ws_bytes)) != MOE_OK) return s;
@@ -555,6 +570,7 @@ moe_status moe_permute(const moe_desc* desc, const void* x, const int32_t* topk_
 
 moe_status moe_grouped_ffn(const moe_desc* desc, const moe_weights* w, const void* x_perm, const int32_t* offsets,
                            const void* x, void* y_perm, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx("moe_grouped_ffn");
   moe_status s = validate(desc);
   if (s != MOE_OK) return s;
   if ((s = check_ws(*desc, ws, ws_bytes)) != MOE_OK) return s;
@@ -568,6 +584,7 @@ moe_status moe_grouped_ffn(const moe_desc* desc, const moe_weights* w, const voi
 
 moe_status moe_reroute(const moe_desc* desc, int32_t* topk_idx, float* topk_w, const int32_t* counts,
                        const int32_t* row_of_slot, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx("moe_reroute");
   moe_status s = validate(desc);
   if (s != MOE_OK) return s;
   if (desc->reroute != 1) return MOE_ERR_INVALID_ARG;
@@ -579,6 +596,7 @@ moe_status moe_reroute(const moe_desc* desc, int32_t* topk_idx, float* topk_w, c
 }
 
 moe_status moe_quantize_rows_e4m3(const void* x, int64_t rows, int32_t d, uint8_t* q, float* s, void* stream) {
+  NvtxRange nvtx("moe_quantize_rows_e4m3");
   if (rows < 0 || d <= 0 || d % 16 != 0) return MOE_ERR_INVALID_ARG;
   if (rows == 0) return MOE_OK;
   if (x == nullptr || q == nullptr || s == nullptr || !aligned16(x) || !aligned16(q)) return MOE_ERR_INVALID_ARG;
@@ -588,6 +606,7 @@ moe_status moe_quantize_rows_e4m3(const void* x, int64_t rows, int32_t d, uint8_
 
 moe_status moe_combine(const moe_desc* desc, const void* y_perm, const int32_t* row_of_slot, const float* topk_w,
                        void* y, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx("moe_combine");
   moe_status s = validate(desc);
   if (s != MOE_OK) return s;
   if ((s = check_ws(*desc, ws, ws_bytes)) != MOE_OK) return s;
@@ -599,16 +618,19 @@ moe_status moe_combine(const moe_desc* desc, const void* y_perm, const int32_t* 
 
 moe_status moe_layer_forward(const moe_desc* desc, const moe_weights* w, const void* x, void* y, int32_t* topk_idx,
                              float* topk_w, int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx("moe_layer_forward");
   return layer_impl(desc, w, x, y, topk_idx, topk_w, counts, ws, ws_bytes, stream, nullptr);
 }
 
 moe_status moe_layer_forward_timed(const moe_desc* desc, const moe_weights* w, const void* x, void* y,
                                    int32_t* topk_idx, float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
                                    void* stream, void* const* events) {
+  NvtxRange nvtx("moe_layer_forward_timed");
   return layer_impl(desc, w, x, y, topk_idx, topk_w, counts, ws, ws_bytes, stream, events);
 }
 
 moe_status moe_load_stats(const moe_desc* desc, const int32_t* counts, double* stats, void* stream) {
+  NvtxRange nvtx("moe_load_stats");
   const moe_status s = validate(desc);
   if (s != MOE_OK) return s;
   if (counts == nullptr || stats == nullptr || (reinterpret_cast<uintptr_t>(counts) & 3) != 0 ||
@@ -637,6 +659,7 @@ moe_status moe_bias_state_init(void* state, size_t state_bytes, void* stream) {
 moe_status moe_update_sel_bias(const moe_desc* desc, const int32_t* topk_idx, int32_t window_tokens, float gamma,
                                void* state, size_t state_bytes, float* sel_bias, int32_t* window_counts,
                                void* stream) {
+  NvtxRange nvtx("moe_update_sel_bias");
   size_t need = 0;
   moe_status s = moe_bias_state_size(desc, window_tokens, &need);
   if (s != MOE_OK) return s;

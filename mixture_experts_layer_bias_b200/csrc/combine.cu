@@ -5,9 +5,9 @@
 // original token order); plumephp.com "MoE 混合专家推理", worked example:
 // output = 0.55 * e0(x) + 0.30 * e3(x), normalised.
 //
-// One warp per token (one CTA per token for S <= 256); lanes stride over
-// 16-byte vectors of the d_model row; fp32 sums in k order, then the shared
-// expert's row (gate 1), one rounding to the output type at the end.
+// One CTA per token; threads stride over 16-byte vectors of the d_model row;
+// fp32 sums in k order, then the shared expert's row (gate 1), one rounding to
+// the output type at the end.
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -18,52 +18,9 @@ namespace moe {
 
 namespace {
 
-constexpr int kCombWarps = 8;
-
-template <typename T>
-__global__ void __launch_bounds__(kCombWarps * 32)
-    combine_kernel(int S, int d, int K, const T* __restrict__ y_perm, const int32_t* __restrict__ row_of_slot,
-                   const float* __restrict__ topk_w, int64_t shared_row0, T* __restrict__ y) {
-  const int t = blockIdx.x * kCombWarps + (threadIdx.x >> 5);
-  if (t >= S) return;
-  const int lane = lane_id();
-  constexpr int V = Vec16<T>::N;
-  const int nvec = d / V;
-  // row indices and gates of this token, one per lane (K <= 32)
-  int my_row = -1;
-  float my_g = 0.0f;
-  if (lane < K) {
-    my_row = __ldg(row_of_slot + static_cast<int64_t>(t) * K + lane);
-    my_g = __ldg(topk_w + static_cast<int64_t>(t) * K + lane);
-  }
-  // warp-uniform loop: every lane takes part in the shuffles below
-  for (int base = 0; base < nvec; base += 32) {
-    const int v = base + lane;
-    const bool act = v < nvec;
-    float acc[V];
-#pragma unroll
-    for (int j = 0; j < V; ++j) acc[j] = 0.0f;
-    for (int k = 0; k < K; ++k) {
-      const int row = __shfl_sync(0xFFFFFFFFu, my_row, k);
-      const float g = __shfl_sync(0xFFFFFFFFu, my_g, k);
-      if (row < 0 || !act) continue;
-      float f[V];
-      unpack16<T>(ldg16(y_perm + static_cast<int64_t>(row) * d + v * V), f);
-#pragma unroll
-      for (int j = 0; j < V; ++j) acc[j] = fmaf(g, f[j], acc[j]);
-    }
-    if (!act) continue;
-    if (shared_row0 >= 0) {
-      float f[V];
-      unpack16<T>(ldg16(y_perm + (shared_row0 + t) * d + v * V), f);
-#pragma unroll
-      for (int j = 0; j < V; ++j) acc[j] += f[j];
-    }
-    stg16(y + static_cast<int64_t>(t) * d + v * V, pack16<T>(acc));
-  }
-}
-
-// Small batches: one CTA per token, its threads split the row.
+// One CTA per token, its threads splitting the row (16-byte vectors): each
+// thread issues the loads of all K rows of its vectors before the sums, so an
+// SM keeps many rows in flight.  Launched under programmatic dependent launch.
 template <typename T>
 __global__ void __launch_bounds__(256)
     combine_cta_kernel(int d, int K, const T* __restrict__ y_perm, const int32_t* __restrict__ row_of_slot,
@@ -80,6 +37,7 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   constexpr int V = Vec16<T>::N;
   const int nvec = d / V;
+#pragma unroll 2
   for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
     float acc[V];
 #pragma unroll
@@ -129,28 +87,19 @@ __global__ void dequant_e4m3_kernel(const uint4* __restrict__ q, uint4* __restri
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream) {
   if (a.S == 0) return cudaSuccess;
-  if (a.S <= 256) {
-    cudaError_t err;
-    if (a.act_dtype == MOE_BF16)
-      err = launch_pdl(combine_cta_kernel<__nv_bfloat16>, dim3(a.S), dim3(256), 0, stream, a.d, a.K,
-                       static_cast<const __nv_bfloat16*>(a.y_perm), a.row_of_slot, a.topk_w, a.shared_row0,
-                       static_cast<__nv_bfloat16*>(a.y));
-    else
-      err = launch_pdl(combine_cta_kernel<float>, dim3(a.S), dim3(256), 0, stream, a.d, a.K,
-                       static_cast<const float*>(a.y_perm), a.row_of_slot, a.topk_w, a.shared_row0,
-                       static_cast<float*>(a.y));
-    if (err != cudaSuccess) return err;
-    return cudaGetLastError();
-  }
-  const int blocks = (a.S + kCombWarps - 1) / kCombWarps;
+  // threads per token: enough 16-byte vectors for each (d / 8 or d / 4 of them), at most 256
+  const int nvec = a.act_dtype == MOE_BF16 ? a.d / 8 : a.d / 4;
+  const int threads = nvec >= 256 ? 256 : (nvec >= 128 ? 128 : 64);
+  cudaError_t err;
   if (a.act_dtype == MOE_BF16)
-    combine_kernel<__nv_bfloat16><<<blocks, kCombWarps * 32, 0, stream>>>(
-        a.S, a.d, a.K, static_cast<const __nv_bfloat16*>(a.y_perm), a.row_of_slot, a.topk_w, a.shared_row0,
-        static_cast<__nv_bfloat16*>(a.y));
+    err = launch_pdl(combine_cta_kernel<__nv_bfloat16>, dim3(a.S), dim3(threads), 0, stream, a.d, a.K,
+                     static_cast<const __nv_bfloat16*>(a.y_perm), a.row_of_slot, a.topk_w, a.shared_row0,
+                     static_cast<__nv_bfloat16*>(a.y));
   else
-    combine_kernel<float><<<blocks, kCombWarps * 32, 0, stream>>>(a.S, a.d, a.K, static_cast<const float*>(a.y_perm),
-                                                                   a.row_of_slot, a.topk_w, a.shared_row0,
-                                                                   static_cast<float*>(a.y));
+    err = launch_pdl(combine_cta_kernel<float>, dim3(a.S), dim3(threads), 0, stream, a.d, a.K,
+                     static_cast<const float*>(a.y_perm), a.row_of_slot, a.topk_w, a.shared_row0,
+                     static_cast<float*>(a.y));
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 

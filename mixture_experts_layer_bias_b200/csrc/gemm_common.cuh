@@ -33,8 +33,10 @@ struct TcParams {
   int max_ksplit;      // 1 = no split-K
   float* partial;      // fp32 [max_ksplit][out_rows][pcols] (split-K partial sums)
   int pcols;           // 2N (SwiGLU: gate then up) or N
+  int* ksplit_out;     // the split chosen on the device (read by the finalize kernel)
+  int inkernel_reduce; // 1: split-K slices are reduced inside the GEMM (tiny groups), 0: by the finalize kernel
   int* tile_count;     // split-K arrival counters, kRegionsPerTile per tile, zero between launches
-  int max_tiles;       // tiles the counters cover (more tiles: no split-K)
+  int max_tiles;       // tiles the counters cover (more tiles: no in-kernel reduction, no split-K)
   int test_stall;      // test hook: the producer delivers nothing (the bounded waits must give up)
   int tma_out;         // 1: the output tensor map is valid (full 32-row quarters use bulk tensor stores)
   const float* row_scale;         // E4M3 activations: per-row scale of the A operand rows (nullptr: none)
@@ -84,17 +86,61 @@ __device__ __forceinline__ bool group_ok(const GroupEntry& g, const TcParams& p)
 // Split-K: every epilogue warp of a CTA owns one region of its tile (32 rows
 // of one TMEM lane quarter x half of the tile's columns) and, per split, writes
 // its raw fp32 accumulators there to the split's slice of the partial buffer.
-// One arrival counter per (tile, region) counts the slices written; the warp
-// whose slice completes the count sums the region's slices in split order
-// (deterministic whatever the arrival order), applies the epilogue and stores
-// the output rows, then resets the counter for the next launch.
+// The slices are then summed in split order (deterministic whatever the
+// arrival order), the epilogue applied and the output stored, in one of two
+// ways chosen on the host:
+//  - tiny groups (decode, at most 16 rows per group): inside the GEMM.  One
+//    arrival counter per (tile, region) counts the slices written; the warp
+//    whose slice completes the count reduces the region (a few rows, so the
+//    one warp's loads are few and all in flight together) and resets the
+//    counter for the next launch.  No extra launch.
+//  - larger groups: splitk_finalize_kernel after the GEMM, one thread per
+//    four output columns of a row, so many rows are reduced in parallel.
 constexpr int kRegionsPerTile = 8;
 
-// The last arriver's reduction of region (q, half) of tile `ti`: rows
-// m_idx*128 + q*32 .. +31 of the group, lane j taking output columns
-// n0 + 2j, n0 + 2j + 1 (SwiGLU, 64 columns per half: gate at n, up at N + n
-// in the slices) or n0 + 4j .. n0 + 4j + 3 (128 columns per half).  Partial
-// sums are read at L2 (ld.global.cg): other CTAs wrote them in this launch.
+// Epilogue of split-K sums: gate/up sums g, u (SwiGLU) or sums v, with the
+// row scale rs, channel scales and bias of column n + j.
+template <int EPI>
+__device__ __forceinline__ float splitk_out(const TcParams& p, int64_t sbase, int n, int j, float g, float u,
+                                            float rs) {
+  float gv = g * rs;
+  if (p.scale0 != nullptr) gv *= p.scale0[sbase + n + j];
+  if (EPI == EPI_SWIGLU) {
+    float uv = u * rs;
+    if (p.scale1 != nullptr) uv *= p.scale1[sbase + n + j];
+    return gv / (1.0f + __expf(-gv)) * uv;
+  }
+  if (EPI == EPI_GELU_BIAS || EPI == EPI_BIAS) gv += p.bias[sbase + n + j];
+  if (EPI == EPI_GELU_BIAS) gv = 0.5f * gv * (1.0f + erff(gv * 0.70710678118654752f));
+  return gv;
+}
+
+// Sum of the ks slices of the float4 at `src` (slice stride `slice`), in split
+// order; the loads are issued four at a time before their sums so that they
+// are in flight together.  Read at L2 (ld.global.cg): other CTAs wrote them.
+__device__ __forceinline__ float4 splitk_sum4(const float* src, int64_t slice, int ks) {
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  int s = 0;
+  for (; s + 4 <= ks; s += 4) {
+    float4 a[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = __ldcg(reinterpret_cast<const float4*>(src + (s + i) * slice));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc.x += a[i].x; acc.y += a[i].y; acc.z += a[i].z; acc.w += a[i].w;
+    }
+  }
+  for (; s < ks; ++s) {
+    const float4 a = __ldcg(reinterpret_cast<const float4*>(src + s * slice));
+    acc.x += a.x; acc.y += a.y; acc.z += a.z; acc.w += a.w;
+  }
+  return acc;
+}
+
+// The last arriver's reduction of region (q, half) of a tile: rows
+// m_row0 .. m_row0 + 31 of the group, the half's output columns split over the
+// lanes in float4 pieces (SwiGLU: 64 columns, lanes 0-15 one row's 16 pieces
+// and lanes 16-31 the next row's; otherwise 128 columns, one row at a time).
 template <int EPI>
 __device__ __forceinline__ void splitk_reduce_region(const TcParams& p, const GroupEntry& grp, int m_row0, int n_tile,
                                                      int ks, int half, int lane) {
@@ -102,69 +148,70 @@ __device__ __forceinline__ void splitk_reduce_region(const TcParams& p, const Gr
   const int64_t slice = p.out_rows * static_cast<int64_t>(p.pcols);
   const int64_t sbase = static_cast<int64_t>(grp.expert) * N;
   const int r1 = min(m_row0 + 32, grp.rows);
-  if (EPI == EPI_SWIGLU) {
-    const int n = n_tile * p.bn_out + half * 64 + 2 * lane;
-    if (n >= N) return;  // N is a multiple of 8, so n + 1 < N as well
-    float c0[2] = {1.0f, 1.0f}, c1[2] = {1.0f, 1.0f};
-    if (p.scale0 != nullptr) { c0[0] = p.scale0[sbase + n]; c0[1] = p.scale0[sbase + n + 1]; }
-    if (p.scale1 != nullptr) { c1[0] = p.scale1[sbase + n]; c1[1] = p.scale1[sbase + n + 1]; }
-    for (int r = m_row0; r < r1; ++r) {
-      const int64_t orow = static_cast<int64_t>(grp.out_row0) + r;
-      const float rs = a_row_scale(p, grp, r);
-      float g[2] = {0.f, 0.f}, u[2] = {0.f, 0.f};
-      for (int s = 0; s < ks; ++s) {
-        const float* src = p.partial + s * slice + orow * p.pcols;
-        const float2 a = __ldcg(reinterpret_cast<const float2*>(src + n));
-        const float2 b = __ldcg(reinterpret_cast<const float2*>(src + N + n));
-        g[0] += a.x; g[1] += a.y; u[0] += b.x; u[1] += b.y;
-      }
-      float o[2];
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        float gv = g[j] * rs;
-        if (p.scale0 != nullptr) gv *= c0[j];
-        float uv = u[j] * rs;
-        if (p.scale1 != nullptr) uv *= c1[j];
-        o[j] = gv / (1.0f + __expf(-gv)) * uv;
-      }
-      if (p.out_f32)
-        *reinterpret_cast<float2*>(static_cast<float*>(p.out) + orow * N + n) = make_float2(o[0], o[1]);
-      else
-        *reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(p.out) + orow * N + n) = pack_bf16x2(o[0], o[1]);
-    }
-    return;
-  }
-  const int n = n_tile * p.bn_out + half * 128 + 4 * lane;
+  constexpr int kRowsPerStep = (EPI == EPI_SWIGLU) ? 2 : 1;
+  constexpr int kHalfCols = (EPI == EPI_SWIGLU) ? 64 : 128;
+  const int piece = (EPI == EPI_SWIGLU) ? (lane & 15) : lane;
+  const int n = n_tile * p.bn_out + half * kHalfCols + 4 * piece;
   if (n >= N) return;  // n is a multiple of 4 and N of 8: n + 3 < N
-  float cs[4] = {1.f, 1.f, 1.f, 1.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    if (p.scale0 != nullptr) cs[j] = p.scale0[sbase + n + j];
-    if (EPI == EPI_GELU_BIAS || EPI == EPI_BIAS) cb[j] = p.bias[sbase + n + j];
-  }
-  for (int r = m_row0; r < r1; ++r) {
+  for (int r0 = m_row0; r0 < r1; r0 += kRowsPerStep) {
+    const int r = r0 + ((EPI == EPI_SWIGLU) ? (lane >> 4) : 0);
+    if (r >= r1) continue;
     const int64_t orow = static_cast<int64_t>(grp.out_row0) + r;
     const float rs = a_row_scale(p, grp, r);
-    float v[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int s = 0; s < ks; ++s) {
-      const float4 a = __ldcg(reinterpret_cast<const float4*>(p.partial + s * slice + orow * p.pcols + n));
-      v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
-    }
+    const float* src = p.partial + orow * p.pcols + n;
+    const float4 g = splitk_sum4(src, slice, ks);
+    float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (EPI == EPI_SWIGLU) u = splitk_sum4(src + N, slice, ks);
     float o[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float z = v[j] * rs;
-      if (p.scale0 != nullptr) z *= cs[j];
-      if (EPI == EPI_GELU_BIAS || EPI == EPI_BIAS) z += cb[j];
-      if (EPI == EPI_GELU_BIAS) z = 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
-      o[j] = z;
-    }
+    o[0] = splitk_out<EPI>(p, sbase, n, 0, g.x, u.x, rs);
+    o[1] = splitk_out<EPI>(p, sbase, n, 1, g.y, u.y, rs);
+    o[2] = splitk_out<EPI>(p, sbase, n, 2, g.z, u.z, rs);
+    o[3] = splitk_out<EPI>(p, sbase, n, 3, g.w, u.w, rs);
     if (p.out_f32) {
       *reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * N + n) = make_float4(o[0], o[1], o[2], o[3]);
     } else {
       const uint2 packed = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
       *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + orow * N + n) = packed;
     }
+  }
+}
+
+// Split-K finalize for larger groups: for every valid row of every group, sum
+// the partial slices in split order and apply the epilogue; one thread per
+// four output columns.  Exits at once when the GEMM ran without a split or
+// reduced its slices itself.  Launched under programmatic dependent launch:
+// it waits for the GEMM before reading.
+template <int EPI>
+__global__ void __launch_bounds__(256) splitk_finalize_kernel(TcParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int ks = *p.ksplit_out;
+  if (ks <= 1 || p.inkernel_reduce) return;
+  const GroupEntry grp = group_at(p, blockIdx.z);
+  const int r = blockIdx.y;
+  if (r >= grp.rows || grp.expert < 0 || grp.expert >= p.num_slabs) return;
+  const int n = (blockIdx.x * 256 + threadIdx.x) * 4;
+  const int N = p.N;
+  if (n >= N) return;
+  const int64_t orow = static_cast<int64_t>(grp.out_row0) + r;
+  if (orow >= p.out_rows) return;
+  const int64_t sbase = static_cast<int64_t>(grp.expert) * N;
+  const int64_t slice = p.out_rows * static_cast<int64_t>(p.pcols);
+  const float rs = a_row_scale(p, grp, r);
+  const float* src = p.partial + orow * p.pcols + n;
+  const float4 g = splitk_sum4(src, slice, ks);
+  float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (EPI == EPI_SWIGLU) u = splitk_sum4(src + N, slice, ks);
+  float o[4];
+  o[0] = splitk_out<EPI>(p, sbase, n, 0, g.x, u.x, rs);
+  o[1] = splitk_out<EPI>(p, sbase, n, 1, g.y, u.y, rs);
+  o[2] = splitk_out<EPI>(p, sbase, n, 2, g.z, u.z, rs);
+  o[3] = splitk_out<EPI>(p, sbase, n, 3, g.w, u.w, rs);
+  if (p.out_f32) {
+    *reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * N + n) = make_float4(o[0], o[1], o[2], o[3]);
+  } else {
+    const uint2 packed = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + orow * N + n) = packed;
   }
 }
 

@@ -328,8 +328,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s.tmem_base;
   const int nk = (p.K + BK - 1) / BK;
   const int tiles = s.tile_start[p.num_groups];
-  // split-K only while every tile has its arrival counters
-  const int ks = tiles <= p.max_tiles ? choose_ksplit(tiles, gridDim.x, nk, p.max_ksplit) : 1;
+  // in-kernel split-K reduction only while every tile has its arrival counters
+  const int ks = (!p.inkernel_reduce || tiles <= p.max_tiles) ? choose_ksplit(tiles, gridDim.x, nk, p.max_ksplit) : 1;
+  if (blockIdx.x == 0 && threadIdx.x == 0 && p.ksplit_out != nullptr) *p.ksplit_out = ks;
   const int total = tiles * ks;  // work units
   volatile int* abort_flag = &s.abort;
 
@@ -456,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         epilogue_store<EPI>(p, ti, tbase, row, valid, lane, half, &tmOut, epi_smem + (warp - 2) * kEpiWarpBytes);
       tc_fence_before();
       mbar_arrive(&s.tempty[acc]);
-      if (ks > 1) {
+      if (ks > 1 && p.inkernel_reduce) {
         // publish this slice of the warp's region, count it; the warp that
         // completes the count reduces the region's slices
         __threadfence();
@@ -488,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int EPI, bool F8>
 cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB0, const CUtensorMap& mB1,
                        const CUtensorMap& mOut, const TcParams& p, int grid, int bma, int stages, size_t smem,
-                       cudaStream_t stream) {
+                       int64_t max_group_rows, cudaStream_t stream) {
   static uint64_t attr_set = 0;  // one bit per device ordinal
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -502,6 +503,10 @@ cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUte
   // programmatic dependent launch: the prologue may overlap the previous kernel
   e = launch_pdl(grouped_gemm_tc_kernel<EPI, F8>, dim3(grid), dim3(kThreads), smem, stream, mA, mA2, mB0, mB1, mOut,
                  p, bma, stages);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaGetLastError()) != cudaSuccess || p.max_ksplit <= 1 || p.inkernel_reduce) return e;
+  dim3 fgrid((p.N + 1023) / 1024, static_cast<unsigned>(max_group_rows), p.num_groups);
+  e = launch_pdl(splitk_finalize_kernel<EPI>, fgrid, dim3(256), 0, stream, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -541,21 +546,21 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
   if (a.fp8) {  // W8A8 runs SwiGLU experts only
     switch (a.epilogue) {
       case EPI_SWIGLU:
-        return launch_epi<EPI_SWIGLU, true>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, stream);
+        return launch_epi<EPI_SWIGLU, true>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
       case EPI_NONE:
-        return launch_epi<EPI_NONE, true>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, stream);
+        return launch_epi<EPI_NONE, true>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
       default: return cudaErrorInvalidValue;
     }
   }
   switch (a.epilogue) {
     case EPI_SWIGLU:
-      return launch_epi<EPI_SWIGLU, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, stream);
+      return launch_epi<EPI_SWIGLU, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
     case EPI_GELU_BIAS:
-      return launch_epi<EPI_GELU_BIAS, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, stream);
+      return launch_epi<EPI_GELU_BIAS, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
     case EPI_BIAS:
-      return launch_epi<EPI_BIAS, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, stream);
+      return launch_epi<EPI_BIAS, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
     case EPI_NONE:
-      return launch_epi<EPI_NONE, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, stream);
+      return launch_epi<EPI_NONE, false>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
     default: return cudaErrorInvalidValue;
   }
 }

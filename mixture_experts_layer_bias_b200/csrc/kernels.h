@@ -112,7 +112,8 @@ struct GemmArgs {
   int64_t max_group_rows;   // upper bound of the rows of one group
   float* partial;           // split-K partial sums (nullptr = no split-K)
   int64_t partial_bytes;    // size of `partial`
-  int* tile_count;          // split-K arrival counters (zero between launches; nullptr = no split-K)
+  int* ksplit_out;          // device int: the split the GEMM chose (read by the finalize kernel)
+  int* tile_count;          // split-K arrival counters (zero between launches; nullptr = none)
   int64_t tile_count_len;   // number of counters
   int fp8;                  // 1: A and B are E4M3 (kind::f8f6f4); A rows scaled by row_scale
   const float* row_scale;        // [a rows] per-row scale of A (fp8 only)

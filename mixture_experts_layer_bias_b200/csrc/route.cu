@@ -29,51 +29,60 @@ using namespace route_detail;
 
 constexpr int kRouteWarps = 8;
 
-// E <= EMAX <= 32, large batches: each warp routes TPW = 32 / EMAX tokens at
-// once, so every router-weight vector it loads (through L1) serves TPW
-// tokens, and the token rows -- the only bytes that must come from HBM --
-// stream at full width (lanes stride over 16-byte vectors of the rows).  The
-// TPW x EMAX = 32 partial dot products per lane are summed over the warp by a
-// reduce-scatter butterfly (31 shuffles: at each step a lane keeps half of
-// its values and receives the partner's partial sums of that half), after
-// which lane i holds logit (token i / EMAX, expert i % EMAX); one shuffle per
-// token hands lane e its expert-e logit for the selection.
-constexpr int kRouteWarpsP = 4;
+// E <= EMAX <= 32, large batches: a set of TPW = 32 / EMAX tokens is routed
+// by kRouteSplit warps, each taking one contiguous part of d for all TPW
+// tokens, so every router-weight vector a warp loads (through L1) serves TPW
+// tokens while the token rows -- the only bytes that must come from HBM --
+// stream with many warps in flight (lanes stride over 16-byte vectors).  In
+// each warp the TPW x EMAX = 32 partial dot products per lane are summed over
+// the warp by a reduce-scatter butterfly (31 shuffles: at each step a lane
+// keeps half of its values and receives the partner's partial sums of that
+// half), after which lane i holds value (token i / EMAX, expert i % EMAX); the
+// warps' values are added in warp order through shared memory, and the set's
+// first warp selects, one shuffle per token handing lane e its expert-e logit.
+constexpr int kRouteWarpsP = 8;
+constexpr int kRouteSplit = 4;  // warps sharing one token set (parts of d)
 
 template <typename T, int EMAX>
 __global__ void __launch_bounds__(kRouteWarpsP * 32)
     route_fused_kernel(int S, int d, const T* __restrict__ x, const T* __restrict__ w_router,
                        const float* __restrict__ router_bias, SelectParams p) {
   constexpr int TPW = 32 / EMAX;
-  const int t0 = (blockIdx.x * kRouteWarpsP + (threadIdx.x >> 5)) * TPW;
-  if (t0 >= S) return;
-  const int lane = lane_id();
+  constexpr int kSets = kRouteWarpsP / kRouteSplit;
+  __shared__ float red[kSets][kRouteSplit][32];
+  const int warp = threadIdx.x >> 5, lane = lane_id();
+  const int set = warp / kRouteSplit, part = warp % kRouteSplit;
+  const int t0 = (blockIdx.x * kSets + set) * TPW;
   constexpr int V = Vec16<T>::N;
   const int nvec = d / V;
+  const int per_part = (nvec + kRouteSplit - 1) / kRouteSplit;
+  const int v0 = part * per_part, v1 = min(nvec, v0 + per_part);
   float acc[TPW * EMAX];
 #pragma unroll
   for (int i = 0; i < TPW * EMAX; ++i) acc[i] = 0.0f;
-  const T* xr[TPW];
+  if (t0 < S) {
+    const T* xr[TPW];
 #pragma unroll
-  for (int tt = 0; tt < TPW; ++tt) xr[tt] = x + static_cast<int64_t>(min(t0 + tt, S - 1)) * d;
+    for (int tt = 0; tt < TPW; ++tt) xr[tt] = x + static_cast<int64_t>(min(t0 + tt, S - 1)) * d;
 #pragma unroll 2
-  for (int v = lane; v < nvec; v += 32) {
-    float xf[TPW][V];
+    for (int v = v0 + lane; v < v1; v += 32) {
+      float xf[TPW][V];
 #pragma unroll
-    for (int tt = 0; tt < TPW; ++tt) unpack16<T>(ldg16(xr[tt] + v * V), xf[tt]);
+      for (int tt = 0; tt < TPW; ++tt) unpack16<T>(ldg16(xr[tt] + v * V), xf[tt]);
 #pragma unroll
-    for (int e = 0; e < EMAX; ++e) {
-      if (e < p.E) {
-        float wf[V];
-        unpack16<T>(ldg16(w_router + static_cast<int64_t>(e) * d + v * V), wf);
+      for (int e = 0; e < EMAX; ++e) {
+        if (e < p.E) {
+          float wf[V];
+          unpack16<T>(ldg16(w_router + static_cast<int64_t>(e) * d + v * V), wf);
 #pragma unroll
-        for (int tt = 0; tt < TPW; ++tt)
+          for (int tt = 0; tt < TPW; ++tt)
 #pragma unroll
-          for (int j = 0; j < V; ++j) acc[tt * EMAX + e] = fmaf(xf[tt][j], wf[j], acc[tt * EMAX + e]);
+            for (int j = 0; j < V; ++j) acc[tt * EMAX + e] = fmaf(xf[tt][j], wf[j], acc[tt * EMAX + e]);
+        }
       }
     }
   }
-  // reduce-scatter over the warp: afterwards acc[0] of lane i is the sum of value i
+  // reduce-scatter over the warp: afterwards acc[0] of lane i is the warp's sum of value i
 #pragma unroll
   for (int s = 16; s >= 1; s >>= 1) {
     const bool upper = (lane & s) != 0;
@@ -84,7 +93,12 @@ __global__ void __launch_bounds__(kRouteWarpsP * 32)
       acc[i] = keep + __shfl_xor_sync(kFull, send, s);
     }
   }
-  const float mine = acc[0];
+  red[set][part][lane] = acc[0];
+  __syncthreads();
+  if (part != 0 || t0 >= S) return;
+  float mine = 0.0f;
+#pragma unroll
+  for (int q = 0; q < kRouteSplit; ++q) mine += red[set][q][lane];
   const float bias = (lane < p.E && router_bias != nullptr) ? __ldg(router_bias + lane) : 0.0f;
 #pragma unroll
   for (int tt = 0; tt < TPW; ++tt) {
@@ -259,7 +273,7 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
       err = launch_pdl(route_token_cta_kernel<T, EM>, dim3(a.S), dim3(kRouteWarps * 32), 0, stream, a.d,       \
                        static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);      \
     } else {                                                                                                   \
-      const int per_cta_tokens = kRouteWarpsP * (32 / EM);                                                     \
+      const int per_cta_tokens = (kRouteWarpsP / kRouteSplit) * (32 / EM);                                     \
       route_fused_kernel<T, EM><<<(a.S + per_cta_tokens - 1) / per_cta_tokens, kRouteWarpsP * 32, 0, stream>>>( \
           a.S, a.d, static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);         \
     }                                                                                                          \

@@ -40,7 +40,7 @@ def test_committed_traffic_record_is_current_or_absent():
     ("mixtral_prefill_w8a8", None, 1 + 4 + 1 + 2 + 1 + 1),  # + quantisation of the hidden rows
     ("fp8_skew_capacity_reroute", None, 2 + 4 + 1 + 2 + 3 + 5 + 1),  # + ranks (3), assignment, gates
     ("mixtral_decode", 1, 1 + 2 + 1),                       # fused route-permute-gather, GEMMs, combine
-    ("mixtral_decode", 32, 1 + 1 + 1 + 2 + 1),              # one-CTA permutation
+    ("mixtral_decode", 32, 1 + 1 + 1 + 2 + 2 + 1),          # one-CTA permutation, split-K finalizes
     ("tiny_f32", None, 1 + 1 + 1 + 2 + 1),                  # fp32: no split-K
 ])
 def test_kernels_per_layer_call(name, S, expected):
