@@ -137,8 +137,8 @@ def kernels_per_step(cfg, S=None):
         n += 2                             # split-K finalize of both GEMMs (S <= 16 reduce inside the GEMMs)
     if cfg.act_quant:
         n += 1                             # per-row E4M3 quantisation of the hidden rows
-    elif cfg.weight_dtype == syn.E4M3:
-        n += 3                             # E4M3 -> bf16 decode of the three stacks
+    elif cfg.weight_dtype == syn.E4M3 and (cfg.d % 16 or cfg.h % 16):
+        n += 3                             # E4M3 -> bf16 decode of the three stacks (else inside the GEMMs)
     if cfg.reroute:
         n += (1 if small else 3) + 2       # ranks, re-route assignment and gates
     n += 1                                 # combine

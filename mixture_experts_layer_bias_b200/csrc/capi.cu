@@ -56,6 +56,13 @@ int64_t routed_rows(const moe_desc& d) {
 
 size_t act_bytes(const moe_desc& d) { return d.act_dtype == MOE_F32 ? 4 : 2; }
 
+// E4M3 weights with bf16 activations: the GEMMs decode the weight tiles
+// themselves when every weight row is a whole number of 16-byte pieces.
+bool w8_in_gemm(const moe_desc& d) {
+  return d.weight_dtype == MOE_E4M3 && d.act_quant == 0 && d.act_dtype == MOE_BF16 && d.d_model % 16 == 0 &&
+         d.d_ff % 16 == 0;
+}
+
 Layout make_layout(const moe_desc& d) {
   Layout L;
   const int64_t S = d.num_tokens, E = d.num_experts, K = d.top_k, h = d.d_ff, dm = d.d_model;
@@ -84,7 +91,9 @@ Layout make_layout(const moe_desc& d) {
   L.hidden = take(static_cast<size_t>(Rt * h) * ab);
   L.y_perm = take(static_cast<size_t>(Rt * dm) * ab);
   const bool w8a8 = d.act_quant == 1;
-  L.wdeq = take(d.weight_dtype == MOE_E4M3 && !w8a8 ? static_cast<size_t>((E + d.num_shared) * 3 * h * dm) * 2 : 0);
+  L.wdeq = take(d.weight_dtype == MOE_E4M3 && !w8a8 && !w8_in_gemm(d)
+                    ? static_cast<size_t>((E + d.num_shared) * 3 * h * dm) * 2
+                    : 0);
   // W8A8: E4M3 codes and row scales of the up GEMM's A rows (permuted
   // tokens; the shared expert's tokens) and of the down GEMM's (hidden rows)
   L.qa = take(w8a8 ? static_cast<size_t>(R * dm) : 0);
@@ -339,9 +348,18 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
       down.a = at<void>(ws, L.qh);
       down.row_scale = at<float>(ws, L.sh);
       down.row_scale_shared = nullptr;
+    } else if (d.weight_dtype == MOE_E4M3 && w8_in_gemm(d)) {
+      // E4M3 weights, bf16 activations: the GEMMs decode each landed weight
+      // tile to bf16 themselves (exact); the per-channel scales are applied to
+      // the fp32 accumulators in the epilogues
+      up.w8 = down.w8 = 1;
+      up.scale0 = w.s_gate;
+      up.scale1 = w.s_up;
+      down.scale0 = w.s_down;
     } else if (d.weight_dtype == MOE_E4M3) {
-      // exact E4M3 -> bf16 decode of this call's weights; the per-channel
-      // scales are applied to the fp32 accumulators in the epilogues
+      // exact E4M3 -> bf16 decode of this call's weights into the workspace
+      // (d or h not a multiple of 16); the per-channel scales are applied to
+      // the fp32 accumulators in the epilogues
       const int64_t n_up = static_cast<int64_t>(slabs) * h * dm;
       char* base = at<char>(ws, L.wdeq);
       void* dg = base;

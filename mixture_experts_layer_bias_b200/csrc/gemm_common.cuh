@@ -264,5 +264,21 @@ inline bool make_map(CUtensorMap* m, const void* base, int64_t rows, int k, int 
 }
 
 
+// 2-D map over E4M3 weights [rows][k] for the W8 GEMM: box = 64 codes (the K
+// extent of one bf16 stage) x 128 rows, no swizzle (the converters read it
+// row by row and write the swizzled bf16 tile).
+inline bool make_map_w8(CUtensorMap* m, const void* base, int64_t rows, int k) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr || rows <= 0 || k <= 0) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || k % 16 != 0) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(k)};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace gemm
 }  // namespace moe

@@ -66,6 +66,12 @@ constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
 constexpr int kEpiWarps = 8;  // two per TMEM lane quarter, each draining half of a tile's columns
 constexpr int kThreads = 64 + 32 * kEpiWarps;
+// E4M3 weights with bf16 activations (W8): four more warps decode each landed
+// E4M3 weight tile into the bf16 B tile of its stage.
+constexpr int kConvWarps = 4;
+constexpr int kThreadsW8 = kThreads + 32 * kConvWarps;
+constexpr int kLandStages = 3;             // landing buffers of E4M3 weight tiles
+constexpr int LAND_BYTES = 256 * 64;       // 256 weight rows x 64 E4M3 codes (one bf16 K step)
 constexpr uint32_t kIdescBf16 = idesc_bf16_f32(128, 256);
 constexpr uint32_t kIdescE4m3 = idesc_e4m3_f32(128, 256);
 
@@ -78,6 +84,8 @@ constexpr int bk_elems() {
 struct SmemCtl {
   uint64_t full[MAX_STAGES];
   uint64_t empty[MAX_STAGES];
+  uint64_t lfull[kLandStages];  // W8: an E4M3 weight tile has landed
+  int conv_ok;                  // W8: the converters' shared go / give-up decision
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -253,8 +261,55 @@ __device__ __forceinline__ void epilogue_partial(const TcParams& p, const TileIn
   }
 }
 
-template <int EPI, bool F8>
-__global__ void __launch_bounds__(kThreads, 1)
+// Four E4M3 codes (bytes of w, lowest first) -> four bf16 values (lo: codes
+// 0, 1; hi: codes 2, 3), exactly: E4M3 -> f16 is exact (every E4M3 value,
+// subnormals included, is a normal f16 or zero) and so is f16 -> bf16 for
+// values with at most four significant bits in the E4M3 range.
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 c0, c1, a, b, c, d;\n\t.reg .b32 h0, h1;\n\t"
+      "mov.b32 {c0, c1}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h0, c0;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h1, c1;\n\t"
+      "mov.b32 {a, b}, h0;\n\t"
+      "cvt.rn.bf16.f16 a, a;\n\t"
+      "cvt.rn.bf16.f16 b, b;\n\t"
+      "mov.b32 %0, {a, b};\n\t"
+      "mov.b32 {c, d}, h1;\n\t"
+      "cvt.rn.bf16.f16 c, c;\n\t"
+      "cvt.rn.bf16.f16 d, d;\n\t"
+      "mov.b32 %1, {c, d};\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+
+// W8: the 128 converter threads decode one landed 256 x 64 E4M3 tile (rows of
+// 64 bytes) into the stage's 256 x 128-byte bf16 B tile in the 128-byte
+// swizzled layout the MMA reads (16-byte chunk j of row r at chunk
+// j ^ (r & 7)).  Thread ct takes the 16-code pieces ct + 128 i.
+__device__ __forceinline__ void convert_tile_w8(const uint8_t* land, uint8_t* b16, int ct) {
+#pragma unroll 2
+  for (int i = 0; i < 8; ++i) {
+    const int piece = ct + 128 * i;  // 1024 pieces of 16 codes
+    const int r = piece >> 2, q4 = piece & 3;
+    const uint4 v = *reinterpret_cast<const uint4*>(land + r * 64 + q4 * 16);
+    uint32_t o[8];
+    e4m3x4_to_bf16x4(v.x, o[0], o[1]);
+    e4m3x4_to_bf16x4(v.y, o[2], o[3]);
+    e4m3x4_to_bf16x4(v.z, o[4], o[5]);
+    e4m3x4_to_bf16x4(v.w, o[6], o[7]);
+    uint8_t* row = b16 + r * BK_BYTES;
+    const int sw = r & 7;
+    *reinterpret_cast<uint4*>(row + (((2 * q4) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(row + (((2 * q4 + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+template <int EPI, bool F8, bool W8>
+__global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                            const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
                            const __grid_constant__ CUtensorMap tmOut, TcParams p, int bma, int STAGES) {
@@ -263,9 +318,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int BK = bk_elems<F8>();
   const int A_TILE = bma * BK_BYTES;
   const int STAGE_BYTES = A_TILE + B_TILE;
-  SmemCtl& s = *reinterpret_cast<SmemCtl*>(ring + STAGES * STAGE_BYTES);
+  uint8_t* land = ring + STAGES * STAGE_BYTES;  // W8 landing buffers (1024-byte aligned)
+  uint8_t* ctl = land + (W8 ? kLandStages * LAND_BYTES : 0);
+  SmemCtl& s = *reinterpret_cast<SmemCtl*>(ctl);
   uint8_t* epi_smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(ring + STAGES * STAGE_BYTES + sizeof(SmemCtl)) + 127) & ~uintptr_t(127));
+      (reinterpret_cast<uintptr_t>(ctl + sizeof(SmemCtl)) + 127) & ~uintptr_t(127));
   const int warp = threadIdx.x >> 5, lane = lane_id();
 
   // Prologue that needs nothing from earlier kernels (barriers, TMEM, tensor
@@ -275,9 +332,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     if (lane == 0) {
       for (int i = 0; i < STAGES; ++i) {
-        mbar_init(&s.full[i], 1);
+        mbar_init(&s.full[i], W8 ? 2 : 1);  // W8: the A copy's arrival plus the converters'
         mbar_init(&s.empty[i], 1);
       }
+      if (W8)
+        for (int i = 0; i < kLandStages; ++i) mbar_init(&s.lfull[i], 1);
       for (int i = 0; i < 2; ++i) {
         mbar_init(&s.tfull[i], 1);
         mbar_init(&s.tempty[i], 32 * kEpiWarps);
@@ -351,13 +410,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&s.full[stage], STAGE_BYTES);
+          mbar_arrive_expect_tx(&s.full[stage], W8 ? A_TILE : STAGE_BYTES);
           armed |= 1u << stage;
           armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
           uint8_t* sa = ring + stage * STAGE_BYTES;
           uint8_t* sb = sa + A_TILE;
           tma_load_2d(sa, mA, kb * BK, a_row, &s.full[stage]);
-          if (EPI == EPI_SWIGLU) {
+          if (W8) {
+            // the converters fill this stage's B tile
+          } else if (EPI == EPI_SWIGLU) {
             tma_load_2d(sb, &tmB0, kb * BK, b_row, &s.full[stage]);
             tma_load_2d(sb + B_HALF, &tmB1, kb * BK, b_row, &s.full[stage]);
           } else {
@@ -431,6 +492,111 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
+  } else if (W8 && warp >= 2 + kEpiWarps) {
+    // W8 converters: for every K step of this CTA's units (the producer's and
+    // the MMA warp's order), wait for the E4M3 tile to land and for the stage's
+    // B tile to be free, decode it, then let the MMA go (second arrival on the
+    // stage's full barrier) and reuse the landing buffer for the K step
+    // kLandStages ahead.  One thread waits on the barriers and issues the
+    // copies; the decision to go on or give up reaches all 128 threads through
+    // shared memory, so they leave together.
+    const int ct = threadIdx.x - (2 + kEpiWarps) * 32;
+    // the K-step sequence, walked twice: `cur` for decoding, `ahd` for issuing copies
+    struct Seq {
+      int u, kb, kb1;
+    };
+    auto seq_begin = [&](Seq& q) {
+      q.u = blockIdx.x;
+      q.kb = 0;
+      q.kb1 = 0;
+      while (q.u < total) {
+        const UnitInfo ui = decode_unit(s, p, q.u, ks, nk);
+        q.kb = ui.kb0;
+        q.kb1 = ui.kb1;
+        if (q.kb < q.kb1) return;
+        q.u += gridDim.x;
+      }
+    };
+    auto seq_next = [&](Seq& q) {
+      if (++q.kb < q.kb1) return;
+      q.u += gridDim.x;
+      while (q.u < total) {
+        const UnitInfo ui = decode_unit(s, p, q.u, ks, nk);
+        q.kb = ui.kb0;
+        q.kb1 = ui.kb1;
+        if (q.kb < q.kb1) return;
+        q.u += gridDim.x;
+      }
+    };
+    auto issue = [&](const Seq& q, int l) {  // E4M3 tile of K step q into landing buffer l
+      const UnitInfo ui = decode_unit(s, p, q.u, ks, nk);
+      const int b_row = ui.ti.grp.expert * p.n_per_slab + ui.ti.n_idx * p.bn_out;
+      uint8_t* dst = land + l * LAND_BYTES;
+      mbar_arrive_expect_tx(&s.lfull[l], LAND_BYTES);
+      if (EPI == EPI_SWIGLU) {
+        tma_load_2d(dst, &tmB0, q.kb * BK, b_row, &s.lfull[l]);
+        tma_load_2d(dst + LAND_BYTES / 2, &tmB1, q.kb * BK, b_row, &s.lfull[l]);
+      } else {
+        tma_load_2d(dst, &tmB0, q.kb * BK, b_row, &s.lfull[l]);
+        tma_load_2d(dst + LAND_BYTES / 2, &tmB0, q.kb * BK, b_row + 128, &s.lfull[l]);
+      }
+    };
+    Seq cur, ahd;
+    seq_begin(cur);
+    seq_begin(ahd);
+    uint32_t armed = 0;  // landing buffers with a copy in flight
+    uint32_t lphase_bits = 0;
+    if (ct == 0 && !p.test_stall) {
+      for (int l = 0; l < kLandStages && ahd.u < total; ++l) {
+        issue(ahd, l);
+        armed |= 1u << l;
+        seq_next(ahd);
+      }
+    }
+    int stage = 0, l = 0;
+    uint32_t phase = 0, lphase = 0;
+    bool ok = true;
+    while (cur.u < total) {
+      if (ct == 0) {
+        int go = !p.test_stall && mbar_wait(&s.lfull[l], lphase, abort_flag) &&
+                 mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag);
+        if (go) armed &= ~(1u << l);
+        s.conv_ok = go;
+      }
+      named_bar_sync(1, 32 * kConvWarps);
+      if (!s.conv_ok) {
+        ok = false;
+        break;
+      }
+      convert_tile_w8(land + l * LAND_BYTES, ring + stage * STAGE_BYTES + A_TILE, ct);
+      fence_proxy_async_smem();  // generic-proxy writes before the tensor core's reads
+      named_bar_sync(1, 32 * kConvWarps);
+      if (ct == 0) {
+        mbar_arrive(&s.full[stage]);
+        if (ahd.u < total) {
+          issue(ahd, l);
+          armed |= 1u << l;
+          lphase_bits = (lphase_bits & ~(1u << l)) | (((lphase + 1u) & 1u) << l);
+          seq_next(ahd);
+        }
+      }
+      seq_next(cur);
+      if (++stage == STAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+      if (++l == kLandStages) {
+        l = 0;
+        lphase ^= 1u;
+      }
+    }
+    if (!ok && ct == 0) {
+      *abort_flag = 1;
+      report(p.status, MOE_STATUS_TIMEOUT, MOE_CNT_TIMEOUT);
+      // let the copies already issued land before the CTA exits
+      for (int i = 0; i < kLandStages; ++i)
+        if (armed & (1u << i)) wait_timed(&s.lfull[i], (lphase_bits >> i) & 1u);
+    }
   } else {
     const int q = warp & 3;                // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;      // which half of the tile's columns it drains
@@ -477,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  if (warp >= 2 && lane == 0) bulk_wait_all();  // this warp's output boxes are written
+  if (warp >= 2 && warp < 2 + kEpiWarps && lane == 0) bulk_wait_all();  // this warp's output boxes are written
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -486,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int EPI, bool F8>
+template <int EPI, bool F8, bool W8 = false>
 cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB0, const CUtensorMap& mB1,
                        const CUtensorMap& mOut, const TcParams& p, int grid, int bma, int stages, size_t smem,
                        int64_t max_group_rows, cudaStream_t stream) {
@@ -495,14 +661,14 @@ cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUte
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64 || !(attr_set & (1ull << dev))) {
-    e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<EPI, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<EPI, F8, W8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemLimitTc));
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set |= 1ull << dev;
   }
   // programmatic dependent launch: the prologue may overlap the previous kernel
-  e = launch_pdl(grouped_gemm_tc_kernel<EPI, F8>, dim3(grid), dim3(kThreads), smem, stream, mA, mA2, mB0, mB1, mOut,
-                 p, bma, stages);
+  e = launch_pdl(grouped_gemm_tc_kernel<EPI, F8, W8>, dim3(grid), dim3(W8 ? kThreadsW8 : kThreads), smem, stream, mA,
+                 mA2, mB0, mB1, mOut, p, bma, stages);
   if (e != cudaSuccess) return e;
   if ((e = cudaGetLastError()) != cudaSuccess || p.max_ksplit <= 1 || p.inkernel_reduce) return e;
   dim3 fgrid((p.N + 1023) / 1024, static_cast<unsigned>(max_group_rows), p.num_groups);
@@ -520,9 +686,11 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
   if (a.max_group_rows > 0 && a.max_group_rows <= 64) bma = static_cast<int>((a.max_group_rows + 15) & ~int64_t(15));
   const size_t stage_bytes = static_cast<size_t>(bma) * BK_BYTES + B_TILE;
   const int eb = a.fp8 ? 1 : 2;  // element bytes of A and B
-  int stages = static_cast<int>((kSmemLimitTc - kCtlBytes) / stage_bytes);
+  const bool w8 = a.w8 != 0 && !a.fp8;
+  const size_t land_bytes = w8 ? static_cast<size_t>(kLandStages) * LAND_BYTES : 0;
+  int stages = static_cast<int>((kSmemLimitTc - kCtlBytes - land_bytes) / stage_bytes);
   if (stages > MAX_STAGES) stages = MAX_STAGES;
-  const size_t smem = stages * stage_bytes + kCtlBytes;
+  const size_t smem = stages * stage_bytes + land_bytes + kCtlBytes;
   CUtensorMap mA, mA2, mB0, mB1, mOut;
   // bf16 outputs: full 32-row quarters go out as bulk tensor stores; fp32 outputs store row by row
   TcParams pp = p;
@@ -534,11 +702,21 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
   } else {
     mA2 = mA;
   }
-  if (!make_map(&mB0, a.b0, a.b_rows, a.K, 128, eb)) return cudaErrorInvalidValue;
-  if (a.epilogue == EPI_SWIGLU) {
-    if (!make_map(&mB1, a.b1, a.b_rows, a.K, 128, eb)) return cudaErrorInvalidValue;
+  if (w8) {
+    // E4M3 weight tiles of one bf16 K step: 64 codes (64 bytes) x 128 rows, unswizzled
+    if (!make_map_w8(&mB0, a.b0, a.b_rows, a.K)) return cudaErrorInvalidValue;
+    if (a.epilogue == EPI_SWIGLU) {
+      if (!make_map_w8(&mB1, a.b1, a.b_rows, a.K)) return cudaErrorInvalidValue;
+    } else {
+      mB1 = mB0;
+    }
   } else {
-    mB1 = mB0;
+    if (!make_map(&mB0, a.b0, a.b_rows, a.K, 128, eb)) return cudaErrorInvalidValue;
+    if (a.epilogue == EPI_SWIGLU) {
+      if (!make_map(&mB1, a.b1, a.b_rows, a.K, 128, eb)) return cudaErrorInvalidValue;
+    } else {
+      mB1 = mB0;
+    }
   }
   // upper bound of the tile count: every group may add one partial m-block
   const int64_t bound = (a.max_total_rows / BM + a.num_groups) * static_cast<int64_t>(p.n_tiles);
@@ -549,6 +727,17 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
         return launch_epi<EPI_SWIGLU, true>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
       case EPI_NONE:
         return launch_epi<EPI_NONE, true>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  if (w8) {  // E4M3 weights, bf16 activations: SwiGLU experts only
+    switch (a.epilogue) {
+      case EPI_SWIGLU:
+        return launch_epi<EPI_SWIGLU, false, true>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem,
+                                                   a.max_group_rows, stream);
+      case EPI_NONE:
+        return launch_epi<EPI_NONE, false, true>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem,
+                                                 a.max_group_rows, stream);
       default: return cudaErrorInvalidValue;
     }
   }

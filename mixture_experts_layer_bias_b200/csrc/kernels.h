@@ -116,6 +116,7 @@ struct GemmArgs {
   int* tile_count;          // split-K arrival counters (zero between launches; nullptr = none)
   int64_t tile_count_len;   // number of counters
   int fp8;                  // 1: A and B are E4M3 (kind::f8f6f4); A rows scaled by row_scale
+  int w8;                   // 1: B (weights) E4M3, A bf16: the GEMM decodes each weight tile to bf16
   const float* row_scale;        // [a rows] per-row scale of A (fp8 only)
   const float* row_scale_shared; // [S] per-row scale of the shared expert's A rows (fp8 only)
   StatusBlock* status;

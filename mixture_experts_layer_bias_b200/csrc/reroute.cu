@@ -11,11 +11,11 @@
 //
 // The visit order makes this a serial assignment.  One CTA runs it in rounds
 // over chunks of up to 1024 excess slots: every slot picks its expert against
-// the room left at the start of the round (8 lanes per slot, splitting the
-// experts; a token's slots in one chunk go to one lane group, in k order, each
-// excluding the previous picks), the
-// picks are ranked per expert in slot order, and the longest prefix of slots
-// whose pick still fits is committed.  A pick made against the round's room
+// the room left at the start of the round (one thread per slot over the
+// token's whole key row; the later slots of a token with several excess slots
+// in the chunk are then fixed up in k order, each excluding the earlier
+// picks), the picks are ranked per expert in slot order, and the longest
+// prefix of slots whose pick still fits is committed.  A pick made against the round's room
 // is the serial pick as long as every earlier slot's pick fit (room only
 // shrinks, and the picked expert is still available), so the committed prefix
 // equals the serial result; the first slot that does not fit had filled its
@@ -30,8 +30,58 @@ namespace {
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxE = 256;
-constexpr int kG = 8;                     // lanes per slot pick (kMaxE / kG <= 32 held bits)
-constexpr int kSpan = kThreads / (kThreads / kG);  // slots per group and round (a chunk over all groups)
+
+// The best candidate expert of excess slot s with room left (room[e] > 0),
+// a finite key, not held by the slot's token (its current K experts) and not
+// in extra[0..n_extra): highest key, ties to the lower index; -1 if none.
+// The key row is read with 16-byte loads issued before the comparisons.
+__device__ int best_pick(int s, int E, int K, const int32_t* topk_idx, const float* cand_key, const int* room,
+                         const int* extra, int n_extra) {
+  const float kNegInf = __int_as_float(0xff800000);
+  const int t = s / K;
+  uint32_t held[kMaxE / 32];
+#pragma unroll
+  for (int i = 0; i < kMaxE / 32; ++i) held[i] = 0;
+  for (int k = 0; k < K; ++k) {
+    const int e = topk_idx[static_cast<int64_t>(t) * K + k];
+    if (e >= 0 && e < E) held[e >> 5] |= 1u << (e & 31);
+  }
+  for (int i = 0; i < n_extra; ++i) held[extra[i] >> 5] |= 1u << (extra[i] & 31);
+  const float* row = cand_key + static_cast<int64_t>(t) * E;
+  float bv = kNegInf;
+  int be = -1;
+  // E is a multiple of 4 here (whole 16-byte loads) or handled one by one
+  const int e4 = (E % 4 == 0) ? E : 0;
+  for (int e0 = 0; e0 < e4; e0 += 32) {
+    float4 v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      v[j] = (e0 + 4 * j < e4) ? __ldg(reinterpret_cast<const float4*>(row + e0 + 4 * j))
+                               : make_float4(kNegInf, kNegInf, kNegInf, kNegInf);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float kv[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int e = e0 + 4 * j + c;
+        if (e >= E || !(kv[c] > kNegInf) || ((held[e >> 5] >> (e & 31)) & 1u) || room[e] <= 0) continue;
+        if (kv[c] > bv) {  // ascending e: a tie keeps the lower index
+          bv = kv[c];
+          be = e;
+        }
+      }
+    }
+  }
+  for (int e = e4; e < E; ++e) {
+    const float kv = __ldg(row + e);
+    if (!(kv > kNegInf) || ((held[e >> 5] >> (e & 31)) & 1u) || room[e] <= 0) continue;
+    if (kv > bv) {
+      bv = kv;
+      be = e;
+    }
+  }
+  return be;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     reroute_assign_kernel(int S, int E, int K, int C, int32_t* __restrict__ topk_idx,
@@ -111,77 +161,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) s_first_bad = m;
     __syncthreads();
     {
-      // groups of kG lanes; group g takes the chunk's slots from the first run
-      // start at or after kSpan*g up to the first run start at or after
-      // kSpan*(g+1), so a token's slots stay in one group and are picked in k
-      // order.  Lane q of a group holds experts q, q + kG, q + 2 kG, ...
-      auto run_start = [&](int i) {  // first i' >= i that starts a token's run (or m)
-        while (i < m && i > 0 && sx[i - 1] / K == sx[i] / K) ++i;
-        return i < m ? i : m;
-      };
-      const int g = tid / kG, q = tid % kG;
-      const int i0 = g == 0 ? 0 : run_start(min(kSpan * g, m));
-      const int i1 = run_start(min(kSpan * (g + 1), m));
-      // the longest range of the warp's groups sets the warp's step count
-      int steps = i1 - i0;
-#pragma unroll
-      for (int off = kG; off < 32; off <<= 1) steps = max(steps, __shfl_xor_sync(0xFFFFFFFFu, steps, off));
-      uint32_t held = 0;  // bit r: expert q + kG*r is held by the current token
-      int cur_t = -1;
-      for (int step = 0; step < steps; ++step) {
-        const int i = i0 + step;
-        const bool act = i < i1;
-        const int s = act ? sx[i] : 0;
-        const int t = s / K;
-        if (act && t != cur_t) {  // the token's current experts, loads issued in batches of 8
-          cur_t = t;
-          held = 0;
-          const int32_t* row = topk_idx + static_cast<int64_t>(t) * K;
-          for (int k0 = 0; k0 < K; k0 += 8) {
-            int ev[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) ev[u] = k0 + u < K ? row[k0 + u] : -1;
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              if (ev[u] >= 0 && ev[u] < E && ev[u] % kG == q) held |= 1u << (ev[u] / kG);
-          }
-        }
-        // the best candidate with room that the token does not hold; key loads in batches of 8
-        float bv = kNegInf;
-        int be = 0x7fffffff;
-        if (act) {
-          const float* key = cand_key + static_cast<int64_t>(t) * E;
-          for (int r0 = 0; r0 * kG < E; r0 += 8) {
-            float kv[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int e = (r0 + u) * kG + q;
-              kv[u] = e < E ? __ldg(key + e) : kNegInf;
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int r = r0 + u, e = r * kG + q;
-              if (!(kv[u] > kNegInf) || ((held >> r) & 1u) || room[e] <= 0) continue;
-              if (kv[u] > bv || (kv[u] == bv && e < be)) {
-                bv = kv[u];
-                be = e;
-              }
-            }
-          }
-        }
-#pragma unroll
-        for (int off = kG / 2; off >= 1; off >>= 1) {
-          const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
-          const int oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
-          if (ov > bv || (ov == bv && oe < be)) {
-            bv = ov;
-            be = oe;
-          }
-        }
-        if (act) {
-          const int best = bv > kNegInf ? be : -1;
-          if (q == 0) ch[i] = best;
-          if (best >= 0 && best % kG == q) held |= 1u << (best / kG);
+      // one thread per slot: the best candidate with room that the token does
+      // not hold, over the token's whole key row (16-byte loads, all issued
+      // together); then the slots of a token that has several excess slots
+      // in this chunk are fixed up in k order, each excluding the earlier
+      // ones' picks
+      if (tid < m) ch[tid] = best_pick(sx[tid], E, K, topk_idx, cand_key, room, nullptr, 0);
+      __syncthreads();
+      if (tid < m && (tid == 0 || sx[tid - 1] / K != sx[tid] / K) && tid + 1 < m && sx[tid + 1] / K == sx[tid] / K) {
+        int taken[32];
+        int nt = 0;
+        if (ch[tid] >= 0) taken[nt++] = ch[tid];
+        for (int j = tid + 1; j < m && sx[j] / K == sx[tid] / K; ++j) {
+          bool clash = false;
+          for (int i = 0; i < nt; ++i) clash |= ch[j] == taken[i];
+          if (clash) ch[j] = best_pick(sx[j], E, K, topk_idx, cand_key, room, taken, nt);
+          if (ch[j] >= 0 && nt < 32) taken[nt++] = ch[j];
         }
       }
     }

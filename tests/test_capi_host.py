@@ -303,3 +303,19 @@ def test_missing_library_fails_loudly():
             "try:\n    ops.lib()\nexcept RuntimeError as e:\n    print('raised', e)\n")
     r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True)
     assert "raised" in r.stdout, (r.stdout, r.stderr)
+
+
+def test_e4m3_workspace_holds_no_decoded_weights():
+    """E4M3 weights with bf16 activations are decoded tile by tile inside the
+    GEMMs: the workspace is no larger than with bf16 weights (no bf16 copy of
+    the weights).  With d or h not a multiple of 16 the layer decodes the
+    weights into the workspace first."""
+    c8 = syn.CONFIGS["fp8_skew_capacity"]
+    c16 = syn.scaled(c8, weight_dtype=syn.BF16)
+    n8 = ops.moe_workspace_size(ops.make_desc(**syn.desc_dict(c8)))
+    n16 = ops.moe_workspace_size(ops.make_desc(**syn.desc_dict(c16)))
+    assert n8 == n16
+    odd8 = syn.scaled(c8, d=2056)
+    odd16 = syn.scaled(c16, d=2056)
+    assert ops.moe_workspace_size(ops.make_desc(**syn.desc_dict(odd8))) > \
+        ops.moe_workspace_size(ops.make_desc(**syn.desc_dict(odd16)))
