@@ -69,6 +69,7 @@ typedef enum { MOE_ACT_GELU = 0, MOE_ACT_SWIGLU = 1 } moe_act;
 #define MOE_STATUS_BAD_EXPERT_ID 0x2u   /* moe_permute saw an id outside [0,E) */
 #define MOE_STATUS_TIMEOUT 0x4u         /* a bounded device wait gave up */
 #define MOE_STATUS_BAD_GROUP 0x8u       /* a group table entry out of range */
+#define MOE_STATUS_DEBUG_CHECK 0x10u    /* an invariant check of a MOE_DEBUG build failed */
 
 /* counters (moe_get_status counters[], MOE_NUM_COUNTERS entries) */
 #define MOE_CNT_NONFINITE 0   /* tokens with a non-finite logit */

@@ -10,6 +10,13 @@ A second library, libmoe_b200_testhooks.so, is linked from the same objects
 except the GEMM launch file, which is compiled with MOE_B200_TEST_HOOKS: it
 adds the failure-detection test hook (moe_test_stall_gemms) that the product
 library does not contain.  Only the failure-detection test loads it.
+
+A third, libmoe_b200_debug.so, is the guard build: the permutation and
+combine files are compiled with MOE_DEBUG, which adds a check kernel after
+every permutation (counts, offsets, row_of_slot and token_of_row agree) and a
+range check of every row the combine reads; a violation sets
+MOE_STATUS_DEBUG_CHECK in the status block.  Its results are otherwise those
+of the product library.
 """
 from __future__ import annotations
 
@@ -28,6 +35,8 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe_b200.so")
 TEST_HOOKS_LIB = os.path.join(PKG, "libmoe_b200_testhooks.so")
 TEST_HOOKS_SOURCE = "gemm_dispatch.cu"
+DEBUG_LIB = os.path.join(PKG, "libmoe_b200_debug.so")
+DEBUG_SOURCES = ("permute.cu", "combine.cu")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",
@@ -78,7 +87,7 @@ def build(force: bool = False, jobs: int = 8, extra=(), out: str = LIB, build_di
           test_hooks: bool = True) -> str:
     """Compile every source (extra nvcc flags, e.g. -D tuning macros, go to
     all of them) into build_dir and link `out`; with test_hooks also link the
-    test-hook library next to the product one."""
+    test-hook and guard (MOE_DEBUG) libraries next to the product one."""
     os.makedirs(build_dir, exist_ok=True)
     srcs = sources()
     with cf.ThreadPoolExecutor(max_workers=jobs) as ex:
@@ -91,6 +100,12 @@ def build(force: bool = False, jobs: int = 8, extra=(), out: str = LIB, build_di
         hook_obj = _compile(hook_src, force, list(extra) + ["-DMOE_B200_TEST_HOOKS"], hook_dir)
         objs_h = [hook_obj if os.path.basename(o) == TEST_HOOKS_SOURCE + ".o" else o for o in objs]
         _link(objs_h, TEST_HOOKS_LIB, force)
+        debug_dir = os.path.join(build_dir, "debug")
+        os.makedirs(debug_dir, exist_ok=True)
+        dbg = {src: _compile(os.path.join(CSRC, src), force, list(extra) + ["-DMOE_DEBUG"], debug_dir)
+               for src in DEBUG_SOURCES}
+        objs_d = [dbg.get(os.path.basename(o)[:-2], o) for o in objs]
+        _link(objs_d, DEBUG_LIB, force)
     return out
 
 

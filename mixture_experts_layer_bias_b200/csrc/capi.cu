@@ -255,11 +255,20 @@ PermuteArgs permute_args(const moe_desc& d, const void* x, const int32_t* topk_i
   return a;
 }
 
+// A MOE_DEBUG build checks the permutation's invariants after it (a no-op
+// otherwise: nothing is launched).
+moe_status debug_check(const PermuteArgs& a, cudaStream_t st) {
+  return cuda_status(launch_debug_check_permutation(a.S, a.E, a.K, a.capacity, a.counts, a.offsets, a.row_of_slot,
+                                                    a.token_of_row, a.num_rows, a.status, st));
+}
+
 moe_status permute_impl(const moe_desc& d, const void* x, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
                         int32_t* row_of_slot, int32_t* token_of_row, void* x_perm, void* ws, cudaStream_t st,
                         bool write_groups = false) {
-  return cuda_status(launch_permute(
-      permute_args(d, x, topk_idx, counts, offsets, row_of_slot, token_of_row, x_perm, ws, write_groups), st));
+  const PermuteArgs a =
+      permute_args(d, x, topk_idx, counts, offsets, row_of_slot, token_of_row, x_perm, ws, write_groups);
+  const moe_status s = cuda_status(launch_permute(a, st));
+  return s != MOE_OK ? s : debug_check(a, st);
 }
 
 // Record stage event `i` of `events` (moe_layer_forward_timed), if given.
@@ -431,8 +440,10 @@ moe_status reroute_impl(const moe_desc& d, int32_t* topk_idx, float* topk_w, con
 }
 
 moe_status combine_impl(const moe_desc& d, const void* y_perm, const int32_t* row_of_slot, const float* topk_w,
-                        void* y, cudaStream_t st) {
+                        void* y, cudaStream_t st, StatusBlock* status = nullptr) {
   CombineArgs a{};
+  a.num_rows = routed_rows(d) + static_cast<int64_t>(d.num_shared) * d.num_tokens;
+  a.status = status;
   a.S = d.num_tokens;
   a.d = d.d_model;
   a.K = d.top_k;
@@ -488,6 +499,7 @@ moe_status layer_impl(const moe_desc* desc, const moe_weights* w, const void* x,
     const RouteArgs ra = route_args(d, w, x, nullptr, idx, gates, ws);
     const PermuteArgs pa = permute_args(d, x, idx, cnt, offs, ros, tor, w8a8 ? nullptr : x_perm, ws, true);
     if (launch_route_permute_small(ra, pa, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if ((s = debug_check(pa, st)) != MOE_OK) return s;
     if (!record(events, 1, st)) return MOE_ERR_CUDA;
     if (w8a8) {
       const bool sh = d.num_shared != 0;
@@ -498,7 +510,7 @@ moe_status layer_impl(const moe_desc* desc, const moe_weights* w, const void* x,
     }
     if (!record(events, 2, st)) return MOE_ERR_CUDA;
     if ((s = ffn_impl(d, *w, x_perm, offs, x, y_perm, ws, st, true, w8a8, events)) != MOE_OK) return s;
-    if ((s = combine_impl(d, y_perm, ros, gates, y, st)) != MOE_OK) return s;
+    if ((s = combine_impl(d, y_perm, ros, gates, y, st, at<StatusBlock>(ws, L.status))) != MOE_OK) return s;
     return record(events, 7, st) ? MOE_OK : MOE_ERR_CUDA;
   }
   if ((s = route_impl(d, w, x, nullptr, idx, gates, ws, st)) != MOE_OK) return s;
@@ -526,7 +538,7 @@ moe_status layer_impl(const moe_desc* desc, const moe_weights* w, const void* x,
     if (!record(events, 2, st)) return MOE_ERR_CUDA;
     if ((s = ffn_impl(d, *w, x_perm, offs, x, y_perm, ws, st, true, false, events)) != MOE_OK) return s;
   }
-  if ((s = combine_impl(d, y_perm, ros, gates, y, st)) != MOE_OK) return s;
+  if ((s = combine_impl(d, y_perm, ros, gates, y, st, at<StatusBlock>(ws, L.status))) != MOE_OK) return s;
   return record(events, 7, st) ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -631,7 +643,8 @@ moe_status moe_combine(const moe_desc* desc, const void* y_perm, const int32_t* 
   if (desc->num_tokens == 0) return MOE_OK;
   if (y_perm == nullptr || row_of_slot == nullptr || topk_w == nullptr || y == nullptr) return MOE_ERR_INVALID_ARG;
   if (!aligned16(y_perm) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
-  return combine_impl(*desc, y_perm, row_of_slot, topk_w, y, static_cast<cudaStream_t>(stream));
+  return combine_impl(*desc, y_perm, row_of_slot, topk_w, y, static_cast<cudaStream_t>(stream),
+                      at<StatusBlock>(ws, make_layout(*desc).status));
 }
 
 moe_status moe_layer_forward(const moe_desc* desc, const moe_weights* w, const void* x, void* y, int32_t* topk_idx,
@@ -699,7 +712,7 @@ moe_status moe_get_status(const void* ws, void* stream, uint32_t* flags, int32_t
   if (flags) *flags = host.flags;
   if (counters) memcpy(counters, host.counters, sizeof(host.counters));
   const uint32_t errors = MOE_STATUS_NONFINITE_LOGIT | MOE_STATUS_BAD_EXPERT_ID | MOE_STATUS_TIMEOUT |
-                          MOE_STATUS_BAD_GROUP;
+                          MOE_STATUS_BAD_GROUP | MOE_STATUS_DEBUG_CHECK;
   return (host.flags & errors) ? MOE_ERR_DEVICE_STATUS : MOE_OK;
 }
 

@@ -24,14 +24,22 @@ namespace {
 template <typename T>
 __global__ void __launch_bounds__(256)
     combine_cta_kernel(int d, int K, const T* __restrict__ y_perm, const int32_t* __restrict__ row_of_slot,
-                       const float* __restrict__ topk_w, int64_t shared_row0, T* __restrict__ y) {
+                       const float* __restrict__ topk_w, int64_t shared_row0, T* __restrict__ y, int64_t num_rows,
+                       StatusBlock* status) {
   __shared__ int32_t rows[32];
   __shared__ float gates[32];
   pdl_wait();
   pdl_trigger();
   const int t = blockIdx.x;
   if (threadIdx.x < K) {
-    rows[threadIdx.x] = row_of_slot[static_cast<int64_t>(t) * K + threadIdx.x];
+    int r = row_of_slot[static_cast<int64_t>(t) * K + threadIdx.x];
+#ifdef MOE_DEBUG
+    if (r >= num_rows) {  // a row outside y_perm: report and skip it
+      report(status, MOE_STATUS_DEBUG_CHECK, -1);
+      r = -1;
+    }
+#endif
+    rows[threadIdx.x] = r;
     gates[threadIdx.x] = topk_w[static_cast<int64_t>(t) * K + threadIdx.x];
   }
   __syncthreads();
@@ -94,11 +102,11 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream) {
   if (a.act_dtype == MOE_BF16)
     err = launch_pdl(combine_cta_kernel<__nv_bfloat16>, dim3(a.S), dim3(threads), 0, stream, a.d, a.K,
                      static_cast<const __nv_bfloat16*>(a.y_perm), a.row_of_slot, a.topk_w, a.shared_row0,
-                     static_cast<__nv_bfloat16*>(a.y));
+                     static_cast<__nv_bfloat16*>(a.y), a.num_rows, a.status);
   else
     err = launch_pdl(combine_cta_kernel<float>, dim3(a.S), dim3(threads), 0, stream, a.d, a.K,
                      static_cast<const float*>(a.y_perm), a.row_of_slot, a.topk_w, a.shared_row0,
-                     static_cast<float*>(a.y));
+                     static_cast<float*>(a.y), a.num_rows, a.status);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }

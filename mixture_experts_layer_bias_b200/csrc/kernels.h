@@ -168,7 +168,19 @@ struct CombineArgs {
   const float* topk_w;
   int64_t shared_row0;  // -1 = no shared expert
   void* y;
+  int64_t num_rows;     // rows of y_perm (debug builds check row_of_slot against it)
+  StatusBlock* status;  // debug builds report a row outside y_perm here (may be nullptr)
 };
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
+
+// --- MOE_DEBUG builds ----------------------------------------------------------
+// Invariants of a permutation: offsets[e+1] - offsets[e] = counts[e] (and the
+// overflow split with a capacity), every row_of_slot in [-1, R), token_of_row
+// the inverse map.  A violation sets MOE_STATUS_DEBUG_CHECK.  Launched after
+// every permutation of a debug build only.
+cudaError_t launch_debug_check_permutation(int S, int E, int K, int capacity, const int32_t* counts,
+                                           const int32_t* offsets, const int32_t* row_of_slot,
+                                           const int32_t* token_of_row, int64_t num_rows, StatusBlock* status,
+                                           cudaStream_t stream);
 
 }  // namespace moe

@@ -456,7 +456,54 @@ __global__ void build_groups_kernel(int S, int E, int K, int capacity, int num_s
   write_groups(S, E, K, capacity, num_shared, offsets, g1);
 }
 
+#ifdef MOE_DEBUG
+__global__ void __launch_bounds__(256)
+    debug_check_permutation_kernel(int S, int E, int K, int capacity, const int32_t* counts, const int32_t* offsets,
+                                   const int32_t* row_of_slot, const int32_t* token_of_row, int64_t num_rows,
+                                   StatusBlock* status) {
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  bool bad = false;
+  if (tid < E) {
+    const int c = counts[tid];
+    if (c < 0 || offsets[tid + 1] - offsets[tid] != c) bad = true;
+    if (capacity > 0) {
+      const int ovf = c > capacity ? c - capacity : 0;
+      if (offsets[E + 1 + tid + 1] - offsets[E + 1 + tid] != ovf) bad = true;
+    }
+  }
+  if (tid == 0 && offsets[0] != 0) bad = true;
+  for (int64_t sl = tid; sl < static_cast<int64_t>(S) * K; sl += nthreads) {
+    const int r = row_of_slot[sl];
+    if (r < -1 || r >= num_rows) {
+      bad = true;
+    } else if (r >= 0 && token_of_row[r] != static_cast<int32_t>(sl / K)) {
+      bad = true;
+    }
+  }
+  if (bad) report(status, MOE_STATUS_DEBUG_CHECK, -1);
+}
+#endif
+
 }  // namespace
+
+cudaError_t launch_debug_check_permutation(int S, int E, int K, int capacity, const int32_t* counts,
+                                           const int32_t* offsets, const int32_t* row_of_slot,
+                                           const int32_t* token_of_row, int64_t num_rows, StatusBlock* status,
+                                           cudaStream_t stream) {
+#ifdef MOE_DEBUG
+  if (S <= 0) return cudaSuccess;
+  const int64_t work = static_cast<int64_t>(S) * K > E ? static_cast<int64_t>(S) * K : E;
+  const int blocks = static_cast<int>(work / 256 + 1 < 1184 ? work / 256 + 1 : 1184);
+  debug_check_permutation_kernel<<<blocks, 256, 0, stream>>>(S, E, K, capacity, counts, offsets, row_of_slot,
+                                                              token_of_row, num_rows, status);
+  return cudaGetLastError();
+#else
+  (void)S; (void)E; (void)K; (void)capacity; (void)counts; (void)offsets; (void)row_of_slot; (void)token_of_row;
+  (void)num_rows; (void)status; (void)stream;
+  return cudaSuccess;
+#endif
+}
 
 bool route_permute_fusable(int S, int E, int K) {
   return S >= 1 && S <= kFusedMaxTokens && E <= 32 && static_cast<int64_t>(S) * K <= kSmallSlots;

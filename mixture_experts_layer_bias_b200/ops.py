@@ -19,6 +19,7 @@ _lib = None
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE_STATUS = range(6)
 MOE_STATUS_NONFINITE_LOGIT, MOE_STATUS_BAD_EXPERT_ID, MOE_STATUS_TIMEOUT, MOE_STATUS_BAD_GROUP = 1, 2, 4, 8
+MOE_STATUS_DEBUG_CHECK = 0x10
 MOE_NUM_COUNTERS = 8
 COUNTER_NAMES = ("nonfinite", "bad_id", "timeout", "overflow_rows", "rerouted")
 
