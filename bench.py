@@ -119,28 +119,28 @@ def workload_desc(cfg):
             f"{', W8A8 (e4m3 activation rows, per-row scales)' if cfg.act_quant else ''}")
 
 
+# E4M3 weights with bf16 activations are decoded inside the GEMMs up to this
+# many routed rows per expert on average, above it by a decode pass
+W8_IN_GEMM_ROWS = 1024
+
+
 def kernels_per_step(cfg, S=None):
     """Launches of this library's kernels in one moe_layer_forward call."""
     S = cfg.S if S is None else S
     small = S * cfg.K <= 4096               # one-CTA permutation for small batches
-    if not cfg.reroute and 1 <= S <= 16 and cfg.E <= 32 and small:
-        n = 1                              # routing, permutation and row gather in one kernel
-        if cfg.act_quant:
-            n += 1                         # the quantising row gather
-    else:
-        n = 1 if (cfg.E <= 32) else 2      # route (fused) or logits GEMM + top-k
-        n += 1 if small else 4             # permutation (+ group table): one kernel, or count, scan, scatter, groups
-        n += 1                             # row gather (quantising for W8A8)
+    n = 1 if (cfg.E <= 32) else 2          # route (logits in the routing kernel) or logits GEMM + top-k
+    n += 1 if small else 4                 # permutation (+ group table): one kernel, or count, scan, scatter, groups
+    n += 1                                 # row gather (quantising for W8A8)
     n += 2                                 # up and down GEMM
     rows = S * cfg.K + cfg.num_shared * S + (cfg.E * cfg.capacity if cfg.capacity else 0)
-    if cfg.act_dtype == syn.BF16 and rows <= 4096 and S > 16:
-        n += 2                             # split-K finalize of both GEMMs (S <= 16 reduce inside the GEMMs)
+    if cfg.act_dtype == syn.BF16 and rows <= 4096:
+        n += 2                             # split-K finalize of both GEMMs
     if cfg.act_quant:
         n += 1                             # per-row E4M3 quantisation of the hidden rows
-    elif cfg.weight_dtype == syn.E4M3 and (cfg.d % 16 or cfg.h % 16):
+    elif cfg.weight_dtype == syn.E4M3 and (cfg.d % 16 or cfg.h % 16 or S * cfg.K > W8_IN_GEMM_ROWS * cfg.E):
         n += 3                             # E4M3 -> bf16 decode of the three stacks (else inside the GEMMs)
     if cfg.reroute:
-        n += (1 if small else 3) + 2       # ranks, re-route assignment and gates
+        n += (1 if small else 3) + 3       # ranks, re-route picks and epochs, gates
     n += 1                                 # combine
     return n
 

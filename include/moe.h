@@ -34,12 +34,8 @@
  *    workspace and never trap; read them with moe_get_status.
  *  - ws / ws_bytes: caller-allocated device scratch of at least
  *    moe_workspace_size() bytes, 256-byte aligned.  Its first 256 bytes hold
- *    the status block, the next 256 KB the grouped GEMMs' split-K arrival
- *    counters (the same place for every desc, so one workspace can serve
- *    several descs); moe_workspace_init zeroes both, and every completed call
- *    leaves the counters zero.  After a MOE_STATUS_TIMEOUT, run
- *    moe_workspace_init again before reusing the workspace.  Calls that share
- *    one workspace must be ordered on one stream.
+ *    the status block; moe_workspace_init zeroes it.  Calls that share one
+ *    workspace must be ordered on one stream.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -69,7 +65,8 @@ typedef enum { MOE_ACT_GELU = 0, MOE_ACT_SWIGLU = 1 } moe_act;
 #define MOE_STATUS_BAD_EXPERT_ID 0x2u   /* moe_permute saw an id outside [0,E) */
 #define MOE_STATUS_TIMEOUT 0x4u         /* a bounded device wait gave up */
 #define MOE_STATUS_BAD_GROUP 0x8u       /* a group table entry out of range */
-#define MOE_STATUS_DEBUG_CHECK 0x10u    /* an invariant check of a MOE_DEBUG build failed */
+#define MOE_STATUS_DEBUG_CHECK 0x10u    /* an internal invariant check failed (the MOE_DEBUG
+                                           build's checks; the re-route assignment's epoch bound) */
 
 /* counters (moe_get_status counters[], MOE_NUM_COUNTERS entries) */
 #define MOE_CNT_NONFINITE 0   /* tokens with a non-finite logit */
@@ -184,8 +181,7 @@ int64_t moe_routed_rows(const moe_desc *desc);
  * calls need no more).  Host only, no CUDA call. */
 moe_status moe_workspace_size(const moe_desc *desc, size_t *bytes);
 
-/* Zero the status block and the split-K counters at the start of `ws` (the
- * first min(ws_bytes, 256 + 262144) bytes; stream-ordered). */
+/* Zero the status block at the start of `ws` (stream-ordered). */
 moe_status moe_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
 /*

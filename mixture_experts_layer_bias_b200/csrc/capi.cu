@@ -31,17 +31,10 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 
 struct Layout {
-  size_t status, counters, logits, chunk_hist, groups, counts, offsets, topk_idx, topk_w, row_of_slot,
+  size_t status, logits, chunk_hist, groups, counts, offsets, topk_idx, topk_w, row_of_slot,
       token_of_row, x_perm, hidden, y_perm, wdeq, ksplit, partial, partial_bytes, qa, sa, qas, sas, qh, sh, rr_key,
-      rr_score, rr_ex, rr_changed, total;
+      rr_score, rr_ex, rr_claim, rr_changed, total;
 };
-
-// Split-K arrival counters of the grouped GEMMs: a fixed region right after
-// the status block, the same for every desc, so a workspace reused across
-// descs (e.g. decode batches of varying size) keeps them valid.  They are zero
-// after moe_workspace_init and every completed GEMM leaves them zero.
-constexpr size_t kCounterInts = 65536;
-constexpr size_t kCounterBytes = kCounterInts * 4;
 
 // Split-K of the tensor-core GEMMs is available to small row spaces (decode-
 // sized batches), where too few output tiles exist to occupy every SM.  The
@@ -56,11 +49,18 @@ int64_t routed_rows(const moe_desc& d) {
 
 size_t act_bytes(const moe_desc& d) { return d.act_dtype == MOE_F32 ? 4 : 2; }
 
-// E4M3 weights with bf16 activations: the GEMMs decode the weight tiles
-// themselves when every weight row is a whole number of 16-byte pieces.
+// E4M3 weights with bf16 activations: the GEMMs decode each weight tile
+// themselves (every weight row a whole number of 16-byte pieces) while the
+// experts have few rows.  Each CTA decodes the tiles it multiplies, so a
+// weight tile is decoded once per 128-row block of its expert: with many row
+// blocks the decode (ALU and shared-memory bandwidth) outgrows the MMA, and a
+// single decode pass into the workspace followed by the bf16 GEMM is faster.
+constexpr int64_t kW8InGemmRowsPerExpert = 1024;
+
 bool w8_in_gemm(const moe_desc& d) {
   return d.weight_dtype == MOE_E4M3 && d.act_quant == 0 && d.act_dtype == MOE_BF16 && d.d_model % 16 == 0 &&
-         d.d_ff % 16 == 0;
+         d.d_ff % 16 == 0 &&
+         static_cast<int64_t>(d.num_tokens) * d.top_k <= kW8InGemmRowsPerExpert * d.num_experts;
 }
 
 Layout make_layout(const moe_desc& d) {
@@ -77,7 +77,6 @@ Layout make_layout(const moe_desc& d) {
     return at;
   };
   L.status = take(kAlign);
-  L.counters = take(kCounterBytes);
   L.logits = take(E > 32 ? static_cast<size_t>(S * E) * 4 : 0);
   L.chunk_hist = take(static_cast<size_t>(nch * E) * 4);
   L.groups = take(static_cast<size_t>(2 * E + 1) * sizeof(GroupEntry));
@@ -102,11 +101,12 @@ Layout make_layout(const moe_desc& d) {
   L.sas = take(w8a8 && d.num_shared ? static_cast<size_t>(S) * 4 : 0);
   L.qh = take(w8a8 ? static_cast<size_t>(Rt * h) : 0);
   L.sh = take(w8a8 ? static_cast<size_t>(Rt) * 4 : 0);
-  // re-routing: every expert's selection key and gate source, the excess-slot list, changed tokens
+  // re-routing: every expert's selection key and gate source, the slots' picks, token claims, changed tokens
   const bool rr = d.reroute == 1;
   L.rr_key = take(rr ? static_cast<size_t>(S * E) * 4 : 0);
   L.rr_score = take(rr ? static_cast<size_t>(S * E) * 4 : 0);
   L.rr_ex = take(rr ? static_cast<size_t>(S * K) * 4 : 0);
+  L.rr_claim = take(rr ? static_cast<size_t>(S) * 4 : 0);
   L.rr_changed = take(rr ? static_cast<size_t>(S) * 4 : 0);
   L.ksplit = take(kAlign);
   L.partial_bytes = 0;
@@ -318,8 +318,6 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
   up.partial = L.partial_bytes ? at<float>(ws, L.partial) : nullptr;
   up.partial_bytes = static_cast<int64_t>(L.partial_bytes);
   up.ksplit_out = at<int>(ws, L.ksplit);
-  up.tile_count = at<int>(ws, L.counters);
-  up.tile_count_len = static_cast<int64_t>(kCounterInts);
 
   GemmArgs down = up;
   down.a_rows_from_out = 1;
@@ -367,8 +365,9 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
       down.scale0 = w.s_down;
     } else if (d.weight_dtype == MOE_E4M3) {
       // exact E4M3 -> bf16 decode of this call's weights into the workspace
-      // (d or h not a multiple of 16); the per-channel scales are applied to
-      // the fp32 accumulators in the epilogues
+      // (many rows per expert, or d or h not a multiple of 16); the
+      // per-channel scales are applied to the fp32 accumulators in the
+      // epilogues
       const int64_t n_up = static_cast<int64_t>(slabs) * h * dm;
       char* base = at<char>(ws, L.wdeq);
       void* dg = base;
@@ -432,7 +431,7 @@ moe_status reroute_impl(const moe_desc& d, int32_t* topk_idx, float* topk_w, con
   int32_t* changed = at<int32_t>(ws, L.rr_changed);
   cudaError_t e = launch_reroute_assign(d.num_tokens, d.num_experts, d.top_k, d.capacity, topk_idx,
                                         at<float>(ws, L.rr_key), counts, row_of_slot, at<int32_t>(ws, L.rr_ex),
-                                        changed, at<StatusBlock>(ws, L.status), st);
+                                        at<int32_t>(ws, L.rr_claim), changed, at<StatusBlock>(ws, L.status), st);
   if (e == cudaSuccess)
     e = launch_reroute_gates(d.num_tokens, d.num_experts, d.top_k, d.score_fn, d.renormalize,
                              at<float>(ws, L.rr_score), changed, topk_idx, topk_w, st);
@@ -493,26 +492,6 @@ moe_status layer_impl(const moe_desc* desc, const moe_weights* w, const void* x,
   void* y_perm = at<void>(ws, L.y_perm);
   if (!record(events, 0, st)) return MOE_ERR_CUDA;
   const bool w8a8 = d.act_quant == 1;
-  if (d.reroute == 0 && route_permute_fusable(d.num_tokens, d.num_experts, d.top_k)) {
-    // tiny batch: routing, permutation (with the group tables) and the row
-    // gather in one kernel; W8A8 gathers E4M3 codes in its own kernel below
-    const RouteArgs ra = route_args(d, w, x, nullptr, idx, gates, ws);
-    const PermuteArgs pa = permute_args(d, x, idx, cnt, offs, ros, tor, w8a8 ? nullptr : x_perm, ws, true);
-    if (launch_route_permute_small(ra, pa, st) != cudaSuccess) return MOE_ERR_CUDA;
-    if ((s = debug_check(pa, st)) != MOE_OK) return s;
-    if (!record(events, 1, st)) return MOE_ERR_CUDA;
-    if (w8a8) {
-      const bool sh = d.num_shared != 0;
-      if (launch_gather_quantize(d.num_tokens, d.d_model, d.top_k, ros, x, at<uint8_t>(ws, L.qa),
-                                 at<float>(ws, L.sa), sh ? at<uint8_t>(ws, L.qas) : nullptr,
-                                 sh ? at<float>(ws, L.sas) : nullptr, st) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    }
-    if (!record(events, 2, st)) return MOE_ERR_CUDA;
-    if ((s = ffn_impl(d, *w, x_perm, offs, x, y_perm, ws, st, true, w8a8, events)) != MOE_OK) return s;
-    if ((s = combine_impl(d, y_perm, ros, gates, y, st, at<StatusBlock>(ws, L.status))) != MOE_OK) return s;
-    return record(events, 7, st) ? MOE_OK : MOE_ERR_CUDA;
-  }
   if ((s = route_impl(d, w, x, nullptr, idx, gates, ws, st)) != MOE_OK) return s;
   if (d.reroute == 1) {
     // capacity ranks of the first choices, then the excess slots move; the
@@ -562,9 +541,7 @@ moe_status moe_workspace_size(const moe_desc* desc, size_t* bytes) {
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   if (ws == nullptr || ws_bytes < kAlign || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0)
     return MOE_ERR_WORKSPACE;
-  // status block and the GEMMs' split-K arrival counters
-  const size_t n = ws_bytes < kAlign + kCounterBytes ? ws_bytes : kAlign + kCounterBytes;
-  return cuda_status(cudaMemsetAsync(ws, 0, n, static_cast<cudaStream_t>(stream)));
+  return cuda_status(cudaMemsetAsync(ws, 0, kAlign, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_route(const moe_desc* desc, const moe_weights* w, const void* x, const float* logits_in,

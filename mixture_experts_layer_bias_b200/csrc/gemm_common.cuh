@@ -34,9 +34,6 @@ struct TcParams {
   float* partial;      // fp32 [max_ksplit][out_rows][pcols] (split-K partial sums)
   int pcols;           // 2N (SwiGLU: gate then up) or N
   int* ksplit_out;     // the split chosen on the device (read by the finalize kernel)
-  int inkernel_reduce; // 1: split-K slices are reduced inside the GEMM (tiny groups), 0: by the finalize kernel
-  int* tile_count;     // split-K arrival counters, kRegionsPerTile per tile, zero between launches
-  int max_tiles;       // tiles the counters cover (more tiles: no in-kernel reduction, no split-K)
   int test_stall;      // test hook: the producer delivers nothing (the bounded waits must give up)
   int tma_out;         // 1: the output tensor map is valid (full 32-row quarters use bulk tensor stores)
   const float* row_scale;         // E4M3 activations: per-row scale of the A operand rows (nullptr: none)
@@ -57,22 +54,21 @@ __device__ __forceinline__ GroupEntry group_at(const TcParams& p, int g) {
 }
 
 // Split-K factor for `tiles` output tiles on `grid` persistent CTAs: the
-// smallest split whose work units fill the CTAs' waves clearly better
-// (>= 5 points of wave efficiency per step up), with >= 4 K-blocks per unit.
+// split that minimises the busiest CTA's work, counted in K-blocks plus one
+// K-block's worth of fixed cost per work unit (its epilogue), with >= 4
+// K-blocks per unit; ties to the smaller split.
 __device__ __forceinline__ int choose_ksplit(int tiles, int grid, int nk, int kmax) {
   if (tiles <= 0 || kmax <= 1) return 1;
-  auto eff = [&](int units) {
-    const int waves = (units + grid - 1) / grid;
-    return static_cast<float>(units) / static_cast<float>(waves * grid);
-  };
+  constexpr int kUnitCost = 1;
   int best = 1;
-  float best_eff = eff(tiles);
+  int64_t best_cost = static_cast<int64_t>((tiles + grid - 1) / grid) * (nk + kUnitCost);
   for (int ks = 2; ks <= kmax; ++ks) {
     if (nk / ks < 4) break;
-    const float e = eff(tiles * ks);
-    if (e > best_eff + 0.05f) {
+    const int64_t units = static_cast<int64_t>(tiles) * ks;
+    const int64_t cost = ((units + grid - 1) / grid) * ((nk + ks - 1) / ks + kUnitCost);
+    if (cost < best_cost) {
       best = ks;
-      best_eff = e;
+      best_cost = cost;
     }
   }
   return best;
@@ -86,17 +82,10 @@ __device__ __forceinline__ bool group_ok(const GroupEntry& g, const TcParams& p)
 // Split-K: every epilogue warp of a CTA owns one region of its tile (32 rows
 // of one TMEM lane quarter x half of the tile's columns) and, per split, writes
 // its raw fp32 accumulators there to the split's slice of the partial buffer.
-// The slices are then summed in split order (deterministic whatever the
-// arrival order), the epilogue applied and the output stored, in one of two
-// ways chosen on the host:
-//  - tiny groups (decode, at most 16 rows per group): inside the GEMM.  One
-//    arrival counter per (tile, region) counts the slices written; the warp
-//    whose slice completes the count reduces the region (a few rows, so the
-//    one warp's loads are few and all in flight together) and resets the
-//    counter for the next launch.  No extra launch.
-//  - larger groups: splitk_finalize_kernel after the GEMM, one thread per
-//    four output columns of a row, so many rows are reduced in parallel.
-constexpr int kRegionsPerTile = 8;
+// splitk_finalize_kernel then sums the slices in split order (deterministic
+// whatever the order the CTAs ran in), applies the epilogue and stores the
+// output: one thread per four output columns of a row, so many rows are
+// reduced in parallel.
 
 // Epilogue of split-K sums: gate/up sums g, u (SwiGLU) or sums v, with the
 // row scale rs, channel scales and bias of column n + j.
@@ -137,56 +126,16 @@ __device__ __forceinline__ float4 splitk_sum4(const float* src, int64_t slice, i
   return acc;
 }
 
-// The last arriver's reduction of region (q, half) of a tile: rows
-// m_row0 .. m_row0 + 31 of the group, the half's output columns split over the
-// lanes in float4 pieces (SwiGLU: 64 columns, lanes 0-15 one row's 16 pieces
-// and lanes 16-31 the next row's; otherwise 128 columns, one row at a time).
-template <int EPI>
-__device__ __forceinline__ void splitk_reduce_region(const TcParams& p, const GroupEntry& grp, int m_row0, int n_tile,
-                                                     int ks, int half, int lane) {
-  const int N = p.N;
-  const int64_t slice = p.out_rows * static_cast<int64_t>(p.pcols);
-  const int64_t sbase = static_cast<int64_t>(grp.expert) * N;
-  const int r1 = min(m_row0 + 32, grp.rows);
-  constexpr int kRowsPerStep = (EPI == EPI_SWIGLU) ? 2 : 1;
-  constexpr int kHalfCols = (EPI == EPI_SWIGLU) ? 64 : 128;
-  const int piece = (EPI == EPI_SWIGLU) ? (lane & 15) : lane;
-  const int n = n_tile * p.bn_out + half * kHalfCols + 4 * piece;
-  if (n >= N) return;  // n is a multiple of 4 and N of 8: n + 3 < N
-  for (int r0 = m_row0; r0 < r1; r0 += kRowsPerStep) {
-    const int r = r0 + ((EPI == EPI_SWIGLU) ? (lane >> 4) : 0);
-    if (r >= r1) continue;
-    const int64_t orow = static_cast<int64_t>(grp.out_row0) + r;
-    const float rs = a_row_scale(p, grp, r);
-    const float* src = p.partial + orow * p.pcols + n;
-    const float4 g = splitk_sum4(src, slice, ks);
-    float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (EPI == EPI_SWIGLU) u = splitk_sum4(src + N, slice, ks);
-    float o[4];
-    o[0] = splitk_out<EPI>(p, sbase, n, 0, g.x, u.x, rs);
-    o[1] = splitk_out<EPI>(p, sbase, n, 1, g.y, u.y, rs);
-    o[2] = splitk_out<EPI>(p, sbase, n, 2, g.z, u.z, rs);
-    o[3] = splitk_out<EPI>(p, sbase, n, 3, g.w, u.w, rs);
-    if (p.out_f32) {
-      *reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * N + n) = make_float4(o[0], o[1], o[2], o[3]);
-    } else {
-      const uint2 packed = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
-      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + orow * N + n) = packed;
-    }
-  }
-}
-
-// Split-K finalize for larger groups: for every valid row of every group, sum
-// the partial slices in split order and apply the epilogue; one thread per
-// four output columns.  Exits at once when the GEMM ran without a split or
-// reduced its slices itself.  Launched under programmatic dependent launch:
-// it waits for the GEMM before reading.
+// Split-K finalize: for every valid row of every group, sum the partial slices
+// in split order and apply the epilogue; one thread per four output columns.
+// Exits at once when the GEMM ran without a split.  Launched under
+// programmatic dependent launch: it waits for the GEMM before reading.
 template <int EPI>
 __global__ void __launch_bounds__(256) splitk_finalize_kernel(TcParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int ks = *p.ksplit_out;
-  if (ks <= 1 || p.inkernel_reduce) return;
+  if (ks <= 1) return;
   const GroupEntry grp = group_at(p, blockIdx.z);
   const int r = blockIdx.y;
   if (r >= grp.rows || grp.expert < 0 || grp.expert >= p.num_slabs) return;

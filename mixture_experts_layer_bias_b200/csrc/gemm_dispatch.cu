@@ -10,9 +10,6 @@ namespace moe {
 
 using namespace gemm;
 
-// Groups of at most this many rows reduce split-K slices inside the GEMM.
-constexpr int64_t kInKernelReduceRows = 16;
-
 #ifdef MOE_B200_TEST_HOOKS
 // Failure-detection test hook, compiled only into the test build of the
 // library (libmoe_b200_testhooks.so): moe_test_stall_gemms(n) makes the next
@@ -54,11 +51,6 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t 
   p.pcols = a.epilogue == EPI_SWIGLU ? 2 * a.N : a.N;
   p.partial = a.partial;
   p.ksplit_out = a.ksplit_out;
-  p.tile_count = a.tile_count;
-  p.max_tiles = static_cast<int>(a.tile_count_len / kRegionsPerTile);
-  // decode-sized groups reduce their split-K slices inside the GEMM (no
-  // finalize launch); larger groups use the finalize kernel
-  p.inkernel_reduce = (a.max_group_rows <= kInKernelReduceRows && a.tile_count != nullptr && p.max_tiles > 0) ? 1 : 0;
   p.max_ksplit = 1;
   if (a.partial != nullptr && a.ksplit_out != nullptr && a.partial_bytes > 0) {
     // as many K slices as the partial buffer holds for every output row

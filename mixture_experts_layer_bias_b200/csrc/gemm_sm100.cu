@@ -66,9 +66,9 @@ constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
 constexpr int kEpiWarps = 8;  // two per TMEM lane quarter, each draining half of a tile's columns
 constexpr int kThreads = 64 + 32 * kEpiWarps;
-// E4M3 weights with bf16 activations (W8): four more warps decode each landed
+// E4M3 weights with bf16 activations (W8): eight more warps decode each landed
 // E4M3 weight tile into the bf16 B tile of its stage.
-constexpr int kConvWarps = 4;
+constexpr int kConvWarps = 8;
 constexpr int kThreadsW8 = kThreads + 32 * kConvWarps;
 constexpr int kLandStages = 3;             // landing buffers of E4M3 weight tiles
 constexpr int LAND_BYTES = 256 * 64;       // 256 weight rows x 64 E4M3 codes (one bf16 K step)
@@ -231,8 +231,7 @@ __device__ __forceinline__ void epilogue_store(const TcParams& p, const TileInfo
 // TMEM lane quarter, and half of the tile's columns -- SwiGLU: output columns
 // half*64 .. +63, i.e. gate chunks {2 half, 2 half + 1} and up chunks
 // {4 + 2 half, 5 + 2 half}, gate stored at column n and up at N + n; other
-// epilogues: columns half*128 .. +127.  A region is then complete in itself
-// (splitk_reduce_region).
+// epilogues: columns half*128 .. +127.
 template <int EPI>
 __device__ __forceinline__ void epilogue_partial(const TcParams& p, const TileInfo& ti, uint32_t tbase, int row,
                                                  bool valid, int split, int half) {
@@ -263,33 +262,36 @@ __device__ __forceinline__ void epilogue_partial(const TcParams& p, const TileIn
 
 // Four E4M3 codes (bytes of w, lowest first) -> four bf16 values (lo: codes
 // 0, 1; hi: codes 2, 3), exactly: E4M3 -> f16 is exact (every E4M3 value,
-// subnormals included, is a normal f16 or zero) and so is f16 -> bf16 for
-// values with at most four significant bits in the E4M3 range.
+// subnormals included, is a normal f16 or zero), f16 -> f32 is exact, and the
+// f32 -> bf16 rounding keeps the value (at most four significant bits, inside
+// bf16's exponent range).  The f16 -> bf16 step goes through f32 because the
+// packed f32 -> bf16x2 conversion is one instruction for two values.
 __device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  asm("{\n\t.reg .b16 c0, c1, a, b, c, d;\n\t.reg .b32 h0, h1;\n\t"
+  asm("{\n\t.reg .b16 c0, c1, a, b, c, d;\n\t.reg .b32 h0, h1;\n\t.reg .f32 fa, fb, fc, fd;\n\t"
       "mov.b32 {c0, c1}, %2;\n\t"
       "cvt.rn.f16x2.e4m3x2 h0, c0;\n\t"
       "cvt.rn.f16x2.e4m3x2 h1, c1;\n\t"
       "mov.b32 {a, b}, h0;\n\t"
-      "cvt.rn.bf16.f16 a, a;\n\t"
-      "cvt.rn.bf16.f16 b, b;\n\t"
-      "mov.b32 %0, {a, b};\n\t"
+      "cvt.f32.f16 fa, a;\n\t"
+      "cvt.f32.f16 fb, b;\n\t"
+      "cvt.rn.bf16x2.f32 %0, fb, fa;\n\t"
       "mov.b32 {c, d}, h1;\n\t"
-      "cvt.rn.bf16.f16 c, c;\n\t"
-      "cvt.rn.bf16.f16 d, d;\n\t"
-      "mov.b32 %1, {c, d};\n\t}"
+      "cvt.f32.f16 fc, c;\n\t"
+      "cvt.f32.f16 fd, d;\n\t"
+      "cvt.rn.bf16x2.f32 %1, fd, fc;\n\t}"
       : "=r"(lo), "=r"(hi)
       : "r"(w));
 }
 
-// W8: the 128 converter threads decode one landed 256 x 64 E4M3 tile (rows of
-// 64 bytes) into the stage's 256 x 128-byte bf16 B tile in the 128-byte
-// swizzled layout the MMA reads (16-byte chunk j of row r at chunk
-// j ^ (r & 7)).  Thread ct takes the 16-code pieces ct + 128 i.
+// W8: the converter threads (kConvWarps warps) decode one landed 256 x 64
+// E4M3 tile (rows of 64 bytes) into the stage's 256 x 128-byte bf16 B tile in
+// the 128-byte swizzled layout the MMA reads (16-byte chunk j of row r at
+// chunk j ^ (r & 7)).  Thread ct takes the 16-code pieces ct + 32 kConvWarps i.
 __device__ __forceinline__ void convert_tile_w8(const uint8_t* land, uint8_t* b16, int ct) {
+  constexpr int kConvThreads = 32 * kConvWarps;
 #pragma unroll 2
-  for (int i = 0; i < 8; ++i) {
-    const int piece = ct + 128 * i;  // 1024 pieces of 16 codes
+  for (int i = 0; i < 1024 / kConvThreads; ++i) {
+    const int piece = ct + kConvThreads * i;  // 1024 pieces of 16 codes
     const int r = piece >> 2, q4 = piece & 3;
     const uint4 v = *reinterpret_cast<const uint4*>(land + r * 64 + q4 * 16);
     uint32_t o[8];
@@ -387,8 +389,7 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
   const uint32_t tmem = s.tmem_base;
   const int nk = (p.K + BK - 1) / BK;
   const int tiles = s.tile_start[p.num_groups];
-  // in-kernel split-K reduction only while every tile has its arrival counters
-  const int ks = (!p.inkernel_reduce || tiles <= p.max_tiles) ? choose_ksplit(tiles, gridDim.x, nk, p.max_ksplit) : 1;
+  const int ks = choose_ksplit(tiles, gridDim.x, nk, p.max_ksplit);
   if (blockIdx.x == 0 && threadIdx.x == 0 && p.ksplit_out != nullptr) *p.ksplit_out = ks;
   const int total = tiles * ks;  // work units
   volatile int* abort_flag = &s.abort;
@@ -498,7 +499,7 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
     // B tile to be free, decode it, then let the MMA go (second arrival on the
     // stage's full barrier) and reuse the landing buffer for the K step
     // kLandStages ahead.  One thread waits on the barriers and issues the
-    // copies; the decision to go on or give up reaches all 128 threads through
+    // copies; the decision to go on or give up reaches all converter threads through
     // shared memory, so they leave together.
     const int ct = threadIdx.x - (2 + kEpiWarps) * 32;
     // the K-step sequence, walked twice: `cur` for decoding, `ahd` for issuing copies
@@ -623,23 +624,6 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
         epilogue_store<EPI>(p, ti, tbase, row, valid, lane, half, &tmOut, epi_smem + (warp - 2) * kEpiWarpBytes);
       tc_fence_before();
       mbar_arrive(&s.tempty[acc]);
-      if (ks > 1 && p.inkernel_reduce) {
-        // publish this slice of the warp's region, count it; the warp that
-        // completes the count reduces the region's slices
-        __threadfence();
-        __syncwarp();
-        int last = 0;
-        int* counter = p.tile_count + static_cast<int64_t>(u / ks) * kRegionsPerTile + q * 2 + half;
-        if (lane == 0) {
-          last = atomicAdd(counter, 1) == ks - 1;
-          if (last) {
-            *counter = 0;  // ready for the next launch
-            __threadfence();
-          }
-        }
-        if (__shfl_sync(0xFFFFFFFFu, last, 0))
-          splitk_reduce_region<EPI>(p, ti.grp, ti.m_idx * BM + q * 32, ti.n_idx, ks, half, lane);
-      }
     }
   }
 
@@ -670,7 +654,7 @@ cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUte
   e = launch_pdl(grouped_gemm_tc_kernel<EPI, F8, W8>, dim3(grid), dim3(W8 ? kThreadsW8 : kThreads), smem, stream, mA,
                  mA2, mB0, mB1, mOut, p, bma, stages);
   if (e != cudaSuccess) return e;
-  if ((e = cudaGetLastError()) != cudaSuccess || p.max_ksplit <= 1 || p.inkernel_reduce) return e;
+  if ((e = cudaGetLastError()) != cudaSuccess || p.max_ksplit <= 1) return e;
   dim3 fgrid((p.N + 1023) / 1024, static_cast<unsigned>(max_group_rows), p.num_groups);
   e = launch_pdl(splitk_finalize_kernel<EPI>, fgrid, dim3(256), 0, stream, p);
   if (e != cudaSuccess) return e;

@@ -35,11 +35,13 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream);
 // --- over-capacity re-routing ------------------------------------------------
 // Excess slots (row_of_slot >= E*C after a capacity-bounded permutation) move,
 // in (token, k) order, to the best-keyed candidate expert with room that the
-// token does not hold; changed[t] marks tokens with a moved slot.  One CTA.
-// ex_scratch: int32 [S*K].  moved_count (optional): device int, += moved slots.
+// token does not hold; changed[t] marks tokens with a moved slot.  A multi-CTA
+// pick kernel, then one CTA running the epochs.  pick_scratch: int32 [S*K],
+// 16-byte aligned; claim_scratch: int32 [S].
 cudaError_t launch_reroute_assign(int S, int E, int K, int capacity, int32_t* topk_idx, const float* cand_key,
-                                  const int32_t* counts, const int32_t* row_of_slot, int32_t* ex_scratch,
-                                  int32_t* changed, StatusBlock* status, cudaStream_t stream);
+                                  const int32_t* counts, const int32_t* row_of_slot, int32_t* pick_scratch,
+                                  int32_t* claim_scratch, int32_t* changed, StatusBlock* status,
+                                  cudaStream_t stream);
 // Gates of the tokens marked in changed[], recomputed over their final experts
 // from the gate sources (the same formulas as the routing kernels).
 cudaError_t launch_reroute_gates(int S, int E, int K, int score_fn, int renormalize, const float* score,
@@ -69,11 +71,6 @@ struct PermuteArgs {
   GroupEntry* g1;
   int num_shared;
 };
-// Tiny batches: routing (logits computed from x, E <= 32), the single-CTA
-// permutation with group tables, and the row gather (pa.x_perm, or none when
-// NULL) in one kernel.  route_permute_fusable says which batches qualify.
-bool route_permute_fusable(int S, int E, int K);
-cudaError_t launch_route_permute_small(const RouteArgs& ra, const PermuteArgs& pa, cudaStream_t stream);
 int permute_num_chunks(int S, int K);
 int permute_tokens_per_chunk(int K);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream);
@@ -113,8 +110,6 @@ struct GemmArgs {
   float* partial;           // split-K partial sums (nullptr = no split-K)
   int64_t partial_bytes;    // size of `partial`
   int* ksplit_out;          // device int: the split the GEMM chose (read by the finalize kernel)
-  int* tile_count;          // split-K arrival counters (zero between launches; nullptr = none)
-  int64_t tile_count_len;   // number of counters
   int fp8;                  // 1: A and B are E4M3 (kind::f8f6f4); A rows scaled by row_scale
   int w8;                   // 1: B (weights) E4M3, A bf16: the GEMM decodes each weight tile to bf16
   const float* row_scale;        // [a rows] per-row scale of A (fp8 only)

@@ -32,8 +32,6 @@ namespace {
 constexpr int kChunkSlots = 1024;  // slots per CTA (whole tokens)
 constexpr int kSmallWarps = 32;
 constexpr int kSmallSlots = 4096;  // the single-CTA permutation handles S*K up to this
-constexpr int kRouteGroupWarps = 8;  // warps routing one token in the fused small-batch kernel
-constexpr int kFusedMaxTokens = 16;  // batches the fused route-permute-gather kernel takes
 constexpr int kPermWarps = 8;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
@@ -250,14 +248,11 @@ __device__ __forceinline__ void write_groups(int S, int E, int K, int capacity, 
 
 // Small batches (decode): histogram, scans, stable ranks, row maps and the
 // group tables in one CTA -- the same counting sort as the chunked path with
-// the whole slot range as one chunk split over 32 warps.  `idx` holds the
-// slots' expert ids (global memory, or shared memory in the fused kernel);
-// ros_mirror (optional, shared memory) receives a copy of row_of_slot.
+// the whole slot range as one chunk split over 32 warps.
 // sm: kSmallWarps * E + 3 * E + 1 ints of shared memory.
 __device__ void permute_small_body(int S, int E, int K, int capacity, int num_shared, const int32_t* idx,
                                    int32_t* counts, int32_t* offsets, int32_t* row_of_slot, int32_t* token_of_row,
-                                   int64_t num_rows, GroupEntry* g1, StatusBlock* status, int32_t* sm,
-                                   int32_t* ros_mirror) {
+                                   int64_t num_rows, GroupEntry* g1, StatusBlock* status, int32_t* sm) {
   int32_t* whist = sm;                      // [32][E]
   int32_t* cnt = sm + kSmallWarps * E;      // [E]
   int32_t* ovf = cnt + E;                   // [E]
@@ -331,7 +326,6 @@ __device__ void permute_small_body(int S, int E, int K, int capacity, int num_sh
     if (e >= 0 && lane == __ffs(peers) - 1) whist[warp * E + e] += __popc(peers);
     if (act) {
       row_of_slot[sl] = row;
-      if (ros_mirror != nullptr) ros_mirror[sl] = row;
       if (row >= 0) token_of_row[row] = sl / K;
     }
     __syncwarp();
@@ -348,86 +342,7 @@ __global__ void __launch_bounds__(kSmallWarps * 32)
   pdl_wait();
   pdl_trigger();
   permute_small_body(S, E, K, capacity, num_shared, topk_idx, counts, offsets, row_of_slot, token_of_row, num_rows,
-                     g1, status, sm, nullptr);
-}
-
-// Routing, permutation and row gather of a tiny batch (S <= kFusedMaxTokens,
-// E <= 32, logits computed here) in one CTA of 32 warps, so a decode step
-// spends one launch where the separate calls spend three.  Routing: groups of
-// 8 warps route one token each (4 tokens at a time), splitting d exactly as
-// the per-token routing kernel does (same partial sums in the same order), and
-// warp 0 of the group selects; the expert ids also go to shared memory.  Then
-// the whole CTA runs the single-CTA permutation on them, and finally copies
-// every token row to its K rows (x_perm NULL: maps only).
-template <typename T, int EMAX>
-__global__ void __launch_bounds__(kSmallWarps * 32, 1)
-    route_permute_small_kernel(int S, int d, const T* __restrict__ x, const T* __restrict__ w_router,
-                               const float* __restrict__ router_bias, route_detail::SelectParams sp, int capacity,
-                               int num_shared, int32_t* counts, int32_t* offsets, int32_t* row_of_slot,
-                               int32_t* token_of_row, int64_t num_rows, GroupEntry* g1, T* x_perm) {
-  extern __shared__ int32_t sm[];
-  __shared__ float part[4][kRouteGroupWarps][EMAX];
-  const int E = sp.E, K = sp.K;
-  int32_t* idx_s = sm + kSmallWarps * E + 3 * E + 1;  // [S*K]
-  int32_t* ros_s = idx_s + S * K;                      // [S*K]
-  pdl_wait();
-  pdl_trigger();
-  sp.idx_mirror = idx_s;
-  const int grp = threadIdx.x / (kRouteGroupWarps * 32);
-  const int gt = threadIdx.x % (kRouteGroupWarps * 32);
-  const int gwarp = gt >> 5, lane = lane_id();
-  constexpr int V = Vec16<T>::N;
-  const int nvec = d / V;
-  for (int t0 = 0; t0 < S; t0 += 4) {
-    const int t = t0 + grp;
-    if (t < S) {
-      float acc[EMAX];
-#pragma unroll
-      for (int e = 0; e < EMAX; ++e) acc[e] = 0.0f;
-      const T* xr = x + static_cast<int64_t>(t) * d;
-      for (int v = gt; v < nvec; v += kRouteGroupWarps * 32) {
-        float xf[V];
-        unpack16<T>(ldg16(xr + v * V), xf);
-#pragma unroll
-        for (int e = 0; e < EMAX; ++e) {
-          if (e < E) {
-            float wf[V];
-            unpack16<T>(ldg16(w_router + static_cast<int64_t>(e) * d + v * V), wf);
-#pragma unroll
-            for (int j = 0; j < V; ++j) acc[e] = fmaf(xf[j], wf[j], acc[e]);
-          }
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < EMAX; ++e) {
-        const float s = route_detail::warp_sum(acc[e]);
-        if (lane == 0) part[grp][gwarp][e] = s;
-      }
-    }
-    __syncthreads();
-    if (t < S && gwarp == 0) {
-      float l[1] = {0.0f};
-      if (lane < E && lane < EMAX) {
-        float s = 0.0f;
-        for (int w = 0; w < kRouteGroupWarps; ++w) s += part[grp][w][lane];
-        l[0] = router_bias != nullptr ? __fadd_rn(s, __ldg(router_bias + lane)) : s;
-      }
-      route_detail::select_topk<1>(l, sp, t);
-    }
-    __syncthreads();
-  }
-  permute_small_body(S, E, K, capacity, num_shared, idx_s, counts, offsets, row_of_slot, token_of_row, num_rows, g1,
-                     sp.status, sm, ros_s);
-  __syncthreads();
-  if (x_perm == nullptr) return;
-  for (int i = threadIdx.x; i < S * nvec; i += blockDim.x) {
-    const int t = i / nvec, v = i - t * nvec;
-    const uint4 val = ldg16(x + static_cast<int64_t>(t) * d + v * V);
-    for (int k = 0; k < K; ++k) {
-      const int row = ros_s[t * K + k];
-      if (row >= 0) stg16(x_perm + static_cast<int64_t>(row) * d + v * V, val);
-    }
-  }
+                     g1, status, sm);
 }
 
 // Row gather for small batches: one CTA per token, its threads split the row.
@@ -503,38 +418,6 @@ cudaError_t launch_debug_check_permutation(int S, int E, int K, int capacity, co
   (void)num_rows; (void)status; (void)stream;
   return cudaSuccess;
 #endif
-}
-
-bool route_permute_fusable(int S, int E, int K) {
-  return S >= 1 && S <= kFusedMaxTokens && E <= 32 && static_cast<int64_t>(S) * K <= kSmallSlots;
-}
-
-cudaError_t launch_route_permute_small(const RouteArgs& ra, const PermuteArgs& pa, cudaStream_t stream) {
-  if (!route_permute_fusable(ra.S, ra.E, ra.K) || ra.logits != nullptr || ra.x == nullptr) return cudaErrorInvalidValue;
-  route_detail::SelectParams sp{ra.E,        ra.K,        ra.score_fn, ra.renormalize, ra.num_groups, ra.topk_groups,
-                                ra.tau,      ra.sel_bias, ra.topk_idx, ra.topk_w,      ra.status,     nullptr,
-                                nullptr,     nullptr};
-  const size_t smem = sizeof(int32_t) * (kSmallWarps * ra.E + 3 * ra.E + 1 + 2 * ra.S * ra.K);
-  cudaError_t err;
-#define MOE_FUSED(T, EM)                                                                                          \
-  err = launch_pdl(route_permute_small_kernel<T, EM>, dim3(1), dim3(kSmallWarps * 32), smem, stream, ra.S, ra.d,      \
-                   static_cast<const T*>(ra.x), static_cast<const T*>(ra.w_router), ra.router_bias, sp, pa.capacity, \
-                   pa.num_shared, pa.counts, pa.offsets, pa.row_of_slot, pa.token_of_row, pa.num_rows, pa.g1,        \
-                   static_cast<T*>(pa.x_perm))
-  if (ra.act_dtype == MOE_BF16) {
-    if (ra.E <= 8)
-      MOE_FUSED(__nv_bfloat16, 8);
-    else
-      MOE_FUSED(__nv_bfloat16, 32);
-  } else {
-    if (ra.E <= 8)
-      MOE_FUSED(float, 8);
-    else
-      MOE_FUSED(float, 32);
-  }
-#undef MOE_FUSED
-  if (err != cudaSuccess) return err;
-  return cudaGetLastError();
 }
 
 int permute_tokens_per_chunk(int K) { return K >= kChunkSlots ? 1 : kChunkSlots / K; }

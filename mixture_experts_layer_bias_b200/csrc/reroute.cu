@@ -9,17 +9,22 @@
 // room and that the token does not already hold (ties to the lower index);
 // an excess slot with no such expert keeps its expert and its overflow row.
 //
-// The visit order makes this a serial assignment.  One CTA runs it in rounds
-// over chunks of up to 1024 excess slots: every slot picks its expert against
-// the room left at the start of the round (one thread per slot over the
-// token's whole key row; the later slots of a token with several excess slots
-// in the chunk are then fixed up in k order, each excluding the earlier
-// picks), the picks are ranked per expert in slot order, and the longest
-// prefix of slots whose pick still fits is committed.  A pick made against the round's room
-// is the serial pick as long as every earlier slot's pick fit (room only
-// shrinks, and the picked expert is still available), so the committed prefix
-// equals the serial result; the first slot that does not fit had filled its
-// expert, so a chunk is cut short at most once per expert.
+// The visit order makes this a serial assignment, but its picks only change
+// when an expert runs out of room, and that happens at most once per expert.
+// So it runs in epochs:
+//  1. every excess slot picks against the room at the start (all SMs, one
+//     thread per token taking its excess slots in k order, each excluding the
+//     token's experts and its earlier picks);
+//  2. one CTA then repeats: find the first slot whose pick overflows its
+//     expert's room (per-expert counts of the uncommitted picks by token
+//     segment, then the exact slot inside one segment); commit every pick
+//     before it (these are the serial picks: no expert they chose was full
+//     when they were made); the experts left without room drop out, and only
+//     the uncommitted slots that picked one of them pick again (with the
+//     later slots of their token that now clash).  Every epoch but the last
+//     fills at least one expert, so there are at most E + 1.
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -27,197 +32,426 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 1024;
-constexpr int kWarps = kThreads / 32;
 constexpr int kMaxE = 256;
+constexpr int kMaskWords = kMaxE / 32;
+constexpr int kPickThreads = 256;
+constexpr int kThreads = 512;
+constexpr int kSegs = kThreads / 32;  // token segments, one per warp of the commit CTA
+constexpr int kScanSlots = 512;       // slots the scanning warp loads at once
+constexpr int kNone = -1;             // excess slot without a candidate
+constexpr int kKept = -2;             // slot within its expert's capacity
 
-// The best candidate expert of excess slot s with room left (room[e] > 0),
-// a finite key, not held by the slot's token (its current K experts) and not
-// in extra[0..n_extra): highest key, ties to the lower index; -1 if none.
-// The key row is read with 16-byte loads issued before the comparisons.
-__device__ int best_pick(int s, int E, int K, const int32_t* topk_idx, const float* cand_key, const int* room,
-                         const int* extra, int n_extra) {
+__device__ __forceinline__ bool bit_of(const uint32_t* m, int e) { return (m[e >> 5] >> (e & 31)) & 1u; }
+
+// Word i of a per-thread expert mask, and setting bit e of it, by unrolled
+// selects, so the mask stays in registers whatever i or e are.
+__device__ __forceinline__ uint32_t word_of(const uint32_t (&m)[kMaskWords], int i) {
+  uint32_t r = 0;
+#pragma unroll
+  for (int j = 0; j < kMaskWords; ++j) r = (i == j) ? m[j] : r;
+  return r;
+}
+__device__ __forceinline__ void set_bit(uint32_t (&m)[kMaskWords], int e) {
+#pragma unroll
+  for (int j = 0; j < kMaskWords; ++j)
+    if ((e >> 5) == j) m[j] |= 1u << (e & 31);
+}
+__device__ __forceinline__ bool has_bit(const uint32_t (&m)[kMaskWords], int e) {
+  return (word_of(m, e >> 5) >> (e & 31)) & 1u;
+}
+
+// The best candidate of token t: highest key among experts in `avail`, not in
+// `held`, with a key above -inf; ties to the lower index; kNone if none.  The
+// key row is read 64 experts at a time with sixteen 16-byte loads in flight.
+__device__ int best_candidate(const float* __restrict__ row, int E, const uint32_t* avail,
+                              const uint32_t (&held)[kMaskWords]) {
   const float kNegInf = __int_as_float(0xff800000);
-  const int t = s / K;
-  uint32_t held[kMaxE / 32];
-#pragma unroll
-  for (int i = 0; i < kMaxE / 32; ++i) held[i] = 0;
-  for (int k = 0; k < K; ++k) {
-    const int e = topk_idx[static_cast<int64_t>(t) * K + k];
-    if (e >= 0 && e < E) held[e >> 5] |= 1u << (e & 31);
-  }
-  for (int i = 0; i < n_extra; ++i) held[extra[i] >> 5] |= 1u << (extra[i] & 31);
-  const float* row = cand_key + static_cast<int64_t>(t) * E;
   float bv = kNegInf;
-  int be = -1;
-  // E is a multiple of 4 here (whole 16-byte loads) or handled one by one
+  int be = kNone;
   const int e4 = (E % 4 == 0) ? E : 0;
-  for (int e0 = 0; e0 < e4; e0 += 32) {
-    float4 v[8];
+  for (int e0 = 0; e0 < e4; e0 += 64) {
+    float4 v[16];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < 16; ++j)
       v[j] = (e0 + 4 * j < e4) ? __ldg(reinterpret_cast<const float4*>(row + e0 + 4 * j))
                                : make_float4(kNegInf, kNegInf, kNegInf, kNegInf);
+    const int w = e0 >> 5;
+    const uint64_t av = static_cast<uint64_t>(avail[w]) | (e0 + 32 < E ? static_cast<uint64_t>(avail[w + 1]) << 32 : 0);
+    const uint64_t hb = static_cast<uint64_t>(word_of(held, w)) | (static_cast<uint64_t>(word_of(held, w + 1)) << 32);
+    const uint64_t ok = av & ~hb;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < 16; ++j) {
       const float kv[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int e = e0 + 4 * j + c;
-        if (e >= E || !(kv[c] > kNegInf) || ((held[e >> 5] >> (e & 31)) & 1u) || room[e] <= 0) continue;
-        if (kv[c] > bv) {  // ascending e: a tie keeps the lower index
-          bv = kv[c];
-          be = e;
-        }
+        if (e >= E || !(kv[c] > bv) || !((ok >> (4 * j + c)) & 1u)) continue;
+        bv = kv[c];  // strictly greater in ascending e: a tie keeps the lower index
+        be = e;
       }
     }
   }
   for (int e = e4; e < E; ++e) {
     const float kv = __ldg(row + e);
-    if (!(kv > kNegInf) || ((held[e >> 5] >> (e & 31)) & 1u) || room[e] <= 0) continue;
-    if (kv > bv) {
-      bv = kv;
-      be = e;
-    }
+    if (!(kv > bv) || has_bit(held, e) || !bit_of(avail, e)) continue;
+    bv = kv;
+    be = e;
   }
   return be;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-    reroute_assign_kernel(int S, int E, int K, int C, int32_t* __restrict__ topk_idx,
-                          const float* __restrict__ cand_key, const int32_t* __restrict__ counts,
-                          const int32_t* __restrict__ row_of_slot, int32_t* __restrict__ ex,
-                          int32_t* __restrict__ changed, StatusBlock* status) {
-  __shared__ int room[kMaxE];
-  __shared__ int wcnt[kWarps][kMaxE];
-  __shared__ int ch[kThreads];
-  __shared__ int sx[kThreads];  // the round's excess slot ids
-  __shared__ int wpre[kWarps];
-  __shared__ int s_total, s_chunk, s_first_bad, s_moved;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const unsigned lt_mask = (1u << lane) - 1u;
-  const int64_t nslots = static_cast<int64_t>(S) * K;
-  const int64_t ovf_row0 = static_cast<int64_t>(E) * C;
-  const float kNegInf = __int_as_float(0xff800000);
+// Bit e set for every expert the token's K slots hold (vec: 16-byte loads,
+// K a multiple of 4 and the row 16-byte aligned).
+__device__ __forceinline__ void held_of(const int32_t* __restrict__ idx_row, int K, int E, bool vec,
+                                        uint32_t (&held)[kMaskWords]) {
+#pragma unroll
+  for (int i = 0; i < kMaskWords; ++i) held[i] = 0;
+  auto add = [&](int e) {
+    if (e >= 0 && e < E) set_bit(held, e);
+  };
+  if (vec) {
+    int4 v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (4 * j < K) v[j] = reinterpret_cast<const int4*>(idx_row)[j];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (4 * j < K) {
+        add(v[j].x); add(v[j].y); add(v[j].z); add(v[j].w);
+      }
+  } else {
+    for (int k = 0; k < K; ++k) add(idx_row[k]);
+  }
+}
 
+// Bit k set for every slot of the token in the overflow region (row >=
+// ovf_row0); vec as for held_of.
+__device__ __forceinline__ uint32_t excess_mask(const int32_t* __restrict__ ros_row, int K, int64_t ovf_row0,
+                                                bool vec) {
+  uint32_t m = 0;
+  if (vec) {
+    int4 v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (4 * j < K) v[j] = reinterpret_cast<const int4*>(ros_row)[j];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (4 * j < K) {
+        m |= (v[j].x >= ovf_row0 ? 1u : 0u) << (4 * j);
+        m |= (v[j].y >= ovf_row0 ? 1u : 0u) << (4 * j + 1);
+        m |= (v[j].z >= ovf_row0 ? 1u : 0u) << (4 * j + 2);
+        m |= (v[j].w >= ovf_row0 ? 1u : 0u) << (4 * j + 3);
+      }
+  } else {
+    for (int k = 0; k < K; ++k) m |= (ros_row[k] >= ovf_row0 ? 1u : 0u) << k;
+  }
+  return m;
+}
+
+// Calls f(s, pick[s]) for every slot s in [lo, hi), reading the pick buffer
+// in 16-byte pieces (four slots; the buffer is 16-byte aligned), four pieces
+// in flight per thread: thread `idx` of `nthreads` takes pieces idx,
+// idx + nthreads, ...
+template <typename F>
+__device__ __forceinline__ void for_picks(const int32_t* __restrict__ pick, int64_t lo, int64_t hi, int idx,
+                                          int nthreads, F&& f) {
+  constexpr int U = 4;
+  if (lo >= hi) return;
+  const int64_t q0 = lo >> 2, q1 = (hi + 3) >> 2;
+  const int4* p4 = reinterpret_cast<const int4*>(pick);
+  for (int64_t qb = q0 + idx; qb < q1; qb += U * static_cast<int64_t>(nthreads)) {
+    int4 v[U];
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      const int64_t q = qb + j * static_cast<int64_t>(nthreads);
+      v[j] = q < q1 ? p4[q] : make_int4(kKept, kKept, kKept, kKept);
+    }
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      const int64_t s0 = (qb + j * static_cast<int64_t>(nthreads)) * 4;
+      const int pv[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if (s0 + c >= lo && s0 + c < hi) f(s0 + c, pv[c]);
+    }
+  }
+}
+
+// Step 1: the picks of every excess slot against the starting room.
+// pick[s] = expert, kNone, or kKept for slots within capacity.
+__global__ void __launch_bounds__(kPickThreads)
+    reroute_pick_kernel(int S, int E, int K, int C, const int32_t* __restrict__ topk_idx,
+                        const float* __restrict__ cand_key, const int32_t* __restrict__ counts,
+                        const int32_t* __restrict__ row_of_slot, int32_t* __restrict__ pick,
+                        int32_t* __restrict__ changed, int32_t* __restrict__ claim, bool vec) {
+  __shared__ uint32_t avail[kMaskWords];
+  if (threadIdx.x < kMaskWords) avail[threadIdx.x] = 0;
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    if (counts[e] < C) atomicOr(&avail[e >> 5], 1u << (e & 31));
+  __syncthreads();
+  const int64_t ovf_row0 = static_cast<int64_t>(E) * C;
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < S; t += gridDim.x * blockDim.x) {
+    changed[t] = 0;
+    claim[t] = 0;
+    const int64_t s0 = static_cast<int64_t>(t) * K;
+    const uint32_t ex = excess_mask(row_of_slot + s0, K, ovf_row0, vec);
+    if (ex == 0) {
+      for (int k = 0; k < K; ++k) pick[s0 + k] = kKept;
+      continue;
+    }
+    uint32_t held[kMaskWords];
+    held_of(topk_idx + s0, K, E, vec, held);
+    for (int k = 0; k < K; ++k) {
+      int p = kKept;
+      if ((ex >> k) & 1u) {
+        p = best_candidate(cand_key + static_cast<int64_t>(t) * E, E, avail, held);
+        if (p >= 0) set_bit(held, p);
+      }
+      pick[s0 + k] = p;
+    }
+  }
+}
+
+// Step 2: the epochs, on one CTA.
+struct CommitSmem {
+  int cnt[kSegs][kMaxE];  // uncommitted picks of each expert in each token segment
+  int sub[kSegs][kMaxE];  // the same within the 32 sub-ranges of one segment
+  int room[kMaxE];
+  int seg_e[kMaxE];       // segment holding expert e's first overflowing pick (kSegs: none)
+  int need_e[kMaxE];      // e's uncommitted picks there before it
+  int sub_e[kMaxE];       // sub-range of that pick, and the picks before it there
+  int need2_e[kMaxE];
+  int run[kMaxE];
+  uint32_t avail[kMaskWords];
+  uint32_t full[kMaskWords];  // experts that ran out of room in this epoch
+  int min_seg, min_sub;
+  long long first_bad;
+  int moved;
+};
+
+// The uncommitted excess slots of token t from slot `first` on pick again, in
+// k order: a slot whose pick ran out of room (in `full`), or that now clashes
+// with an earlier slot's new pick, takes the best candidate among the experts
+// still available; the segment counts follow every change.
+__device__ __noinline__ void repick_token(int t, int64_t first, int E, int K, bool vec, int seg,
+                                          const int32_t* __restrict__ topk_idx, const float* __restrict__ cand_key,
+                                          int32_t* __restrict__ pick, CommitSmem& sm) {
+  const int64_t s0 = static_cast<int64_t>(t) * K;
+  const int k0 = static_cast<int>((first > s0 ? first : s0) - s0);
+  int pk[32];  // the token's picks, loaded together with its experts
+#pragma unroll
+  for (int k = 0; k < 32; ++k)
+    if (k < K) pk[k] = pick[s0 + k];
+  uint32_t held[kMaskWords];
+  held_of(topk_idx + s0, K, E, vec, held);  // the token's committed picks are in topk_idx already
+  for (int k = k0; k < K; ++k) {
+    int p = pk[k];
+    if (p == kKept) continue;
+    if (p >= 0 && (bit_of(sm.full, p) || has_bit(held, p))) {
+      const int q = best_candidate(cand_key + static_cast<int64_t>(t) * E, E, sm.avail, held);
+      atomicSub(&sm.cnt[seg][p], 1);
+      if (q >= 0) atomicAdd(&sm.cnt[seg][q], 1);
+      pick[s0 + k] = q;
+      p = q;
+    }
+    if (p >= 0) set_bit(held, p);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    reroute_commit_kernel(int S, int E, int K, int C, int32_t* __restrict__ topk_idx,
+                          const float* __restrict__ cand_key, const int32_t* __restrict__ counts,
+                          int32_t* __restrict__ pick, int32_t* __restrict__ changed, int32_t* __restrict__ claim,
+                          bool vec, StatusBlock* status) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  CommitSmem& sm = *reinterpret_cast<CommitSmem*>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t nslots = static_cast<int64_t>(S) * K;
+  const int seg_len = (S + kSegs - 1) / kSegs;  // tokens per segment
+  auto seg_of = [&](int64_t s) { return static_cast<int>((s / K) / seg_len); };
+  auto seg_begin = [&](int w) { return static_cast<int64_t>(min(S, w * seg_len)) * K; };
+
+  for (int i = tid; i < kSegs * kMaxE; i += kThreads) (&sm.cnt[0][0])[i] = 0;
+  if (tid < kMaskWords) sm.avail[tid] = 0;
+  if (tid == 0) sm.moved = 0;
+  __syncthreads();
   for (int e = tid; e < E; e += kThreads) {
     const int c = counts[e];
-    room[e] = C - (c < C ? (c > 0 ? c : 0) : C);
+    sm.room[e] = C - (c < C ? (c > 0 ? c : 0) : C);
+    if (sm.room[e] > 0) atomicOr(&sm.avail[e >> 5], 1u << (e & 31));
   }
-  for (int t = tid; t < S; t += kThreads) changed[t] = 0;
-  if (tid == 0) {
-    s_total = 0;
-    s_moved = 0;
-  }
+  // each warp counts the picks of its own segment
+  for_picks(pick, seg_begin(warp), seg_begin(warp + 1), lane, 32, [&](int64_t, int p) {
+    if (p >= 0) atomicAdd(&sm.cnt[warp][p], 1);
+  });
   __syncthreads();
 
-  // 1. the excess slots (overflow rows of the permutation), in slot order;
-  //    each thread looks at kPer consecutive slots per pass
-  constexpr int kPer = 8;
-  for (int64_t base = 0; base < nslots; base += static_cast<int64_t>(kThreads) * kPer) {
-    const int64_t s0 = base + static_cast<int64_t>(tid) * kPer;
-    unsigned bits = 0;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j)
-      if (s0 + j < nslots && row_of_slot[s0 + j] >= ovf_row0) bits |= 1u << j;
-    const int n = __popc(bits);
-    int incl = n;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-      if (lane >= off) incl += o;
+  int64_t start = 0;  // first uncommitted slot
+  int moved = 0;
+  bool ok = true;
+  for (int epoch = 0; epoch <= E + 1; ++epoch) {
+    // 1. for each available expert, the segment of its first overflowing pick
+    if (tid == 0) {
+      sm.min_seg = kSegs;
+      sm.min_sub = kSegs;
+      sm.first_bad = nslots;
     }
-    if (lane == 31) wpre[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-      const int v = wpre[lane];
-      int winc = v;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int o = __shfl_up_sync(0xFFFFFFFFu, winc, off);
-        if (lane >= off) winc += o;
-      }
-      wpre[lane] = winc - v;
-      if (lane == 31) s_chunk = winc;
-    }
-    __syncthreads();
-    int pos = s_total + wpre[warp] + incl - n;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j)
-      if (bits & (1u << j)) ex[pos++] = static_cast<int32_t>(s0 + j);
-    __syncthreads();
-    if (tid == 0) s_total += s_chunk;
-    __syncthreads();
-  }
-  const int n_ex = s_total;
-
-  // 2. rounds over chunks of excess slots
-  int base = 0;
-  while (base < n_ex) {
-    const int m = min(kThreads, n_ex - base);
-    ch[tid] = -1;
-    sx[tid] = tid < m ? ex[base + tid] : 0;
-    for (int i = tid; i < kWarps * kMaxE; i += kThreads) (&wcnt[0][0])[i] = 0;
-    if (tid == 0) s_first_bad = m;
-    __syncthreads();
-    {
-      // one thread per slot: the best candidate with room that the token does
-      // not hold, over the token's whole key row (16-byte loads, all issued
-      // together); then the slots of a token that has several excess slots
-      // in this chunk are fixed up in k order, each excluding the earlier
-      // ones' picks
-      if (tid < m) ch[tid] = best_pick(sx[tid], E, K, topk_idx, cand_key, room, nullptr, 0);
-      __syncthreads();
-      if (tid < m && (tid == 0 || sx[tid - 1] / K != sx[tid] / K) && tid + 1 < m && sx[tid + 1] / K == sx[tid] / K) {
-        int taken[32];
-        int nt = 0;
-        if (ch[tid] >= 0) taken[nt++] = ch[tid];
-        for (int j = tid + 1; j < m && sx[j] / K == sx[tid] / K; ++j) {
-          bool clash = false;
-          for (int i = 0; i < nt; ++i) clash |= ch[j] == taken[i];
-          if (clash) ch[j] = best_pick(sx[j], E, K, topk_idx, cand_key, room, taken, nt);
-          if (ch[j] >= 0 && nt < 32) taken[nt++] = ch[j];
+    for (int e = tid; e < E; e += kThreads) {
+      int seg = kSegs, acc = 0, need = 0;
+      if (bit_of(sm.avail, e)) {
+        for (int w = 0; w < kSegs; ++w) {
+          const int c = sm.cnt[w][e];
+          if (acc + c > sm.room[e]) {
+            seg = w;
+            need = sm.room[e] - acc;
+            break;
+          }
+          acc += c;
         }
       }
+      sm.seg_e[e] = seg;
+      sm.need_e[e] = need;
     }
     __syncthreads();
-    // rank of each pick among the earlier picks of the same expert in this chunk
-    const int c = tid < m ? ch[tid] : -1;
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, c);
-    const int wrank = __popc(peers & lt_mask);
-    if (c >= 0 && wrank == 0) wcnt[warp][c] = __popc(peers);
+    for (int e = tid; e < E; e += kThreads)
+      if (sm.seg_e[e] < kSegs) atomicMin(&sm.min_seg, sm.seg_e[e]);
+    for (int i = tid; i < kSegs * kMaxE; i += kThreads) (&sm.sub[0][0])[i] = 0;
     __syncthreads();
-    bool bad = false;
-    if (c >= 0) {
-      int rank = wrank;
-      for (int w = 0; w < warp; ++w) rank += wcnt[w][c];
-      bad = rank >= room[c];
+    const int ms = sm.min_seg;
+    int64_t P = nslots;
+    if (ms < kSegs) {
+      // 2. the exact slot: sub-range counts of the candidate experts' picks
+      //    within segment ms, then a scan of one sub-range in slot order
+      const int64_t a = max(seg_begin(ms), start), b = seg_begin(ms + 1);
+      const int64_t span = (b - a + kSegs - 1) / kSegs;
+      const int64_t lo = min(b, a + warp * span), hi = min(b, lo + span);
+      for_picks(pick, lo, hi, lane, 32, [&](int64_t, int p) {
+        if (p >= 0 && sm.seg_e[p] == ms) atomicAdd(&sm.sub[warp][p], 1);
+      });
+      __syncthreads();
+      for (int e = tid; e < E; e += kThreads) {
+        int w_hit = kSegs, acc = 0, need2 = 0;
+        if (sm.seg_e[e] == ms) {
+          for (int w = 0; w < kSegs; ++w) {
+            const int c = sm.sub[w][e];
+            if (acc + c > sm.need_e[e]) {
+              w_hit = w;
+              need2 = sm.need_e[e] - acc;
+              break;
+            }
+            acc += c;
+          }
+          atomicMin(&sm.min_sub, w_hit);
+        }
+        sm.sub_e[e] = w_hit;
+        sm.need2_e[e] = need2;
+        sm.run[e] = 0;
+      }
+      __syncthreads();
+      const int wm = sm.min_sub;
+      if (warp == wm) {
+        // the sub-range is loaded kScanSlots slots at a time (all loads in
+        // flight together), each piece scanned 32 slots at a time in slot order
+        const int64_t slo = min(b, a + wm * span), shi = min(b, slo + span);
+        const unsigned lt = (1u << lane) - 1u;
+        bool found = false;
+        for (int64_t c0 = slo; c0 < shi && !found; c0 += kScanSlots) {
+          int pv[kScanSlots / 32];
+#pragma unroll
+          for (int j = 0; j < kScanSlots / 32; ++j) {
+            const int64_t s = c0 + 32 * j + lane;
+            pv[j] = s < shi ? pick[s] : kKept;
+          }
+#pragma unroll
+          for (int j = 0; j < kScanSlots / 32; ++j) {
+            const int p = pv[j];
+            const bool cand = p >= 0 && sm.seg_e[p] == ms && sm.sub_e[p] == wm;
+            const unsigned peers = __match_any_sync(0xFFFFFFFFu, p);
+            const int rank = __popc(peers & lt);
+            const bool hit = cand && sm.run[p] + rank == sm.need2_e[p];
+            const unsigned hits = __ballot_sync(0xFFFFFFFFu, hit);
+            if (hits != 0) {
+              if (lane == 0) sm.first_bad = c0 + 32 * j + __ffs(hits) - 1;
+              found = true;
+              break;
+            }
+            if (cand && rank == 0) sm.run[p] += __popc(peers);
+            __syncwarp();
+          }
+        }
+      }
+      __syncthreads();
+      P = sm.first_bad;
+      if (P >= nslots) {  // the counts promised an overflow in this segment: cannot happen
+        ok = false;
+        break;
+      }
     }
-    if (bad) atomicMin(&s_first_bad, tid);
-    __syncthreads();
-    const int p = s_first_bad;  // >= 1: the chunk's first pick always fits
-    if (tid < p && c >= 0) {
-      const int s = ex[base + tid];
-      topk_idx[s] = c;
-      atomicSub(&room[c], 1);
+    // 3. commit the picks of [start, P)
+    for_picks(pick, start, P, tid, kThreads, [&](int64_t s, int p) {
+      if (p < 0) return;
+      topk_idx[s] = p;
+      atomicSub(&sm.room[p], 1);
+      atomicSub(&sm.cnt[seg_of(s)][p], 1);
       changed[s / K] = 1;
-      atomicAdd(&s_moved, 1);
-    }
+      ++moved;
+    });
+    if (tid < kMaskWords) sm.full[tid] = 0;
     __syncthreads();
-    base += p;
+    start = P;
+    if (P >= nslots) break;
+    // 4. experts left without room drop out
+    for (int e = tid; e < E; e += kThreads)
+      if (bit_of(sm.avail, e) && sm.room[e] <= 0) atomicOr(&sm.full[e >> 5], 1u << (e & 31));
+    __syncthreads();
+    if (tid < kMaskWords) sm.avail[tid] &= ~sm.full[tid];
+    __syncthreads();
+    // 5. the tokens with an uncommitted slot that picked a full expert pick
+    //    again; the first thread to see such a slot claims the token for this
+    //    epoch and re-picks it
+    for_picks(pick, P, nslots, tid, kThreads, [&](int64_t s, int p) {
+      if (p < 0 || !bit_of(sm.full, p)) return;
+      const int t = static_cast<int>(s / K);
+      if (atomicMax(&claim[t], epoch + 1) < epoch + 1)
+        repick_token(t, P, E, K, vec, seg_of(s), topk_idx, cand_key, pick, sm);
+    });
+    __syncthreads();
   }
-  if (tid == 0 && status != nullptr && s_moved > 0) atomicAdd(&status->counters[MOE_CNT_REROUTED], s_moved);
+  if (!ok || start < nslots) report(status, MOE_STATUS_DEBUG_CHECK, -1);
+  if (moved > 0) atomicAdd(&sm.moved, moved);
+  __syncthreads();
+  if (tid == 0 && status != nullptr && sm.moved > 0) atomicAdd(&status->counters[MOE_CNT_REROUTED], sm.moved);
 }
 
 }  // namespace
 
 cudaError_t launch_reroute_assign(int S, int E, int K, int capacity, int32_t* topk_idx, const float* cand_key,
-                                  const int32_t* counts, const int32_t* row_of_slot, int32_t* ex_scratch,
-                                  int32_t* changed, StatusBlock* status, cudaStream_t stream) {
+                                  const int32_t* counts, const int32_t* row_of_slot, int32_t* pick_scratch,
+                                  int32_t* claim_scratch, int32_t* changed, StatusBlock* status,
+                                  cudaStream_t stream) {
   if (S <= 0) return cudaSuccess;
   if (E < 1 || E > kMaxE || K < 1 || K > 32 || capacity <= 0) return cudaErrorInvalidValue;
-  reroute_assign_kernel<<<1, kThreads, 0, stream>>>(S, E, K, capacity, topk_idx, cand_key, counts, row_of_slot,
-                                                    ex_scratch, changed, status);
+  if ((reinterpret_cast<uintptr_t>(pick_scratch) & 15) != 0) return cudaErrorInvalidValue;
+  const bool vec = K % 4 == 0 && (reinterpret_cast<uintptr_t>(topk_idx) & 15) == 0 &&
+                   (reinterpret_cast<uintptr_t>(row_of_slot) & 15) == 0;
+  const int want = (S + kPickThreads - 1) / kPickThreads;
+  reroute_pick_kernel<<<want < 148 * 8 ? want : 148 * 8, kPickThreads, 0, stream>>>(
+      S, E, K, capacity, topk_idx, cand_key, counts, row_of_slot, pick_scratch, changed, claim_scratch, vec);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const size_t smem = sizeof(CommitSmem);
+  static std::atomic<uint64_t> attr_set{0};  // one bit per device ordinal
+  int dev = 0;
+  if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+  if (dev >= 64 || !(attr_set.load() & (1ull << dev))) {
+    err = cudaFuncSetAttribute(reroute_commit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    if (dev < 64) attr_set.fetch_or(1ull << dev);
+  }
+  reroute_commit_kernel<<<1, kThreads, smem, stream>>>(S, E, K, capacity, topk_idx, cand_key, counts, pick_scratch,
+                                                       changed, claim_scratch, vec, status);
   return cudaGetLastError();
 }
 

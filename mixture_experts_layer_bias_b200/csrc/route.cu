@@ -260,7 +260,7 @@ cudaError_t launch_topk_ni(const RouteArgs& a, const float* logits, const Select
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
   if (a.S == 0) return cudaSuccess;
   SelectParams sp{a.E,        a.K,      a.score_fn, a.renormalize, a.num_groups,   a.topk_groups, a.tau,
-                  a.sel_bias, a.topk_idx, a.topk_w, a.status,      a.cand_key_out, a.score_out, nullptr};
+                  a.sel_bias, a.topk_idx, a.topk_w, a.status,      a.cand_key_out, a.score_out};
   const int blocks = (a.S + kRouteWarps - 1) / kRouteWarps;
   const float* logits = a.logits;
   if (logits == nullptr && a.E <= 32) {

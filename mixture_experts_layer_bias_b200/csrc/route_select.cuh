@@ -84,7 +84,6 @@ struct SelectParams {
   StatusBlock* status;
   float* cand_key;   // optional [S][E]: selection key of each candidate expert, -inf for the others
   float* score_out;  // optional [S][E]: the gate source (logit, or sigmoid score) of every expert
-  int32_t* idx_mirror;  // optional: a second copy of topk_idx (shared memory of a fused kernel)
 };
 
 // Gate of this lane's selected expert (lanes < K hold one each, my_score its
@@ -255,7 +254,6 @@ __device__ void select_topk(const float (&l)[NI], const SelectParams& p, int t) 
   if (mine) {
     p.topk_idx[static_cast<int64_t>(t) * p.K + lane] = my_e;
     p.topk_w[static_cast<int64_t>(t) * p.K + lane] = g;
-    if (p.idx_mirror != nullptr) p.idx_mirror[t * p.K + lane] = my_e;
   }
 }
 

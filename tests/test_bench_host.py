@@ -34,13 +34,13 @@ def test_committed_traffic_record_is_current_or_absent():
 
 
 @pytest.mark.parametrize("name,S,expected", [
-    ("mixtral_prefill", None, 1 + 4 + 1 + 2 + 1),           # fused route, chunked permutation + groups, gather, GEMMs, combine
+    ("mixtral_prefill", None, 1 + 4 + 1 + 2 + 1),           # route, chunked permutation + groups, gather, GEMMs, combine
     ("dsv3_grouped", None, 2 + 4 + 1 + 2 + 1),              # router GEMM + top-k
-    ("fp8_skew_capacity", None, 2 + 4 + 1 + 2 + 1),         # E = 64: router GEMM + top-k; E4M3 decoded in the GEMMs
+    ("fp8_skew_capacity", None, 2 + 4 + 1 + 2 + 3 + 1),     # E = 64: router GEMM + top-k; 2048 rows per expert: decode pass
     ("mixtral_prefill_w8a8", None, 1 + 4 + 1 + 2 + 1 + 1),  # + quantisation of the hidden rows
-    ("fp8_skew_capacity_reroute", None, 2 + 4 + 1 + 2 + 5 + 1),  # + ranks (3), assignment, gates
-    ("mixtral_decode", 1, 1 + 2 + 1),                       # fused route-permute-gather, GEMMs, combine
-    ("mixtral_decode", 32, 1 + 1 + 1 + 2 + 2 + 1),          # one-CTA permutation, split-K finalizes
+    ("fp8_skew_capacity_reroute", None, 2 + 4 + 1 + 2 + 3 + 6 + 1),  # + ranks (3), picks, epochs, gates
+    ("mixtral_decode", 1, 1 + 1 + 1 + 2 + 2 + 1),           # one-CTA permutation, split-K finalizes
+    ("mixtral_decode", 32, 1 + 1 + 1 + 2 + 2 + 1),
     ("tiny_f32", None, 1 + 1 + 1 + 2 + 1),                  # fp32: no split-K
 ])
 def test_kernels_per_layer_call(name, S, expected):

@@ -305,17 +305,20 @@ def test_missing_library_fails_loudly():
     assert "raised" in r.stdout, (r.stdout, r.stderr)
 
 
-def test_e4m3_workspace_holds_no_decoded_weights():
+def test_e4m3_workspace_decoded_weights_only_for_many_rows():
     """E4M3 weights with bf16 activations are decoded tile by tile inside the
-    GEMMs: the workspace is no larger than with bf16 weights (no bf16 copy of
-    the weights).  With d or h not a multiple of 16 the layer decodes the
-    weights into the workspace first."""
-    c8 = syn.CONFIGS["fp8_skew_capacity"]
+    GEMMs while the experts have at most 1024 routed rows each on average:
+    the workspace is then no larger than with bf16 weights (no bf16 copy of
+    the weights).  With more rows per expert, or with d or h not a multiple
+    of 16, the layer decodes the weights into the workspace first."""
+    c8 = syn.scaled(syn.CONFIGS["fp8_skew_capacity"], S=8192)      # 8192 * 8 / 64 = 1024 rows per expert
     c16 = syn.scaled(c8, weight_dtype=syn.BF16)
-    n8 = ops.moe_workspace_size(ops.make_desc(**syn.desc_dict(c8)))
-    n16 = ops.moe_workspace_size(ops.make_desc(**syn.desc_dict(c16)))
-    assert n8 == n16
+    size = lambda c: ops.moe_workspace_size(ops.make_desc(**syn.desc_dict(c)))
+    assert size(c8) == size(c16)
+    big8 = syn.scaled(c8, S=8200)
+    assert size(big8) > size(syn.scaled(c16, S=8200))
+    n_dec = 3 * (big8.E + big8.num_shared) * big8.h * big8.d * 2      # the three decoded bf16 stacks
+    assert size(big8) - size(syn.scaled(c16, S=8200)) >= n_dec
     odd8 = syn.scaled(c8, d=2056)
     odd16 = syn.scaled(c16, d=2056)
-    assert ops.moe_workspace_size(ops.make_desc(**syn.desc_dict(odd8))) > \
-        ops.moe_workspace_size(ops.make_desc(**syn.desc_dict(odd16)))
+    assert size(odd8) > size(odd16)

@@ -29,7 +29,7 @@ ops._LIB_PATH = DEBUG_LIB
 from parity import run_layer, compare_layer, new_ws
 res = {{}}
 cases = {{
-    "decode_fused": syn.scaled(syn.CONFIGS["mixtral_decode"], S=4, d=512, h=512),
+    "decode": syn.scaled(syn.CONFIGS["mixtral_decode"], S=4, d=512, h=512),
     "prefill": syn.scaled(syn.CONFIGS["mixtral_prefill"], S=300, d=256, h=256),
     "capacity": syn.scaled(syn.CONFIGS["fp8_skew_capacity"], S=700, d=256, h=128),
     "grouped": syn.scaled(syn.CONFIGS["dsv3_grouped"], S=96, d=256, h=128),
@@ -72,7 +72,7 @@ def test_guard_build_agrees_and_reports():
     assert r.returncode == 0, r.stderr[-3000:]
     line = [l for l in r.stdout.splitlines() if l.startswith("RESULT ")][-1]
     res = json.loads(line[len("RESULT "):])
-    for name in ("decode_fused", "prefill", "capacity", "grouped"):
+    for name in ("decode", "prefill", "capacity", "grouped"):
         assert res[name]["ok"], (name, res[name])
         assert res[name]["flags"] == 0 and res[name]["code"] == 0, (name, res[name])
     bad = res["bad_row"]

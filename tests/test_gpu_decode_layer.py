@@ -1,10 +1,8 @@
-"""The tiny-batch layer path: routing, permutation and row gather in one
-kernel (route_permute_small_kernel) for S <= 16 tokens and E <= 32.
-
-Its maps and outputs must be exactly those of the separate stage calls
-(moe_route -> moe_permute -> moe_grouped_ffn -> moe_combine, whose routing
-kernel splits the dot products the same way), and the layer must match the
-oracle within the contract's tolerances.
+"""Decode-sized layer calls (S <= 16 tokens): the layer call must give
+exactly the outputs of the separate stage calls (moe_route -> moe_permute ->
+moe_grouped_ffn -> moe_combine), match the oracle within the contract's
+tolerances, repeat bit-identically, and let one workspace serve several batch
+sizes.
 """
 import dataclasses
 
@@ -51,12 +49,12 @@ CASES = [
     ("tiny_f32", dict(S=3)),
     ("tiny_f32", dict(S=16, E=32, K=4)),
     ("mixtral_decode", dict(S=7, d=512, h=512, E=32, K=4, capacity=1)),   # capacity with overflow rows
-    ("mixtral_prefill_w8a8", dict(S=9, d=512, h=512)),                  # fused routing, quantising gather
+    ("mixtral_prefill_w8a8", dict(S=9, d=512, h=512)),                  # quantising gather
 ]
 
 
 @pytest.mark.parametrize("name,kw", CASES)
-def test_fused_tiny_layer_equals_stage_calls_and_oracle(name, kw):
+def test_small_layer_equals_stage_calls_and_oracle(name, kw):
     base = syn.CONFIGS.get(name) or syn.VARIANTS[name]
     cfg = syn.scaled(base, **kw)
     inp = syn.make_inputs(cfg, "cuda", seed=11)
@@ -77,9 +75,9 @@ def test_fused_tiny_layer_equals_stage_calls_and_oracle(name, kw):
         assert counters["overflow_rows"] == int(np.maximum(ref["counts"].cpu().numpy() - cfg.capacity, 0).sum())
 
 
-def test_fused_path_repeats_bit_identically():
-    """Two layer calls on one workspace give the same bits (the split-K
-    arrival counters are left at zero by every call)."""
+def test_small_layer_repeats_bit_identically():
+    """Repeated layer calls on one workspace give the same bits (split-K
+    slices are summed in a fixed order)."""
     cfg = syn.scaled(syn.CONFIGS["mixtral_decode"], S=2, d=1024, h=2048)
     inp = syn.make_inputs(cfg, "cuda", seed=12)
     desc = ops.make_desc(**syn.desc_dict(cfg))
@@ -96,8 +94,7 @@ def test_fused_path_repeats_bit_identically():
 
 
 def test_one_workspace_serves_several_batch_sizes():
-    """A workspace sized for the largest batch serves smaller ones (the
-    split-K counters sit at a fixed place for every desc)."""
+    """A workspace sized for the largest batch serves smaller ones."""
     base = syn.scaled(syn.CONFIGS["mixtral_decode"], d=1024, h=2048)
     inp = syn.make_inputs(syn.scaled(base, S=128), "cuda", seed=13)
     big = ops.make_desc(**syn.desc_dict(base, 128))

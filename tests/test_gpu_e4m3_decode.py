@@ -1,5 +1,7 @@
-"""E4M3 expert weights with bf16 activations: the GEMM decodes every landed
-E4M3 weight tile to bf16 itself (no separate decode pass).
+"""E4M3 expert weights with bf16 activations: while the experts have at most
+1024 routed rows each on average, the GEMM decodes every landed E4M3 weight
+tile to bf16 itself (no separate decode pass); above that, one decode pass
+writes the bf16 weights to the workspace first.
 
 With all channel scales 1, the layer on E4M3 weights must give exactly the
 layer on the same weights decoded to bf16 beforehand (E4M3 -> bf16 is exact,
@@ -30,7 +32,8 @@ def _all_codes(shape, seed):
     return codes.to(torch.uint8)
 
 
-@pytest.mark.parametrize("S,E,K,cap", [(256, 8, 2, 0), (5, 8, 2, 0), (700, 16, 4, 180)])
+@pytest.mark.parametrize("S,E,K,cap", [(256, 8, 2, 0), (5, 8, 2, 0), (700, 16, 4, 180),
+                                       (4200, 4, 1, 0)])   # 1050 rows per expert: the decode pass
 def test_e4m3_layer_equals_bf16_layer_on_decoded_weights(S, E, K, cap):
     d, h = 256, 384
     cfg8 = syn.LayerConfig("e4m3_exact", S=S, d=d, E=E, K=K, h=h, weight_dtype=syn.E4M3, capacity=cap)

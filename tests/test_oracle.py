@@ -768,68 +768,141 @@ def test_selection_margin_hand_computed_and_stability():
     assert set(idx3[t].tolist()) != set(idx[t].tolist())
 
 
-def _reroute_in_rounds(topk_idx, keys, cand, capacity, chunk):
-    """The round structure the GPU assignment uses, restated on the host: every
-    slot of a chunk picks against the room at the round's start (a token's
-    slots in order, each excluding the earlier picks), picks are ranked per
-    expert in slot order, and the longest prefix whose picks fit is
-    committed."""
-    idx = np.array(topk_idx, dtype=np.int32, copy=True)
-    S, K = idx.shape
+def _reroute_in_epochs(topk_idx, keys, cand, capacity, nsegs):
+    """The epoch structure the GPU assignment uses, restated on the host.
+
+    Every excess slot first picks against the starting room (a token's slots
+    in k order, each excluding the token's experts and its earlier picks).
+    Then, per epoch: the first slot whose pick is the (room+1)-th pick of its
+    expert among the uncommitted slots is found through per-expert counts by
+    token segment (nsegs segments), then sub-ranges of that segment, then a
+    scan of one sub-range; the picks before it are committed; the experts
+    left without room drop out; the uncommitted slots that picked one of them
+    pick again, in k order per token, with the token's later slots that now
+    clash with a new pick.  Returns (topk_idx, epochs)."""
+    KEPT, NONE = -2, -1
+    idx = np.array(topk_idx, dtype=np.int64, copy=True).reshape(-1)
+    S, K = np.asarray(topk_idx).shape
     E = keys.shape[1]
-    P = O.expert_permutation(idx, E, capacity)
-    ex = np.nonzero(P["row_of_slot"] >= E * capacity)[0]
-    room = capacity - np.minimum(O.expert_counts(idx, E), capacity)
-    base = 0
-    rounds = 0
-    while base < len(ex):
-        m = min(chunk, len(ex) - base)
-        picks, held_t, held = [], -1, None
-        for i in range(m):
-            t = ex[base + i] // K
-            if t != held_t:
-                held_t, held = t, set(idx[t].tolist())
-            ok = [e for e in range(E) if room[e] > 0 and e not in held and cand[t, e] and keys[t, e] > -np.inf]
-            b = max(ok, key=lambda e: (keys[t, e], -e)) if ok else -1
-            picks.append(b)
-            if b >= 0:
-                held.add(b)
-        seen = np.zeros(E, np.int64)
-        p = m
-        for i, b in enumerate(picks):
-            if b >= 0:
-                if seen[b] >= room[b]:
-                    p = i
-                    break
-                seen[b] += 1
-        assert p >= 1
-        for i in range(p):
-            if picks[i] >= 0:
-                s = ex[base + i]
-                idx[s // K, s % K] = picks[i]
-                room[picks[i]] -= 1
-        base += p
-        rounds += 1
-    return idx, rounds
+    key = np.where(cand, keys, -np.inf)
+    counts = O.expert_counts(np.asarray(topk_idx), E)
+    ros = O.expert_permutation(np.asarray(topk_idx), E, capacity)["row_of_slot"]
+    room = capacity - np.minimum(counts, capacity)
+    avail = room > 0
+
+    def best(t, held):
+        bv, be = -np.inf, NONE
+        for e in range(E):
+            if key[t, e] > bv and not held[e] and avail[e]:
+                bv, be = key[t, e], e
+        return be
+
+    pick = np.full(S * K, KEPT)
+    for t in range(S):
+        held = np.zeros(E, bool)
+        held[idx[t * K:(t + 1) * K]] = True
+        for k in range(K):
+            if ros[t * K + k] >= E * capacity:
+                pick[t * K + k] = best(t, held)
+                if pick[t * K + k] >= 0:
+                    held[pick[t * K + k]] = True
+    seg_len = -(-S // nsegs)
+    seg_of = lambda s: (s // K) // seg_len
+    seg_begin = lambda w: min(S, w * seg_len) * K
+    cnt = np.zeros((nsegs, E), np.int64)
+    for s in np.nonzero(pick >= 0)[0]:
+        cnt[seg_of(s), pick[s]] += 1
+
+    def first_over(counts_by_part, limit):  # part holding the (limit+1)-th pick, picks before it there
+        acc = 0
+        for w, c in enumerate(counts_by_part):
+            if acc + c > limit:
+                return w, limit - acc
+            acc += c
+        return len(counts_by_part), 0
+
+    start, epochs = 0, 0
+    for _ in range(E + 2):
+        epochs += 1
+        seg_e, need_e = np.full(E, nsegs), np.zeros(E, np.int64)
+        for e in np.nonzero(avail)[0]:
+            seg_e[e], need_e[e] = first_over(cnt[:, e], room[e])
+        ms, P = int(seg_e.min()), S * K
+        if ms < nsegs:
+            a, b = max(seg_begin(ms), start), seg_begin(ms + 1)
+            span = -(-(b - a) // nsegs)
+            sub = np.zeros((nsegs, E), np.int64)
+            for w in range(nsegs):
+                lo = min(b, a + w * span)
+                for s in range(lo, min(b, lo + span)):
+                    if pick[s] >= 0 and seg_e[pick[s]] == ms:
+                        sub[w, pick[s]] += 1
+            sub_e, need2 = np.full(E, nsegs), np.zeros(E, np.int64)
+            for e in np.nonzero(seg_e == ms)[0]:
+                sub_e[e], need2[e] = first_over(sub[:, e], need_e[e])
+            wm = int(sub_e.min())
+            lo = min(b, a + wm * span)
+            run, P = np.zeros(E, np.int64), None
+            for s in range(lo, min(b, lo + span)):
+                p = pick[s]
+                if p >= 0 and seg_e[p] == ms and sub_e[p] == wm:
+                    if run[p] == need2[p]:
+                        P = s
+                        break
+                    run[p] += 1
+            assert P is not None
+        for s in range(start, P):
+            if pick[s] >= 0:
+                idx[s] = pick[s]
+                room[pick[s]] -= 1
+                cnt[seg_of(s), pick[s]] -= 1
+        start = P
+        if P >= S * K:
+            break
+        full = avail & (room <= 0)
+        avail &= ~full
+        done = set()
+        for s in range(P, S * K):
+            t = s // K
+            if pick[s] < 0 or not full[pick[s]] or t in done:
+                continue
+            done.add(t)
+            held = np.zeros(E, bool)
+            held[idx[t * K:(t + 1) * K]] = True
+            for k in range(max(P, t * K) - t * K, K):
+                p = pick[t * K + k]
+                if p >= 0 and (full[p] or held[p]):
+                    q = best(t, held)
+                    cnt[seg_of(t * K), p] -= 1
+                    if q >= 0:
+                        cnt[seg_of(t * K), q] += 1
+                    pick[t * K + k] = p = q
+                if p >= 0:
+                    held[p] = True
+    assert start >= S * K
+    return idx.reshape(S, K).astype(np.int32), epochs
 
 
-@pytest.mark.parametrize("chunk", [1, 4, 16, 1024])
-def test_reroute_rounds_equal_the_serial_assignment(chunk):
-    """The committed prefix of every round is the serial result: the round
-    structure reproduces reroute_over_capacity exactly, for any chunk size,
-    with at most ceil(excess / chunk) + E rounds."""
-    rng = np.random.default_rng(24 + chunk)
-    for trial in range(6):
-        S, E, K = int(rng.integers(50, 400)), int(rng.choice([8, 16, 32])), int(rng.integers(1, 5))
+@pytest.mark.parametrize("nsegs", [1, 3, 16])
+def test_reroute_epochs_equal_the_serial_assignment(nsegs):
+    """The epoch structure reproduces reroute_over_capacity exactly, for any
+    number of token segments, with ties in the keys, and with at most one
+    epoch per expert that runs out of room, plus one."""
+    rng = np.random.default_rng(24 + nsegs)
+    for trial in range(12):
+        S, E, K = int(rng.integers(20, 300)), int(rng.choice([4, 8, 16, 32])), int(rng.integers(1, 5))
         keys = (rng.normal(size=(S, E)) + 1.5 * rng.normal(size=E)[None, :]).astype(np.float32)
+        if trial % 3 == 0:
+            keys = np.round(keys).astype(np.float32)         # many equal keys
         cand = rng.random((S, E)) > 0.1
         idx, _ = O.select_experts(np.where(cand, keys, -np.inf).astype(np.float32), K)
         C = max(1, int(np.ceil(rng.uniform(0.7, 1.3) * S * K / E)))
         ref, _ = O.reroute_over_capacity(idx, keys, cand, C)
-        got, rounds = _reroute_in_rounds(idx, keys, cand, C, chunk)
+        got, epochs = _reroute_in_epochs(idx, keys, cand, C, nsegs)
         np.testing.assert_array_equal(got, ref)
-        n_ex = int((O.expert_permutation(idx, E, C)["row_of_slot"] >= E * C).sum())
-        assert rounds <= -(-n_ex // chunk) + E + 1
+        room = C - np.minimum(O.expert_counts(idx, E), C)
+        filled = int(((room > 0) & (O.expert_counts(ref, E) >= C)).sum())
+        assert epochs <= filled + 1, (epochs, filled)
 
 
 def test_skew_recipe_gives_max_over_mean_near_four():
