@@ -70,6 +70,8 @@ L2_FLUSH_BYTES = 256 << 20
 # of the current sources yet).
 GEMM_TRAFFIC_CAPTURE = {
     "workload": "mixtral_prefill",
+    # dram__bytes_read.sum + dram__bytes_write.sum of the up and down GEMM launches of one layer call,
+    # one-pass ncu capture of the full-size workload (None: not captured on the current GEMM sources)
     "bytes": None,
     "sources": ("common.cuh", "gemm_common.cuh", "gemm_sm100.cu"),
     "sha1": None,
@@ -359,12 +361,15 @@ def roofline_for(cfg, S, stages, peaks, workload_name):
             "peak_source": f"{peaks['source']} {kind}"}
 
 
-def decode_sweep(base_inp, device, peaks, reps=20):
-    """Decode-regime calls S in {1, 8, 32, 128} on the prefill weights with
-    the decode router offsets, captured in a CUDA graph; reports us per call,
-    tokens/s and the HBM fraction of the expert weights touched."""
+def decode_sweep(base_inp, device, peaks, reps=20, dcfg0=None):
+    """Decode-regime calls S in {1, 8, 32, 128} on the prefill weights (or
+    dcfg0's) with the decode router offsets, captured in a CUDA graph; reports
+    us per call (median of five batches of `reps` replays), tokens/s and the
+    HBM fraction of the expert weights touched
+    (their stored bytes: 2 per bf16 weight, 1 per E4M3 code plus the fp32
+    channel scales)."""
     out = {}
-    dcfg0 = syn.CONFIGS["mixtral_decode"]
+    dcfg0 = dcfg0 or syn.CONFIGS["mixtral_decode"]
     for S in syn.DECODE_SIZES:
         cfg = syn.scaled(dcfg0, S=S)
         dinp = syn.make_inputs(cfg, device, seed=0, x_only=True)
@@ -382,15 +387,22 @@ def decode_sweep(base_inp, device, peaks, reps=20):
             run.call(stream=s)
         g.replay()
         torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(reps):
-            g.replay()
-        e1.record()
-        torch.cuda.synchronize()
-        us = e0.elapsed_time(e1) * 1e3 / reps
+        # five batches of `reps` replays; the median batch's time per call
+        batches = []
+        for _ in range(5):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            batches.append(e0.elapsed_time(e1) * 1e3 / reps)
+        us = statistics.median(batches)
         touched = int((run.counts > 0).sum().item())
-        wbytes = touched * 3 * cfg.d * cfg.h * 2
+        if cfg.weight_dtype == syn.E4M3:
+            wbytes = touched * (3 * cfg.d * cfg.h + (2 * cfg.h + cfg.d) * 4)
+        else:
+            wbytes = touched * 3 * cfg.d * cfg.h * 2
         gbs = wbytes / (us * 1e-6) / 1e9
         out[str(S)] = {"us_per_call": round(us, 2), "tokens_per_s": round(S / (us * 1e-6), 1),
                        "experts_touched": touched, "weight_bytes": wbytes, "hbm_gbs": round(gbs, 1),
@@ -663,13 +675,21 @@ def main():
 
     e2e = e2e_run(run, args.steps, args.warmup, world, dist)
     bias_us = time_bias_update(cfg, device, S)
-    dec = None
+    dec = dec8 = None
     if not args.no_decode and args.workload == WORKLOAD:
         dec = decode_sweep(run.inp, device, peaks)
     inp = run.inp
     del run
     gc.collect()
     torch.cuda.empty_cache()
+    if not args.no_decode and args.workload == WORKLOAD:
+        # the same decode sizes on E4M3 expert weights (decoded inside the GEMMs)
+        c8 = syn.VARIANTS["mixtral_decode_e4m3"]
+        inp8 = syn.make_inputs(c8, device, seed=0)
+        dec8 = decode_sweep(inp8, device, peaks, dcfg0=c8)
+        del inp8
+        gc.collect()
+        torch.cuda.empty_cache()
     workloads = None
     if not args.no_workloads and args.workload == WORKLOAD:
         workloads = {}
@@ -695,7 +715,8 @@ def main():
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": kernels_per_step(cfg) * args.steps, "clocks": clk,
             "stages_ms": {k: round(v, 4) for k, v in stages.items()},
-            "load": load, "decode_sweep": dec, "bias_update_us": bias_us, "counters": counters,
+            "load": load, "decode_sweep": dec, "decode_sweep_e4m3": dec8, "bias_update_us": bias_us,
+            "counters": counters,
             "workloads": workloads}
     print(json.dumps(line), flush=True)
 

@@ -35,6 +35,7 @@ struct TcParams {
   int pcols;           // 2N (SwiGLU: gate then up) or N
   int* ksplit_out;     // the split chosen on the device (read by the finalize kernel)
   int test_stall;      // test hook: the producer delivers nothing (the bounded waits must give up)
+  int land_stages;     // E4M3-weight kernel: landing buffers of E4M3 weight tiles
   int tma_out;         // 1: the output tensor map is valid (full 32-row quarters use bulk tensor stores)
   const float* row_scale;         // E4M3 activations: per-row scale of the A operand rows (nullptr: none)
   const float* row_scale_shared;  // ... of the shared expert's A rows (indexed by row within the group)

@@ -70,7 +70,7 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;
 // E4M3 weight tile into the bf16 B tile of its stage.
 constexpr int kConvWarps = 8;
 constexpr int kThreadsW8 = kThreads + 32 * kConvWarps;
-constexpr int kLandStages = 3;             // landing buffers of E4M3 weight tiles
+constexpr int kMaxLandStages = 8;          // landing buffers of E4M3 weight tiles (at most)
 constexpr int LAND_BYTES = 256 * 64;       // 256 weight rows x 64 E4M3 codes (one bf16 K step)
 constexpr uint32_t kIdescBf16 = idesc_bf16_f32(128, 256);
 constexpr uint32_t kIdescE4m3 = idesc_e4m3_f32(128, 256);
@@ -84,7 +84,7 @@ constexpr int bk_elems() {
 struct SmemCtl {
   uint64_t full[MAX_STAGES];
   uint64_t empty[MAX_STAGES];
-  uint64_t lfull[kLandStages];  // W8: an E4M3 weight tile has landed
+  uint64_t lfull[kMaxLandStages];  // W8: an E4M3 weight tile has landed
   int conv_ok;                  // W8: the converters' shared go / give-up decision
   uint64_t tfull[2];
   uint64_t tempty[2];
@@ -321,7 +321,8 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
   const int A_TILE = bma * BK_BYTES;
   const int STAGE_BYTES = A_TILE + B_TILE;
   uint8_t* land = ring + STAGES * STAGE_BYTES;  // W8 landing buffers (1024-byte aligned)
-  uint8_t* ctl = land + (W8 ? kLandStages * LAND_BYTES : 0);
+  const int LAND = W8 ? p.land_stages : 0;       // W8 landing buffers in use
+  uint8_t* ctl = land + LAND * LAND_BYTES;
   SmemCtl& s = *reinterpret_cast<SmemCtl*>(ctl);
   uint8_t* epi_smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(ctl + sizeof(SmemCtl)) + 127) & ~uintptr_t(127));
@@ -338,7 +339,7 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
         mbar_init(&s.empty[i], 1);
       }
       if (W8)
-        for (int i = 0; i < kLandStages; ++i) mbar_init(&s.lfull[i], 1);
+        for (int i = 0; i < LAND; ++i) mbar_init(&s.lfull[i], 1);
       for (int i = 0; i < 2; ++i) {
         mbar_init(&s.tfull[i], 1);
         mbar_init(&s.tempty[i], 32 * kEpiWarps);
@@ -498,7 +499,7 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
     // the MMA warp's order), wait for the E4M3 tile to land and for the stage's
     // B tile to be free, decode it, then let the MMA go (second arrival on the
     // stage's full barrier) and reuse the landing buffer for the K step
-    // kLandStages ahead.  One thread waits on the barriers and issues the
+    // LAND ahead.  One thread waits on the barriers and issues the
     // copies; the decision to go on or give up reaches all converter threads through
     // shared memory, so they leave together.
     const int ct = threadIdx.x - (2 + kEpiWarps) * 32;
@@ -548,7 +549,7 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
     uint32_t armed = 0;  // landing buffers with a copy in flight
     uint32_t lphase_bits = 0;
     if (ct == 0 && !p.test_stall) {
-      for (int l = 0; l < kLandStages && ahd.u < total; ++l) {
+      for (int l = 0; l < LAND && ahd.u < total; ++l) {
         issue(ahd, l);
         armed |= 1u << l;
         seq_next(ahd);
@@ -586,7 +587,7 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
         stage = 0;
         phase ^= 1u;
       }
-      if (++l == kLandStages) {
+      if (++l == LAND) {
         l = 0;
         lphase ^= 1u;
       }
@@ -595,7 +596,7 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
       *abort_flag = 1;
       report(p.status, MOE_STATUS_TIMEOUT, MOE_CNT_TIMEOUT);
       // let the copies already issued land before the CTA exits
-      for (int i = 0; i < kLandStages; ++i)
+      for (int i = 0; i < LAND; ++i)
         if (armed & (1u << i)) wait_timed(&s.lfull[i], (lphase_bits >> i) & 1u);
     }
   } else {
@@ -671,13 +672,29 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
   const size_t stage_bytes = static_cast<size_t>(bma) * BK_BYTES + B_TILE;
   const int eb = a.fp8 ? 1 : 2;  // element bytes of A and B
   const bool w8 = a.w8 != 0 && !a.fp8;
-  const size_t land_bytes = w8 ? static_cast<size_t>(kLandStages) * LAND_BYTES : 0;
-  int stages = static_cast<int>((kSmemLimitTc - kCtlBytes - land_bytes) / stage_bytes);
-  if (stages > MAX_STAGES) stages = MAX_STAGES;
+  int stages, land = 0;
+  if (w8) {
+    // E4M3 weights: the HBM latency is covered by the landing buffers (a
+    // weight tile is decoded into a bf16 stage only when the MMA is about to
+    // need it), so three bf16 stages and as many landing buffers as fit
+    stages = 3;
+    land = static_cast<int>((kSmemLimitTc - kCtlBytes - stages * stage_bytes) / LAND_BYTES);
+    if (land < 2) {
+      stages = 2;
+      land = static_cast<int>((kSmemLimitTc - kCtlBytes - stages * stage_bytes) / LAND_BYTES);
+    }
+    if (land > kMaxLandStages) land = kMaxLandStages;
+    if (land < 2) return cudaErrorInvalidValue;
+  } else {
+    stages = static_cast<int>((kSmemLimitTc - kCtlBytes) / stage_bytes);
+    if (stages > MAX_STAGES) stages = MAX_STAGES;
+  }
+  const size_t land_bytes = static_cast<size_t>(land) * LAND_BYTES;
   const size_t smem = stages * stage_bytes + land_bytes + kCtlBytes;
   CUtensorMap mA, mA2, mB0, mB1, mOut;
   // bf16 outputs: full 32-row quarters go out as bulk tensor stores; fp32 outputs store row by row
   TcParams pp = p;
+  pp.land_stages = land;
   pp.tma_out = !a.out_f32 && make_store_map(&mOut, a.out, a.out_rows, a.N, 2) ? 1 : 0;
   if (!pp.tma_out) memset(&mOut, 0, sizeof(mOut));
   if (!make_map(&mA, a.a, a.a_rows, a.K, bma, eb)) return cudaErrorInvalidValue;

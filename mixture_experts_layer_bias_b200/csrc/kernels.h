@@ -37,11 +37,11 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream);
 // in (token, k) order, to the best-keyed candidate expert with room that the
 // token does not hold; changed[t] marks tokens with a moved slot.  A multi-CTA
 // pick kernel, then one CTA running the epochs.  pick_scratch: int32 [S*K],
-// 16-byte aligned; claim_scratch: int32 [S].
+// 16-byte aligned; claim_scratch, list_scratch: int32 [S].
 cudaError_t launch_reroute_assign(int S, int E, int K, int capacity, int32_t* topk_idx, const float* cand_key,
                                   const int32_t* counts, const int32_t* row_of_slot, int32_t* pick_scratch,
-                                  int32_t* claim_scratch, int32_t* changed, StatusBlock* status,
-                                  cudaStream_t stream);
+                                  int32_t* claim_scratch, int32_t* list_scratch, int32_t* changed,
+                                  StatusBlock* status, cudaStream_t stream);
 // Gates of the tokens marked in changed[], recomputed over their final experts
 // from the gate sources (the same formulas as the routing kernels).
 cudaError_t launch_reroute_gates(int S, int E, int K, int score_fn, int renormalize, const float* score,

@@ -32,6 +32,7 @@ namespace {
 constexpr int kChunkSlots = 1024;  // slots per CTA (whole tokens)
 constexpr int kSmallWarps = 32;
 constexpr int kSmallSlots = 4096;  // the single-CTA permutation handles S*K up to this
+constexpr int64_t kFoldGatherBytes = 256 << 10;  // ... and also copies the rows up to this many bytes
 constexpr int kPermWarps = 8;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
@@ -333,16 +334,28 @@ __device__ void permute_small_body(int S, int E, int K, int capacity, int num_sh
   if (g1 != nullptr) write_groups(S, E, K, capacity, num_shared, offs_s, g1);
 }
 
+// x / x_perm (optional): the row gather of a tiny batch folded in -- every
+// token row (row_chunks 16-byte pieces) copied to its slots' rows once the
+// maps are written, so a decode step spends no launch on it.
 __global__ void __launch_bounds__(kSmallWarps * 32)
     permute_small_kernel(int S, int E, int K, int capacity, int num_shared, const int32_t* topk_idx,
                          int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                          int32_t* __restrict__ row_of_slot, int32_t* __restrict__ token_of_row, int64_t num_rows,
-                         GroupEntry* __restrict__ g1, StatusBlock* status) {
+                         GroupEntry* __restrict__ g1, StatusBlock* status, const uint4* __restrict__ x,
+                         uint4* __restrict__ x_perm, int row_chunks) {
   extern __shared__ int32_t sm[];
   pdl_wait();
   pdl_trigger();
   permute_small_body(S, E, K, capacity, num_shared, topk_idx, counts, offsets, row_of_slot, token_of_row, num_rows,
                      g1, status, sm);
+  if (x == nullptr) return;
+  __syncthreads();  // the row maps written above are read back below
+  const int64_t n = static_cast<int64_t>(S) * K * row_chunks;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
+    const int64_t sl = i / row_chunks, c = i - sl * row_chunks;
+    const int row = row_of_slot[sl];
+    if (row >= 0) x_perm[static_cast<int64_t>(row) * row_chunks + c] = x[(sl / K) * row_chunks + c];
+  }
 }
 
 // Row gather for small batches: one CTA per token, its threads split the row.
@@ -437,11 +450,16 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
     return err;
   }
   cudaError_t err;
+  const int64_t row_bytes = static_cast<int64_t>(a.d) * (a.act_dtype == MOE_BF16 ? 2 : 4);
+  bool gathered = false;
   if (static_cast<int64_t>(a.S) * a.K <= kSmallSlots) {
     const size_t smem = sizeof(int32_t) * (kSmallWarps * a.E + 3 * a.E + 1);
+    // tiny batches: the one CTA also copies the rows (a few hundred KB at most)
+    gathered = a.x != nullptr && a.x_perm != nullptr && static_cast<int64_t>(a.S) * a.K * row_bytes <= kFoldGatherBytes;
     err = launch_pdl(permute_small_kernel, dim3(1), dim3(kSmallWarps * 32), smem, stream, a.S, a.E, a.K, a.capacity,
                      a.num_shared, a.topk_idx, a.counts, a.offsets, a.row_of_slot, a.token_of_row, a.num_rows, a.g1,
-                     a.status);
+                     a.status, gathered ? static_cast<const uint4*>(a.x) : nullptr,
+                     gathered ? static_cast<uint4*>(a.x_perm) : nullptr, static_cast<int>(row_bytes / 16));
     if (err != cudaSuccess || (err = cudaGetLastError()) != cudaSuccess) return err;
   } else {
     const int tpc = permute_tokens_per_chunk(a.K);
@@ -468,7 +486,7 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
       if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
   }
-  if (a.x == nullptr || a.x_perm == nullptr) return cudaSuccess;
+  if (a.x == nullptr || a.x_perm == nullptr || gathered) return cudaSuccess;
   if (a.S <= 256) {
 #define MOE_GATHER_CTA(T)                                                                                    \
   err = launch_pdl(gather_rows_cta_kernel<T>, dim3(a.S), dim3(256), 0, stream, a.d, a.K,                       \

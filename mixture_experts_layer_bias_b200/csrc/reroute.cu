@@ -228,6 +228,7 @@ struct CommitSmem {
   int min_seg, min_sub;
   long long first_bad;
   int moved;
+  int nlist;  // tokens listed for re-picking in this epoch
 };
 
 // The uncommitted excess slots of token t from slot `first` on pick again, in
@@ -263,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     reroute_commit_kernel(int S, int E, int K, int C, int32_t* __restrict__ topk_idx,
                           const float* __restrict__ cand_key, const int32_t* __restrict__ counts,
                           int32_t* __restrict__ pick, int32_t* __restrict__ changed, int32_t* __restrict__ claim,
-                          bool vec, StatusBlock* status) {
+                          int32_t* __restrict__ list, bool vec, StatusBlock* status) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   CommitSmem& sm = *reinterpret_cast<CommitSmem*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -398,6 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++moved;
     });
     if (tid < kMaskWords) sm.full[tid] = 0;
+    if (tid == 0) sm.nlist = 0;
     __syncthreads();
     start = P;
     if (P >= nslots) break;
@@ -408,14 +410,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid < kMaskWords) sm.avail[tid] &= ~sm.full[tid];
     __syncthreads();
     // 5. the tokens with an uncommitted slot that picked a full expert pick
-    //    again; the first thread to see such a slot claims the token for this
-    //    epoch and re-picks it
+    //    again: the first thread to see such a slot claims the token for this
+    //    epoch and lists it; then the listed tokens are re-picked, one per
+    //    thread (so the threads of a warp re-pick side by side)
     for_picks(pick, P, nslots, tid, kThreads, [&](int64_t s, int p) {
       if (p < 0 || !bit_of(sm.full, p)) return;
       const int t = static_cast<int>(s / K);
-      if (atomicMax(&claim[t], epoch + 1) < epoch + 1)
-        repick_token(t, P, E, K, vec, seg_of(s), topk_idx, cand_key, pick, sm);
+      if (atomicMax(&claim[t], epoch + 1) < epoch + 1) list[atomicAdd(&sm.nlist, 1)] = t;
     });
+    __syncthreads();
+    const int nl = sm.nlist;
+    for (int i = tid; i < nl; i += kThreads) {
+      const int t = list[i];
+      repick_token(t, P, E, K, vec, seg_of(static_cast<int64_t>(t) * K), topk_idx, cand_key, pick, sm);
+    }
     __syncthreads();
   }
   if (!ok || start < nslots) report(status, MOE_STATUS_DEBUG_CHECK, -1);
@@ -428,8 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_reroute_assign(int S, int E, int K, int capacity, int32_t* topk_idx, const float* cand_key,
                                   const int32_t* counts, const int32_t* row_of_slot, int32_t* pick_scratch,
-                                  int32_t* claim_scratch, int32_t* changed, StatusBlock* status,
-                                  cudaStream_t stream) {
+                                  int32_t* claim_scratch, int32_t* list_scratch, int32_t* changed,
+                                  StatusBlock* status, cudaStream_t stream) {
   if (S <= 0) return cudaSuccess;
   if (E < 1 || E > kMaxE || K < 1 || K > 32 || capacity <= 0) return cudaErrorInvalidValue;
   if ((reinterpret_cast<uintptr_t>(pick_scratch) & 15) != 0) return cudaErrorInvalidValue;
@@ -451,7 +459,7 @@ cudaError_t launch_reroute_assign(int S, int E, int K, int capacity, int32_t* to
     if (dev < 64) attr_set.fetch_or(1ull << dev);
   }
   reroute_commit_kernel<<<1, kThreads, smem, stream>>>(S, E, K, capacity, topk_idx, cand_key, counts, pick_scratch,
-                                                       changed, claim_scratch, vec, status);
+                                                       changed, claim_scratch, list_scratch, vec, status);
   return cudaGetLastError();
 }
 

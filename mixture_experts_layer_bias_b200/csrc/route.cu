@@ -95,29 +95,33 @@ __global__ void __launch_bounds__(kRouteWarpsP * 32)
   }
   red[set][part][lane] = acc[0];
   __syncthreads();
-  if (part != 0 || t0 >= S) return;
-  float mine = 0.0f;
-#pragma unroll
-  for (int q = 0; q < kRouteSplit; ++q) mine += red[set][q][lane];
+  // the set's warps select its tokens in parallel: warp `part` takes tokens
+  // t0 + part, t0 + part + kRouteSplit, ...; a token's logit of expert e is
+  // the sum of the four parts' value tt * EMAX + e, added in part order
   const float bias = (lane < p.E && router_bias != nullptr) ? __ldg(router_bias + lane) : 0.0f;
-#pragma unroll
-  for (int tt = 0; tt < TPW; ++tt) {
+  for (int tt = part; tt < TPW; tt += kRouteSplit) {
     if (t0 + tt >= S) break;  // warp-uniform
-    float l[1];
-    l[0] = __shfl_sync(kFull, mine, tt * EMAX + (lane % EMAX));
+    float l[1] = {0.0f};
+    if (lane < EMAX) {
+#pragma unroll
+      for (int q = 0; q < kRouteSplit; ++q) l[0] += red[set][q][tt * EMAX + lane];
+    }
     if (lane < p.E && router_bias != nullptr) l[0] = __fadd_rn(l[0], bias);
     select_topk<1>(l, p, t0 + tt);
   }
 }
 
-// Small batches (decode): one CTA per token, its 8 warps split d so the
-// token's dot products are not serialised on one warp.  Per-warp partial sums
-// are added in warp order (deterministic), then warp 0 selects.
+// Small batches (decode): one CTA per token, its 16 warps split d (d = 4096
+// in bf16 is one 16-byte vector per thread, so every load of the token is in
+// flight at once).  Per-warp partial sums are added in warp order
+// (deterministic), then warp 0 selects.
+constexpr int kRouteTokenWarps = 16;
+
 template <typename T, int EMAX>
-__global__ void __launch_bounds__(kRouteWarps * 32)
+__global__ void __launch_bounds__(kRouteTokenWarps * 32)
     route_token_cta_kernel(int d, const T* __restrict__ x, const T* __restrict__ w_router,
                            const float* __restrict__ router_bias, SelectParams p) {
-  __shared__ float part[kRouteWarps][EMAX];
+  __shared__ float part[kRouteTokenWarps][EMAX];
   pdl_wait();
   pdl_trigger();
   const int t = blockIdx.x;
@@ -128,7 +132,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
 #pragma unroll
   for (int e = 0; e < EMAX; ++e) acc[e] = 0.0f;
   const T* xr = x + static_cast<int64_t>(t) * d;
-  for (int v = threadIdx.x; v < nvec; v += kRouteWarps * 32) {
+  for (int v = threadIdx.x; v < nvec; v += kRouteTokenWarps * 32) {
     float xf[V];
     unpack16<T>(ldg16(xr + v * V), xf);
 #pragma unroll
@@ -151,7 +155,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
   float l[1] = {0.0f};
   if (lane < p.E && lane < EMAX) {
     float s = 0.0f;
-    for (int w = 0; w < kRouteWarps; ++w) s += part[w][lane];
+    for (int w = 0; w < kRouteTokenWarps; ++w) s += part[w][lane];
     l[0] = router_bias != nullptr ? __fadd_rn(s, __ldg(router_bias + lane)) : s;
   }
   select_topk<1>(l, p, t);
@@ -270,7 +274,7 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
 #define MOE_ROUTE_LAUNCH(T, EM)                                                                                \
   do {                                                                                                         \
     if (per_cta) {                                                                                             \
-      err = launch_pdl(route_token_cta_kernel<T, EM>, dim3(a.S), dim3(kRouteWarps * 32), 0, stream, a.d,       \
+      err = launch_pdl(route_token_cta_kernel<T, EM>, dim3(a.S), dim3(kRouteTokenWarps * 32), 0, stream, a.d,  \
                        static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);      \
     } else {                                                                                                   \
       const int per_cta_tokens = (kRouteWarpsP / kRouteSplit) * (32 / EM);                                     \

@@ -1,7 +1,7 @@
 // Expert selection of one token held by one warp: scores (softmax logits
 // with temperature, or the operationally defined sigmoid), selection bias,
 // group-limited candidates, K rounds of arg-max and the gate weights.  Shared
-// by the routing kernels and the fused small-batch route-permute kernel.
+// by the routing kernels.
 //
 // jsqmd.com "第11章 MoE模型推理" 11.1.1 (R(x) = Softmax(W_r x) with the TopK
 // sparsifier), 11.3.3 (soft routing with a temperature); ybb.press

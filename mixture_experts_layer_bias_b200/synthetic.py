@@ -97,6 +97,9 @@ VARIANTS = {
     # the skewed capacity-bounded layer with over-capacity re-routing instead of the overflow pass
     "fp8_skew_capacity_reroute": dataclasses.replace(CONFIGS["fp8_skew_capacity"], name="fp8_skew_capacity_reroute",
                                                      reroute=1),
+    # decode with the Mixtral-shaped expert weights stored as E4M3 (per-channel scales), bf16 activations
+    "mixtral_decode_e4m3": dataclasses.replace(CONFIGS["mixtral_decode"], name="mixtral_decode_e4m3",
+                                               weight_dtype=E4M3),
 }
 
 DECODE_SIZES = (1, 8, 32, 128)

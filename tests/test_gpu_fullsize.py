@@ -138,6 +138,26 @@ def test_mixtral_decode_sweep_full_weights():
     _free()
 
 
+def test_mixtral_decode_e4m3_weights_full_size():
+    """The decode sizes on the Mixtral-shaped weights stored as E4M3 with
+    per-channel scales and bf16 activations: the GEMMs decode the weight
+    tiles themselves.  Every token against the oracle (FP8 tolerance)."""
+    base = syn.VARIANTS["mixtral_decode_e4m3"]
+    weights = syn.make_inputs(syn.scaled(base, S=1), "cuda", seed=0)
+    for S in (1, 8, 32):
+        cfg = syn.scaled(base, S=S)
+        inp = dict(weights)
+        inp["x"] = syn.make_inputs(cfg, "cuda", seed=S, x_only=True)["x"]
+        gpu = run_layer(inp, cfg)
+        code, flags, counters = ops.moe_get_status(gpu["ws"])
+        assert flags == 0, (flags, counters)
+        rep = compare_layer(gpu, inp, cfg)
+        print(cfg.name, S, rep)
+        assert rep["ok"], rep
+    del weights
+    _free()
+
+
 def test_dsv3_grouped_full_size():
     cfg = syn.CONFIGS["dsv3_grouped"]
     inp = syn.make_inputs(cfg, "cuda", seed=0)
