@@ -50,8 +50,8 @@ int64_t routed_rows(const moe_desc& d) {
 size_t act_bytes(const moe_desc& d) { return d.act_dtype == MOE_F32 ? 4 : 2; }
 
 // E4M3 weights with bf16 activations: the GEMMs decode each weight tile
-// themselves (every weight row a whole number of 16-byte pieces) while the
-// experts have few rows.  Each CTA decodes the tiles it multiplies, so a
+// themselves (every weight row a whole number of 16-byte pieces, at least 128
+// codes) while the experts have few rows.  Each CTA decodes the tiles it multiplies, so a
 // weight tile is decoded once per 128-row block of its expert: with many row
 // blocks the decode (ALU and shared-memory bandwidth) outgrows the MMA, and a
 // single decode pass into the workspace followed by the bf16 GEMM is faster.
@@ -59,7 +59,7 @@ constexpr int64_t kW8InGemmRowsPerExpert = 1024;
 
 bool w8_in_gemm(const moe_desc& d) {
   return d.weight_dtype == MOE_E4M3 && d.act_quant == 0 && d.act_dtype == MOE_BF16 && d.d_model % 16 == 0 &&
-         d.d_ff % 16 == 0 &&
+         d.d_ff % 16 == 0 && d.d_model >= 128 && d.d_ff >= 128 &&
          static_cast<int64_t>(d.num_tokens) * d.top_k <= kW8InGemmRowsPerExpert * d.num_experts;
 }
 

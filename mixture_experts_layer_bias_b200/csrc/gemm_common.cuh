@@ -220,10 +220,10 @@ inline bool make_map(CUtensorMap* m, const void* base, int64_t rows, int k, int 
 inline bool make_map_w8(CUtensorMap* m, const void* base, int64_t rows, int k) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr || rows <= 0 || k <= 0) return false;
-  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || k % 16 != 0) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || k % 16 != 0 || k < 128) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(k)};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {128, 128};  // two bf16 K steps of 128 weight rows
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

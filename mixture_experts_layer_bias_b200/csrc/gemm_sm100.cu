@@ -71,7 +71,7 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kConvWarps = 8;
 constexpr int kThreadsW8 = kThreads + 32 * kConvWarps;
 constexpr int kMaxLandStages = 8;          // landing buffers of E4M3 weight tiles (at most)
-constexpr int LAND_BYTES = 256 * 64;       // 256 weight rows x 64 E4M3 codes (one bf16 K step)
+constexpr int LAND_BYTES = 256 * 128;      // 256 weight rows x 128 E4M3 codes (two bf16 K steps)
 constexpr uint32_t kIdescBf16 = idesc_bf16_f32(128, 256);
 constexpr uint32_t kIdescE4m3 = idesc_e4m3_f32(128, 256);
 
@@ -283,17 +283,19 @@ __device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint3
       : "r"(w));
 }
 
-// W8: the converter threads (kConvWarps warps) decode one landed 256 x 64
-// E4M3 tile (rows of 64 bytes) into the stage's 256 x 128-byte bf16 B tile in
-// the 128-byte swizzled layout the MMA reads (16-byte chunk j of row r at
-// chunk j ^ (r & 7)).  Thread ct takes the 16-code pieces ct + 32 kConvWarps i.
+// W8: the converter threads (kConvWarps warps) decode the 64 codes of one K
+// step from each of the 256 rows of a landing buffer (rows of 128 bytes, two
+// K steps; `land` points at the step's first code of row 0) into the stage's
+// 256 x 128-byte bf16 B tile in the 128-byte swizzled layout the MMA reads
+// (16-byte chunk j of row r at chunk j ^ (r & 7)).  Thread ct takes the
+// 16-code pieces ct + 32 kConvWarps i.
 __device__ __forceinline__ void convert_tile_w8(const uint8_t* land, uint8_t* b16, int ct) {
   constexpr int kConvThreads = 32 * kConvWarps;
 #pragma unroll 2
   for (int i = 0; i < 1024 / kConvThreads; ++i) {
     const int piece = ct + kConvThreads * i;  // 1024 pieces of 16 codes
     const int r = piece >> 2, q4 = piece & 3;
-    const uint4 v = *reinterpret_cast<const uint4*>(land + r * 64 + q4 * 16);
+    const uint4 v = *reinterpret_cast<const uint4*>(land + r * 128 + q4 * 16);
     uint32_t o[8];
     e4m3x4_to_bf16x4(v.x, o[0], o[1]);
     e4m3x4_to_bf16x4(v.y, o[2], o[3]);
@@ -495,17 +497,20 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
     }
     __syncwarp();
   } else if (W8 && warp >= 2 + kEpiWarps) {
-    // W8 converters: for every K step of this CTA's units (the producer's and
-    // the MMA warp's order), wait for the E4M3 tile to land and for the stage's
-    // B tile to be free, decode it, then let the MMA go (second arrival on the
-    // stage's full barrier) and reuse the landing buffer for the K step
-    // LAND ahead.  One thread waits on the barriers and issues the
-    // copies; the decision to go on or give up reaches all converter threads through
-    // shared memory, so they leave together.
+    // W8 converters.  A landing buffer holds the E4M3 codes of two K steps
+    // of a weight tile (256 rows x 128 bytes: DRAM reads of 128 contiguous
+    // bytes per row).  For every K step of this CTA's units (the producer's
+    // and the MMA warp's order) wait for its codes to land and for the stage's
+    // B tile to be free, decode them, then let the MMA go (second arrival on
+    // the stage's full barrier); a landing buffer is refilled with the pair
+    // LAND pairs ahead once both of its K steps are decoded.  One thread
+    // waits on the barriers and issues the copies; the decision to go on or
+    // give up reaches all converter threads through shared memory, so they
+    // leave together.
     const int ct = threadIdx.x - (2 + kEpiWarps) * 32;
-    // the K-step sequence, walked twice: `cur` for decoding, `ahd` for issuing copies
+    // the sequence of K-step pairs, walked twice: `cur` for decoding, `ahd` for issuing copies
     struct Seq {
-      int u, kb, kb1;
+      int u, kb, kb1;  // unit, first K step of the pair, end of the unit's K range
     };
     auto seq_begin = [&](Seq& q) {
       q.u = blockIdx.x;
@@ -520,7 +525,8 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
       }
     };
     auto seq_next = [&](Seq& q) {
-      if (++q.kb < q.kb1) return;
+      q.kb += 2;
+      if (q.kb < q.kb1) return;
       q.u += gridDim.x;
       while (q.u < total) {
         const UnitInfo ui = decode_unit(s, p, q.u, ks, nk);
@@ -530,7 +536,7 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
         q.u += gridDim.x;
       }
     };
-    auto issue = [&](const Seq& q, int l) {  // E4M3 tile of K step q into landing buffer l
+    auto issue = [&](const Seq& q, int l) {  // E4M3 codes of pair q into landing buffer l
       const UnitInfo ui = decode_unit(s, p, q.u, ks, nk);
       const int b_row = ui.ti.grp.expert * p.n_per_slab + ui.ti.n_idx * p.bn_out;
       uint8_t* dst = land + l * LAND_BYTES;
@@ -558,35 +564,37 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
     int stage = 0, l = 0;
     uint32_t phase = 0, lphase = 0;
     bool ok = true;
-    while (cur.u < total) {
-      if (ct == 0) {
-        int go = !p.test_stall && mbar_wait(&s.lfull[l], lphase, abort_flag) &&
-                 mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag);
-        if (go) armed &= ~(1u << l);
-        s.conv_ok = go;
-      }
-      named_bar_sync(1, 32 * kConvWarps);
-      if (!s.conv_ok) {
-        ok = false;
-        break;
-      }
-      convert_tile_w8(land + l * LAND_BYTES, ring + stage * STAGE_BYTES + A_TILE, ct);
-      fence_proxy_async_smem();  // generic-proxy writes before the tensor core's reads
-      named_bar_sync(1, 32 * kConvWarps);
-      if (ct == 0) {
-        mbar_arrive(&s.full[stage]);
-        if (ahd.u < total) {
-          issue(ahd, l);
-          armed |= 1u << l;
-          lphase_bits = (lphase_bits & ~(1u << l)) | (((lphase + 1u) & 1u) << l);
-          seq_next(ahd);
+    while (cur.u < total && ok) {
+      const int n = min(2, cur.kb1 - cur.kb);  // K steps in this pair
+      for (int h = 0; h < n; ++h) {
+        if (ct == 0) {
+          int go = !p.test_stall && (h > 0 || mbar_wait(&s.lfull[l], lphase, abort_flag)) &&
+                   mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag);
+          if (go && h == 0) armed &= ~(1u << l);
+          s.conv_ok = go;
+        }
+        named_bar_sync(1, 32 * kConvWarps);
+        if (!s.conv_ok) {
+          ok = false;
+          break;
+        }
+        convert_tile_w8(land + l * LAND_BYTES + h * 64, ring + stage * STAGE_BYTES + A_TILE, ct);
+        fence_proxy_async_smem();  // generic-proxy writes before the tensor core's reads
+        named_bar_sync(1, 32 * kConvWarps);
+        if (ct == 0) mbar_arrive(&s.full[stage]);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
-      seq_next(cur);
-      if (++stage == STAGES) {
-        stage = 0;
-        phase ^= 1u;
+      if (!ok) break;
+      if (ct == 0 && ahd.u < total) {
+        issue(ahd, l);
+        armed |= 1u << l;
+        lphase_bits = (lphase_bits & ~(1u << l)) | (((lphase + 1u) & 1u) << l);
+        seq_next(ahd);
       }
+      seq_next(cur);
       if (++l == LAND) {
         l = 0;
         lphase ^= 1u;

@@ -29,85 +29,95 @@ using namespace route_detail;
 
 constexpr int kRouteWarps = 8;
 
-// E <= EMAX <= 32, large batches: a set of TPW = 32 / EMAX tokens is routed
-// by kRouteSplit warps, each taking one contiguous part of d for all TPW
-// tokens, so every router-weight vector a warp loads (through L1) serves TPW
-// tokens while the token rows -- the only bytes that must come from HBM --
-// stream with many warps in flight (lanes stride over 16-byte vectors).  In
-// each warp the TPW x EMAX = 32 partial dot products per lane are summed over
-// the warp by a reduce-scatter butterfly (31 shuffles: at each step a lane
-// keeps half of its values and receives the partner's partial sums of that
-// half), after which lane i holds value (token i / EMAX, expert i % EMAX); the
-// warps' values are added in warp order through shared memory, and the set's
-// first warp selects, one shuffle per token handing lane e its expert-e logit.
-constexpr int kRouteWarpsP = 8;
-constexpr int kRouteSplit = 4;  // warps sharing one token set (parts of d)
+// E <= EMAX <= 32, large batches: every warp routes TPW tokens (2 for
+// EMAX = 8, 1 for EMAX = 32) over the whole of d, lanes striding over 16-byte
+// vectors; 8 (EMAX = 8) or 4 vectors of each token are loaded together per
+// lane (a token row's loads in two rounds at d = 4096 in bf16), so the
+// token rows -- the bytes that must come from HBM -- stream with many loads in
+// flight and no block-wide barrier.  The router weights sit in shared memory
+// when they fit in 64 KB (else they are read through L1).  The TPW x EMAX
+// partial dot products of a lane are summed over the warp by a reduce-scatter
+// butterfly (lane i ends with value i: token i / EMAX, expert i % EMAX), then
+// the warp selects its tokens.  The grid is persistent: warps loop over token
+// sets.
+constexpr int kRouteRowWarps = 8;
+constexpr int kRouteWSmemBytes = 64 << 10;
 
-template <typename T, int EMAX>
-__global__ void __launch_bounds__(kRouteWarpsP * 32)
-    route_fused_kernel(int S, int d, const T* __restrict__ x, const T* __restrict__ w_router,
-                       const float* __restrict__ router_bias, SelectParams p) {
-  constexpr int TPW = 32 / EMAX;
-  constexpr int kSets = kRouteWarpsP / kRouteSplit;
-  __shared__ float red[kSets][kRouteSplit][32];
-  const int warp = threadIdx.x >> 5, lane = lane_id();
-  const int set = warp / kRouteSplit, part = warp % kRouteSplit;
-  const int t0 = (blockIdx.x * kSets + set) * TPW;
+template <typename T, int EMAX, bool WSMEM>
+__global__ void __launch_bounds__(kRouteRowWarps * 32, 2)
+    route_rows_kernel(int S, int d, const T* __restrict__ x, const T* __restrict__ w_router,
+                      const float* __restrict__ router_bias, SelectParams p) {
+  constexpr int TPW = EMAX >= 16 ? 1 : 16 / EMAX;
+  constexpr int NV = TPW * EMAX;  // 16 or 32 partial sums per lane
+  constexpr int kRouteBatch = EMAX >= 16 ? 4 : 8;
+  constexpr int kExpertUnroll = (!WSMEM && EMAX >= 16) ? 8 : EMAX;  // W from global: fewer loads in flight
   constexpr int V = Vec16<T>::N;
+  extern __shared__ uint4 wsm[];
+  const int warp = threadIdx.x >> 5, lane = lane_id();
   const int nvec = d / V;
-  const int per_part = (nvec + kRouteSplit - 1) / kRouteSplit;
-  const int v0 = part * per_part, v1 = min(nvec, v0 + per_part);
-  float acc[TPW * EMAX];
-#pragma unroll
-  for (int i = 0; i < TPW * EMAX; ++i) acc[i] = 0.0f;
-  if (t0 < S) {
+  if (WSMEM) {
+    const int n16 = p.E * nvec;
+    for (int i = threadIdx.x; i < n16; i += blockDim.x) wsm[i] = ldg16(w_router + static_cast<int64_t>(i) * V);
+    __syncthreads();
+  }
+  const float bias = (lane < p.E && router_bias != nullptr) ? __ldg(router_bias + lane) : 0.0f;
+  const int num_sets = (S + TPW - 1) / TPW;
+  for (int set = blockIdx.x * kRouteRowWarps + warp; set < num_sets; set += gridDim.x * kRouteRowWarps) {
+    const int t0 = set * TPW;
     const T* xr[TPW];
 #pragma unroll
     for (int tt = 0; tt < TPW; ++tt) xr[tt] = x + static_cast<int64_t>(min(t0 + tt, S - 1)) * d;
-#pragma unroll 2
-    for (int v = v0 + lane; v < v1; v += 32) {
-      float xf[TPW][V];
+    float acc[NV];
 #pragma unroll
-      for (int tt = 0; tt < TPW; ++tt) unpack16<T>(ldg16(xr[tt] + v * V), xf[tt]);
+    for (int i = 0; i < NV; ++i) acc[i] = 0.0f;
+    for (int vb = lane; vb < nvec; vb += 32 * kRouteBatch) {
+      uint4 xv[TPW][kRouteBatch];
 #pragma unroll
-      for (int e = 0; e < EMAX; ++e) {
-        if (e < p.E) {
-          float wf[V];
-          unpack16<T>(ldg16(w_router + static_cast<int64_t>(e) * d + v * V), wf);
+      for (int b = 0; b < kRouteBatch; ++b)
 #pragma unroll
-          for (int tt = 0; tt < TPW; ++tt)
+        for (int tt = 0; tt < TPW; ++tt)
+          xv[tt][b] = (vb + 32 * b < nvec) ? ldg16(xr[tt] + (vb + 32 * b) * V) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-            for (int j = 0; j < V; ++j) acc[tt * EMAX + e] = fmaf(xf[tt][j], wf[j], acc[tt * EMAX + e]);
+      for (int b = 0; b < kRouteBatch; ++b) {
+        const int v = vb + 32 * b;
+        if (v >= nvec) break;
+        float xf[TPW][V];
+#pragma unroll
+        for (int tt = 0; tt < TPW; ++tt) unpack16<T>(xv[tt][b], xf[tt]);
+#pragma unroll kExpertUnroll
+        for (int e = 0; e < EMAX; ++e) {
+          if (e < p.E) {
+            float wf[V];
+            unpack16<T>(WSMEM ? wsm[e * nvec + v] : ldg16(w_router + (static_cast<int64_t>(e) * nvec + v) * V), wf);
+#pragma unroll
+            for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+              for (int j = 0; j < V; ++j) acc[tt * EMAX + e] = fmaf(xf[tt][j], wf[j], acc[tt * EMAX + e]);
+          }
         }
       }
     }
-  }
-  // reduce-scatter over the warp: afterwards acc[0] of lane i is the warp's sum of value i
+    // reduce-scatter over the warp: afterwards acc[0] of lane i is the warp's sum of value i % NV
 #pragma unroll
-  for (int s = 16; s >= 1; s >>= 1) {
-    const bool upper = (lane & s) != 0;
+    for (int s = NV / 2; s >= 1; s >>= 1) {
+      const bool upper = (lane & s) != 0;
 #pragma unroll
-    for (int i = 0; i < s; ++i) {
-      const float send = upper ? acc[i] : acc[i + s];
-      const float keep = upper ? acc[i + s] : acc[i];
-      acc[i] = keep + __shfl_xor_sync(kFull, send, s);
+      for (int i = 0; i < s; ++i) {
+        const float send = upper ? acc[i] : acc[i + s];
+        const float keep = upper ? acc[i + s] : acc[i];
+        acc[i] = keep + __shfl_xor_sync(kFull, send, s);
+      }
     }
-  }
-  red[set][part][lane] = acc[0];
-  __syncthreads();
-  // the set's warps select its tokens in parallel: warp `part` takes tokens
-  // t0 + part, t0 + part + kRouteSplit, ...; a token's logit of expert e is
-  // the sum of the four parts' value tt * EMAX + e, added in part order
-  const float bias = (lane < p.E && router_bias != nullptr) ? __ldg(router_bias + lane) : 0.0f;
-  for (int tt = part; tt < TPW; tt += kRouteSplit) {
-    if (t0 + tt >= S) break;  // warp-uniform
-    float l[1] = {0.0f};
-    if (lane < EMAX) {
 #pragma unroll
-      for (int q = 0; q < kRouteSplit; ++q) l[0] += red[set][q][tt * EMAX + lane];
+    for (int s = NV; s < 32; s <<= 1) acc[0] += __shfl_xor_sync(kFull, acc[0], s);
+#pragma unroll
+    for (int tt = 0; tt < TPW; ++tt) {
+      if (t0 + tt >= S) break;  // warp-uniform
+      float l[1];
+      l[0] = __shfl_sync(kFull, acc[0], tt * EMAX + (lane % EMAX));
+      if (lane < p.E && router_bias != nullptr) l[0] = __fadd_rn(l[0], bias);
+      select_topk<1>(l, p, t0 + tt);
     }
-    if (lane < p.E && router_bias != nullptr) l[0] = __fadd_rn(l[0], bias);
-    select_topk<1>(l, p, t0 + tt);
   }
 }
 
@@ -265,10 +275,9 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
   if (a.S == 0) return cudaSuccess;
   SelectParams sp{a.E,        a.K,      a.score_fn, a.renormalize, a.num_groups,   a.topk_groups, a.tau,
                   a.sel_bias, a.topk_idx, a.topk_w, a.status,      a.cand_key_out, a.score_out};
-  const int blocks = (a.S + kRouteWarps - 1) / kRouteWarps;
   const float* logits = a.logits;
   if (logits == nullptr && a.E <= 32) {
-    // decode-sized batches: a CTA per token; otherwise a warp per token
+    // decode-sized batches: a CTA per token; otherwise warps streaming token rows
     const bool per_cta = a.S <= 512;
     cudaError_t err = cudaSuccess;
 #define MOE_ROUTE_LAUNCH(T, EM)                                                                                \
@@ -277,9 +286,22 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
       err = launch_pdl(route_token_cta_kernel<T, EM>, dim3(a.S), dim3(kRouteTokenWarps * 32), 0, stream, a.d,  \
                        static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);      \
     } else {                                                                                                   \
-      const int per_cta_tokens = (kRouteWarpsP / kRouteSplit) * (32 / EM);                                     \
-      route_fused_kernel<T, EM><<<(a.S + per_cta_tokens - 1) / per_cta_tokens, kRouteWarpsP * 32, 0, stream>>>( \
-          a.S, a.d, static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);         \
+      constexpr int TPW = EM >= 16 ? 1 : 16 / EM;                                                              \
+      const int sets = (a.S + TPW - 1) / TPW;                                                                  \
+      const int want = (sets + kRouteRowWarps - 1) / kRouteRowWarps;                                           \
+      const int cap = (a.num_sms > 0 ? a.num_sms : 148) * 2;                                                   \
+      const int grid = want < cap ? want : cap;                                                                \
+      const size_t wbytes = static_cast<size_t>(a.E) * a.d * sizeof(T);                                        \
+      if (wbytes <= static_cast<size_t>(kRouteWSmemBytes)) {                                                   \
+        err = cudaFuncSetAttribute(route_rows_kernel<T, EM, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                   kRouteWSmemBytes);                                                          \
+        if (err == cudaSuccess)                                                                                \
+          route_rows_kernel<T, EM, true><<<grid, kRouteRowWarps * 32, wbytes, stream>>>(                        \
+              a.S, a.d, static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);     \
+      } else {                                                                                                 \
+        route_rows_kernel<T, EM, false><<<grid, kRouteRowWarps * 32, 0, stream>>>(                              \
+            a.S, a.d, static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);       \
+      }                                                                                                        \
     }                                                                                                          \
   } while (0)
     if (a.act_dtype == MOE_BF16) {
