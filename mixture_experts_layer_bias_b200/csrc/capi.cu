@@ -33,7 +33,7 @@ size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 struct Layout {
   size_t status, logits, chunk_hist, groups, counts, offsets, topk_idx, topk_w, row_of_slot,
       token_of_row, x_perm, hidden, y_perm, wdeq, ksplit, partial, partial_bytes, qa, sa, qas, sas, qh, sh, rr_key,
-      rr_score, rr_ex, rr_claim, rr_list, rr_changed, total;
+      rr_score, rr_ex, rr_pick8, rr_exl, rr_excount, rr_claim, rr_list, rr_changed, total;
 };
 
 // Split-K of the tensor-core GEMMs is available to small row spaces (decode-
@@ -101,12 +101,15 @@ Layout make_layout(const moe_desc& d) {
   L.sas = take(w8a8 && d.num_shared ? static_cast<size_t>(S) * 4 : 0);
   L.qh = take(w8a8 ? static_cast<size_t>(Rt * h) : 0);
   L.sh = take(w8a8 ? static_cast<size_t>(Rt) * 4 : 0);
-  // re-routing: every expert's selection key and gate source, the slots' picks, token claims and lists,
-  // changed tokens
+  // re-routing: every expert's selection key and gate source, the slots' picks, the excess-slot list and
+  // its count, token claims and lists, changed tokens
   const bool rr = d.reroute == 1;
   L.rr_key = take(rr ? static_cast<size_t>(S * E) * 4 : 0);
   L.rr_score = take(rr ? static_cast<size_t>(S * E) * 4 : 0);
   L.rr_ex = take(rr ? static_cast<size_t>(S * K) * 4 : 0);
+  L.rr_pick8 = take(rr ? (static_cast<size_t>(S * K) + 15) & ~size_t(15) : 0);
+  L.rr_exl = take(rr ? static_cast<size_t>(S * K) * 4 : 0);
+  L.rr_excount = take(rr ? 4 : 0);
   L.rr_claim = take(rr ? static_cast<size_t>(S) * 4 : 0);
   L.rr_list = take(rr ? static_cast<size_t>(S) * 4 : 0);
   L.rr_changed = take(rr ? static_cast<size_t>(S) * 4 : 0);
@@ -431,9 +434,10 @@ moe_status reroute_impl(const moe_desc& d, int32_t* topk_idx, float* topk_w, con
                         const int32_t* row_of_slot, void* ws, cudaStream_t st) {
   const Layout L = make_layout(d);
   int32_t* changed = at<int32_t>(ws, L.rr_changed);
+  RerouteScratch scratch{at<int32_t>(ws, L.rr_ex),      at<int8_t>(ws, L.rr_pick8), at<int32_t>(ws, L.rr_exl),
+                         at<int32_t>(ws, L.rr_excount), at<int32_t>(ws, L.rr_claim), at<int32_t>(ws, L.rr_list)};
   cudaError_t e = launch_reroute_assign(d.num_tokens, d.num_experts, d.top_k, d.capacity, topk_idx,
-                                        at<float>(ws, L.rr_key), counts, row_of_slot, at<int32_t>(ws, L.rr_ex),
-                                        at<int32_t>(ws, L.rr_claim), at<int32_t>(ws, L.rr_list), changed,
+                                        at<float>(ws, L.rr_key), counts, row_of_slot, scratch, changed,
                                         at<StatusBlock>(ws, L.status), st);
   if (e == cudaSuccess)
     e = launch_reroute_gates(d.num_tokens, d.num_experts, d.top_k, d.score_fn, d.renormalize,

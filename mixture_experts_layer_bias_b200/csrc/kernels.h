@@ -36,12 +36,18 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream);
 // Excess slots (row_of_slot >= E*C after a capacity-bounded permutation) move,
 // in (token, k) order, to the best-keyed candidate expert with room that the
 // token does not hold; changed[t] marks tokens with a moved slot.  A multi-CTA
-// pick kernel, then one CTA running the epochs.  pick_scratch: int32 [S*K],
-// 16-byte aligned; claim_scratch, list_scratch: int32 [S].
+// pick kernel, one CTA running the epochs, a multi-CTA apply kernel.
+struct RerouteScratch {
+  int32_t* pick;      // [S*K], 16-byte aligned
+  int8_t* pick8;      // [S*K] rounded up to 16, 16-byte aligned: a byte copy of the picks (E <= 127)
+  int32_t* ex;        // [S*K], 16-byte aligned: the excess slots
+  int32_t* ex_count;  // one int
+  int32_t* claim;     // [S]
+  int32_t* list;      // [S]
+};
 cudaError_t launch_reroute_assign(int S, int E, int K, int capacity, int32_t* topk_idx, const float* cand_key,
-                                  const int32_t* counts, const int32_t* row_of_slot, int32_t* pick_scratch,
-                                  int32_t* claim_scratch, int32_t* list_scratch, int32_t* changed,
-                                  StatusBlock* status, cudaStream_t stream);
+                                  const int32_t* counts, const int32_t* row_of_slot, const RerouteScratch& w,
+                                  int32_t* changed, StatusBlock* status, cudaStream_t stream);
 // Gates of the tokens marked in changed[], recomputed over their final experts
 // from the gate sources (the same formulas as the routing kernels).
 cudaError_t launch_reroute_gates(int S, int E, int K, int score_fn, int renormalize, const float* score,
