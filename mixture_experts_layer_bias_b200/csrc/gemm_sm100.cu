@@ -69,6 +69,8 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;
 // E4M3 weights with bf16 activations (W8): eight more warps decode each landed
 // E4M3 weight tile into the bf16 B tile of its stage.
 constexpr int kConvWarps = 8;
+constexpr int kConvGroups = 2;  // the two K steps of a landing buffer are decoded side by side
+constexpr int kGroupThreads = 32 * kConvWarps / kConvGroups;
 constexpr int kThreadsW8 = kThreads + 32 * kConvWarps;
 constexpr int kMaxLandStages = 8;          // landing buffers of E4M3 weight tiles (at most)
 constexpr int LAND_BYTES = 256 * 128;      // 256 weight rows x 128 E4M3 codes (two bf16 K steps)
@@ -85,7 +87,9 @@ struct SmemCtl {
   uint64_t full[MAX_STAGES];
   uint64_t empty[MAX_STAGES];
   uint64_t lfull[kMaxLandStages];  // W8: an E4M3 weight tile has landed
-  int conv_ok;                  // W8: the converters' shared go / give-up decision
+  uint64_t ldone[kMaxLandStages];  // W8: the first K step of a two-step landing buffer is decoded
+  int land_parity[kMaxLandStages]; // W8: parity of the latest copy into each landing buffer (-1: none)
+  int conv_ok[kConvGroups];        // W8: each converter group's shared go / give-up decision
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -283,17 +287,16 @@ __device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint3
       : "r"(w));
 }
 
-// W8: the converter threads (kConvWarps warps) decode the 64 codes of one K
-// step from each of the 256 rows of a landing buffer (rows of 128 bytes, two
-// K steps; `land` points at the step's first code of row 0) into the stage's
-// 256 x 128-byte bf16 B tile in the 128-byte swizzled layout the MMA reads
-// (16-byte chunk j of row r at chunk j ^ (r & 7)).  Thread ct takes the
-// 16-code pieces ct + 32 kConvWarps i.
-__device__ __forceinline__ void convert_tile_w8(const uint8_t* land, uint8_t* b16, int ct) {
-  constexpr int kConvThreads = 32 * kConvWarps;
+// W8: one converter group (kGroupThreads threads) decodes the 64 codes of
+// one K step from each of the 256 rows of a landing buffer (rows of 128
+// bytes, two K steps; `land` points at the step's first code of row 0) into
+// the stage's 256 x 128-byte bf16 B tile in the 128-byte swizzled layout the
+// MMA reads (16-byte chunk j of row r at chunk j ^ (r & 7)).  Thread gt takes
+// the 16-code pieces gt + kGroupThreads i.
+__device__ __forceinline__ void convert_tile_w8(const uint8_t* land, uint8_t* b16, int gt) {
 #pragma unroll 2
-  for (int i = 0; i < 1024 / kConvThreads; ++i) {
-    const int piece = ct + kConvThreads * i;  // 1024 pieces of 16 codes
+  for (int i = 0; i < 1024 / kGroupThreads; ++i) {
+    const int piece = gt + kGroupThreads * i;  // 1024 pieces of 16 codes
     const int r = piece >> 2, q4 = piece & 3;
     const uint4 v = *reinterpret_cast<const uint4*>(land + r * 128 + q4 * 16);
     uint32_t o[8];
@@ -341,7 +344,11 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
         mbar_init(&s.empty[i], 1);
       }
       if (W8)
-        for (int i = 0; i < LAND; ++i) mbar_init(&s.lfull[i], 1);
+        for (int i = 0; i < LAND; ++i) {
+          mbar_init(&s.lfull[i], 1);
+          mbar_init(&s.ldone[i], 1);
+          s.land_parity[i] = -1;
+        }
       for (int i = 0; i < 2; ++i) {
         mbar_init(&s.tfull[i], 1);
         mbar_init(&s.tempty[i], 32 * kEpiWarps);
@@ -497,17 +504,19 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
     }
     __syncwarp();
   } else if (W8 && warp >= 2 + kEpiWarps) {
-    // W8 converters.  A landing buffer holds the E4M3 codes of two K steps
-    // of a weight tile (256 rows x 128 bytes: DRAM reads of 128 contiguous
-    // bytes per row).  For every K step of this CTA's units (the producer's
-    // and the MMA warp's order) wait for its codes to land and for the stage's
-    // B tile to be free, decode them, then let the MMA go (second arrival on
-    // the stage's full barrier); a landing buffer is refilled with the pair
-    // LAND pairs ahead once both of its K steps are decoded.  One thread
-    // waits on the barriers and issues the copies; the decision to go on or
-    // give up reaches all converter threads through shared memory, so they
-    // leave together.
+    // W8 converters, two groups of four warps.  A landing buffer holds the
+    // E4M3 codes of two K steps of a weight tile (256 rows x 128 bytes: DRAM
+    // reads of 128 contiguous bytes per row); group 0 decodes the first K
+    // step, group 1 the second, side by side.  For its K step a group waits
+    // for the codes to land and for the stage's B tile to be free, decodes,
+    // then lets the MMA go (second arrival on the stage's full barrier).  The
+    // group decoding a buffer's last K step refills it with the pair LAND
+    // pairs ahead (group 1 first waits for group 0's half: ldone).  Both
+    // groups walk the whole K-step sequence, so they agree on stages, phases
+    // and buffers.  Each group's first thread waits on the barriers; the go /
+    // give-up decision reaches the group through shared memory.
     const int ct = threadIdx.x - (2 + kEpiWarps) * 32;
+    const int g = ct / kGroupThreads, gt = ct % kGroupThreads;
     // the sequence of K-step pairs, walked twice: `cur` for decoding, `ahd` for issuing copies
     struct Seq {
       int u, kb, kb1;  // unit, first K step of the pair, end of the unit's K range
@@ -536,10 +545,11 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
         q.u += gridDim.x;
       }
     };
-    auto issue = [&](const Seq& q, int l) {  // E4M3 codes of pair q into landing buffer l
+    auto issue = [&](const Seq& q, int l, uint32_t parity) {  // E4M3 codes of pair q into landing buffer l
       const UnitInfo ui = decode_unit(s, p, q.u, ks, nk);
       const int b_row = ui.ti.grp.expert * p.n_per_slab + ui.ti.n_idx * p.bn_out;
       uint8_t* dst = land + l * LAND_BYTES;
+      s.land_parity[l] = static_cast<int>(parity);
       mbar_arrive_expect_tx(&s.lfull[l], LAND_BYTES);
       if (EPI == EPI_SWIGLU) {
         tma_load_2d(dst, &tmB0, q.kb * BK, b_row, &s.lfull[l]);
@@ -552,60 +562,71 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
     Seq cur, ahd;
     seq_begin(cur);
     seq_begin(ahd);
-    uint32_t armed = 0;  // landing buffers with a copy in flight
-    uint32_t lphase_bits = 0;
-    if (ct == 0 && !p.test_stall) {
+    if (g == 0 && gt == 0 && !p.test_stall) {
       for (int l = 0; l < LAND && ahd.u < total; ++l) {
-        issue(ahd, l);
-        armed |= 1u << l;
+        issue(ahd, l, 0u);
         seq_next(ahd);
       }
+    } else {
+      for (int l = 0; l < LAND && ahd.u < total; ++l) seq_next(ahd);
     }
     int stage = 0, l = 0;
-    uint32_t phase = 0, lphase = 0;
+    uint32_t phase = 0, lphase = 0, ld_bits = 0;
     bool ok = true;
     while (cur.u < total && ok) {
       const int n = min(2, cur.kb1 - cur.kb);  // K steps in this pair
       for (int h = 0; h < n; ++h) {
-        if (ct == 0) {
-          int go = !p.test_stall && (h > 0 || mbar_wait(&s.lfull[l], lphase, abort_flag)) &&
-                   mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag);
-          if (go && h == 0) armed &= ~(1u << l);
-          s.conv_ok = go;
+        if (h == g) {
+          if (gt == 0) {
+            const int go = !p.test_stall && mbar_wait(&s.lfull[l], lphase, abort_flag) &&
+                           mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag);
+            s.conv_ok[g] = go;
+          }
+          named_bar_sync(1 + g, kGroupThreads);
+          if (!s.conv_ok[g]) {
+            ok = false;
+            break;
+          }
+          convert_tile_w8(land + l * LAND_BYTES + h * 64, ring + stage * STAGE_BYTES + A_TILE, gt);
+          fence_proxy_async_smem();  // generic-proxy writes before the tensor core's reads
+          named_bar_sync(1 + g, kGroupThreads);
+          if (gt == 0) {
+            mbar_arrive(&s.full[stage]);
+            if (g == 0 && n == 2) mbar_arrive(&s.ldone[l]);
+          }
         }
-        named_bar_sync(1, 32 * kConvWarps);
-        if (!s.conv_ok) {
-          ok = false;
-          break;
-        }
-        convert_tile_w8(land + l * LAND_BYTES + h * 64, ring + stage * STAGE_BYTES + A_TILE, ct);
-        fence_proxy_async_smem();  // generic-proxy writes before the tensor core's reads
-        named_bar_sync(1, 32 * kConvWarps);
-        if (ct == 0) mbar_arrive(&s.full[stage]);
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
         }
       }
       if (!ok) break;
-      if (ct == 0 && ahd.u < total) {
-        issue(ahd, l);
-        armed |= 1u << l;
-        lphase_bits = (lphase_bits & ~(1u << l)) | (((lphase + 1u) & 1u) << l);
-        seq_next(ahd);
+      // the group that decoded the pair's last K step refills the buffer
+      if (g == n - 1 && gt == 0 && ahd.u < total) {
+        if (n == 2 && !mbar_wait(&s.ldone[l], (ld_bits >> l) & 1u, abort_flag)) {
+          ok = false;
+        } else {
+          issue(ahd, l, (lphase + 1u) & 1u);
+        }
       }
+      if (n == 2) ld_bits ^= 1u << l;
+      if (g == n - 1 && gt == 0) s.conv_ok[g] = ok;
+      named_bar_sync(1 + g, kGroupThreads);
+      if (g == n - 1 && !s.conv_ok[g]) ok = false;
+      if (!ok) break;
+      seq_next(ahd);
       seq_next(cur);
       if (++l == LAND) {
         l = 0;
         lphase ^= 1u;
       }
     }
-    if (!ok && ct == 0) {
+    if (!ok && gt == 0) {
       *abort_flag = 1;
       report(p.status, MOE_STATUS_TIMEOUT, MOE_CNT_TIMEOUT);
       // let the copies already issued land before the CTA exits
       for (int i = 0; i < LAND; ++i)
-        if (armed & (1u << i)) wait_timed(&s.lfull[i], (lphase_bits >> i) & 1u);
+        if (s.land_parity[i] >= 0) wait_timed(&s.lfull[i], static_cast<uint32_t>(s.land_parity[i]));
     }
   } else {
     const int q = warp & 3;                // TMEM lane quarter this warp may access

@@ -28,7 +28,10 @@ from mixture_experts_layer_bias_b200.build import TEST_HOOKS_LIB
 ops._LIB_PATH = TEST_HOOKS_LIB
 ops.lib().moe_test_stall_gemms(1)
 from parity import run_layer, compare_layer
-cfg = syn.scaled(syn.CONFIGS["mixtral_prefill"], S=64, d=256, h=256)
+if {e4m3!r}:   # E4M3 weights decoded inside the GEMM: its converter warps must give up too
+    cfg = syn.scaled(syn.VARIANTS["mixtral_decode_e4m3"], S=4, d=256, h=384)
+else:
+    cfg = syn.scaled(syn.CONFIGS["mixtral_prefill"], S=64, d=256, h=256)
 inp = syn.make_inputs(cfg, "cuda", seed=0)
 first = run_layer(inp, cfg)                     # its first GEMM launch stalls
 code1, flags1, cnt1 = ops.moe_get_status(first["ws"])
@@ -41,8 +44,9 @@ print("RESULT " + json.dumps(dict(code1=code1, flags1=flags1, timeouts=cnt1["tim
 """
 
 
-def test_bounded_wait_gives_up_and_context_survives():
-    code = CHILD.format(root=ROOT, tests=os.path.join(ROOT, "tests"))
+@pytest.mark.parametrize("e4m3", [False, True])
+def test_bounded_wait_gives_up_and_context_survives(e4m3):
+    code = CHILD.format(root=ROOT, tests=os.path.join(ROOT, "tests"), e4m3=e4m3)
     r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-3000:]
     line = [l for l in r.stdout.splitlines() if l.startswith("RESULT ")][-1]
