@@ -72,9 +72,9 @@ GEMM_TRAFFIC_CAPTURE = {
     "workload": "mixtral_prefill",
     # dram__bytes_read.sum + dram__bytes_write.sum of the up and down GEMM launches of one layer call,
     # one-pass ncu capture of the full-size workload (None: not captured on the current GEMM sources)
-    "bytes": None,
+    "bytes": 3669935616,  # 1947710464 + 228175616 (up) + 1432751360 + 61298176 (down)
     "sources": ("common.cuh", "gemm_common.cuh", "gemm_sm100.cu"),
-    "sha1": None,
+    "sha1": "563130c49bd44542c11bfafe51775933c0eeb9b2",
 }
 
 
@@ -132,7 +132,9 @@ def kernels_per_step(cfg, S=None):
     small = S * cfg.K <= 4096               # one-CTA permutation for small batches
     n = 1 if (cfg.E <= 32) else 2          # route (logits in the routing kernel) or logits GEMM + top-k
     n += 1 if small else 4                 # permutation (+ group table): one kernel, or count, scan, scatter, groups
-    n += 1                                 # row gather (quantising for W8A8)
+    elem = 4 if cfg.act_dtype == syn.F32 else 2
+    if cfg.act_quant or not (small and S * cfg.K * cfg.d * elem <= 256 * 1024):
+        n += 1                             # row gather (quantising for W8A8); tiny batches: inside the permutation
     n += 2                                 # up and down GEMM
     rows = S * cfg.K + cfg.num_shared * S + (cfg.E * cfg.capacity if cfg.capacity else 0)
     if cfg.act_dtype == syn.BF16 and rows <= 4096:
@@ -142,7 +144,7 @@ def kernels_per_step(cfg, S=None):
     elif cfg.weight_dtype == syn.E4M3 and (cfg.d % 16 or cfg.h % 16 or S * cfg.K > W8_IN_GEMM_ROWS * cfg.E):
         n += 3                             # E4M3 -> bf16 decode of the three stacks (else inside the GEMMs)
     if cfg.reroute:
-        n += (1 if small else 3) + 3       # ranks, re-route picks and epochs, gates
+        n += (1 if small else 3) + 4       # ranks, re-route picks, epochs and apply, gates
     n += 1                                 # combine
     return n
 

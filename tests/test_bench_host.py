@@ -38,10 +38,11 @@ def test_committed_traffic_record_is_current_or_absent():
     ("dsv3_grouped", None, 2 + 4 + 1 + 2 + 1),              # router GEMM + top-k
     ("fp8_skew_capacity", None, 2 + 4 + 1 + 2 + 3 + 1),     # E = 64: router GEMM + top-k; 2048 rows per expert: decode pass
     ("mixtral_prefill_w8a8", None, 1 + 4 + 1 + 2 + 1 + 1),  # + quantisation of the hidden rows
-    ("fp8_skew_capacity_reroute", None, 2 + 4 + 1 + 2 + 3 + 6 + 1),  # + ranks (3), picks, epochs, gates
-    ("mixtral_decode", 1, 1 + 1 + 1 + 2 + 2 + 1),           # one-CTA permutation, split-K finalizes
-    ("mixtral_decode", 32, 1 + 1 + 1 + 2 + 2 + 1),
-    ("tiny_f32", None, 1 + 1 + 1 + 2 + 1),                  # fp32: no split-K
+    ("fp8_skew_capacity_reroute", None, 2 + 4 + 1 + 2 + 3 + 7 + 1),  # + ranks (3), picks, epochs, apply, gates
+    ("mixtral_decode", 1, 1 + 1 + 2 + 2 + 1),               # one-CTA permutation with the gather, split-K finalizes
+    ("mixtral_decode", 8, 1 + 1 + 2 + 2 + 1),               # 8 x 2 rows of 8 KB: gathered by the permutation
+    ("mixtral_decode", 32, 1 + 1 + 1 + 2 + 2 + 1),          # 512 KB of rows: the gather kernel
+    ("tiny_f32", None, 1 + 1 + 2 + 1),                      # fp32: no split-K; 64 x 2 rows of 512 B: folded gather
 ])
 def test_kernels_per_layer_call(name, S, expected):
     cfg = syn.CONFIGS.get(name) or syn.VARIANTS[name]
