@@ -381,7 +381,9 @@ struct CommitSmem {
   uint32_t full[kMaskWords];  // experts that ran out of room in this epoch
   int min_seg, min_sub;
   long long first_bad;
-  int nlist;  // tokens listed for re-picking in this epoch
+  int nlist;     // tokens listed for re-picking in this epoch
+  int nf;        // experts that ran out of room in this epoch, and the first four of them
+  int flist[4];
 };
 
 // The excess slots of token t from slot `first` on pick again, in k order: a
@@ -482,6 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       sm.min_sub = kSegs;
       sm.first_bad = nslots;
       sm.nlist = 0;
+      sm.nf = 0;
     }
     for (int e = tid; e < E; e += kThreads) {
       int seg = kSegs, acc = 0, need = 0;
@@ -595,7 +598,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     start = P;
     // 4. experts left without room drop out
     for (int e = tid; e < E; e += kThreads)
-      if (bit_of(sm.avail, e) && sm.room[e] <= 0) atomicOr(&sm.full[e >> 5], 1u << (e & 31));
+      if (bit_of(sm.avail, e) && sm.room[e] <= 0) {
+        atomicOr(&sm.full[e >> 5], 1u << (e & 31));
+        const int i = atomicAdd(&sm.nf, 1);
+        if (i < 4) sm.flist[i] = e;
+      }
     __syncthreads();
     if (tid < kMaskWords) sm.avail[tid] &= ~sm.full[tid];
     __syncthreads();
@@ -608,10 +615,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t = static_cast<int>(s / K);
       if (atomicMax(&claim[t], epoch + 1) < epoch + 1) list[atomicAdd(&sm.nlist, 1)] = t;
     };
-    if constexpr (SM)
-      pick.for_range(P, nslots, tid, kThreads, claim_slot);
-    else
+    if constexpr (SM) {
+      if (sm.nf <= 4 && 16 % K == 0) {
+        // a 16-slot piece holds whole tokens, so one thread sees all of a
+        // token's slots and lists it without a claim; four picks per word are
+        // compared at once with the (at most four) experts that filled up
+        uint32_t fb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) fb[i] = 0x01010101u * static_cast<uint32_t>(sm.flist[i < sm.nf ? i : 0]);
+        const uint4* s4 = reinterpret_cast<const uint4*>(pick.s);
+        const uint32_t tmask = (K >= 16) ? 0xFFFFu : ((1u << K) - 1u);
+        for (int64_t q = (P >> 4) + tid; q < ((nslots + 15) >> 4); q += kThreads) {
+          const uint4 v = s4[q];
+          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+          uint32_t hit = 0;  // bit c: slot q*16 + c picked a full expert
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t m = 0;
+#pragma unroll
+            for (int f = 0; f < 4; ++f) m |= __vcmpeq4(wv[i], fb[f]);
+            hit |= ((m & 1u) | ((m >> 7) & 2u) | ((m >> 14) & 4u) | ((m >> 21) & 8u)) << (4 * i);
+          }
+          if (hit == 0) continue;
+          const int64_t s_lo = q * 16;
+          if (s_lo < P) hit &= ~((1u << static_cast<int>(P - s_lo)) - 1u);  // committed slots
+          if (s_lo + 16 > nslots) hit &= (1u << static_cast<int>(nslots - s_lo)) - 1u;
+          for (int c0 = 0; c0 < 16; c0 += K)
+            if ((hit >> c0) & tmask) list[atomicAdd(&sm.nlist, 1)] = static_cast<int>((s_lo + c0) / K);
+        }
+      } else {
+        pick.for_range(P, nslots, tid, kThreads, claim_slot);
+      }
+    } else {
       for_excess(ex, n_ex, pick_g, tid, kThreads, claim_slot);
+    }
     __syncthreads();
     const int nl = sm.nlist;
     for (int i = tid; i < nl; i += kThreads) {
