@@ -387,7 +387,9 @@ def decode_sweep(base_inp, device, peaks, reps=20, dcfg0=None):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=s):
             run.call(stream=s)
-        g.replay()
+        # untimed replays first (tens of ms), so that the clocks have left any idle state
+        for _ in range(100):
+            g.replay()
         torch.cuda.synchronize()
         # five batches of `reps` replays; the median batch's time per call
         batches = []
@@ -679,6 +681,9 @@ def main():
     bias_us = time_bias_update(cfg, device, S)
     dec = dec8 = None
     if not args.no_decode and args.workload == WORKLOAD:
+        # right after the power-capped prefill loop the clocks are still held down for a
+        # moment; the decode sweep measures the steady decode regime after a short pause
+        time.sleep(3.0)
         dec = decode_sweep(run.inp, device, peaks)
     inp = run.inp
     del run
