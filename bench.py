@@ -74,7 +74,7 @@ GEMM_TRAFFIC_CAPTURE = {
     # one-pass ncu capture of the full-size workload (None: not captured on the current GEMM sources)
     "bytes": 3669935616,  # 1947710464 + 228175616 (up) + 1432751360 + 61298176 (down)
     "sources": ("common.cuh", "gemm_common.cuh", "gemm_sm100.cu"),
-    "sha1": "563130c49bd44542c11bfafe51775933c0eeb9b2",
+    "sha1": "d2bc3eb5235db093b2f9627641f98a3e7983c2c7",
 }
 
 

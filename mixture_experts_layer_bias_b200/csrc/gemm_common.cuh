@@ -1,6 +1,6 @@
 // Pieces shared by the tensor-core grouped GEMM kernel: launch parameters,
-// group lookup, the device-side split-K choice, the split-K reduction of the
-// last-arriving slice and tensor-map encoding.
+// group lookup, the device-side split-K choice, the split-K finalize kernel
+// and tensor-map encoding.
 #pragma once
 
 #include <math.h>
