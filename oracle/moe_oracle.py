@@ -761,6 +761,48 @@ def quantize_rows_e4m3(rows: np.ndarray):
     return f32_to_e4m3_bits(ratio), s
 
 
+def split_rows_e4m3(rows: np.ndarray):
+    """Two-term E4M3 codes of float32 rows holding bf16 values: the
+    activation operand of E4M3-weight layers with bf16 activations.  The
+    pages give E4M3 only as the expert weights' storage format (ybb.press
+    3.3); the library's tensor-core GEMMs have no bf16 x E4M3 product, so it
+    writes each bf16 value as a power-of-two multiple of the sum of two E4M3
+    values.  Per row:
+
+        k  = the largest integer with amax * 2**k <= 448 (0 for an all-zero
+             row), clamped to [-126, 126]
+        v  = x * 2**k                 (float32 product)
+        c1 = E4M3(v)                  (round to nearest even)
+        c2 = E4M3(v - value(c1))      (float32 difference)
+        scale = 2**-k                 (NaN when the row holds an inf or NaN;
+                                       v = x * 0 then)
+
+    Returns (c1 uint8 [n, d], c2 uint8 [n, d], scale float32 [n]); the row is
+    (value(c1) + value(c2)) * scale."""
+    x = np.asarray(rows, dtype=np.float32)
+    n, d = x.shape
+    c1 = np.zeros((n, d), dtype=np.uint8)
+    c2 = np.zeros((n, d), dtype=np.uint8)
+    scale = np.zeros(n, dtype=np.float32)
+    for i in range(n):
+        row = x[i]
+        if not np.all(np.isfinite(row)):
+            mult, scale[i] = np.float32(0.0), np.float32(np.nan)
+        else:
+            amax = float(np.max(np.abs(row.astype(np.float64)))) if d else 0.0
+            k = 0
+            if amax > 0.0:
+                f, ex = math.frexp(amax)  # amax = f * 2**ex, f in [0.5, 1); 448 = 0.875 * 2**9
+                k = (9 if f <= 0.875 else 8) - ex
+                k = max(-126, min(126, k))
+            mult, scale[i] = np.float32(math.ldexp(1.0, k)), np.float32(math.ldexp(1.0, -k))
+        v = np.multiply(row, mult, dtype=np.float32)
+        c1[i] = f32_to_e4m3_bits(v)
+        rest = np.subtract(v, e4m3_bits_to_f64(c1[i]).astype(np.float32), dtype=np.float32)
+        c2[i] = f32_to_e4m3_bits(rest)
+    return c1, c2, scale
+
+
 def expert_swiglu_w8a8(x, q_gate, q_up, q_down, s_gate, s_up, s_down, round_hidden_bf16=True):
     """SwiGLU expert with E4M3 weights (per-output-channel scales) applied to
     E4M3-quantised activations: x rows are quantised per row

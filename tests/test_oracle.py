@@ -609,6 +609,65 @@ def test_quantize_rows_round_trip_error_bound():
     assert np.all(np.abs(O.e4m3_bits_to_f64(q[np.arange(50), top]))[nz] == 448.0)
 
 
+def _bf16_rows(rng, n, d, spread):
+    """Random float32 rows holding bf16 values: |x| = amax_row * 2**-u, u
+    uniform in [0, spread), random signs, bf16 mantissas."""
+    amax = np.exp2(rng.integers(-20, 20, size=(n, 1))) * rng.uniform(1, 2, size=(n, 1))
+    x = amax * np.exp2(-rng.uniform(0, spread, size=(n, d))) * rng.choice([-1.0, 1.0], size=(n, d))
+    return O.bf16_bits_to_f64(O.f64_to_bf16_bits(x)).astype(np.float32)
+
+
+def test_split_rows_hand_example():
+    """x = [1 + 2**-7, -0.5, 0, 3]: amax 3 = 0.75 * 2**2, so k = 7 (3 * 2**7 =
+    384 <= 448 < 768); v = [129, -64, 0, 384].  129 lies on the grid of
+    spacing 16 in [128, 256) and rounds to 128 = code 0x70 (exponent field
+    14), leaving 1 = code 0x38; -64 = code 0xE8, 384 = 1.5 * 2**8 = code 0x7C,
+    all exact; scale 2**-7."""
+    c1, c2, s = O.split_rows_e4m3(np.array([[1.0078125, -0.5, 0.0, 3.0]], np.float32))
+    assert list(c1[0]) == [0x70, 0xE8, 0x00, 0x7C]
+    assert list(c2[0]) == [0x38, 0x00, 0x00, 0x00]
+    assert s[0] == np.float32(2.0 ** -7)
+
+
+def test_split_rows_reconstruct_bf16_exactly():
+    """Every bf16 value of at least 2**-9 of its row's largest magnitude is
+    the exact sum of its two terms times the row scale (the scaled value is at
+    least 224 * 2**-9 > 1/4, so the remainder after the first term, at most 4
+    significant bits, lies on the E4M3 grid); the scale is the largest power
+    of two bringing the row maximum to at most 448."""
+    rng = np.random.default_rng(31)
+    x = _bf16_rows(rng, 40, 96, 9.0)
+    c1, c2, s = O.split_rows_e4m3(x)
+    v1, v2 = O.e4m3_bits_to_f64(c1), O.e4m3_bits_to_f64(c2)
+    assert np.array_equal((v1 + v2) * s[:, None].astype(np.float64), x.astype(np.float64))
+    top = np.max(np.abs(x.astype(np.float64)), axis=1) / s
+    assert np.all((top > 224.0) & (top <= 448.0))
+    # the first term alone is the value rounded to 4 significant bits
+    assert np.all(np.abs(v2) <= np.abs(v1) * 2.0 ** -4)
+
+
+def test_split_rows_error_bound_and_special_rows():
+    """Values far below the row maximum lose at most 2**-10 of the scaled
+    value (half the E4M3 subnormal spacing); a zero row has scale 1 and zero
+    codes; a row maximum of exactly 448 * 2**j gives scale 2**j; a row with an
+    infinity or a NaN gets the scale NaN."""
+    rng = np.random.default_rng(32)
+    x = _bf16_rows(rng, 30, 128, 30.0)
+    c1, c2, s = O.split_rows_e4m3(x)
+    v = x.astype(np.float64) / s[:, None]
+    err = np.abs(O.e4m3_bits_to_f64(c1) + O.e4m3_bits_to_f64(c2) - v)
+    assert np.all(err <= 2.0 ** -10)
+    assert np.any(err > 0)  # the spread reaches below the exact range
+    y = np.zeros((4, 16), np.float32)
+    y[1, 3] = 448.0 * 8
+    y[2, 5] = np.inf
+    y[3, 0] = np.nan
+    c1, c2, s = O.split_rows_e4m3(y)
+    assert s[0] == 1.0 and not c1[0].any() and not c2[0].any()
+    assert s[1] == 8.0 and c1[1, 3] == 0x7E and c2[1, 3] == 0
+    assert np.isnan(s[2]) and np.isnan(s[3])
+
+
 def test_w8a8_expert_close_to_exact_expert():
     """With 8-bit activations the expert output stays within the quantisation
     noise of the same expert on unquantised activations (relative L2 a few
