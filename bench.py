@@ -72,9 +72,9 @@ GEMM_TRAFFIC_CAPTURE = {
     "workload": "mixtral_prefill",
     # dram__bytes_read.sum + dram__bytes_write.sum of the up and down GEMM launches of one layer call,
     # one-pass ncu capture of the full-size workload (None: not captured on the current GEMM sources)
-    "bytes": 3669935616,  # 1947710464 + 228175616 (up) + 1432751360 + 61298176 (down)
+    "bytes": None,
     "sources": ("common.cuh", "gemm_common.cuh", "gemm_sm100.cu"),
-    "sha1": "d2bc3eb5235db093b2f9627641f98a3e7983c2c7",
+    "sha1": None,
 }
 
 
@@ -121,9 +121,11 @@ def workload_desc(cfg):
             f"{', W8A8 (e4m3 activation rows, per-row scales)' if cfg.act_quant else ''}")
 
 
-# E4M3 weights with bf16 activations are decoded inside the GEMMs up to this
-# many routed rows per expert on average, above it by a decode pass
-W8_IN_GEMM_ROWS = 1024
+def coded_a_rows(cfg):
+    """The expert GEMMs read E4M3 codes of their A rows: W8A8, or E4M3 weights
+    with bf16 activations (two-term codes; d and h multiples of 16)."""
+    return bool(cfg.act_quant) or (cfg.weight_dtype == syn.E4M3 and cfg.act_dtype == syn.BF16
+                                   and cfg.d % 16 == 0 and cfg.h % 16 == 0)
 
 
 def kernels_per_step(cfg, S=None):
@@ -133,16 +135,17 @@ def kernels_per_step(cfg, S=None):
     n = 1 if (cfg.E <= 32) else 2          # route (logits in the routing kernel) or logits GEMM + top-k
     n += 1 if small else 4                 # permutation (+ group table): one kernel, or count, scan, scatter, groups
     elem = 4 if cfg.act_dtype == syn.F32 else 2
-    if cfg.act_quant or not (small and S * cfg.K * cfg.d * elem <= 256 * 1024):
-        n += 1                             # row gather (quantising for W8A8); tiny batches: inside the permutation
+    coded = coded_a_rows(cfg)
+    if coded or not (small and S * cfg.K * cfg.d * elem <= 256 * 1024):
+        n += 1                             # row gather (writing E4M3 codes); tiny bf16 batches: inside the permutation
     n += 2                                 # up and down GEMM
     rows = S * cfg.K + cfg.num_shared * S + (cfg.E * cfg.capacity if cfg.capacity else 0)
     if cfg.act_dtype == syn.BF16 and rows <= 4096:
         n += 2                             # split-K finalize of both GEMMs
-    if cfg.act_quant:
-        n += 1                             # per-row E4M3 quantisation of the hidden rows
-    elif cfg.weight_dtype == syn.E4M3 and (cfg.d % 16 or cfg.h % 16 or S * cfg.K > W8_IN_GEMM_ROWS * cfg.E):
-        n += 3                             # E4M3 -> bf16 decode of the three stacks (else inside the GEMMs)
+    if coded:
+        n += 1                             # per-row E4M3 codes of the hidden rows
+    elif cfg.weight_dtype == syn.E4M3:
+        n += 3                             # E4M3 -> bf16 decode of the three stacks (d or h not a multiple of 16)
     if cfg.reroute:
         n += (1 if small else 3) + 4       # ranks, re-route picks, epochs and apply, gates
     n += 1                                 # combine
@@ -350,7 +353,10 @@ def roofline_for(cfg, S, stages, peaks, workload_name):
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     kind = "bf16 burst"
-    if cfg.act_quant:
+    if cfg.weight_dtype == syn.E4M3 and not cfg.act_quant and coded_a_rows(cfg):
+        # two E4M3 MMAs (one per activation term) per product: the fp8 peak / 2, i.e. the bf16 peak
+        kind = "bf16 burst (two-term E4M3 activations: two E4M3 MMAs per product, half the nominal e4m3 rate)"
+    elif cfg.act_quant:
         # E4M3 x E4M3: the measured bf16 peak times the nominal fp8 : bf16 ratio (4.5 : 2.25)
         peak, sustained = 2 * peak, 2 * sustained
         kind = "bf16 burst x 2 (nominal e4m3 : bf16 ratio)"
@@ -690,7 +696,7 @@ def main():
     gc.collect()
     torch.cuda.empty_cache()
     if not args.no_decode and args.workload == WORKLOAD:
-        # the same decode sizes on E4M3 expert weights (decoded inside the GEMMs)
+        # the same decode sizes on E4M3 expert weights (two-term E4M3 activations)
         c8 = syn.VARIANTS["mixtral_decode_e4m3"]
         inp8 = syn.make_inputs(c8, device, seed=0)
         dec8 = decode_sweep(inp8, device, peaks, dcfg0=c8)

@@ -17,6 +17,7 @@
  * Around them: moe_reroute (over-capacity re-routing between two
  * permutations), moe_update_sel_bias (sliding-window selection-bias update),
  * moe_quantize_rows_e4m3 (the W8A8 activation quantiser on its own),
+ * moe_split_rows_e4m3 (the two-term activation codes of E4M3-weight layers),
  * moe_permute_static (moe_permute without a workspace), and the workspace /
  * status helpers.
  *
@@ -101,8 +102,13 @@ typedef enum { MOE_ACT_GELU = 0, MOE_ACT_SWIGLU = 1 } moe_act;
  *     primary block, the rest in an overflow region (ybb.press 2.2,
  *     overflow buffering) whose rows the expert GEMMs process right after
  *     that expert's primary rows.  No token is dropped.
- *   act_quant: 0 = the expert GEMMs read bf16 activations (E4M3 weights are
- *     decoded to bf16 first); 1 = W8A8: each A row of both expert GEMMs
+ *   act_quant: 0 = the expert GEMMs compute on the bf16 activations.  With
+ *     E4M3 weights (d and h multiples of 16) each bf16 A row is written as two
+ *     E4M3 terms with a power-of-two row scale (moe_split_rows_e4m3), exact
+ *     but for elements below about 2^-10.8 of the row's largest magnitude,
+ *     and the GEMMs multiply the stored weight codes by both terms in one
+ *     fp32 sum; otherwise the weights are decoded to bf16 first.
+ *     1 = W8A8: each A row of both expert GEMMs
  *     (the permuted tokens, then the bf16 hidden rows) is quantised to E4M3
  *     with one fp32 scale per row (moe_quantize_rows_e4m3) and the GEMMs run
  *     on 8-bit operands, the epilogue applying row and channel scales.  The
@@ -290,6 +296,29 @@ moe_status moe_reroute(const moe_desc *desc, int32_t *topk_idx, float *topk_w, c
  * the launch fails.  There is no workspace or status block.
  */
 moe_status moe_quantize_rows_e4m3(const void *x, int64_t rows, int32_t d, uint8_t *q, float *s, void *stream);
+
+/*
+ * Two-term E4M3 codes of bf16 rows, the activation step of the E4M3-weight
+ * path with bf16 activations (act_quant = 0), exposed on its own.  The
+ * tensor cores have no bf16 x E4M3 product (ybb.press "MoE 推理工程深层实战"
+ * 3.3 gives E4M3 as the expert weights' storage format), so each bf16 value
+ * becomes two E4M3 terms that the GEMM multiplies with the weight codes.
+ * For each row i of x [rows][d] (bf16, row-major, DEVICE, 16-byte aligned,
+ * d a multiple of 16):
+ *   k       = the largest integer with max_j |x[i][j]| * 2^k <= 448,
+ *             clamped to [-126, 126] (0 for an all-zero row);
+ *   v_j     = x[i][j] * 2^k (exact);
+ *   q[i][j]     = E4M3(v_j), round to nearest even;
+ *   q[i][d + j] = E4M3(v_j - q[i][j]) (the difference exact in fp32);
+ *   s[i]    = 2^-k, or NaN when the row holds an infinity or a NaN.
+ * Then q[i][j] + q[i][d+j] = v_j exactly whenever |v_j| >= 1/4; below that
+ * the error is at most 2^-10 in v_j.  q [rows][2d] uint8 and s [rows] fp32
+ * are caller-owned DEVICE buffers (q 16-byte aligned).  Launches one kernel
+ * on `stream`, allocates nothing.  rows = 0 is a no-op.  Errors:
+ * MOE_ERR_INVALID_ARG for a NULL or misaligned pointer, rows < 0 or d not a
+ * positive multiple of 16; MOE_ERR_CUDA when the launch fails.
+ */
+moe_status moe_split_rows_e4m3(const void *x, int64_t rows, int32_t d, uint8_t *q, float *s, void *stream);
 
 /*
  * Gate-weighted combine back into token order (11.3.1 step 6; plumephp.com

@@ -49,18 +49,16 @@ int64_t routed_rows(const moe_desc& d) {
 
 size_t act_bytes(const moe_desc& d) { return d.act_dtype == MOE_F32 ? 4 : 2; }
 
-// E4M3 weights with bf16 activations: the GEMMs decode each weight tile
-// themselves (every weight row a whole number of 16-byte pieces, at least 128
-// codes) while the experts have few rows.  Each CTA decodes the tiles it multiplies, so a
-// weight tile is decoded once per 128-row block of its expert: with many row
-// blocks the decode (ALU and shared-memory bandwidth) outgrows the MMA, and a
-// single decode pass into the workspace followed by the bf16 GEMM is faster.
-constexpr int64_t kW8InGemmRowsPerExpert = 1024;
-
-bool w8_in_gemm(const moe_desc& d) {
-  return d.weight_dtype == MOE_E4M3 && d.act_quant == 0 && d.act_dtype == MOE_BF16 && d.d_model % 16 == 0 &&
-         d.d_ff % 16 == 0 && d.d_model >= 128 && d.d_ff >= 128 &&
-         static_cast<int64_t>(d.num_tokens) * d.top_k <= kW8InGemmRowsPerExpert * d.num_experts;
+// Codes of the expert GEMMs' A rows: 0 = the GEMMs read bf16 (or fp32) rows;
+// 1 = W8A8 (one E4M3 code per element, scale amax / 448); 2 = E4M3 weights
+// with bf16 activations: each bf16 element as two E4M3 terms with a
+// power-of-two row scale (quant.cu), so the GEMMs multiply the stored weight
+// codes directly.  Rows must be whole 16-byte pieces of codes (d and h
+// multiples of 16); otherwise the weights are decoded to bf16 first.
+int a_terms(const moe_desc& d) {
+  if (d.act_quant == 1) return 1;
+  if (d.weight_dtype == MOE_E4M3 && d.act_dtype == MOE_BF16 && d.d_model % 16 == 0 && d.d_ff % 16 == 0) return 2;
+  return 0;
 }
 
 Layout make_layout(const moe_desc& d) {
@@ -86,21 +84,22 @@ Layout make_layout(const moe_desc& d) {
   L.topk_w = take(static_cast<size_t>(S * K) * 4);
   L.row_of_slot = take(static_cast<size_t>(S * K) * 4);
   L.token_of_row = take(static_cast<size_t>(R) * 4);
-  L.x_perm = take(static_cast<size_t>(R * dm) * ab);
+  // (E4M3 A rows: the row gather writes codes, no bf16 copy of the permuted rows)
+  L.x_perm = take(a_terms(d) ? 0 : static_cast<size_t>(R * dm) * ab);
   L.hidden = take(static_cast<size_t>(Rt * h) * ab);
   L.y_perm = take(static_cast<size_t>(Rt * dm) * ab);
-  const bool w8a8 = d.act_quant == 1;
-  L.wdeq = take(d.weight_dtype == MOE_E4M3 && !w8a8 && !w8_in_gemm(d)
-                    ? static_cast<size_t>((E + d.num_shared) * 3 * h * dm) * 2
-                    : 0);
-  // W8A8: E4M3 codes and row scales of the up GEMM's A rows (permuted
-  // tokens; the shared expert's tokens) and of the down GEMM's (hidden rows)
-  L.qa = take(w8a8 ? static_cast<size_t>(R * dm) : 0);
-  L.sa = take(w8a8 ? static_cast<size_t>(R) * 4 : 0);
-  L.qas = take(w8a8 && d.num_shared ? static_cast<size_t>(S * dm) : 0);
-  L.sas = take(w8a8 && d.num_shared ? static_cast<size_t>(S) * 4 : 0);
-  L.qh = take(w8a8 ? static_cast<size_t>(Rt * h) : 0);
-  L.sh = take(w8a8 ? static_cast<size_t>(Rt) * 4 : 0);
+  const int terms = a_terms(d);
+  L.wdeq = take(d.weight_dtype == MOE_E4M3 && terms == 0 ? static_cast<size_t>((E + d.num_shared) * 3 * h * dm) * 2
+                                                          : 0);
+  // E4M3 A rows (W8A8, or two-term codes): codes and row scales of the up
+  // GEMM's A rows (permuted tokens; the shared expert's tokens) and of the
+  // down GEMM's (hidden rows)
+  L.qa = take(static_cast<size_t>(terms * R * dm));
+  L.sa = take(terms ? static_cast<size_t>(R) * 4 : 0);
+  L.qas = take(d.num_shared ? static_cast<size_t>(terms * S * dm) : 0);
+  L.sas = take(terms && d.num_shared ? static_cast<size_t>(S) * 4 : 0);
+  L.qh = take(static_cast<size_t>(terms * Rt * h));
+  L.sh = take(terms ? static_cast<size_t>(Rt) * 4 : 0);
   // re-routing: every expert's selection key and gate source, the slots' picks, the excess-slot list and
   // its count, token claims and lists, changed tokens
   const bool rr = d.reroute == 1;
@@ -346,10 +345,13 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
     down.bias = w.b2;
   } else {
     const void *wg = w.w_gate, *wu = w.w_up, *wd = w.w_down, *w1 = w.w1, *w2 = w.w2;
-    if (d.act_quant == 1) {
-      // W8A8: the GEMMs read the E4M3 weights as they are; A rows are
-      // quantised per row right before each GEMM (below)
+    if (a_terms(d) > 0) {
+      // E4M3 weights read as they are by kind::f8f6f4 GEMMs; the A rows are
+      // E4M3 codes (W8A8: one per element; bf16 activations: two terms per
+      // element), made per row right before each GEMM (below) or by the row
+      // gather; the epilogue applies the row and the channel scales
       up.fp8 = down.fp8 = 1;
+      up.a_terms = down.a_terms = a_terms(d);
       up.scale0 = w.s_gate;
       up.scale1 = w.s_up;
       down.scale0 = w.s_down;
@@ -360,14 +362,6 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
       down.a = at<void>(ws, L.qh);
       down.row_scale = at<float>(ws, L.sh);
       down.row_scale_shared = nullptr;
-    } else if (d.weight_dtype == MOE_E4M3 && w8_in_gemm(d)) {
-      // E4M3 weights, bf16 activations: the GEMMs decode each landed weight
-      // tile to bf16 themselves (exact); the per-channel scales are applied to
-      // the fp32 accumulators in the epilogues
-      up.w8 = down.w8 = 1;
-      up.scale0 = w.s_gate;
-      up.scale1 = w.s_up;
-      down.scale0 = w.s_down;
     } else if (d.weight_dtype == MOE_E4M3) {
       // exact E4M3 -> bf16 decode of this call's weights into the workspace
       // (many rows per expert, or d or h not a multiple of 16); the
@@ -408,22 +402,24 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
   auto run = [&](const GemmArgs& g) {
     return d.act_dtype == MOE_F32 ? launch_grouped_gemm_f32(g, st) : launch_grouped_gemm_tc(g, sms, st);
   };
-  // W8A8: E4M3 codes + row scales of the A rows a GEMM over `g` reads
+  // E4M3 A rows: codes + row scales of the A rows a GEMM over `g` reads
+  const int terms = a_terms(d);
   auto quant_up = [&](const GemmArgs& g) {
     return launch_quantize_group_rows(g.groups, g.num_groups, 0, g.shared_slab, x_perm, at<uint8_t>(ws, L.qa),
                                       at<float>(ws, L.sa), R, x, d.num_shared ? at<uint8_t>(ws, L.qas) : nullptr,
-                                      d.num_shared ? at<float>(ws, L.sas) : nullptr, S, dm, g.max_group_rows, st);
+                                      d.num_shared ? at<float>(ws, L.sas) : nullptr, S, dm, g.max_total_rows, terms,
+                                      st);
   };
   auto quant_down = [&](const GemmArgs& g) {
     return launch_quantize_group_rows(g.groups, g.num_groups, 1, -1, hidden, at<uint8_t>(ws, L.qh),
-                                      at<float>(ws, L.sh), Rt, nullptr, nullptr, nullptr, 0, h, g.max_group_rows, st);
+                                      at<float>(ws, L.sh), Rt, nullptr, nullptr, nullptr, 0, h, g.max_total_rows,
+                                      terms, st);
   };
-  const bool w8a8 = d.act_quant == 1;
-  if (w8a8 && !a_quantized && (err = quant_up(up)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (terms && !a_quantized && (err = quant_up(up)) != cudaSuccess) return MOE_ERR_CUDA;
   if (!record(events, 3, st)) return MOE_ERR_CUDA;
   if ((err = run(up)) != cudaSuccess) return MOE_ERR_CUDA;
   if (!record(events, 4, st)) return MOE_ERR_CUDA;
-  if (w8a8 && (err = quant_down(down)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (terms && (err = quant_down(down)) != cudaSuccess) return MOE_ERR_CUDA;
   if (!record(events, 5, st)) return MOE_ERR_CUDA;
   if ((err = run(down)) != cudaSuccess) return MOE_ERR_CUDA;
   if (!record(events, 6, st)) return MOE_ERR_CUDA;
@@ -498,7 +494,7 @@ moe_status layer_impl(const moe_desc* desc, const moe_weights* w, const void* x,
   void* x_perm = at<void>(ws, L.x_perm);
   void* y_perm = at<void>(ws, L.y_perm);
   if (!record(events, 0, st)) return MOE_ERR_CUDA;
-  const bool w8a8 = d.act_quant == 1;
+  const int terms = a_terms(d);
   if ((s = route_impl(d, w, x, nullptr, idx, gates, ws, st)) != MOE_OK) return s;
   if (d.reroute == 1) {
     // capacity ranks of the first choices, then the excess slots move; the
@@ -508,13 +504,13 @@ moe_status layer_impl(const moe_desc* desc, const moe_weights* w, const void* x,
   }
   if (!record(events, 1, st)) return MOE_ERR_CUDA;
   // the permutation also writes the GEMM group tables, so the FFN skips that launch
-  if (w8a8) {
-    // W8A8: the row gather writes E4M3 codes and row scales straight away
-    // (no bf16 copy of the permuted rows)
+  if (terms) {
+    // E4M3 A rows: the row gather writes the codes and row scales straight
+    // away (no bf16 copy of the permuted rows)
     if ((s = permute_impl(d, nullptr, idx, cnt, offs, ros, tor, nullptr, ws, st, true)) != MOE_OK) return s;
     const bool sh = d.num_shared != 0;
     if (launch_gather_quantize(d.num_tokens, d.d_model, d.top_k, ros, x, at<uint8_t>(ws, L.qa), at<float>(ws, L.sa),
-                               sh ? at<uint8_t>(ws, L.qas) : nullptr, sh ? at<float>(ws, L.sas) : nullptr,
+                               sh ? at<uint8_t>(ws, L.qas) : nullptr, sh ? at<float>(ws, L.sas) : nullptr, terms,
                                st) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (!record(events, 2, st)) return MOE_ERR_CUDA;
@@ -615,7 +611,16 @@ moe_status moe_quantize_rows_e4m3(const void* x, int64_t rows, int32_t d, uint8_
   if (rows == 0) return MOE_OK;
   if (x == nullptr || q == nullptr || s == nullptr || !aligned16(x) || !aligned16(q)) return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(s) & 3) != 0) return MOE_ERR_INVALID_ARG;
-  return cuda_status(launch_quantize_rows(x, q, s, rows, d, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_quantize_rows(x, q, s, rows, d, 1, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_split_rows_e4m3(const void* x, int64_t rows, int32_t d, uint8_t* q, float* s, void* stream) {
+  NvtxRange nvtx("moe_split_rows_e4m3");
+  if (rows < 0 || d <= 0 || d % 16 != 0) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (x == nullptr || q == nullptr || s == nullptr || !aligned16(x) || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(s) & 3) != 0) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_quantize_rows(x, q, s, rows, d, 2, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_combine(const moe_desc* desc, const void* y_perm, const int32_t* row_of_slot, const float* topk_w,

@@ -35,7 +35,7 @@ struct TcParams {
   int pcols;           // 2N (SwiGLU: gate then up) or N
   int* ksplit_out;     // the split chosen on the device (read by the finalize kernel)
   int test_stall;      // test hook: the producer delivers nothing (the bounded waits must give up)
-  int land_stages;     // E4M3-weight kernel: landing buffers of E4M3 weight tiles
+  int a_terms;         // E4M3 activations: 1, or 2 for two-term codes (A rows of 2K codes, term 2 at column K)
   int tma_out;         // 1: the output tensor map is valid (full 32-row quarters use bulk tensor stores)
   const float* row_scale;         // E4M3 activations: per-row scale of the A operand rows (nullptr: none)
   const float* row_scale_shared;  // ... of the shared expert's A rows (indexed by row within the group)
@@ -213,22 +213,6 @@ inline bool make_map(CUtensorMap* m, const void* base, int64_t rows, int k, int 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-
-// 2-D map over E4M3 weights [rows][k] for the W8 GEMM: box = 64 codes (the K
-// extent of one bf16 stage) x 128 rows, no swizzle (the converters read it
-// row by row and write the swizzled bf16 tile).
-inline bool make_map_w8(CUtensorMap* m, const void* base, int64_t rows, int k) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (enc == nullptr || rows <= 0 || k <= 0) return false;
-  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || k % 16 != 0 || k < 128) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(k)};
-  cuuint32_t box[2] = {128, 128};  // two bf16 K steps of 128 weight rows
-  cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 }  // namespace gemm
 }  // namespace moe

@@ -14,11 +14,14 @@
 // silu(gate) * up (x per-channel scales for FP8 weights) as bf16.
 // Down projection: 256 output columns per tile, optional bias / scale.
 //
-// With E4M3 activations and weights (W8A8) the same kernel runs on 8-bit
-// operands: a stage still holds 128-byte rows, now 128 K elements, and the
-// MMA kind is f8f6f4 (K = 32 per instruction); the epilogue multiplies each
-// accumulator row by its activation row scale and each column by the weight
-// channel scale.
+// With E4M3 weights the same kernel runs on 8-bit operands: a stage still
+// holds 128-byte rows, now 128 K elements, and the MMA kind is f8f6f4 (K = 32
+// per instruction); the epilogue multiplies each accumulator row by its
+// activation row scale and each column by the weight channel scale.  The A
+// rows are E4M3 codes of the activations: one code per element (W8A8), or,
+// for bf16 activations, two codes per element (x * 2^k = c1 + c2, rows
+// [c1 | c2] of 2K codes): a stage then holds both A tiles and the MMA warp
+// issues both terms against the same weight tile into one fp32 sum.
 //
 // Structure (one CTA per SM, 320 threads):
 //   warp 0      TMA producer: A tile 128x64 and B tile 256x64 (bf16, 128-byte
@@ -66,14 +69,6 @@ constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
 constexpr int kEpiWarps = 8;  // two per TMEM lane quarter, each draining half of a tile's columns
 constexpr int kThreads = 64 + 32 * kEpiWarps;
-// E4M3 weights with bf16 activations (W8): eight more warps decode each landed
-// E4M3 weight tile into the bf16 B tile of its stage.
-constexpr int kConvWarps = 8;
-constexpr int kConvGroups = 2;  // the two K steps of a landing buffer are decoded side by side
-constexpr int kGroupThreads = 32 * kConvWarps / kConvGroups;
-constexpr int kThreadsW8 = kThreads + 32 * kConvWarps;
-constexpr int kMaxLandStages = 8;          // landing buffers of E4M3 weight tiles (at most)
-constexpr int LAND_BYTES = 256 * 128;      // 256 weight rows x 128 E4M3 codes (two bf16 K steps)
 constexpr uint32_t kIdescBf16 = idesc_bf16_f32(128, 256);
 constexpr uint32_t kIdescE4m3 = idesc_e4m3_f32(128, 256);
 
@@ -86,10 +81,6 @@ constexpr int bk_elems() {
 struct SmemCtl {
   uint64_t full[MAX_STAGES];
   uint64_t empty[MAX_STAGES];
-  uint64_t lfull[kMaxLandStages];  // W8: an E4M3 weight tile has landed
-  uint64_t ldone[kMaxLandStages];  // W8: the first K step of a two-step landing buffer is decoded
-  int land_parity[kMaxLandStages]; // W8: parity of the latest copy into each landing buffer (-1: none)
-  int conv_ok[kConvGroups];        // W8: each converter group's shared go / give-up decision
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -264,70 +255,19 @@ __device__ __forceinline__ void epilogue_partial(const TcParams& p, const TileIn
   }
 }
 
-// Four E4M3 codes (bytes of w, lowest first) -> four bf16 values (lo: codes
-// 0, 1; hi: codes 2, 3), exactly: E4M3 -> f16 is exact (every E4M3 value,
-// subnormals included, is a normal f16 or zero), f16 -> f32 is exact, and the
-// f32 -> bf16 rounding keeps the value (at most four significant bits, inside
-// bf16's exponent range).  The f16 -> bf16 step goes through f32 because the
-// packed f32 -> bf16x2 conversion is one instruction for two values.
-__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  asm("{\n\t.reg .b16 c0, c1, a, b, c, d;\n\t.reg .b32 h0, h1;\n\t.reg .f32 fa, fb, fc, fd;\n\t"
-      "mov.b32 {c0, c1}, %2;\n\t"
-      "cvt.rn.f16x2.e4m3x2 h0, c0;\n\t"
-      "cvt.rn.f16x2.e4m3x2 h1, c1;\n\t"
-      "mov.b32 {a, b}, h0;\n\t"
-      "cvt.f32.f16 fa, a;\n\t"
-      "cvt.f32.f16 fb, b;\n\t"
-      "cvt.rn.bf16x2.f32 %0, fb, fa;\n\t"
-      "mov.b32 {c, d}, h1;\n\t"
-      "cvt.f32.f16 fc, c;\n\t"
-      "cvt.f32.f16 fd, d;\n\t"
-      "cvt.rn.bf16x2.f32 %1, fd, fc;\n\t}"
-      : "=r"(lo), "=r"(hi)
-      : "r"(w));
-}
-
-// W8: one converter group (kGroupThreads threads) decodes the 64 codes of
-// one K step from each of the 256 rows of a landing buffer (rows of 128
-// bytes, two K steps; `land` points at the step's first code of row 0) into
-// the stage's 256 x 128-byte bf16 B tile in the 128-byte swizzled layout the
-// MMA reads (16-byte chunk j of row r at chunk j ^ (r & 7)).  Thread gt takes
-// the 16-code pieces gt + kGroupThreads i.
-__device__ __forceinline__ void convert_tile_w8(const uint8_t* land, uint8_t* b16, int gt) {
-#pragma unroll 2
-  for (int i = 0; i < 1024 / kGroupThreads; ++i) {
-    const int piece = gt + kGroupThreads * i;  // 1024 pieces of 16 codes
-    const int r = piece >> 2, q4 = piece & 3;
-    const uint4 v = *reinterpret_cast<const uint4*>(land + r * 128 + q4 * 16);
-    uint32_t o[8];
-    e4m3x4_to_bf16x4(v.x, o[0], o[1]);
-    e4m3x4_to_bf16x4(v.y, o[2], o[3]);
-    e4m3x4_to_bf16x4(v.z, o[4], o[5]);
-    e4m3x4_to_bf16x4(v.w, o[6], o[7]);
-    uint8_t* row = b16 + r * BK_BYTES;
-    const int sw = r & 7;
-    *reinterpret_cast<uint4*>(row + (((2 * q4) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-    *reinterpret_cast<uint4*>(row + (((2 * q4 + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
-  }
-}
-
-__device__ __forceinline__ void named_bar_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-
-template <int EPI, bool F8, bool W8>
-__global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
+template <int EPI, bool F8>
+__global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                            const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
                            const __grid_constant__ CUtensorMap tmOut, TcParams p, int bma, int STAGES) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int BK = bk_elems<F8>();
-  const int A_TILE = bma * BK_BYTES;
+  const int A_TERM = bma * BK_BYTES;              // one A tile (rows x 128 bytes of K)
+  const int A_TERMS = F8 ? p.a_terms : 1;         // two-term E4M3 activations: two A tiles per stage
+  const int A_TILE = A_TERM * A_TERMS;
   const int STAGE_BYTES = A_TILE + B_TILE;
-  uint8_t* land = ring + STAGES * STAGE_BYTES;  // W8 landing buffers (1024-byte aligned)
-  const int LAND = W8 ? p.land_stages : 0;       // W8 landing buffers in use
-  uint8_t* ctl = land + LAND * LAND_BYTES;
+  uint8_t* ctl = ring + STAGES * STAGE_BYTES;
   SmemCtl& s = *reinterpret_cast<SmemCtl*>(ctl);
   uint8_t* epi_smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(ctl + sizeof(SmemCtl)) + 127) & ~uintptr_t(127));
@@ -340,15 +280,9 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
   if (warp == 1) {
     if (lane == 0) {
       for (int i = 0; i < STAGES; ++i) {
-        mbar_init(&s.full[i], W8 ? 2 : 1);  // W8: the A copy's arrival plus the converters'
+        mbar_init(&s.full[i], 1);
         mbar_init(&s.empty[i], 1);
       }
-      if (W8)
-        for (int i = 0; i < LAND; ++i) {
-          mbar_init(&s.lfull[i], 1);
-          mbar_init(&s.ldone[i], 1);
-          s.land_parity[i] = -1;
-        }
       for (int i = 0; i < 2; ++i) {
         mbar_init(&s.tfull[i], 1);
         mbar_init(&s.tempty[i], 32 * kEpiWarps);
@@ -421,15 +355,14 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&s.full[stage], W8 ? A_TILE : STAGE_BYTES);
+          mbar_arrive_expect_tx(&s.full[stage], STAGE_BYTES);
           armed |= 1u << stage;
           armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
           uint8_t* sa = ring + stage * STAGE_BYTES;
           uint8_t* sb = sa + A_TILE;
           tma_load_2d(sa, mA, kb * BK, a_row, &s.full[stage]);
-          if (W8) {
-            // the converters fill this stage's B tile
-          } else if (EPI == EPI_SWIGLU) {
+          if (F8 && A_TERMS == 2) tma_load_2d(sa + A_TERM, mA, p.K + kb * BK, a_row, &s.full[stage]);
+          if (EPI == EPI_SWIGLU) {
             tma_load_2d(sb, &tmB0, kb * BK, b_row, &s.full[stage]);
             tma_load_2d(sb + B_HALF, &tmB1, kb * BK, b_row, &s.full[stage]);
           } else {
@@ -476,12 +409,17 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
           tc_fence_after();
           const uint32_t a_base = smem_u32(ring + stage * STAGE_BYTES);
           const uint32_t b_base = a_base + A_TILE;
+          if (F8) {
+            // one or two A terms against the same weight tile, one fp32 sum
+            for (int t = 0; t < A_TERMS; ++t) {
 #pragma unroll
-          for (int kk = 0; kk < BK_BYTES / 32; ++kk) {  // 32 bytes of K per MMA (16 bf16 or 32 E4M3)
-            if (F8)
-              tc_mma_f8(d_tmem, smem_desc_sw128(a_base + kk * 32), smem_desc_sw128(b_base + kk * 32), kIdescE4m3,
-                        (kb > kb0 || kk > 0) ? 1u : 0u);
-            else
+              for (int kk = 0; kk < BK_BYTES / 32; ++kk)  // 32 E4M3 of K per MMA
+                tc_mma_f8(d_tmem, smem_desc_sw128(a_base + t * A_TERM + kk * 32), smem_desc_sw128(b_base + kk * 32),
+                          kIdescE4m3, (kb > kb0 || kk > 0 || t > 0) ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < BK_BYTES / 32; ++kk)  // 16 bf16 of K per MMA
               tc_mma_f16(d_tmem, smem_desc_sw128(a_base + kk * 32), smem_desc_sw128(b_base + kk * 32), kIdescBf16,
                          (kb > kb0 || kk > 0) ? 1u : 0u);
           }
@@ -503,131 +441,6 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (W8 && warp >= 2 + kEpiWarps) {
-    // W8 converters, two groups of four warps.  A landing buffer holds the
-    // E4M3 codes of two K steps of a weight tile (256 rows x 128 bytes: DRAM
-    // reads of 128 contiguous bytes per row); group 0 decodes the first K
-    // step, group 1 the second, side by side.  For its K step a group waits
-    // for the codes to land and for the stage's B tile to be free, decodes,
-    // then lets the MMA go (second arrival on the stage's full barrier).  The
-    // group decoding a buffer's last K step refills it with the pair LAND
-    // pairs ahead (group 1 first waits for group 0's half: ldone).  Both
-    // groups walk the whole K-step sequence, so they agree on stages, phases
-    // and buffers.  Each group's first thread waits on the barriers; the go /
-    // give-up decision reaches the group through shared memory.
-    const int ct = threadIdx.x - (2 + kEpiWarps) * 32;
-    const int g = ct / kGroupThreads, gt = ct % kGroupThreads;
-    // the sequence of K-step pairs, walked twice: `cur` for decoding, `ahd` for issuing copies
-    struct Seq {
-      int u, kb, kb1;  // unit, first K step of the pair, end of the unit's K range
-    };
-    auto seq_begin = [&](Seq& q) {
-      q.u = blockIdx.x;
-      q.kb = 0;
-      q.kb1 = 0;
-      while (q.u < total) {
-        const UnitInfo ui = decode_unit(s, p, q.u, ks, nk);
-        q.kb = ui.kb0;
-        q.kb1 = ui.kb1;
-        if (q.kb < q.kb1) return;
-        q.u += gridDim.x;
-      }
-    };
-    auto seq_next = [&](Seq& q) {
-      q.kb += 2;
-      if (q.kb < q.kb1) return;
-      q.u += gridDim.x;
-      while (q.u < total) {
-        const UnitInfo ui = decode_unit(s, p, q.u, ks, nk);
-        q.kb = ui.kb0;
-        q.kb1 = ui.kb1;
-        if (q.kb < q.kb1) return;
-        q.u += gridDim.x;
-      }
-    };
-    auto issue = [&](const Seq& q, int l, uint32_t parity) {  // E4M3 codes of pair q into landing buffer l
-      const UnitInfo ui = decode_unit(s, p, q.u, ks, nk);
-      const int b_row = ui.ti.grp.expert * p.n_per_slab + ui.ti.n_idx * p.bn_out;
-      uint8_t* dst = land + l * LAND_BYTES;
-      s.land_parity[l] = static_cast<int>(parity);
-      mbar_arrive_expect_tx(&s.lfull[l], LAND_BYTES);
-      if (EPI == EPI_SWIGLU) {
-        tma_load_2d(dst, &tmB0, q.kb * BK, b_row, &s.lfull[l]);
-        tma_load_2d(dst + LAND_BYTES / 2, &tmB1, q.kb * BK, b_row, &s.lfull[l]);
-      } else {
-        tma_load_2d(dst, &tmB0, q.kb * BK, b_row, &s.lfull[l]);
-        tma_load_2d(dst + LAND_BYTES / 2, &tmB0, q.kb * BK, b_row + 128, &s.lfull[l]);
-      }
-    };
-    Seq cur, ahd;
-    seq_begin(cur);
-    seq_begin(ahd);
-    if (g == 0 && gt == 0 && !p.test_stall) {
-      for (int l = 0; l < LAND && ahd.u < total; ++l) {
-        issue(ahd, l, 0u);
-        seq_next(ahd);
-      }
-    } else {
-      for (int l = 0; l < LAND && ahd.u < total; ++l) seq_next(ahd);
-    }
-    int stage = 0, l = 0;
-    uint32_t phase = 0, lphase = 0, ld_bits = 0;
-    bool ok = true;
-    while (cur.u < total && ok) {
-      const int n = min(2, cur.kb1 - cur.kb);  // K steps in this pair
-      for (int h = 0; h < n; ++h) {
-        if (h == g) {
-          if (gt == 0) {
-            const int go = !p.test_stall && mbar_wait(&s.lfull[l], lphase, abort_flag) &&
-                           mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag);
-            s.conv_ok[g] = go;
-          }
-          named_bar_sync(1 + g, kGroupThreads);
-          if (!s.conv_ok[g]) {
-            ok = false;
-            break;
-          }
-          convert_tile_w8(land + l * LAND_BYTES + h * 64, ring + stage * STAGE_BYTES + A_TILE, gt);
-          fence_proxy_async_smem();  // generic-proxy writes before the tensor core's reads
-          named_bar_sync(1 + g, kGroupThreads);
-          if (gt == 0) {
-            mbar_arrive(&s.full[stage]);
-            if (g == 0 && n == 2) mbar_arrive(&s.ldone[l]);
-          }
-        }
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
-      if (!ok) break;
-      // the group that decoded the pair's last K step refills the buffer
-      if (g == n - 1 && gt == 0 && ahd.u < total) {
-        if (n == 2 && !mbar_wait(&s.ldone[l], (ld_bits >> l) & 1u, abort_flag)) {
-          ok = false;
-        } else {
-          issue(ahd, l, (lphase + 1u) & 1u);
-        }
-      }
-      if (n == 2) ld_bits ^= 1u << l;
-      if (g == n - 1 && gt == 0) s.conv_ok[g] = ok;
-      named_bar_sync(1 + g, kGroupThreads);
-      if (g == n - 1 && !s.conv_ok[g]) ok = false;
-      if (!ok) break;
-      seq_next(ahd);
-      seq_next(cur);
-      if (++l == LAND) {
-        l = 0;
-        lphase ^= 1u;
-      }
-    }
-    if (!ok && gt == 0) {
-      *abort_flag = 1;
-      report(p.status, MOE_STATUS_TIMEOUT, MOE_CNT_TIMEOUT);
-      // let the copies already issued land before the CTA exits
-      for (int i = 0; i < LAND; ++i)
-        if (s.land_parity[i] >= 0) wait_timed(&s.lfull[i], static_cast<uint32_t>(s.land_parity[i]));
-    }
   } else {
     const int q = warp & 3;                // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;      // which half of the tile's columns it drains
@@ -666,7 +479,7 @@ __global__ void __launch_bounds__(W8 ? kThreadsW8 : kThreads, 1)
   }
 }
 
-template <int EPI, bool F8, bool W8 = false>
+template <int EPI, bool F8>
 cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB0, const CUtensorMap& mB1,
                        const CUtensorMap& mOut, const TcParams& p, int grid, int bma, int stages, size_t smem,
                        int64_t max_group_rows, cudaStream_t stream) {
@@ -675,13 +488,13 @@ cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUte
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64 || !(attr_set & (1ull << dev))) {
-    e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<EPI, F8, W8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<EPI, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemLimitTc));
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set |= 1ull << dev;
   }
   // programmatic dependent launch: the prologue may overlap the previous kernel
-  e = launch_pdl(grouped_gemm_tc_kernel<EPI, F8, W8>, dim3(grid), dim3(W8 ? kThreadsW8 : kThreads), smem, stream, mA,
+  e = launch_pdl(grouped_gemm_tc_kernel<EPI, F8>, dim3(grid), dim3(kThreads), smem, stream, mA,
                  mA2, mB0, mB1, mOut, p, bma, stages);
   if (e != cudaSuccess) return e;
   if ((e = cudaGetLastError()) != cudaSuccess || p.max_ksplit <= 1) return e;
@@ -698,76 +511,39 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
   // A rows loaded per stage: all 128, or (every group fitting) the largest group rounded up to 16
   int bma = BM;
   if (a.max_group_rows > 0 && a.max_group_rows <= 64) bma = static_cast<int>((a.max_group_rows + 15) & ~int64_t(15));
-  const size_t stage_bytes = static_cast<size_t>(bma) * BK_BYTES + B_TILE;
+  const int terms = a.fp8 && a.a_terms == 2 ? 2 : 1;  // two-term E4M3 activations: A rows of 2K codes
+  const size_t stage_bytes = static_cast<size_t>(bma) * BK_BYTES * terms + B_TILE;
   const int eb = a.fp8 ? 1 : 2;  // element bytes of A and B
-  const bool w8 = a.w8 != 0 && !a.fp8;
-  int stages, land = 0;
-  if (w8) {
-    // E4M3 weights: the HBM latency is covered by the landing buffers (a
-    // weight tile is decoded into a bf16 stage only when the MMA is about to
-    // need it), so three bf16 stages and as many landing buffers as fit
-    stages = 3;
-    land = static_cast<int>((kSmemLimitTc - kCtlBytes - stages * stage_bytes) / LAND_BYTES);
-    if (land < 2) {
-      stages = 2;
-      land = static_cast<int>((kSmemLimitTc - kCtlBytes - stages * stage_bytes) / LAND_BYTES);
-    }
-    if (land > kMaxLandStages) land = kMaxLandStages;
-    if (land < 2) return cudaErrorInvalidValue;
-  } else {
-    stages = static_cast<int>((kSmemLimitTc - kCtlBytes) / stage_bytes);
-    if (stages > MAX_STAGES) stages = MAX_STAGES;
-  }
-  const size_t land_bytes = static_cast<size_t>(land) * LAND_BYTES;
-  const size_t smem = stages * stage_bytes + land_bytes + kCtlBytes;
+  int stages = static_cast<int>((kSmemLimitTc - kCtlBytes) / stage_bytes);
+  if (stages > MAX_STAGES) stages = MAX_STAGES;
+  const size_t smem = stages * stage_bytes + kCtlBytes;
   CUtensorMap mA, mA2, mB0, mB1, mOut;
   // bf16 outputs: full 32-row quarters go out as bulk tensor stores; fp32 outputs store row by row
   TcParams pp = p;
-  pp.land_stages = land;
   pp.tma_out = !a.out_f32 && make_store_map(&mOut, a.out, a.out_rows, a.N, 2) ? 1 : 0;
   if (!pp.tma_out) memset(&mOut, 0, sizeof(mOut));
-  if (!make_map(&mA, a.a, a.a_rows, a.K, bma, eb)) return cudaErrorInvalidValue;
+  pp.a_terms = terms;
+  if (!make_map(&mA, a.a, a.a_rows, a.K * terms, bma, eb)) return cudaErrorInvalidValue;
   if (a.a_shared != nullptr) {
-    if (!make_map(&mA2, a.a_shared, a.a_shared_rows, a.K, bma, eb)) return cudaErrorInvalidValue;
+    if (!make_map(&mA2, a.a_shared, a.a_shared_rows, a.K * terms, bma, eb)) return cudaErrorInvalidValue;
   } else {
     mA2 = mA;
   }
-  if (w8) {
-    // E4M3 weight tiles of one bf16 K step: 64 codes (64 bytes) x 128 rows, unswizzled
-    if (!make_map_w8(&mB0, a.b0, a.b_rows, a.K)) return cudaErrorInvalidValue;
-    if (a.epilogue == EPI_SWIGLU) {
-      if (!make_map_w8(&mB1, a.b1, a.b_rows, a.K)) return cudaErrorInvalidValue;
-    } else {
-      mB1 = mB0;
-    }
+  if (!make_map(&mB0, a.b0, a.b_rows, a.K, 128, eb)) return cudaErrorInvalidValue;
+  if (a.epilogue == EPI_SWIGLU) {
+    if (!make_map(&mB1, a.b1, a.b_rows, a.K, 128, eb)) return cudaErrorInvalidValue;
   } else {
-    if (!make_map(&mB0, a.b0, a.b_rows, a.K, 128, eb)) return cudaErrorInvalidValue;
-    if (a.epilogue == EPI_SWIGLU) {
-      if (!make_map(&mB1, a.b1, a.b_rows, a.K, 128, eb)) return cudaErrorInvalidValue;
-    } else {
-      mB1 = mB0;
-    }
+    mB1 = mB0;
   }
   // upper bound of the tile count: every group may add one partial m-block
   const int64_t bound = (a.max_total_rows / BM + a.num_groups) * static_cast<int64_t>(p.n_tiles);
   const int grid = static_cast<int>(bound < num_sms ? (bound > 0 ? bound : 1) : num_sms);
-  if (a.fp8) {  // W8A8 runs SwiGLU experts only
+  if (a.fp8) {  // E4M3 x E4M3 runs SwiGLU experts only
     switch (a.epilogue) {
       case EPI_SWIGLU:
         return launch_epi<EPI_SWIGLU, true>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
       case EPI_NONE:
         return launch_epi<EPI_NONE, true>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem, a.max_group_rows, stream);
-      default: return cudaErrorInvalidValue;
-    }
-  }
-  if (w8) {  // E4M3 weights, bf16 activations: SwiGLU experts only
-    switch (a.epilogue) {
-      case EPI_SWIGLU:
-        return launch_epi<EPI_SWIGLU, false, true>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem,
-                                                   a.max_group_rows, stream);
-      case EPI_NONE:
-        return launch_epi<EPI_NONE, false, true>(mA, mA2, mB0, mB1, mOut, pp, grid, bma, stages, smem,
-                                                 a.max_group_rows, stream);
       default: return cudaErrorInvalidValue;
     }
   }

@@ -117,7 +117,7 @@ struct GemmArgs {
   int64_t partial_bytes;    // size of `partial`
   int* ksplit_out;          // device int: the split the GEMM chose (read by the finalize kernel)
   int fp8;                  // 1: A and B are E4M3 (kind::f8f6f4); A rows scaled by row_scale
-  int w8;                   // 1: B (weights) E4M3, A bf16: the GEMM decodes each weight tile to bf16
+  int a_terms;              // fp8: 2 = A rows hold two-term codes [c1 | c2] (2K codes), summed in one accumulator
   const float* row_scale;        // [a rows] per-row scale of A (fp8 only)
   const float* row_scale_shared; // [S] per-row scale of the shared expert's A rows (fp8 only)
   StatusBlock* status;
@@ -133,23 +133,28 @@ cudaError_t launch_grouped_gemm_f32(const GemmArgs& a, cudaStream_t stream);
 cudaError_t launch_dequant_e4m3(const uint8_t* q, void* out_bf16, int64_t n, cudaStream_t stream);
 
 // --- E4M3 activations (W8A8) -------------------------------------------------
-// Per-row quantisation of bf16 rows: s = amax / 448 (1 for an all-zero row
-// or a row holding a NaN), q = RNE satfinite E4M3 (x / s), both float32
-// divisions.
-cudaError_t launch_quantize_rows(const void* src, uint8_t* dst, float* scale, int64_t rows, int d, cudaStream_t stream);
+// Per-row quantisation of bf16 rows.  terms = 1 (W8A8): s = amax / 448 (1
+// for an all-zero row or a row holding a NaN), q = RNE satfinite E4M3
+// (x / s), both float32 divisions; rows of d codes.  terms = 2 (E4M3
+// weights, bf16 activations): two-term codes c1 | c2 with x * 2^k = c1 + c2
+// and s = 2^-k (quant.cu); rows of 2d codes.
+cudaError_t launch_quantize_rows(const void* src, uint8_t* dst, float* scale, int64_t rows, int d, int terms,
+                                 cudaStream_t stream);
 // The row gather of the permutation fused with that quantisation: token t's
 // codes and scale go to rows row_of_slot[t*K + k] (>= 0) of q_perm / s_perm
 // and, when q_x is given, to row t of q_x / s_x.
 cudaError_t launch_gather_quantize(int S, int d, int K, const int32_t* row_of_slot, const void* x, uint8_t* q_perm,
-                                   float* s_perm, uint8_t* q_x, float* s_x, cudaStream_t stream);
+                                   float* s_perm, uint8_t* q_x, float* s_x, int terms, cudaStream_t stream);
 // The same for the rows of a group table: rows a_row0 + r (or out_row0 + r
 // with use_out_rows) of src, at most dst_rows; the shared-expert group's
 // rows come from src_shared and go to dst_shared / scale_shared (index r,
-// at most shared_rows).
+// at most shared_rows).  max_total_rows bounds the rows of all groups
+// together (it sizes the grid).
 cudaError_t launch_quantize_group_rows(const GroupEntry* groups, int num_groups, int use_out_rows, int shared_slab,
                                        const void* src, uint8_t* dst, float* scale, int64_t dst_rows,
                                        const void* src_shared, uint8_t* dst_shared, float* scale_shared,
-                                       int64_t shared_rows, int d, int64_t max_group_rows, cudaStream_t stream);
+                                       int64_t shared_rows, int d, int64_t max_total_rows, int terms,
+                                       cudaStream_t stream);
 
 // --- sliding-window load and selection-bias update ---------------------------
 size_t bias_state_bytes(int E, int K, int window);

@@ -33,7 +33,7 @@ WEIGHT_FIELDS = ("w_router", "router_bias", "sel_bias", "w1", "b1", "w2", "b2", 
 EXPORTED = ("moe_routed_rows", "moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute",
             "moe_permute_static", "moe_grouped_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_timed",
             "moe_load_stats", "moe_bias_state_size", "moe_bias_state_init", "moe_update_sel_bias",
-            "moe_quantize_rows_e4m3", "moe_reroute", "moe_get_status", "moe_strerror")
+            "moe_quantize_rows_e4m3", "moe_split_rows_e4m3", "moe_reroute", "moe_get_status", "moe_strerror")
 
 MOE_NUM_STAGE_EVENTS = 8
 MOE_NUM_LOAD_STATS = 6
@@ -80,6 +80,7 @@ def lib():
         "moe_bias_state_init": (I, [P, SZ, P]),
         "moe_update_sel_bias": (I, [pd, P, ctypes.c_int32, ctypes.c_float, P, SZ, P, P, P]),
         "moe_quantize_rows_e4m3": (I, [P, ctypes.c_int64, ctypes.c_int32, P, P, P]),
+        "moe_split_rows_e4m3": (I, [P, ctypes.c_int64, ctypes.c_int32, P, P, P]),
         "moe_reroute": (I, [pd, P, P, P, P, P, SZ, P]),
         "moe_get_status": (I, [P, P, ctypes.POINTER(ctypes.c_uint32), ctypes.POINTER(ctypes.c_int32)]),
         "moe_strerror": (ctypes.c_char_p, [I]),
@@ -247,6 +248,14 @@ def moe_quantize_rows_e4m3(x, q, s, stream=None):
     rows, d = int(x.shape[0]), int(x.shape[1])
     _check(lib().moe_quantize_rows_e4m3(_ptr(x), rows, d, _ptr(q), _ptr(s), _stream(stream)),
            "moe_quantize_rows_e4m3")
+
+
+def moe_split_rows_e4m3(x, q, s, stream=None):
+    """Two-term E4M3 codes q [rows][2d] (uint8: first terms, then second
+    terms) and power-of-two scales s [rows] (fp32) of the bf16 rows x
+    [rows][d]."""
+    rows, d = int(x.shape[0]), int(x.shape[1])
+    _check(lib().moe_split_rows_e4m3(_ptr(x), rows, d, _ptr(q), _ptr(s), _stream(stream)), "moe_split_rows_e4m3")
 
 
 def moe_get_status(ws, stream=None):

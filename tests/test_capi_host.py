@@ -182,32 +182,34 @@ def test_bias_state_size_and_argument_errors():
 
 @pytest.mark.parametrize("name", [n for n, c in syn.VARIANTS.items() if c.act_quant])
 def test_w8a8_workspace_holds_codes_and_scales(name):
-    """W8A8 replaces the bf16 weight copy with the 8-bit activation rows."""
+    """W8A8 holds one E4M3 code per activation element and a scale per row;
+    the same layer on bf16 activations holds two codes per element (two-term
+    codes) and the same scales."""
     cfg = syn.VARIANTS[name]
     d8 = _desc(name)
     d16 = ops.make_desc(**dict(syn.desc_dict(cfg), act_quant=0))
     R = ops.moe_routed_rows(d8)
     Rt = R + cfg.num_shared * cfg.S
     n8, n16 = ops.moe_workspace_size(d8), ops.moe_workspace_size(d16)
-    wdeq = (cfg.E + cfg.num_shared) * 3 * cfg.h * cfg.d * 2
     codes = R * cfg.d + Rt * cfg.h + (R + Rt) * 4
     assert n8 >= codes
-    assert n8 - (n16 - wdeq) >= codes
+    assert R * cfg.d + Rt * cfg.h <= n16 - n8 <= R * cfg.d + Rt * cfg.h + 8 * 4096
 
 
-def test_quantize_rows_argument_errors():
-    L = ops.lib()
+@pytest.mark.parametrize("name", ["moe_quantize_rows_e4m3", "moe_split_rows_e4m3"])
+def test_quantize_rows_argument_errors(name):
+    fn = getattr(ops.lib(), name)
     p = ctypes.c_void_p(0x1000)
-    assert L.moe_quantize_rows_e4m3(p, 0, 32, p, p, None) == ops.MOE_OK       # nothing to do
-    assert L.moe_quantize_rows_e4m3(p, -1, 32, p, p, None) == ops.MOE_ERR_INVALID_ARG
-    assert L.moe_quantize_rows_e4m3(p, 4, 24, p, p, None) == ops.MOE_ERR_INVALID_ARG
-    assert L.moe_quantize_rows_e4m3(p, 4, 0, p, p, None) == ops.MOE_ERR_INVALID_ARG
-    assert L.moe_quantize_rows_e4m3(None, 4, 32, p, p, None) == ops.MOE_ERR_INVALID_ARG
-    assert L.moe_quantize_rows_e4m3(p, 4, 32, None, p, None) == ops.MOE_ERR_INVALID_ARG
-    assert L.moe_quantize_rows_e4m3(p, 4, 32, p, None, None) == ops.MOE_ERR_INVALID_ARG
-    assert L.moe_quantize_rows_e4m3(ctypes.c_void_p(0x1008), 4, 32, p, p, None) == ops.MOE_ERR_INVALID_ARG
-    assert L.moe_quantize_rows_e4m3(p, 4, 32, ctypes.c_void_p(0x1004), p, None) == ops.MOE_ERR_INVALID_ARG
-    assert L.moe_quantize_rows_e4m3(p, 4, 32, p, ctypes.c_void_p(0x1002), None) == ops.MOE_ERR_INVALID_ARG
+    assert fn(p, 0, 32, p, p, None) == ops.MOE_OK       # nothing to do
+    assert fn(p, -1, 32, p, p, None) == ops.MOE_ERR_INVALID_ARG
+    assert fn(p, 4, 24, p, p, None) == ops.MOE_ERR_INVALID_ARG
+    assert fn(p, 4, 0, p, p, None) == ops.MOE_ERR_INVALID_ARG
+    assert fn(None, 4, 32, p, p, None) == ops.MOE_ERR_INVALID_ARG
+    assert fn(p, 4, 32, None, p, None) == ops.MOE_ERR_INVALID_ARG
+    assert fn(p, 4, 32, p, None, None) == ops.MOE_ERR_INVALID_ARG
+    assert fn(ctypes.c_void_p(0x1008), 4, 32, p, p, None) == ops.MOE_ERR_INVALID_ARG
+    assert fn(p, 4, 32, ctypes.c_void_p(0x1004), p, None) == ops.MOE_ERR_INVALID_ARG
+    assert fn(p, 4, 32, p, ctypes.c_void_p(0x1002), None) == ops.MOE_ERR_INVALID_ARG
 
 
 def test_reroute_workspace_and_argument_errors():
@@ -305,20 +307,22 @@ def test_missing_library_fails_loudly():
     assert "raised" in r.stdout, (r.stdout, r.stderr)
 
 
-def test_e4m3_workspace_decoded_weights_only_for_many_rows():
-    """E4M3 weights with bf16 activations are decoded tile by tile inside the
-    GEMMs while the experts have at most 1024 routed rows each on average:
-    the workspace is then no larger than with bf16 weights (no bf16 copy of
-    the weights).  With more rows per expert, or with d or h not a multiple
-    of 16, the layer decodes the weights into the workspace first."""
-    c8 = syn.scaled(syn.CONFIGS["fp8_skew_capacity"], S=8192)      # 8192 * 8 / 64 = 1024 rows per expert
-    c16 = syn.scaled(c8, weight_dtype=syn.BF16)
+def test_e4m3_workspace_two_term_codes_instead_of_decoded_weights():
+    """E4M3 weights with bf16 activations: the GEMMs read the stored weight
+    codes, so the workspace holds no bf16 copy of the weights.  The token
+    rows' two-term codes (2 bytes per element) take the place of the bf16
+    copy of the permuted rows, and the hidden rows get their codes beside the
+    bf16 hidden rows, with one fp32 scale per row.  With d or h not a
+    multiple of 16 the layer decodes the weights into the workspace first."""
     size = lambda c: ops.moe_workspace_size(ops.make_desc(**syn.desc_dict(c)))
-    assert size(c8) == size(c16)
-    big8 = syn.scaled(c8, S=8200)
-    assert size(big8) > size(syn.scaled(c16, S=8200))
-    n_dec = 3 * (big8.E + big8.num_shared) * big8.h * big8.d * 2      # the three decoded bf16 stacks
-    assert size(big8) - size(syn.scaled(c16, S=8200)) >= n_dec
+    for S in (64, 8192, 16384):
+        c8 = syn.scaled(syn.CONFIGS["fp8_skew_capacity"], S=S)
+        c16 = syn.scaled(c8, weight_dtype=syn.BF16)
+        R = ops.moe_routed_rows(ops.make_desc(**syn.desc_dict(c8)))
+        extra = 2 * R * c8.h + 4 * 2 * R                                  # hidden codes, scales
+        assert extra <= size(c8) - size(c16) <= extra + 8 * 4096, S       # alignment slack only
+    c8 = syn.scaled(syn.CONFIGS["fp8_skew_capacity"], S=1024)
     odd8 = syn.scaled(c8, d=2056)
-    odd16 = syn.scaled(c16, d=2056)
-    assert size(odd8) > size(odd16)
+    odd16 = syn.scaled(c8, d=2056, weight_dtype=syn.BF16)
+    n_dec = 3 * (odd8.E + odd8.num_shared) * odd8.h * odd8.d * 2
+    assert size(odd8) - size(odd16) >= n_dec
