@@ -1,9 +1,11 @@
-// Per-row E4M3 quantisation of bf16 activation rows, the activation half of
-// the W8A8 expert path.
+// Per-row E4M3 codes of bf16 activation rows, for the expert GEMMs that run
+// on the E4M3 tensor-core kind.
 //
 // ybb.press "MoE 推理工程深层实战" 3.3 lists FP8 (E4M3) as the production
-// format for expert weights.  Running the expert GEMMs on 8-bit activations
-// as well needs one scale per activation row; the reading used here:
+// format for expert weights.  Two ways of feeding the activations:
+//
+// W8A8 (one term).  Running the expert GEMMs on 8-bit activations as well
+// needs one scale per activation row; the reading used here:
 //
 //     s   = amax_j |x_j| / 448          (float32 division; 1 for an all-zero
 //                                        row or a row holding a NaN)
@@ -12,9 +14,7 @@
 //                                        NaN -> 0x7F)
 //
 // so that x_j ~= q_j * s, and the GEMM epilogue multiplies each accumulator
-// row by its s.  One warp per row, two passes over the row (max, then
-// encode; the second pass mostly hits L1/L2), 16-byte loads of 8 bf16 and
-// 8-byte stores of 8 codes.
+// row by its s.
 //
 // Two-term codes (E4M3 weights with bf16 activations).  The tensor cores
 // have no bf16 x E4M3 product, so a bf16 row is written as two E4M3 terms
@@ -34,6 +34,13 @@
 // |v_j| < 0.25 (|x_j| below about amax * 2^-10.8); there the error is at
 // most 2^-10 in v, 2^-17.8 * amax in x.  A row holding an infinity or a NaN
 // gets the scale NaN, so its outputs are NaN.
+//
+// Layout of the work: a row is read twice (max, then codes; the second read
+// mostly hits L1/L2) by a warp, or, when there are few rows (decode), by a
+// whole CTA so that the row's loads spread over 8 warps.  Codes are made two
+// at a time by the paired float -> E4M3 conversion, and the value of c1 is
+// recovered with integer and float arithmetic (below), so the conversion unit
+// sees one instruction per two codes of each term.
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -43,11 +50,24 @@ namespace moe {
 
 namespace {
 
-constexpr int kWarps = 8;  // rows per CTA
+constexpr int kWarps = 8;  // warps per CTA
+constexpr unsigned kFull = 0xFFFFFFFFu;
 
-__device__ __forceinline__ uint8_t e4m3_code(float v) {
-  if (isnan(v)) return 0x7F;
-  return static_cast<uint8_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
+// Two float32 values -> their E4M3 codes (round to nearest even, saturating
+// at +-448; a NaN gives 0x7F), first value in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+  uint32_t q = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  if (isnan(a)) q = (q & 0xFF00u) | 0x7Fu;
+  if (isnan(b)) q = (q & 0x00FFu) | 0x7F00u;
+  return q & 0xFFFFu;
+}
+
+// Value of a finite E4M3 code, exactly: its exponent and mantissa bits placed
+// at the bottom of a float's exponent field and the top of its mantissa give
+// the value times 2^-120 (an E4M3 subnormal becomes a float subnormal, with
+// the same mantissa), and one multiply by 2^120 restores it.
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+  return __uint_as_float(((c & 0x7Fu) << 20) | ((c & 0x80u) << 24)) * 0x1p120f;
 }
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& w, float* f) {
@@ -59,60 +79,63 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& w, float* f) {
   }
 }
 
-// Row scale of d bf16 values (d % 8 == 0), computed by the calling warp.
-__device__ __forceinline__ float row_scale_e4m3(const __nv_bfloat16* __restrict__ src, int d, int lane) {
-  float amax = 0.0f;
-  bool nan = false;
+// Max |x| of a row and whether it holds a NaN / a non-finite value, over T
+// threads (a warp, or the whole CTA) with thread index `tid`.
+template <int T>
+__device__ __forceinline__ void row_amax(const __nv_bfloat16* __restrict__ src, int d, int tid, float& amax,
+                                         bool& nan, bool& nonfinite) {
+  float m = 0.0f;
+  bool n = false, nf = false;
 #pragma unroll 4
-  for (int c = lane * 8; c < d; c += 256) {
+  for (int c = tid * 8; c < d; c += T * 8) {
     float f[8];
     bf16x8_to_f32(ldg16(src + c), f);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      amax = fmaxf(amax, fabsf(f[j]));
-      nan |= isnan(f[j]);
+      m = fmaxf(m, fabsf(f[j]));
+      n |= isnan(f[j]);
+      nf |= !isfinite(f[j]);
     }
   }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-  nan = __any_sync(0xFFFFFFFFu, nan);
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+  n = __any_sync(kFull, n);
+  nf = __any_sync(kFull, nf);
+  if (T > 32) {
+    __shared__ float wm[kWarps];
+    __shared__ int wf[kWarps];
+    const int w = tid >> 5;
+    if ((tid & 31) == 0) {
+      wm[w] = m;
+      wf[w] = (n ? 1 : 0) | (nf ? 2 : 0);
+    }
+    __syncthreads();
+    m = wm[0];
+    int fl = wf[0];
+#pragma unroll
+    for (int i = 1; i < T / 32; ++i) {
+      m = fmaxf(m, wm[i]);
+      fl |= wf[i];
+    }
+    n = fl & 1;
+    nf = fl & 2;
+    __syncthreads();  // the next row's maxima reuse wm / wf
+  }
+  amax = m;
+  nan = n;
+  nonfinite = nf;
+}
+
+// W8A8 scale: amax / 448 (1 for an all-zero row or a row holding a NaN).
+__device__ __forceinline__ float w8a8_scale(float amax, bool nan) {
   return (!nan && amax > 0.0f) ? __fdiv_rn(amax, 448.0f) : 1.0f;
 }
 
-// E4M3 codes of 8 bf16 values for the row scale s, packed in memory order.
-__device__ __forceinline__ uint2 encode8_e4m3(const uint4& w, float s) {
-  float f[8];
-  bf16x8_to_f32(w, f);
-  uint32_t lo = 0, hi = 0;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    lo |= static_cast<uint32_t>(e4m3_code(__fdiv_rn(f[j], s))) << (8 * j);
-    hi |= static_cast<uint32_t>(e4m3_code(__fdiv_rn(f[4 + j], s))) << (8 * j);
-  }
-  return make_uint2(lo, hi);
-}
-
-// Two-term codes: the row's multiplier 2^k (0 for a row with a non-finite
-// value) and its scale 2^-k (NaN for such a row), computed by the calling warp.
-__device__ __forceinline__ float row_pow2_e4m3(const __nv_bfloat16* __restrict__ src, int d, int lane,
-                                               float* scale) {
-  float amax = 0.0f;
-  bool bad = false;
-#pragma unroll 4
-  for (int c = lane * 8; c < d; c += 256) {
-    float f[8];
-    bf16x8_to_f32(ldg16(src + c), f);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      amax = fmaxf(amax, fabsf(f[j]));
-      bad |= !isfinite(f[j]);
-    }
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-  bad = __any_sync(0xFFFFFFFFu, bad);
-  if (bad) {
-    *scale = __int_as_float(0x7FC00000);
+// Two-term multiplier 2^k (0 for a row with a non-finite value) and scale
+// 2^-k (NaN for such a row).
+__device__ __forceinline__ float two_term_mult(float amax, bool nonfinite, float& scale) {
+  if (nonfinite) {
+    scale = __int_as_float(0x7FC00000);
     return 0.0f;
   }
   int k = 0;
@@ -122,104 +145,126 @@ __device__ __forceinline__ float row_pow2_e4m3(const __nv_bfloat16* __restrict__
     k = (f <= 0.875f ? 9 : 8) - ex;     // 448 = 0.875 * 2^9
     k = max(-126, min(126, k));
   }
-  *scale = __int_as_float((127 - k) << 23);
+  scale = __int_as_float((127 - k) << 23);
   return __int_as_float((127 + k) << 23);
 }
 
-__device__ __forceinline__ float e4m3_value(uint8_t c) {
-  return __half2float(__half(__nv_cvt_fp8_to_halfraw(c, __NV_E4M3)));
+// W8A8 codes of 8 bf16 values for the row scale s, in memory order.
+__device__ __forceinline__ uint2 encode8_w8a8(const uint4& w, float s) {
+  float f[8];
+  bf16x8_to_f32(w, f);
+  uint32_t q[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) q[j] = e4m3x2(__fdiv_rn(f[2 * j], s), __fdiv_rn(f[2 * j + 1], s));
+  return make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
 }
 
-// Two-term codes of 8 bf16 values for the multiplier m, each term packed in memory order.
+// Two-term codes of 8 bf16 values for the multiplier m, each term in memory order.
 __device__ __forceinline__ void encode8_two_term(const uint4& w, float m, uint2& t1, uint2& t2) {
   float f[8];
   bf16x8_to_f32(w, f);
-  uint32_t a[2] = {0, 0}, b[2] = {0, 0};
+  uint32_t a[4], b[4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float v = f[j] * m;
-    const uint8_t c1 = e4m3_code(v);
-    const uint8_t c2 = e4m3_code(v - e4m3_value(c1));
-    a[j >> 2] |= static_cast<uint32_t>(c1) << (8 * (j & 3));
-    b[j >> 2] |= static_cast<uint32_t>(c2) << (8 * (j & 3));
+  for (int j = 0; j < 4; ++j) {
+    const float v0 = f[2 * j] * m, v1 = f[2 * j + 1] * m;
+    a[j] = e4m3x2(v0, v1);
+    b[j] = e4m3x2(v0 - e4m3_value(a[j] & 0xFFu), v1 - e4m3_value(a[j] >> 8));
   }
-  t1 = make_uint2(a[0], a[1]);
-  t2 = make_uint2(b[0], b[1]);
+  t1 = make_uint2(a[0] | (a[1] << 16), a[2] | (a[3] << 16));
+  t2 = make_uint2(b[0] | (b[1] << 16), b[2] | (b[3] << 16));
 }
 
-// Two-term codes of one row (d % 8 == 0): term 1 at dst[0, d), term 2 at dst[d, 2d).
-__device__ __forceinline__ void two_term_row(const __nv_bfloat16* __restrict__ src, uint8_t* __restrict__ dst,
-                                             float* __restrict__ scale, int d, int lane) {
-  float sc;
-  const float m = row_pow2_e4m3(src, d, lane, &sc);
+// Codes of one row of d bf16 values (d % 8 == 0) by T threads (thread `tid`):
+// TERMS = 1 (d codes) or 2 (2d codes: first terms, then second terms); the
+// row's scale goes to *scale.
+template <int T>
+__device__ __forceinline__ void code_row(const __nv_bfloat16* __restrict__ src, uint8_t* __restrict__ dst,
+                                         float* __restrict__ scale, int d, int terms, int tid) {
+  float amax;
+  bool nan, nonfinite;
+  row_amax<T>(src, d, tid, amax, nan, nonfinite);
+  if (terms == 2) {
+    float sc;
+    const float m = two_term_mult(amax, nonfinite, sc);
 #pragma unroll 4
-  for (int c = lane * 8; c < d; c += 256) {
-    uint2 t1, t2;
-    encode8_two_term(ldg16(src + c), m, t1, t2);
-    *reinterpret_cast<uint2*>(dst + c) = t1;
-    *reinterpret_cast<uint2*>(dst + d + c) = t2;
+    for (int c = tid * 8; c < d; c += T * 8) {
+      uint2 t1, t2;
+      encode8_two_term(ldg16(src + c), m, t1, t2);
+      *reinterpret_cast<uint2*>(dst + c) = t1;
+      *reinterpret_cast<uint2*>(dst + d + c) = t2;
+    }
+    if (tid == 0) *scale = sc;
+  } else {
+    const float s = w8a8_scale(amax, nan);
+#pragma unroll 4
+    for (int c = tid * 8; c < d; c += T * 8) *reinterpret_cast<uint2*>(dst + c) = encode8_w8a8(ldg16(src + c), s);
+    if (tid == 0) *scale = s;
   }
-  if (lane == 0) *scale = sc;
 }
 
-// Quantise one row of d bf16 values (d % 8 == 0) with the calling warp.
-__device__ __forceinline__ void quantize_row(const __nv_bfloat16* __restrict__ src, uint8_t* __restrict__ dst,
-                                             float* __restrict__ scale, int d, int lane) {
-  const float s = row_scale_e4m3(src, d, lane);
-#pragma unroll 4
-  for (int c = lane * 8; c < d; c += 256) *reinterpret_cast<uint2*>(dst + c) = encode8_e4m3(ldg16(src + c), s);
-  if (lane == 0) *scale = s;
-}
-
-// The permutation's row gather fused with the quantisation: a warp per
-// token computes the token row's scale and codes once and writes them to the
+// The permutation's row gather fused with the coding: token t's row is coded
+// once (by a warp, or by the CTA with T = 256) and the codes go to the
 // token's K rows of the expert-sorted buffer (row_of_slot; -1 = none), and to
-// row t of q_x / s_x when given (the shared expert's operand).  TERMS = 1:
-// W8A8 codes (rows of d bytes); TERMS = 2: two-term codes (rows of 2d bytes).
-template <int TERMS>
+// row t of q_x / s_x when given (the shared expert's operand).  Rows of
+// terms * d codes.
+template <int T>
 __global__ void __launch_bounds__(kWarps * 32)
-    gather_quantize_kernel(int S, int d, int K, const int32_t* __restrict__ row_of_slot,
+    gather_quantize_kernel(int S, int d, int K, int terms, const int32_t* __restrict__ row_of_slot,
                            const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ q_perm,
                            float* __restrict__ s_perm, uint8_t* __restrict__ q_x, float* __restrict__ s_x) {
-  const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
-  if (t >= S) return;
-  const int lane = lane_id();
-  const int my_row = lane < K ? __ldg(row_of_slot + static_cast<int64_t>(t) * K + lane) : -1;
+  const int per_cta = kWarps * 32 / T;
+  const int t = blockIdx.x * per_cta + static_cast<int>(threadIdx.x) / T;
+  const int tid = static_cast<int>(threadIdx.x) % T;
+  if (t >= S) return;  // T = 256: the whole CTA leaves together
+  __shared__ int rows[kWarps][32];
+  int* my_rows = rows[threadIdx.x >> 5];
+  if (T == 32) {
+    if (tid < K) my_rows[tid] = __ldg(row_of_slot + static_cast<int64_t>(t) * K + tid);
+    __syncwarp();
+  } else {
+    if (tid < K) rows[0][tid] = __ldg(row_of_slot + static_cast<int64_t>(t) * K + tid);
+    my_rows = rows[0];
+    __syncthreads();
+  }
   const __nv_bfloat16* src = x + static_cast<int64_t>(t) * d;
-  const int64_t pitch = static_cast<int64_t>(TERMS) * d;
+  const int64_t pitch = static_cast<int64_t>(terms) * d;
+  float amax;
+  bool nan, nonfinite;
+  row_amax<T>(src, d, tid, amax, nan, nonfinite);
   float s = 1.0f, m = 1.0f;
-  if (TERMS == 1)
-    s = row_scale_e4m3(src, d, lane);
+  if (terms == 2)
+    m = two_term_mult(amax, nonfinite, s);
   else
-    m = row_pow2_e4m3(src, d, lane, &s);
-  for (int c = lane * 8; c < d; c += 256) {
+    s = w8a8_scale(amax, nan);
+  for (int c = tid * 8; c < d; c += T * 8) {
     uint2 q, q2 = make_uint2(0, 0);
-    if (TERMS == 1)
-      q = encode8_e4m3(ldg16(src + c), s);
-    else
+    if (terms == 2)
       encode8_two_term(ldg16(src + c), m, q, q2);
+    else
+      q = encode8_w8a8(ldg16(src + c), s);
     for (int k = 0; k < K; ++k) {
-      const int row = __shfl_sync(0xFFFFFFFFu, my_row, k);
+      const int row = my_rows[k];
       if (row >= 0) {
         *reinterpret_cast<uint2*>(q_perm + row * pitch + c) = q;
-        if (TERMS == 2) *reinterpret_cast<uint2*>(q_perm + row * pitch + d + c) = q2;
+        if (terms == 2) *reinterpret_cast<uint2*>(q_perm + row * pitch + d + c) = q2;
       }
     }
     if (q_x != nullptr) {
       *reinterpret_cast<uint2*>(q_x + t * pitch + c) = q;
-      if (TERMS == 2) *reinterpret_cast<uint2*>(q_x + t * pitch + d + c) = q2;
+      if (terms == 2) *reinterpret_cast<uint2*>(q_x + t * pitch + d + c) = q2;
     }
   }
-  if (my_row >= 0) s_perm[my_row] = s;
-  if (lane == 0 && s_x != nullptr) s_x[t] = s;
+  if (tid < K && my_rows[tid] >= 0) s_perm[my_rows[tid]] = s;
+  if (tid == 0 && s_x != nullptr) s_x[t] = s;
 }
 
 // Rows of a group table (groups != nullptr) or `single_rows` contiguous rows.
 // The rows of all groups form one flat range (a prefix over the groups'
-// row counts in shared memory); each warp takes rows of it with a grid
-// stride, so the grid is sized by the rows there are, not by groups x the
-// largest group.
+// row counts in shared memory); each warp (T = 32) or CTA (T = 256) takes
+// rows of it with a grid stride, so the grid is sized by the rows there are,
+// not by groups x the largest group.
 constexpr int kQuantMaxGroups = 520;
+template <int T>
 __global__ void __launch_bounds__(kWarps * 32)
     quantize_rows_kernel(const GroupEntry* __restrict__ groups, int num_groups, int use_out_rows, int shared_slab,
                          int64_t single_rows, const __nv_bfloat16* __restrict__ src, uint8_t* __restrict__ dst,
@@ -238,19 +283,21 @@ __global__ void __launch_bounds__(kWarps * 32)
         int64_t incl = rows;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
-          const int64_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+          const int64_t o = __shfl_up_sync(kFull, incl, off);
           if (lane >= off) incl += o;
         }
         if (g < num_groups) start[g] = carry + incl - rows;
-        carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        carry += __shfl_sync(kFull, incl, 31);
       }
       if (lane == 0) start[num_groups] = carry;
     }
     __syncthreads();
     total = start[num_groups];
   }
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * kWarps + warp; i < total;
-       i += static_cast<int64_t>(gridDim.x) * kWarps) {
+  const int per_cta = kWarps * 32 / T;
+  const int tid = static_cast<int>(threadIdx.x) % T;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * per_cta + static_cast<int>(threadIdx.x) / T; i < total;
+       i += static_cast<int64_t>(gridDim.x) * per_cta) {
     int64_t row;
     bool shared = false;
     if (groups == nullptr) {
@@ -269,54 +316,76 @@ __global__ void __launch_bounds__(kWarps * 32)
       row = (shared ? 0 : (use_out_rows ? g.out_row0 : g.a_row0)) + (i - start[lo]);
     }
     // rows outside the buffers (a corrupt table) are skipped; the GEMM reports the group
+    // (uniform over the T threads of the row, so a CTA row never splits at its barriers)
     if (row < 0 || row >= (shared ? sh_rows : dst_rows)) continue;
     const __nv_bfloat16* in = shared ? src_sh + row * d : src + row * d;
     uint8_t* out = (shared ? dst_sh : dst) + row * terms * d;
     float* sc = (shared ? scale_sh : scale) + row;
-    if (terms == 2)
-      two_term_row(in, out, sc, d, lane);
-    else
-      quantize_row(in, out, sc, d, lane);
+    code_row<T>(in, out, sc, d, terms, tid);
   }
 }
 
-}  // namespace
-
-// Grid of the row quantisation: enough warps for `rows`, at most 16 CTAs per SM.
-dim3 quantize_grid(int64_t rows) {
+int device_sms() {
   static int sms = 0;
   if (sms == 0) {
     int dev = 0;
     cudaGetDevice(&dev);
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
   }
-  const int64_t want = (rows + kWarps - 1) / kWarps;
-  return dim3(static_cast<unsigned>(want < 16 * sms ? (want > 0 ? want : 1) : 16 * sms));
+  return sms;
 }
+
+// Few rows (up to four per SM): a CTA per row; otherwise a warp per row.
+bool cta_rows(int64_t rows) { return rows <= 4 * static_cast<int64_t>(device_sms()); }
+
+// Grid of the row coding: enough warps (or CTAs) for `rows`, at most 16 CTAs per SM.
+dim3 quantize_grid(int64_t rows) {
+  const int64_t per_cta = cta_rows(rows) ? 1 : kWarps;
+  const int64_t want = (rows + per_cta - 1) / per_cta;
+  const int64_t cap = 16 * static_cast<int64_t>(device_sms());
+  return dim3(static_cast<unsigned>(want < cap ? (want > 0 ? want : 1) : cap));
+}
+
+cudaError_t launch_rows(const GroupEntry* groups, int num_groups, int use_out_rows, int shared_slab,
+                        int64_t single_rows, const void* src, uint8_t* dst, float* scale, int64_t dst_rows,
+                        const void* src_sh, uint8_t* dst_sh, float* scale_sh, int64_t sh_rows, int d, int terms,
+                        int64_t max_rows, cudaStream_t stream) {
+  const dim3 grid = quantize_grid(max_rows);
+  const auto* s = static_cast<const __nv_bfloat16*>(src);
+  const auto* ss = static_cast<const __nv_bfloat16*>(src_sh);
+  if (cta_rows(max_rows))
+    quantize_rows_kernel<kWarps * 32><<<grid, kWarps * 32, 0, stream>>>(groups, num_groups, use_out_rows,
+                                                                         shared_slab, single_rows, s, dst, scale,
+                                                                         dst_rows, ss, dst_sh, scale_sh, sh_rows, d,
+                                                                         terms);
+  else
+    quantize_rows_kernel<32><<<grid, kWarps * 32, 0, stream>>>(groups, num_groups, use_out_rows, shared_slab,
+                                                               single_rows, s, dst, scale, dst_rows, ss, dst_sh,
+                                                               scale_sh, sh_rows, d, terms);
+  return cudaGetLastError();
+}
+
+}  // namespace
 
 cudaError_t launch_quantize_rows(const void* src, uint8_t* dst, float* scale, int64_t rows, int d, int terms,
                                  cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
   if (d <= 0 || d % 8 != 0 || (terms != 1 && terms != 2)) return cudaErrorInvalidValue;
-  quantize_rows_kernel<<<quantize_grid(rows), kWarps * 32, 0, stream>>>(
-      nullptr, 0, 0, -1, rows, static_cast<const __nv_bfloat16*>(src), dst, scale, rows, nullptr, nullptr, nullptr, 0,
-      d, terms);
-  return cudaGetLastError();
+  return launch_rows(nullptr, 0, 0, -1, rows, src, dst, scale, rows, nullptr, nullptr, nullptr, 0, d, terms, rows,
+                     stream);
 }
 
 cudaError_t launch_gather_quantize(int S, int d, int K, const int32_t* row_of_slot, const void* x, uint8_t* q_perm,
                                    float* s_perm, uint8_t* q_x, float* s_x, int terms, cudaStream_t stream) {
   if (S <= 0) return cudaSuccess;
   if (d <= 0 || d % 8 != 0 || K < 1 || K > 32 || (terms != 1 && terms != 2)) return cudaErrorInvalidValue;
-  const dim3 grid((S + kWarps - 1) / kWarps);
-  if (terms == 2)
-    gather_quantize_kernel<2><<<grid, kWarps * 32, 0, stream>>>(S, d, K, row_of_slot,
-                                                                 static_cast<const __nv_bfloat16*>(x), q_perm,
-                                                                 s_perm, q_x, s_x);
+  const auto* xs = static_cast<const __nv_bfloat16*>(x);
+  if (cta_rows(S))
+    gather_quantize_kernel<kWarps * 32><<<S, kWarps * 32, 0, stream>>>(S, d, K, terms, row_of_slot, xs, q_perm,
+                                                                        s_perm, q_x, s_x);
   else
-    gather_quantize_kernel<1><<<grid, kWarps * 32, 0, stream>>>(S, d, K, row_of_slot,
-                                                                 static_cast<const __nv_bfloat16*>(x), q_perm,
-                                                                 s_perm, q_x, s_x);
+    gather_quantize_kernel<32><<<(S + kWarps - 1) / kWarps, kWarps * 32, 0, stream>>>(S, d, K, terms, row_of_slot,
+                                                                                      xs, q_perm, s_perm, q_x, s_x);
   return cudaGetLastError();
 }
 
@@ -328,10 +397,8 @@ cudaError_t launch_quantize_group_rows(const GroupEntry* groups, int num_groups,
   if (num_groups <= 0 || max_total_rows <= 0) return cudaSuccess;
   if (num_groups > kQuantMaxGroups || d <= 0 || d % 8 != 0 || (terms != 1 && terms != 2))
     return cudaErrorInvalidValue;
-  quantize_rows_kernel<<<quantize_grid(max_total_rows), kWarps * 32, 0, stream>>>(
-      groups, num_groups, use_out_rows, shared_slab, 0, static_cast<const __nv_bfloat16*>(src), dst, scale, dst_rows,
-      static_cast<const __nv_bfloat16*>(src_shared), dst_shared, scale_shared, shared_rows, d, terms);
-  return cudaGetLastError();
+  return launch_rows(groups, num_groups, use_out_rows, shared_slab, 0, src, dst, scale, dst_rows, src_shared,
+                     dst_shared, scale_shared, shared_rows, d, terms, max_total_rows, stream);
 }
 
 }  // namespace moe
