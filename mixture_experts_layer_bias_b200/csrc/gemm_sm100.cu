@@ -266,7 +266,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int A_TERM = bma * BK_BYTES;              // one A tile (rows x 128 bytes of K)
   const int A_TERMS = F8 ? p.a_terms : 1;         // two-term E4M3 activations: two A tiles per stage
   const int A_TILE = A_TERM * A_TERMS;
-  const int STAGE_BYTES = A_TILE + B_TILE;
+  // Stage layout.  Usually [A term 1][A term 2][B].  Packed two-term A (groups
+  // of at most 64 rows): [B][A term 1 at rows 0..][A term 2 at rows 64..], so
+  // one M=128 MMA multiplies both terms (accumulator lanes 0..63 and 64..127;
+  // the 128-row read runs past the stage's end into garbage rows that are
+  // never stored).
+  const bool PACK = F8 && p.a_pack;
+  const int B_OFF = PACK ? 0 : A_TILE;
+  const int A_OFF = PACK ? B_TILE : 0;
+  const int A2_OFF = PACK ? B_TILE + 64 * BK_BYTES : A_TERM;
+  const int STAGE_BYTES = PACK ? B_TILE + 64 * BK_BYTES + A_TERM : A_TILE + B_TILE;
   uint8_t* ctl = ring + STAGES * STAGE_BYTES;
   SmemCtl& s = *reinterpret_cast<SmemCtl*>(ctl);
   uint8_t* epi_smem = reinterpret_cast<uint8_t*>(
@@ -333,8 +342,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s.tmem_base;
   const int nk = (p.K + BK - 1) / BK;
   const int tiles = s.tile_start[p.num_groups];
-  const int ks = choose_ksplit(tiles, gridDim.x, nk, p.max_ksplit);
-  if (blockIdx.x == 0 && threadIdx.x == 0 && p.ksplit_out != nullptr) *p.ksplit_out = ks;
+  // packed two-term A: the second term's accumulator rows are one more set of
+  // K slices, so every unit writes partial sums and the finalize adds 2 ks slices
+  const int ks = choose_ksplit(tiles, gridDim.x, nk, PACK ? p.max_ksplit / 2 : p.max_ksplit);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && p.ksplit_out != nullptr) *p.ksplit_out = PACK ? 2 * ks : ks;
   const int total = tiles * ks;  // work units
   volatile int* abort_flag = &s.abort;
 
@@ -355,13 +366,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&s.full[stage], STAGE_BYTES);
+          mbar_arrive_expect_tx(&s.full[stage], A_TILE + B_TILE);
           armed |= 1u << stage;
           armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
-          uint8_t* sa = ring + stage * STAGE_BYTES;
-          uint8_t* sb = sa + A_TILE;
-          tma_load_2d(sa, mA, kb * BK, a_row, &s.full[stage]);
-          if (F8 && A_TERMS == 2) tma_load_2d(sa + A_TERM, mA, p.K + kb * BK, a_row, &s.full[stage]);
+          uint8_t* st = ring + stage * STAGE_BYTES;
+          uint8_t* sb = st + B_OFF;
+          tma_load_2d(st + A_OFF, mA, kb * BK, a_row, &s.full[stage]);
+          if (F8 && A_TERMS == 2) tma_load_2d(st + A2_OFF, mA, p.K + kb * BK, a_row, &s.full[stage]);
           if (EPI == EPI_SWIGLU) {
             tma_load_2d(sb, &tmB0, kb * BK, b_row, &s.full[stage]);
             tma_load_2d(sb + B_HALF, &tmB1, kb * BK, b_row, &s.full[stage]);
@@ -407,11 +418,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(ring + stage * STAGE_BYTES);
-          const uint32_t b_base = a_base + A_TILE;
+          const uint32_t st_base = smem_u32(ring + stage * STAGE_BYTES);
+          const uint32_t a_base = st_base + A_OFF;
+          const uint32_t b_base = st_base + B_OFF;
           if (F8) {
             // one or two A terms against the same weight tile, one fp32 sum
-            for (int t = 0; t < A_TERMS; ++t) {
+            // (packed: one MMA covers both terms' rows)
+            for (int t = 0; t < (PACK ? 1 : A_TERMS); ++t) {
 #pragma unroll
               for (int kk = 0; kk < BK_BYTES / 32; ++kk)  // 32 E4M3 of K per MMA
                 tc_mma_f8(d_tmem, smem_desc_sw128(a_base + t * A_TERM + kk * 32), smem_desc_sw128(b_base + kk * 32),
@@ -458,10 +471,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int row = ti.m_idx * BM + q * 32 + lane;
+      // packed two-term A: lane quarters 2, 3 hold the second term's sums of
+      // the rows of quarters 0, 1, written as K slices ks .. 2 ks - 1
+      const int row = ti.m_idx * BM + (PACK ? (q & 1) : q) * 32 + lane;
       const bool valid = row < ti.grp.rows;
       const uint32_t tbase = tmem + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16);
-      if (ks > 1)
+      if (PACK)
+        epilogue_partial<EPI>(p, ti, tbase, row, valid, ui.split + (q >> 1) * ks, half);
+      else if (ks > 1)
         epilogue_partial<EPI>(p, ti, tbase, row, valid, ui.split, half);
       else
         epilogue_store<EPI>(p, ti, tbase, row, valid, lane, half, &tmOut, epi_smem + (warp - 2) * kEpiWarpBytes);
@@ -512,7 +529,10 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
   int bma = BM;
   if (a.max_group_rows > 0 && a.max_group_rows <= 64) bma = static_cast<int>((a.max_group_rows + 15) & ~int64_t(15));
   const int terms = a.fp8 && a.a_terms == 2 ? 2 : 1;  // two-term E4M3 activations: A rows of 2K codes
-  const size_t stage_bytes = static_cast<size_t>(bma) * BK_BYTES * terms + B_TILE;
+  // both terms in one MMA when every group fits in 64 rows (split-K buffer needed for the second term's sums)
+  const bool pack = terms == 2 && bma <= 64 && p.max_ksplit >= 2;
+  const size_t stage_bytes = pack ? static_cast<size_t>(B_TILE + 64 * BK_BYTES + bma * BK_BYTES)
+                                  : static_cast<size_t>(bma) * BK_BYTES * terms + B_TILE;
   const int eb = a.fp8 ? 1 : 2;  // element bytes of A and B
   int stages = static_cast<int>((kSmemLimitTc - kCtlBytes) / stage_bytes);
   if (stages > MAX_STAGES) stages = MAX_STAGES;
@@ -523,6 +543,7 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
   pp.tma_out = !a.out_f32 && make_store_map(&mOut, a.out, a.out_rows, a.N, 2) ? 1 : 0;
   if (!pp.tma_out) memset(&mOut, 0, sizeof(mOut));
   pp.a_terms = terms;
+  pp.a_pack = pack ? 1 : 0;
   if (!make_map(&mA, a.a, a.a_rows, a.K * terms, bma, eb)) return cudaErrorInvalidValue;
   if (a.a_shared != nullptr) {
     if (!make_map(&mA2, a.a_shared, a.a_shared_rows, a.K * terms, bma, eb)) return cudaErrorInvalidValue;

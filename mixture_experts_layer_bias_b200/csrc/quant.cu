@@ -79,24 +79,42 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& w, float* f) {
   }
 }
 
-// Max |x| of a row and whether it holds a NaN / a non-finite value, over T
-// threads (a warp, or the whole CTA) with thread index `tid`.
+// A row's 16-byte pieces held by one of T threads (a warp, or the whole CTA):
+// pieces tid, tid + T, ... up to kVec of them stay in registers, so the row
+// is read from memory once; pieces beyond T * kVec (rows longer than the
+// launch's choice of T allows) are read again when coded.
+constexpr int kVec = 8;
+
 template <int T>
-__device__ __forceinline__ void row_amax(const __nv_bfloat16* __restrict__ src, int d, int tid, float& amax,
-                                         bool& nan, bool& nonfinite) {
+struct RowPieces {
+  uint4 v[kVec];
+};
+
+// Loads the thread's pieces and reduces max |x| and the NaN / non-finite
+// flags over the T threads.
+template <int T>
+__device__ __forceinline__ void row_load_amax(const __nv_bfloat16* __restrict__ src, int d, int tid,
+                                              RowPieces<T>& rp, float& amax, bool& nan, bool& nonfinite) {
   float m = 0.0f;
   bool n = false, nf = false;
-#pragma unroll 4
-  for (int c = tid * 8; c < d; c += T * 8) {
+#pragma unroll
+  for (int i = 0; i < kVec; ++i) {
+    const int c = (tid + i * T) * 8;
+    rp.v[i] = c < d ? ldg16(src + c) : make_uint4(0, 0, 0, 0);
+  }
+  auto acc = [&](const uint4& w) {
     float f[8];
-    bf16x8_to_f32(ldg16(src + c), f);
+    bf16x8_to_f32(w, f);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       m = fmaxf(m, fabsf(f[j]));
       n |= isnan(f[j]);
       nf |= !isfinite(f[j]);
     }
-  }
+  };
+#pragma unroll
+  for (int i = 0; i < kVec; ++i) acc(rp.v[i]);  // zero pieces past the row change nothing
+  for (int c = (tid + kVec * T) * 8; c < d; c += T * 8) acc(ldg16(src + c));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
   n = __any_sync(kFull, n);
@@ -174,32 +192,48 @@ __device__ __forceinline__ void encode8_two_term(const uint4& w, float m, uint2&
   t2 = make_uint2(b[0] | (b[1] << 16), b[2] | (b[3] << 16));
 }
 
+// Scale (and two-term multiplier) of a row from its maximum.
+__device__ __forceinline__ void row_scale(int terms, float amax, bool nan, bool nonfinite, float& s, float& m) {
+  if (terms == 2) {
+    m = two_term_mult(amax, nonfinite, s);
+  } else {
+    s = w8a8_scale(amax, nan);
+    m = 1.0f;
+  }
+}
+
+// Codes of the row piece starting at column c: term codes to dst[c..] (and
+// dst[d + c..] for two terms).
+__device__ __forceinline__ void code_piece(const uint4& w, uint8_t* __restrict__ dst, int d, int c, int terms,
+                                           float s, float m) {
+  if (terms == 2) {
+    uint2 t1, t2;
+    encode8_two_term(w, m, t1, t2);
+    *reinterpret_cast<uint2*>(dst + c) = t1;
+    *reinterpret_cast<uint2*>(dst + d + c) = t2;
+  } else {
+    *reinterpret_cast<uint2*>(dst + c) = encode8_w8a8(w, s);
+  }
+}
+
 // Codes of one row of d bf16 values (d % 8 == 0) by T threads (thread `tid`):
-// TERMS = 1 (d codes) or 2 (2d codes: first terms, then second terms); the
+// terms = 1 (d codes) or 2 (2d codes: first terms, then second terms); the
 // row's scale goes to *scale.
 template <int T>
 __device__ __forceinline__ void code_row(const __nv_bfloat16* __restrict__ src, uint8_t* __restrict__ dst,
                                          float* __restrict__ scale, int d, int terms, int tid) {
-  float amax;
+  RowPieces<T> rp;
+  float amax, s, m;
   bool nan, nonfinite;
-  row_amax<T>(src, d, tid, amax, nan, nonfinite);
-  if (terms == 2) {
-    float sc;
-    const float m = two_term_mult(amax, nonfinite, sc);
-#pragma unroll 4
-    for (int c = tid * 8; c < d; c += T * 8) {
-      uint2 t1, t2;
-      encode8_two_term(ldg16(src + c), m, t1, t2);
-      *reinterpret_cast<uint2*>(dst + c) = t1;
-      *reinterpret_cast<uint2*>(dst + d + c) = t2;
-    }
-    if (tid == 0) *scale = sc;
-  } else {
-    const float s = w8a8_scale(amax, nan);
-#pragma unroll 4
-    for (int c = tid * 8; c < d; c += T * 8) *reinterpret_cast<uint2*>(dst + c) = encode8_w8a8(ldg16(src + c), s);
-    if (tid == 0) *scale = s;
+  row_load_amax<T>(src, d, tid, rp, amax, nan, nonfinite);
+  row_scale(terms, amax, nan, nonfinite, s, m);
+#pragma unroll
+  for (int i = 0; i < kVec; ++i) {
+    const int c = (tid + i * T) * 8;
+    if (c < d) code_piece(rp.v[i], dst, d, c, terms, s, m);
   }
+  for (int c = (tid + kVec * T) * 8; c < d; c += T * 8) code_piece(ldg16(src + c), dst, d, c, terms, s, m);
+  if (tid == 0) *scale = s;
 }
 
 // The permutation's row gather fused with the coding: token t's row is coded
@@ -228,20 +262,17 @@ __global__ void __launch_bounds__(kWarps * 32)
   }
   const __nv_bfloat16* src = x + static_cast<int64_t>(t) * d;
   const int64_t pitch = static_cast<int64_t>(terms) * d;
-  float amax;
+  RowPieces<T> rp;
+  float amax, s, m;
   bool nan, nonfinite;
-  row_amax<T>(src, d, tid, amax, nan, nonfinite);
-  float s = 1.0f, m = 1.0f;
-  if (terms == 2)
-    m = two_term_mult(amax, nonfinite, s);
-  else
-    s = w8a8_scale(amax, nan);
-  for (int c = tid * 8; c < d; c += T * 8) {
+  row_load_amax<T>(src, d, tid, rp, amax, nan, nonfinite);
+  row_scale(terms, amax, nan, nonfinite, s, m);
+  auto put = [&](const uint4& w, int c) {
     uint2 q, q2 = make_uint2(0, 0);
     if (terms == 2)
-      encode8_two_term(ldg16(src + c), m, q, q2);
+      encode8_two_term(w, m, q, q2);
     else
-      q = encode8_w8a8(ldg16(src + c), s);
+      q = encode8_w8a8(w, s);
     for (int k = 0; k < K; ++k) {
       const int row = my_rows[k];
       if (row >= 0) {
@@ -253,7 +284,13 @@ __global__ void __launch_bounds__(kWarps * 32)
       *reinterpret_cast<uint2*>(q_x + t * pitch + c) = q;
       if (terms == 2) *reinterpret_cast<uint2*>(q_x + t * pitch + d + c) = q2;
     }
+  };
+#pragma unroll
+  for (int i = 0; i < kVec; ++i) {
+    const int c = (tid + i * T) * 8;
+    if (c < d) put(rp.v[i], c);
   }
+  for (int c = (tid + kVec * T) * 8; c < d; c += T * 8) put(ldg16(src + c), c);
   if (tid < K && my_rows[tid] >= 0) s_perm[my_rows[tid]] = s;
   if (tid == 0 && s_x != nullptr) s_x[t] = s;
 }
@@ -335,12 +372,15 @@ int device_sms() {
   return sms;
 }
 
-// Few rows (up to four per SM): a CTA per row; otherwise a warp per row.
-bool cta_rows(int64_t rows) { return rows <= 4 * static_cast<int64_t>(device_sms()); }
+// A CTA per row when there are few rows (up to four per SM: decode) or rows
+// too long for a warp to hold in registers; otherwise a warp per row.
+bool cta_rows(int64_t rows, int d) {
+  return rows <= 4 * static_cast<int64_t>(device_sms()) || d > 32 * 8 * kVec;
+}
 
 // Grid of the row coding: enough warps (or CTAs) for `rows`, at most 16 CTAs per SM.
-dim3 quantize_grid(int64_t rows) {
-  const int64_t per_cta = cta_rows(rows) ? 1 : kWarps;
+dim3 quantize_grid(int64_t rows, int d) {
+  const int64_t per_cta = cta_rows(rows, d) ? 1 : kWarps;
   const int64_t want = (rows + per_cta - 1) / per_cta;
   const int64_t cap = 16 * static_cast<int64_t>(device_sms());
   return dim3(static_cast<unsigned>(want < cap ? (want > 0 ? want : 1) : cap));
@@ -350,10 +390,10 @@ cudaError_t launch_rows(const GroupEntry* groups, int num_groups, int use_out_ro
                         int64_t single_rows, const void* src, uint8_t* dst, float* scale, int64_t dst_rows,
                         const void* src_sh, uint8_t* dst_sh, float* scale_sh, int64_t sh_rows, int d, int terms,
                         int64_t max_rows, cudaStream_t stream) {
-  const dim3 grid = quantize_grid(max_rows);
+  const dim3 grid = quantize_grid(max_rows, d);
   const auto* s = static_cast<const __nv_bfloat16*>(src);
   const auto* ss = static_cast<const __nv_bfloat16*>(src_sh);
-  if (cta_rows(max_rows))
+  if (cta_rows(max_rows, d))
     quantize_rows_kernel<kWarps * 32><<<grid, kWarps * 32, 0, stream>>>(groups, num_groups, use_out_rows,
                                                                          shared_slab, single_rows, s, dst, scale,
                                                                          dst_rows, ss, dst_sh, scale_sh, sh_rows, d,
@@ -380,7 +420,7 @@ cudaError_t launch_gather_quantize(int S, int d, int K, const int32_t* row_of_sl
   if (S <= 0) return cudaSuccess;
   if (d <= 0 || d % 8 != 0 || K < 1 || K > 32 || (terms != 1 && terms != 2)) return cudaErrorInvalidValue;
   const auto* xs = static_cast<const __nv_bfloat16*>(x);
-  if (cta_rows(S))
+  if (cta_rows(S, d))
     gather_quantize_kernel<kWarps * 32><<<S, kWarps * 32, 0, stream>>>(S, d, K, terms, row_of_slot, xs, q_perm,
                                                                         s_perm, q_x, s_x);
   else
