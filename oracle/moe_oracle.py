@@ -775,7 +775,7 @@ def split_rows_e4m3(rows: np.ndarray):
         c1 = E4M3(v)                  (round to nearest even)
         c2 = E4M3(v - value(c1))      (float32 difference)
         scale = 2**-k                 (NaN when the row holds an inf or NaN;
-                                       v = x * 0 then)
+                                       its codes are then all zero)
 
     Returns (c1 uint8 [n, d], c2 uint8 [n, d], scale float32 [n]); the row is
     (value(c1) + value(c2)) * scale."""
@@ -787,7 +787,8 @@ def split_rows_e4m3(rows: np.ndarray):
     for i in range(n):
         row = x[i]
         if not np.all(np.isfinite(row)):
-            mult, scale[i] = np.float32(0.0), np.float32(np.nan)
+            scale[i] = np.float32(np.nan)  # the row's outputs are NaN through its scale
+            continue
         else:
             amax = float(np.max(np.abs(row.astype(np.float64)))) if d else 0.0
             k = 0

@@ -650,7 +650,7 @@ def test_split_rows_error_bound_and_special_rows():
     """Values far below the row maximum lose at most 2**-10 of the scaled
     value (half the E4M3 subnormal spacing); a zero row has scale 1 and zero
     codes; a row maximum of exactly 448 * 2**j gives scale 2**j; a row with an
-    infinity or a NaN gets the scale NaN."""
+    infinity or a NaN gets the scale NaN and zero codes."""
     rng = np.random.default_rng(32)
     x = _bf16_rows(rng, 30, 128, 30.0)
     c1, c2, s = O.split_rows_e4m3(x)
@@ -666,6 +666,7 @@ def test_split_rows_error_bound_and_special_rows():
     assert s[0] == 1.0 and not c1[0].any() and not c2[0].any()
     assert s[1] == 8.0 and c1[1, 3] == 0x7E and c2[1, 3] == 0
     assert np.isnan(s[2]) and np.isnan(s[3])
+    assert not c1[2:].any() and not c2[2:].any()
 
 
 def test_w8a8_expert_close_to_exact_expert():
