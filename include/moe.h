@@ -310,7 +310,8 @@ moe_status moe_quantize_rows_e4m3(const void *x, int64_t rows, int32_t d, uint8_
  *   v_j     = x[i][j] * 2^k (exact);
  *   q[i][j]     = E4M3(v_j), round to nearest even;
  *   q[i][d + j] = E4M3(v_j - q[i][j]) (the difference exact in fp32);
- *   s[i]    = 2^-k, or NaN when the row holds an infinity or a NaN.
+ *   s[i]    = 2^-k, or NaN when the row holds an infinity or a NaN
+ *             (its codes are then all zero).
  * Then q[i][j] + q[i][d+j] = v_j exactly whenever |v_j| >= 1/4; below that
  * the error is at most 2^-10 in v_j.  q [rows][2d] uint8 and s [rows] fp32
  * are caller-owned DEVICE buffers (q 16-byte aligned).  Launches one kernel

@@ -408,12 +408,12 @@ moe_status ffn_impl(const moe_desc& d, const moe_weights& w, const void* x_perm,
     return launch_quantize_group_rows(g.groups, g.num_groups, 0, g.shared_slab, x_perm, at<uint8_t>(ws, L.qa),
                                       at<float>(ws, L.sa), R, x, d.num_shared ? at<uint8_t>(ws, L.qas) : nullptr,
                                       d.num_shared ? at<float>(ws, L.sas) : nullptr, S, dm, g.max_total_rows, terms,
-                                      st);
+                                      status, st);
   };
   auto quant_down = [&](const GemmArgs& g) {
     return launch_quantize_group_rows(g.groups, g.num_groups, 1, -1, hidden, at<uint8_t>(ws, L.qh),
                                       at<float>(ws, L.sh), Rt, nullptr, nullptr, nullptr, 0, h, g.max_total_rows,
-                                      terms, st);
+                                      terms, status, st);
   };
   if (terms && !a_quantized && (err = quant_up(up)) != cudaSuccess) return MOE_ERR_CUDA;
   if (!record(events, 3, st)) return MOE_ERR_CUDA;

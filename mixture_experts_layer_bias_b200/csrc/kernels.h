@@ -154,7 +154,7 @@ cudaError_t launch_quantize_group_rows(const GroupEntry* groups, int num_groups,
                                        const void* src, uint8_t* dst, float* scale, int64_t dst_rows,
                                        const void* src_shared, uint8_t* dst_shared, float* scale_shared,
                                        int64_t shared_rows, int d, int64_t max_total_rows, int terms,
-                                       cudaStream_t stream);
+                                       StatusBlock* status, cudaStream_t stream);
 
 // --- sliding-window load and selection-bias update ---------------------------
 size_t bias_state_bytes(int E, int K, int window);

@@ -43,6 +43,8 @@
 // sees one instruction per two codes of each term.
 #include <cuda_fp8.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -53,13 +55,18 @@ namespace {
 constexpr int kWarps = 8;  // warps per CTA
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
-// Two float32 values -> their E4M3 codes (round to nearest even, saturating
-// at +-448; a NaN gives 0x7F), first value in the low byte.
+// Two finite float32 values -> their E4M3 codes (round to nearest even,
+// saturating at +-448), first value in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2_finite(float a, float b) {
+  return __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3) & 0xFFFFu;
+}
+
+// The same for any values, a NaN giving 0x7F.
 __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
-  uint32_t q = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  uint32_t q = e4m3x2_finite(a, b);
   if (isnan(a)) q = (q & 0xFF00u) | 0x7Fu;
   if (isnan(b)) q = (q & 0x00FFu) | 0x7F00u;
-  return q & 0xFFFFu;
+  return q;
 }
 
 // Value of a finite E4M3 code, exactly: its exponent and mantissa bits placed
@@ -149,8 +156,8 @@ __device__ __forceinline__ float w8a8_scale(float amax, bool nan) {
   return (!nan && amax > 0.0f) ? __fdiv_rn(amax, 448.0f) : 1.0f;
 }
 
-// Two-term multiplier 2^k (0 for a row with a non-finite value) and scale
-// 2^-k (NaN for such a row).
+// Two-term multiplier 2^k (0 for a row with a non-finite value, whose codes
+// are all zero) and scale 2^-k (NaN for such a row).
 __device__ __forceinline__ float two_term_mult(float amax, bool nonfinite, float& scale) {
   if (nonfinite) {
     scale = __int_as_float(0x7FC00000);
@@ -177,16 +184,21 @@ __device__ __forceinline__ uint2 encode8_w8a8(const uint4& w, float s) {
   return make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
 }
 
-// Two-term codes of 8 bf16 values for the multiplier m, each term in memory order.
+// Two-term codes of 8 bf16 values for the multiplier m, each term in memory
+// order (zero codes for m = 0: a row with a non-finite value).
 __device__ __forceinline__ void encode8_two_term(const uint4& w, float m, uint2& t1, uint2& t2) {
+  if (m == 0.0f) {
+    t1 = t2 = make_uint2(0, 0);
+    return;
+  }
   float f[8];
   bf16x8_to_f32(w, f);
   uint32_t a[4], b[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const float v0 = f[2 * j] * m, v1 = f[2 * j + 1] * m;
-    a[j] = e4m3x2(v0, v1);
-    b[j] = e4m3x2(v0 - e4m3_value(a[j] & 0xFFu), v1 - e4m3_value(a[j] >> 8));
+    const float v0 = f[2 * j] * m, v1 = f[2 * j + 1] * m;  // finite, |v| <= 448
+    a[j] = e4m3x2_finite(v0, v1);
+    b[j] = e4m3x2_finite(v0 - e4m3_value(a[j] & 0xFFu), v1 - e4m3_value(a[j] >> 8));
   }
   t1 = make_uint2(a[0] | (a[1] << 16), a[2] | (a[3] << 16));
   t2 = make_uint2(b[0] | (b[1] << 16), b[2] | (b[3] << 16));
@@ -362,6 +374,164 @@ __global__ void __launch_bounds__(kWarps * 32)
   }
 }
 
+// 1-D bulk copy global -> shared of `bytes` (a multiple of 16, both addresses
+// 16-byte aligned), completion counted on `bar` in bytes.  No multicast.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(smem_dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// Many rows of at most kStagedMaxCols columns: each CTA codes chunks of
+// `chunk` consecutive rows of the flat row range.  Warp 0 stages a chunk's
+// rows in shared memory by bulk copies (one per row), into one of two chunk
+// buffers, so the next chunk streams in while the warps code this one (a row
+// per warp: max, then codes, both from shared memory).  The waits on the
+// copies are bounded; a CTA that gives up reports MOE_STATUS_TIMEOUT, lets its
+// copies in flight land (bounded again) and exits.
+constexpr int kStagedMaxCols = 4096;
+constexpr int kMaxChunk = 32;
+__global__ void __launch_bounds__(kWarps * 32)
+    quantize_rows_staged_kernel(const GroupEntry* __restrict__ groups, int num_groups, int use_out_rows,
+                                int shared_slab, int64_t single_rows, const __nv_bfloat16* __restrict__ src,
+                                uint8_t* __restrict__ dst, float* __restrict__ scale, int64_t dst_rows,
+                                const __nv_bfloat16* __restrict__ src_sh, uint8_t* __restrict__ dst_sh,
+                                float* __restrict__ scale_sh, int64_t sh_rows, int d, int terms, int chunk,
+                                StatusBlock* status) {
+  extern __shared__ __align__(128) uint8_t stage[];  // [2][chunk][d] bf16
+  __shared__ int64_t start[kQuantMaxGroups + 1];
+  __shared__ __align__(8) uint64_t full[2];
+  __shared__ int64_t row_of[2][kMaxChunk];  // staged row -> its row in src / src_sh (-1: none)
+  __shared__ int8_t sh_of[2][kMaxChunk];    // 1: the shared expert's row (src_sh)
+  __shared__ int fail;
+  __shared__ int issued[2];                 // parity + 1 of the last copies into each buffer, 0: none
+  const int lane = lane_id(), warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    fail = 0;
+    issued[0] = issued[1] = 0;
+    fence_mbar_init();
+  }
+  int64_t total = single_rows;
+  if (groups != nullptr && warp == 0) {
+    int64_t carry = 0;
+    for (int base = 0; base < num_groups; base += 32) {
+      const int g = base + lane;
+      const int64_t rows = g < num_groups ? max(groups[g].rows, 0) : 0;
+      int64_t incl = rows;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int64_t o = __shfl_up_sync(kFull, incl, off);
+        if (lane >= off) incl += o;
+      }
+      if (g < num_groups) start[g] = carry + incl - rows;
+      carry += __shfl_sync(kFull, incl, 31);
+    }
+    if (lane == 0) start[num_groups] = carry;
+  }
+  __syncthreads();
+  if (groups != nullptr) total = start[num_groups];
+  const int64_t nchunks = (total + chunk - 1) / chunk;
+  const uint32_t row_bytes = static_cast<uint32_t>(d) * 2;
+  uint32_t phase[2] = {0, 0};
+  int abort_flag = 0;
+  // warp 0: rows of chunk c into buffer b
+  auto issue = [&](int64_t c, int b) {
+    int n_valid = 0;
+    for (int r = lane; r < chunk; r += 32) {
+      const int64_t i = c * chunk + r;
+      int64_t row = -1;
+      int sh = 0;
+      if (i < total) {
+        if (groups == nullptr) {
+          row = i;
+        } else {
+          int lo = 0, hi = num_groups;  // start[lo] <= i < start[lo + 1]
+          while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (start[mid] <= i)
+              lo = mid;
+            else
+              hi = mid;
+          }
+          const GroupEntry g = groups[lo];
+          sh = g.expert == shared_slab && src_sh != nullptr;
+          row = (sh ? 0 : (use_out_rows ? g.out_row0 : g.a_row0)) + (i - start[lo]);
+        }
+        // rows outside the buffers (a corrupt table) are skipped; the GEMM reports the group
+        if (row < 0 || row >= (sh ? sh_rows : dst_rows)) row = -1;
+      }
+      row_of[b][r] = row;
+      sh_of[b][r] = static_cast<int8_t>(sh);
+      n_valid += row >= 0;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) n_valid += __shfl_xor_sync(kFull, n_valid, off);
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&full[b], static_cast<uint32_t>(n_valid) * row_bytes);
+      issued[b] = static_cast<int>(phase[b]) + 1;
+    }
+    __syncwarp();
+    for (int r = lane; r < chunk; r += 32) {
+      const int64_t row = row_of[b][r];
+      if (row >= 0)
+        bulk_load(stage + (static_cast<size_t>(b) * chunk + r) * row_bytes, (sh_of[b][r] ? src_sh : src) + row * d,
+                  row_bytes, &full[b]);
+    }
+  };
+  int b = 0;
+  int64_t c = blockIdx.x;
+  if (warp == 0 && c < nchunks) issue(c, 0);
+  for (; c < nchunks; c += gridDim.x) {
+    const int64_t cn = c + gridDim.x;
+    if (warp == 0 && cn < nchunks) issue(cn, b ^ 1);  // released by the barrier ending the previous chunk
+    if (!mbar_wait(&full[b], phase[b], &abort_flag)) atomicOr(&fail, 1);
+    __syncthreads();
+    if (fail) break;
+    if (threadIdx.x == 0) issued[b] = 0;
+    phase[b] ^= 1u;
+    for (int r = warp; r < chunk; r += kWarps) {
+      const int64_t row = row_of[b][r];
+      if (row < 0) continue;
+      const bool sh = sh_of[b][r];
+      const uint8_t* rs = stage + (static_cast<size_t>(b) * chunk + r) * row_bytes;
+      float m = 0.0f;
+      bool nan = false, nonfinite = false;
+      for (int col = lane * 8; col < d; col += 256) {
+        float f[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(rs + col * 2), f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          m = fmaxf(m, fabsf(f[j]));
+          nan |= isnan(f[j]);
+          nonfinite |= !isfinite(f[j]);
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+      nan = __any_sync(kFull, nan);
+      nonfinite = __any_sync(kFull, nonfinite);
+      float sc, mult;
+      row_scale(terms, m, nan, nonfinite, sc, mult);
+      uint8_t* out = (sh ? dst_sh : dst) + row * terms * d;
+      for (int col = lane * 8; col < d; col += 256)
+        code_piece(*reinterpret_cast<const uint4*>(rs + col * 2), out, d, col, terms, sc, mult);
+      if (lane == 0) (sh ? scale_sh : scale)[row] = sc;
+    }
+    __syncthreads();  // buffer b is free again
+    b ^= 1;
+  }
+  if (fail && threadIdx.x == 0) {
+    report(status, MOE_STATUS_TIMEOUT, MOE_CNT_TIMEOUT);
+    // copies still in flight must land before the CTA's shared memory goes away
+    int never = 0;
+    for (int i = 0; i < 2; ++i)
+      if (issued[i]) mbar_wait(&full[i], static_cast<uint32_t>(issued[i] - 1), &never);
+  }
+}
+
 int device_sms() {
   static int sms = 0;
   if (sms == 0) {
@@ -389,10 +559,32 @@ dim3 quantize_grid(int64_t rows, int d) {
 cudaError_t launch_rows(const GroupEntry* groups, int num_groups, int use_out_rows, int shared_slab,
                         int64_t single_rows, const void* src, uint8_t* dst, float* scale, int64_t dst_rows,
                         const void* src_sh, uint8_t* dst_sh, float* scale_sh, int64_t sh_rows, int d, int terms,
-                        int64_t max_rows, cudaStream_t stream) {
-  const dim3 grid = quantize_grid(max_rows, d);
+                        int64_t max_rows, StatusBlock* status, cudaStream_t stream) {
   const auto* s = static_cast<const __nv_bfloat16*>(src);
   const auto* ss = static_cast<const __nv_bfloat16*>(src_sh);
+  if (!cta_rows(max_rows, d) && d <= kStagedMaxCols) {
+    // staged chunks: a multiple of 8 rows (one per warp), about 24 KB per chunk buffer (two per CTA)
+    const int chunk = std::min(kMaxChunk, std::max(kWarps, (12288 / d) / kWarps * kWarps));
+    const size_t smem = static_cast<size_t>(2) * chunk * d * 2;
+    static bool attr = false;
+    if (!attr) {
+      cudaError_t e = cudaFuncSetAttribute(quantize_rows_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           2 * kMaxChunk * kStagedMaxCols);
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    const int64_t chunks = (max_rows + chunk - 1) / chunk;
+    // as many CTAs as are resident at once (shared memory, 8 CTAs of 256 threads at most)
+    const int per_sm = static_cast<int>(std::max<size_t>(1, std::min<size_t>(8, 232448 / (smem + 6144))));
+    const int64_t cap = static_cast<int64_t>(per_sm) * device_sms();
+    const dim3 grid(static_cast<unsigned>(chunks < cap ? chunks : cap));
+    quantize_rows_staged_kernel<<<grid, kWarps * 32, smem, stream>>>(groups, num_groups, use_out_rows, shared_slab,
+                                                                      single_rows, s, dst, scale, dst_rows, ss,
+                                                                      dst_sh, scale_sh, sh_rows, d, terms, chunk,
+                                                                      status);
+    return cudaGetLastError();
+  }
+  const dim3 grid = quantize_grid(max_rows, d);
   if (cta_rows(max_rows, d))
     quantize_rows_kernel<kWarps * 32><<<grid, kWarps * 32, 0, stream>>>(groups, num_groups, use_out_rows,
                                                                          shared_slab, single_rows, s, dst, scale,
@@ -412,7 +604,7 @@ cudaError_t launch_quantize_rows(const void* src, uint8_t* dst, float* scale, in
   if (rows <= 0) return cudaSuccess;
   if (d <= 0 || d % 8 != 0 || (terms != 1 && terms != 2)) return cudaErrorInvalidValue;
   return launch_rows(nullptr, 0, 0, -1, rows, src, dst, scale, rows, nullptr, nullptr, nullptr, 0, d, terms, rows,
-                     stream);
+                     nullptr, stream);
 }
 
 cudaError_t launch_gather_quantize(int S, int d, int K, const int32_t* row_of_slot, const void* x, uint8_t* q_perm,
@@ -433,12 +625,12 @@ cudaError_t launch_quantize_group_rows(const GroupEntry* groups, int num_groups,
                                        const void* src, uint8_t* dst, float* scale, int64_t dst_rows,
                                        const void* src_shared, uint8_t* dst_shared, float* scale_shared,
                                        int64_t shared_rows, int d, int64_t max_total_rows, int terms,
-                                       cudaStream_t stream) {
+                                       StatusBlock* status, cudaStream_t stream) {
   if (num_groups <= 0 || max_total_rows <= 0) return cudaSuccess;
   if (num_groups > kQuantMaxGroups || d <= 0 || d % 8 != 0 || (terms != 1 && terms != 2))
     return cudaErrorInvalidValue;
   return launch_rows(groups, num_groups, use_out_rows, shared_slab, 0, src, dst, scale, dst_rows, src_shared,
-                     dst_shared, scale_shared, shared_rows, d, terms, max_total_rows, stream);
+                     dst_shared, scale_shared, shared_rows, d, terms, max_total_rows, status, stream);
 }
 
 }  // namespace moe

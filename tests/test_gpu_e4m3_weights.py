@@ -37,12 +37,11 @@ def _all_codes(shape, seed):
     return codes.to(torch.uint8)
 
 
-def _edge_rows(d):
+def _edge_rows(d, n=40):
     """bf16 rows with every kind of value: spreads from 2**-30 to 1 of the row
     maximum, bf16 subnormals, huge and tiny maxima, maxima of exactly
     448 * 2**j, a zero row, rows holding an infinity or a NaN."""
-    rng = np.random.default_rng(77)
-    n = 40
+    rng = np.random.default_rng(77 + n)
     amax = np.exp2(rng.integers(-30, 30, size=(n, 1))).astype(np.float64) * rng.uniform(1, 2, size=(n, 1))
     x = amax * np.exp2(-rng.uniform(0, 30, size=(n, d))) * rng.choice([-1.0, 1.0], size=(n, d))
     x[0] = 0.0
@@ -56,9 +55,11 @@ def _edge_rows(d):
     return t
 
 
-@pytest.mark.parametrize("d", [16, 272, 4096])
-def test_split_rows_bit_exact(d):
-    x = _edge_rows(d)
+@pytest.mark.parametrize("n,d", [(40, 16), (40, 272), (40, 4096), (1500, 272), (700, 2048)])
+def test_split_rows_bit_exact(n, d):
+    """Few rows (a CTA per row) and many rows (rows staged in shared memory by
+    bulk copies)."""
+    x = _edge_rows(d, n)
     xd = x.cuda()
     q = torch.empty((x.shape[0], 2 * d), dtype=torch.uint8, device="cuda")
     s = torch.empty((x.shape[0],), dtype=torch.float32, device="cuda")
