@@ -47,6 +47,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "pdl.cuh"
 
 namespace moe {
 
@@ -261,6 +262,8 @@ __global__ void __launch_bounds__(kWarps * 32)
   const int per_cta = kWarps * 32 / T;
   const int t = blockIdx.x * per_cta + static_cast<int>(threadIdx.x) / T;
   const int tid = static_cast<int>(threadIdx.x) % T;
+  pdl_wait();
+  pdl_trigger();
   if (t >= S) return;  // T = 256: the whole CTA leaves together
   __shared__ int rows[kWarps][32];
   int* my_rows = rows[threadIdx.x >> 5];
@@ -322,6 +325,8 @@ __global__ void __launch_bounds__(kWarps * 32)
                          int terms) {
   __shared__ int64_t start[kQuantMaxGroups + 1];
   const int lane = lane_id(), warp = threadIdx.x >> 5;
+  pdl_wait();
+  pdl_trigger();
   int64_t total = single_rows;
   if (groups != nullptr) {
     if (warp == 0) {
@@ -414,6 +419,8 @@ __global__ void __launch_bounds__(kWarps * 32)
     issued[0] = issued[1] = 0;
     fence_mbar_init();
   }
+  pdl_wait();
+  pdl_trigger();
   int64_t total = single_rows;
   if (groups != nullptr && warp == 0) {
     int64_t carry = 0;
@@ -566,35 +573,33 @@ cudaError_t launch_rows(const GroupEntry* groups, int num_groups, int use_out_ro
     // staged chunks: a multiple of 8 rows (one per warp), about 24 KB per chunk buffer (two per CTA)
     const int chunk = std::min(kMaxChunk, std::max(kWarps, (12288 / d) / kWarps * kWarps));
     const size_t smem = static_cast<size_t>(2) * chunk * d * 2;
-    static bool attr = false;
-    if (!attr) {
+    static size_t attr_bytes = 0;  // the largest dynamic shared memory enabled so far
+    if (smem > attr_bytes) {
       cudaError_t e = cudaFuncSetAttribute(quantize_rows_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           2 * kMaxChunk * kStagedMaxCols);
+                                           static_cast<int>(smem));
       if (e != cudaSuccess) return e;
-      attr = true;
+      attr_bytes = smem;
     }
     const int64_t chunks = (max_rows + chunk - 1) / chunk;
     // as many CTAs as are resident at once (shared memory, 8 CTAs of 256 threads at most)
     const int per_sm = static_cast<int>(std::max<size_t>(1, std::min<size_t>(8, 232448 / (smem + 6144))));
     const int64_t cap = static_cast<int64_t>(per_sm) * device_sms();
     const dim3 grid(static_cast<unsigned>(chunks < cap ? chunks : cap));
-    quantize_rows_staged_kernel<<<grid, kWarps * 32, smem, stream>>>(groups, num_groups, use_out_rows, shared_slab,
-                                                                      single_rows, s, dst, scale, dst_rows, ss,
-                                                                      dst_sh, scale_sh, sh_rows, d, terms, chunk,
-                                                                      status);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(quantize_rows_staged_kernel, grid, dim3(kWarps * 32), smem, stream, groups, num_groups,
+                               use_out_rows, shared_slab, single_rows, s, dst, scale, dst_rows, ss, dst_sh, scale_sh,
+                               sh_rows, d, terms, chunk, status);
+    return e != cudaSuccess ? e : cudaGetLastError();
   }
   const dim3 grid = quantize_grid(max_rows, d);
+  cudaError_t e;
   if (cta_rows(max_rows, d))
-    quantize_rows_kernel<kWarps * 32><<<grid, kWarps * 32, 0, stream>>>(groups, num_groups, use_out_rows,
-                                                                         shared_slab, single_rows, s, dst, scale,
-                                                                         dst_rows, ss, dst_sh, scale_sh, sh_rows, d,
-                                                                         terms);
+    e = launch_pdl(quantize_rows_kernel<kWarps * 32>, grid, dim3(kWarps * 32), 0, stream, groups, num_groups,
+                   use_out_rows, shared_slab, single_rows, s, dst, scale, dst_rows, ss, dst_sh, scale_sh, sh_rows, d,
+                   terms);
   else
-    quantize_rows_kernel<32><<<grid, kWarps * 32, 0, stream>>>(groups, num_groups, use_out_rows, shared_slab,
-                                                               single_rows, s, dst, scale, dst_rows, ss, dst_sh,
-                                                               scale_sh, sh_rows, d, terms);
-  return cudaGetLastError();
+    e = launch_pdl(quantize_rows_kernel<32>, grid, dim3(kWarps * 32), 0, stream, groups, num_groups, use_out_rows,
+                   shared_slab, single_rows, s, dst, scale, dst_rows, ss, dst_sh, scale_sh, sh_rows, d, terms);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace
@@ -612,13 +617,14 @@ cudaError_t launch_gather_quantize(int S, int d, int K, const int32_t* row_of_sl
   if (S <= 0) return cudaSuccess;
   if (d <= 0 || d % 8 != 0 || K < 1 || K > 32 || (terms != 1 && terms != 2)) return cudaErrorInvalidValue;
   const auto* xs = static_cast<const __nv_bfloat16*>(x);
+  cudaError_t e;
   if (cta_rows(S, d))
-    gather_quantize_kernel<kWarps * 32><<<S, kWarps * 32, 0, stream>>>(S, d, K, terms, row_of_slot, xs, q_perm,
-                                                                        s_perm, q_x, s_x);
+    e = launch_pdl(gather_quantize_kernel<kWarps * 32>, dim3(S), dim3(kWarps * 32), 0, stream, S, d, K, terms,
+                   row_of_slot, xs, q_perm, s_perm, q_x, s_x);
   else
-    gather_quantize_kernel<32><<<(S + kWarps - 1) / kWarps, kWarps * 32, 0, stream>>>(S, d, K, terms, row_of_slot,
-                                                                                      xs, q_perm, s_perm, q_x, s_x);
-  return cudaGetLastError();
+    e = launch_pdl(gather_quantize_kernel<32>, dim3((S + kWarps - 1) / kWarps), dim3(kWarps * 32), 0, stream, S, d, K,
+                   terms, row_of_slot, xs, q_perm, s_perm, q_x, s_x);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_quantize_group_rows(const GroupEntry* groups, int num_groups, int use_out_rows, int shared_slab,
