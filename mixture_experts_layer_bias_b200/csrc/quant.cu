@@ -70,12 +70,27 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
   return q;
 }
 
-// Value of a finite E4M3 code, exactly: its exponent and mantissa bits placed
-// at the bottom of a float's exponent field and the top of its mantissa give
-// the value times 2^-120 (an E4M3 subnormal becomes a float subnormal, with
-// the same mantissa), and one multiply by 2^120 restores it.
-__device__ __forceinline__ float e4m3_value(uint32_t c) {
-  return __uint_as_float(((c & 0x7Fu) << 20) | ((c & 0x80u) << 24)) * 0x1p120f;
+// Magnitude of the finite E4M3 code in the low byte of c, exactly: its
+// exponent and mantissa bits placed at the bottom of a float's exponent field
+// and the top of its mantissa give the value times 2^-120 (an E4M3 subnormal
+// becomes a float subnormal, with the same mantissa), and one multiply by
+// 2^120 restores it.
+__device__ __forceinline__ float e4m3_magnitude(uint32_t c) {
+  return __uint_as_float((c & 0x7Fu) << 20) * 0x1p120f;
+}
+
+// Largest |x| of bf16 values kept as bit patterns: the magnitude bits of a
+// bf16 (sign cleared) order like the values, with +inf = 0x7F80 above every
+// finite value and NaNs above it, so two 16-bit unsigned maxima per 32-bit
+// word track the row's maximum and whether it holds an infinity or a NaN.
+__device__ __forceinline__ uint32_t absmax_bits2(uint32_t acc, uint32_t w) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(acc), "r"(w & 0x7FFF7FFFu));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t absmax_bits8(uint32_t acc, const uint4& w) {
+  return absmax_bits2(absmax_bits2(absmax_bits2(absmax_bits2(acc, w.x), w.y), w.z), w.w);
 }
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& w, float* f) {
@@ -103,53 +118,28 @@ struct RowPieces {
 template <int T>
 __device__ __forceinline__ void row_load_amax(const __nv_bfloat16* __restrict__ src, int d, int tid,
                                               RowPieces<T>& rp, float& amax, bool& nan, bool& nonfinite) {
-  float m = 0.0f;
-  bool n = false, nf = false;
+  uint32_t acc = 0;
 #pragma unroll
   for (int i = 0; i < kVec; ++i) {
     const int c = (tid + i * T) * 8;
     rp.v[i] = c < d ? ldg16(src + c) : make_uint4(0, 0, 0, 0);
   }
-  auto acc = [&](const uint4& w) {
-    float f[8];
-    bf16x8_to_f32(w, f);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      m = fmaxf(m, fabsf(f[j]));
-      n |= isnan(f[j]);
-      nf |= !isfinite(f[j]);
-    }
-  };
-#pragma unroll
-  for (int i = 0; i < kVec; ++i) acc(rp.v[i]);  // zero pieces past the row change nothing
-  for (int c = (tid + kVec * T) * 8; c < d; c += T * 8) acc(ldg16(src + c));
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
-  n = __any_sync(kFull, n);
-  nf = __any_sync(kFull, nf);
+  for (int i = 0; i < kVec; ++i) acc = absmax_bits8(acc, rp.v[i]);  // zero pieces past the row change nothing
+  for (int c = (tid + kVec * T) * 8; c < d; c += T * 8) acc = absmax_bits8(acc, ldg16(src + c));
+  uint32_t bits = __reduce_max_sync(kFull, max(acc & 0xFFFFu, acc >> 16));
   if (T > 32) {
-    __shared__ float wm[kWarps];
-    __shared__ int wf[kWarps];
-    const int w = tid >> 5;
-    if ((tid & 31) == 0) {
-      wm[w] = m;
-      wf[w] = (n ? 1 : 0) | (nf ? 2 : 0);
-    }
+    __shared__ uint32_t wm[kWarps];
+    if ((tid & 31) == 0) wm[tid >> 5] = bits;
     __syncthreads();
-    m = wm[0];
-    int fl = wf[0];
+    bits = wm[0];
 #pragma unroll
-    for (int i = 1; i < T / 32; ++i) {
-      m = fmaxf(m, wm[i]);
-      fl |= wf[i];
-    }
-    n = fl & 1;
-    nf = fl & 2;
-    __syncthreads();  // the next row's maxima reuse wm / wf
+    for (int i = 1; i < T / 32; ++i) bits = max(bits, wm[i]);
+    __syncthreads();  // the next row's maxima reuse wm
   }
-  amax = m;
-  nan = n;
-  nonfinite = nf;
+  amax = __uint_as_float(bits << 16);
+  nan = bits > 0x7F80u;
+  nonfinite = bits >= 0x7F80u;
 }
 
 // W8A8 scale: amax / 448 (1 for an all-zero row or a row holding a NaN).
@@ -199,7 +189,8 @@ __device__ __forceinline__ void encode8_two_term(const uint4& w, float m, uint2&
   for (int j = 0; j < 4; ++j) {
     const float v0 = f[2 * j] * m, v1 = f[2 * j + 1] * m;  // finite, |v| <= 448
     a[j] = e4m3x2_finite(v0, v1);
-    b[j] = e4m3x2_finite(v0 - e4m3_value(a[j] & 0xFFu), v1 - e4m3_value(a[j] >> 8));
+    // c1 carries v's sign (or is zero), so v - c1 = v - copysign(|c1|, v)
+    b[j] = e4m3x2_finite(v0 - copysignf(e4m3_magnitude(a[j]), v0), v1 - copysignf(e4m3_magnitude(a[j] >> 8), v1));
   }
   t1 = make_uint2(a[0] | (a[1] << 16), a[2] | (a[3] << 16));
   t2 = make_uint2(b[0] | (b[1] << 16), b[2] | (b[3] << 16));
@@ -504,24 +495,12 @@ __global__ void __launch_bounds__(kWarps * 32)
       if (row < 0) continue;
       const bool sh = sh_of[b][r];
       const uint8_t* rs = stage + (static_cast<size_t>(b) * chunk + r) * row_bytes;
-      float m = 0.0f;
-      bool nan = false, nonfinite = false;
-      for (int col = lane * 8; col < d; col += 256) {
-        float f[8];
-        bf16x8_to_f32(*reinterpret_cast<const uint4*>(rs + col * 2), f);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          m = fmaxf(m, fabsf(f[j]));
-          nan |= isnan(f[j]);
-          nonfinite |= !isfinite(f[j]);
-        }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
-      nan = __any_sync(kFull, nan);
-      nonfinite = __any_sync(kFull, nonfinite);
+      uint32_t acc = 0;
+      for (int col = lane * 8; col < d; col += 256)
+        acc = absmax_bits8(acc, *reinterpret_cast<const uint4*>(rs + col * 2));
+      const uint32_t bits = __reduce_max_sync(kFull, max(acc & 0xFFFFu, acc >> 16));
       float sc, mult;
-      row_scale(terms, m, nan, nonfinite, sc, mult);
+      row_scale(terms, __uint_as_float(bits << 16), bits > 0x7F80u, bits >= 0x7F80u, sc, mult);
       uint8_t* out = (sh ? dst_sh : dst) + row * terms * d;
       for (int col = lane * 8; col < d; col += 256)
         code_piece(*reinterpret_cast<const uint4*>(rs + col * 2), out, d, col, terms, sc, mult);
