@@ -642,9 +642,10 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=sorted(syn.CONFIGS) + sorted(syn.VARIANTS)
                     + ["profile_small", "profile_small_w8a8", "profile_small_dsv3"],
-                    help="profile_small*: smaller cases of the same kernels (0.4-1.5 GB of weights) for ncu "
-                         "captures: Mixtral-shaped S=2048, h=4096 (bf16 or W8A8); DeepSeek-shaped S=512 with "
-                         "16 routed experts (~256 rows each) + the shared one")
+                    help="profile_small*: smaller cases of the same kernels (0.4-2.9 GB of weights) for ncu "
+                         "captures: Mixtral-shaped S=2048, h=4096 (bf16 or W8A8); DeepSeek-shaped S=1024 with "
+                         "32 routed experts in 4 groups (top-2 groups, biased selection: uneven loads around "
+                         "256 rows) + the shared one")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))
@@ -667,7 +668,7 @@ def main():
     elif args.workload == "profile_small_w8a8":
         cfg = syn.scaled(syn.VARIANTS["mixtral_prefill_w8a8"], S=2048, h=4096)
     elif args.workload == "profile_small_dsv3":
-        cfg = syn.scaled(syn.CONFIGS["dsv3_grouped"], S=512, E=16, num_groups=1, topk_groups=1)
+        cfg = syn.scaled(syn.CONFIGS["dsv3_grouped"], S=1024, E=32, num_groups=4, topk_groups=2)
     else:
         cfg = get_cfg(args.workload)
     S = cfg.S
