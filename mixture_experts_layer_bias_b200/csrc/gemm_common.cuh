@@ -106,26 +106,34 @@ __device__ __forceinline__ float splitk_out(const TcParams& p, int64_t sbase, in
   return gv;
 }
 
-// Sum of the ks slices of the float4 at `src` (slice stride `slice`), in split
-// order; the loads are issued four at a time before their sums so that they
+// Sums of the ks slices of the float4 at `src` and, with TWO, of the float4
+// at `src + off` (slice stride `slice`), each in split order; up to eight
+// slices of each are loaded before their sums, so that all loads of a batch
 // are in flight together.  Read at L2 (ld.global.cg): other CTAs wrote them.
-__device__ __forceinline__ float4 splitk_sum4(const float* src, int64_t slice, int ks) {
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  int s = 0;
-  for (; s + 4 <= ks; s += 4) {
-    float4 a[4];
+template <bool TWO>
+__device__ __forceinline__ void splitk_sums4(const float* src, int64_t off, int64_t slice, int ks, float4& g,
+                                             float4& u) {
+  g = make_float4(0.f, 0.f, 0.f, 0.f);
+  u = g;
+  for (int s = 0; s < ks; s += 8) {
+    float4 a[8], b[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) a[i] = __ldcg(reinterpret_cast<const float4*>(src + (s + i) * slice));
+    for (int i = 0; i < 8; ++i) {
+      if (s + i < ks) {
+        a[i] = __ldcg(reinterpret_cast<const float4*>(src + (s + i) * slice));
+        if (TWO) b[i] = __ldcg(reinterpret_cast<const float4*>(src + off + (s + i) * slice));
+      }
+    }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      acc.x += a[i].x; acc.y += a[i].y; acc.z += a[i].z; acc.w += a[i].w;
+    for (int i = 0; i < 8; ++i) {
+      if (s + i < ks) {
+        g.x += a[i].x; g.y += a[i].y; g.z += a[i].z; g.w += a[i].w;
+        if (TWO) {
+          u.x += b[i].x; u.y += b[i].y; u.z += b[i].z; u.w += b[i].w;
+        }
+      }
     }
   }
-  for (; s < ks; ++s) {
-    const float4 a = __ldcg(reinterpret_cast<const float4*>(src + s * slice));
-    acc.x += a.x; acc.y += a.y; acc.z += a.z; acc.w += a.w;
-  }
-  return acc;
 }
 
 // Split-K finalize: for every valid row of every group, sum the partial slices
@@ -150,9 +158,8 @@ __global__ void __launch_bounds__(256) splitk_finalize_kernel(TcParams p) {
   const int64_t slice = p.out_rows * static_cast<int64_t>(p.pcols);
   const float rs = a_row_scale(p, grp, r);
   const float* src = p.partial + orow * p.pcols + n;
-  const float4 g = splitk_sum4(src, slice, ks);
-  float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (EPI == EPI_SWIGLU) u = splitk_sum4(src + N, slice, ks);
+  float4 g, u;
+  splitk_sums4<EPI == EPI_SWIGLU>(src, N, slice, ks, g, u);
   float o[4];
   o[0] = splitk_out<EPI>(p, sbase, n, 0, g.x, u.x, rs);
   o[1] = splitk_out<EPI>(p, sbase, n, 1, g.y, u.y, rs);
