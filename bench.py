@@ -132,9 +132,10 @@ def kernels_per_step(cfg, S=None):
     """Launches of this library's kernels in one moe_layer_forward call."""
     S = cfg.S if S is None else S
     small = S * cfg.K <= 4096               # one-CTA permutation for small batches
-    n = 1 if (cfg.E <= 32) else 2          # route (logits in the routing kernel) or logits GEMM + top-k
-    n += 1 if small else 4                 # permutation (+ group table): one kernel, or count, scan, scatter, groups
     elem = 4 if cfg.act_dtype == syn.F32 else 2
+    logits_first = cfg.E > 32 or (S > 512 and cfg.E * cfg.d * elem > 64 * 1024)
+    n = 2 if logits_first else 1           # logits GEMM + top-k, or the routing kernel computing the logits
+    n += 1 if small else 4                 # permutation (+ group table): one kernel, or count, scan, scatter, groups
     coded = coded_a_rows(cfg)
     if coded or not (small and S * cfg.K * cfg.d * elem <= 256 * 1024):
         n += 1                             # row gather (writing E4M3 codes); tiny bf16 batches: inside the permutation

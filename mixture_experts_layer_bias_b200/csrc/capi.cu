@@ -75,7 +75,7 @@ Layout make_layout(const moe_desc& d) {
     return at;
   };
   L.status = take(kAlign);
-  L.logits = take(E > 32 ? static_cast<size_t>(S * E) * 4 : 0);
+  L.logits = take(route_logits_first(S, E, dm, static_cast<int>(act_bytes(d))) ? static_cast<size_t>(S * E) * 4 : 0);
   L.chunk_hist = take(static_cast<size_t>(nch * E) * 4);
   L.groups = take(static_cast<size_t>(2 * E + 1) * sizeof(GroupEntry));
   L.counts = take(static_cast<size_t>(E) * 4);

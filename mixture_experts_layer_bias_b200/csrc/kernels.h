@@ -12,6 +12,16 @@ namespace moe {
 struct StatusBlock;
 
 // --- routing ---------------------------------------------------------------
+// Router logits: E <= 32 are computed inside the routing kernels (a CTA per
+// token for S <= 512, else warps streaming token rows against a copy of W_r in
+// shared memory of at most kRouteWSmemBytes); otherwise (E > 32, or W_r too
+// large for that copy when S > 512) one logits GEMM into the workspace first,
+// then the selection.
+constexpr int kRouteWSmemBytes = 64 << 10;
+inline bool route_logits_first(int64_t S, int64_t E, int64_t d, int elem_bytes) {
+  return E > 32 || (S > 512 && E * d * elem_bytes > kRouteWSmemBytes);
+}
+
 struct RouteArgs {
   int S, d, E, K;
   int score_fn, renormalize, num_groups, topk_groups;
@@ -20,7 +30,7 @@ struct RouteArgs {
   const void* x;            // [S][d] (unused when logits given)
   const void* w_router;     // [E][d]
   const float* logits;      // [S][E] fp32 or nullptr (then computed)
-  float* logits_scratch;    // [S][E] fp32 scratch for E > 32
+  float* logits_scratch;    // [S][E] fp32 scratch (route_logits_first)
   const float* router_bias; // [E] or nullptr
   const float* sel_bias;    // [E] or nullptr
   int32_t* topk_idx;        // [S][K]

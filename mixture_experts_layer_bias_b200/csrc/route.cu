@@ -35,27 +35,26 @@ constexpr int kRouteWarps = 8;
 // lane (a token row's loads in two rounds at d = 4096 in bf16), so the
 // token rows -- the bytes that must come from HBM -- stream with many loads in
 // flight and no block-wide barrier.  The router weights sit in shared memory
-// when they fit in 64 KB (else they are read through L1).  The TPW x EMAX
+// (at most 64 KB: larger router matrices go through the logits GEMM, see
+// route_logits_first).  The TPW x EMAX
 // partial dot products of a lane are summed over the warp by a reduce-scatter
 // butterfly (lane i ends with value i: token i / EMAX, expert i % EMAX), then
 // the warp selects its tokens.  The grid is persistent: warps loop over token
 // sets.
 constexpr int kRouteRowWarps = 8;
-constexpr int kRouteWSmemBytes = 64 << 10;
 
-template <typename T, int EMAX, bool WSMEM>
+template <typename T, int EMAX>
 __global__ void __launch_bounds__(kRouteRowWarps * 32, 2)
     route_rows_kernel(int S, int d, const T* __restrict__ x, const T* __restrict__ w_router,
                       const float* __restrict__ router_bias, SelectParams p) {
   constexpr int TPW = EMAX >= 16 ? 1 : 16 / EMAX;
   constexpr int NV = TPW * EMAX;  // 16 or 32 partial sums per lane
   constexpr int kRouteBatch = EMAX >= 16 ? 4 : 8;
-  constexpr int kExpertUnroll = (!WSMEM && EMAX >= 16) ? 8 : EMAX;  // W from global: fewer loads in flight
   constexpr int V = Vec16<T>::N;
   extern __shared__ uint4 wsm[];
   const int warp = threadIdx.x >> 5, lane = lane_id();
   const int nvec = d / V;
-  if (WSMEM) {
+  {
     const int n16 = p.E * nvec;
     for (int i = threadIdx.x; i < n16; i += blockDim.x) wsm[i] = ldg16(w_router + static_cast<int64_t>(i) * V);
     __syncthreads();
@@ -84,11 +83,11 @@ __global__ void __launch_bounds__(kRouteRowWarps * 32, 2)
         float xf[TPW][V];
 #pragma unroll
         for (int tt = 0; tt < TPW; ++tt) unpack16<T>(xv[tt][b], xf[tt]);
-#pragma unroll kExpertUnroll
+#pragma unroll
         for (int e = 0; e < EMAX; ++e) {
           if (e < p.E) {
             float wf[V];
-            unpack16<T>(WSMEM ? wsm[e * nvec + v] : ldg16(w_router + (static_cast<int64_t>(e) * nvec + v) * V), wf);
+            unpack16<T>(wsm[e * nvec + v], wf);
 #pragma unroll
             for (int tt = 0; tt < TPW; ++tt)
 #pragma unroll
@@ -276,7 +275,8 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
   SelectParams sp{a.E,        a.K,      a.score_fn, a.renormalize, a.num_groups,   a.topk_groups, a.tau,
                   a.sel_bias, a.topk_idx, a.topk_w, a.status,      a.cand_key_out, a.score_out};
   const float* logits = a.logits;
-  if (logits == nullptr && a.E <= 32) {
+  const int elem = a.act_dtype == MOE_F32 ? 4 : 2;
+  if (logits == nullptr && !route_logits_first(a.S, a.E, a.d, elem)) {
     // decode-sized batches: a CTA per token; otherwise warps streaming token rows
     const bool per_cta = a.S <= 512;
     cudaError_t err = cudaSuccess;
@@ -291,17 +291,12 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
       const int want = (sets + kRouteRowWarps - 1) / kRouteRowWarps;                                           \
       const int cap = (a.num_sms > 0 ? a.num_sms : 148) * 2;                                                   \
       const int grid = want < cap ? want : cap;                                                                \
-      const size_t wbytes = static_cast<size_t>(a.E) * a.d * sizeof(T);                                        \
-      if (wbytes <= static_cast<size_t>(kRouteWSmemBytes)) {                                                   \
-        err = cudaFuncSetAttribute(route_rows_kernel<T, EM, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                                   kRouteWSmemBytes);                                                          \
-        if (err == cudaSuccess)                                                                                \
-          route_rows_kernel<T, EM, true><<<grid, kRouteRowWarps * 32, wbytes, stream>>>(                        \
-              a.S, a.d, static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);     \
-      } else {                                                                                                 \
-        route_rows_kernel<T, EM, false><<<grid, kRouteRowWarps * 32, 0, stream>>>(                              \
+      const size_t wbytes = static_cast<size_t>(a.E) * a.d * sizeof(T); /* <= kRouteWSmemBytes here */       \
+      err = cudaFuncSetAttribute(route_rows_kernel<T, EM>, cudaFuncAttributeMaxDynamicSharedMemorySize,         \
+                                 kRouteWSmemBytes);                                                            \
+      if (err == cudaSuccess)                                                                                  \
+        route_rows_kernel<T, EM><<<grid, kRouteRowWarps * 32, wbytes, stream>>>(                                \
             a.S, a.d, static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);       \
-      }                                                                                                        \
     }                                                                                                          \
   } while (0)
     if (a.act_dtype == MOE_BF16) {
