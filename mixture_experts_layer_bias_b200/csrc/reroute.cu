@@ -427,69 +427,6 @@ __device__ __forceinline__ void repick_token(int t, int64_t first, int E, int K,
   }
 }
 
-// repick_token with four threads of a warp (`quad_lane` 0..3, lanes `qmask`)
-// per token, for E <= 64 with E a multiple of 4: lane j holds the keys of
-// experts 16j .. 16j+15 in registers, each slot's best candidate is the best
-// of the four lanes' local bests (highest key, ties to the lower index, the
-// same choice as the serial scan), and lane 0 commits it.  Four tokens per
-// warp are re-picked side by side instead of one per thread, so an epoch's
-// re-picks take a quarter of the key registers per thread and a short
-// reduction per slot.
-template <bool SM>
-__device__ __forceinline__ void repick_token_quad(int t, int64_t first, int E, int K, bool vec, int seg,
-                                                  const int32_t* __restrict__ topk_idx,
-                                                  const float* __restrict__ cand_key, const Picks<SM>& pick,
-                                                  CommitSmem& sm, int quad_lane, unsigned qmask) {
-  const int64_t s0 = static_cast<int64_t>(t) * K;
-  const int k0 = static_cast<int>((first > s0 ? first : s0) - s0);
-  const float kNegInf = __int_as_float(0xff800000);
-  const int e0 = 16 * quad_lane;
-  const float4* row4 = reinterpret_cast<const float4*>(cand_key + static_cast<int64_t>(t) * E + e0);
-  float4 kv[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    kv[j] = (e0 + 4 * j < E) ? __ldg(row4 + j) : make_float4(kNegInf, kNegInf, kNegInf, kNegInf);
-  uint32_t held[kMaskWords];
-  held_of(topk_idx + s0, K, E, vec, held);
-  for (int k = 0; k < K; ++k) {
-    int p = pick.get(s0 + k);
-    if (p == kKept) continue;
-    if (k >= k0 && p >= 0 && (bit_of(sm.full, p) || has_bit(held, p))) {
-      // this lane's 16 experts that are available and not held
-      const uint64_t av = static_cast<uint64_t>(sm.avail[0]) | (E > 32 ? static_cast<uint64_t>(sm.avail[1]) << 32 : 0);
-      const uint64_t ok = (av & ~(static_cast<uint64_t>(held[0]) | (static_cast<uint64_t>(held[1]) << 32))) >> e0;
-      float bv = kNegInf;
-      int be = kNone;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float v4[4] = {kv[j].x, kv[j].y, kv[j].z, kv[j].w};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (!(v4[c] > bv) || !((ok >> (4 * j + c)) & 1u)) continue;
-          bv = v4[c];  // strictly greater in ascending e: a tie keeps the lower index
-          be = e0 + 4 * j + c;
-        }
-      }
-#pragma unroll
-      for (int off = 1; off < 4; off <<= 1) {
-        const float ov = __shfl_xor_sync(qmask, bv, off);
-        const int oe = __shfl_xor_sync(qmask, be, off);
-        if (oe != kNone && (be == kNone || ov > bv || (ov == bv && oe < be))) {
-          bv = ov;
-          be = oe;
-        }
-      }
-      if (quad_lane == 0) {
-        atomicSub(&sm.cnt[seg][p], 1);
-        if (be >= 0) atomicAdd(&sm.cnt[seg][be], 1);
-        pick.set(s0 + k, be);
-      }
-      p = be;
-    }
-    if (p >= 0) set_bit(held, p);
-  }
-}
-
 template <bool SM>
 __global__ void __launch_bounds__(kThreads, 1)
     reroute_commit_kernel(int S, int E, int K, int C, const int32_t* __restrict__ topk_idx,
@@ -714,19 +651,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
     const int nl = sm.nlist;
-    if (E <= 64 && E % 4 == 0) {
-      const int ql = tid & 3;
-      const unsigned qmask = 0xFu << (tid & 28);
-      for (int i = tid >> 2; i < nl; i += kThreads / 4) {
-        const int t = list[i];
-        repick_token_quad<SM>(t, P, E, K, vec, seg_of(static_cast<int64_t>(t) * K), topk_idx, cand_key, pick, sm,
-                              ql, qmask);
-      }
-    } else {
-      for (int i = tid; i < nl; i += kThreads) {
-        const int t = list[i];
-        repick_token<SM>(t, P, E, K, vec, seg_of(static_cast<int64_t>(t) * K), topk_idx, cand_key, pick, sm);
-      }
+    for (int i = tid; i < nl; i += kThreads) {
+      const int t = list[i];
+      repick_token<SM>(t, P, E, K, vec, seg_of(static_cast<int64_t>(t) * K), topk_idx, cand_key, pick, sm);
     }
     __syncthreads();
   }
