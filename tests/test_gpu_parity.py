@@ -119,14 +119,19 @@ def test_route_worked_example():
     np.testing.assert_allclose(gw[0], [0.55, 0.30], rtol=1e-6)
 
 
-@pytest.mark.parametrize("name,S", [("tiny_f32", 64), ("mixtral_prefill", 512), ("fp8_skew_capacity", 1024),
-                                    ("dsv3_grouped", 256)])
-def test_route_computed_logits_within_margin(name, S):
-    """The router computes its own logits (fused kernel for E <= 32, logits
-    GEMM otherwise); indices must agree with the oracle wherever the
-    selection margin is >= 1e-4 (excluded tokens are counted), and the gates
-    within the fp32 tolerance."""
-    cfg = syn.scaled(syn.CONFIGS[name], S=S)
+@pytest.mark.parametrize("name,S,over", [("tiny_f32", 64, {}), ("mixtral_prefill", 512, {}),
+                                         ("mixtral_prefill", 1500, {}), ("fp8_skew_capacity", 1024, {}),
+                                         ("dsv3_grouped", 256, {}),
+                                         ("dsv3_grouped", 1024, dict(E=32, num_groups=4, topk_groups=2))])
+def test_route_computed_logits_within_margin(name, S, over):
+    """The router computes its own logits: a CTA per token (S <= 512), warps
+    streaming token rows against W_r in shared memory (S > 512, E <= 32, W_r
+    of at most 64 KB: the Mixtral-shaped case at S = 1500), or the logits GEMM
+    then the selection (E > 32, or a larger W_r: 32 experts x 7168 here);
+    indices must agree with the oracle wherever the selection margin is
+    >= 1e-4 (excluded tokens are counted), and the gates within the fp32
+    tolerance."""
+    cfg = syn.scaled(syn.CONFIGS[name], S=S, **over)
     # routing only reads x and the router; small experts keep the draw cheap
     inp = syn.make_inputs(syn.scaled(cfg, h=8), "cuda", seed=1)
     desc = ops.make_desc(**syn.desc_dict(cfg, S))
