@@ -276,6 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int A_OFF = PACK ? B_TILE : 0;
   const int A2_OFF = PACK ? B_TILE + 64 * BK_BYTES : A_TERM;
   const int STAGE_BYTES = PACK ? B_TILE + 64 * BK_BYTES + A_TERM : A_TILE + B_TILE;
+  const int BMX = PACK ? 64 : BM;  // rows of an m-block (packed: 64, both terms in one M=128 MMA)
   uint8_t* ctl = ring + STAGES * STAGE_BYTES;
   SmemCtl& s = *reinterpret_cast<SmemCtl*>(ctl);
   uint8_t* epi_smem = reinterpret_cast<uint8_t*>(
@@ -320,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (g < p.num_groups) {
         const GroupEntry ge = group_at(p, g);
         if (group_ok(ge, p))
-          tiles = ((ge.rows + BM - 1) / BM) * p.n_tiles;
+          tiles = ((ge.rows + BMX - 1) / BMX) * p.n_tiles;
         else if (ge.rows != 0)
           report(p.status, MOE_STATUS_BAD_GROUP, -1);
       }
@@ -356,9 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t armed = 0, armed_phase = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < total && ok && !p.test_stall; u += gridDim.x) {
-        const UnitInfo ui = decode_unit(s, p, u, ks, nk);
+        const UnitInfo ui = decode_unit(s, p, u, ks, nk, BMX);
         const TileInfo& ti = ui.ti;
-        const int a_row = (p.a_rows_from_out ? ti.grp.out_row0 : ti.grp.a_row0) + ti.m_idx * BM;
+        const int a_row = (p.a_rows_from_out ? ti.grp.out_row0 : ti.grp.a_row0) + ti.m_idx * BMX;
         const CUtensorMap* mA = (ti.grp.expert == p.shared_slab) ? &tmA2 : &tmA;
         const int b_row = ti.grp.expert * p.n_per_slab + ti.n_idx * p.bn_out;
         for (int kb = ui.kb0; kb < ui.kb1; ++kb) {
@@ -459,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = (warp - 2) >> 2;      // which half of the tile's columns it drains
     int local = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x, ++local) {
-      const UnitInfo ui = decode_unit(s, p, u, ks, nk);
+      const UnitInfo ui = decode_unit(s, p, u, ks, nk, BMX);
       const TileInfo& ti = ui.ti;
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
@@ -473,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       // packed two-term A: lane quarters 2, 3 hold the second term's sums of
       // the rows of quarters 0, 1, written as K slices ks .. 2 ks - 1
-      const int row = ti.m_idx * BM + (PACK ? (q & 1) : q) * 32 + lane;
+      const int row = ti.m_idx * BMX + (PACK ? (q & 1) : q) * 32 + lane;
       const bool valid = row < ti.grp.rows;
       const uint32_t tbase = tmem + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16);
       if (PACK)
@@ -529,8 +530,10 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
   int bma = BM;
   if (a.max_group_rows > 0 && a.max_group_rows <= 64) bma = static_cast<int>((a.max_group_rows + 15) & ~int64_t(15));
   const int terms = a.fp8 && a.a_terms == 2 ? 2 : 1;  // two-term E4M3 activations: A rows of 2K codes
-  // both terms in one MMA when every group fits in 64 rows (split-K buffer needed for the second term's sums)
-  const bool pack = terms == 2 && bma <= 64 && p.max_ksplit >= 2;
+  // both terms in one MMA, in m-blocks of 64 rows, when no group exceeds 128 rows (decode; the split-K
+  // buffer holds the second term's sums)
+  const bool pack = terms == 2 && a.max_group_rows > 0 && a.max_group_rows <= 128 && p.max_ksplit >= 2;
+  if (pack && bma > 64) bma = 64;
   const size_t stage_bytes = pack ? static_cast<size_t>(B_TILE + 64 * BK_BYTES + bma * BK_BYTES)
                                   : static_cast<size_t>(bma) * BK_BYTES * terms + B_TILE;
   const int eb = a.fp8 ? 1 : 2;  // element bytes of A and B
@@ -557,7 +560,7 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
     mB1 = mB0;
   }
   // upper bound of the tile count: every group may add one partial m-block
-  const int64_t bound = (a.max_total_rows / BM + a.num_groups) * static_cast<int64_t>(p.n_tiles);
+  const int64_t bound = (a.max_total_rows / (pack ? 64 : BM) + a.num_groups) * static_cast<int64_t>(p.n_tiles);
   const int grid = static_cast<int>(bound < num_sms ? (bound > 0 ? bound : 1) : num_sms);
   if (a.fp8) {  // E4M3 x E4M3 runs SwiGLU experts only
     switch (a.epilogue) {

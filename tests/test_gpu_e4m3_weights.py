@@ -76,6 +76,7 @@ def test_split_rows_bit_exact(n, d):
 
 
 @pytest.mark.parametrize("S,E,K,cap,d,h", [(256, 8, 2, 0, 256, 384), (5, 8, 2, 0, 256, 384),
+                                           (100, 4, 2, 0, 256, 384),   # groups up to 100 rows: 64-row m-blocks
                                            (700, 16, 4, 180, 256, 384), (4200, 4, 1, 0, 256, 384),
                                            (64, 8, 2, 0, 264, 392)])   # d, h not multiples of 16: decode pass
 def test_e4m3_layer_against_bf16_layer_on_decoded_weights(S, E, K, cap, d, h):

@@ -140,11 +140,13 @@ def test_mixtral_decode_sweep_full_weights():
 
 def test_mixtral_decode_e4m3_weights_full_size():
     """The decode sizes on the Mixtral-shaped weights stored as E4M3 with
-    per-channel scales and bf16 activations: the GEMMs decode the weight
-    tiles themselves.  Every token against the oracle (FP8 tolerance)."""
+    per-channel scales and bf16 activations: the GEMMs multiply the weight
+    codes by two-term codes of the activations (both terms in one MMA, in
+    64-row m-blocks at S = 128).  Every token against the oracle (FP8
+    tolerance)."""
     base = syn.VARIANTS["mixtral_decode_e4m3"]
     weights = syn.make_inputs(syn.scaled(base, S=1), "cuda", seed=0)
-    for S in (1, 8, 32):
+    for S in (1, 8, 32, 128):
         cfg = syn.scaled(base, S=S)
         inp = dict(weights)
         inp["x"] = syn.make_inputs(cfg, "cuda", seed=S, x_only=True)["x"]
