@@ -36,7 +36,8 @@ struct TcParams {
   int* ksplit_out;     // the split chosen on the device (read by the finalize kernel)
   int test_stall;      // test hook: the producer delivers nothing (the bounded waits must give up)
   int a_terms;         // E4M3 activations: 1, or 2 for two-term codes (A rows of 2K codes, term 2 at column K)
-  int a_pack;          // two-term codes with groups of <= 64 rows: both terms in one M=128 MMA (rows 0.., 64..)
+  int a_pack;          // two-term codes, 64-row m-blocks: both terms in one M=128 MMA (A rows 0.., 64..)
+  int bm;              // rows of an m-block: 128, or 64 when no group exceeds 128 rows
   int tma_out;         // 1: the output tensor map is valid (full 32-row quarters use bulk tensor stores)
   const float* row_scale;         // E4M3 activations: per-row scale of the A operand rows (nullptr: none)
   const float* row_scale_shared;  // ... of the shared expert's A rows (indexed by row within the group)

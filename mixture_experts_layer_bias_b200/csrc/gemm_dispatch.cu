@@ -67,6 +67,7 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t 
   p.tma_out = 0;  // set by the launcher when it can map the output
   p.a_terms = 1;  // set by the launcher
   p.a_pack = 0;
+  p.bm = 128;  // set by the launcher
   p.row_scale = a.fp8 ? a.row_scale : nullptr;
   p.row_scale_shared = a.fp8 ? a.row_scale_shared : nullptr;
   if (a.fp8 && a.row_scale == nullptr) return cudaErrorInvalidValue;

@@ -42,6 +42,8 @@
 // in flight, frees its TMEM and exits.  No load uses cluster multicast.
 #include <math.h>
 
+#include <algorithm>
+
 #include <stdlib.h>
 #include <string.h>
 
@@ -57,11 +59,13 @@ using namespace gemm;
 constexpr int BM = 128;
 constexpr int BK_BYTES = 128;  // one swizzle row: 64 bf16 or 128 E4M3 elements of K per stage
 // Ring: one stage = A rows (bma x 64 bf16, bma <= 128) then B (256 x 64 bf16).
-// Prefill loads all 128 token rows of A (4 stages of 48 KB).  When every group
-// fits in bma < 128 rows (decode), only those rows are loaded and the shared
-// memory saved becomes extra stages, i.e. more weight bytes in flight; the
-// MMA still reads 128 A rows, the rows past bma being the start of the same
-// stage's B tile, and their accumulator rows are never stored.
+// Prefill loads all 128 token rows of A (4 stages of 48 KB).  When no group
+// exceeds 128 rows (decode), m-blocks have 64 rows and only the bma <= 64 rows
+// the largest group can fill are loaded; the shared memory saved becomes extra
+// stages, i.e. more weight bytes in flight.  The MMA still reads 128 A rows,
+// the rows past bma being the start of the next tile in shared memory, and
+// their accumulator rows are never stored (with two-term codes the second
+// term's rows sit at A rows 64.. and share the MMA).
 constexpr int MAX_STAGES = 8;
 constexpr int B_HALF = 128 * BK_BYTES;        // 16 KB
 constexpr int B_TILE = 2 * B_HALF;            // 32 KB
@@ -276,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int A_OFF = PACK ? B_TILE : 0;
   const int A2_OFF = PACK ? B_TILE + 64 * BK_BYTES : A_TERM;
   const int STAGE_BYTES = PACK ? B_TILE + 64 * BK_BYTES + A_TERM : A_TILE + B_TILE;
-  const int BMX = PACK ? 64 : BM;  // rows of an m-block (packed: 64, both terms in one M=128 MMA)
+  const int BMX = p.bm;  // rows of an m-block: 128, or 64 for groups of at most 128 rows (decode)
   uint8_t* ctl = ring + STAGES * STAGE_BYTES;
   SmemCtl& s = *reinterpret_cast<SmemCtl*>(ctl);
   uint8_t* epi_smem = reinterpret_cast<uint8_t*>(
@@ -473,16 +477,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       // packed two-term A: lane quarters 2, 3 hold the second term's sums of
-      // the rows of quarters 0, 1, written as K slices ks .. 2 ks - 1
-      const int row = ti.m_idx * BMX + (PACK ? (q & 1) : q) * 32 + lane;
-      const bool valid = row < ti.grp.rows;
-      const uint32_t tbase = tmem + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16);
-      if (PACK)
-        epilogue_partial<EPI>(p, ti, tbase, row, valid, ui.split + (q >> 1) * ks, half);
-      else if (ks > 1)
-        epilogue_partial<EPI>(p, ti, tbase, row, valid, ui.split, half);
-      else
-        epilogue_store<EPI>(p, ti, tbase, row, valid, lane, half, &tmOut, epi_smem + (warp - 2) * kEpiWarpBytes);
+      // the rows of quarters 0, 1, written as K slices ks .. 2 ks - 1; with
+      // 64-row m-blocks and one term, quarters 2, 3 hold no rows of the block
+      const int qrow = PACK ? (q & 1) : q;
+      if (qrow * 32 < BMX) {  // warp-uniform
+        const int row = ti.m_idx * BMX + qrow * 32 + lane;
+        const bool valid = row < ti.grp.rows;
+        const uint32_t tbase = tmem + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16);
+        if (PACK)
+          epilogue_partial<EPI>(p, ti, tbase, row, valid, ui.split + (q >> 1) * ks, half);
+        else if (ks > 1)
+          epilogue_partial<EPI>(p, ti, tbase, row, valid, ui.split, half);
+        else
+          epilogue_store<EPI>(p, ti, tbase, row, valid, lane, half, &tmOut, epi_smem + (warp - 2) * kEpiWarpBytes);
+      }
       tc_fence_before();
       mbar_arrive(&s.tempty[acc]);
     }
@@ -526,14 +534,15 @@ cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUte
 
 // Token-rows kernel launch; `p` is filled by launch_grouped_gemm_tc.
 cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& p, int num_sms, cudaStream_t stream) {
-  // A rows loaded per stage: all 128, or (every group fitting) the largest group rounded up to 16
-  int bma = BM;
-  if (a.max_group_rows > 0 && a.max_group_rows <= 64) bma = static_cast<int>((a.max_group_rows + 15) & ~int64_t(15));
+  // m-blocks of 128 rows; when no group exceeds 128 rows (decode), m-blocks of 64 rows, of which
+  // only the rows the largest group can fill (rounded up to 16) are loaded: the shared memory saved
+  // becomes extra stages, i.e. more weight bytes in flight
+  const bool half = a.max_group_rows > 0 && a.max_group_rows <= 128;
+  const int bm = half ? 64 : BM;
+  const int bma = half ? static_cast<int>(std::min<int64_t>(64, (a.max_group_rows + 15) & ~int64_t(15))) : BM;
   const int terms = a.fp8 && a.a_terms == 2 ? 2 : 1;  // two-term E4M3 activations: A rows of 2K codes
-  // both terms in one MMA, in m-blocks of 64 rows, when no group exceeds 128 rows (decode; the split-K
-  // buffer holds the second term's sums)
-  const bool pack = terms == 2 && a.max_group_rows > 0 && a.max_group_rows <= 128 && p.max_ksplit >= 2;
-  if (pack && bma > 64) bma = 64;
+  // both terms in one MMA (64-row m-blocks; the split-K buffer holds the second term's sums)
+  const bool pack = terms == 2 && half && p.max_ksplit >= 2;
   const size_t stage_bytes = pack ? static_cast<size_t>(B_TILE + 64 * BK_BYTES + bma * BK_BYTES)
                                   : static_cast<size_t>(bma) * BK_BYTES * terms + B_TILE;
   const int eb = a.fp8 ? 1 : 2;  // element bytes of A and B
@@ -547,6 +556,7 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
   if (!pp.tma_out) memset(&mOut, 0, sizeof(mOut));
   pp.a_terms = terms;
   pp.a_pack = pack ? 1 : 0;
+  pp.bm = bm;
   if (!make_map(&mA, a.a, a.a_rows, a.K * terms, bma, eb)) return cudaErrorInvalidValue;
   if (a.a_shared != nullptr) {
     if (!make_map(&mA2, a.a_shared, a.a_shared_rows, a.K * terms, bma, eb)) return cudaErrorInvalidValue;
@@ -560,7 +570,7 @@ cudaError_t launch_grouped_gemm_single(const GemmArgs& a, const gemm::TcParams& 
     mB1 = mB0;
   }
   // upper bound of the tile count: every group may add one partial m-block
-  const int64_t bound = (a.max_total_rows / (pack ? 64 : BM) + a.num_groups) * static_cast<int64_t>(p.n_tiles);
+  const int64_t bound = (a.max_total_rows / bm + a.num_groups) * static_cast<int64_t>(p.n_tiles);
   const int grid = static_cast<int>(bound < num_sms ? (bound > 0 ? bound : 1) : num_sms);
   if (a.fp8) {  // E4M3 x E4M3 runs SwiGLU experts only
     switch (a.epilogue) {
