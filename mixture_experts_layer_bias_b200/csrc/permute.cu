@@ -24,6 +24,7 @@
 #include "kernels.h"
 #include "pdl.cuh"
 #include "route_select.cuh"
+#include "row_coding.cuh"
 
 namespace moe {
 
@@ -334,20 +335,81 @@ __device__ void permute_small_body(int S, int E, int K, int capacity, int num_sh
   if (g1 != nullptr) write_groups(S, E, K, capacity, num_shared, offs_s, g1);
 }
 
+// Coded row gather of a tiny batch inside the one-CTA permutation: a warp per
+// token codes the row once (coding::row_load_amax / row_scale, as
+// gather_quantize_kernel) and writes the codes to the token's K rows of q_perm
+// and, when given, to row t of q_x (the shared expert's operand).
+struct FoldCodes {
+  const __nv_bfloat16* x;
+  uint8_t* q_perm;
+  float* s_perm;
+  uint8_t* q_x;
+  float* s_x;
+  int terms, d;
+};
+
+__device__ void code_gather_small(int S, int K, const int32_t* __restrict__ row_of_slot, const FoldCodes& f) {
+  using namespace coding;
+  const int warp = threadIdx.x >> 5, lane = lane_id();
+  const int d = f.d;
+  const int64_t pitch = static_cast<int64_t>(f.terms) * d;
+  for (int t = warp; t < S; t += kSmallWarps) {
+    const __nv_bfloat16* src = f.x + static_cast<int64_t>(t) * d;
+    RowPieces<32> rp;
+    float amax, s, m;
+    bool nan, nonfinite;
+    row_load_amax<32>(src, d, lane, rp, amax, nan, nonfinite);
+    row_scale(f.terms, amax, nan, nonfinite, s, m);
+    const int my_row = lane < K ? row_of_slot[static_cast<int64_t>(t) * K + lane] : -1;
+    auto put = [&](const uint4& w, int c) {
+      uint2 q, q2 = make_uint2(0, 0);
+      if (f.terms == 2)
+        encode8_two_term(w, m, q, q2);
+      else
+        q = encode8_w8a8(w, s);
+      for (int k = 0; k < K; ++k) {
+        const int row = __shfl_sync(kFull, my_row, k);
+        if (row >= 0) {
+          *reinterpret_cast<uint2*>(f.q_perm + row * pitch + c) = q;
+          if (f.terms == 2) *reinterpret_cast<uint2*>(f.q_perm + row * pitch + d + c) = q2;
+        }
+      }
+      if (f.q_x != nullptr) {
+        *reinterpret_cast<uint2*>(f.q_x + t * pitch + c) = q;
+        if (f.terms == 2) *reinterpret_cast<uint2*>(f.q_x + t * pitch + d + c) = q2;
+      }
+    };
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) {
+      const int c = (lane + i * 32) * 8;
+      if (c < d) put(rp.v[i], c);
+    }
+    for (int c = (lane + kVec * 32) * 8; c < d; c += 256) put(ldg16(src + c), c);
+    if (my_row >= 0) f.s_perm[my_row] = s;
+    if (lane == 0 && f.s_x != nullptr) f.s_x[t] = s;
+  }
+}
+
 // x / x_perm (optional): the row gather of a tiny batch folded in -- every
 // token row (row_chunks 16-byte pieces) copied to its slots' rows once the
-// maps are written, so a decode step spends no launch on it.
+// maps are written, so a decode step spends no launch on it; or, with
+// codes.q_perm, the coded row gather (code_gather_small).
 __global__ void __launch_bounds__(kSmallWarps * 32)
     permute_small_kernel(int S, int E, int K, int capacity, int num_shared, const int32_t* topk_idx,
                          int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                          int32_t* __restrict__ row_of_slot, int32_t* __restrict__ token_of_row, int64_t num_rows,
                          GroupEntry* __restrict__ g1, StatusBlock* status, const uint4* __restrict__ x,
-                         uint4* __restrict__ x_perm, int row_chunks) {
+                         uint4* __restrict__ x_perm, int row_chunks, FoldCodes codes) {
   extern __shared__ int32_t sm[];
   pdl_wait();
   pdl_trigger();
   permute_small_body(S, E, K, capacity, num_shared, topk_idx, counts, offsets, row_of_slot, token_of_row, num_rows,
                      g1, status, sm);
+  if (codes.q_perm != nullptr) {
+    __syncthreads();  // the row maps written above are read back below
+    code_gather_small(S, K, row_of_slot, codes);
+    return;
+  }
   if (x == nullptr) return;
   __syncthreads();  // the row maps written above are read back below
   const int64_t n = static_cast<int64_t>(S) * K * row_chunks;
@@ -452,14 +514,24 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
   cudaError_t err;
   const int64_t row_bytes = static_cast<int64_t>(a.d) * (a.act_dtype == MOE_BF16 ? 2 : 4);
   bool gathered = false;
+  const bool coded = a.terms > 0 && a.x != nullptr && a.q_perm != nullptr;
+  FoldCodes codes{};
   if (static_cast<int64_t>(a.S) * a.K <= kSmallSlots) {
     const size_t smem = sizeof(int32_t) * (kSmallWarps * a.E + 3 * a.E + 1);
-    // tiny batches: the one CTA also copies the rows (a few hundred KB at most)
-    gathered = a.x != nullptr && a.x_perm != nullptr && static_cast<int64_t>(a.S) * a.K * row_bytes <= kFoldGatherBytes;
+    // tiny batches: the one CTA also copies (or codes) the rows (a few hundred KB at most)
+    if (coded) {
+      gathered = static_cast<int64_t>(a.S) * a.K * a.d * a.terms <= kFoldGatherBytes && a.S <= kSmallWarps;
+      if (gathered)
+        codes = FoldCodes{static_cast<const __nv_bfloat16*>(a.x), a.q_perm, a.s_perm, a.q_x, a.s_x, a.terms, a.d};
+    } else {
+      gathered = a.x != nullptr && a.x_perm != nullptr &&
+                 static_cast<int64_t>(a.S) * a.K * row_bytes <= kFoldGatherBytes;
+    }
+    const bool copy = gathered && !coded;
     err = launch_pdl(permute_small_kernel, dim3(1), dim3(kSmallWarps * 32), smem, stream, a.S, a.E, a.K, a.capacity,
                      a.num_shared, a.topk_idx, a.counts, a.offsets, a.row_of_slot, a.token_of_row, a.num_rows, a.g1,
-                     a.status, gathered ? static_cast<const uint4*>(a.x) : nullptr,
-                     gathered ? static_cast<uint4*>(a.x_perm) : nullptr, static_cast<int>(row_bytes / 16));
+                     a.status, copy ? static_cast<const uint4*>(a.x) : nullptr,
+                     copy ? static_cast<uint4*>(a.x_perm) : nullptr, static_cast<int>(row_bytes / 16), codes);
     if (err != cudaSuccess || (err = cudaGetLastError()) != cudaSuccess) return err;
   } else {
     const int tpc = permute_tokens_per_chunk(a.K);
@@ -485,6 +557,11 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
       build_groups_kernel<<<1, 256, 0, stream>>>(a.S, a.E, a.K, a.capacity, a.num_shared, a.offsets, a.g1);
       if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
+  }
+  if (coded) {
+    if (gathered) return cudaSuccess;
+    return launch_gather_quantize(a.S, a.d, a.K, a.row_of_slot, a.x, a.q_perm, a.s_perm, a.q_x, a.s_x, a.terms,
+                                  stream);
   }
   if (a.x == nullptr || a.x_perm == nullptr || gathered) return cudaSuccess;
   if (a.S <= 256) {

@@ -50,6 +50,9 @@ CASES = [
     ("tiny_f32", dict(S=16, E=32, K=4)),
     ("mixtral_decode", dict(S=7, d=512, h=512, E=32, K=4, capacity=1)),   # capacity with overflow rows
     ("mixtral_prefill_w8a8", dict(S=9, d=512, h=512)),                  # quantising gather
+    ("mixtral_decode", dict(S=120, d=512, h=512, E=2, K=2)),            # groups of 120 rows: two 64-row blocks
+    ("mixtral_decode_e4m3", dict(S=120, d=512, h=512, E=2, K=2)),       # the same, both E4M3 terms in one MMA
+    ("mixtral_prefill_w8a8", dict(S=120, d=512, h=512, E=2, K=2)),      # the same with one E4M3 term
 ]
 
 
