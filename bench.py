@@ -138,7 +138,7 @@ def kernels_per_step(cfg, S=None):
     n += 1 if small else 4                 # permutation (+ group table): one kernel, or count, scan, scatter, groups
     coded = coded_a_rows(cfg)
     terms = 1 if cfg.act_quant else 2
-    folded = small and ((S * cfg.K * cfg.d * terms <= 256 * 1024 and S <= 32) if coded
+    folded = small and ((S * cfg.K * cfg.d * terms <= 256 * 1024 and S <= 8) if coded
                         else S * cfg.K * cfg.d * elem <= 256 * 1024)
     if not folded:
         n += 1                             # row gather (writing E4M3 codes when coded); tiny batches: inside the permutation
