@@ -137,11 +137,8 @@ def kernels_per_step(cfg, S=None):
     n = 2 if logits_first else 1           # logits GEMM + top-k, or the routing kernel computing the logits
     n += 1 if small else 4                 # permutation (+ group table): one kernel, or count, scan, scatter, groups
     coded = coded_a_rows(cfg)
-    terms = 1 if cfg.act_quant else 2
-    folded = small and ((S * cfg.K * cfg.d * terms <= 256 * 1024 and S <= 8) if coded
-                        else S * cfg.K * cfg.d * elem <= 256 * 1024)
-    if not folded:
-        n += 1                             # row gather (writing E4M3 codes when coded); tiny batches: inside the permutation
+    if coded or not (small and S * cfg.K * cfg.d * elem <= 256 * 1024):
+        n += 1                             # row gather (writing E4M3 codes); tiny bf16 batches: inside the permutation
     n += 2                                 # up and down GEMM
     rows = S * cfg.K + cfg.num_shared * S + (cfg.E * cfg.capacity if cfg.capacity else 0)
     if cfg.act_dtype == syn.BF16 and rows <= 4096:

@@ -268,21 +268,9 @@ moe_status debug_check(const PermuteArgs& a, cudaStream_t st) {
 
 moe_status permute_impl(const moe_desc& d, const void* x, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
                         int32_t* row_of_slot, int32_t* token_of_row, void* x_perm, void* ws, cudaStream_t st,
-                        bool write_groups = false, bool coded_rows = false) {
-  PermuteArgs a =
+                        bool write_groups = false) {
+  const PermuteArgs a =
       permute_args(d, x, topk_idx, counts, offsets, row_of_slot, token_of_row, x_perm, ws, write_groups);
-  if (coded_rows) {
-    // E4M3 A rows: the row gather writes the codes and row scales of the
-    // tokens (and of the shared expert's rows) instead of bf16 rows
-    const Layout L = make_layout(d);
-    const bool sh = d.num_shared != 0;
-    a.x_perm = nullptr;
-    a.terms = a_terms(d);
-    a.q_perm = at<uint8_t>(ws, L.qa);
-    a.s_perm = at<float>(ws, L.sa);
-    a.q_x = sh ? at<uint8_t>(ws, L.qas) : nullptr;
-    a.s_x = sh ? at<float>(ws, L.sas) : nullptr;
-  }
   const moe_status s = cuda_status(launch_permute(a, st));
   return s != MOE_OK ? s : debug_check(a, st);
 }
@@ -518,8 +506,13 @@ moe_status layer_impl(const moe_desc* desc, const moe_weights* w, const void* x,
   // the permutation also writes the GEMM group tables, so the FFN skips that launch
   if (terms) {
     // E4M3 A rows: the row gather writes the codes and row scales straight
-    // away (no bf16 copy of the permuted rows; tiny batches inside the permutation)
-    if ((s = permute_impl(d, x, idx, cnt, offs, ros, tor, nullptr, ws, st, true, true)) != MOE_OK) return s;
+    // away (no bf16 copy of the permuted rows)
+    if ((s = permute_impl(d, nullptr, idx, cnt, offs, ros, tor, nullptr, ws, st, true)) != MOE_OK) return s;
+    const bool sh = d.num_shared != 0;
+    if (launch_gather_quantize(d.num_tokens, d.d_model, d.top_k, ros, x, at<uint8_t>(ws, L.qa), at<float>(ws, L.sa),
+                               sh ? at<uint8_t>(ws, L.qas) : nullptr, sh ? at<float>(ws, L.sas) : nullptr, terms,
+                               st) != cudaSuccess)
+      return MOE_ERR_CUDA;
     if (!record(events, 2, st)) return MOE_ERR_CUDA;
     if ((s = ffn_impl(d, *w, x_perm, offs, x, y_perm, ws, st, true, true, events)) != MOE_OK) return s;
   } else {

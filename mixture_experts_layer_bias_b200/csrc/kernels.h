@@ -86,14 +86,6 @@ struct PermuteArgs {
   // optional: also write the GEMM group table (see GroupEntry)
   GroupEntry* g1;
   int num_shared;
-  // optional (terms 1 or 2, x given, x_perm nullptr): the row gather writes
-  // E4M3 codes and row scales instead of bf16 rows (launch_gather_quantize),
-  // folded into the one-CTA permutation for tiny batches
-  int terms;
-  uint8_t* q_perm;
-  float* s_perm;
-  uint8_t* q_x;
-  float* s_x;
 };
 int permute_num_chunks(int S, int K);
 int permute_tokens_per_chunk(int K);

@@ -24,7 +24,6 @@
 #include "kernels.h"
 #include "pdl.cuh"
 #include "route_select.cuh"
-#include "row_coding.cuh"
 
 namespace moe {
 
@@ -335,104 +334,20 @@ __device__ void permute_small_body(int S, int E, int K, int capacity, int num_sh
   if (g1 != nullptr) write_groups(S, E, K, capacity, num_shared, offs_s, g1);
 }
 
-// Coded row gather of a tiny batch (S <= kFoldCodeTokens) inside the one-CTA
-// permutation: the CTA's 1024 threads split into S groups of G = 1024 / S'
-// threads (S' = S rounded up to a power of two), one token per group.  A group
-// reads its row once into registers, reduces the row maximum over its warps
-// (shuffles, then shared memory and a named barrier of the group), and writes
-// the codes (coding::row_scale / encode, as gather_quantize_kernel) to the
-// token's K rows of q_perm and, when given, to row t of q_x.
-constexpr int kFoldCodeTokens = 8;
-
-struct FoldCodes {
-  const __nv_bfloat16* x;
-  uint8_t* q_perm;
-  float* s_perm;
-  uint8_t* q_x;
-  float* s_x;
-  int terms, d;
-};
-
-__device__ void code_gather_small(int S, int K, const int32_t* __restrict__ row_of_slot, const FoldCodes& f) {
-  using namespace coding;
-  __shared__ uint32_t red[kSmallWarps];
-  const int sp = S <= 1 ? 1 : S <= 2 ? 2 : S <= 4 ? 4 : 8;
-  const int G = kSmallWarps * 32 / sp;  // threads per token: 1024 .. 128
-  const int t = threadIdx.x / G, gt = threadIdx.x % G;
-  if (t >= S) return;  // whole groups only
-  const int warp = threadIdx.x >> 5, lane = lane_id();
-  const int d = f.d;
-  const int64_t pitch = static_cast<int64_t>(f.terms) * d;
-  const __nv_bfloat16* src = f.x + static_cast<int64_t>(t) * d;
-  constexpr int kFoldVec = 4;  // pieces held in registers (d = 4096 at 128 threads per token)
-  uint4 v[kFoldVec];
-  uint32_t acc = 0;
-#pragma unroll
-  for (int i = 0; i < kFoldVec; ++i) {
-    const int c = (gt + i * G) * 8;
-    v[i] = c < d ? ldg16(src + c) : make_uint4(0, 0, 0, 0);
-  }
-#pragma unroll
-  for (int i = 0; i < kFoldVec; ++i) acc = absmax_bits8(acc, v[i]);
-  for (int c = (gt + kFoldVec * G) * 8; c < d; c += G * 8) acc = absmax_bits8(acc, ldg16(src + c));
-  red[warp] = __reduce_max_sync(kFull, max(acc & 0xFFFFu, acc >> 16));
-  // the group's warps: named barrier 1 + t (barrier 0 is __syncthreads)
-  asm volatile("bar.sync %0, %1;" ::"r"(1 + t), "r"(G) : "memory");
-  uint32_t bits = 0;
-  for (int w = t * (G / 32); w < (t + 1) * (G / 32); ++w) bits = max(bits, red[w]);
-  float s, m;
-  row_scale(f.terms, __uint_as_float(bits << 16), bits > 0x7F80u, bits >= 0x7F80u, s, m);
-  auto put = [&](const uint4& w, int c) {
-    uint2 q, q2 = make_uint2(0, 0);
-    if (f.terms == 2)
-      encode8_two_term(w, m, q, q2);
-    else
-      q = encode8_w8a8(w, s);
-    for (int k = 0; k < K; ++k) {
-      const int row = row_of_slot[static_cast<int64_t>(t) * K + k];
-      if (row >= 0) {
-        *reinterpret_cast<uint2*>(f.q_perm + row * pitch + c) = q;
-        if (f.terms == 2) *reinterpret_cast<uint2*>(f.q_perm + row * pitch + d + c) = q2;
-      }
-    }
-    if (f.q_x != nullptr) {
-      *reinterpret_cast<uint2*>(f.q_x + t * pitch + c) = q;
-      if (f.terms == 2) *reinterpret_cast<uint2*>(f.q_x + t * pitch + d + c) = q2;
-    }
-  };
-#pragma unroll
-  for (int i = 0; i < kFoldVec; ++i) {
-    const int c = (gt + i * G) * 8;
-    if (c < d) put(v[i], c);
-  }
-  for (int c = (gt + kFoldVec * G) * 8; c < d; c += G * 8) put(ldg16(src + c), c);
-  if (gt < K) {
-    const int row = row_of_slot[static_cast<int64_t>(t) * K + gt];
-    if (row >= 0) f.s_perm[row] = s;
-  }
-  if (gt == 0 && f.s_x != nullptr) f.s_x[t] = s;
-}
-
 // x / x_perm (optional): the row gather of a tiny batch folded in -- every
 // token row (row_chunks 16-byte pieces) copied to its slots' rows once the
-// maps are written, so a decode step spends no launch on it; or, with
-// codes.q_perm, the coded row gather (code_gather_small).
+// maps are written, so a decode step spends no launch on it.
 __global__ void __launch_bounds__(kSmallWarps * 32)
     permute_small_kernel(int S, int E, int K, int capacity, int num_shared, const int32_t* topk_idx,
                          int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                          int32_t* __restrict__ row_of_slot, int32_t* __restrict__ token_of_row, int64_t num_rows,
                          GroupEntry* __restrict__ g1, StatusBlock* status, const uint4* __restrict__ x,
-                         uint4* __restrict__ x_perm, int row_chunks, FoldCodes codes) {
+                         uint4* __restrict__ x_perm, int row_chunks) {
   extern __shared__ int32_t sm[];
   pdl_wait();
   pdl_trigger();
   permute_small_body(S, E, K, capacity, num_shared, topk_idx, counts, offsets, row_of_slot, token_of_row, num_rows,
                      g1, status, sm);
-  if (codes.q_perm != nullptr) {
-    __syncthreads();  // the row maps written above are read back below
-    code_gather_small(S, K, row_of_slot, codes);
-    return;
-  }
   if (x == nullptr) return;
   __syncthreads();  // the row maps written above are read back below
   const int64_t n = static_cast<int64_t>(S) * K * row_chunks;
@@ -537,24 +452,14 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
   cudaError_t err;
   const int64_t row_bytes = static_cast<int64_t>(a.d) * (a.act_dtype == MOE_BF16 ? 2 : 4);
   bool gathered = false;
-  const bool coded = a.terms > 0 && a.x != nullptr && a.q_perm != nullptr;
-  FoldCodes codes{};
   if (static_cast<int64_t>(a.S) * a.K <= kSmallSlots) {
     const size_t smem = sizeof(int32_t) * (kSmallWarps * a.E + 3 * a.E + 1);
-    // tiny batches: the one CTA also copies (or codes) the rows (a few hundred KB at most)
-    if (coded) {
-      gathered = static_cast<int64_t>(a.S) * a.K * a.d * a.terms <= kFoldGatherBytes && a.S <= kFoldCodeTokens;
-      if (gathered)
-        codes = FoldCodes{static_cast<const __nv_bfloat16*>(a.x), a.q_perm, a.s_perm, a.q_x, a.s_x, a.terms, a.d};
-    } else {
-      gathered = a.x != nullptr && a.x_perm != nullptr &&
-                 static_cast<int64_t>(a.S) * a.K * row_bytes <= kFoldGatherBytes;
-    }
-    const bool copy = gathered && !coded;
+    // tiny batches: the one CTA also copies the rows (a few hundred KB at most)
+    gathered = a.x != nullptr && a.x_perm != nullptr && static_cast<int64_t>(a.S) * a.K * row_bytes <= kFoldGatherBytes;
     err = launch_pdl(permute_small_kernel, dim3(1), dim3(kSmallWarps * 32), smem, stream, a.S, a.E, a.K, a.capacity,
                      a.num_shared, a.topk_idx, a.counts, a.offsets, a.row_of_slot, a.token_of_row, a.num_rows, a.g1,
-                     a.status, copy ? static_cast<const uint4*>(a.x) : nullptr,
-                     copy ? static_cast<uint4*>(a.x_perm) : nullptr, static_cast<int>(row_bytes / 16), codes);
+                     a.status, gathered ? static_cast<const uint4*>(a.x) : nullptr,
+                     gathered ? static_cast<uint4*>(a.x_perm) : nullptr, static_cast<int>(row_bytes / 16));
     if (err != cudaSuccess || (err = cudaGetLastError()) != cudaSuccess) return err;
   } else {
     const int tpc = permute_tokens_per_chunk(a.K);
@@ -580,11 +485,6 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t stream) {
       build_groups_kernel<<<1, 256, 0, stream>>>(a.S, a.E, a.K, a.capacity, a.num_shared, a.offsets, a.g1);
       if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
-  }
-  if (coded) {
-    if (gathered) return cudaSuccess;
-    return launch_gather_quantize(a.S, a.d, a.K, a.row_of_slot, a.x, a.q_perm, a.s_perm, a.q_x, a.s_x, a.terms,
-                                  stream);
   }
   if (a.x == nullptr || a.x_perm == nullptr || gathered) return cudaSuccess;
   if (a.S <= 256) {

@@ -39,8 +39,7 @@ def test_committed_traffic_record_is_current_or_absent():
     ("fp8_skew_capacity", None, 2 + 4 + 1 + 2 + 1 + 1),     # E = 64: router GEMM + top-k; codes of the hidden rows
     ("mixtral_prefill_w8a8", None, 1 + 4 + 1 + 2 + 1 + 1),  # + quantisation of the hidden rows
     ("fp8_skew_capacity_reroute", None, 2 + 4 + 1 + 2 + 1 + 7 + 1),  # + ranks (3), picks, epochs, apply, gates
-    ("mixtral_decode_e4m3", 1, 1 + 1 + 2 + 2 + 1 + 1),      # coded gather in the permutation, split-K finalizes, hidden codes
-    ("mixtral_decode_e4m3", 32, 1 + 1 + 1 + 2 + 2 + 1 + 1),  # 32 x 2 rows of 8 KB of codes: the coding gather kernel
+    ("mixtral_decode_e4m3", 1, 1 + 1 + 1 + 2 + 2 + 1 + 1),  # coded gather, split-K finalizes, hidden codes
     ("mixtral_decode", 1, 1 + 1 + 2 + 2 + 1),               # one-CTA permutation with the gather, split-K finalizes
     ("mixtral_decode", 8, 1 + 1 + 2 + 2 + 1),               # 8 x 2 rows of 8 KB: gathered by the permutation
     ("mixtral_decode", 32, 1 + 1 + 1 + 2 + 2 + 1),          # 512 KB of rows: the gather kernel
