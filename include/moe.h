@@ -250,11 +250,14 @@ moe_status moe_permute_static(const moe_desc *desc, const void *x, const int32_t
  *   The hidden activations live in the workspace.  Rows outside any group
  *   (unused capacity rows) are not written.  With a capacity, each expert's
  *   overflow rows are processed in the same GEMM launches, right after its
- *   primary rows.  E4M3 weights with act_quant = 0 are decoded exactly to
- *   bf16 into the workspace on every call (the channel scales multiply the
- *   fp32 accumulators); with act_quant = 1 the A rows of both GEMMs (x_perm
- *   rows and, for the shared expert, x rows; then the hidden rows) are
- *   quantised per row into the workspace and the GEMMs read E4M3 codes.
+ *   primary rows.  With E4M3 weights the A rows of both GEMMs (x_perm rows
+ *   and, for the shared expert, x rows; then the hidden rows) are coded per
+ *   row into the workspace -- two-term codes (moe_split_rows_e4m3) with
+ *   act_quant = 0, W8A8 codes (moe_quantize_rows_e4m3) with act_quant = 1 --
+ *   and the GEMMs multiply them with the stored weight codes; the row and
+ *   channel scales multiply the fp32 accumulators.  E4M3 weights with d or h
+ *   not a multiple of 16 (act_quant = 0) are instead decoded exactly to bf16
+ *   into the workspace on every call.
  */
 moe_status moe_grouped_ffn(const moe_desc *desc, const moe_weights *w, const void *x_perm,
                            const int32_t *offsets, const void *x, void *y_perm, void *ws, size_t ws_bytes,
@@ -348,7 +351,7 @@ moe_status moe_layer_forward(const moe_desc *desc, const moe_weights *w, const v
  * NULL (skipped) or an event created on the current device:
  *   [0] before routing             [1] after routing (and re-routing)
  *   [2] after the permutation       [3] before the up-projection GEMM (after
- *   any E4M3 weight decode or activation quantisation of the FFN)
+ *   any E4M3 weight decode or coding of the A rows in the FFN)
  *   [4] after the up-projection GEMM   [5] before the down-projection GEMM
  *   [6] after the down-projection GEMM [7] after the combine.
  * Errors as moe_layer_forward; MOE_ERR_CUDA when an event record fails.
