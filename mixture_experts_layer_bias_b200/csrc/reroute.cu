@@ -407,14 +407,12 @@ __device__ __forceinline__ void repick_token(int t, int64_t first, int E, int K,
   for (int j = 0; j < 16; ++j)
     kv[j] = (regs && 4 * j < E) ? __ldg(reinterpret_cast<const float4*>(row) + j)
                                 : make_float4(kNegInf, kNegInf, kNegInf, kNegInf);
-  int pk[32];  // the token's picks, loaded together with its experts and keys
-#pragma unroll
-  for (int k = 0; k < 32; ++k)
-    if (k < K) pk[k] = pick.get(s0 + k);
   uint32_t held[kMaskWords];
   held_of(topk_idx + s0, K, E, vec, held);
+  // the picks are read slot by slot: an array of them indexed by k would live
+  // in local memory, which with the picks filling shared memory misses L1
   for (int k = 0; k < K; ++k) {
-    int p = pk[k];
+    int p = pick.get(s0 + k);
     if (p == kKept) continue;
     if (k >= k0 && p >= 0 && (bit_of(sm.full, p) || has_bit(held, p))) {
       const int q = regs ? best_candidate_regs(kv, E, sm.avail, held) : best_candidate(row, E, sm.avail, held);
