@@ -669,6 +669,32 @@ def test_split_rows_error_bound_and_special_rows():
     assert not c1[2:].any() and not c2[2:].any()
 
 
+def test_split_rows_expert_equals_bf16_expert_within_bound():
+    """A SwiGLU expert fed the two-term reconstruction of bf16 rows
+    ((c1 + c2) * scale) equals the expert on the bf16 rows themselves within
+    the bound the split guarantees (every element within 2**-10 * scale of its
+    value), propagated through the up projections: |x W| changes by at most
+    2**-10 * scale * sum_k |W[n, k]|.  On rows of limited spread (every value
+    at least 2**-9 of its row maximum) the two agree exactly."""
+    rng = np.random.default_rng(33)
+    d, h = 48, 40
+    wg, wu = rng.normal(size=(h, d)) / 7, rng.normal(size=(h, d)) / 7
+    for spread, exact in ((9.0, True), (24.0, False)):
+        x = _bf16_rows(rng, 25, d, spread).astype(np.float64)
+        c1, c2, sc = O.split_rows_e4m3(x.astype(np.float32))
+        xr = (O.e4m3_bits_to_f64(c1) + O.e4m3_bits_to_f64(c2)) * sc[:, None].astype(np.float64)
+        if exact:
+            assert np.array_equal(xr, x)
+        bound_x = 2.0 ** -10 * sc[:, None].astype(np.float64)
+        assert np.all(np.abs(xr - x) <= bound_x)
+        g, u = x @ wg.T, x @ wu.T
+        gr, ur = xr @ wg.T, xr @ wu.T
+        bg = bound_x * np.abs(wg).sum(axis=1)[None, :]
+        bu = bound_x * np.abs(wu).sum(axis=1)[None, :]
+        assert np.all(np.abs(gr - g) <= bg * (1 + 1e-9) + 1e-300)
+        assert np.all(np.abs(ur - u) <= bu * (1 + 1e-9) + 1e-300)
+
+
 def test_w8a8_expert_close_to_exact_expert():
     """With 8-bit activations the expert output stays within the quantisation
     noise of the same expert on unquantised activations (relative L2 a few
