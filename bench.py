@@ -74,7 +74,7 @@ GEMM_TRAFFIC_CAPTURE = {
     # one-pass ncu capture of the full-size workload (None: not captured on the current GEMM sources)
     "bytes": 3669152512,  # 1946752512 + 228090368 (up) + 1432097536 + 62212096 (down)
     "sources": ("common.cuh", "gemm_common.cuh", "gemm_sm100.cu"),
-    "sha1": "2a55588aef87395e1041b3421018faabd9bb7801",
+    "sha1": "112b954715e693cb4ff154f8fa636d82bd54d4db",
 }
 
 

@@ -43,6 +43,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include <stdlib.h>
 #include <string.h>
@@ -509,15 +510,15 @@ template <int EPI, bool F8>
 cudaError_t launch_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB0, const CUtensorMap& mB1,
                        const CUtensorMap& mOut, const TcParams& p, int grid, int bma, int stages, size_t smem,
                        int64_t max_group_rows, cudaStream_t stream) {
-  static uint64_t attr_set = 0;  // one bit per device ordinal
+  static std::atomic<uint64_t> attr_set{0};  // one bit per device ordinal (host threads may launch concurrently)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 64 || !(attr_set & (1ull << dev))) {
+  if (dev >= 64 || !(attr_set.load(std::memory_order_relaxed) & (1ull << dev))) {
     e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<EPI, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemLimitTc));
     if (e != cudaSuccess) return e;
-    if (dev < 64) attr_set |= 1ull << dev;
+    if (dev < 64) attr_set.fetch_or(1ull << dev, std::memory_order_relaxed);
   }
   // programmatic dependent launch: the prologue may overlap the previous kernel
   e = launch_pdl(grouped_gemm_tc_kernel<EPI, F8>, dim3(grid), dim3(kThreads), smem, stream, mA,

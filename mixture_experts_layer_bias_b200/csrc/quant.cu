@@ -44,6 +44,7 @@
 #include <cuda_fp8.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -336,12 +337,22 @@ __global__ void __launch_bounds__(kWarps * 32)
   }
 }
 
+// Per-device host caches (atomics: host threads may launch concurrently).
+constexpr int kMaxDevices = 64;
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) dev = 0;
+  return dev;
+}
+
 int device_sms() {
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
+  static std::atomic<int> cache[kMaxDevices];
+  const int dev = current_device();
+  int sms = dev < kMaxDevices ? cache[dev].load(std::memory_order_relaxed) : 0;
+  if (sms <= 0) {
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
+    if (dev < kMaxDevices) cache[dev].store(sms, std::memory_order_relaxed);
   }
   return sms;
 }
@@ -370,12 +381,18 @@ cudaError_t launch_rows(const GroupEntry* groups, int num_groups, int use_out_ro
     // staged chunks: a multiple of 8 rows (one per warp), about 24 KB per chunk buffer (two per CTA)
     const int chunk = std::min(kMaxChunk, std::max(kWarps, (12288 / d) / kWarps * kWarps));
     const size_t smem = static_cast<size_t>(2) * chunk * d * 2;
-    static size_t attr_bytes = 0;  // the largest dynamic shared memory enabled so far
-    if (smem > attr_bytes) {
+    // the largest dynamic shared memory enabled so far, per device (the attribute is per device)
+    static std::atomic<size_t> attr_bytes[kMaxDevices];
+    const int dev = current_device();
+    if (dev >= kMaxDevices || smem > attr_bytes[dev].load(std::memory_order_relaxed)) {
       cudaError_t e = cudaFuncSetAttribute(quantize_rows_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
       if (e != cudaSuccess) return e;
-      attr_bytes = smem;
+      if (dev < kMaxDevices) {
+        size_t cur = attr_bytes[dev].load(std::memory_order_relaxed);
+        while (smem > cur && !attr_bytes[dev].compare_exchange_weak(cur, smem, std::memory_order_relaxed)) {
+        }
+      }
     }
     const int64_t chunks = (max_rows + chunk - 1) / chunk;
     // as many CTAs as are resident at once (shared memory, 8 CTAs of 256 threads at most)
