@@ -442,6 +442,42 @@ def time_bias_update(cfg, device, S, window=1000, reps=50):
     return round(e0.elapsed_time(e1) * 1e3 / reps, 2)
 
 
+def time_routing(run, peaks, reps=20, nbuf=5):
+    """The routing call alone (moe_route: logits, scoring, top-K), `reps`
+    calls captured in a CUDA graph over `nbuf` token buffers together larger
+    than L2; us per call (median of seven replays) and the HBM fraction of
+    its algorithmic bytes (x, W_r, the ids and gates written)."""
+    cfg, S, dev = run.cfg, run.S, run.device
+    xs = [run.inp["x"]] + [syn.make_inputs(cfg, dev, seed=100 + i, x_only=True)["x"] for i in range(nbuf - 1)]
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            ops.moe_route(run.desc, run.w, xs[0], None, run.idx, run.gw, run.ws, stream=s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for i in range(reps):
+            ops.moe_route(run.desc, run.w, xs[i % nbuf], None, run.idx, run.gw, run.ws, stream=s)
+    g.replay()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(7):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e3 / reps)
+    del g
+    us = statistics.median(times)
+    b = 2 if cfg.act_dtype == syn.BF16 else 4
+    nbytes = S * cfg.d * b + cfg.E * cfg.d * b + S * cfg.K * 8
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"us_per_call": round(us, 2), "bytes": nbytes, "hbm_gbs": round(gbs, 1),
+            "hbm_frac": round(gbs / peaks["hbm_gbs"], 3),
+            "note": f"{reps} calls in a CUDA graph over {nbuf} token buffers ({nbuf * S * cfg.d * b / 1e6:.0f} MB)"}
+
+
 # ---------------------------------------------------------------------------
 # the CPU oracle as a baseline (rank 0, bounded samples)
 # ---------------------------------------------------------------------------
@@ -687,6 +723,7 @@ def main():
 
     e2e = e2e_run(run, args.steps, args.warmup, world, dist)
     bias_us = time_bias_update(cfg, device, S)
+    routing = time_routing(run, peaks)
     dec = dec8 = None
     if not args.no_decode and args.workload == WORKLOAD:
         # right after the power-capped prefill loop the clocks are still held down for a
@@ -731,7 +768,7 @@ def main():
             "gpu_launches": kernels_per_step(cfg) * args.steps, "clocks": clk,
             "stages_ms": {k: round(v, 4) for k, v in stages.items()},
             "load": load, "decode_sweep": dec, "decode_sweep_e4m3": dec8, "bias_update_us": bias_us,
-            "counters": counters,
+            "routing": routing, "counters": counters,
             "workloads": workloads}
     print(json.dumps(line), flush=True)
 

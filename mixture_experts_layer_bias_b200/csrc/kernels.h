@@ -13,10 +13,11 @@ struct StatusBlock;
 
 // --- routing ---------------------------------------------------------------
 // Router logits: E <= 32 are computed inside the routing kernels (a CTA per
-// token for S <= 512, else warps streaming token rows against a copy of W_r in
-// shared memory of at most kRouteWSmemBytes); otherwise (E > 32, or W_r too
-// large for that copy when S > 512) one logits GEMM into the workspace first,
-// then the selection.
+// token for S <= 512; else, with W_r of at most kRouteWSmemBytes, tensor-core
+// products over 16 tokens per CTA with W_r read from L1/L2 (bf16), or warps
+// streaming token rows against a copy of W_r in shared memory (fp32));
+// otherwise (E > 32, or a larger W_r when S > 512, which every CTA would read
+// again) one logits GEMM into the workspace first, then the selection.
 constexpr int kRouteWSmemBytes = 64 << 10;
 inline bool route_logits_first(int64_t S, int64_t E, int64_t d, int elem_bytes) {
   return E > 32 || (S > 512 && E * d * elem_bytes > kRouteWSmemBytes);

@@ -29,10 +29,11 @@ using namespace route_detail;
 
 constexpr int kRouteWarps = 8;
 
-// E <= EMAX <= 32, large batches: every warp routes TPW tokens (2 for
+// fp32 activations, E <= EMAX <= 32, large batches (bf16 rows take the
+// tensor-core kernel below): every warp routes TPW tokens (2 for
 // EMAX = 8, 1 for EMAX = 32) over the whole of d, lanes striding over 16-byte
 // vectors; 8 (EMAX = 8) or 4 vectors of each token are loaded together per
-// lane (a token row's loads in two rounds at d = 4096 in bf16), so the
+// lane (a token row's loads in four rounds at d = 4096), so the
 // token rows -- the bytes that must come from HBM -- stream with many loads in
 // flight and no block-wide barrier.  The router weights sit in shared memory
 // (at most 64 KB: larger router matrices go through the logits GEMM, see
@@ -117,6 +118,148 @@ __global__ void __launch_bounds__(kRouteRowWarps * 32, 2)
       if (lane < p.E && router_bias != nullptr) l[0] = __fadd_rn(l[0], bias);
       select_topk<1>(l, p, t0 + tt);
     }
+  }
+}
+
+// bf16, E <= EMAX <= 32, large batches: the logits of 16 tokens against 8
+// experts over 16 columns of d are one m16n8k16 tensor-core product (bf16
+// operands, fp32 accumulation), so streaming the token rows costs no
+// per-element unpacking or FMA work and the pass is bound by reading x.  A
+// CTA owns 16 tokens; its warps split d into 32-column chunks (warp w takes
+// chunks w, w + 8, ...).  Per chunk, lane (g = lane / 4, q = lane % 4) loads
+// the 16 bytes at column 32c + 8q of token rows g and g + 8 and of router row
+// 8nt + g (L1/L2-resident): the quad's four lanes hold the chunk's 32
+// columns, and since the A and B fragments give a lane the same fragment
+// slots, columns 8q..8q+3 (8q+4..8q+7) fill slots {2q, 2q+1, 2q+8, 2q+9} of
+// the chunk's first (second) product and every column is summed once.  The
+// warps' partial logits are added in warp order through shared memory, then
+// each warp selects two of the CTA's tokens.
+constexpr int kRouteMmaWarps = 8;
+constexpr int kRouteMmaTokens = 16;
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// 16-byte read-only loads kept in program order with the products (volatile
+// asm), so a lane's U chunks are all in flight before the first product;
+// token rows are read once and bypass L1, router rows stay in L1
+__device__ __forceinline__ uint4 ld16_stream(const void* ptr) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(ptr));
+  return r;
+}
+__device__ __forceinline__ uint4 ld16_keep(const void* ptr) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(ptr));
+  return r;
+}
+
+template <int EMAX>
+__global__ void __launch_bounds__(kRouteMmaWarps * 32, 2)
+    route_rows_mma_kernel(int S, int d, const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w,
+                          const float* __restrict__ router_bias, SelectParams p) {
+  constexpr int NT = EMAX / 8;                  // n-tiles of 8 experts
+  constexpr int ACC = NT == 1 ? 2 : 1;          // independent accumulator chains per n-tile
+  constexpr int U = NT == 1 ? 8 : 3;            // chunks in flight per lane
+  __shared__ float part[kRouteMmaWarps][kRouteMmaTokens][EMAX];
+  const int warp = threadIdx.x >> 5, lane = lane_id();
+  const int g = lane >> 2, q = lane & 3;
+  const int t0 = blockIdx.x * kRouteMmaTokens;
+  const __nv_bfloat16* xa = x + static_cast<int64_t>(min(t0 + g, S - 1)) * d;
+  const __nv_bfloat16* xb = x + static_cast<int64_t>(min(t0 + g + 8, S - 1)) * d;
+  const __nv_bfloat16* wr[NT];
+  bool wok[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int n = nt * 8 + g;
+    wok[nt] = n < p.E;
+    wr[nt] = w + static_cast<int64_t>(wok[nt] ? n : 0) * d;
+  }
+  float acc[ACC][NT][4];
+#pragma unroll
+  for (int s = 0; s < ACC; ++s)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[s][nt][i] = 0.0f;
+  const uint4 zero = make_uint4(0, 0, 0, 0);
+  // full chunks, U per lane at a time: unconditional loads (rows of absent
+  // experts read router row 0 and are zeroed after the load)
+  const int nfull = d / 32;
+  int c0 = warp;
+  for (; c0 + (U - 1) * kRouteMmaWarps < nfull; c0 += kRouteMmaWarps * U) {
+    uint4 va[U], vb[U], vw[U][NT];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int col = (c0 + u * kRouteMmaWarps) * 32 + q * 8;
+      va[u] = ld16_stream(xa + col);
+      vb[u] = ld16_stream(xb + col);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint4 v = ld16_keep(wr[nt] + col);
+        vw[u][nt] = wok[nt] ? v : zero;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        float(&c)[4] = acc[u % ACC][nt];
+        mma_bf16_16816(c, va[u].x, vb[u].x, va[u].y, vb[u].y, vw[u][nt].x, vw[u][nt].y);
+        mma_bf16_16816(c, va[u].z, vb[u].z, va[u].w, vb[u].w, vw[u][nt].z, vw[u][nt].w);
+      }
+  }
+  // the remaining chunks one at a time; the last may be partial (d % 8 == 0:
+  // a lane's 8 columns are all inside d or all outside)
+  const int nch = (d + 31) / 32;
+  for (; c0 < nch; c0 += kRouteMmaWarps) {
+    const int col = c0 * 32 + q * 8;
+    const bool ok = col < d;
+    const uint4 va = ok ? ldg16(xa + col) : zero;
+    const uint4 vb = ok ? ldg16(xb + col) : zero;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const uint4 vw = (ok && wok[nt]) ? ldg16(wr[nt] + col) : zero;
+      mma_bf16_16816(acc[0][nt], va.x, vb.x, va.y, vb.y, vw.x, vw.y);
+      mma_bf16_16816(acc[0][nt], va.z, vb.z, va.w, vb.w, vw.z, vw.w);
+    }
+  }
+  // C fragment: c0, c1 = token g, experts 8nt + 2q + {0, 1}; c2, c3 = token g + 8
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[i] = ACC == 2 ? acc[0][nt][i] + acc[ACC - 1][nt][i] : acc[0][nt][i];
+    const int n = nt * 8 + 2 * q;
+    part[warp][g][n] = c[0];
+    part[warp][g][n + 1] = c[1];
+    part[warp][g + 8][n] = c[2];
+    part[warp][g + 8][n + 1] = c[3];
+  }
+  __syncthreads();
+  const float bias = (lane < p.E && router_bias != nullptr) ? __ldg(router_bias + lane) : 0.0f;
+#pragma unroll
+  for (int i = 0; i < kRouteMmaTokens / kRouteMmaWarps; ++i) {
+    const int tl = warp * (kRouteMmaTokens / kRouteMmaWarps) + i;
+    if (t0 + tl >= S) break;  // warp-uniform
+    float l[1] = {0.0f};
+    if (lane < EMAX) {
+      float s = 0.0f;
+#pragma unroll
+      for (int w2 = 0; w2 < kRouteMmaWarps; ++w2) s += part[w2][tl][lane];
+      l[0] = (lane < p.E && router_bias != nullptr) ? __fadd_rn(s, bias) : s;
+    }
+    select_topk<1>(l, p, t0 + tl);
   }
 }
 
@@ -268,6 +411,37 @@ cudaError_t launch_topk_ni(const RouteArgs& a, const float* logits, const Select
   return cudaGetLastError();
 }
 
+template <typename T, int EM>
+cudaError_t launch_route_token_cta(const RouteArgs& a, const SelectParams& sp, cudaStream_t st) {
+  return launch_pdl(route_token_cta_kernel<T, EM>, dim3(a.S), dim3(kRouteTokenWarps * 32), 0, st, a.d,
+                    static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);
+}
+
+template <int EM>
+cudaError_t launch_route_rows_mma(const RouteArgs& a, const SelectParams& sp, cudaStream_t st) {
+  const dim3 grid((a.S + kRouteMmaTokens - 1) / kRouteMmaTokens);
+  route_rows_mma_kernel<EM><<<grid, kRouteMmaWarps * 32, 0, st>>>(a.S, a.d, static_cast<const __nv_bfloat16*>(a.x),
+                                                                   static_cast<const __nv_bfloat16*>(a.w_router),
+                                                                   a.router_bias, sp);
+  return cudaGetLastError();
+}
+
+template <int EM>
+cudaError_t launch_route_rows_f32(const RouteArgs& a, const SelectParams& sp, cudaStream_t st) {
+  constexpr int TPW = EM >= 16 ? 1 : 16 / EM;
+  const int sets = (a.S + TPW - 1) / TPW;
+  const int want = (sets + kRouteRowWarps - 1) / kRouteRowWarps;
+  const int cap = (a.num_sms > 0 ? a.num_sms : 148) * 2;
+  const int grid = want < cap ? want : cap;
+  const size_t wbytes = static_cast<size_t>(a.E) * a.d * sizeof(float);  // <= kRouteWSmemBytes here
+  cudaError_t err =
+      cudaFuncSetAttribute(route_rows_kernel<float, EM>, cudaFuncAttributeMaxDynamicSharedMemorySize, kRouteWSmemBytes);
+  if (err != cudaSuccess) return err;
+  route_rows_kernel<float, EM><<<grid, kRouteRowWarps * 32, wbytes, st>>>(
+      a.S, a.d, static_cast<const float*>(a.x), static_cast<const float*>(a.w_router), a.router_bias, sp);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
@@ -277,40 +451,24 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
   const float* logits = a.logits;
   const int elem = a.act_dtype == MOE_F32 ? 4 : 2;
   if (logits == nullptr && !route_logits_first(a.S, a.E, a.d, elem)) {
-    // decode-sized batches: a CTA per token; otherwise warps streaming token rows
+    // decode-sized batches: a CTA per token; otherwise 16 tokens per CTA on
+    // the tensor cores (bf16; d % 8 == 0 for every layer) or warps streaming
+    // token rows (fp32)
     const bool per_cta = a.S <= 512;
-    cudaError_t err = cudaSuccess;
-#define MOE_ROUTE_LAUNCH(T, EM)                                                                                \
-  do {                                                                                                         \
-    if (per_cta) {                                                                                             \
-      err = launch_pdl(route_token_cta_kernel<T, EM>, dim3(a.S), dim3(kRouteTokenWarps * 32), 0, stream, a.d,  \
-                       static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);      \
-    } else {                                                                                                   \
-      constexpr int TPW = EM >= 16 ? 1 : 16 / EM;                                                              \
-      const int sets = (a.S + TPW - 1) / TPW;                                                                  \
-      const int want = (sets + kRouteRowWarps - 1) / kRouteRowWarps;                                           \
-      const int cap = (a.num_sms > 0 ? a.num_sms : 148) * 2;                                                   \
-      const int grid = want < cap ? want : cap;                                                                \
-      const size_t wbytes = static_cast<size_t>(a.E) * a.d * sizeof(T); /* <= kRouteWSmemBytes here */       \
-      err = cudaFuncSetAttribute(route_rows_kernel<T, EM>, cudaFuncAttributeMaxDynamicSharedMemorySize,         \
-                                 kRouteWSmemBytes);                                                            \
-      if (err == cudaSuccess)                                                                                  \
-        route_rows_kernel<T, EM><<<grid, kRouteRowWarps * 32, wbytes, stream>>>(                                \
-            a.S, a.d, static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.router_bias, sp);       \
-    }                                                                                                          \
-  } while (0)
+    const bool wide = a.E > 8;
+    cudaError_t err;
     if (a.act_dtype == MOE_BF16) {
-      if (a.E <= 8)
-        MOE_ROUTE_LAUNCH(__nv_bfloat16, 8);
+      if (per_cta)
+        err = wide ? launch_route_token_cta<__nv_bfloat16, 32>(a, sp, stream)
+                   : launch_route_token_cta<__nv_bfloat16, 8>(a, sp, stream);
       else
-        MOE_ROUTE_LAUNCH(__nv_bfloat16, 32);
+        err = wide ? launch_route_rows_mma<32>(a, sp, stream) : launch_route_rows_mma<8>(a, sp, stream);
     } else {
-      if (a.E <= 8)
-        MOE_ROUTE_LAUNCH(float, 8);
+      if (per_cta)
+        err = wide ? launch_route_token_cta<float, 32>(a, sp, stream) : launch_route_token_cta<float, 8>(a, sp, stream);
       else
-        MOE_ROUTE_LAUNCH(float, 32);
+        err = wide ? launch_route_rows_f32<32>(a, sp, stream) : launch_route_rows_f32<8>(a, sp, stream);
     }
-#undef MOE_ROUTE_LAUNCH
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
   }

@@ -122,12 +122,18 @@ def test_route_worked_example():
 @pytest.mark.parametrize("name,S,over", [("tiny_f32", 64, {}), ("mixtral_prefill", 512, {}),
                                          ("mixtral_prefill", 1500, {}), ("fp8_skew_capacity", 1024, {}),
                                          ("dsv3_grouped", 256, {}),
-                                         ("dsv3_grouped", 1024, dict(E=32, num_groups=4, topk_groups=2))])
+                                         ("dsv3_grouped", 1024, dict(E=32, num_groups=4, topk_groups=2)),
+                                         ("mixtral_prefill", 1000, dict(d=520, E=6)),
+                                         ("mixtral_prefill", 777, dict(d=1000, E=13, K=3)),
+                                         ("mixtral_prefill", 2049, dict(d=264, E=32, K=4))])
 def test_route_computed_logits_within_margin(name, S, over):
-    """The router computes its own logits: a CTA per token (S <= 512), warps
-    streaming token rows against W_r in shared memory (S > 512, E <= 32, W_r
-    of at most 64 KB: the Mixtral-shaped case at S = 1500), or the logits GEMM
-    then the selection (E > 32, or a larger W_r: 32 experts x 7168 here);
+    """The router computes its own logits: a CTA per token (S <= 512), for
+    S > 512, E <= 32 and W_r of at most 64 KB tensor-core products over 16
+    tokens per CTA (bf16: the Mixtral-shaped case at S = 1500, and ragged
+    cases with d not a multiple of 32, E not a multiple of 8 and S not a
+    multiple of 16) or warps streaming token rows against W_r in shared memory
+    (fp32), or the logits GEMM then the selection (E > 32, or a larger W_r:
+    32 experts x 7168 here);
     indices must agree with the oracle wherever the selection margin is
     >= 1e-4 (excluded tokens are counted), and the gates within the fp32
     tolerance."""
